@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Throughput of the 3LC codec on B200, one JSON line on stdout (rank 0).
+
+A step is one pass of the whole hot path over one synthetic gradient:
+tlc_compress (error feedback, magnitude, ternary quantization with sparsity
+multiplication, quartic packing, zero-run encoding), tlc_decompress (dense
+fp32 output) and tlc_decompress_accumulate (the stream added into a dense
+fp32 aggregation buffer).  The workload is the flat 2^28-value fp32 tensor,
+Laplace(0, 1e-4) with 90% exact zeros in geometric runs (mean 64), s = 1.9,
+with the error buffer carried from step to step.  Inputs (2 GiB of x + err)
+exceed the 126 MB L2, so every step streams from HBM.
+
+value = 4n bytes of fp32 input per step and GPU / device time per step.
+Under torchrun each rank compresses its own tensor (replicas, weak scaling);
+the step time is the maximum over ranks.  `--impl reference` times the CPU
+oracle on a bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("compress & decompress GB/s of fp32 input on 1 B200; % of HBM roofline; "
+          "bits/value")
+S_PARAM = 1.9
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--log2n", type=int, default=28, help="tensor size 2^k (default 28)")
+    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--cpu-baseline-log2n", type=int, default=26)
+    p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    return p.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def workload_config(n, log2n):
+    return {
+        "workload": (f"flat fp32 tensor of 2^{log2n} values, Laplace(0,1e-4) with 90% exact "
+                     f"zeros in geometric runs (mean 64), s={S_PARAM}; step = compress + "
+                     "decompress + decompress-accumulate (K=1), error buffer carried"),
+        "n": n,
+        "s": S_PARAM,
+        "input_bytes_per_step": 4 * n,
+        "l2": "inputs (x + err = 8n bytes) larger than the 126 MB L2; no flush",
+    }
+
+
+# ----------------------------------------------------------- clock sampler --
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id=None):
+        self.proc = None
+        self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "50"]
+        if bus_id:
+            cmd += ["-i", bus_id]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        self.tmp.seek(0)
+        rows = [r.split(",") for r in self.tmp.read().strip().splitlines() if r.count(",") >= 8]
+        os.unlink(self.tmp.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ ours ----
+
+def run_ours(args, rank, world, local):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import gradient_traffic_compression_b200 as tlc
+    import synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    n = 1 << args.log2n
+    x_h = synth.flat_tensor(3, n=n, step=rank)       # each rank: its own gradient
+
+    x = torch.from_numpy(x_h).to(dev)
+    err = torch.zeros(n, dtype=torch.float32, device=dev)
+    cap = tlc.tlc_compress_bound(n)
+    out = torch.empty(cap, dtype=torch.uint8, device=dev)
+    out_len = torch.zeros(1, dtype=torch.int64, device=dev)
+    y = torch.empty(n, dtype=torch.float32, device=dev)
+    acc = torch.zeros(n, dtype=torch.float32, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        tlc.tlc_compress(x, S_PARAM, err, out, out_len, status, stream)
+        tlc.tlc_decompress(out, n, y, in_len=out_len, in_cap=cap, dev_status=status,
+                           stream=stream)
+        tlc.tlc_decompress_accumulate([out], n, acc, in_lens=out_len, in_caps=[cap],
+                                      dev_status=status, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during warm-up")
+
+    bus = None
+    try:
+        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+    except Exception:
+        bus = None
+
+    # per-leg events (compress | decompress | accumulate) and library kernel timing
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(bus)
+    time.sleep(0.15)
+    tlc.tlc_kernel_timing(True)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        e = ev[k]
+        e[0].record(stream)
+        tlc.tlc_compress(x, S_PARAM, err, out, out_len, status, stream)
+        e[1].record(stream)
+        tlc.tlc_decompress(out, n, y, in_len=out_len, in_cap=cap, dev_status=status,
+                           stream=stream)
+        e[2].record(stream)
+        tlc.tlc_decompress_accumulate([out], n, acc, in_lens=out_len, in_caps=[cap],
+                                      dev_status=status, stream=stream)
+        e[3].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    tlc.tlc_kernel_timing(False)
+    kern = tlc.tlc_kernel_timing_read()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the timed region")
+
+    total_ms = t_start.elapsed_time(t_end)
+    legs = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)) for i in range(3)]
+    if world > 1:
+        t = torch.tensor([total_ms] + legs, dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, legs = float(t[0]), [float(v) for v in t[1:]]
+
+    L = int(out_len.item())
+    nnz = int(torch.count_nonzero(y).item())
+    ms_step = total_ms / args.steps
+    in_bytes = 4 * n
+    value = world * in_bytes / (ms_step * 1e-3) / 1e9
+    peak, peak_kind = load_peaks()
+
+    algo = {
+        "k_absmax": 8 * n,
+        "k_quant_zre": 12 * n + L,
+        "k_decode_write": L + 4 * n,
+        "k_decode_accumulate": L + 8 * nnz,
+    }
+    kernels = {}
+    for name, (launches, ms) in kern.items():
+        if launches == 0:
+            continue
+        per = ms / launches
+        gbs = algo[name] / (per * 1e-3) / 1e9
+        kernels[name] = {"launches": launches, "avg_ms": round(per, 5),
+                         "algo_bytes_per_launch": algo[name], "achieved_gbs": round(gbs, 1),
+                         "frac": round(gbs / peak, 4)}
+    dom = max(kernels, key=lambda k: kern[k][1])
+    c_ms, d_ms, a_ms = (v / args.steps for v in legs)
+    compress_bytes = algo["k_absmax"] + algo["k_quant_zre"]
+    decompress_bytes = algo["k_decode_write"]
+    result = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": workload_config(n, args.log2n) | {"parallelism": f"replicas x{world}"},
+        "clocks": clocks,
+        "gpu_launches": int(sum(v[0] for v in kern.values())),
+        "roofline": {
+            "bound": "hbm",
+            "kernel": dom,
+            "achieved": kernels[dom]["achieved_gbs"],
+            "peak": peak,
+            "peak_source": f"{peak_kind} hbm_gbs",
+            "unit": "GB/s",
+            "frac": kernels[dom]["frac"],
+            "traffic": traffic_for(dom, n),
+        },
+        "legs": {
+            "compress_gbs": round(in_bytes / (c_ms * 1e-3) / 1e9, 1),
+            "compress_ms": round(c_ms, 5),
+            "compress_hbm_frac": round(compress_bytes / (c_ms * 1e-3) / 1e9 / peak, 4),
+            "decompress_gbs": round(in_bytes / (d_ms * 1e-3) / 1e9, 1),
+            "decompress_ms": round(d_ms, 5),
+            "decompress_hbm_frac": round(decompress_bytes / (d_ms * 1e-3) / 1e9 / peak, 4),
+            "accumulate_gbs": round(in_bytes / (a_ms * 1e-3) / 1e9, 1),
+            "accumulate_ms": round(a_ms, 5),
+            "stream_bytes": L,
+            "bits_per_value": round(8 * L / n, 5),
+            "nonzero_values": nnz,
+        },
+        "kernels": kernels,
+    }
+
+    if not args.no_e2e:
+        result["e2e"] = run_e2e(args, tlc, torch, dev, x_h, n, cap, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args)
+    return result
+
+
+def run_e2e(args, tlc, torch, dev, x_h, n, cap, world):
+    """Same step through the public API with host buffers: pinned host x and
+    err copied in, stream, err and y copied out, every step."""
+    import numpy as np
+    import torch.distributed as dist
+    xh = torch.from_numpy(x_h).pin_memory()
+    eh = torch.zeros(n, dtype=torch.float32).pin_memory()
+    yh = torch.empty(n, dtype=torch.float32).pin_memory()
+    sh = torch.empty(cap, dtype=torch.uint8).pin_memory()
+    x = torch.empty(n, dtype=torch.float32, device=dev)
+    err = torch.empty(n, dtype=torch.float32, device=dev)
+    out = torch.empty(cap, dtype=torch.uint8, device=dev)
+    out_len = torch.zeros(1, dtype=torch.int64, device=dev)
+    y = torch.empty(n, dtype=torch.float32, device=dev)
+    acc = torch.zeros(n, dtype=torch.float32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    d2h = [0]
+
+    def step():
+        x.copy_(xh, non_blocking=True)
+        err.copy_(eh, non_blocking=True)
+        tlc.tlc_compress(x, S_PARAM, err, out, out_len, st)
+        L = int(out_len.item())
+        sh[:L].copy_(out[:L], non_blocking=True)
+        eh.copy_(err, non_blocking=True)
+        tlc.tlc_decompress(out, n, y, in_len=out_len, in_cap=cap, dev_status=st)
+        tlc.tlc_decompress_accumulate([out], n, acc, in_lens=out_len, in_caps=[cap],
+                                      dev_status=st)
+        yh.copy_(y, non_blocking=True)
+        torch.cuda.synchronize()
+        d2h[0] = L + 8 * n
+
+    step()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(args.e2e_steps):
+        step()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = t0.elapsed_time(t1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t[0])
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the e2e run")
+    return {"value": round(world * 4 * n / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "ms_per_step": round(ms, 3), "steps": args.e2e_steps,
+            "h2d_bytes_per_step": 8 * n, "d2h_bytes_per_step": d2h[0],
+            "path": "pinned host x, err -> device; tlc_compress; stream + err -> host; "
+                    "tlc_decompress; tlc_decompress_accumulate; y -> host"}
+
+
+# ------------------------------------------------------- CPU oracle timing --
+
+def oracle_step(oracle, x, n, acc):
+    import numpy as np
+    rc, st, e = oracle.compress(x, S_PARAM, np.zeros(n, np.float32))
+    rc2, y = oracle.decompress(st, n)
+    rc3, acc = oracle.decompress_accumulate([st], n, acc)
+    if rc or rc2 or rc3:
+        raise RuntimeError(f"oracle status {rc}/{rc2}/{rc3}")
+    return st.size, acc
+
+
+def cpu_baseline(args):
+    """The CPU oracle (single-threaded C, as it stands) on a bounded sample of
+    the same workload: repeated compress + decompress + accumulate steps."""
+    import numpy as np
+    import oracle
+    import synth
+    ns = 1 << args.cpu_baseline_log2n
+    x = synth.flat_tensor(3, n=ns)
+    acc = np.zeros(ns, np.float32)
+    oracle_step(oracle, x, ns, acc)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(oracle, x, ns, acc)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= args.cpu_baseline_seconds and reps >= 2:
+            break
+    return {"value": round(4 * ns * reps / el / 1e9, 4), "unit": "GB/s", "cores": 1,
+            "kind": "oracle", "seconds": round(el, 2),
+            "sample": f"{reps} steps of the same workload at n = 2^{args.cpu_baseline_log2n} "
+                      "(first-step error buffer), compress + decompress + accumulate",
+            "cpu": cpu_model()}
+
+
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip() + f" ({os.cpu_count()} threads visible)"
+    except OSError:
+        pass
+    return None
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import numpy as np
+    import oracle
+    import synth
+    ns = 1 << min(args.log2n, 24)
+    x = synth.flat_tensor(3, n=ns)
+    acc = np.zeros(ns, np.float32)
+    for _ in range(args.warmup):
+        oracle_step(oracle, x, ns, acc)
+    t0 = time.perf_counter()
+    L = 0
+    for _ in range(args.steps):
+        L, acc = oracle_step(oracle, x, ns, acc)
+    el = time.perf_counter() - t0
+    ms = el * 1e3 / args.steps
+    v = round(4 * ns / (ms * 1e-3) / 1e9, 4)
+    n = 1 << args.log2n
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_config(n, args.log2n) | {"parallelism": "single CPU core"},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": f"each step: the same workload at n = 2^{min(args.log2n, 24)} "
+                                   "(a bounded sample of the 2^28 tensor's distribution)",
+                         "cpu": cpu_model()},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "bits_per_value": round(8 * L / ns, 5),
+    }
+
+
+# ---------------------------------------------------------------- traffic ---
+
+def traffic_for(kernel, n):
+    """DRAM bytes per launch of `kernel` at size n from the committed ncu
+    summary (profiles/dram_traffic.txt), scaled by n; None when there is no
+    capture for it or the kernel sources changed since the capture."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    from gradient_traffic_compression_b200.build import source_digest
+    digest = source_digest()
+    with open(path) as f:
+        for line in f:
+            t = line.split()
+            if len(t) == 4 and not line.startswith("#") and t[0] == kernel:
+                n_cap, bytes_cap, dig = int(t[1]), float(t[2]), t[3]
+                if dig != digest:
+                    return None
+                return int(bytes_cap * n / n_cap)
+    return None
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    try:
+        res = run_ours(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,28 @@
+"""3LC state-change compression for NVIDIA B200 (sm_100a).
+
+The codec itself is the C ABI in include/tlc.h, built into libtlc.so from
+csrc/ (hand-written CUDA kernels).  ``tlc`` is its ctypes binding; torch is
+used only for device memory and streams.
+"""
+from .tlc import (  # noqa: F401
+    CORRUPT,
+    CUDA_ERROR,
+    INVALID_ARG,
+    NONFINITE,
+    OK,
+    TIMEOUT,
+    TLCError,
+    compress,
+    decompress,
+    lib,
+    status_string,
+    tlc_compress,
+    tlc_compress_bound,
+    tlc_decompress,
+    tlc_decompress_accumulate,
+    tlc_kernel_timing,
+    tlc_kernel_timing_read,
+    tlc_set_wait_limit,
+    tlc_test_wait_timeout,
+    version,
+)

@@ -1,0 +1,552 @@
+// tlc_compress.cu -- compression kernels for the 3LC pipeline on sm_100a.
+//
+// Source: review page "3LC: Lightweight and Effective Traffic Compression for
+// Distributed Machine Learning", section "Proposed method":
+//   bullet 1  3-value quantization with sparsity multiplication and an
+//             error-accumulation buffer  -> k_absmax + first half of k_quant_zre
+//   bullet 2  quartic encoding (five ternary values per byte) -> k_quant_zre
+//   bullet 3  zero-run encoding of all-zero byte groups       -> k_quant_zre
+// bullet 5 of the same section asks for vectorised, byte-level processing
+// with low overhead; here that is 128-bit coalesced loads, one pass per
+// dependency, and a single-pass scan so no byte intermediate touches HBM.
+//
+// Two launches per call:
+//   k_absmax     x' = x + err and M = max|x'| (as a max over the uint32 bit
+//                patterns of |x'|; NaN/Inf sort above every finite value).
+//                It also clears the scan state that k_quant_zre uses.
+//   k_quant_zre  per tile of 4096 byte groups (20480 values): recompute x',
+//                q = round(x'/(M s)), err' = x' - q M s (written back), pack
+//                the quartic bytes into shared memory, zero-run encode them,
+//                and place the tile's output with a decoupled look-back over
+//                earlier tiles.  Tiles are taken in order from a ticket
+//                counter, so every tile a tile waits on is already running.
+//
+// Zero-run emission order.  A maximal run of L bytes equal to 121 emits
+// floor(L/14) bytes 255 (one at the end of each full chunk of 14), then, if
+// L mod 14 = r != 0, one remainder byte (121 for r = 1, else 241 + r).  The
+// remainder is written by the first non-121 byte after the run (just before
+// that byte's own literal), or by the last tile at the end of the stream.
+// The output sequence is the canonical one -- full chunks from the start of
+// the run, remainder last -- but no tile needs to look at the next tile.
+//
+// Tile summary (aggregate) for a segment of bytes, as a function of the
+// incoming run length t (mod 14) of 121-bytes that precede it:
+//   all    the segment is entirely 121s (then A = its length)
+//   A      length of its leading 121-run
+//   R      bytes emitted from position A onwards (literals, full chunks of
+//          runs that start inside, remainders before literals)
+//   tc     length mod 14 of the trailing 121-run (if not all)
+// emitted(t) = (all ? floor : ceil)((t + A) / 14) + R
+// t_out(t)   = all ? (t + A) mod 14 : tc
+// Two segments compose associatively (see compose()).
+#include "tlc_device.cuh"
+#include "tlc_internal.h"
+
+namespace tlc {
+
+// ------------------------------------------------------------ k_absmax ----
+constexpr int kAbsThreads = 512;
+constexpr int kAbsUnroll = 4;
+
+__device__ __forceinline__ uint32_t abs_bits(float v) {
+  return __float_as_uint(v) & 0x7fffffffu;
+}
+
+template <bool kVec>
+__global__ void __launch_bounds__(kAbsThreads)
+k_absmax(const float *__restrict__ x, const float *__restrict__ err, uint64_t n,
+         uint32_t *__restrict__ partial, uint64_t *__restrict__ zero_words,
+         uint32_t n_zero) {
+  uint32_t m = 0;
+  const uint64_t gtid = (uint64_t)blockIdx.x * kAbsThreads + threadIdx.x;
+  const uint64_t nth = (uint64_t)gridDim.x * kAbsThreads;
+  if (kVec) {
+    const uint64_t n4 = n >> 2;
+    const float4 *x4 = reinterpret_cast<const float4 *>(x);
+    const float4 *e4 = reinterpret_cast<const float4 *>(err);
+    uint64_t i = gtid;
+    for (; i + (kAbsUnroll - 1) * nth < n4; i += kAbsUnroll * nth) {
+      float4 a[kAbsUnroll], b[kAbsUnroll];
+#pragma unroll
+      for (int u = 0; u < kAbsUnroll; ++u) {
+        a[u] = __ldg(x4 + i + u * nth);
+        b[u] = __ldg(e4 + i + u * nth);
+      }
+#pragma unroll
+      for (int u = 0; u < kAbsUnroll; ++u) {
+        m = max(m, abs_bits(__fadd_rn(a[u].x, b[u].x)));
+        m = max(m, abs_bits(__fadd_rn(a[u].y, b[u].y)));
+        m = max(m, abs_bits(__fadd_rn(a[u].z, b[u].z)));
+        m = max(m, abs_bits(__fadd_rn(a[u].w, b[u].w)));
+      }
+    }
+    for (; i < n4; i += nth) {
+      const float4 a = __ldg(x4 + i), b = __ldg(e4 + i);
+      m = max(m, abs_bits(__fadd_rn(a.x, b.x)));
+      m = max(m, abs_bits(__fadd_rn(a.y, b.y)));
+      m = max(m, abs_bits(__fadd_rn(a.z, b.z)));
+      m = max(m, abs_bits(__fadd_rn(a.w, b.w)));
+    }
+    const uint64_t rem = n - (n4 << 2);
+    if (gtid < rem) {
+      const uint64_t k = (n4 << 2) + gtid;
+      m = max(m, abs_bits(__fadd_rn(x[k], err[k])));
+    }
+  } else {
+    for (uint64_t i = gtid; i < n; i += nth) m = max(m, abs_bits(__fadd_rn(x[i], err[i])));
+  }
+  for (uint64_t w = gtid; w < n_zero; w += nth) zero_words[w] = 0;
+
+  __shared__ uint32_t wmax[kAbsThreads / kWarp];
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < kWarp) {
+    uint32_t v = threadIdx.x < kAbsThreads / kWarp ? wmax[threadIdx.x] : 0u;
+    v = __reduce_max_sync(0xffffffffu, v);
+    if (threadIdx.x == 0) partial[blockIdx.x] = v;
+  }
+}
+
+// --------------------------------------------------------- k_quant_zre ----
+constexpr int kQThreads = 256;
+constexpr int kQWarps = kQThreads / kWarp;
+constexpr int kChunkElems = 640;   // one warp step: 32 lanes x 5 float4
+constexpr int kChunkGroups = 128;  // = kChunkElems / 5
+constexpr int kQIters = 4;
+constexpr int kTileGroups = kQWarps * kQIters * kChunkGroups;  // 4096
+constexpr uint64_t kTileElems = 5ull * kTileGroups;            // 20480
+constexpr int kZBytes = kTileGroups / kQThreads;               // 16 per thread
+static_assert(kZBytes == 16, "ZRE stage reads one uint4 per thread");
+
+struct ZAgg {
+  uint32_t all, A, R, tc;
+};
+
+__device__ __forceinline__ uint64_t pack_agg(const ZAgg &a) {
+  return kFlagAgg | (uint64_t)a.A | ((uint64_t)a.R << 16) | ((uint64_t)a.tc << 32) |
+         ((uint64_t)a.all << 36);
+}
+__device__ __forceinline__ ZAgg unpack_agg(uint64_t w) {
+  ZAgg a;
+  a.A = (uint32_t)(w & 0xffffu);
+  a.R = (uint32_t)((w >> 16) & 0xffffu);
+  a.tc = (uint32_t)((w >> 32) & 0xfu);
+  a.all = (uint32_t)((w >> 36) & 1u);
+  return a;
+}
+// Inclusive prefix: emitted count C (< 2^32) and run length mod 14.
+__device__ __forceinline__ uint64_t pack_prefix(uint32_t C, uint32_t t) {
+  return kFlagPrefix | (uint64_t)C | ((uint64_t)t << 32);
+}
+
+__device__ __forceinline__ uint32_t lead_count(const ZAgg &a, uint32_t t) {
+  const uint32_t v = t + a.A;
+  return a.all ? v / 14u : (v + 13u) / 14u;
+}
+
+__device__ __forceinline__ void eval_agg(uint32_t &C, uint32_t &t, const ZAgg &a) {
+  C += lead_count(a, t) + a.R;
+  t = a.all ? (t + a.A) % 14u : a.tc;
+}
+
+// Aggregate of segment a1 followed by segment a2.
+__device__ __forceinline__ ZAgg compose(const ZAgg &a1, const ZAgg &a2) {
+  ZAgg r;
+  if (!a1.all) {
+    r.all = 0;
+    r.A = a1.A;
+    r.R = a1.R + lead_count(a2, a1.tc) + a2.R;
+    r.tc = a2.all ? (a1.tc + a2.A) % 14u : a2.tc;
+  } else {
+    r.all = a2.all;
+    r.A = a1.A + a2.A;
+    r.R = a2.R;
+    r.tc = a2.tc;
+  }
+  return r;
+}
+
+__device__ __forceinline__ uint8_t remainder_byte(uint32_t r) {
+  return r == 1 ? uint8_t(121) : uint8_t(241 + r);
+}
+
+// One element: digit q+1 of round(x'/scale) with ties away from zero, and
+// the updated error x' - q*scale.  M = 0 gives q = 0 with no division.
+__device__ __forceinline__ uint32_t quant_digit(float xp, float scale, bool mzero, float &e) {
+  uint32_t d = 1;
+  if (!mzero) {
+    const float r = __fdiv_rn(xp, scale);
+    if (fabsf(r) >= 0.5f) d = (r > 0.0f) ? 2u : 0u;
+  }
+  e = (d == 1) ? xp : __fsub_rn(xp, d == 2 ? scale : -scale);
+  return d;
+}
+
+// Quartic byte of five digits, first digit most significant (Horner in base 3).
+__device__ __forceinline__ uint32_t pack_groups4(const uint32_t w[5]) {
+  uint32_t out = 0;
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint32_t v = 0;
+#pragma unroll
+    for (int d = 0; d < 5; ++d) {
+      const int i = 5 * g + d;
+      v = v * 3u + ((w[i >> 2] >> (8 * (i & 3))) & 0xffu);
+    }
+    out |= v << (8 * g);
+  }
+  return out;
+}
+
+struct QuantArgs {
+  const float *x;
+  float *err;
+  uint64_t n;
+  uint64_t groups;
+  float s;
+  const uint32_t *partial;
+  uint32_t n_partial;
+  uint8_t *out;
+  uint64_t out_cap;
+  uint64_t *out_len;
+  uint64_t *status;
+  uint32_t *ticket;
+  uint32_t n_tiles;
+  int32_t *dev_status;
+  uint32_t max_polls;
+};
+
+__device__ __forceinline__ void put_out(const QuantArgs &a, uint64_t pos, uint8_t v) {
+  if (4 + pos < a.out_cap) a.out[4 + pos] = v;
+}
+
+template <bool kVec>
+__global__ void __launch_bounds__(kQThreads)
+k_quant_zre(const QuantArgs a) {
+  __shared__ __align__(16) uint32_t dig_s[kQWarps][kChunkElems / 4];
+  __shared__ __align__(16) uint32_t tile_s[kTileGroups / 4];
+  __shared__ uint32_t scan_s[kQWarps + 1];
+  __shared__ uint32_t tile_id_s, A_s, cin_s, tin_s;
+  __shared__ float scale_s;
+  __shared__ int state_s;  // 0 ok, 1 M == 0, 2 non-finite
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  // M from the per-block partial maxima of k_absmax.
+  if (warp == 0) {
+    uint32_t mb = 0;
+    for (uint32_t i = lane; i < a.n_partial; i += kWarp) mb = max(mb, a.partial[i]);
+    mb = __reduce_max_sync(0xffffffffu, mb);
+    if (lane == 0) {
+      int st = 0;
+      float scale = 0.0f;
+      if (mb >= 0x7f800000u) {
+        st = 2;
+      } else {
+        scale = __fmul_rn(__uint_as_float(mb), a.s);
+        if (!isfinite(scale)) st = 2;
+        else if (mb == 0) st = 1;
+      }
+      scale_s = scale;
+      state_s = st;
+    }
+  }
+  __syncthreads();
+  if (state_s == 2) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      report(a.dev_status, TLC_ERR_NONFINITE);
+      *a.out_len = 0;
+    }
+    return;
+  }
+  const float scale = scale_s;
+  const bool mzero = state_s == 1;
+
+  for (;;) {
+    if (threadIdx.x == 0) {
+      tile_id_s = atomicAdd(a.ticket, 1u);
+      A_s = 0xffffffffu;
+    }
+    __syncthreads();
+    const uint32_t t = tile_id_s;
+    if (t >= a.n_tiles) break;
+
+    const uint64_t g0 = (uint64_t)t * kTileGroups;
+    const uint32_t tgv = (uint32_t)umin64(kTileGroups, a.groups - g0);
+    const uint64_t e_tile = g0 * 5;
+    const bool full = kVec && (e_tile + kTileElems <= a.n);
+
+    // ---- quantize + error update + quartic pack ------------------------
+#pragma unroll 1
+    for (int it = 0; it < kQIters; ++it) {
+      const int c = it * kQWarps + warp;
+      const uint64_t e0 = e_tile + (uint64_t)c * kChunkElems;
+      if (full) {
+        const float4 *x4 = reinterpret_cast<const float4 *>(a.x + e0);
+        float4 *err4 = reinterpret_cast<float4 *>(a.err + e0);
+        float4 xv[5], ev[5];
+#pragma unroll
+        for (int j = 0; j < 5; ++j) {
+          xv[j] = __ldg(x4 + lane + 32 * j);
+          ev[j] = err4[lane + 32 * j];
+        }
+#pragma unroll
+        for (int j = 0; j < 5; ++j) {
+          float4 o;
+          uint32_t dw;
+          dw = quant_digit(__fadd_rn(xv[j].x, ev[j].x), scale, mzero, o.x);
+          dw |= quant_digit(__fadd_rn(xv[j].y, ev[j].y), scale, mzero, o.y) << 8;
+          dw |= quant_digit(__fadd_rn(xv[j].z, ev[j].z), scale, mzero, o.z) << 16;
+          dw |= quant_digit(__fadd_rn(xv[j].w, ev[j].w), scale, mzero, o.w) << 24;
+          err4[lane + 32 * j] = o;
+          dig_s[warp][lane + 32 * j] = dw;
+        }
+      } else {
+#pragma unroll 1
+        for (int j = 0; j < 5; ++j) {
+          uint32_t dw = 0;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t e = e0 + 4 * (uint64_t)(lane + 32 * j) + k;
+            uint32_t d = 1;
+            if (e < a.n) {
+              float o;
+              d = quant_digit(__fadd_rn(a.x[e], a.err[e]), scale, mzero, o);
+              a.err[e] = o;
+            }
+            dw |= d << (8 * k);
+          }
+          dig_s[warp][lane + 32 * j] = dw;
+        }
+      }
+      __syncwarp();
+      uint32_t w5[5];
+#pragma unroll
+      for (int k = 0; k < 5; ++k) w5[k] = dig_s[warp][5 * lane + k];
+      tile_s[c * (kChunkGroups / 4) + lane] = pack_groups4(w5);
+      __syncwarp();
+    }
+    __syncthreads();
+
+    // ---- zero-run encoding: local analysis -----------------------------
+    const uint4 q4 = reinterpret_cast<const uint4 *>(tile_s)[threadIdx.x];
+    const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
+    const int p0 = (int)threadIdx.x * kZBytes;
+    int fnz = -1, lnz = -1;
+#pragma unroll
+    for (int k = 0; k < kZBytes; ++k) {
+      const uint32_t b = (qw[k >> 2] >> (8 * (k & 3))) & 0xffu;
+      const int p = p0 + k;
+      if (p < (int)tgv && b != 121u) {
+        if (fnz < 0) fnz = p;
+        lnz = p;
+      }
+    }
+    int32_t lnz_all;
+    const int prev_in = block_exclusive_max<kQThreads>(lnz, reinterpret_cast<int32_t *>(scan_s), lnz_all);
+    if (prev_in < 0 && fnz >= 0) A_s = (uint32_t)fnz;
+
+    uint32_t cnt = 0;
+    {
+      int prev = prev_in;
+#pragma unroll
+      for (int k = 0; k < kZBytes; ++k) {
+        const uint32_t b = (qw[k >> 2] >> (8 * (k & 3))) & 0xffu;
+        const int p = p0 + k;
+        if (p >= (int)tgv) break;
+        if (b == 121u) {
+          if (prev >= 0 && (p - prev - 1) % 14 == 13) ++cnt;
+        } else {
+          if (prev >= 0 && (p - 1 - prev) % 14 != 0) ++cnt;
+          ++cnt;
+          prev = p;
+        }
+      }
+    }
+    uint32_t R;
+    const uint32_t off = block_exclusive_sum<kQThreads>(cnt, scan_s, R);
+
+    ZAgg agg;
+    agg.all = lnz_all < 0 ? 1u : 0u;
+    agg.A = agg.all ? tgv : A_s;
+    agg.R = R;
+    agg.tc = agg.all ? 0u : (uint32_t)((int)tgv - 1 - lnz_all) % 14u;
+
+    // ---- decoupled look-back -------------------------------------------
+    if (warp == 0) {
+      if (t == 0) {
+        if (lane == 0) {
+          uint32_t C = 0, tt = 0;
+          eval_agg(C, tt, agg);
+          st_relaxed_u64(a.status, pack_prefix(C, tt));
+          cin_s = 0;
+          tin_s = 0;
+        }
+      } else {
+        if (lane == 0) st_relaxed_u64(a.status + t, pack_agg(agg));
+        bool timed_out = false;
+        bool have_suffix = false;
+        ZAgg suffix = {0, 0, 0, 0};
+        int64_t end = (int64_t)t - 1;
+        uint32_t C = 0, tt = 0;
+        for (;;) {
+          const int64_t idx = end - lane;
+          const uint64_t w =
+              idx >= 0 ? wait_flag(a.status + idx, a.max_polls, timed_out) : pack_prefix(0, 0);
+          const uint32_t pmask = __ballot_sync(0xffffffffu, (w >> kFlagShift) == 2);
+          if (pmask) {
+            const int pl = __ffs(pmask) - 1;
+            const uint64_t wp = __shfl_sync(0xffffffffu, w, pl);
+            C = (uint32_t)(wp & 0xffffffffu);
+            tt = (uint32_t)((wp >> 32) & 0xfu);
+            for (int l = pl - 1; l >= 0; --l) {
+              const uint64_t wl = __shfl_sync(0xffffffffu, w, l);
+              eval_agg(C, tt, unpack_agg(wl));
+            }
+            if (have_suffix) eval_agg(C, tt, suffix);
+            break;
+          }
+          ZAgg acc = unpack_agg(__shfl_sync(0xffffffffu, w, 31));
+          for (int l = 30; l >= 0; --l)
+            acc = compose(acc, unpack_agg(__shfl_sync(0xffffffffu, w, l)));
+          suffix = have_suffix ? compose(acc, suffix) : acc;
+          have_suffix = true;
+          end -= kWarp;
+        }
+        if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(a.dev_status, TLC_ERR_TIMEOUT);
+        if (lane == 0) {
+          cin_s = C;
+          tin_s = tt;
+          uint32_t Ci = C, ti = tt;
+          eval_agg(Ci, ti, agg);
+          st_relaxed_u64(a.status + t, pack_prefix(Ci, ti));
+        }
+      }
+    }
+    __syncthreads();
+    const uint32_t cin = cin_s, tin = tin_s;
+
+    // ---- emission --------------------------------------------------------
+    {
+      uint64_t k_out = (uint64_t)cin + lead_count(agg, tin) + off;
+      int prev = prev_in;
+#pragma unroll
+      for (int k = 0; k < kZBytes; ++k) {
+        const uint32_t b = (qw[k >> 2] >> (8 * (k & 3))) & 0xffu;
+        const int p = p0 + k;
+        if (p >= (int)tgv) break;
+        if (b == 121u) {
+          if (prev < 0) {
+            if ((tin + p) % 14u == 13u) put_out(a, cin + (tin + p) / 14u, 255);
+          } else if ((p - prev - 1) % 14 == 13) {
+            put_out(a, k_out++, 255);
+          }
+        } else {
+          if (prev < 0) {
+            const uint32_t r = (tin + p) % 14u;
+            if (r) put_out(a, cin + (tin + p) / 14u, remainder_byte(r));
+          } else {
+            const uint32_t r = (uint32_t)(p - 1 - prev) % 14u;
+            if (r) put_out(a, k_out++, remainder_byte(r));
+          }
+          put_out(a, k_out++, (uint8_t)b);
+          prev = p;
+        }
+      }
+    }
+    if (threadIdx.x == 0) {
+      if (t == 0) {
+        const uint32_t sb = __float_as_uint(scale);
+        a.out[0] = sb & 0xff;
+        a.out[1] = (sb >> 8) & 0xff;
+        a.out[2] = (sb >> 16) & 0xff;
+        a.out[3] = (sb >> 24) & 0xff;
+      }
+      if (t == a.n_tiles - 1) {
+        uint32_t C = cin, tt = tin;
+        eval_agg(C, tt, agg);
+        if (tt) put_out(a, C, remainder_byte(tt));
+        *a.out_len = 4ull + C + (tt ? 1u : 0u);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------- launcher ---
+uint32_t compress_tiles(uint64_t n) {
+  const uint64_t g = (n + 4) / 5;
+  return (uint32_t)((g + kTileGroups - 1) / kTileGroups);
+}
+
+uint32_t compress_partials(const DeviceInfo &dev, uint64_t n) {
+  const uint64_t per_block = (uint64_t)kAbsThreads * 4 * kAbsUnroll;
+  uint64_t want = (n + per_block - 1) / per_block;
+  const uint64_t cap = (uint64_t)dev.sm_count * 4;
+  if (want > cap) want = cap;
+  if (want < 1) want = 1;
+  return (uint32_t)want;
+}
+
+cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, float s,
+                            float *err, uint8_t *out, uint64_t out_cap, uint64_t *out_len,
+                            int32_t *dev_status, uint32_t max_polls, void *scratch,
+                            cudaStream_t stream) {
+  const uint32_t n_tiles = compress_tiles(n);
+  const uint32_t n_part = compress_partials(dev, n);
+  CompressScratch sc = compress_scratch_layout(scratch, n_part, n_tiles);
+  const bool vec = ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(err)) & 15) == 0;
+
+  // status words and the ticket are cleared by k_absmax (ticket sits in
+  // the word right after the status array).
+  timing_begin(kKindAbsmax, stream);
+  if (vec)
+    k_absmax<true><<<n_part, kAbsThreads, 0, stream>>>(x, err, n, sc.partial, sc.status,
+                                                        n_tiles + 1);
+  else
+    k_absmax<false><<<n_part, kAbsThreads, 0, stream>>>(x, err, n, sc.partial, sc.status,
+                                                         n_tiles + 1);
+  timing_end(kKindAbsmax, stream);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+
+  QuantArgs qa;
+  qa.x = x;
+  qa.err = err;
+  qa.n = n;
+  qa.groups = (n + 4) / 5;
+  qa.s = s;
+  qa.partial = sc.partial;
+  qa.n_partial = n_part;
+  qa.out = out;
+  qa.out_cap = out_cap;
+  qa.out_len = out_len;
+  qa.status = sc.status;
+  qa.ticket = sc.ticket;
+  qa.n_tiles = n_tiles;
+  qa.dev_status = dev_status;
+  qa.max_polls = max_polls;
+
+  int occ = vec ? dev.occ_quant_vec : dev.occ_quant_scalar;
+  uint32_t grid = (uint32_t)dev.sm_count * (uint32_t)(occ > 0 ? occ : 1);
+  if (grid > n_tiles) grid = n_tiles;
+  timing_begin(kKindQuantZre, stream);
+  if (vec)
+    k_quant_zre<true><<<grid, kQThreads, 0, stream>>>(qa);
+  else
+    k_quant_zre<false><<<grid, kQThreads, 0, stream>>>(qa);
+  timing_end(kKindQuantZre, stream);
+  return cudaGetLastError();
+}
+
+int occupancy_quant(bool vec) {
+  int occ = 0;
+  if (vec)
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_quant_zre<true>, kQThreads, 0);
+  else
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_quant_zre<false>, kQThreads, 0);
+  return occ;
+}
+
+}  // namespace tlc

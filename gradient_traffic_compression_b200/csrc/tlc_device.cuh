@@ -1,0 +1,137 @@
+// tlc_device.cuh -- device-side helpers shared by the compress and decode
+// kernels: status-word publication for single-pass (decoupled look-back)
+// scans, bounded waits, block-wide scans, and error reporting.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/tlc.h"
+
+namespace tlc {
+
+constexpr int kWarp = 32;
+
+__host__ __device__ __forceinline__ uint64_t umin64(uint64_t a, uint64_t b) { return a < b ? a : b; }
+
+// ---------------------------------------------------------------------------
+// Tile status words.  Each tile of a single-pass scan owns one 64-bit word:
+// bits 62..63 hold the flag, the rest the tile's value.  A word is written
+// first with its aggregate (flag 1) and later with its inclusive prefix
+// (flag 2); both values are self-contained, so relaxed 64-bit accesses at
+// GPU scope are enough (a reader sees one whole word or the other).
+// ---------------------------------------------------------------------------
+constexpr uint64_t kFlagShift = 62;
+constexpr uint64_t kFlagAgg = 1ull << kFlagShift;
+constexpr uint64_t kFlagPrefix = 2ull << kFlagShift;
+constexpr uint64_t kValueMask = (1ull << kFlagShift) - 1;
+
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t *p) {
+  uint64_t v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Record a data-dependent failure; the first error wins, zero is never written.
+__device__ __forceinline__ void report(int32_t *dev_status, int code) {
+  if (dev_status) atomicCAS(reinterpret_cast<int *>(dev_status), 0, code);
+}
+
+// Poll a status word until its flag is set, at most `max_polls` times.
+// Returns the word, or kFlagPrefix with value 0 after giving up (the caller
+// then reports TLC_ERR_TIMEOUT; the result is wrong but every write stays
+// in bounds, and later tiles can still finish).
+__device__ __forceinline__ uint64_t wait_flag(const uint64_t *p, uint32_t max_polls,
+                                              bool &timed_out) {
+  uint64_t w = ld_relaxed_u64(p);
+  uint32_t polls = 0;
+  unsigned ns = 32;
+  while ((w >> kFlagShift) == 0) {
+    if (++polls >= max_polls) {
+      timed_out = true;
+      return kFlagPrefix;
+    }
+    __nanosleep(ns);
+    if (ns < 512) ns <<= 1;
+    w = ld_relaxed_u64(p);
+  }
+  return w;
+}
+
+// ---------------------------------------------------------------------------
+// Block-wide exclusive scans for blocks of kThreads threads (multiple of 32).
+// `scratch` needs kThreads/32 + 1 words of shared memory.  Every thread
+// receives the block total as well.
+// ---------------------------------------------------------------------------
+template <int kThreads>
+__device__ __forceinline__ uint32_t block_exclusive_sum(uint32_t v, uint32_t *scratch,
+                                                        uint32_t &total) {
+  constexpr int kWarps = kThreads / kWarp;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t inc = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc += t;
+  }
+  if (lane == 31) scratch[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = lane < kWarps ? scratch[lane] : 0;
+    uint32_t wi = w;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      uint32_t t = __shfl_up_sync(0xffffffffu, wi, d);
+      if (lane >= d) wi += t;
+    }
+    if (lane < kWarps) scratch[lane] = wi - w;   // exclusive warp offsets
+    if (lane == kWarps - 1) scratch[kWarps] = wi;
+  }
+  __syncthreads();
+  uint32_t r = scratch[warp] + inc - v;
+  total = scratch[kWarps];
+  __syncthreads();
+  return r;
+}
+
+// Exclusive max-scan of signed values (identity -1); also returns the block max.
+template <int kThreads>
+__device__ __forceinline__ int32_t block_exclusive_max(int32_t v, int32_t *scratch,
+                                                       int32_t &total) {
+  constexpr int kWarps = kThreads / kWarp;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t inc = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    int32_t t = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc = max(inc, t);
+  }
+  int32_t exc_in_warp = __shfl_up_sync(0xffffffffu, inc, 1);
+  if (lane == 0) exc_in_warp = -1;
+  if (lane == 31) scratch[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = lane < kWarps ? scratch[lane] : -1;
+    int32_t wi = w;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      int32_t t = __shfl_up_sync(0xffffffffu, wi, d);
+      if (lane >= d) wi = max(wi, t);
+    }
+    int32_t we = __shfl_up_sync(0xffffffffu, wi, 1);
+    if (lane == 0) we = -1;
+    if (lane < kWarps) scratch[lane] = we;
+    if (lane == kWarps - 1) scratch[kWarps] = wi;
+  }
+  __syncthreads();
+  int32_t r = max(scratch[warp], exc_in_warp);
+  total = scratch[kWarps];
+  __syncthreads();
+  return r;
+}
+
+}  // namespace tlc

@@ -1,0 +1,209 @@
+"""Python binding of the C ABI in include/tlc.h (argument marshalling only).
+
+Every function forwards to libtlc.so: tensors become raw device pointers and
+sizes, the stream is torch's current CUDA stream unless one is given.  All
+compression and decompression work runs in the library's CUDA kernels; if the
+library cannot be loaded, or a tensor is not on a CUDA device, these
+functions raise instead of computing anything elsewhere.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+from . import build as _build
+
+OK, INVALID_ARG, NONFINITE, CORRUPT, TIMEOUT, CUDA_ERROR = 0, 1, 2, 3, 4, 5
+
+_lib = None
+
+
+class TLCError(RuntimeError):
+    """A host-detected failure returned by the C ABI."""
+
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn}: {status_string(code)} (status {code})")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtlc.so (building it with nvcc first if it does not exist)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = _build.library_path()
+    if not os.path.exists(path):
+        _build.build_library()
+    L = ctypes.CDLL(path)
+    P, S, U64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint64
+    L.tlc_compress_bound.argtypes = [S]
+    L.tlc_compress_bound.restype = S
+    L.tlc_compress.argtypes = [P, S, ctypes.c_float, P, P, S, P, P, P]
+    L.tlc_compress.restype = ctypes.c_int
+    L.tlc_decompress.argtypes = [P, P, S, S, P, P, P]
+    L.tlc_decompress.restype = ctypes.c_int
+    L.tlc_decompress_accumulate.argtypes = [P, P, P, ctypes.c_int, S, P, P, P]
+    L.tlc_decompress_accumulate.restype = ctypes.c_int
+    L.tlc_status_string.argtypes = [ctypes.c_int]
+    L.tlc_status_string.restype = ctypes.c_char_p
+    L.tlc_version.argtypes = []
+    L.tlc_version.restype = ctypes.c_char_p
+    L.tlc_set_wait_limit.argtypes = [ctypes.c_uint32]
+    L.tlc_set_wait_limit.restype = None
+    L.tlc_test_wait_timeout.argtypes = [ctypes.c_uint32, P, P]
+    L.tlc_test_wait_timeout.restype = ctypes.c_int
+    L.tlc_kernel_timing.argtypes = [ctypes.c_int]
+    L.tlc_kernel_timing.restype = None
+    L.tlc_kernel_timing_read.argtypes = [P, P, ctypes.c_int]
+    L.tlc_kernel_timing_read.restype = ctypes.c_int
+    L.tlc_kernel_name.argtypes = [ctypes.c_int]
+    L.tlc_kernel_name.restype = ctypes.c_char_p
+    _ = U64
+    _lib = L
+    return L
+
+
+# ------------------------------------------------------------- marshalling --
+
+def _dev_ptr(t, name: str, dtype=None):
+    """Raw device pointer of a contiguous CUDA tensor (None stays NULL)."""
+    if t is None:
+        return None
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(fn: str, code: int) -> int:
+    if code != OK:
+        raise TLCError(fn, code)
+    return code
+
+
+def status_string(code: int) -> str:
+    return lib().tlc_status_string(code).decode()
+
+
+def version() -> str:
+    return lib().tlc_version().decode()
+
+
+def tlc_compress_bound(n: int) -> int:
+    """4 + ceil(n/5): the largest stream for n values (0 if n is out of range)."""
+    return int(lib().tlc_compress_bound(n))
+
+
+def tlc_compress(x, s: float, err, out, out_len, dev_status=None, stream=None) -> int:
+    """Compress x (fp32, CUDA) with sparsity multiplier s; updates err in place.
+
+    out: uint8 CUDA tensor of at least tlc_compress_bound(x.numel()) bytes;
+    out_len: uint64/int64 CUDA tensor of one element (stream length);
+    dev_status: optional int32 CUDA tensor of one element (set it to 0 first).
+    """
+    import torch
+    n = x.numel()
+    code = lib().tlc_compress(
+        _dev_ptr(x, "x", torch.float32), n, float(s), _dev_ptr(err, "err", torch.float32),
+        _dev_ptr(out, "out", torch.uint8), out.numel(), _dev_ptr(out_len, "out_len"),
+        _dev_ptr(dev_status, "dev_status", torch.int32), _stream(stream))
+    return _check("tlc_compress", code)
+
+
+def tlc_decompress(stream_buf, n: int, y, in_len=None, in_cap=None, dev_status=None,
+                   stream=None) -> int:
+    """Decompress a stream into y (fp32 CUDA tensor of n values).
+
+    in_len: optional one-element uint64/int64 CUDA tensor holding the length;
+    without it, in_cap (default stream_buf.numel()) is the exact length.
+    """
+    import torch
+    cap = stream_buf.numel() if in_cap is None else int(in_cap)
+    code = lib().tlc_decompress(
+        _dev_ptr(stream_buf, "in", torch.uint8), _dev_ptr(in_len, "in_len"), cap, n,
+        _dev_ptr(y, "y", torch.float32), _dev_ptr(dev_status, "dev_status", torch.int32),
+        _stream(stream))
+    return _check("tlc_decompress", code)
+
+
+def tlc_decompress_accumulate(streams, n: int, acc, in_lens=None, in_caps=None,
+                              dev_status=None, stream=None) -> int:
+    """acc += sum over streams (in order) of their decompressed values.
+
+    streams: list of uint8 CUDA tensors; in_lens: optional uint64/int64 CUDA
+    tensor of len(streams) lengths; in_caps: optional list of readable sizes
+    (default each tensor's numel, the exact length when in_lens is None).
+    """
+    import torch
+    k = len(streams)
+    ptrs = (ctypes.c_void_p * k)(*[_dev_ptr(s_, "in", torch.uint8) for s_ in streams])
+    caps_l = [s_.numel() for s_ in streams] if in_caps is None else [int(c) for c in in_caps]
+    caps = (ctypes.c_size_t * k)(*caps_l)
+    code = lib().tlc_decompress_accumulate(
+        ptrs, _dev_ptr(in_lens, "in_lens"), caps, k, n, _dev_ptr(acc, "acc", torch.float32),
+        _dev_ptr(dev_status, "dev_status", torch.int32), _stream(stream))
+    return _check("tlc_decompress_accumulate", code)
+
+
+def tlc_set_wait_limit(max_polls: int) -> None:
+    lib().tlc_set_wait_limit(int(max_polls))
+
+
+def tlc_test_wait_timeout(max_polls: int, dev_status, stream=None) -> int:
+    import torch
+    code = lib().tlc_test_wait_timeout(int(max_polls),
+                                       _dev_ptr(dev_status, "dev_status", torch.int32),
+                                       _stream(stream))
+    return _check("tlc_test_wait_timeout", code)
+
+
+def tlc_kernel_timing(enable: bool) -> None:
+    lib().tlc_kernel_timing(1 if enable else 0)
+
+
+def tlc_kernel_timing_read() -> dict:
+    """{kernel name: (launches, total device ms)} since timing was enabled."""
+    L = lib()
+    k = 8
+    launches = (ctypes.c_uint64 * k)()
+    ms = (ctypes.c_double * k)()
+    nk = L.tlc_kernel_timing_read(launches, ms, k)
+    return {L.tlc_kernel_name(i).decode(): (int(launches[i]), float(ms[i])) for i in range(nk)}
+
+
+# ----------------------------------------------------------- conveniences --
+
+def compress(x, s: float, err, stream=None):
+    """Allocate the outputs and compress: returns (out, out_len, dev_status),
+    all CUDA tensors; nothing is synchronised."""
+    import torch
+    n = x.numel()
+    out = torch.empty(tlc_compress_bound(n), dtype=torch.uint8, device=x.device)
+    out_len = torch.zeros(1, dtype=torch.int64, device=x.device)
+    st = torch.zeros(1, dtype=torch.int32, device=x.device)
+    tlc_compress(x, s, err, out, out_len, st, stream)
+    return out, out_len, st
+
+
+def decompress(stream_buf, n: int, in_len=None, stream=None):
+    """Allocate y and decompress: returns (y, dev_status)."""
+    import torch
+    y = torch.empty(n, dtype=torch.float32, device=stream_buf.device)
+    st = torch.zeros(1, dtype=torch.int32, device=stream_buf.device)
+    tlc_decompress(stream_buf, n, y, in_len=in_len, dev_status=st, stream=stream)
+    return y, st

@@ -253,12 +253,18 @@ static float dequant(int qi, float scale)
     return (float)qi * scale;
 }
 
-/* Decode one stream into q and its scale. */
+/* Decode one stream into q and its scale.  The encoder only writes a
+ * finite, non-negative scale (M >= 0, s >= 1, overflow is refused), so a
+ * header with the sign bit set or an all-ones exponent marks the stream as
+ * corrupt. */
 static int decode_stream(const uint8_t *in, size_t in_len, size_t n,
                          int8_t *q, float *scale_out)
 {
     if (in_len < 4)
         return ORC_INVALID;
+    float sc = get_f32le(in);
+    if (!(isfinite(sc) && !signbit(sc)))
+        return ORC_CORRUPT;
     size_t g = orc_groups(n);
     uint8_t *b = (uint8_t *)malloc(g);
     if (!b)

@@ -19,6 +19,8 @@ base XOR splitmix64(k * 2^20 + t); values and masks use separate streams.
 """
 from __future__ import annotations
 
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 from .gen import (bernoulli, key_for, laplace, normal, splitmix64_mix,
@@ -97,8 +99,10 @@ def tensor_set(cfg: int, step: int, limit: int | None = None):
         shapes = bert_large_shapes()
     else:
         raise ValueError(f"config {cfg} is a flat tensor")
-    out = []
-    for t, shp in enumerate(shapes[:limit] if limit else shapes):
+    todo = list(enumerate(shapes[:limit] if limit else shapes))
+
+    def one(item):
+        t, shp = item
         seed = tensor_seed(0, step, t)
         n = _numel(shp)
         x = normal(key_for(seed, P_VALUES), n, 1e-3)
@@ -107,8 +111,11 @@ def tensor_set(cfg: int, step: int, limit: int | None = None):
         elif t == 0:   # word embedding: whole rows zero with p = 0.99
             rows = bernoulli(key_for(seed, P_MASK), shp[0], 0.99)
             x.reshape(shp)[rows, :] = 0.0
-        out.append(x)
-    return out
+        return x
+
+    # tensors are independent; a separate pool from the chunk pool in gen.py
+    with ThreadPoolExecutor(4) as pool:
+        return list(pool.map(one, todo))
 
 
 def config_step_inputs(cfg: int, step: int = 0):

@@ -1,13 +1,36 @@
 """Counter-based random streams (splitmix64) and the distributions built on them."""
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 
 MASK64 = (1 << 64) - 1
 GOLDEN_RATIO64 = 0x9E3779B97F4A7C15
 _M1 = np.uint64(0xBF58476D1CE4E5B9)
 _M2 = np.uint64(0x94D049BB133111EB)
-_CHUNK = 1 << 22
+_CHUNK = 1 << 20
+_POOL = None
+
+
+def _threads() -> int:
+    return max(1, min(16, os.cpu_count() or 1))
+
+
+def _chunked(count: int, fill) -> None:
+    """Run fill(a, b) over [0, count) in chunks, in parallel threads (numpy
+    releases the GIL).  Every chunk depends only on its own counters, so the
+    result does not depend on the thread count."""
+    global _POOL
+    spans = [(a, min(count, a + _CHUNK)) for a in range(0, count, _CHUNK)]
+    if len(spans) <= 1:
+        for a, b in spans:
+            fill(a, b)
+        return
+    if _POOL is None:
+        _POOL = ThreadPoolExecutor(_threads())
+    list(_POOL.map(lambda ab: fill(*ab), spans))
 
 
 def splitmix64_mix(z):
@@ -46,42 +69,49 @@ def _raw(key: int, start: int, count: int) -> np.ndarray:
 def uniforms(key: int, count: int, start: int = 0) -> np.ndarray:
     """float64 uniforms in (0, 1) from stream `key`."""
     out = np.empty(count, np.float64)
-    for a in range(0, count, _CHUNK):
-        b = min(count, a + _CHUNK)
+
+    def fill(a, b):
         r = _raw(key, start + a, b - a)
         out[a:b] = ((r >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
+    _chunked(count, fill)
     return out
 
 
 def normal(key: int, count: int, sigma: float) -> np.ndarray:
     """fp32 N(0, sigma^2) by Box-Muller (uniform pairs 2i, 2i+1)."""
     out = np.empty(count, np.float32)
-    for a in range(0, count, _CHUNK):
-        b = min(count, a + _CHUNK)
-        u = uniforms(key, 2 * (b - a), start=2 * a)
+
+    def fill(a, b):
+        r = _raw(key, 2 * a, 2 * (b - a))
+        u = ((r >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53)
         u1, u2 = u[0::2], u[1::2]
         z = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
         out[a:b] = (sigma * z).astype(np.float32)
+    _chunked(count, fill)
     return out
 
 
 def laplace(key: int, count: int, b_scale: float) -> np.ndarray:
     """fp32 Laplace(0, b) by the inverse CDF."""
     out = np.empty(count, np.float32)
-    for a in range(0, count, _CHUNK):
-        b = min(count, a + _CHUNK)
-        u = uniforms(key, b - a, start=a) - 0.5
+
+    def fill(a, b):
+        r = _raw(key, a, b - a)
+        u = ((r >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53) - 0.5
         v = -b_scale * np.sign(u) * np.log1p(-2.0 * np.abs(u))
         out[a:b] = v.astype(np.float32)
+    _chunked(count, fill)
     return out
 
 
 def bernoulli(key: int, count: int, p: float) -> np.ndarray:
     """bool mask, True with probability p."""
     out = np.empty(count, bool)
-    for a in range(0, count, _CHUNK):
-        b = min(count, a + _CHUNK)
-        out[a:b] = uniforms(key, b - a, start=a) < p
+
+    def fill(a, b):
+        r = _raw(key, a, b - a)
+        out[a:b] = ((r >> np.uint64(11)).astype(np.float64) + 0.5) * (2.0 ** -53) < p
+    _chunked(count, fill)
     return out
 
 

@@ -1,0 +1,426 @@
+"""CUDA path against the CPU oracle, element by element (needs a B200).
+
+Everything goes through the C ABI (libtlc.so) via its Python binding.  The
+bar is bit-exactness: the stream bytes and length, the updated error buffer,
+the decompressed values and the accumulated sums must equal the oracle's on
+the same seeded inputs.  Output buffers carry guard bytes to catch any write
+outside them.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from conftest import load_quantizer_cases
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+GUARD = 256
+CANARY = 0xA5
+
+
+@pytest.fixture(scope="module")
+def g():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import gradient_traffic_compression_b200 as g
+    g.lib()
+    return g
+
+
+def bits(a):
+    return np.ascontiguousarray(a, np.float32).view(np.uint32)
+
+
+def _dev_f32(a, offset=0):
+    """fp32 CUDA copy of `a`; offset > 0 shifts the start by that many
+    floats (offset 1 makes the pointer 4- but not 16-byte aligned)."""
+    buf = torch.empty(a.size + offset, dtype=torch.float32, device="cuda")
+    t = buf[offset:]
+    t.copy_(torch.from_numpy(np.ascontiguousarray(a, np.float32)))
+    return t
+
+
+def _guarded_f32(n, offset=0):
+    buf = torch.full((n + 2 * GUARD + offset,), float("nan"), dtype=torch.float32, device="cuda")
+    buf.view(torch.int32).fill_(0x7FA5A5A5)
+    return buf, buf[GUARD + offset:GUARD + offset + n]
+
+
+def _check_f32_guards(buf, n, offset=0):
+    raw = buf.view(torch.int32).cpu().numpy()
+    assert np.all(raw[:GUARD + offset] == 0x7FA5A5A5)
+    assert np.all(raw[GUARD + offset + n:] == 0x7FA5A5A5)
+
+
+def gpu_compress(g, x, s, err, offset=0):
+    """(status, stream, err', out_len) through tlc_compress."""
+    n = x.size
+    xt, et = _dev_f32(x, offset), _dev_f32(err, offset)
+    cap = g.tlc_compress_bound(n)
+    obuf = torch.full((cap + 2 * GUARD,), CANARY, dtype=torch.uint8, device="cuda")
+    out = obuf[GUARD:GUARD + cap]
+    out_len = torch.zeros(1, dtype=torch.int64, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g.tlc_compress(xt, s, et, out, out_len, st)
+    torch.cuda.synchronize()
+    L = int(out_len.item())
+    ob = obuf.cpu().numpy()
+    assert np.all(ob[:GUARD] == CANARY)
+    assert np.all(ob[GUARD + L:] == CANARY), "write past the stream end"
+    assert np.array_equal(xt.cpu().numpy().view(np.uint32), bits(x)), "x was modified"
+    return int(st.item()), ob[GUARD:GUARD + L].copy(), et.cpu().numpy(), L
+
+
+def gpu_decompress(g, stream, n, offset=0, in_len=None, cap=None):
+    buf, y = _guarded_f32(n, offset)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cap = stream.size if cap is None else cap
+    sb = torch.full((max(cap, 1),), CANARY, dtype=torch.uint8, device="cuda")
+    if stream.size:
+        sb[:stream.size].copy_(torch.from_numpy(stream))
+    lt = None
+    if in_len is not None:
+        lt = torch.tensor([in_len], dtype=torch.int64, device="cuda")
+    g.tlc_decompress(sb[:cap] if cap else sb[:0], n, y, in_len=lt, in_cap=cap, dev_status=st)
+    torch.cuda.synchronize()
+    _check_f32_guards(buf, n, offset)
+    return int(st.item()), y.cpu().numpy()
+
+
+def gpu_accumulate(g, streams, n, acc0, offset=0, device_lens=False):
+    buf, acc = _guarded_f32(n, offset)
+    acc.copy_(torch.from_numpy(np.ascontiguousarray(acc0, np.float32)))
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ts = [torch.from_numpy(np.ascontiguousarray(s_, np.uint8)).cuda() for s_ in streams]
+    lens = None
+    caps = None
+    if device_lens:
+        lens = torch.tensor([s_.size for s_ in streams], dtype=torch.int64, device="cuda")
+        ts = [torch.cat([t, torch.full((37,), CANARY, dtype=torch.uint8, device="cuda")])
+              for t in ts]
+        caps = [t.numel() for t in ts]
+    g.tlc_decompress_accumulate(ts, n, acc, in_lens=lens, in_caps=caps, dev_status=st)
+    torch.cuda.synchronize()
+    _check_f32_guards(buf, n, offset)
+    return int(st.item()), acc.cpu().numpy()
+
+
+def assert_compress_parity(g, x, s, err, offset=0):
+    rc_o, st_o, e_o = oracle.compress(x, s, err)
+    rc_g, st_g, e_g, L = gpu_compress(g, x, s, err, offset)
+    assert rc_g == rc_o
+    assert L == st_o.size
+    if not np.array_equal(st_g, st_o):
+        i = int(np.argmax(st_g[:min(st_g.size, st_o.size)] != st_o[:min(st_g.size, st_o.size)]))
+        raise AssertionError(f"stream differs at byte {i} of {st_o.size}: "
+                             f"gpu {st_g[max(0, i - 4):i + 8]} oracle {st_o[max(0, i - 4):i + 8]}")
+    d = np.flatnonzero(bits(e_g) != bits(e_o))
+    assert d.size == 0, f"err differs at {d[:8]}: gpu {e_g[d[:4]]} oracle {e_o[d[:4]]}"
+    return st_o, e_o
+
+
+def assert_roundtrip_parity(g, stream, n, offset=0):
+    rc_o, y_o = oracle.decompress(stream, n)
+    rc_g, y_g = gpu_decompress(g, stream, n, offset)
+    assert rc_g == rc_o
+    d = np.flatnonzero(bits(y_g) != bits(y_o))
+    assert d.size == 0, f"y differs at {d[:8]}"
+
+
+def mixed_case(seed, n, zero_frac=0.6):
+    x = synth.normal(synth.key_for(seed, 0), n, 1e-3)
+    x[synth.bernoulli(synth.key_for(seed, 3), n, zero_frac)] = 0.0
+    err = synth.laplace(synth.key_for(seed, 1), n, 3e-4)
+    s = float(np.float32(1.0 + 0.999 * synth.uniforms(synth.key_for(seed, 2), 1)[0]))
+    return x, err, s
+
+
+# ------------------------------------------------------------------ cases --
+
+TILE_VALUES = 20480          # compress tile: 4096 groups
+RAGGED = sorted(set(
+    list(range(1, 13)) + [19, 20, 21, 39, 40, 41, 639, 640, 641, 5119, 5120, 5121,
+                          TILE_VALUES - 1, TILE_VALUES, TILE_VALUES + 1, TILE_VALUES + 5,
+                          2 * TILE_VALUES - 3, 2 * TILE_VALUES + 17, 3 * TILE_VALUES + 4,
+                          5 * 2048 * 14 + 3, 131071, 131072, 131073]))
+
+
+@pytest.mark.parametrize("n", RAGGED)
+def test_ragged_sizes(g, n):
+    x, err, s = mixed_case(1000 + n, n)
+    st, _ = assert_compress_parity(g, x, s, err)
+    assert_roundtrip_parity(g, st, n)
+
+
+def test_random_sizes_cover_every_tail(g):
+    key = synth.key_for(77, 1)
+    ns = (1 + synth.uniforms(key, 80) * 5000).astype(int)
+    ns = sorted(set(ns.tolist()) | set(range(4980, 5000)))
+    assert {n % 20 for n in ns} == set(range(20))
+    for n in ns:
+        x, err, s = mixed_case(2000 + n, n, zero_frac=0.3 + 0.6 * ((n * 7) % 10) / 10)
+        st, _ = assert_compress_parity(g, x, s, err)
+        assert_roundtrip_parity(g, st, n)
+
+
+@pytest.mark.parametrize("case", load_quantizer_cases(), ids=lambda c: c["name"])
+def test_golden_cases_on_gpu(g, case):
+    rc, st, e, L = gpu_compress(g, case["x"], case["s"], case["err"])
+    assert rc == case["status"]
+    assert st.tolist() == case["stream"].tolist()
+    assert np.array_equal(bits(e), bits(case["err_out"]))
+    if rc == 0:
+        assert_roundtrip_parity(g, st, case["x"].size)
+
+
+def _literal_groups_case(n, groups):
+    """x = 0 except +-1 at the first value of each listed group (M = 1, s = 1):
+    the quartic bytes are 121 everywhere else."""
+    x = np.zeros(n, np.float32)
+    for k, gi in enumerate(groups):
+        x[5 * gi] = 1.0 if k % 2 == 0 else -1.0
+    return x
+
+
+RUN_CASES = {
+    # runs that end exactly at, just past, or far past compress tile edges
+    # (4096 groups per tile), with lengths = 0, 1, 13 (mod 14) on each side
+    "edge_mod0": [4096 - 15, 4096 + 13],
+    "edge_mod1": [4096 - 16, 4096 + 14],
+    "edge_mod13": [4096 - 14, 4096 + 12],
+    "end_at_edge": [4096 - 1, 4096, 8191],
+    "start_at_edge": [4095, 4096 + 27],
+    "span_many_tiles": [100, 4096 * 5 + 57],
+    "span_exact_tiles": [4095, 4096 * 3 - 1],
+    "long_tail_run": [3],
+    "long_head_run": [4096 * 4 + 1],
+    "dense_then_empty": list(range(0, 300)) + [4096 * 2 + 7],
+}
+
+
+@pytest.mark.parametrize("name", list(RUN_CASES))
+def test_runs_across_tiles(g, name):
+    groups = RUN_CASES[name]
+    n = 5 * (4096 * 6 + 11) + 3
+    x = _literal_groups_case(n, groups)
+    st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
+    assert_roundtrip_parity(g, st, n)
+
+
+@pytest.mark.parametrize("tail", [0, 1, 13, 14, 15, 27, 28])
+def test_run_lengths_at_stream_end(g, tail):
+    gtot = 4096 * 2 + tail + 1
+    n = 5 * gtot
+    x = _literal_groups_case(n, [gtot - tail - 1])     # then `tail` zero groups
+    st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
+    assert_roundtrip_parity(g, st, n)
+
+
+def test_all_zero_and_single_values(g):
+    for n in (1, 5, 70, 71, 4096 * 5, 4096 * 5 * 3 + 1):
+        st, _ = assert_compress_parity(g, np.zeros(n, np.float32), 1.0, np.zeros(n, np.float32))
+        assert_roundtrip_parity(g, st, n)
+    x = np.zeros(100003, np.float32)
+    x[100002] = -3.0
+    st, _ = assert_compress_parity(g, x, 1.5, np.zeros(x.size, np.float32))
+    assert_roundtrip_parity(g, st, x.size)
+
+
+def test_config1_full(g):
+    x = synth.flat_tensor(1)
+    err = np.zeros_like(x)
+    st, e = assert_compress_parity(g, x, 1.0, err)
+    assert_roundtrip_parity(g, st, x.size)
+    acc0 = synth.normal(synth.key_for(11, 0), x.size, 1e-3)
+    rc_o, a_o = oracle.decompress_accumulate([st], x.size, acc0)
+    rc_g, a_g = gpu_accumulate(g, [st], x.size, acc0)
+    assert rc_g == rc_o == 0 and np.array_equal(bits(a_g), bits(a_o))
+
+
+def test_config2_twenty_steps(g):
+    shapes = synth.resnet110_conv_shapes()
+    errs = [np.zeros(int(np.prod(s_)), np.float32) for s_ in shapes]
+    for step in range(20):
+        xs = synth.tensor_set(2, step)
+        for t, x in enumerate(xs):
+            st, errs[t] = assert_compress_parity(g, x, 1.75, errs[t])
+            if t % 27 == 0:
+                assert_roundtrip_parity(g, st, x.size)
+
+
+@pytest.mark.parametrize("log2n", list(range(20, 25)))
+def test_config3_sweep(g, log2n):
+    n = 1 << log2n
+    x = synth.flat_tensor(3, n=n)
+    st, _ = assert_compress_parity(g, x, 1.9, np.zeros(n, np.float32))
+    assert_roundtrip_parity(g, st, n)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("log2n", [25, 26, 27, 28])
+def test_config3_sweep_large(g, log2n):
+    n = 1 << log2n
+    x = synth.flat_tensor(3, n=n)
+    st, _ = assert_compress_parity(g, x, 1.9, np.zeros(n, np.float32))
+    assert_roundtrip_parity(g, st, n)
+
+
+@pytest.mark.slow
+def test_config4_five_steps(g):
+    shapes = synth.bert_large_shapes()
+    errs = [np.zeros(int(np.prod(s_)), np.float32) for s_ in shapes]
+    for step in range(5):
+        xs = synth.tensor_set(4, step)
+        for t, x in enumerate(xs):
+            st, errs[t] = assert_compress_parity(g, x, 1.5, errs[t])
+            if t in (0, 5, 390):
+                assert_roundtrip_parity(g, st, x.size)
+
+
+def test_config5_accumulate_k8(g):
+    n = synth.CONFIGS[5]["n"]
+    streams = []
+    for w in range(8):
+        x = synth.flat_tensor(5, worker=w)
+        rc, st, _ = oracle.compress(x, 1.75, np.zeros(n, np.float32))
+        assert rc == 0
+        streams.append(st)
+    # the GPU encoder gives the same bytes for one worker (checked in full)
+    assert_compress_parity(g, synth.flat_tensor(5, worker=3), 1.75, np.zeros(n, np.float32))
+    acc0 = np.zeros(n, np.float32)
+    rc_o, a_o = oracle.decompress_accumulate(streams, n, acc0)
+    rc_g, a_g = gpu_accumulate(g, streams, n, acc0)
+    assert rc_o == rc_g == 0
+    assert np.array_equal(bits(a_g), bits(a_o))
+
+
+def test_accumulate_dense_streams_and_device_lengths(g):
+    n = 300_001
+    streams = []
+    for w in range(5):
+        x, err, s = mixed_case(500 + w, n, zero_frac=0.1)
+        streams.append(oracle.compress(x, 1.0, err)[1])
+    acc0 = synth.normal(synth.key_for(12, 0), n, 1e-3)
+    acc0[::5] = -0.0
+    rc_o, a_o = oracle.decompress_accumulate(streams, n, acc0)
+    for dl in (False, True):
+        rc_g, a_g = gpu_accumulate(g, streams, n, acc0, device_lens=dl)
+        assert rc_g == rc_o == 0 and np.array_equal(bits(a_g), bits(a_o))
+
+
+@pytest.mark.parametrize("offset", [1, 2, 3])
+def test_unaligned_pointers(g, offset):
+    n = 3 * TILE_VALUES + 123
+    x, err, s = mixed_case(42 + offset, n)
+    st, _ = assert_compress_parity(g, x, s, err, offset=offset)
+    assert_roundtrip_parity(g, st, n, offset=offset)
+    acc0 = synth.normal(synth.key_for(13, offset), n, 1e-3)
+    rc_o, a_o = oracle.decompress_accumulate([st, st], n, acc0)
+    rc_g, a_g = gpu_accumulate(g, [st, st], n, acc0, offset=offset)
+    assert rc_g == rc_o == 0 and np.array_equal(bits(a_g), bits(a_o))
+
+
+def test_device_side_length(g):
+    n = 77_777
+    x, err, s = mixed_case(9, n)
+    _, st, _ = oracle.compress(x, s, err)
+    rc_o, y_o = oracle.decompress(st, n)
+    padded = np.concatenate([st, np.full(50, CANARY, np.uint8)])
+    rc_g, y_g = gpu_decompress(g, padded, n, in_len=st.size, cap=padded.size)
+    assert rc_g == 0 and np.array_equal(bits(y_g), bits(y_o))
+    # a device length beyond the capacity is corrupt, not an overrun
+    rc_g, _ = gpu_decompress(g, padded, n, in_len=padded.size + 1, cap=padded.size)
+    assert rc_g == 3
+
+
+def test_nonfinite_inputs(g):
+    n = 50_000
+    for where, val in (("x", np.nan), ("x", np.inf), ("err", -np.inf), ("x", -np.nan)):
+        x, err, s = mixed_case(3, n)
+        (x if where == "x" else err)[31_337] = val
+        rc, st, e, L = gpu_compress(g, x, s, err)
+        assert rc == 2 and L == 0
+        assert np.array_equal(bits(e), bits(err))          # err untouched
+    x = np.zeros(n, np.float32)
+    x[7] = 3e38
+    rc, st, e, L = gpu_compress(g, x, 1.5, np.zeros(n, np.float32))
+    assert rc == 2 and L == 0                               # M*s overflows
+
+
+def test_corrupt_streams(g):
+    n = 40_000
+    x, err, s = mixed_case(5, n)
+    _, st, _ = oracle.compress(x, s, err)
+    key = synth.key_for(99, 0)
+    cases = {
+        "truncated": st[:-1],
+        "truncated_more": st[: st.size // 2],
+        "extended": np.concatenate([st, np.array([7], np.uint8)]),
+        "extra_escape": np.concatenate([st[:-1], np.array([255], np.uint8)]),
+        "negative_scale": np.concatenate([st[:3], np.array([st[3] | 0x80], np.uint8), st[4:]]),
+        "nan_scale": np.concatenate([np.array([0, 0, 0xC0, 0x7F], np.uint8), st[4:]]),
+        "header_only": st[:4],
+    }
+    for trial in range(10):
+        flip = st.copy()
+        pos = 4 + int(synth.uniforms(key, 1, start=trial)[0] * (st.size - 4))
+        flip[pos] = 243 + (trial % 13)
+        cases[f"flip{trial}"] = flip
+    for name, bad in cases.items():
+        rc_o, _ = oracle.decompress(bad, n)
+        if bad.size - 4 > (n + 4) // 5:
+            continue                                        # host rejects this length
+        rc_g, _ = gpu_decompress(g, bad, n)
+        assert rc_g == rc_o, name
+        rc_ga, _ = gpu_accumulate(g, [bad], n, np.zeros(n, np.float32))
+        assert rc_ga == rc_o, name
+
+
+def test_deterministic_over_repeats(g):
+    n = 4_000_000
+    x, err, s = mixed_case(17, n, zero_frac=0.5)
+    first = gpu_compress(g, x, s, err)
+    for _ in range(20):
+        again = gpu_compress(g, x, s, err)
+        assert again[1].tolist() == first[1].tolist()
+        assert np.array_equal(bits(again[2]), bits(first[2]))
+
+
+def test_checkpoint_resume(g):
+    n = 36_864
+    err = np.zeros(n, np.float32)
+    xs = [synth.normal(synth.key_for(400 + k, 0), n, 1e-3) for k in range(12)]
+    for k in range(10):
+        _, _, err, _ = gpu_compress(g, xs[k], 1.75, err)
+    saved = err.copy()
+    _, s1, e1, _ = gpu_compress(g, xs[10], 1.75, err)
+    _, s2, e2, _ = gpu_compress(g, xs[10], 1.75, saved)
+    assert s1.tolist() == s2.tolist() and np.array_equal(bits(e1), bits(e2))
+
+
+def test_status_word_keeps_first_error(g):
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    bad = torch.tensor([0, 0, 0x80, 0xBF, 1], dtype=torch.uint8, device="cuda")   # scale -1
+    y = torch.empty(5, dtype=torch.float32, device="cuda")
+    g.tlc_decompress(bad, 5, y, dev_status=st)
+    x = torch.tensor([1.0, float("nan")], device="cuda")
+    e = torch.zeros(2, device="cuda")
+    out = torch.empty(g.tlc_compress_bound(2), dtype=torch.uint8, device="cuda")
+    ln = torch.zeros(1, dtype=torch.int64, device="cuda")
+    g.tlc_compress(x, 1.0, e, out, ln, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 3
+
+
+def test_bounded_wait_reports_timeout(g):
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g.tlc_test_wait_timeout(64, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 4
+    # the context is still usable afterwards
+    x, err, s = mixed_case(1, 1000)
+    assert_compress_parity(g, x, s, err)

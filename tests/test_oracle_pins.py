@@ -280,6 +280,13 @@ def test_decompress_flags_corrupt_and_short(orc):
     assert orc.decompress(st[:3], 6)[0] == orc.INVALID    # no full header
 
 
+def test_decompress_rejects_headers_the_encoder_cannot_write(orc):
+    for bad in (-1.0, -0.0, float("inf"), float("nan")):
+        st = _hand_stream([1, 0, 0, 0, 0], bad)
+        assert orc.decompress(st, 5)[0] == orc.CORRUPT
+        assert orc.decompress_accumulate([st], 5, np.zeros(5, np.float32))[0] == orc.CORRUPT
+
+
 def test_accumulate_exact_on_power_of_two_scales(orc):
     n, scales = 503, [0.5, 0.25, 1.0, 2.0]
     key = synth.key_for(77, 0)
