@@ -38,7 +38,7 @@ S_PARAM = 1.9
 def parse_args():
     p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--steps", type=int, default=400)
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--log2n", type=int, default=28, help="tensor size 2^k (default 28)")
@@ -81,7 +81,7 @@ def workload_config(n, log2n):
 # ----------------------------------------------------------- clock sampler --
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -97,9 +97,14 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def mark(self, which):
+        """Record the host time at which the timed region starts / ends."""
+        setattr(self, which, time.time())
+
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.06)
         self.proc.terminate()
         try:
             self.proc.wait(5)
@@ -109,6 +114,18 @@ class ClockSampler:
         self.tmp.seek(0)
         rows = [r.split(",") for r in self.tmp.read().strip().splitlines() if r.count(",") >= 8]
         os.unlink(self.tmp.name)
+        t0, t1 = getattr(self, "start", None), getattr(self, "end", None)
+        if t0 is not None and t1 is not None:
+            import datetime as _dt
+            kept = []
+            for r in rows:
+                try:
+                    ts = _dt.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                except ValueError:
+                    continue
+                if t0 - 0.03 <= ts <= t1 + 0.03:
+                    kept.append(r)
+            rows = kept or rows
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
@@ -161,7 +178,9 @@ def run_ours(args, rank, world, local):
 
     bus = None
     try:
-        bus = torch.cuda.get_device_properties(dev).pci_bus_id
+        pr = torch.cuda.get_device_properties(dev)
+        bus = "%08X:%02X:%02X.0" % (int(pr.pci_domain_id), int(pr.pci_bus_id),
+                                    int(pr.pci_device_id))
     except Exception:
         bus = None
 
@@ -171,8 +190,9 @@ def run_ours(args, rank, world, local):
         dist.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(bus)
-    time.sleep(0.15)
+    time.sleep(0.2)
     tlc.tlc_kernel_timing(True)
+    sampler.mark("start")
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -189,6 +209,7 @@ def run_ours(args, rank, world, local):
         e[3].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
+    sampler.mark("end")
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
