@@ -171,16 +171,31 @@ __device__ __forceinline__ uint8_t remainder_byte(uint32_t r) {
   return r == 1 ? uint8_t(121) : uint8_t(241 + r);
 }
 
+// Rounding without the division.  With r = fl(x'/scale) the correctly
+// rounded quotient and |x'| <= M <= scale, q = round(r) is non-zero exactly
+// when fl(|x'|/scale) >= 1/2.  The fp32 neighbour below 1/2 is 1/2 - 2^-25,
+// and the midpoint 1/2 - 2^-26 rounds to 1/2 (its even neighbour), so
+//   fl(|x'|/scale) >= 1/2  <=>  |x'|/scale >= 1/2 - 2^-26
+//                          <=>  |x'| >= scale * (1/2 - 2^-26)   (exact reals)
+//                          <=>  |x'| >= T,  T = the least fp32 value that is
+//                                            >= scale * (1/2 - 2^-26).
+// scale has 24 significant bits and 1/2 - 2^-26 has 25, so the product is
+// exact in fp64 and T is that product rounded towards +infinity.  The test
+// gives the same q as the division for every input, subnormals included.
+// M = 0 uses T = +inf (every q = 0, no division).
+__device__ __forceinline__ float zero_band_threshold(float scale, bool mzero) {
+  if (mzero) return __int_as_float(0x7f800000);
+  const double t = __dmul_rn((double)scale, 0.5 - 0x1p-26);
+  return __double2float_ru(t);
+}
+
 // One element: digit q+1 of round(x'/scale) with ties away from zero, and
-// the updated error x' - q*scale.  M = 0 gives q = 0 with no division.
-__device__ __forceinline__ uint32_t quant_digit(float xp, float scale, bool mzero, float &e) {
-  uint32_t d = 1;
-  if (!mzero) {
-    const float r = __fdiv_rn(xp, scale);
-    if (fabsf(r) >= 0.5f) d = (r > 0.0f) ? 2u : 0u;
-  }
-  e = (d == 1) ? xp : __fsub_rn(xp, d == 2 ? scale : -scale);
-  return d;
+// the updated error x' - q*scale.
+__device__ __forceinline__ uint32_t quant_digit(float xp, float scale, float thr, float &e) {
+  const bool nz = fabsf(xp) >= thr;
+  const bool neg = __float_as_uint(xp) >> 31;
+  e = nz ? __fsub_rn(xp, neg ? -scale : scale) : xp;
+  return nz ? (neg ? 0u : 2u) : 1u;
 }
 
 // Quartic byte of five digits, first digit most significant (Horner in base 3).
@@ -219,6 +234,88 @@ struct QuantArgs {
 
 __device__ __forceinline__ void put_out(const QuantArgs &a, uint64_t pos, uint8_t v) {
   if (4 + pos < a.out_cap) a.out[4 + pos] = v;
+}
+
+// Decoupled look-back for tile t (whole block calls; warp 0 works): publish
+// the tile's aggregate, combine earlier tiles' words until an inclusive
+// prefix is found, publish this tile's inclusive prefix, and return the
+// exclusive prefix (emitted count, incoming run length mod 14) to all threads.
+__device__ __forceinline__ void lookback_tile(const QuantArgs &a, uint32_t t, const ZAgg &agg,
+                                              uint32_t &cin, uint32_t &tin, uint32_t &cin_s,
+                                              uint32_t &tin_s) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp == 0) {
+    if (t == 0) {
+      if (lane == 0) {
+        uint32_t C = 0, tt = 0;
+        eval_agg(C, tt, agg);
+        st_relaxed_u64(a.status, pack_prefix(C, tt));
+        cin_s = 0;
+        tin_s = 0;
+      }
+    } else {
+      if (lane == 0) st_relaxed_u64(a.status + t, pack_agg(agg));
+      bool timed_out = false;
+      bool have_suffix = false;
+      ZAgg suffix = {0, 0, 0, 0};
+      int64_t end = (int64_t)t - 1;
+      uint32_t C = 0, tt = 0;
+      for (;;) {
+        const int64_t idx = end - lane;
+        const uint64_t w =
+            idx >= 0 ? wait_flag(a.status + idx, a.max_polls, timed_out) : pack_prefix(0, 0);
+        const uint32_t pmask = __ballot_sync(0xffffffffu, (w >> kFlagShift) == 2);
+        if (pmask) {
+          const int pl = __ffs(pmask) - 1;
+          const uint64_t wp = __shfl_sync(0xffffffffu, w, pl);
+          C = (uint32_t)(wp & 0xffffffffu);
+          tt = (uint32_t)((wp >> 32) & 0xfu);
+          for (int l = pl - 1; l >= 0; --l) {
+            const uint64_t wl = __shfl_sync(0xffffffffu, w, l);
+            eval_agg(C, tt, unpack_agg(wl));
+          }
+          if (have_suffix) eval_agg(C, tt, suffix);
+          break;
+        }
+        ZAgg acc = unpack_agg(__shfl_sync(0xffffffffu, w, 31));
+        for (int l = 30; l >= 0; --l)
+          acc = compose(acc, unpack_agg(__shfl_sync(0xffffffffu, w, l)));
+        suffix = have_suffix ? compose(acc, suffix) : acc;
+        have_suffix = true;
+        end -= kWarp;
+      }
+      if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(a.dev_status, TLC_ERR_TIMEOUT);
+      if (lane == 0) {
+        cin_s = C;
+        tin_s = tt;
+        uint32_t Ci = C, ti = tt;
+        eval_agg(Ci, ti, agg);
+        st_relaxed_u64(a.status + t, pack_prefix(Ci, ti));
+      }
+    }
+  }
+  __syncthreads();
+  cin = cin_s;
+  tin = tin_s;
+}
+
+// Stream header (first tile) and the closing remainder + length (last tile).
+__device__ __forceinline__ void finish_tile(const QuantArgs &a, uint32_t t, const ZAgg &agg,
+                                            uint32_t cin, uint32_t tin, float scale) {
+  if (threadIdx.x != 0) return;
+  if (t == 0) {
+    const uint32_t sb = __float_as_uint(scale);
+    a.out[0] = sb & 0xff;
+    a.out[1] = (sb >> 8) & 0xff;
+    a.out[2] = (sb >> 16) & 0xff;
+    a.out[3] = (sb >> 24) & 0xff;
+  }
+  if (t == a.n_tiles - 1) {
+    uint32_t C = cin, tt = tin;
+    eval_agg(C, tt, agg);
+    if (tt) put_out(a, C, remainder_byte(tt));
+    *a.out_len = 4ull + C + (tt ? 1u : 0u);
+  }
 }
 
 template <bool kVec>
@@ -261,7 +358,7 @@ k_quant_zre(const QuantArgs a) {
     return;
   }
   const float scale = scale_s;
-  const bool mzero = state_s == 1;
+  const float thr = zero_band_threshold(scale, state_s == 1);
 
   for (;;) {
     if (threadIdx.x == 0) {
@@ -295,10 +392,10 @@ k_quant_zre(const QuantArgs a) {
         for (int j = 0; j < 5; ++j) {
           float4 o;
           uint32_t dw;
-          dw = quant_digit(__fadd_rn(xv[j].x, ev[j].x), scale, mzero, o.x);
-          dw |= quant_digit(__fadd_rn(xv[j].y, ev[j].y), scale, mzero, o.y) << 8;
-          dw |= quant_digit(__fadd_rn(xv[j].z, ev[j].z), scale, mzero, o.z) << 16;
-          dw |= quant_digit(__fadd_rn(xv[j].w, ev[j].w), scale, mzero, o.w) << 24;
+          dw = quant_digit(__fadd_rn(xv[j].x, ev[j].x), scale, thr, o.x);
+          dw |= quant_digit(__fadd_rn(xv[j].y, ev[j].y), scale, thr, o.y) << 8;
+          dw |= quant_digit(__fadd_rn(xv[j].z, ev[j].z), scale, thr, o.z) << 16;
+          dw |= quant_digit(__fadd_rn(xv[j].w, ev[j].w), scale, thr, o.w) << 24;
           err4[lane + 32 * j] = o;
           dig_s[warp][lane + 32 * j] = dw;
         }
@@ -312,7 +409,7 @@ k_quant_zre(const QuantArgs a) {
             uint32_t d = 1;
             if (e < a.n) {
               float o;
-              d = quant_digit(__fadd_rn(a.x[e], a.err[e]), scale, mzero, o);
+              d = quant_digit(__fadd_rn(a.x[e], a.err[e]), scale, thr, o);
               a.err[e] = o;
             }
             dw |= d << (8 * k);
@@ -332,6 +429,20 @@ k_quant_zre(const QuantArgs a) {
     // ---- zero-run encoding: local analysis -----------------------------
     const uint4 q4 = reinterpret_cast<const uint4 *>(tile_s)[threadIdx.x];
     const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
+    // groups past the end of the tensor are all-zero (121) by construction
+    const bool tile_all = __syncthreads_and(q4.x == 0x79797979u && q4.y == 0x79797979u &&
+                                            q4.z == 0x79797979u && q4.w == 0x79797979u);
+    if (tile_all) {
+      // Entirely 121s: only full 14-chunks of the run end inside the tile.
+      ZAgg agg = {1u, tgv, 0u, 0u};
+      uint32_t cin, tin;
+      lookback_tile(a, t, agg, cin, tin, cin_s, tin_s);
+      const uint32_t cnt = (tin + tgv) / 14u;
+      for (uint32_t i = threadIdx.x; i < cnt; i += kQThreads) put_out(a, (uint64_t)cin + i, 255);
+      finish_tile(a, t, agg, cin, tin, scale);
+      __syncthreads();
+      continue;
+    }
     const int p0 = (int)threadIdx.x * kZBytes;
     int fnz = -1, lnz = -1;
 #pragma unroll
@@ -374,58 +485,8 @@ k_quant_zre(const QuantArgs a) {
     agg.tc = agg.all ? 0u : (uint32_t)((int)tgv - 1 - lnz_all) % 14u;
 
     // ---- decoupled look-back -------------------------------------------
-    if (warp == 0) {
-      if (t == 0) {
-        if (lane == 0) {
-          uint32_t C = 0, tt = 0;
-          eval_agg(C, tt, agg);
-          st_relaxed_u64(a.status, pack_prefix(C, tt));
-          cin_s = 0;
-          tin_s = 0;
-        }
-      } else {
-        if (lane == 0) st_relaxed_u64(a.status + t, pack_agg(agg));
-        bool timed_out = false;
-        bool have_suffix = false;
-        ZAgg suffix = {0, 0, 0, 0};
-        int64_t end = (int64_t)t - 1;
-        uint32_t C = 0, tt = 0;
-        for (;;) {
-          const int64_t idx = end - lane;
-          const uint64_t w =
-              idx >= 0 ? wait_flag(a.status + idx, a.max_polls, timed_out) : pack_prefix(0, 0);
-          const uint32_t pmask = __ballot_sync(0xffffffffu, (w >> kFlagShift) == 2);
-          if (pmask) {
-            const int pl = __ffs(pmask) - 1;
-            const uint64_t wp = __shfl_sync(0xffffffffu, w, pl);
-            C = (uint32_t)(wp & 0xffffffffu);
-            tt = (uint32_t)((wp >> 32) & 0xfu);
-            for (int l = pl - 1; l >= 0; --l) {
-              const uint64_t wl = __shfl_sync(0xffffffffu, w, l);
-              eval_agg(C, tt, unpack_agg(wl));
-            }
-            if (have_suffix) eval_agg(C, tt, suffix);
-            break;
-          }
-          ZAgg acc = unpack_agg(__shfl_sync(0xffffffffu, w, 31));
-          for (int l = 30; l >= 0; --l)
-            acc = compose(acc, unpack_agg(__shfl_sync(0xffffffffu, w, l)));
-          suffix = have_suffix ? compose(acc, suffix) : acc;
-          have_suffix = true;
-          end -= kWarp;
-        }
-        if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(a.dev_status, TLC_ERR_TIMEOUT);
-        if (lane == 0) {
-          cin_s = C;
-          tin_s = tt;
-          uint32_t Ci = C, ti = tt;
-          eval_agg(Ci, ti, agg);
-          st_relaxed_u64(a.status + t, pack_prefix(Ci, ti));
-        }
-      }
-    }
-    __syncthreads();
-    const uint32_t cin = cin_s, tin = tin_s;
+    uint32_t cin, tin;
+    lookback_tile(a, t, agg, cin, tin, cin_s, tin_s);
 
     // ---- emission --------------------------------------------------------
     {
@@ -455,21 +516,7 @@ k_quant_zre(const QuantArgs a) {
         }
       }
     }
-    if (threadIdx.x == 0) {
-      if (t == 0) {
-        const uint32_t sb = __float_as_uint(scale);
-        a.out[0] = sb & 0xff;
-        a.out[1] = (sb >> 8) & 0xff;
-        a.out[2] = (sb >> 16) & 0xff;
-        a.out[3] = (sb >> 24) & 0xff;
-      }
-      if (t == a.n_tiles - 1) {
-        uint32_t C = cin, tt = tin;
-        eval_agg(C, tt, agg);
-        if (tt) put_out(a, C, remainder_byte(tt));
-        *a.out_len = 4ull + C + (tt ? 1u : 0u);
-      }
-    }
+    finish_tile(a, t, agg, cin, tin, scale);
     __syncthreads();
   }
 }

@@ -215,14 +215,27 @@ k_decode(const DecodeArgs a) {
           v0 = v1 = 0;
           for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) a.y[e] = value_at(e);
         } else {
+          // Values 4v..4v+3 lie in group g = 4v/5 (digits d0..) and, when
+          // d0 >= 2, spill into group g+1; both groups' digit words are
+          // joined so one shift lines the four digits up.
           float4 *y4 = reinterpret_cast<float4 *>(a.y);
           for (uint64_t v = v0 + threadIdx.x; v < v1; v += kDThreads) {
-            const uint64_t e = 4 * v;
+            const uint32_t e0 = (uint32_t)(4 * v);
+            const uint32_t g = e0 / 5u;
+            const uint32_t d0 = e0 - 5u * g;
+            const uint32_t li = g - o32;
+            const uint32_t b0 = grp_s[li];
+            const uint32_t b1 = d0 >= 2u ? (uint32_t)grp_s[li + 1] : 121u;
             float4 o;
-            o.x = value_at(e);
-            o.y = value_at(e + 1);
-            o.z = value_at(e + 2);
-            o.w = value_at(e + 3);
+            if (b0 == 121u && b1 == 121u) {
+              o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            } else {
+              const uint32_t w = ((uint32_t)lut_s[b0] | ((uint32_t)lut_s[b1] << 10)) >> (2u * d0);
+              o.x = dequant(w & 3u, scale);
+              o.y = dequant((w >> 2) & 3u, scale);
+              o.z = dequant((w >> 4) & 3u, scale);
+              o.w = dequant((w >> 6) & 3u, scale);
+            }
             y4[v] = o;
           }
           if (threadIdx.x < 4) {
