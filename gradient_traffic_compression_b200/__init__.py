@@ -8,6 +8,7 @@ from .tlc import (  # noqa: F401
     CORRUPT,
     CUDA_ERROR,
     INVALID_ARG,
+    NOALLOC_MAX_N,
     NONFINITE,
     OK,
     TIMEOUT,
@@ -18,6 +19,7 @@ from .tlc import (  # noqa: F401
     status_string,
     tlc_compress,
     tlc_compress_bound,
+    tlc_compress_noalloc,
     tlc_decompress,
     tlc_decompress_accumulate,
     tlc_kernel_timing,

@@ -14,7 +14,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["tlc_api.cu", "tlc_compress.cu", "tlc_decode.cu"]
+SOURCES = ["tlc_api.cu", "tlc_compress.cu", "tlc_decode.cu", "tlc_noalloc.cu"]
 HEADERS = ["tlc_device.cuh", "tlc_internal.h"]
 LIB_NAME = "libtlc.so"
 

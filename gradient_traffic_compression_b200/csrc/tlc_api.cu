@@ -112,6 +112,13 @@ const char *const kKindNames[tlc::kKindCount] = {"k_absmax", "k_quant_zre", "k_d
 }  // namespace
 
 namespace tlc {
+const DeviceInfo *device_info(int d) {
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  std::call_once(g_dev_once[d], init_device, d);
+  return g_dev_err[d] == cudaSuccess ? &g_dev[d] : nullptr;
+}
+uint32_t wait_limit() { return ::wait_limit(); }
+
 void timing_begin(int kind, cudaStream_t stream) {
   if (!g_timing.on.load(std::memory_order_relaxed)) return;
   std::lock_guard<std::mutex> lk(g_timing.mu);

@@ -44,6 +44,11 @@ inline CompressScratch compress_scratch_layout(void *base, uint32_t n_part, uint
   return s;
 }
 
+// Per-device facts for device d (initialised on first use); nullptr on error.
+const DeviceInfo *device_info(int d);
+// The current cross-block wait limit (polls).
+uint32_t wait_limit();
+
 // Kernel kinds for the optional per-launch timing (see tlc_kernel_timing).
 enum KernelKind { kKindAbsmax = 0, kKindQuantZre, kKindDecodeWrite, kKindDecodeAccumulate,
                   kKindCount };

@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
     L.tlc_set_wait_limit.restype = None
     L.tlc_test_wait_timeout.argtypes = [ctypes.c_uint32, P, P]
     L.tlc_test_wait_timeout.restype = ctypes.c_int
+    L.tlc_compress_noalloc.argtypes = [P, S, ctypes.c_float, P, P, S, P, P, P]
+    L.tlc_compress_noalloc.restype = ctypes.c_int
     L.tlc_kernel_timing.argtypes = [ctypes.c_int]
     L.tlc_kernel_timing.restype = None
     L.tlc_kernel_timing_read.argtypes = [P, P, ctypes.c_int]
@@ -123,6 +125,22 @@ def tlc_compress(x, s: float, err, out, out_len, dev_status=None, stream=None) -
         _dev_ptr(out, "out", torch.uint8), out.numel(), _dev_ptr(out_len, "out_len"),
         _dev_ptr(dev_status, "dev_status", torch.int32), _stream(stream))
     return _check("tlc_compress", code)
+
+
+NOALLOC_MAX_N = 1 << 29
+
+
+def tlc_compress_noalloc(x, s: float, err, out, out_len, dev_status=None, stream=None) -> int:
+    """tlc_compress without any device allocation (scratch is a fixed array
+    inside the library), for callers that cannot allocate; n <= 2^29.  Calls
+    that overlap on the GPU share that array and must be ordered."""
+    import torch
+    n = x.numel()
+    code = lib().tlc_compress_noalloc(
+        _dev_ptr(x, "x", torch.float32), n, float(s), _dev_ptr(err, "err", torch.float32),
+        _dev_ptr(out, "out", torch.uint8), out.numel(), _dev_ptr(out_len, "out_len"),
+        _dev_ptr(dev_status, "dev_status", torch.int32), _stream(stream))
+    return _check("tlc_compress_noalloc", code)
 
 
 def tlc_decompress(stream_buf, n: int, y, in_len=None, in_cap=None, dev_status=None,

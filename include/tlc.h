@@ -139,6 +139,35 @@ tlc_status tlc_decompress_accumulate(const uint8_t *const *ins,
                                      float *acc, int32_t *dev_status,
                                      tlc_stream_t stream);
 
+/* Largest n accepted by tlc_compress_noalloc. */
+#define TLC_NOALLOC_MAX_N ((size_t)1 << 29)
+
+/* tlc_compress without any device memory allocation.
+ *
+ * This has no counterpart on the page; it exists for callers that cannot
+ * allocate device memory while they run: a process whose device memory is
+ * all handed to a framework's caching allocator up front, code that must not
+ * allocate on its hot path (real-time or certified loops), or a runtime
+ * without stream-ordered memory pools.  tlc_compress takes its scratch from
+ * a pool; this call takes it from a fixed 256 KiB array inside the library's
+ * own device memory, which every device that loads the library holds until
+ * the process exits.  It calls no allocation or free routine.
+ *
+ * Arguments, results and errors are those of tlc_compress, and the output is
+ * bit-identical to it, with one more limit: n <= TLC_NOALLOC_MAX_N (2^29),
+ * else TLC_ERR_INVALID_ARG and nothing is enqueued.
+ * - The first call on a device resolves the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ * - Every call on a device shares the one array.  Calls whose work overlaps
+ *   on the GPU (different streams, or different host threads without
+ *   ordering between their streams) race on it and give wrong results;
+ *   order them, e.g. keep them on one stream.  The kernels clear what they
+ *   need at the start of each call, so a call never sees an earlier call's
+ *   leftovers. */
+tlc_status tlc_compress_noalloc(const float *x, size_t n, float s, float *err,
+                                uint8_t *out, size_t out_cap, uint64_t *out_len,
+                                int32_t *dev_status, tlc_stream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char *tlc_status_string(tlc_status status);
 
