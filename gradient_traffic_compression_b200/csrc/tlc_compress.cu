@@ -109,15 +109,64 @@ k_absmax(const float *__restrict__ x, const float *__restrict__ err, uint64_t n,
 }
 
 // --------------------------------------------------------- k_quant_zre ----
+// Tile shape (compile-time knobs; defaults are the tuned values).
+#ifndef TLC_Q_ITERS
+#define TLC_Q_ITERS 4
+#endif
+#ifndef TLC_Q_MINB
+#define TLC_Q_MINB 6
+#endif
+#ifndef TLC_Q_STREAMING
+#define TLC_Q_STREAMING 0
+#endif
+#ifndef TLC_Q_PREFETCH
+#define TLC_Q_PREFETCH 0
+#endif
+#ifndef TLC_Q_EARLY
+#define TLC_Q_EARLY 0
+#endif
 constexpr int kQThreads = 256;
 constexpr int kQWarps = kQThreads / kWarp;
 constexpr int kChunkElems = 640;   // one warp step: 32 lanes x 5 float4
 constexpr int kChunkGroups = 128;  // = kChunkElems / 5
-constexpr int kQIters = 4;
-constexpr int kTileGroups = kQWarps * kQIters * kChunkGroups;  // 4096
-constexpr uint64_t kTileElems = 5ull * kTileGroups;            // 20480
-constexpr int kZBytes = kTileGroups / kQThreads;               // 16 per thread
-static_assert(kZBytes == 16, "ZRE stage reads one uint4 per thread");
+constexpr int kQIters = TLC_Q_ITERS;
+constexpr int kTileGroups = kQWarps * kQIters * kChunkGroups;  // 4096 by default
+constexpr uint64_t kTileElems = 5ull * kTileGroups;            // 20480 by default
+constexpr int kZBytes = kTileGroups / kQThreads;               // 16 per thread by default
+constexpr int kZWords = kZBytes / 4;                           // u32 words per thread
+static_assert((kZBytes == 8 || kZBytes % 16 == 0) && kTileGroups < 65536, "tile shape");
+#ifndef TLC_Q_LOOKV
+#define TLC_Q_LOOKV 1
+#endif
+constexpr int kLookV = TLC_Q_LOOKV;  // look-back words per lane per round trip
+
+// Ask L2 to fetch [p, p + bytes) ahead of use (bytes a multiple of 16,
+// p 16-byte aligned).  No data moves into the SM; nothing to wait for.
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ float4 ld_in(const float4 *p) {
+#if TLC_Q_STREAMING
+  return __ldcs(p);
+#else
+  return __ldg(p);
+#endif
+}
+__device__ __forceinline__ float4 ld_err(const float4 *p) {
+#if TLC_Q_STREAMING
+  return __ldcs(p);
+#else
+  return *p;
+#endif
+}
+__device__ __forceinline__ void st_err(float4 *p, float4 v) {
+#if TLC_Q_STREAMING
+  __stcs(p, v);
+#else
+  *p = v;
+#endif
+}
 
 struct ZAgg {
   uint32_t all, A, R, tc;
@@ -240,6 +289,8 @@ __device__ __forceinline__ void put_out(const QuantArgs &a, uint64_t pos, uint8_
 // the tile's aggregate, combine earlier tiles' words until an inclusive
 // prefix is found, publish this tile's inclusive prefix, and return the
 // exclusive prefix (emitted count, incoming run length mod 14) to all threads.
+// Each round trip reads 32 * kLookV earlier words: every lane first folds
+// its kLookV words (oldest to nearest), then lane 0 folds the lanes.
 __device__ __forceinline__ void lookback_tile(const QuantArgs &a, uint32_t t, const ZAgg &agg,
                                               uint32_t &cin, uint32_t &tin, uint32_t &cin_s,
                                               uint32_t &tin_s) {
@@ -261,28 +312,63 @@ __device__ __forceinline__ void lookback_tile(const QuantArgs &a, uint32_t t, co
       int64_t end = (int64_t)t - 1;
       uint32_t C = 0, tt = 0;
       for (;;) {
-        const int64_t idx = end - lane;
-        const uint64_t w =
-            idx >= 0 ? wait_flag(a.status + idx, a.max_polls, timed_out) : pack_prefix(0, 0);
-        const uint32_t pmask = __ballot_sync(0xffffffffu, (w >> kFlagShift) == 2);
-        if (pmask) {
-          const int pl = __ffs(pmask) - 1;
-          const uint64_t wp = __shfl_sync(0xffffffffu, w, pl);
-          C = (uint32_t)(wp & 0xffffffffu);
-          tt = (uint32_t)((wp >> 32) & 0xfu);
-          for (int l = pl - 1; l >= 0; --l) {
-            const uint64_t wl = __shfl_sync(0xffffffffu, w, l);
-            eval_agg(C, tt, unpack_agg(wl));
+        uint64_t w[kLookV];
+        load_window(a.status, end, pack_prefix(0, 0), a.max_polls, timed_out, w);
+        int jp = kLookV;
+        uint64_t wp = 0;
+#pragma unroll
+        for (int j = 0; j < kLookV; ++j)
+          if (jp == kLookV && (w[j] >> kFlagShift) == 2) {
+            jp = j;
+            wp = w[j];
           }
+        // this lane's words nearer than its prefix (or all of them), folded
+        // from the oldest to the nearest
+        ZAgg lagg = {1u, 0u, 0u, 0u};
+        bool have = false;
+#pragma unroll
+        for (int j = kLookV - 1; j >= 0; --j) {
+          if (j < jp) {
+            const ZAgg aj = unpack_agg(w[j]);
+            lagg = have ? compose(lagg, aj) : aj;
+            have = true;
+          }
+        }
+        uint32_t lC = 0, lt = 0;  // this lane's state after its prefix
+        if (jp < kLookV) {
+          lC = (uint32_t)(wp & 0xffffffffu);
+          lt = (uint32_t)((wp >> 32) & 0xfu);
+          if (have) eval_agg(lC, lt, lagg);
+        }
+        const uint32_t pmask = __ballot_sync(0xffffffffu, jp < kLookV);
+        const int pl = pmask ? __ffs(pmask) - 1 : kWarp;
+        if (pmask) {
+          C = __shfl_sync(0xffffffffu, lC, pl);
+          tt = __shfl_sync(0xffffffffu, lt, pl);
+        }
+        // lanes pl-1 .. 0 (or 31 .. 0 without a prefix), oldest first
+        ZAgg acc = {1u, 0u, 0u, 0u};
+        bool acc_have = false;
+        for (int l = pl - 1; l >= 0; --l) {
+          ZAgg al;
+          al.all = __shfl_sync(0xffffffffu, lagg.all, l);
+          al.A = __shfl_sync(0xffffffffu, lagg.A, l);
+          al.R = __shfl_sync(0xffffffffu, lagg.R, l);
+          al.tc = __shfl_sync(0xffffffffu, lagg.tc, l);
+          if (pmask) {
+            eval_agg(C, tt, al);
+          } else {
+            acc = acc_have ? compose(acc, al) : al;
+            acc_have = true;
+          }
+        }
+        if (pmask) {
           if (have_suffix) eval_agg(C, tt, suffix);
           break;
         }
-        ZAgg acc = unpack_agg(__shfl_sync(0xffffffffu, w, 31));
-        for (int l = 30; l >= 0; --l)
-          acc = compose(acc, unpack_agg(__shfl_sync(0xffffffffu, w, l)));
         suffix = have_suffix ? compose(acc, suffix) : acc;
         have_suffix = true;
-        end -= kWarp;
+        end -= kWarp * kLookV;
       }
       if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(a.dev_status, TLC_ERR_TIMEOUT);
       if (lane == 0) {
@@ -318,8 +404,13 @@ __device__ __forceinline__ void finish_tile(const QuantArgs &a, uint32_t t, cons
   }
 }
 
+#if TLC_Q_MINB > 1
+#define TLC_Q_BOUNDS __launch_bounds__(kQThreads, TLC_Q_MINB)
+#else
+#define TLC_Q_BOUNDS __launch_bounds__(kQThreads)
+#endif
 template <bool kVec>
-__global__ void __launch_bounds__(kQThreads)
+__global__ void TLC_Q_BOUNDS
 k_quant_zre(const QuantArgs a) {
   __shared__ __align__(16) uint32_t dig_s[kQWarps][kChunkElems / 4];
   __shared__ __align__(16) uint32_t tile_s[kTileGroups / 4];
@@ -360,9 +451,14 @@ k_quant_zre(const QuantArgs a) {
   const float scale = scale_s;
   const float thr = zero_band_threshold(scale, state_s == 1);
 
+#if TLC_Q_EARLY
+  if (threadIdx.x == 0) tile_id_s = atomicAdd(a.ticket, 1u);
+#endif
   for (;;) {
     if (threadIdx.x == 0) {
+#if !TLC_Q_EARLY
       tile_id_s = atomicAdd(a.ticket, 1u);
+#endif
       A_s = 0xffffffffu;
     }
     __syncthreads();
@@ -385,8 +481,8 @@ k_quant_zre(const QuantArgs a) {
         float4 xv[5], ev[5];
 #pragma unroll
         for (int j = 0; j < 5; ++j) {
-          xv[j] = __ldg(x4 + lane + 32 * j);
-          ev[j] = err4[lane + 32 * j];
+          xv[j] = ld_in(x4 + lane + 32 * j);
+          ev[j] = ld_err(err4 + lane + 32 * j);
         }
 #pragma unroll
         for (int j = 0; j < 5; ++j) {
@@ -396,7 +492,7 @@ k_quant_zre(const QuantArgs a) {
           dw |= quant_digit(__fadd_rn(xv[j].y, ev[j].y), scale, thr, o.y) << 8;
           dw |= quant_digit(__fadd_rn(xv[j].z, ev[j].z), scale, thr, o.z) << 16;
           dw |= quant_digit(__fadd_rn(xv[j].w, ev[j].w), scale, thr, o.w) << 24;
-          err4[lane + 32 * j] = o;
+          st_err(err4 + lane + 32 * j, o);
           dig_s[warp][lane + 32 * j] = dw;
         }
       } else {
@@ -425,13 +521,44 @@ k_quant_zre(const QuantArgs a) {
       __syncwarp();
     }
     __syncthreads();
+#if TLC_Q_EARLY
+    // The next tile's ticket is taken now, so its loads can start (through
+    // L2) while this tile is encoded.  A block handles its tickets in
+    // increasing order, so no look-back ever waits on a later ticket.
+    if (threadIdx.x == 0) {
+      const uint32_t tn = atomicAdd(a.ticket, 1u);
+      tile_id_s = tn;
+#if TLC_Q_PREFETCH
+      const uint64_t en = (uint64_t)tn * kTileElems;
+      if (kVec && tn < a.n_tiles && en + kTileElems <= a.n) {
+        prefetch_l2(a.x + en, (uint32_t)(kTileElems * 4));
+        prefetch_l2(a.err + en, (uint32_t)(kTileElems * 4));
+      }
+#endif
+    }
+#endif
 
     // ---- zero-run encoding: local analysis -----------------------------
-    const uint4 q4 = reinterpret_cast<const uint4 *>(tile_s)[threadIdx.x];
-    const uint32_t qw[4] = {q4.x, q4.y, q4.z, q4.w};
+    uint32_t qw[kZWords];
+    if constexpr (kZWords == 2) {
+      const uint2 q2 = reinterpret_cast<const uint2 *>(tile_s)[threadIdx.x];
+      qw[0] = q2.x;
+      qw[1] = q2.y;
+    } else {
+#pragma unroll
+      for (int v = 0; v < kZWords / 4; ++v) {
+        const uint4 q4 = reinterpret_cast<const uint4 *>(tile_s)[threadIdx.x * (kZWords / 4) + v];
+        qw[4 * v] = q4.x;
+        qw[4 * v + 1] = q4.y;
+        qw[4 * v + 2] = q4.z;
+        qw[4 * v + 3] = q4.w;
+      }
+    }
+    bool mine_all = true;
+#pragma unroll
+    for (int w = 0; w < kZWords; ++w) mine_all = mine_all && qw[w] == 0x79797979u;
     // groups past the end of the tensor are all-zero (121) by construction
-    const bool tile_all = __syncthreads_and(q4.x == 0x79797979u && q4.y == 0x79797979u &&
-                                            q4.z == 0x79797979u && q4.w == 0x79797979u);
+    const bool tile_all = __syncthreads_and(mine_all);
     if (tile_all) {
       // Entirely 121s: only full 14-chunks of the run end inside the tile.
       ZAgg agg = {1u, tgv, 0u, 0u};

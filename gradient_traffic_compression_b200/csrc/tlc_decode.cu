@@ -24,11 +24,27 @@
 
 namespace tlc {
 
+// Payload bytes per thread (multiple of 4): small tiles balance the dense
+// write mode best; the accumulate mode touches little memory per tile and
+// prefers fewer, larger tiles.
+#ifndef TLC_D_BYTES_WRITE
+#define TLC_D_BYTES_WRITE 4
+#endif
+#ifndef TLC_D_BYTES_ACC
+#define TLC_D_BYTES_ACC 8
+#endif
 constexpr int kDThreads = 256;
-constexpr int kDBytes = 8;                  // payload bytes per thread
-constexpr int kDTile = kDThreads * kDBytes; // 2048
-constexpr int kDMaxGroups = kDTile * 14;    // largest expansion of a tile
 constexpr int kWrite = 0, kAccumulate = 1;
+template <int kMode>
+struct DecodeShape {
+  static constexpr int kBytes = kMode == kWrite ? TLC_D_BYTES_WRITE : TLC_D_BYTES_ACC;
+  static constexpr int kTile = kDThreads * kBytes;   // payload bytes per tile
+  static constexpr int kMaxGroups = kTile * 14;      // largest expansion of a tile
+};
+#ifndef TLC_D_LOOKV
+#define TLC_D_LOOKV 1
+#endif
+constexpr int kLookV = TLC_D_LOOKV;   // look-back words per lane per round trip
 
 struct DecodeArgs {
   const uint8_t *in;
@@ -50,7 +66,8 @@ __device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
 }
 
 // Exclusive prefix (in groups) of tile u, by warp 0.  Publishes the tile's
-// aggregate first and its inclusive prefix last.
+// aggregate first and its inclusive prefix last.  Each round trip reads
+// 32 * kLookV earlier tiles' words.
 __device__ uint64_t lookback_sum(uint64_t *status, uint32_t u, uint64_t E, uint32_t max_polls,
                                  bool &timed_out) {
   const int lane = threadIdx.x & 31;
@@ -62,16 +79,26 @@ __device__ uint64_t lookback_sum(uint64_t *status, uint32_t u, uint64_t E, uint3
   uint64_t sum = 0;
   int64_t end = (int64_t)u - 1;
   for (;;) {
-    const int64_t idx = end - lane;
-    const uint64_t w = idx >= 0 ? wait_flag(status + idx, max_polls, timed_out) : kFlagPrefix;
-    const uint32_t pmask = __ballot_sync(0xffffffffu, (w >> kFlagShift) == 2);
+    uint64_t w[kLookV];
+    load_window(status, end, kFlagPrefix, max_polls, timed_out, w);
+    // nearest prefix of this lane, and the sum up to and including it
+    int jp = kLookV;
+    uint64_t part = 0;
+#pragma unroll
+    for (int j = 0; j < kLookV; ++j) {
+      if (jp == kLookV) {
+        part += w[j] & kValueMask;
+        if ((w[j] >> kFlagShift) == 2) jp = j;
+      }
+    }
+    const uint32_t pmask = __ballot_sync(0xffffffffu, jp < kLookV);
     if (pmask) {
       const int pl = __ffs(pmask) - 1;
-      sum += warp_sum_u64(lane <= pl ? (w & kValueMask) : 0);
+      sum += warp_sum_u64(lane <= pl ? part : 0);
       break;
     }
-    sum += warp_sum_u64(w & kValueMask);
-    end -= kWarp;
+    sum += warp_sum_u64(part);
+    end -= kWarp * kLookV;
   }
   if (lane == 0) st_relaxed_u64(status + u, kFlagPrefix | (sum + E));
   return sum;
@@ -92,7 +119,9 @@ __device__ __forceinline__ float dequant(uint32_t dig, float scale) {
 template <int kMode, bool kVec>
 __global__ void __launch_bounds__(kDThreads)
 k_decode(const DecodeArgs a) {
-  extern __shared__ __align__(16) uint8_t grp_s[];  // kWrite: kDMaxGroups + 16 bytes
+  constexpr int kDBytes = DecodeShape<kMode>::kBytes;
+  constexpr int kDTile = DecodeShape<kMode>::kTile;
+  extern __shared__ __align__(16) uint8_t grp_s[];  // kWrite: kMaxGroups + 16 bytes
   __shared__ uint16_t lut_s[256];
   __shared__ uint32_t scan_s[kDThreads / kWarp + 1];
   __shared__ uint64_t o_s, m_s;
@@ -136,12 +165,14 @@ k_decode(const DecodeArgs a) {
 
     // ---- load 8 payload bytes, expansion counts, block scan ------------
     const uint64_t b0 = (uint64_t)u * kDTile + (uint64_t)threadIdx.x * kDBytes;
-    uint32_t bw[2] = {0x79797979u, 0x79797979u};
+    uint32_t bw[kDBytes / 4];
+#pragma unroll
+    for (int k = 0; k < kDBytes / 4; ++k) bw[k] = 0x79797979u;
     int nvalid = 0;
     if (b0 + kDBytes <= m && ((reinterpret_cast<uintptr_t>(payload + b0) & 3) == 0)) {
       const uint32_t *p32 = reinterpret_cast<const uint32_t *>(payload + b0);
-      bw[0] = __ldg(p32);
-      bw[1] = __ldg(p32 + 1);
+#pragma unroll
+      for (int k = 0; k < kDBytes / 4; ++k) bw[k] = __ldg(p32 + k);
       nvalid = kDBytes;
     } else {
 #pragma unroll
@@ -284,13 +315,19 @@ __global__ void k_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_s
 
 // ------------------------------------------------------------- launchers --
 uint32_t decode_tiles_max(uint64_t cap, uint64_t groups) {
+  // sized for the smaller of the two tile shapes, so it covers both modes
+  constexpr int kSmallest = DecodeShape<kWrite>::kTile < DecodeShape<kAccumulate>::kTile
+                                ? DecodeShape<kWrite>::kTile
+                                : DecodeShape<kAccumulate>::kTile;
   uint64_t m = cap >= 4 ? cap - 4 : 0;
   if (m > groups) m = groups;
-  uint64_t t = (m + kDTile - 1) / kDTile;
+  uint64_t t = (m + kSmallest - 1) / kSmallest;
   return (uint32_t)(t < 1 ? 1 : t);
 }
 
-size_t decode_smem_bytes(bool accumulate) { return accumulate ? 0 : (size_t)kDMaxGroups + 16; }
+size_t decode_smem_bytes(bool accumulate) {
+  return accumulate ? 0 : (size_t)DecodeShape<kWrite>::kMaxGroups + 16;
+}
 
 template <int kMode, bool kVec>
 static cudaError_t launch_one(const DeviceInfo &dev, const DecodeArgs &a, uint32_t tiles,

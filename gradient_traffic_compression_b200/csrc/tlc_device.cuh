@@ -62,6 +62,27 @@ __device__ __forceinline__ uint64_t wait_flag(const uint64_t *p, uint32_t max_po
   return w;
 }
 
+// Look-back window: each lane of the looking-back warp reads V consecutive
+// status words per round trip (32 * V tiles per trip): the words
+// end - (lane*V + j), j = 0..V-1 (nearest first), with every load issued
+// before any is waited on; indices below 0 read as `origin` (an inclusive
+// prefix).  Then it waits (bounded) for any word that has no flag yet.
+template <int V>
+__device__ __forceinline__ void load_window(const uint64_t *status, int64_t end, uint64_t origin,
+                                            uint32_t max_polls, bool &timed_out, uint64_t (&w)[V]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    const int64_t idx = end - (int64_t)(lane * V + j);
+    w[j] = idx >= 0 ? ld_relaxed_u64(status + idx) : origin;
+  }
+#pragma unroll
+  for (int j = 0; j < V; ++j) {
+    const int64_t idx = end - (int64_t)(lane * V + j);
+    if ((w[j] >> kFlagShift) == 0) w[j] = wait_flag(status + idx, max_polls, timed_out);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Block-wide exclusive scans for blocks of kThreads threads (multiple of 32).
 // `scratch` needs kThreads/32 + 1 words of shared memory.  Every thread

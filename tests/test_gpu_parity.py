@@ -220,6 +220,23 @@ def test_run_lengths_at_stream_end(g, tail):
     assert_roundtrip_parity(g, st, n)
 
 
+@pytest.mark.parametrize("groups", [1023, 1024, 1025, 2047, 2048, 2049, 3 * 1024 + 1,
+                                    8 * 2048 - 1, 8 * 2048 + 1])
+def test_dense_streams_at_decode_tile_edges(g, groups):
+    # uniform values with s = 1 make almost every group a literal, so the
+    # payload length is close to the group count (decode tiles: 1024 bytes
+    # for dense output, 2048 for accumulation)
+    n = 5 * groups - (groups % 3)
+    x = (synth.uniforms(synth.key_for(groups, 5), n) * 2 - 1).astype(np.float32)
+    st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
+    assert st.size - 4 > 0.9 * ((n + 4) // 5)
+    assert_roundtrip_parity(g, st, n)
+    acc0 = synth.normal(synth.key_for(groups, 6), n, 1.0)
+    rc_o, a_o = oracle.decompress_accumulate([st, st], n, acc0)
+    rc_g, a_g = gpu_accumulate(g, [st, st], n, acc0)
+    assert rc_g == rc_o == 0 and np.array_equal(bits(a_g), bits(a_o))
+
+
 def test_all_zero_and_single_values(g):
     for n in (1, 5, 70, 71, 4096 * 5, 4096 * 5 * 3 + 1):
         st, _ = assert_compress_parity(g, np.zeros(n, np.float32), 1.0, np.zeros(n, np.float32))
