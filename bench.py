@@ -448,7 +448,7 @@ def traffic_for(kernel, n):
     if not os.path.exists(path):
         return None
     from gradient_traffic_compression_b200.build import source_digest
-    digest = source_digest()
+    digest = source_digest(kernel)
     with open(path) as f:
         for line in f:
             t = line.split()

@@ -65,12 +65,23 @@ def build_library(verbose: bool = False, ptxas_info: bool = False) -> str:
     return out
 
 
-def source_digest() -> str:
-    """Short SHA-256 over the kernel sources and headers (identifies which
-    build a stored profile belongs to)."""
+KERNEL_SOURCES = {
+    "k_absmax": ["tlc_compress.cu", "tlc_device.cuh"],
+    "k_quant_zre": ["tlc_compress.cu", "tlc_device.cuh"],
+    "k_decode_write": ["tlc_decode.cu", "tlc_device.cuh"],
+    "k_decode_accumulate": ["tlc_decode.cu", "tlc_device.cuh"],
+}
+
+
+def source_digest(kernel: str | None = None) -> str:
+    """Short SHA-256 over the compiler flags and the sources of one kernel
+    (or of the whole library); identifies which build a stored profile
+    belongs to."""
     import hashlib
-    h = hashlib.sha256()
-    for p in _inputs():
+    h = hashlib.sha256(" ".join(NVCC_FLAGS).encode())
+    paths = ([os.path.join(CSRC, f) for f in KERNEL_SOURCES[kernel]] if kernel
+             else list(_inputs()))
+    for p in paths:
         with open(p, "rb") as f:
             h.update(os.path.basename(p).encode() + b"\0" + f.read())
     return h.hexdigest()[:12]
