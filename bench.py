@@ -47,6 +47,9 @@ def parse_args():
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4, 5],
+                   help="workload: 3 (default, the headline) or another of the five "
+                        "parity configs, measured the same way (extra lines)")
     return p.parse_args()
 
 
@@ -150,8 +153,14 @@ def run_ours(args, rank, world, local):
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    global S_PARAM
+    if args.config == 1:
+        S_PARAM = synth.CONFIGS[1]["s"]
+        args.log2n = 20
+        args.no_e2e = True
+        args.no_cpu_baseline = True
     n = 1 << args.log2n
-    x_h = synth.flat_tensor(3, n=n, step=rank)       # each rank: its own gradient
+    x_h = synth.flat_tensor(args.config, n=n, step=rank)   # each rank: its own gradient
 
     x = torch.from_numpy(x_h).to(dev)
     err = torch.zeros(n, dtype=torch.float32, device=dev)
@@ -264,7 +273,9 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": workload_config(n, args.log2n) | {"parallelism": f"replicas x{world}"},
+        "config": (workload_config(n, args.log2n) if args.config == 3 else
+                   {"workload": synth.CONFIGS[args.config]["name"], "n": n, "s": S_PARAM,
+                    "l2": "L2-resident (x + err = 8 MiB)"}) | {"parallelism": f"replicas x{world}"},
         "clocks": clocks,
         "gpu_launches": int(sum(v[0] for v in kern.values())),
         "roofline": {
@@ -355,6 +366,113 @@ def run_e2e(args, tlc, torch, dev, x_h, n, cap, world):
             "h2d_bytes_per_step": 8 * n, "d2h_bytes_per_step": d2h[0],
             "path": "pinned host x, err -> device; tlc_compress; stream + err -> host; "
                     "tlc_decompress; tlc_decompress_accumulate; y -> host"}
+
+
+# ------------------------------------------- tensor sets and K streams ----
+
+def run_config_set(args, rank, world, local):
+    """Configs 2 and 4 (per-layer tensors, one call per tensor, error buffers
+    carried) and 5 (K = 8 workers' streams summed).  Same legs and timing as
+    the headline; extra lines, not the headline workload."""
+    import torch
+    import torch.distributed as dist
+
+    import gradient_traffic_compression_b200 as tlc
+    import synth
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    cfg = synth.CONFIGS[args.config]
+    s = cfg["s"]
+    if args.config == 5:
+        xs_h = [synth.flat_tensor(5, worker=w) for w in range(cfg["k"])]
+    else:
+        xs_h = synth.tensor_set(args.config, rank)
+    xs = [torch.from_numpy(a).to(dev) for a in xs_h]
+    ns = [a.size for a in xs_h]
+    total = sum(ns)
+    errs = [torch.zeros(n, dtype=torch.float32, device=dev) for n in ns]
+    caps = [tlc.tlc_compress_bound(n) for n in ns]
+    outs = [torch.empty(c, dtype=torch.uint8, device=dev) for c in caps]
+    lens = torch.zeros(len(ns), dtype=torch.int64, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    if args.config == 5:
+        acc = torch.zeros(ns[0], dtype=torch.float32, device=dev)
+        ys, accs = None, None
+    else:
+        ys = [torch.empty(n, dtype=torch.float32, device=dev) for n in ns]
+        accs = [torch.zeros(n, dtype=torch.float32, device=dev) for n in ns]
+
+    def legs():
+        for i in range(len(ns)):
+            tlc.tlc_compress(xs[i], s, errs[i], outs[i], lens[i:i + 1], status, stream)
+        yield
+        if args.config == 5:
+            yield
+            tlc.tlc_decompress_accumulate(outs, ns[0], acc, in_lens=lens, in_caps=caps,
+                                          dev_status=status, stream=stream)
+        else:
+            for i in range(len(ns)):
+                tlc.tlc_decompress(outs[i], ns[i], ys[i], in_len=lens[i:i + 1], in_cap=caps[i],
+                                   dev_status=status, stream=stream)
+            yield
+            for i in range(len(ns)):
+                tlc.tlc_decompress_accumulate([outs[i]], ns[i], accs[i], in_lens=lens[i:i + 1],
+                                              in_caps=[caps[i]], dev_status=status,
+                                              stream=stream)
+        yield
+
+    for _ in range(max(3, args.warmup)):
+        for _ in legs():
+            pass
+    torch.cuda.synchronize()
+    steps = max(1, min(args.steps, 50))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    tlc.tlc_kernel_timing(True)
+    for k in range(steps):
+        ev[k][0].record(stream)
+        for j, _ in enumerate(legs()):
+            ev[k][j + 1].record(stream)
+    torch.cuda.synchronize()
+    tlc.tlc_kernel_timing(False)
+    kern = tlc.tlc_kernel_timing_read()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())}")
+    legs_ms = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)) / steps
+               for i in range(3)]
+    step_ms = sum(legs_ms)
+    L = int(lens.sum().item())
+    in_bytes = 4 * total
+    peak, _ = load_peaks()
+    res = {
+        "metric": METRIC, "value": round(world * in_bytes / (step_ms * 1e-3) / 1e9, 2),
+        "unit": "GB/s", "n_gpus": world, "steps": steps, "ms_per_step": round(step_ms, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": cfg["name"], "tensors": len(ns), "values": total, "s": s,
+                   "calls": "one C-ABI call per tensor and leg"},
+        "legs": {"compress_ms": round(legs_ms[0], 4),
+                 "compress_gbs": round(in_bytes / (legs_ms[0] * 1e-3) / 1e9, 1),
+                 "stream_bytes": L, "bits_per_value": round(8 * L / total, 5)},
+        "kernels": {k: {"launches": v[0], "avg_ms": round(v[1] / max(v[0], 1), 5)}
+                    for k, v in kern.items() if v[0]},
+        "gpu_launches": int(sum(v[0] for v in kern.values())),
+    }
+    if args.config == 5:
+        res["legs"]["accumulate_ms"] = round(legs_ms[2], 4)
+        res["legs"]["accumulate_gbs_of_fp32_input"] = round(
+            in_bytes / (legs_ms[2] * 1e-3) / 1e9, 1)
+        res["legs"]["accumulate_dense_bytes_frac"] = round(
+            (8 * ns[0]) / (legs_ms[2] * 1e-3) / 1e9 / peak, 4)
+    else:
+        res["legs"]["decompress_ms"] = round(legs_ms[1], 4)
+        res["legs"]["decompress_gbs"] = round(in_bytes / (legs_ms[1] * 1e-3) / 1e9, 1)
+        res["legs"]["accumulate_ms"] = round(legs_ms[2], 4)
+    return res
 
 
 # ------------------------------------------------------- CPU oracle timing --
@@ -476,7 +594,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     try:
-        res = run_ours(args, rank, world, local)
+        if args.config in (1, 3):
+            res = run_ours(args, rank, world, local)
+        else:
+            res = run_config_set(args, rank, world, local)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
