@@ -495,7 +495,8 @@ k_quant_zre(const QuantArgs a) {
           st_err(err4 + lane + 32 * j, o);
           dig_s[warp][lane + 32 * j] = dw;
         }
-      } else {
+      } else if (e0 < a.n) {
+        // tail or unaligned chunk: scalar and bounds-checked
 #pragma unroll 1
         for (int j = 0; j < 5; ++j) {
           uint32_t dw = 0;
@@ -512,6 +513,10 @@ k_quant_zre(const QuantArgs a) {
           }
           dig_s[warp][lane + 32 * j] = dw;
         }
+      } else {
+        // chunk entirely past the end: all-zero groups
+#pragma unroll
+        for (int j = 0; j < 5; ++j) dig_s[warp][lane + 32 * j] = 0x01010101u;
       }
       __syncwarp();
       uint32_t w5[5];

@@ -10,13 +10,15 @@
 //   kWrite       dense output: y_i = +scale, -scale or +0.0
 //   kAccumulate  acc_i += y_i only where q_i != 0 (acc keeps its bits at
 //                zeros), one launch per worker stream, in worker order
-// Each tile is 2048 payload bytes.  Per tile: expansion counts e_k (an
-// escape byte b >= 243 stands for b - 241 groups of 121, any other byte for
-// itself), a block scan, and a decoupled look-back over earlier tiles for the
-// tile's first group index O.  In kWrite mode the tile's groups are expanded
-// in shared memory (at most 14 * 2048 bytes) and turned into fp32 with
-// coalesced 128-bit stores; in kAccumulate mode only literal bytes other
-// than 121 are visited, so work and traffic follow the non-zeros.
+// A tile is 1024 (kWrite) or 2048 (kAccumulate) payload bytes.  Per tile:
+// expansion counts e_k (an escape byte b >= 243 stands for b - 241 groups of
+// 121, any other byte for itself), a block scan, and a decoupled look-back
+// over earlier tiles for the tile's first group index O.  The tile's groups
+// are then expanded in shared memory (at most 14 bytes per payload byte) and
+// walked as float4 columns with coalesced 128-bit accesses: written in kWrite
+// mode, read-modify-written (all-zero columns skipped) in kAccumulate mode.
+// An accumulate tile made mostly of escapes instead visits only its literal
+// groups, so there work and traffic follow the non-zeros.
 // Every write is clamped to the ceil(n/5) groups of the tensor; a stream that
 // does not expand to exactly that many groups is reported as corrupt.
 #include "tlc_device.cuh"
@@ -121,7 +123,7 @@ __global__ void __launch_bounds__(kDThreads)
 k_decode(const DecodeArgs a) {
   constexpr int kDBytes = DecodeShape<kMode>::kBytes;
   constexpr int kDTile = DecodeShape<kMode>::kTile;
-  extern __shared__ __align__(16) uint8_t grp_s[];  // kWrite: kMaxGroups + 16 bytes
+  extern __shared__ __align__(16) uint8_t grp_s[];  // kMaxGroups + 16 bytes
   __shared__ uint16_t lut_s[256];
   __shared__ uint32_t scan_s[kDThreads / kWarp + 1];
   __shared__ uint64_t o_s, m_s;
@@ -145,8 +147,7 @@ k_decode(const DecodeArgs a) {
     scale_s = __uint_as_float(hb);
     m_s = bad ? 0 : L - 4;
   }
-  if (kMode == kWrite)
-    for (int v = threadIdx.x; v < 256; v += kDThreads) lut_s[v] = v < 243 ? digits_of(v) : 0;
+  for (int v = threadIdx.x; v < 256; v += kDThreads) lut_s[v] = v < 243 ? digits_of(v) : 0;
   __syncthreads();
   if (bad_s) {
     if (blockIdx.x == 0 && threadIdx.x == 0) report(a.dev_status, TLC_ERR_CORRUPT);
@@ -192,6 +193,11 @@ k_decode(const DecodeArgs a) {
     }
     uint32_t E;
     const uint32_t off = block_exclusive_sum<kDThreads>(esum, scan_s, E);
+    // Dense output always expands the tile's groups in shared memory.  The
+    // accumulate mode does so too when the tile is mostly literals (then a
+    // coalesced float4 pass over acc is cheapest); for escape-heavy tiles it
+    // visits only the literal groups.
+    const bool expand = kMode == kWrite || E <= 4u * (uint32_t)kDTile;
 
     // ---- look-back (warp 0); the other warps pre-fill zero groups ----------
     if (warp == 0) {
@@ -199,7 +205,7 @@ k_decode(const DecodeArgs a) {
       const uint64_t O = lookback_sum(a.status, u, E, a.max_polls, timed_out);
       if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(a.dev_status, TLC_ERR_TIMEOUT);
       if (lane == 0) o_s = O;
-    } else if (kMode == kWrite) {
+    } else if (expand) {
       const uint32_t words = (E + 15) / 16;
       for (uint32_t w = threadIdx.x - kWarp; w < words; w += kDThreads - kWarp)
         reinterpret_cast<uint4 *>(grp_s)[w] = make_uint4(0x79797979u, 0x79797979u, 0x79797979u,
@@ -213,7 +219,7 @@ k_decode(const DecodeArgs a) {
     }
     const uint64_t Ec = O >= a.groups ? 0 : umin64(E, a.groups - O);
 
-    if (kMode == kWrite) {
+    if (expand) {
       // literal bytes into the expanded group buffer
       uint32_t pos = off;
 #pragma unroll
@@ -241,10 +247,21 @@ k_decode(const DecodeArgs a) {
           const uint32_t dig = (lut_s[grp_s[g - o32]] >> (2 * d)) & 3u;
           return dequant(dig, scale);
         };
+        // one value: written (dense output) or added where non-zero (accumulate)
+        auto put = [&](uint64_t e) {
+          if (kMode == kWrite) {
+            a.y[e] = value_at(e);
+          } else {
+            const uint32_t e32 = (uint32_t)e;
+            const uint32_t g = e32 / 5u;
+            const uint32_t dig = (lut_s[grp_s[g - o32]] >> (2 * (e32 - 5u * g))) & 3u;
+            if (dig != 1u) a.y[e] = __fadd_rn(a.y[e], dequant(dig, scale));
+          }
+        };
         uint64_t v0 = (e_begin + 3) / 4, v1 = e_end / 4;
         if (!kVec || v1 <= v0) {
           v0 = v1 = 0;
-          for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) a.y[e] = value_at(e);
+          for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) put(e);
         } else {
           // Values 4v..4v+3 lie in group g = 4v/5 (digits d0..) and, when
           // d0 >= 2, spill into group g+1; both groups' digit words are
@@ -257,29 +274,44 @@ k_decode(const DecodeArgs a) {
             const uint32_t li = g - o32;
             const uint32_t b0 = grp_s[li];
             const uint32_t b1 = d0 >= 2u ? (uint32_t)grp_s[li + 1] : 121u;
-            float4 o;
-            if (b0 == 121u && b1 == 121u) {
-              o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            } else {
+            if (kMode == kWrite) {
+              float4 o;
+              if (b0 == 121u && b1 == 121u) {
+                o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+              } else {
+                const uint32_t w =
+                    ((uint32_t)lut_s[b0] | ((uint32_t)lut_s[b1] << 10)) >> (2u * d0);
+                o.x = dequant(w & 3u, scale);
+                o.y = dequant((w >> 2) & 3u, scale);
+                o.z = dequant((w >> 4) & 3u, scale);
+                o.w = dequant((w >> 6) & 3u, scale);
+              }
+              y4[v] = o;
+            } else if (b0 != 121u || b1 != 121u) {
               const uint32_t w = ((uint32_t)lut_s[b0] | ((uint32_t)lut_s[b1] << 10)) >> (2u * d0);
-              o.x = dequant(w & 3u, scale);
-              o.y = dequant((w >> 2) & 3u, scale);
-              o.z = dequant((w >> 4) & 3u, scale);
-              o.w = dequant((w >> 6) & 3u, scale);
+              if ((w & 0xffu) != 0x55u) {  // some of the four digits is not zero
+                float4 o = y4[v];
+                if ((w & 3u) != 1u) o.x = __fadd_rn(o.x, dequant(w & 3u, scale));
+                if (((w >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, dequant((w >> 2) & 3u, scale));
+                if (((w >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, dequant((w >> 4) & 3u, scale));
+                if (((w >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, dequant((w >> 6) & 3u, scale));
+                y4[v] = o;
+              }
             }
-            y4[v] = o;
           }
           if (threadIdx.x < 4) {
             const uint64_t e = e_begin + threadIdx.x;
-            if (e < 4 * v0) a.y[e] = value_at(e);
+            if (e < 4 * v0) put(e);
           } else if (threadIdx.x < 8) {
             const uint64_t e = 4 * v1 + (threadIdx.x - 4);
-            if (e < e_end) a.y[e] = value_at(e);
+            if (e < e_end) put(e);
           }
         }
       }
     } else {
-      // accumulate: visit literal groups other than the all-zero 121
+      // accumulate, escape-heavy tile: visit only literal groups other than
+      // the all-zero 121; each group's (up to five) acc values are loaded
+      // before any is added
       uint64_t g = O + off;
 #pragma unroll
       for (int k = 0; k < kDBytes; ++k) {
@@ -290,11 +322,17 @@ k_decode(const DecodeArgs a) {
           } else {
             if (b != 121u && g < a.groups) {
               const uint16_t dg = digits_of(b);
+              float v[5];
+#pragma unroll
+              for (int d = 0; d < 5; ++d) {
+                const uint64_t e = 5 * g + d;
+                v[d] = (((dg >> (2 * d)) & 3u) != 1u && e < a.n) ? a.y[e] : 0.0f;
+              }
 #pragma unroll
               for (int d = 0; d < 5; ++d) {
                 const uint32_t dig = (dg >> (2 * d)) & 3u;
                 const uint64_t e = 5 * g + d;
-                if (dig != 1u && e < a.n) a.y[e] = __fadd_rn(a.y[e], dequant(dig, scale));
+                if (dig != 1u && e < a.n) a.y[e] = __fadd_rn(v[d], dequant(dig, scale));
               }
             }
             ++g;
@@ -326,7 +364,8 @@ uint32_t decode_tiles_max(uint64_t cap, uint64_t groups) {
 }
 
 size_t decode_smem_bytes(bool accumulate) {
-  return accumulate ? 0 : (size_t)DecodeShape<kWrite>::kMaxGroups + 16;
+  return (size_t)(accumulate ? DecodeShape<kAccumulate>::kMaxGroups
+                             : DecodeShape<kWrite>::kMaxGroups) + 16;
 }
 
 template <int kMode, bool kVec>
@@ -360,7 +399,9 @@ cudaError_t launch_decode(const DeviceInfo &dev, const uint8_t *in, const uint64
   a.max_polls = max_polls;
   const uint32_t tiles = decode_tiles_max(cap, a.groups);
   const bool vec = (reinterpret_cast<uintptr_t>(y) & 15) == 0;
-  if (accumulate) return launch_one<kAccumulate, false>(dev, a, tiles, stream);
+  if (accumulate)
+    return vec ? launch_one<kAccumulate, true>(dev, a, tiles, stream)
+               : launch_one<kAccumulate, false>(dev, a, tiles, stream);
   return vec ? launch_one<kWrite, true>(dev, a, tiles, stream)
              : launch_one<kWrite, false>(dev, a, tiles, stream);
 }
@@ -375,7 +416,11 @@ int occupancy_decode(bool accumulate) {
   int occ = 0;
   const size_t smem = decode_smem_bytes(accumulate);
   if (accumulate) {
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode<kAccumulate, false>, kDThreads,
+    cudaFuncSetAttribute(k_decode<kAccumulate, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    cudaFuncSetAttribute(k_decode<kAccumulate, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode<kAccumulate, true>, kDThreads,
                                                   smem);
   } else {
     cudaFuncSetAttribute(k_decode<kWrite, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
