@@ -11,6 +11,7 @@ from .tlc import (  # noqa: F401
     NOALLOC_MAX_N,
     NONFINITE,
     OK,
+    Plan,
     TIMEOUT,
     TLCError,
     compress,
@@ -18,11 +19,17 @@ from .tlc import (  # noqa: F401
     lib,
     status_string,
     tlc_compress,
+    tlc_compress_batch,
     tlc_compress_bound,
     tlc_compress_noalloc,
     tlc_decompress,
+    tlc_decompress_batch,
     tlc_decompress_accumulate,
     tlc_kernel_timing,
+    tlc_plan_arena_bytes,
+    tlc_plan_create,
+    tlc_plan_destroy,
+    tlc_plan_stream_offset,
     tlc_kernel_timing_read,
     tlc_set_wait_limit,
     tlc_test_wait_timeout,

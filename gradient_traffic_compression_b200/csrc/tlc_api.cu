@@ -34,6 +34,9 @@ void init_device(int d) {
     di.occ_quant_scalar = tlc::occupancy_quant(false);
     di.occ_decode_write = tlc::occupancy_decode(false);
     di.occ_decode_acc = tlc::occupancy_decode(true);
+    di.occ_quant_batch = tlc::occupancy_quant_batch();
+    di.occ_decode_batch_write = tlc::occupancy_decode_batch(false);
+    di.occ_decode_batch_acc = tlc::occupancy_decode_batch(true);
     cudaMemPoolProps props;
     std::memset(&props, 0, sizeof(props));
     props.allocType = cudaMemAllocationTypePinned;
@@ -289,6 +292,173 @@ tlc_status tlc_decompress_accumulate(const uint8_t *const *ins, const uint64_t *
   }
   const cudaError_t fe = cudaFreeAsync(scratch, st);
   return (ce == cudaSuccess && fe == cudaSuccess) ? TLC_OK : TLC_ERR_CUDA;
+}
+
+// ---- plans: a fixed list of tensors, one launch set per step ---------------
+
+}  // extern "C"
+
+struct tlc_plan_s {
+  int device = -1;
+  int count = 0;
+  std::vector<uint64_t> offsets;  // count + 1 arena offsets
+  bool has_inputs = false, has_outputs = false;
+  void *dmem = nullptr;
+  tlc::BatchPlanDev dev{};
+  int32_t *spare_status = nullptr;
+};
+
+extern "C" {
+
+tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
+                           float *const *errs, float *const *ys, tlc_plan *plan) {
+  if (!plan) return TLC_ERR_INVALID_ARG;
+  *plan = nullptr;
+  if (count < 1 || !ns || (!xs && !ys) || (xs && !errs) || (!xs && errs))
+    return TLC_ERR_INVALID_ARG;
+  for (int i = 0; i < count; ++i) {
+    if (!n_ok(ns[i])) return TLC_ERR_INVALID_ARG;
+    if (xs && (!xs[i] || !errs[i])) return TLC_ERR_INVALID_ARG;
+    if (ys && !ys[i]) return TLC_ERR_INVALID_ARG;
+    const size_t fb = ns[i] * sizeof(float);
+    if (xs && overlaps(xs[i], fb, errs[i], fb)) return TLC_ERR_INVALID_ARG;
+  }
+  cudaError_t ce;
+  const tlc::DeviceInfo *dev = current_device(ce);
+  if (!dev) return TLC_ERR_CUDA;
+
+  std::vector<tlc::BatchTensor> T(count);
+  std::vector<tlc::BatchChunk> chunks;
+  std::vector<uint32_t> qtt, dtt;
+  std::vector<uint64_t> offsets(count + 1, 0);
+  const uint32_t dtile = tlc::decode_tile_payload_bytes(false);
+  for (int i = 0; i < count; ++i) {
+    tlc::BatchTensor &t = T[i];
+    t.x = xs ? xs[i] : nullptr;
+    t.err = xs ? errs[i] : nullptr;
+    t.y = ys ? ys[i] : nullptr;
+    t.n = ns[i];
+    t.groups = groups_of(ns[i]);
+    t.cap = 4 + t.groups;
+    t.arena_off = offsets[i];
+    offsets[i + 1] = tlc::align_up(offsets[i] + t.cap, 16);
+    t.q_tile_begin = (uint32_t)qtt.size();
+    t.q_tiles = tlc::compress_tiles(t.n);
+    for (uint32_t k = 0; k < t.q_tiles; ++k) qtt.push_back((uint32_t)i);
+    t.d_tile_begin = (uint32_t)dtt.size();
+    t.d_tiles = (uint32_t)((t.groups + dtile - 1) / dtile);
+    for (uint32_t k = 0; k < t.d_tiles; ++k) dtt.push_back((uint32_t)i);
+    t.vec_q = xs && (((reinterpret_cast<uintptr_t>(t.x) | reinterpret_cast<uintptr_t>(t.err)) &
+                      15) == 0);
+    t.vec_y = ys && ((reinterpret_cast<uintptr_t>(t.y) & 15) == 0);
+    for (uint64_t b = 0; b < t.n; b += tlc::kBatchChunk) chunks.push_back({(uint32_t)i, 0u, b});
+    if (qtt.size() >= (1ull << 31) || dtt.size() >= (1ull << 31) ||
+        chunks.size() >= (1ull << 31))
+      return TLC_ERR_INVALID_ARG;
+  }
+  // device layout: tables, then the zeroed-per-call scratch of each direction
+  const size_t sz_T = tlc::align_up(sizeof(tlc::BatchTensor) * count, 256);
+  const size_t sz_C = tlc::align_up(sizeof(tlc::BatchChunk) * chunks.size(), 256);
+  const size_t sz_Q = tlc::align_up(4 * qtt.size(), 256);
+  const size_t sz_D = tlc::align_up(4 * dtt.size(), 256);
+  const size_t sz_M = tlc::align_up(4 * (size_t)count + 8, 256);      // mbits, q_ticket
+  const size_t sz_QS = tlc::align_up(8 * qtt.size(), 256);
+  const size_t sz_DS = tlc::align_up(8 * (dtt.size() + 1), 256);     // d_ticket, d_status
+  const size_t total = sz_T + sz_C + sz_Q + sz_D + sz_M + sz_QS + sz_DS + 256;
+  tlc_plan_s *P = new tlc_plan_s();
+  P->device = dev->device;
+  P->count = count;
+  P->offsets = offsets;
+  P->has_inputs = xs != nullptr;
+  P->has_outputs = ys != nullptr;
+  if (cudaMalloc(&P->dmem, total) != cudaSuccess) {
+    delete P;
+    return TLC_ERR_CUDA;
+  }
+  char *b = static_cast<char *>(P->dmem);
+  tlc::BatchPlanDev &D = P->dev;
+  D.tensors = reinterpret_cast<tlc::BatchTensor *>(b);
+  D.count = (uint32_t)count;
+  D.chunks = reinterpret_cast<tlc::BatchChunk *>(b + sz_T);
+  D.n_chunks = (uint32_t)chunks.size();
+  D.q_tile_tensor = reinterpret_cast<uint32_t *>(b + sz_T + sz_C);
+  D.n_q_tiles = (uint32_t)qtt.size();
+  D.d_tile_tensor = reinterpret_cast<uint32_t *>(b + sz_T + sz_C + sz_Q);
+  D.n_d_tiles = (uint32_t)dtt.size();
+  char *zq = b + sz_T + sz_C + sz_Q + sz_D;
+  D.mbits = reinterpret_cast<uint32_t *>(zq);
+  D.q_ticket = reinterpret_cast<uint32_t *>(zq + 4 * (size_t)count);
+  D.q_status = reinterpret_cast<uint64_t *>(zq + sz_M);
+  D.q_zero_base = zq;
+  D.q_zero_bytes = sz_M + 8 * qtt.size();
+  char *zd = zq + sz_M + sz_QS;
+  D.d_ticket = reinterpret_cast<uint32_t *>(zd);
+  D.d_status = reinterpret_cast<uint64_t *>(zd + 8);
+  D.d_zero_base = zd;
+  D.d_zero_bytes = 8 * (dtt.size() + 1);
+  P->spare_status = reinterpret_cast<int32_t *>(zd + sz_DS);
+  ce = cudaMemcpy(b, T.data(), sizeof(tlc::BatchTensor) * count, cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess && !chunks.empty())
+    ce = cudaMemcpy(b + sz_T, chunks.data(), sizeof(tlc::BatchChunk) * chunks.size(),
+                    cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpy(b + sz_T + sz_C, qtt.data(), 4 * qtt.size(), cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess)
+    ce = cudaMemcpy(b + sz_T + sz_C + sz_Q, dtt.data(), 4 * dtt.size(), cudaMemcpyHostToDevice);
+  if (ce != cudaSuccess) {
+    cudaFree(P->dmem);
+    delete P;
+    return TLC_ERR_CUDA;
+  }
+  *plan = P;
+  return TLC_OK;
+}
+
+void tlc_plan_destroy(tlc_plan plan) {
+  if (!plan) return;
+  int cur = -1;
+  cudaGetDevice(&cur);
+  if (cur != plan->device) cudaSetDevice(plan->device);
+  cudaFree(plan->dmem);
+  if (cur >= 0 && cur != plan->device) cudaSetDevice(cur);
+  delete plan;
+}
+
+size_t tlc_plan_arena_bytes(tlc_plan plan) { return plan ? plan->offsets.back() : 0; }
+
+size_t tlc_plan_stream_offset(tlc_plan plan, int i) {
+  if (!plan || i < 0 || i >= plan->count) return (size_t)-1;
+  return plan->offsets[i];
+}
+
+static const tlc::DeviceInfo *plan_device(tlc_plan plan) {
+  int cur = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess || cur != plan->device) return nullptr;
+  return tlc::device_info(cur);
+}
+
+tlc_status tlc_compress_batch(tlc_plan plan, float s, uint8_t *arena, uint64_t *out_lens,
+                              int32_t *dev_status, tlc_stream_t stream) {
+  if (!plan || !plan->has_inputs || !arena || !out_lens) return TLC_ERR_INVALID_ARG;
+  if (!(s >= 1.0f && s < 2.0f)) return TLC_ERR_INVALID_ARG;
+  const tlc::DeviceInfo *dev = plan_device(plan);
+  if (!dev) return TLC_ERR_INVALID_ARG;
+  const cudaError_t ce = tlc::launch_compress_batch(
+      *dev, plan->dev, s, arena, out_lens, dev_status ? dev_status : plan->spare_status,
+      wait_limit(), reinterpret_cast<cudaStream_t>(stream));
+  return ce == cudaSuccess ? TLC_OK : TLC_ERR_CUDA;
+}
+
+tlc_status tlc_decompress_batch(tlc_plan plan, const uint8_t *arena, const uint64_t *in_lens,
+                                int accumulate, int32_t *dev_status, tlc_stream_t stream) {
+  if (!plan || !plan->has_outputs || !arena || !in_lens) return TLC_ERR_INVALID_ARG;
+  const tlc::DeviceInfo *dev = plan_device(plan);
+  if (!dev) return TLC_ERR_INVALID_ARG;
+  const cudaError_t ce = tlc::launch_decode_batch(
+      *dev, plan->dev, arena, in_lens, accumulate != 0,
+      dev_status ? dev_status : plan->spare_status, wait_limit(),
+      reinterpret_cast<cudaStream_t>(stream));
+  return ce == cudaSuccess ? TLC_OK : TLC_ERR_CUDA;
 }
 
 tlc_status tlc_test_wait_timeout(uint32_t max_polls, int32_t *dev_status, tlc_stream_t stream) {

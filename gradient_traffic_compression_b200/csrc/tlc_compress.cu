@@ -116,15 +116,6 @@ k_absmax(const float *__restrict__ x, const float *__restrict__ err, uint64_t n,
 #ifndef TLC_Q_MINB
 #define TLC_Q_MINB 6
 #endif
-#ifndef TLC_Q_STREAMING
-#define TLC_Q_STREAMING 0
-#endif
-#ifndef TLC_Q_PREFETCH
-#define TLC_Q_PREFETCH 0
-#endif
-#ifndef TLC_Q_EARLY
-#define TLC_Q_EARLY 0
-#endif
 constexpr int kQThreads = 256;
 constexpr int kQWarps = kQThreads / kWarp;
 constexpr int kChunkElems = 640;   // one warp step: 32 lanes x 5 float4
@@ -140,33 +131,6 @@ static_assert((kZBytes == 8 || kZBytes % 16 == 0) && kTileGroups < 65536, "tile 
 #endif
 constexpr int kLookV = TLC_Q_LOOKV;  // look-back words per lane per round trip
 
-// Ask L2 to fetch [p, p + bytes) ahead of use (bytes a multiple of 16,
-// p 16-byte aligned).  No data moves into the SM; nothing to wait for.
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ float4 ld_in(const float4 *p) {
-#if TLC_Q_STREAMING
-  return __ldcs(p);
-#else
-  return __ldg(p);
-#endif
-}
-__device__ __forceinline__ float4 ld_err(const float4 *p) {
-#if TLC_Q_STREAMING
-  return __ldcs(p);
-#else
-  return *p;
-#endif
-}
-__device__ __forceinline__ void st_err(float4 *p, float4 v) {
-#if TLC_Q_STREAMING
-  __stcs(p, v);
-#else
-  *p = v;
-#endif
-}
 
 struct ZAgg {
   uint32_t all, A, R, tc;
@@ -263,26 +227,30 @@ __device__ __forceinline__ uint32_t pack_groups4(const uint32_t w[5]) {
   return out;
 }
 
-struct QuantArgs {
+// One tensor's compression job, as the tile function sees it.
+struct TileJob {
   const float *x;
   float *err;
   uint64_t n;
   uint64_t groups;
-  float s;
-  const uint32_t *partial;
-  uint32_t n_partial;
-  uint8_t *out;
+  uint8_t *out;       // stream: header then payload
   uint64_t out_cap;
   uint64_t *out_len;
-  uint64_t *status;
-  uint32_t *ticket;
+  uint64_t *status;   // this tensor's tile status words
   uint32_t n_tiles;
-  int32_t *dev_status;
-  uint32_t max_polls;
+  bool vec;           // x and err are 16-byte aligned
 };
 
-__device__ __forceinline__ void put_out(const QuantArgs &a, uint64_t pos, uint8_t v) {
-  if (4 + pos < a.out_cap) a.out[4 + pos] = v;
+// Shared memory of one compress block.
+struct QuantSmem {
+  __align__(16) uint32_t dig[kQWarps][kChunkElems / 4];  // digits q+1, one byte per value
+  __align__(16) uint32_t tile[kTileGroups / 4];          // the tile's quartic bytes
+  uint32_t scan[kQWarps + 1];
+  uint32_t A, cin, tin;
+};
+
+__device__ __forceinline__ void put_out(const TileJob &j, uint64_t pos, uint8_t v) {
+  if (4 + pos < j.out_cap) j.out[4 + pos] = v;
 }
 
 // Decoupled look-back for tile t (whole block calls; warp 0 works): publish
@@ -291,21 +259,21 @@ __device__ __forceinline__ void put_out(const QuantArgs &a, uint64_t pos, uint8_
 // exclusive prefix (emitted count, incoming run length mod 14) to all threads.
 // Each round trip reads 32 * kLookV earlier words: every lane first folds
 // its kLookV words (oldest to nearest), then lane 0 folds the lanes.
-__device__ __forceinline__ void lookback_tile(const QuantArgs &a, uint32_t t, const ZAgg &agg,
-                                              uint32_t &cin, uint32_t &tin, uint32_t &cin_s,
-                                              uint32_t &tin_s) {
+__device__ __forceinline__ void lookback_tile(const TileJob &j, uint32_t t, const ZAgg &agg,
+                                              uint32_t &cin, uint32_t &tin, QuantSmem &sm,
+                                              int32_t *dev_status, uint32_t max_polls) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (warp == 0) {
     if (t == 0) {
       if (lane == 0) {
         uint32_t C = 0, tt = 0;
         eval_agg(C, tt, agg);
-        st_relaxed_u64(a.status, pack_prefix(C, tt));
-        cin_s = 0;
-        tin_s = 0;
+        st_relaxed_u64(j.status, pack_prefix(C, tt));
+        sm.cin = 0;
+        sm.tin = 0;
       }
     } else {
-      if (lane == 0) st_relaxed_u64(a.status + t, pack_agg(agg));
+      if (lane == 0) st_relaxed_u64(j.status + t, pack_agg(agg));
       bool timed_out = false;
       bool have_suffix = false;
       ZAgg suffix = {0, 0, 0, 0};
@@ -313,24 +281,24 @@ __device__ __forceinline__ void lookback_tile(const QuantArgs &a, uint32_t t, co
       uint32_t C = 0, tt = 0;
       for (;;) {
         uint64_t w[kLookV];
-        load_window(a.status, end, pack_prefix(0, 0), a.max_polls, timed_out, w);
+        load_window(j.status, end, pack_prefix(0, 0), max_polls, timed_out, w);
         int jp = kLookV;
         uint64_t wp = 0;
 #pragma unroll
-        for (int j = 0; j < kLookV; ++j)
-          if (jp == kLookV && (w[j] >> kFlagShift) == 2) {
-            jp = j;
-            wp = w[j];
+        for (int k = 0; k < kLookV; ++k)
+          if (jp == kLookV && (w[k] >> kFlagShift) == 2) {
+            jp = k;
+            wp = w[k];
           }
         // this lane's words nearer than its prefix (or all of them), folded
         // from the oldest to the nearest
         ZAgg lagg = {1u, 0u, 0u, 0u};
         bool have = false;
 #pragma unroll
-        for (int j = kLookV - 1; j >= 0; --j) {
-          if (j < jp) {
-            const ZAgg aj = unpack_agg(w[j]);
-            lagg = have ? compose(lagg, aj) : aj;
+        for (int k = kLookV - 1; k >= 0; --k) {
+          if (k < jp) {
+            const ZAgg ak = unpack_agg(w[k]);
+            lagg = have ? compose(lagg, ak) : ak;
             have = true;
           }
         }
@@ -370,286 +338,384 @@ __device__ __forceinline__ void lookback_tile(const QuantArgs &a, uint32_t t, co
         have_suffix = true;
         end -= kWarp * kLookV;
       }
-      if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(a.dev_status, TLC_ERR_TIMEOUT);
+      if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(dev_status, TLC_ERR_TIMEOUT);
       if (lane == 0) {
-        cin_s = C;
-        tin_s = tt;
+        sm.cin = C;
+        sm.tin = tt;
         uint32_t Ci = C, ti = tt;
         eval_agg(Ci, ti, agg);
-        st_relaxed_u64(a.status + t, pack_prefix(Ci, ti));
+        st_relaxed_u64(j.status + t, pack_prefix(Ci, ti));
       }
     }
   }
   __syncthreads();
-  cin = cin_s;
-  tin = tin_s;
+  cin = sm.cin;
+  tin = sm.tin;
 }
 
 // Stream header (first tile) and the closing remainder + length (last tile).
-__device__ __forceinline__ void finish_tile(const QuantArgs &a, uint32_t t, const ZAgg &agg,
+__device__ __forceinline__ void finish_tile(const TileJob &j, uint32_t t, const ZAgg &agg,
                                             uint32_t cin, uint32_t tin, float scale) {
   if (threadIdx.x != 0) return;
   if (t == 0) {
     const uint32_t sb = __float_as_uint(scale);
-    a.out[0] = sb & 0xff;
-    a.out[1] = (sb >> 8) & 0xff;
-    a.out[2] = (sb >> 16) & 0xff;
-    a.out[3] = (sb >> 24) & 0xff;
+    j.out[0] = sb & 0xff;
+    j.out[1] = (sb >> 8) & 0xff;
+    j.out[2] = (sb >> 16) & 0xff;
+    j.out[3] = (sb >> 24) & 0xff;
   }
-  if (t == a.n_tiles - 1) {
+  if (t == j.n_tiles - 1) {
     uint32_t C = cin, tt = tin;
     eval_agg(C, tt, agg);
-    if (tt) put_out(a, C, remainder_byte(tt));
-    *a.out_len = 4ull + C + (tt ? 1u : 0u);
+    if (tt) put_out(j, C, remainder_byte(tt));
+    *j.out_len = 4ull + C + (tt ? 1u : 0u);
   }
 }
+
+// One tile of 4096 byte groups (20480 values) of one tensor: quantize and
+// update the error buffer, pack the quartic bytes into shared memory,
+// zero-run encode them and place the output after the look-back.  The whole
+// block calls it; it ends with the block synchronised.
+__device__ __forceinline__ void quant_tile(const TileJob &j, uint32_t t, float scale, float thr,
+                                           QuantSmem &sm, int32_t *dev_status,
+                                           uint32_t max_polls) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) sm.A = 0xffffffffu;
+  const uint64_t g0 = (uint64_t)t * kTileGroups;
+  const uint32_t tgv = (uint32_t)umin64(kTileGroups, j.groups - g0);
+  const uint64_t e_tile = g0 * 5;
+  const bool full = j.vec && (e_tile + kTileElems <= j.n);
+
+  // ---- quantize + error update + quartic pack --------------------------
+#pragma unroll 1
+  for (int it = 0; it < kQIters; ++it) {
+    const int c = it * kQWarps + warp;
+    const uint64_t e0 = e_tile + (uint64_t)c * kChunkElems;
+    if (full) {
+      const float4 *x4 = reinterpret_cast<const float4 *>(j.x + e0);
+      float4 *err4 = reinterpret_cast<float4 *>(j.err + e0);
+      float4 xv[5], ev[5];
+#pragma unroll
+      for (int k = 0; k < 5; ++k) {
+        xv[k] = __ldg(x4 + lane + 32 * k);
+        ev[k] = err4[lane + 32 * k];
+      }
+#pragma unroll
+      for (int k = 0; k < 5; ++k) {
+        float4 o;
+        uint32_t dw;
+        dw = quant_digit(__fadd_rn(xv[k].x, ev[k].x), scale, thr, o.x);
+        dw |= quant_digit(__fadd_rn(xv[k].y, ev[k].y), scale, thr, o.y) << 8;
+        dw |= quant_digit(__fadd_rn(xv[k].z, ev[k].z), scale, thr, o.z) << 16;
+        dw |= quant_digit(__fadd_rn(xv[k].w, ev[k].w), scale, thr, o.w) << 24;
+        err4[lane + 32 * k] = o;
+        sm.dig[warp][lane + 32 * k] = dw;
+      }
+    } else if (e0 < j.n) {
+      // tail or unaligned chunk: scalar and bounds-checked
+#pragma unroll 1
+      for (int k = 0; k < 5; ++k) {
+        uint32_t dw = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint64_t e = e0 + 4 * (uint64_t)(lane + 32 * k) + q;
+          uint32_t d = 1;
+          if (e < j.n) {
+            float o;
+            d = quant_digit(__fadd_rn(j.x[e], j.err[e]), scale, thr, o);
+            j.err[e] = o;
+          }
+          dw |= d << (8 * q);
+        }
+        sm.dig[warp][lane + 32 * k] = dw;
+      }
+    } else {
+      // chunk entirely past the end: all-zero groups
+#pragma unroll
+      for (int k = 0; k < 5; ++k) sm.dig[warp][lane + 32 * k] = 0x01010101u;
+    }
+    __syncwarp();
+    uint32_t w5[5];
+#pragma unroll
+    for (int k = 0; k < 5; ++k) w5[k] = sm.dig[warp][5 * lane + k];
+    sm.tile[c * (kChunkGroups / 4) + lane] = pack_groups4(w5);
+    __syncwarp();
+  }
+  __syncthreads();
+
+  // ---- zero-run encoding: local analysis ---------------------------------
+  uint32_t qw[kZWords];
+  if constexpr (kZWords == 2) {
+    const uint2 q2 = reinterpret_cast<const uint2 *>(sm.tile)[threadIdx.x];
+    qw[0] = q2.x;
+    qw[1] = q2.y;
+  } else {
+#pragma unroll
+    for (int v = 0; v < kZWords / 4; ++v) {
+      const uint4 q4 = reinterpret_cast<const uint4 *>(sm.tile)[threadIdx.x * (kZWords / 4) + v];
+      qw[4 * v] = q4.x;
+      qw[4 * v + 1] = q4.y;
+      qw[4 * v + 2] = q4.z;
+      qw[4 * v + 3] = q4.w;
+    }
+  }
+  bool mine_all = true;
+#pragma unroll
+  for (int w = 0; w < kZWords; ++w) mine_all = mine_all && qw[w] == 0x79797979u;
+  // groups past the end of the tensor are all-zero (121) by construction
+  if (__syncthreads_and(mine_all)) {
+    // Entirely 121s: only full 14-chunks of the run end inside the tile.
+    const ZAgg agg = {1u, tgv, 0u, 0u};
+    uint32_t cin, tin;
+    lookback_tile(j, t, agg, cin, tin, sm, dev_status, max_polls);
+    const uint32_t cnt = (tin + tgv) / 14u;
+    for (uint32_t i = threadIdx.x; i < cnt; i += kQThreads) put_out(j, (uint64_t)cin + i, 255);
+    finish_tile(j, t, agg, cin, tin, scale);
+    __syncthreads();
+    return;
+  }
+  const int p0 = (int)threadIdx.x * kZBytes;
+  int fnz = -1, lnz = -1;
+#pragma unroll
+  for (int k = 0; k < kZBytes; ++k) {
+    const uint32_t b = (qw[k >> 2] >> (8 * (k & 3))) & 0xffu;
+    const int p = p0 + k;
+    if (p < (int)tgv && b != 121u) {
+      if (fnz < 0) fnz = p;
+      lnz = p;
+    }
+  }
+  int32_t lnz_all;
+  const int prev_in =
+      block_exclusive_max<kQThreads>(lnz, reinterpret_cast<int32_t *>(sm.scan), lnz_all);
+  if (prev_in < 0 && fnz >= 0) sm.A = (uint32_t)fnz;
+
+  uint32_t cnt = 0;
+  {
+    int prev = prev_in;
+#pragma unroll
+    for (int k = 0; k < kZBytes; ++k) {
+      const uint32_t b = (qw[k >> 2] >> (8 * (k & 3))) & 0xffu;
+      const int p = p0 + k;
+      if (p >= (int)tgv) break;
+      if (b == 121u) {
+        if (prev >= 0 && (p - prev - 1) % 14 == 13) ++cnt;
+      } else {
+        if (prev >= 0 && (p - 1 - prev) % 14 != 0) ++cnt;
+        ++cnt;
+        prev = p;
+      }
+    }
+  }
+  uint32_t R;
+  const uint32_t off = block_exclusive_sum<kQThreads>(cnt, sm.scan, R);
+
+  ZAgg agg;
+  agg.all = lnz_all < 0 ? 1u : 0u;
+  agg.A = agg.all ? tgv : sm.A;
+  agg.R = R;
+  agg.tc = agg.all ? 0u : (uint32_t)((int)tgv - 1 - lnz_all) % 14u;
+
+  // ---- decoupled look-back -----------------------------------------------
+  uint32_t cin, tin;
+  lookback_tile(j, t, agg, cin, tin, sm, dev_status, max_polls);
+
+  // ---- emission ------------------------------------------------------------
+  {
+    uint64_t k_out = (uint64_t)cin + lead_count(agg, tin) + off;
+    int prev = prev_in;
+#pragma unroll
+    for (int k = 0; k < kZBytes; ++k) {
+      const uint32_t b = (qw[k >> 2] >> (8 * (k & 3))) & 0xffu;
+      const int p = p0 + k;
+      if (p >= (int)tgv) break;
+      if (b == 121u) {
+        if (prev < 0) {
+          if ((tin + p) % 14u == 13u) put_out(j, cin + (tin + p) / 14u, 255);
+        } else if ((p - prev - 1) % 14 == 13) {
+          put_out(j, k_out++, 255);
+        }
+      } else {
+        if (prev < 0) {
+          const uint32_t r = (tin + p) % 14u;
+          if (r) put_out(j, cin + (tin + p) / 14u, remainder_byte(r));
+        } else {
+          const uint32_t r = (uint32_t)(p - 1 - prev) % 14u;
+          if (r) put_out(j, k_out++, remainder_byte(r));
+        }
+        put_out(j, k_out++, (uint8_t)b);
+        prev = p;
+      }
+    }
+  }
+  finish_tile(j, t, agg, cin, tin, scale);
+  __syncthreads();
+}
+
+// scale = M * s and the zero-band threshold from the bits of M; false when
+// the step is non-finite (M not finite, or M * s overflows).
+__device__ __forceinline__ bool scale_from_max(uint32_t mbits, float s, float &scale,
+                                               float &thr) {
+  if (mbits >= 0x7f800000u) return false;
+  scale = __fmul_rn(__uint_as_float(mbits), s);
+  if (!isfinite(scale)) return false;
+  thr = zero_band_threshold(scale, mbits == 0);
+  return true;
+}
+
+struct QuantArgs {
+  const float *x;
+  float *err;
+  uint64_t n;
+  uint64_t groups;
+  float s;
+  const uint32_t *partial;
+  uint32_t n_partial;
+  uint8_t *out;
+  uint64_t out_cap;
+  uint64_t *out_len;
+  uint64_t *status;
+  uint32_t *ticket;
+  uint32_t n_tiles;
+  int32_t *dev_status;
+  uint32_t max_polls;
+};
 
 #if TLC_Q_MINB > 1
 #define TLC_Q_BOUNDS __launch_bounds__(kQThreads, TLC_Q_MINB)
 #else
 #define TLC_Q_BOUNDS __launch_bounds__(kQThreads)
 #endif
-template <bool kVec>
-__global__ void TLC_Q_BOUNDS
-k_quant_zre(const QuantArgs a) {
-  __shared__ __align__(16) uint32_t dig_s[kQWarps][kChunkElems / 4];
-  __shared__ __align__(16) uint32_t tile_s[kTileGroups / 4];
-  __shared__ uint32_t scan_s[kQWarps + 1];
-  __shared__ uint32_t tile_id_s, A_s, cin_s, tin_s;
-  __shared__ float scale_s;
-  __shared__ int state_s;  // 0 ok, 1 M == 0, 2 non-finite
 
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+template <bool kVec>
+__global__ void TLC_Q_BOUNDS k_quant_zre(const QuantArgs a) {
+  __shared__ QuantSmem sm;
+  __shared__ uint32_t tile_id_s;
+  __shared__ float scale_s, thr_s;
+  __shared__ int ok_s;
 
   // M from the per-block partial maxima of k_absmax.
-  if (warp == 0) {
+  if (threadIdx.x < kWarp) {
     uint32_t mb = 0;
-    for (uint32_t i = lane; i < a.n_partial; i += kWarp) mb = max(mb, a.partial[i]);
+    for (uint32_t i = threadIdx.x; i < a.n_partial; i += kWarp) mb = max(mb, a.partial[i]);
     mb = __reduce_max_sync(0xffffffffu, mb);
-    if (lane == 0) {
-      int st = 0;
-      float scale = 0.0f;
-      if (mb >= 0x7f800000u) {
-        st = 2;
-      } else {
-        scale = __fmul_rn(__uint_as_float(mb), a.s);
-        if (!isfinite(scale)) st = 2;
-        else if (mb == 0) st = 1;
-      }
+    if (threadIdx.x == 0) {
+      float scale = 0.0f, thr = 0.0f;
+      ok_s = scale_from_max(mb, a.s, scale, thr) ? 1 : 0;
       scale_s = scale;
-      state_s = st;
+      thr_s = thr;
     }
   }
   __syncthreads();
-  if (state_s == 2) {
+  if (!ok_s) {
     if (blockIdx.x == 0 && threadIdx.x == 0) {
       report(a.dev_status, TLC_ERR_NONFINITE);
       *a.out_len = 0;
     }
     return;
   }
-  const float scale = scale_s;
-  const float thr = zero_band_threshold(scale, state_s == 1);
-
-#if TLC_Q_EARLY
-  if (threadIdx.x == 0) tile_id_s = atomicAdd(a.ticket, 1u);
-#endif
+  const float scale = scale_s, thr = thr_s;
+  const TileJob job = {a.x, a.err, a.n, a.groups, a.out, a.out_cap, a.out_len,
+                       a.status, a.n_tiles, kVec};
   for (;;) {
-    if (threadIdx.x == 0) {
-#if !TLC_Q_EARLY
-      tile_id_s = atomicAdd(a.ticket, 1u);
-#endif
-      A_s = 0xffffffffu;
-    }
+    if (threadIdx.x == 0) tile_id_s = atomicAdd(a.ticket, 1u);
     __syncthreads();
     const uint32_t t = tile_id_s;
     if (t >= a.n_tiles) break;
+    quant_tile(job, t, scale, thr, sm, a.dev_status, a.max_polls);
+  }
+}
 
-    const uint64_t g0 = (uint64_t)t * kTileGroups;
-    const uint32_t tgv = (uint32_t)umin64(kTileGroups, a.groups - g0);
-    const uint64_t e_tile = g0 * 5;
-    const bool full = kVec && (e_tile + kTileElems <= a.n);
-
-    // ---- quantize + error update + quartic pack ------------------------
-#pragma unroll 1
-    for (int it = 0; it < kQIters; ++it) {
-      const int c = it * kQWarps + warp;
-      const uint64_t e0 = e_tile + (uint64_t)c * kChunkElems;
-      if (full) {
-        const float4 *x4 = reinterpret_cast<const float4 *>(a.x + e0);
-        float4 *err4 = reinterpret_cast<float4 *>(a.err + e0);
-        float4 xv[5], ev[5];
+// ------------------------------------------------- batched (tensor lists) --
+// Magnitude pass over a list of tensors: one block per chunk of up to
+// kBatchChunk values of one tensor, one atomic maximum per tensor.
+__global__ void __launch_bounds__(kAbsThreads)
+k_absmax_batch(const BatchTensor *__restrict__ tensors, const BatchChunk *__restrict__ chunks,
+               uint32_t *__restrict__ mbits) {
+  const BatchChunk ch = chunks[blockIdx.x];
+  const BatchTensor &T = tensors[ch.tensor];
+  const uint64_t b = ch.start, e = umin64(ch.start + kBatchChunk, T.n);
+  uint32_t m = 0;
+  if (T.vec_q) {
+    // b is a multiple of kBatchChunk, so x + b and err + b stay 16-byte aligned
+    const uint64_t n4 = (e - b) >> 2;
+    const float4 *x4 = reinterpret_cast<const float4 *>(T.x + b);
+    const float4 *e4 = reinterpret_cast<const float4 *>(T.err + b);
+    constexpr int kU = kBatchChunk / 4 / kAbsThreads;
+    float4 xa[kU], ea[kU];
 #pragma unroll
-        for (int j = 0; j < 5; ++j) {
-          xv[j] = ld_in(x4 + lane + 32 * j);
-          ev[j] = ld_err(err4 + lane + 32 * j);
-        }
-#pragma unroll
-        for (int j = 0; j < 5; ++j) {
-          float4 o;
-          uint32_t dw;
-          dw = quant_digit(__fadd_rn(xv[j].x, ev[j].x), scale, thr, o.x);
-          dw |= quant_digit(__fadd_rn(xv[j].y, ev[j].y), scale, thr, o.y) << 8;
-          dw |= quant_digit(__fadd_rn(xv[j].z, ev[j].z), scale, thr, o.z) << 16;
-          dw |= quant_digit(__fadd_rn(xv[j].w, ev[j].w), scale, thr, o.w) << 24;
-          st_err(err4 + lane + 32 * j, o);
-          dig_s[warp][lane + 32 * j] = dw;
-        }
-      } else if (e0 < a.n) {
-        // tail or unaligned chunk: scalar and bounds-checked
-#pragma unroll 1
-        for (int j = 0; j < 5; ++j) {
-          uint32_t dw = 0;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t e = e0 + 4 * (uint64_t)(lane + 32 * j) + k;
-            uint32_t d = 1;
-            if (e < a.n) {
-              float o;
-              d = quant_digit(__fadd_rn(a.x[e], a.err[e]), scale, thr, o);
-              a.err[e] = o;
-            }
-            dw |= d << (8 * k);
-          }
-          dig_s[warp][lane + 32 * j] = dw;
-        }
+    for (int u = 0; u < kU; ++u) {
+      const uint64_t i = threadIdx.x + (uint64_t)u * kAbsThreads;
+      if (i < n4) {
+        xa[u] = __ldg(x4 + i);
+        ea[u] = __ldg(e4 + i);
       } else {
-        // chunk entirely past the end: all-zero groups
-#pragma unroll
-        for (int j = 0; j < 5; ++j) dig_s[warp][lane + 32 * j] = 0x01010101u;
+        xa[u] = ea[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
-      __syncwarp();
-      uint32_t w5[5];
+    }
 #pragma unroll
-      for (int k = 0; k < 5; ++k) w5[k] = dig_s[warp][5 * lane + k];
-      tile_s[c * (kChunkGroups / 4) + lane] = pack_groups4(w5);
-      __syncwarp();
+    for (int u = 0; u < kU; ++u) {
+      m = max(m, abs_bits(__fadd_rn(xa[u].x, ea[u].x)));
+      m = max(m, abs_bits(__fadd_rn(xa[u].y, ea[u].y)));
+      m = max(m, abs_bits(__fadd_rn(xa[u].z, ea[u].z)));
+      m = max(m, abs_bits(__fadd_rn(xa[u].w, ea[u].w)));
     }
-    __syncthreads();
-#if TLC_Q_EARLY
-    // The next tile's ticket is taken now, so its loads can start (through
-    // L2) while this tile is encoded.  A block handles its tickets in
-    // increasing order, so no look-back ever waits on a later ticket.
-    if (threadIdx.x == 0) {
-      const uint32_t tn = atomicAdd(a.ticket, 1u);
-      tile_id_s = tn;
-#if TLC_Q_PREFETCH
-      const uint64_t en = (uint64_t)tn * kTileElems;
-      if (kVec && tn < a.n_tiles && en + kTileElems <= a.n) {
-        prefetch_l2(a.x + en, (uint32_t)(kTileElems * 4));
-        prefetch_l2(a.err + en, (uint32_t)(kTileElems * 4));
-      }
-#endif
-    }
-#endif
+    const uint64_t r = b + (n4 << 2) + threadIdx.x;
+    if (r < e) m = max(m, abs_bits(__fadd_rn(T.x[r], T.err[r])));
+  } else {
+    for (uint64_t i = b + threadIdx.x; i < e; i += kAbsThreads)
+      m = max(m, abs_bits(__fadd_rn(T.x[i], T.err[i])));
+  }
+  __shared__ uint32_t wmax[kAbsThreads / kWarp];
+  m = __reduce_max_sync(0xffffffffu, m);
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < kWarp) {
+    uint32_t v = threadIdx.x < kAbsThreads / kWarp ? wmax[threadIdx.x] : 0u;
+    v = __reduce_max_sync(0xffffffffu, v);
+    if (threadIdx.x == 0) atomicMax(mbits + ch.tensor, v);
+  }
+}
 
-    // ---- zero-run encoding: local analysis -----------------------------
-    uint32_t qw[kZWords];
-    if constexpr (kZWords == 2) {
-      const uint2 q2 = reinterpret_cast<const uint2 *>(tile_s)[threadIdx.x];
-      qw[0] = q2.x;
-      qw[1] = q2.y;
-    } else {
-#pragma unroll
-      for (int v = 0; v < kZWords / 4; ++v) {
-        const uint4 q4 = reinterpret_cast<const uint4 *>(tile_s)[threadIdx.x * (kZWords / 4) + v];
-        qw[4 * v] = q4.x;
-        qw[4 * v + 1] = q4.y;
-        qw[4 * v + 2] = q4.z;
-        qw[4 * v + 3] = q4.w;
+struct BatchQuantArgs {
+  const BatchTensor *tensors;
+  const uint32_t *tile_tensor;  // tensor of each global tile
+  const uint32_t *mbits;        // per-tensor bits of M
+  float s;
+  uint8_t *arena;
+  uint64_t *out_lens;
+  uint64_t *status;             // all tensors' tile status words
+  uint32_t *ticket;
+  uint32_t n_tiles;             // over all tensors
+  int32_t *dev_status;
+  uint32_t max_polls;
+};
+
+// Quantize + encode over a list of tensors: tiles of all tensors in one
+// ticket order (tensor by tensor), each look-back confined to its tensor.
+__global__ void TLC_Q_BOUNDS k_quant_zre_batch(const BatchQuantArgs a) {
+  __shared__ QuantSmem sm;
+  __shared__ uint32_t tile_id_s;
+  for (;;) {
+    if (threadIdx.x == 0) tile_id_s = atomicAdd(a.ticket, 1u);
+    __syncthreads();
+    const uint32_t u = tile_id_s;
+    if (u >= a.n_tiles) break;
+    const uint32_t id = a.tile_tensor[u];
+    const BatchTensor &T = a.tensors[id];
+    const uint32_t t = u - T.q_tile_begin;
+    float scale = 0.0f, thr = 0.0f;
+    if (!scale_from_max(a.mbits[id], a.s, scale, thr)) {
+      if (t == 0 && threadIdx.x == 0) {
+        report(a.dev_status, TLC_ERR_NONFINITE);
+        a.out_lens[id] = 0;
       }
-    }
-    bool mine_all = true;
-#pragma unroll
-    for (int w = 0; w < kZWords; ++w) mine_all = mine_all && qw[w] == 0x79797979u;
-    // groups past the end of the tensor are all-zero (121) by construction
-    const bool tile_all = __syncthreads_and(mine_all);
-    if (tile_all) {
-      // Entirely 121s: only full 14-chunks of the run end inside the tile.
-      ZAgg agg = {1u, tgv, 0u, 0u};
-      uint32_t cin, tin;
-      lookback_tile(a, t, agg, cin, tin, cin_s, tin_s);
-      const uint32_t cnt = (tin + tgv) / 14u;
-      for (uint32_t i = threadIdx.x; i < cnt; i += kQThreads) put_out(a, (uint64_t)cin + i, 255);
-      finish_tile(a, t, agg, cin, tin, scale);
       __syncthreads();
       continue;
     }
-    const int p0 = (int)threadIdx.x * kZBytes;
-    int fnz = -1, lnz = -1;
-#pragma unroll
-    for (int k = 0; k < kZBytes; ++k) {
-      const uint32_t b = (qw[k >> 2] >> (8 * (k & 3))) & 0xffu;
-      const int p = p0 + k;
-      if (p < (int)tgv && b != 121u) {
-        if (fnz < 0) fnz = p;
-        lnz = p;
-      }
-    }
-    int32_t lnz_all;
-    const int prev_in = block_exclusive_max<kQThreads>(lnz, reinterpret_cast<int32_t *>(scan_s), lnz_all);
-    if (prev_in < 0 && fnz >= 0) A_s = (uint32_t)fnz;
-
-    uint32_t cnt = 0;
-    {
-      int prev = prev_in;
-#pragma unroll
-      for (int k = 0; k < kZBytes; ++k) {
-        const uint32_t b = (qw[k >> 2] >> (8 * (k & 3))) & 0xffu;
-        const int p = p0 + k;
-        if (p >= (int)tgv) break;
-        if (b == 121u) {
-          if (prev >= 0 && (p - prev - 1) % 14 == 13) ++cnt;
-        } else {
-          if (prev >= 0 && (p - 1 - prev) % 14 != 0) ++cnt;
-          ++cnt;
-          prev = p;
-        }
-      }
-    }
-    uint32_t R;
-    const uint32_t off = block_exclusive_sum<kQThreads>(cnt, scan_s, R);
-
-    ZAgg agg;
-    agg.all = lnz_all < 0 ? 1u : 0u;
-    agg.A = agg.all ? tgv : A_s;
-    agg.R = R;
-    agg.tc = agg.all ? 0u : (uint32_t)((int)tgv - 1 - lnz_all) % 14u;
-
-    // ---- decoupled look-back -------------------------------------------
-    uint32_t cin, tin;
-    lookback_tile(a, t, agg, cin, tin, cin_s, tin_s);
-
-    // ---- emission --------------------------------------------------------
-    {
-      uint64_t k_out = (uint64_t)cin + lead_count(agg, tin) + off;
-      int prev = prev_in;
-#pragma unroll
-      for (int k = 0; k < kZBytes; ++k) {
-        const uint32_t b = (qw[k >> 2] >> (8 * (k & 3))) & 0xffu;
-        const int p = p0 + k;
-        if (p >= (int)tgv) break;
-        if (b == 121u) {
-          if (prev < 0) {
-            if ((tin + p) % 14u == 13u) put_out(a, cin + (tin + p) / 14u, 255);
-          } else if ((p - prev - 1) % 14 == 13) {
-            put_out(a, k_out++, 255);
-          }
-        } else {
-          if (prev < 0) {
-            const uint32_t r = (tin + p) % 14u;
-            if (r) put_out(a, cin + (tin + p) / 14u, remainder_byte(r));
-          } else {
-            const uint32_t r = (uint32_t)(p - 1 - prev) % 14u;
-            if (r) put_out(a, k_out++, remainder_byte(r));
-          }
-          put_out(a, k_out++, (uint8_t)b);
-          prev = p;
-        }
-      }
-    }
-    finish_tile(a, t, agg, cin, tin, scale);
-    __syncthreads();
+    const TileJob job = {T.x, T.err, T.n, T.groups, a.arena + T.arena_off, T.cap,
+                         a.out_lens + id, a.status + T.q_tile_begin, T.q_tiles, T.vec_q != 0};
+    quant_tile(job, t, scale, thr, sm, a.dev_status, a.max_polls);
   }
 }
 
@@ -717,6 +783,43 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
     k_quant_zre<false><<<grid, kQThreads, 0, stream>>>(qa);
   timing_end(kKindQuantZre, stream);
   return cudaGetLastError();
+}
+
+cudaError_t launch_compress_batch(const DeviceInfo &dev, const BatchPlanDev &p, float s,
+                                  uint8_t *arena, uint64_t *out_lens, int32_t *dev_status,
+                                  uint32_t max_polls, cudaStream_t stream) {
+  // the per-tensor maxima, the ticket and the tile status words start at 0
+  cudaError_t e = cudaMemsetAsync(p.q_zero_base, 0, p.q_zero_bytes, stream);
+  if (e != cudaSuccess) return e;
+  timing_begin(kKindAbsmax, stream);
+  k_absmax_batch<<<p.n_chunks, kAbsThreads, 0, stream>>>(p.tensors, p.chunks, p.mbits);
+  timing_end(kKindAbsmax, stream);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  BatchQuantArgs qa;
+  qa.tensors = p.tensors;
+  qa.tile_tensor = p.q_tile_tensor;
+  qa.mbits = p.mbits;
+  qa.s = s;
+  qa.arena = arena;
+  qa.out_lens = out_lens;
+  qa.status = p.q_status;
+  qa.ticket = p.q_ticket;
+  qa.n_tiles = p.n_q_tiles;
+  qa.dev_status = dev_status;
+  qa.max_polls = max_polls;
+  uint32_t grid = (uint32_t)dev.sm_count * (uint32_t)(dev.occ_quant_batch > 0 ? dev.occ_quant_batch : 1);
+  if (grid > p.n_q_tiles) grid = p.n_q_tiles;
+  timing_begin(kKindQuantZre, stream);
+  k_quant_zre_batch<<<grid, kQThreads, 0, stream>>>(qa);
+  timing_end(kKindQuantZre, stream);
+  return cudaGetLastError();
+}
+
+int occupancy_quant_batch() {
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_quant_zre_batch, kQThreads, 0);
+  return occ;
 }
 
 int occupancy_quant(bool vec) {

@@ -48,6 +48,8 @@ struct DecodeShape {
 #endif
 constexpr int kLookV = TLC_D_LOOKV;   // look-back words per lane per round trip
 
+size_t decode_smem_bytes(bool accumulate);
+
 struct DecodeArgs {
   const uint8_t *in;
   const uint64_t *len_dev;
@@ -118,229 +120,329 @@ __device__ __forceinline__ float dequant(uint32_t dig, float scale) {
   return dig == 1u ? 0.0f : (dig == 2u ? scale : -scale);
 }
 
+// One stream's decode job, as the tile function sees it.
+struct DecodeJob {
+  const uint8_t *payload;  // stream bytes after the 4-byte header
+  uint64_t m;              // payload length
+  uint64_t n, groups;
+  float scale;
+  float *y;                // output (kWrite) or accumulation buffer
+  uint64_t *status;        // this stream's tile status words
+  uint32_t n_tiles;        // tiles actually present: ceil(m / tile)
+  bool vec;                // y is 16-byte aligned
+};
+
+struct DecodeSmem {
+  uint16_t lut[256];       // base-3 digits of every quartic byte
+  uint32_t scan[kDThreads / kWarp + 1];
+  uint64_t o;
+};
+
+// Validate a stream (length and header) and return its payload length and
+// scale.  Corrupt when the length is below 4 or above the readable capacity,
+// the payload would be longer than the tensor's groups or empty, or the
+// header is negative or not finite.
+__device__ __forceinline__ bool read_stream_header(const uint8_t *in, const uint64_t *len_dev,
+                                                   uint64_t cap, uint64_t groups, uint64_t &m,
+                                                   float &scale) {
+  const uint64_t L = len_dev ? *len_dev : cap;
+  if (L < 4 || L > cap || L - 4 > groups || L == 4) return false;
+  const uint32_t hb = (uint32_t)in[0] | ((uint32_t)in[1] << 8) | ((uint32_t)in[2] << 16) |
+                      ((uint32_t)in[3] << 24);
+  if (hb >= 0x7f800000u) return false;  // negative, infinite or NaN scale
+  m = L - 4;
+  scale = __uint_as_float(hb);
+  return true;
+}
+
+// One tile of one stream; the whole block calls it and it ends synchronised.
+template <int kMode>
+__device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, DecodeSmem &sm,
+                                            uint8_t *grp_s, int32_t *dev_status,
+                                            uint32_t max_polls) {
+  constexpr int kDBytes = DecodeShape<kMode>::kBytes;
+  constexpr int kDTile = DecodeShape<kMode>::kTile;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float scale = j.scale;
+
+  // ---- load the tile's payload bytes, expansion counts, block scan -------
+  const uint64_t b0 = (uint64_t)u * kDTile + (uint64_t)threadIdx.x * kDBytes;
+  uint32_t bw[kDBytes / 4];
+#pragma unroll
+  for (int k = 0; k < kDBytes / 4; ++k) bw[k] = 0x79797979u;
+  int nvalid = 0;
+  if (b0 + kDBytes <= j.m && ((reinterpret_cast<uintptr_t>(j.payload + b0) & 3) == 0)) {
+    const uint32_t *p32 = reinterpret_cast<const uint32_t *>(j.payload + b0);
+#pragma unroll
+    for (int k = 0; k < kDBytes / 4; ++k) bw[k] = __ldg(p32 + k);
+    nvalid = kDBytes;
+  } else {
+#pragma unroll
+    for (int k = 0; k < kDBytes; ++k) {
+      if (b0 + k < j.m) {
+        const uint32_t b = __ldg(j.payload + b0 + k);
+        bw[k >> 2] = (bw[k >> 2] & ~(0xffu << (8 * (k & 3)))) | (b << (8 * (k & 3)));
+        nvalid = k + 1;
+      }
+    }
+  }
+  uint32_t esum = 0;
+#pragma unroll
+  for (int k = 0; k < kDBytes; ++k) {
+    const uint32_t b = (bw[k >> 2] >> (8 * (k & 3))) & 0xffu;
+    if (k < nvalid) esum += b >= 243u ? b - 241u : 1u;
+  }
+  uint32_t E;
+  const uint32_t off = block_exclusive_sum<kDThreads>(esum, sm.scan, E);
+  // Dense output always expands the tile's groups in shared memory.  The
+  // accumulate mode does so too when the tile is mostly literals (then a
+  // coalesced float4 pass over acc is cheapest); for escape-heavy tiles it
+  // visits only the literal groups.
+  const bool expand = kMode == kWrite || E <= 4u * (uint32_t)kDTile;
+
+  // ---- look-back (warp 0); the other warps pre-fill zero groups ----------
+  if (warp == 0) {
+    bool timed_out = false;
+    const uint64_t O = lookback_sum(j.status, u, E, max_polls, timed_out);
+    if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(dev_status, TLC_ERR_TIMEOUT);
+    if (lane == 0) sm.o = O;
+  } else if (expand) {
+    const uint32_t words = (E + 15) / 16;
+    for (uint32_t w = threadIdx.x - kWarp; w < words; w += kDThreads - kWarp)
+      reinterpret_cast<uint4 *>(grp_s)[w] =
+          make_uint4(0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u);
+  }
+  __syncthreads();
+  const uint64_t O = sm.o;
+  if (threadIdx.x == 0) {
+    const bool last = (u == j.n_tiles - 1);
+    if (O + E > j.groups || (last && O + E != j.groups)) report(dev_status, TLC_ERR_CORRUPT);
+  }
+  const uint64_t Ec = O >= j.groups ? 0 : umin64(E, j.groups - O);
+
+  if (expand) {
+    // literal bytes into the expanded group buffer
+    uint32_t pos = off;
+#pragma unroll
+    for (int k = 0; k < kDBytes; ++k) {
+      const uint32_t b = (bw[k >> 2] >> (8 * (k & 3))) & 0xffu;
+      if (k < nvalid) {
+        if (b >= 243u) {
+          pos += b - 241u;
+        } else {
+          grp_s[pos] = (uint8_t)b;
+          ++pos;
+        }
+      }
+    }
+    __syncthreads();
+    // groups [O, O+Ec) -> values [5 O, min(5 (O+Ec), n))
+    const uint64_t e_begin = 5 * O;
+    const uint64_t e_end = umin64(5 * (O + Ec), j.n);
+    if (e_end > e_begin) {
+      const uint32_t o32 = (uint32_t)O;
+      // one value: written (dense output) or added where non-zero (accumulate)
+      auto put = [&](uint64_t e) {
+        const uint32_t e32 = (uint32_t)e;
+        const uint32_t g = e32 / 5u;
+        const uint32_t dig = (sm.lut[grp_s[g - o32]] >> (2 * (e32 - 5u * g))) & 3u;
+        if (kMode == kWrite)
+          j.y[e] = dequant(dig, scale);
+        else if (dig != 1u)
+          j.y[e] = __fadd_rn(j.y[e], dequant(dig, scale));
+      };
+      const uint64_t v0 = (e_begin + 3) / 4, v1 = e_end / 4;
+      if (!j.vec || v1 <= v0) {
+        for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) put(e);
+      } else {
+        // Values 4v..4v+3 lie in group g = 4v/5 (digits d0..) and, when
+        // d0 >= 2, spill into group g+1; both groups' digit words are joined
+        // so one shift lines the four digits up.
+        float4 *y4 = reinterpret_cast<float4 *>(j.y);
+        for (uint64_t v = v0 + threadIdx.x; v < v1; v += kDThreads) {
+          const uint32_t e0 = (uint32_t)(4 * v);
+          const uint32_t g = e0 / 5u;
+          const uint32_t d0 = e0 - 5u * g;
+          const uint32_t li = g - o32;
+          const uint32_t c0 = grp_s[li];
+          const uint32_t c1 = d0 >= 2u ? (uint32_t)grp_s[li + 1] : 121u;
+          if (kMode == kWrite) {
+            float4 o;
+            if (c0 == 121u && c1 == 121u) {
+              o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            } else {
+              const uint32_t w =
+                  ((uint32_t)sm.lut[c0] | ((uint32_t)sm.lut[c1] << 10)) >> (2u * d0);
+              o.x = dequant(w & 3u, scale);
+              o.y = dequant((w >> 2) & 3u, scale);
+              o.z = dequant((w >> 4) & 3u, scale);
+              o.w = dequant((w >> 6) & 3u, scale);
+            }
+            y4[v] = o;
+          } else if (c0 != 121u || c1 != 121u) {
+            const uint32_t w = ((uint32_t)sm.lut[c0] | ((uint32_t)sm.lut[c1] << 10)) >> (2u * d0);
+            if ((w & 0xffu) != 0x55u) {  // some of the four digits is not zero
+              float4 o = y4[v];
+              if ((w & 3u) != 1u) o.x = __fadd_rn(o.x, dequant(w & 3u, scale));
+              if (((w >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, dequant((w >> 2) & 3u, scale));
+              if (((w >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, dequant((w >> 4) & 3u, scale));
+              if (((w >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, dequant((w >> 6) & 3u, scale));
+              y4[v] = o;
+            }
+          }
+        }
+        if (threadIdx.x < 4) {
+          const uint64_t e = e_begin + threadIdx.x;
+          if (e < 4 * v0) put(e);
+        } else if (threadIdx.x < 8) {
+          const uint64_t e = 4 * v1 + (threadIdx.x - 4);
+          if (e < e_end) put(e);
+        }
+      }
+    }
+  } else {
+    // accumulate, escape-heavy tile: visit only literal groups other than
+    // the all-zero 121; each group's (up to five) acc values are loaded
+    // before any is added
+    uint64_t g = O + off;
+#pragma unroll
+    for (int k = 0; k < kDBytes; ++k) {
+      const uint32_t b = (bw[k >> 2] >> (8 * (k & 3))) & 0xffu;
+      if (k < nvalid) {
+        if (b >= 243u) {
+          g += b - 241u;
+        } else {
+          if (b != 121u && g < j.groups) {
+            const uint16_t dg = digits_of(b);
+            float v[5];
+#pragma unroll
+            for (int d = 0; d < 5; ++d) {
+              const uint64_t e = 5 * g + d;
+              v[d] = (((dg >> (2 * d)) & 3u) != 1u && e < j.n) ? j.y[e] : 0.0f;
+            }
+#pragma unroll
+            for (int d = 0; d < 5; ++d) {
+              const uint32_t dig = (dg >> (2 * d)) & 3u;
+              const uint64_t e = 5 * g + d;
+              if (dig != 1u && e < j.n) j.y[e] = __fadd_rn(v[d], dequant(dig, scale));
+            }
+          }
+          ++g;
+        }
+      }
+    }
+  }
+  __syncthreads();
+}
+
 template <int kMode, bool kVec>
 __global__ void __launch_bounds__(kDThreads)
 k_decode(const DecodeArgs a) {
-  constexpr int kDBytes = DecodeShape<kMode>::kBytes;
   constexpr int kDTile = DecodeShape<kMode>::kTile;
   extern __shared__ __align__(16) uint8_t grp_s[];  // kMaxGroups + 16 bytes
-  __shared__ uint16_t lut_s[256];
-  __shared__ uint32_t scan_s[kDThreads / kWarp + 1];
-  __shared__ uint64_t o_s, m_s;
+  __shared__ DecodeSmem sm;
+  __shared__ uint64_t m_s;
   __shared__ uint32_t tile_s;
   __shared__ float scale_s;
-  __shared__ int bad_s;
-
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  __shared__ int ok_s;
 
   if (threadIdx.x == 0) {
-    const uint64_t L = a.len_dev ? *a.len_dev : a.cap;
-    int bad = (L < 4 || L > a.cap) ? 1 : 0;
-    uint32_t hb = 0;
-    if (!bad) {
-      if (L - 4 > a.groups || L == 4) bad = 1;
-      hb = (uint32_t)a.in[0] | ((uint32_t)a.in[1] << 8) | ((uint32_t)a.in[2] << 16) |
-           ((uint32_t)a.in[3] << 24);
-      if (hb >= 0x7f800000u) bad = 1;  // negative, infinite or NaN scale
-    }
-    bad_s = bad;
-    scale_s = __uint_as_float(hb);
-    m_s = bad ? 0 : L - 4;
+    uint64_t m = 0;
+    float scale = 0.0f;
+    ok_s = read_stream_header(a.in, a.len_dev, a.cap, a.groups, m, scale) ? 1 : 0;
+    m_s = m;
+    scale_s = scale;
   }
-  for (int v = threadIdx.x; v < 256; v += kDThreads) lut_s[v] = v < 243 ? digits_of(v) : 0;
+  for (int v = threadIdx.x; v < 256; v += kDThreads) sm.lut[v] = v < 243 ? digits_of(v) : 0;
   __syncthreads();
-  if (bad_s) {
+  if (!ok_s) {
     if (blockIdx.x == 0 && threadIdx.x == 0) report(a.dev_status, TLC_ERR_CORRUPT);
     return;
   }
-  const uint64_t m = m_s;
-  const uint32_t n_tiles = (uint32_t)((m + kDTile - 1) / kDTile);
-  const float scale = scale_s;
-  const uint8_t *payload = a.in + 4;
-
+  DecodeJob job;
+  job.payload = a.in + 4;
+  job.m = m_s;
+  job.n = a.n;
+  job.groups = a.groups;
+  job.scale = scale_s;
+  job.y = a.y;
+  job.status = a.status;
+  job.n_tiles = (uint32_t)((job.m + kDTile - 1) / kDTile);
+  job.vec = kVec;
   for (;;) {
     if (threadIdx.x == 0) tile_s = atomicAdd(a.ticket, 1u);
     __syncthreads();
     const uint32_t u = tile_s;
-    if (u >= n_tiles) break;
+    if (u >= job.n_tiles) break;
+    decode_tile<kMode>(job, u, sm, grp_s, a.dev_status, a.max_polls);
+  }
+}
 
-    // ---- load 8 payload bytes, expansion counts, block scan ------------
-    const uint64_t b0 = (uint64_t)u * kDTile + (uint64_t)threadIdx.x * kDBytes;
-    uint32_t bw[kDBytes / 4];
-#pragma unroll
-    for (int k = 0; k < kDBytes / 4; ++k) bw[k] = 0x79797979u;
-    int nvalid = 0;
-    if (b0 + kDBytes <= m && ((reinterpret_cast<uintptr_t>(payload + b0) & 3) == 0)) {
-      const uint32_t *p32 = reinterpret_cast<const uint32_t *>(payload + b0);
-#pragma unroll
-      for (int k = 0; k < kDBytes / 4; ++k) bw[k] = __ldg(p32 + k);
-      nvalid = kDBytes;
-    } else {
-#pragma unroll
-      for (int k = 0; k < kDBytes; ++k) {
-        if (b0 + k < m) {
-          const uint32_t b = __ldg(payload + b0 + k);
-          bw[k >> 2] = (bw[k >> 2] & ~(0xffu << (8 * (k & 3)))) | (b << (8 * (k & 3)));
-          nvalid = k + 1;
-        }
-      }
-    }
-    uint32_t esum = 0;
-#pragma unroll
-    for (int k = 0; k < kDBytes; ++k) {
-      const uint32_t b = (bw[k >> 2] >> (8 * (k & 3))) & 0xffu;
-      if (k < nvalid) esum += b >= 243u ? b - 241u : 1u;
-    }
-    uint32_t E;
-    const uint32_t off = block_exclusive_sum<kDThreads>(esum, scan_s, E);
-    // Dense output always expands the tile's groups in shared memory.  The
-    // accumulate mode does so too when the tile is mostly literals (then a
-    // coalesced float4 pass over acc is cheapest); for escape-heavy tiles it
-    // visits only the literal groups.
-    const bool expand = kMode == kWrite || E <= 4u * (uint32_t)kDTile;
+struct BatchDecodeArgs {
+  const BatchTensor *tensors;
+  const uint32_t *tile_tensor;  // tensor of each global (upper-bound) tile
+  const uint8_t *arena;
+  const uint64_t *in_lens;      // per-tensor stream lengths
+  uint64_t *status;
+  uint32_t *ticket;
+  uint32_t n_tiles;             // upper bound over all tensors
+  int32_t *dev_status;
+  uint32_t max_polls;
+};
 
-    // ---- look-back (warp 0); the other warps pre-fill zero groups ----------
-    if (warp == 0) {
-      bool timed_out = false;
-      const uint64_t O = lookback_sum(a.status, u, E, a.max_polls, timed_out);
-      if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(a.dev_status, TLC_ERR_TIMEOUT);
-      if (lane == 0) o_s = O;
-    } else if (expand) {
-      const uint32_t words = (E + 15) / 16;
-      for (uint32_t w = threadIdx.x - kWarp; w < words; w += kDThreads - kWarp)
-        reinterpret_cast<uint4 *>(grp_s)[w] = make_uint4(0x79797979u, 0x79797979u, 0x79797979u,
-                                                          0x79797979u);
-    }
-    __syncthreads();
-    const uint64_t O = o_s;
+// Decode the streams of a list of tensors from their arena slots: tiles of
+// all tensors in one ticket order, each look-back confined to its stream;
+// tiles past a stream's actual length do nothing.
+template <int kMode>
+__global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArgs a) {
+  constexpr int kDTile = DecodeShape<kMode>::kTile;
+  extern __shared__ __align__(16) uint8_t grp_s[];
+  __shared__ DecodeSmem sm;
+  __shared__ uint64_t m_s;
+  __shared__ uint32_t tile_s;
+  __shared__ float scale_s;
+  __shared__ int ok_s;
+  for (int v = threadIdx.x; v < 256; v += kDThreads) sm.lut[v] = v < 243 ? digits_of(v) : 0;
+  for (;;) {
     if (threadIdx.x == 0) {
-      const bool last = (u == n_tiles - 1);
-      if (O + E > a.groups || (last && O + E != a.groups)) report(a.dev_status, TLC_ERR_CORRUPT);
-    }
-    const uint64_t Ec = O >= a.groups ? 0 : umin64(E, a.groups - O);
-
-    if (expand) {
-      // literal bytes into the expanded group buffer
-      uint32_t pos = off;
-#pragma unroll
-      for (int k = 0; k < kDBytes; ++k) {
-        const uint32_t b = (bw[k >> 2] >> (8 * (k & 3))) & 0xffu;
-        if (k < nvalid) {
-          if (b >= 243u) {
-            pos += b - 241u;
-          } else {
-            grp_s[pos] = (uint8_t)b;
-            ++pos;
-          }
-        }
-      }
-      __syncthreads();
-      // groups [O, O+Ec) -> values [5 O, min(5 (O+Ec), n))
-      const uint64_t e_begin = 5 * O;
-      const uint64_t e_end = umin64(5 * (O + Ec), a.n);
-      if (e_end > e_begin) {
-        const uint32_t o32 = (uint32_t)O;
-        auto value_at = [&](uint64_t e) -> float {
-          const uint32_t e32 = (uint32_t)e;
-          const uint32_t g = e32 / 5u;
-          const uint32_t d = e32 - 5u * g;
-          const uint32_t dig = (lut_s[grp_s[g - o32]] >> (2 * d)) & 3u;
-          return dequant(dig, scale);
-        };
-        // one value: written (dense output) or added where non-zero (accumulate)
-        auto put = [&](uint64_t e) {
-          if (kMode == kWrite) {
-            a.y[e] = value_at(e);
-          } else {
-            const uint32_t e32 = (uint32_t)e;
-            const uint32_t g = e32 / 5u;
-            const uint32_t dig = (lut_s[grp_s[g - o32]] >> (2 * (e32 - 5u * g))) & 3u;
-            if (dig != 1u) a.y[e] = __fadd_rn(a.y[e], dequant(dig, scale));
-          }
-        };
-        uint64_t v0 = (e_begin + 3) / 4, v1 = e_end / 4;
-        if (!kVec || v1 <= v0) {
-          v0 = v1 = 0;
-          for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) put(e);
-        } else {
-          // Values 4v..4v+3 lie in group g = 4v/5 (digits d0..) and, when
-          // d0 >= 2, spill into group g+1; both groups' digit words are
-          // joined so one shift lines the four digits up.
-          float4 *y4 = reinterpret_cast<float4 *>(a.y);
-          for (uint64_t v = v0 + threadIdx.x; v < v1; v += kDThreads) {
-            const uint32_t e0 = (uint32_t)(4 * v);
-            const uint32_t g = e0 / 5u;
-            const uint32_t d0 = e0 - 5u * g;
-            const uint32_t li = g - o32;
-            const uint32_t b0 = grp_s[li];
-            const uint32_t b1 = d0 >= 2u ? (uint32_t)grp_s[li + 1] : 121u;
-            if (kMode == kWrite) {
-              float4 o;
-              if (b0 == 121u && b1 == 121u) {
-                o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-              } else {
-                const uint32_t w =
-                    ((uint32_t)lut_s[b0] | ((uint32_t)lut_s[b1] << 10)) >> (2u * d0);
-                o.x = dequant(w & 3u, scale);
-                o.y = dequant((w >> 2) & 3u, scale);
-                o.z = dequant((w >> 4) & 3u, scale);
-                o.w = dequant((w >> 6) & 3u, scale);
-              }
-              y4[v] = o;
-            } else if (b0 != 121u || b1 != 121u) {
-              const uint32_t w = ((uint32_t)lut_s[b0] | ((uint32_t)lut_s[b1] << 10)) >> (2u * d0);
-              if ((w & 0xffu) != 0x55u) {  // some of the four digits is not zero
-                float4 o = y4[v];
-                if ((w & 3u) != 1u) o.x = __fadd_rn(o.x, dequant(w & 3u, scale));
-                if (((w >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, dequant((w >> 2) & 3u, scale));
-                if (((w >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, dequant((w >> 4) & 3u, scale));
-                if (((w >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, dequant((w >> 6) & 3u, scale));
-                y4[v] = o;
-              }
-            }
-          }
-          if (threadIdx.x < 4) {
-            const uint64_t e = e_begin + threadIdx.x;
-            if (e < 4 * v0) put(e);
-          } else if (threadIdx.x < 8) {
-            const uint64_t e = 4 * v1 + (threadIdx.x - 4);
-            if (e < e_end) put(e);
-          }
-        }
-      }
-    } else {
-      // accumulate, escape-heavy tile: visit only literal groups other than
-      // the all-zero 121; each group's (up to five) acc values are loaded
-      // before any is added
-      uint64_t g = O + off;
-#pragma unroll
-      for (int k = 0; k < kDBytes; ++k) {
-        const uint32_t b = (bw[k >> 2] >> (8 * (k & 3))) & 0xffu;
-        if (k < nvalid) {
-          if (b >= 243u) {
-            g += b - 241u;
-          } else {
-            if (b != 121u && g < a.groups) {
-              const uint16_t dg = digits_of(b);
-              float v[5];
-#pragma unroll
-              for (int d = 0; d < 5; ++d) {
-                const uint64_t e = 5 * g + d;
-                v[d] = (((dg >> (2 * d)) & 3u) != 1u && e < a.n) ? a.y[e] : 0.0f;
-              }
-#pragma unroll
-              for (int d = 0; d < 5; ++d) {
-                const uint32_t dig = (dg >> (2 * d)) & 3u;
-                const uint64_t e = 5 * g + d;
-                if (dig != 1u && e < a.n) a.y[e] = __fadd_rn(v[d], dequant(dig, scale));
-              }
-            }
-            ++g;
-          }
-        }
+      const uint32_t u = atomicAdd(a.ticket, 1u);
+      tile_s = u;
+      if (u < a.n_tiles) {
+        const BatchTensor &T = a.tensors[a.tile_tensor[u]];
+        uint64_t m = 0;
+        float scale = 0.0f;
+        ok_s = read_stream_header(a.arena + T.arena_off, a.in_lens + a.tile_tensor[u], T.cap,
+                                  T.groups, m, scale) ? 1 : 0;
+        m_s = m;
+        scale_s = scale;
       }
     }
     __syncthreads();
+    const uint32_t u = tile_s;
+    if (u >= a.n_tiles) break;
+    const uint32_t id = a.tile_tensor[u];
+    const BatchTensor &T = a.tensors[id];
+    const uint32_t t = u - T.d_tile_begin;
+    if (!ok_s) {
+      if (t == 0 && threadIdx.x == 0) report(a.dev_status, TLC_ERR_CORRUPT);
+      __syncthreads();
+      continue;
+    }
+    DecodeJob job;
+    job.payload = a.arena + T.arena_off + 4;
+    job.m = m_s;
+    job.n = T.n;
+    job.groups = T.groups;
+    job.scale = scale_s;
+    job.y = T.y;
+    job.status = a.status + T.d_tile_begin;
+    job.n_tiles = (uint32_t)((job.m + kDTile - 1) / kDTile);
+    job.vec = T.vec_y != 0;
+    if (t >= job.n_tiles) {  // this stream is shorter than its slot
+      __syncthreads();
+      continue;
+    }
+    decode_tile<kMode>(job, t, sm, grp_s, a.dev_status, a.max_polls);
   }
 }
 
@@ -404,6 +506,59 @@ cudaError_t launch_decode(const DeviceInfo &dev, const uint8_t *in, const uint64
                : launch_one<kAccumulate, false>(dev, a, tiles, stream);
   return vec ? launch_one<kWrite, true>(dev, a, tiles, stream)
              : launch_one<kWrite, false>(dev, a, tiles, stream);
+}
+
+uint32_t decode_tile_payload_bytes(bool accumulate) {
+  return accumulate ? DecodeShape<kAccumulate>::kTile : DecodeShape<kWrite>::kTile;
+}
+
+template <int kMode>
+static cudaError_t launch_batch_one(const DeviceInfo &dev, const BatchDecodeArgs &a,
+                                    cudaStream_t stream) {
+  const size_t smem = decode_smem_bytes(kMode == kAccumulate);
+  const int occ = kMode == kWrite ? dev.occ_decode_batch_write : dev.occ_decode_batch_acc;
+  uint32_t grid = (uint32_t)dev.sm_count * (uint32_t)(occ > 0 ? occ : 1);
+  if (grid > a.n_tiles) grid = a.n_tiles;
+  const int kind = kMode == kWrite ? kKindDecodeWrite : kKindDecodeAccumulate;
+  timing_begin(kind, stream);
+  k_decode_batch<kMode><<<grid, kDThreads, smem, stream>>>(a);
+  timing_end(kind, stream);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
+                                const uint8_t *arena, const uint64_t *in_lens, bool accumulate,
+                                int32_t *dev_status, uint32_t max_polls, cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(p.d_zero_base, 0, p.d_zero_bytes, stream);
+  if (e != cudaSuccess) return e;
+  BatchDecodeArgs a;
+  a.tensors = p.tensors;
+  a.tile_tensor = p.d_tile_tensor;
+  a.arena = arena;
+  a.in_lens = in_lens;
+  a.status = p.d_status;
+  a.ticket = p.d_ticket;
+  a.n_tiles = p.n_d_tiles;
+  a.dev_status = dev_status;
+  a.max_polls = max_polls;
+  return accumulate ? launch_batch_one<kAccumulate>(dev, a, stream)
+                    : launch_batch_one<kWrite>(dev, a, stream);
+}
+
+int occupancy_decode_batch(bool accumulate) {
+  int occ = 0;
+  const size_t smem = decode_smem_bytes(accumulate);
+  if (accumulate) {
+    cudaFuncSetAttribute(k_decode_batch<kAccumulate>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_batch<kAccumulate>, kDThreads,
+                                                  smem);
+  } else {
+    cudaFuncSetAttribute(k_decode_batch<kWrite>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_batch<kWrite>, kDThreads, smem);
+  }
+  return occ;
 }
 
 cudaError_t launch_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_status,

@@ -16,6 +16,9 @@ struct DeviceInfo {
   int occ_quant_scalar = 0;
   int occ_decode_write = 0;
   int occ_decode_acc = 0;
+  int occ_quant_batch = 0;
+  int occ_decode_batch_write = 0;
+  int occ_decode_batch_acc = 0;
   cudaMemPool_t pool = nullptr;
 };
 
@@ -43,6 +46,61 @@ inline CompressScratch compress_scratch_layout(void *base, uint32_t n_part, uint
   s.spare_status = reinterpret_cast<int32_t *>(s.partial + n_part);
   return s;
 }
+
+// ---- tensor lists (plans) ---------------------------------------------------
+// Values per block of the batched magnitude pass (a multiple of 4 * 512).
+constexpr uint32_t kBatchChunk = 8192;
+
+// One tensor of a plan, as the batched kernels see it (device memory).
+struct BatchTensor {
+  const float *x;
+  float *err;
+  float *y;              // decompress target (or accumulation buffer)
+  uint64_t n, groups;
+  uint64_t arena_off;    // the tensor's stream slot in the arena
+  uint64_t cap;          // slot size = 4 + ceil(n/5)
+  uint32_t q_tile_begin, q_tiles;  // compress tiles (global numbering)
+  uint32_t d_tile_begin, d_tiles;  // decode tiles (global numbering, upper bound)
+  uint32_t vec_q;        // x and err 16-byte aligned
+  uint32_t vec_y;        // y 16-byte aligned
+};
+
+struct BatchChunk {
+  uint32_t tensor;
+  uint32_t pad;
+  uint64_t start;        // first value of the chunk
+};
+
+// Device-side view of a plan: descriptor tables and scratch.
+struct BatchPlanDev {
+  const BatchTensor *tensors;
+  uint32_t count;
+  const BatchChunk *chunks;
+  uint32_t n_chunks;
+  const uint32_t *q_tile_tensor;
+  uint32_t n_q_tiles;
+  const uint32_t *d_tile_tensor;
+  uint32_t n_d_tiles;
+  uint32_t *mbits;        // per-tensor max bits
+  uint32_t *q_ticket;
+  uint64_t *q_status;
+  void *q_zero_base;      // mbits, q_ticket and q_status, contiguous
+  size_t q_zero_bytes;
+  uint32_t *d_ticket;
+  uint64_t *d_status;
+  void *d_zero_base;      // d_ticket and d_status, contiguous
+  size_t d_zero_bytes;
+};
+
+cudaError_t launch_compress_batch(const DeviceInfo &dev, const BatchPlanDev &p, float s,
+                                  uint8_t *arena, uint64_t *out_lens, int32_t *dev_status,
+                                  uint32_t max_polls, cudaStream_t stream);
+cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
+                                const uint8_t *arena, const uint64_t *in_lens, bool accumulate,
+                                int32_t *dev_status, uint32_t max_polls, cudaStream_t stream);
+int occupancy_quant_batch();
+int occupancy_decode_batch(bool accumulate);
+uint32_t decode_tile_payload_bytes(bool accumulate);
 
 // Per-device facts for device d (initialised on first use); nullptr on error.
 const DeviceInfo *device_info(int d);

@@ -54,6 +54,18 @@ def lib() -> ctypes.CDLL:
     L.tlc_test_wait_timeout.restype = ctypes.c_int
     L.tlc_compress_noalloc.argtypes = [P, S, ctypes.c_float, P, P, S, P, P, P]
     L.tlc_compress_noalloc.restype = ctypes.c_int
+    L.tlc_plan_create.argtypes = [ctypes.c_int, P, P, P, P, P]
+    L.tlc_plan_create.restype = ctypes.c_int
+    L.tlc_plan_destroy.argtypes = [P]
+    L.tlc_plan_destroy.restype = None
+    L.tlc_plan_arena_bytes.argtypes = [P]
+    L.tlc_plan_arena_bytes.restype = S
+    L.tlc_plan_stream_offset.argtypes = [P, ctypes.c_int]
+    L.tlc_plan_stream_offset.restype = S
+    L.tlc_compress_batch.argtypes = [P, ctypes.c_float, P, P, P, P]
+    L.tlc_compress_batch.restype = ctypes.c_int
+    L.tlc_decompress_batch.argtypes = [P, P, P, ctypes.c_int, P, P]
+    L.tlc_decompress_batch.restype = ctypes.c_int
     L.tlc_kernel_timing.argtypes = [ctypes.c_int]
     L.tlc_kernel_timing.restype = None
     L.tlc_kernel_timing_read.argtypes = [P, P, ctypes.c_int]
@@ -176,6 +188,98 @@ def tlc_decompress_accumulate(streams, n: int, acc, in_lens=None, in_caps=None,
         ptrs, _dev_ptr(in_lens, "in_lens"), caps, k, n, _dev_ptr(acc, "acc", torch.float32),
         _dev_ptr(dev_status, "dev_status", torch.int32), _stream(stream))
     return _check("tlc_decompress_accumulate", code)
+
+
+# ------------------------------------------------------------ tensor lists --
+
+def _ptr_array(ts, name, dtype):
+    if ts is None:
+        return None
+    return (ctypes.c_void_p * len(ts))(*[_dev_ptr(t, name, dtype) for t in ts])
+
+
+def tlc_plan_create(ns, xs=None, errs=None, ys=None) -> int:
+    """Create a plan for a fixed list of tensors; returns the handle.
+
+    ns: sizes; xs/errs: fp32 CUDA tensors (inputs and error buffers of
+    tlc_compress_batch); ys: fp32 CUDA tensors (outputs of
+    tlc_decompress_batch).  The caller keeps the tensors alive."""
+    import torch
+    ns = [int(n) for n in ns]
+    h = ctypes.c_void_p()
+    code = lib().tlc_plan_create(
+        len(ns), (ctypes.c_size_t * len(ns))(*ns), _ptr_array(xs, "x", torch.float32),
+        _ptr_array(errs, "err", torch.float32), _ptr_array(ys, "y", torch.float32),
+        ctypes.byref(h))
+    _check("tlc_plan_create", code)
+    return h.value
+
+
+def tlc_plan_destroy(plan: int) -> None:
+    lib().tlc_plan_destroy(plan)
+
+
+def tlc_plan_arena_bytes(plan: int) -> int:
+    return int(lib().tlc_plan_arena_bytes(plan))
+
+
+def tlc_plan_stream_offset(plan: int, i: int) -> int:
+    return int(lib().tlc_plan_stream_offset(plan, i))
+
+
+def tlc_compress_batch(plan: int, s: float, arena, out_lens, dev_status=None,
+                       stream=None) -> int:
+    """Compress every tensor of the plan into its arena slot; out_lens is a
+    uint64/int64 CUDA tensor with one entry per tensor."""
+    import torch
+    code = lib().tlc_compress_batch(plan, float(s), _dev_ptr(arena, "arena", torch.uint8),
+                                    _dev_ptr(out_lens, "out_lens"),
+                                    _dev_ptr(dev_status, "dev_status", torch.int32),
+                                    _stream(stream))
+    return _check("tlc_compress_batch", code)
+
+
+def tlc_decompress_batch(plan: int, arena, in_lens, accumulate: bool = False,
+                         dev_status=None, stream=None) -> int:
+    """Decompress every arena slot into the plan's ys (overwrite, or add
+    where q != 0 when accumulate is true)."""
+    import torch
+    code = lib().tlc_decompress_batch(plan, _dev_ptr(arena, "arena", torch.uint8),
+                                      _dev_ptr(in_lens, "in_lens"), 1 if accumulate else 0,
+                                      _dev_ptr(dev_status, "dev_status", torch.int32),
+                                      _stream(stream))
+    return _check("tlc_decompress_batch", code)
+
+
+class Plan:
+    """A plan with its tensors kept alive; see tlc_plan_create."""
+
+    def __init__(self, xs=None, errs=None, ys=None):
+        lists = [v for v in (xs, ys) if v is not None]
+        if not lists:
+            raise ValueError("a plan needs inputs (xs, errs) or outputs (ys)")
+        self.ns = [t.numel() for t in lists[0]]
+        self._tensors = (xs, errs, ys)
+        self.handle = tlc_plan_create(self.ns, xs, errs, ys)
+        self.arena_bytes = tlc_plan_arena_bytes(self.handle)
+        self.offsets = [tlc_plan_stream_offset(self.handle, i) for i in range(len(self.ns))]
+
+    def compress(self, s, arena, out_lens, dev_status=None, stream=None):
+        return tlc_compress_batch(self.handle, s, arena, out_lens, dev_status, stream)
+
+    def decompress(self, arena, in_lens, accumulate=False, dev_status=None, stream=None):
+        return tlc_decompress_batch(self.handle, arena, in_lens, accumulate, dev_status, stream)
+
+    def close(self):
+        if self.handle:
+            tlc_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def tlc_set_wait_limit(max_polls: int) -> None:

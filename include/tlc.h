@@ -139,6 +139,56 @@ tlc_status tlc_decompress_accumulate(const uint8_t *const *ins,
                                      float *acc, int32_t *dev_status,
                                      tlc_stream_t stream);
 
+/* ---- Tensor lists ------------------------------------------------------
+ * A training step compresses many tensors (one per layer).  A plan binds a
+ * fixed list of tensors once; each step then compresses (or decompresses)
+ * the whole list with one launch set, each tensor with its own M, scale and
+ * error buffer, exactly as tlc_compress / tlc_decompress would one by one.
+ * The streams live in one caller-owned arena: tensor i's stream starts at
+ * tlc_plan_stream_offset(plan, i) and has room for 4 + ceil(n_i/5) bytes.
+ *
+ * A plan holds device memory for its descriptor tables and scratch (allocated
+ * once, at creation) and belongs to the device current at creation; calls
+ * must be made with that device current.  Calls with the same plan share its
+ * scratch, so their work must not overlap on the GPU (keep them on one
+ * stream or order the streams).  Different plans are independent. */
+typedef struct tlc_plan_s *tlc_plan;
+
+/* Create a plan for count tensors of ns[i] values.  xs/errs (arrays of
+ * count device pointers; both or neither) are the inputs and error buffers
+ * of tlc_compress_batch; ys (count device pointers, or NULL) are the outputs
+ * of tlc_decompress_batch.  Synchronous (copies the tables to the device).
+ * TLC_ERR_INVALID_ARG for count < 1, a bad n, a NULL entry, or x/err
+ * overlap; TLC_ERR_CUDA if the device allocation fails. */
+tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
+                           float *const *errs, float *const *ys, tlc_plan *plan);
+
+/* Free a plan (synchronous; no call using it may still be running). */
+void tlc_plan_destroy(tlc_plan plan);
+
+/* Arena size for one set of streams, and tensor i's stream offset in it
+ * (16-byte aligned); (size_t)-1 for a bad i. */
+size_t tlc_plan_arena_bytes(tlc_plan plan);
+size_t tlc_plan_stream_offset(tlc_plan plan, int i);
+
+/* Compress every tensor of the plan ("Proposed method" bullets 1-3), each
+ * as tlc_compress would: err_i is updated in place, stream i is written at
+ * its arena offset and its length to out_lens[i] (device uint64[count]).  A
+ * non-finite tensor gets out_lens[i] = 0 and its err_i unchanged;
+ * TLC_ERR_NONFINITE goes to *dev_status while the other tensors are still
+ * compressed.  Launches: one memset, a magnitude pass, one quantize+encode
+ * pass over all tensors. */
+tlc_status tlc_compress_batch(tlc_plan plan, float s, uint8_t *arena, uint64_t *out_lens,
+                              int32_t *dev_status, tlc_stream_t stream);
+
+/* Decompress every tensor's stream from the arena (lengths in in_lens,
+ * device uint64[count]) into the plan's ys: overwrite (accumulate = 0, as
+ * tlc_decompress) or add where q != 0 (accumulate = 1, as one stream of
+ * tlc_decompress_accumulate).  A corrupt stream sets TLC_ERR_CORRUPT and
+ * leaves its y unspecified; the others are still decoded. */
+tlc_status tlc_decompress_batch(tlc_plan plan, const uint8_t *arena, const uint64_t *in_lens,
+                                int accumulate, int32_t *dev_status, tlc_stream_t stream);
+
 /* Largest n accepted by tlc_compress_noalloc. */
 #define TLC_NOALLOC_MAX_N ((size_t)1 << 29)
 

@@ -110,3 +110,23 @@ def test_binding_refuses_cpu_tensors(L):
     x = torch.zeros(10)
     with pytest.raises(ValueError):
         g.compress(x, 1.0, torch.zeros(10))
+
+
+def test_plan_create_rejects_bad_arguments_on_the_host(L):
+    h = ctypes.c_void_p()
+    ns = (ctypes.c_size_t * 2)(10, 20)
+    ptrs = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    errs = (ctypes.c_void_p * 2)(0x30000, 0x40000)
+    INV = 1
+    assert L.tlc_plan_create(0, ns, ptrs, errs, None, ctypes.byref(h)) == INV
+    assert L.tlc_plan_create(2, None, ptrs, errs, None, ctypes.byref(h)) == INV
+    assert L.tlc_plan_create(2, ns, ptrs, None, None, ctypes.byref(h)) == INV   # x without err
+    assert L.tlc_plan_create(2, ns, None, None, None, ctypes.byref(h)) == INV   # nothing bound
+    bad_n = (ctypes.c_size_t * 2)(10, 0)
+    assert L.tlc_plan_create(2, bad_n, ptrs, errs, None, ctypes.byref(h)) == INV
+    overl = (ctypes.c_void_p * 2)(0x10000, 0x20010)
+    assert L.tlc_plan_create(2, ns, ptrs, overl, None, ctypes.byref(h)) == INV  # x/err overlap
+    assert L.tlc_plan_create(2, ns, ptrs, errs, None, None) == INV
+    assert L.tlc_compress_batch(None, 1.0, None, None, None, None) == INV
+    assert L.tlc_decompress_batch(None, None, None, 0, None, None) == INV
+    assert L.tlc_plan_arena_bytes(None) == 0

@@ -1,0 +1,162 @@
+"""Tensor lists (plans) on the GPU against the CPU oracle, tensor by tensor.
+
+tlc_compress_batch must give, for every tensor, exactly the stream and error
+buffer that one tlc_compress call (and the oracle) gives; tlc_decompress_batch
+exactly what tlc_decompress / one stream of tlc_decompress_accumulate gives.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def g():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import gradient_traffic_compression_b200 as g
+    g.lib()
+    return g
+
+
+def bits(a):
+    return np.ascontiguousarray(a, np.float32).view(np.uint32)
+
+
+def dev_f32(a, offset=0):
+    buf = torch.empty(a.size + offset, dtype=torch.float32, device="cuda")
+    t = buf[offset:]
+    t.copy_(torch.from_numpy(np.ascontiguousarray(a, np.float32)))
+    return t
+
+
+class Batch:
+    """Device tensors, a plan over them, an arena and length/status words."""
+
+    def __init__(self, g, xs_h, errs_h, offsets=None, with_y=True):
+        offsets = offsets or [0] * len(xs_h)
+        self.xs = [dev_f32(x, o) for x, o in zip(xs_h, offsets)]
+        self.errs = [dev_f32(e, o) for e, o in zip(errs_h, offsets)]
+        self.ys = ([dev_f32(np.zeros(x.size, np.float32), o) for x, o in zip(xs_h, offsets)]
+                   if with_y else None)
+        self.plan = g.Plan(self.xs, self.errs, self.ys)
+        self.arena = torch.full((self.plan.arena_bytes,), 0xA5, dtype=torch.uint8, device="cuda")
+        self.lens = torch.zeros(len(xs_h), dtype=torch.int64, device="cuda")
+        self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
+
+    def stream(self, i):
+        L = int(self.lens[i].item())
+        o = self.plan.offsets[i]
+        return self.arena[o:o + L].cpu().numpy()
+
+
+def mixed(seed, n, zero_frac=0.6, sigma=1e-3):
+    x = synth.normal(synth.key_for(seed, 0), n, sigma)
+    x[synth.bernoulli(synth.key_for(seed, 3), n, zero_frac)] = 0.0
+    e = synth.laplace(synth.key_for(seed, 1), n, 3e-4)
+    return x, e
+
+
+SIZES = [1, 7, 432, 2304, 4099, 20479, 20480, 20481, 36864, 100_003, 262_144, 1_000_001]
+
+
+@pytest.mark.parametrize("unaligned", [False, True])
+def test_batch_matches_oracle_over_three_steps(g, unaligned):
+    xs0, errs = zip(*[mixed(50 + i, n) for i, n in enumerate(SIZES)])
+    errs = [e.copy() for e in errs]
+    offsets = [(i % 3) if unaligned else 0 for i in range(len(SIZES))]
+    b = Batch(g, list(xs0), errs, offsets)
+    s = 1.75
+    for step in range(3):
+        xs = [mixed(1000 * step + i, n)[0] for i, n in enumerate(SIZES)]
+        for t, x in zip(b.xs, xs):
+            t.copy_(torch.from_numpy(x))
+        b.plan.compress(s, b.arena, b.lens, b.status)
+        b.plan.decompress(b.arena, b.lens, accumulate=False, dev_status=b.status)
+        torch.cuda.synchronize()
+        assert int(b.status.item()) == 0
+        for i, x in enumerate(xs):
+            rc, st, e2 = oracle.compress(x, s, errs[i])
+            assert rc == 0
+            assert b.stream(i).tolist() == st.tolist(), f"tensor {i} (n={x.size}) step {step}"
+            assert np.array_equal(bits(b.errs[i].cpu().numpy()), bits(e2)), f"err {i}"
+            _, y = oracle.decompress(st, x.size)
+            assert np.array_equal(bits(b.ys[i].cpu().numpy()), bits(y)), f"y {i}"
+            errs[i] = e2
+
+
+def test_batch_accumulate_mode(g):
+    sizes = [5, 1234, 20480 * 2 + 9, 300_001]
+    xs, errs = zip(*[mixed(70 + i, n, zero_frac=0.1, sigma=1.0) for i, n in enumerate(sizes)])
+    b = Batch(g, list(xs), list(errs))
+    accs0 = [synth.normal(synth.key_for(80 + i, 2), n, 1.0) for i, n in enumerate(sizes)]
+    for t, a in zip(b.ys, accs0):
+        t.copy_(torch.from_numpy(a))
+    b.plan.compress(1.0, b.arena, b.lens, b.status)
+    b.plan.decompress(b.arena, b.lens, accumulate=True, dev_status=b.status)
+    b.plan.decompress(b.arena, b.lens, accumulate=True, dev_status=b.status)   # a second worker
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    for i, x in enumerate(xs):
+        _, st, _ = oracle.compress(x, 1.0, errs[i])
+        _, want = oracle.decompress_accumulate([st, st], x.size, accs0[i])
+        assert np.array_equal(bits(b.ys[i].cpu().numpy()), bits(want))
+
+
+def test_batch_config2_twenty_steps(g):
+    shapes = synth.resnet110_conv_shapes()
+    ns = [int(np.prod(s_)) for s_ in shapes]
+    errs = [np.zeros(n, np.float32) for n in ns]
+    b = Batch(g, [np.zeros(n, np.float32) for n in ns], errs, with_y=False)
+    for step in range(20):
+        xs = synth.tensor_set(2, step)
+        for t, x in zip(b.xs, xs):
+            t.copy_(torch.from_numpy(x))
+        b.plan.compress(1.75, b.arena, b.lens, b.status)
+        torch.cuda.synchronize()
+        assert int(b.status.item()) == 0
+        for i, x in enumerate(xs):
+            rc, st, errs[i] = oracle.compress(x, 1.75, errs[i])
+            assert b.stream(i).tolist() == st.tolist(), f"step {step} tensor {i}"
+        if step % 5 == 4:
+            for i in range(len(ns)):
+                assert np.array_equal(bits(b.errs[i].cpu().numpy()), bits(errs[i]))
+
+
+def test_batch_isolates_a_nonfinite_tensor(g):
+    sizes = [1000, 30000, 5000]
+    xs, errs = [list(v) for v in zip(*[mixed(90 + i, n) for i, n in enumerate(sizes)])]
+    xs[1] = xs[1].copy()
+    xs[1][12345] = np.nan
+    b = Batch(g, xs, errs)
+    b.plan.compress(1.5, b.arena, b.lens, b.status)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 2
+    assert int(b.lens[1].item()) == 0
+    assert np.array_equal(bits(b.errs[1].cpu().numpy()), bits(errs[1]))      # untouched
+    for i in (0, 2):
+        _, st, e2 = oracle.compress(xs[i], 1.5, errs[i])
+        assert b.stream(i).tolist() == st.tolist()
+        assert np.array_equal(bits(b.errs[i].cpu().numpy()), bits(e2))
+
+
+def test_batch_isolates_a_corrupt_stream(g):
+    sizes = [3000, 3000]
+    xs, errs = zip(*[mixed(95 + i, n) for i, n in enumerate(sizes)])
+    b = Batch(g, list(xs), list(errs))
+    b.plan.compress(1.5, b.arena, b.lens, b.status)
+    torch.cuda.synchronize()
+    lens = b.lens.clone()
+    lens[0] -= 1                                   # stream 0 now one byte short
+    b.plan.decompress(b.arena, lens, dev_status=b.status)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 3
+    _, st, _ = oracle.compress(xs[1], 1.5, errs[1])
+    _, y = oracle.decompress(st, sizes[1])
+    assert np.array_equal(bits(b.ys[1].cpu().numpy()), bits(y))
