@@ -35,6 +35,7 @@ void init_device(int d) {
     di.occ_decode_write = tlc::occupancy_decode(false);
     di.occ_decode_acc = tlc::occupancy_decode(true);
     di.occ_quant_batch = tlc::occupancy_quant_batch();
+    tlc::occupancy_split(di.occ_pack_vec, di.occ_pack_scalar, di.occ_encode);
     di.occ_decode_batch_write = tlc::occupancy_decode_batch(false);
     di.occ_decode_batch_acc = tlc::occupancy_decode_batch(true);
     cudaMemPoolProps props;
@@ -110,7 +111,7 @@ struct Timing {
 Timing g_timing;
 
 const char *const kKindNames[tlc::kKindCount] = {"k_absmax", "k_quant_zre", "k_decode_write",
-                                                 "k_decode_accumulate"};
+                                                 "k_decode_accumulate", "k_zre_encode"};
 
 }  // namespace
 
@@ -212,16 +213,14 @@ tlc_status tlc_compress(const float *x, size_t n, float s, float *err, uint8_t *
   const tlc::DeviceInfo *dev = current_device(ce);
   if (!dev) return TLC_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const uint32_t n_tiles = tlc::compress_tiles(n);
-  const uint32_t n_part = tlc::compress_partials(*dev, n);
   void *scratch = nullptr;
-  if (scratch_alloc(*dev, tlc::compress_scratch_bytes(n_part, n_tiles), &scratch, st) !=
-      cudaSuccess)
-    return TLC_ERR_CUDA;
+  const size_t bytes = tlc::compress_scratch_bytes_for(*dev, n, true);
+  if (scratch_alloc(*dev, bytes + 256, &scratch, st) != cudaSuccess) return TLC_ERR_CUDA;
+  // a status word for calls without one, past everything the kernels use
   int32_t *status_ptr =
-      dev_status ? dev_status : tlc::compress_scratch_layout(scratch, n_part, n_tiles).spare_status;
+      dev_status ? dev_status : reinterpret_cast<int32_t *>(static_cast<char *>(scratch) + bytes);
   ce = tlc::launch_compress(*dev, x, n, s, err, out, out_cap, out_len, status_ptr, wait_limit(),
-                            scratch, st);
+                            scratch, st, true);
   const cudaError_t fe = cudaFreeAsync(scratch, st);
   return (ce == cudaSuccess && fe == cudaSuccess) ? TLC_OK : TLC_ERR_CUDA;
 }

@@ -441,3 +441,46 @@ def test_bounded_wait_reports_timeout(g):
     # the context is still usable afterwards
     x, err, s = mixed_case(1, 1000)
     assert_compress_parity(g, x, s, err)
+
+
+# ---- large tensors: streaming quantize + separate zero-run encode ---------
+
+SPLIT_MIN = 1 << 22            # sizes from here on take the split path
+ENC_TILE_VALUES = 5 * 16384    # values per encode tile (16384 groups)
+
+
+@pytest.mark.parametrize("n,offset", [(SPLIT_MIN, 0), (SPLIT_MIN + 1, 0),
+                                      (SPLIT_MIN + 12345, 0), (SPLIT_MIN + 7, 1),
+                                      (SPLIT_MIN + 640 * 3 + 9, 3)])
+def test_split_path_sizes(g, n, offset):
+    x, err, s = mixed_case(3000 + n % 997, n, zero_frac=0.7)
+    st, _ = assert_compress_parity(g, x, s, err, offset=offset)
+    assert_roundtrip_parity(g, st, n, offset=offset)
+
+
+SPLIT_RUNS = {
+    "enc_edge_mod0": [16384 - 15, 16384 + 13],
+    "enc_edge_mod1": [16384 - 16, 16384 + 14],
+    "enc_edge_mod13": [2 * 16384 - 14, 2 * 16384 + 12],
+    "enc_end_at_edge": [3 * 16384 - 1, 3 * 16384, 4 * 16384 - 1],
+    "enc_span_many": [100, 16384 * 40 + 57],
+    "enc_dense_block": list(range(5 * 16384 - 200, 5 * 16384 + 200)),
+}
+
+
+@pytest.mark.parametrize("name", list(SPLIT_RUNS))
+def test_split_runs_across_encode_tiles(g, name):
+    n = SPLIT_MIN + 3
+    x = _literal_groups_case(n, SPLIT_RUNS[name])
+    st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
+    assert_roundtrip_parity(g, st, n)
+
+
+def test_split_path_nonfinite_and_zero(g):
+    n = SPLIT_MIN + 5
+    x, err, s = mixed_case(4, n)
+    x[n - 3] = np.inf
+    rc, st, e, L = gpu_compress(g, x, s, err)
+    assert rc == 2 and L == 0 and np.array_equal(bits(e), bits(err))
+    st, _ = assert_compress_parity(g, np.zeros(n, np.float32), 1.5, np.zeros(n, np.float32))
+    assert_roundtrip_parity(g, st, n)
