@@ -259,9 +259,11 @@ __device__ __forceinline__ void put_out(const TileJob &j, uint64_t pos, uint8_t 
 // exclusive prefix (emitted count, incoming run length mod 14) to all threads.
 // Each round trip reads 32 * kLookV earlier words: every lane first folds
 // its kLookV words (oldest to nearest), then lane 0 folds the lanes.
+template <int kV>
 __device__ __forceinline__ void lookback_tile(const TileJob &j, uint32_t t, const ZAgg &agg,
                                               uint32_t &cin, uint32_t &tin, QuantSmem &sm,
                                               int32_t *dev_status, uint32_t max_polls) {
+  constexpr int kLookV = kV;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (warp == 0) {
     if (t == 0) {
@@ -436,7 +438,7 @@ __device__ __forceinline__ uint32_t quant_chunk(const float *x, float *err, uint
 // kZB consecutive bytes (p0 = threadIdx.x * kZB onwards) in qw; tgv bytes of
 // the tile are valid.  Local analysis (block scans), decoupled look-back,
 // emission, header / closing byte.  Whole block; ends synchronised.
-template <int kZB>
+template <int kZB, int kV>
 __device__ __forceinline__ void zre_encode_tile(const TileJob &j, uint32_t t, uint32_t tgv,
                                                 const uint32_t (&qw)[kZB / 4], float scale,
                                                 QuantSmem &sm, int32_t *dev_status,
@@ -450,7 +452,7 @@ __device__ __forceinline__ void zre_encode_tile(const TileJob &j, uint32_t t, ui
     // Entirely 121s: only full 14-chunks of the run end inside the tile.
     const ZAgg agg = {1u, tgv, 0u, 0u};
     uint32_t cin, tin;
-    lookback_tile(j, t, agg, cin, tin, sm, dev_status, max_polls);
+    lookback_tile<kV>(j, t, agg, cin, tin, sm, dev_status, max_polls);
     const uint32_t cnt = (tin + tgv) / 14u;
     for (uint32_t i = threadIdx.x; i < cnt; i += blockDim.x) put_out(j, (uint64_t)cin + i, 255);
     finish_tile(j, t, agg, cin, tin, scale);
@@ -500,7 +502,7 @@ __device__ __forceinline__ void zre_encode_tile(const TileJob &j, uint32_t t, ui
   agg.tc = agg.all ? 0u : (uint32_t)((int)tgv - 1 - lnz_all) % 14u;
 
   uint32_t cin, tin;
-  lookback_tile(j, t, agg, cin, tin, sm, dev_status, max_polls);
+  lookback_tile<kV>(j, t, agg, cin, tin, sm, dev_status, max_polls);
 
   {
     uint64_t k_out = (uint64_t)cin + lead_count(agg, tin) + off;
@@ -568,7 +570,7 @@ __device__ __forceinline__ void quant_tile(const TileJob &j, uint32_t t, float s
       qw[4 * v + 3] = q4.w;
     }
   }
-  zre_encode_tile<kZBytes>(j, t, tgv, qw, scale, sm, dev_status, max_polls);
+  zre_encode_tile<kZBytes, kLookV>(j, t, tgv, qw, scale, sm, dev_status, max_polls);
 }
 
 // scale = M * s and the zero-band threshold from the bits of M; false when
@@ -651,6 +653,12 @@ __global__ void TLC_Q_BOUNDS k_quant_zre(const QuantArgs a) {
 // quantization as a pure streaming kernel that also writes the quartic
 // bytes (n/5 bytes) to scratch, then zero-run encodes them in large tiles.
 constexpr int kEncBytesPerThread = 64;
+// Encode tiles are light, so the prefix frontier of the look-back is what
+// limits them: read 8 words per lane (256 tiles) per round trip.
+#ifndef TLC_ENC_LOOKV
+#define TLC_ENC_LOOKV 8
+#endif
+constexpr int kEncLookV = TLC_ENC_LOOKV;
 constexpr uint32_t kEncTileGroups = kQThreads * kEncBytesPerThread;  // 16384
 static_assert(kEncTileGroups < 65536, "aggregate fields are 16 bits");
 
@@ -767,7 +775,8 @@ __global__ void __launch_bounds__(kQThreads, 2) k_zre_encode(const EncodeArgs a)
       if (p + k >= a.groups)
         qw[k >> 2] = (qw[k >> 2] & ~(0xffu << (8 * (k & 3)))) | (121u << (8 * (k & 3)));
     }
-    zre_encode_tile<kEncBytesPerThread>(job, t, tgv, qw, scale, sm, a.dev_status, a.max_polls);
+    zre_encode_tile<kEncBytesPerThread, kEncLookV>(job, t, tgv, qw, scale, sm, a.dev_status,
+                                                   a.max_polls);
   }
 }
 
