@@ -152,6 +152,7 @@ def run_ours(args, rank, world, local):
 
     import gradient_traffic_compression_b200 as tlc
     import synth
+    from gradient_traffic_compression_b200.exchange import max_over_ranks
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -231,10 +232,7 @@ def run_ours(args, rank, world, local):
 
     total_ms = t_start.elapsed_time(t_end)
     legs = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)) for i in range(3)]
-    if world > 1:
-        t = torch.tensor([total_ms] + legs, dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, legs = float(t[0]), [float(v) for v in t[1:]]
+    total_ms, *legs = max_over_ranks([total_ms] + legs, device=dev)
 
     L = int(out_len.item())
     nnz = int(torch.count_nonzero(y).item())
@@ -324,8 +322,9 @@ def run_ours(args, rank, world, local):
 def run_e2e(args, tlc, torch, dev, x_h, n, cap, world):
     """Same step through the public API with host buffers: pinned host x and
     err copied in, stream, err and y copied out, every step."""
-    import numpy as np
     import torch.distributed as dist
+
+    from gradient_traffic_compression_b200.exchange import max_over_ranks
     xh = torch.from_numpy(x_h).pin_memory()
     eh = torch.zeros(n, dtype=torch.float32).pin_memory()
     yh = torch.empty(n, dtype=torch.float32).pin_memory()
@@ -364,11 +363,7 @@ def run_e2e(args, tlc, torch, dev, x_h, n, cap, world):
         step()
     t1.record()
     torch.cuda.synchronize()
-    ms = t0.elapsed_time(t1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t[0])
+    ms = max_over_ranks([t0.elapsed_time(t1) / args.e2e_steps], device=dev)[0]
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())} in the e2e run")
     return {"value": round(world * 4 * n / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
