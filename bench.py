@@ -241,15 +241,12 @@ def run_ours(args, rank, world, local):
     value = world * in_bytes / (ms_step * 1e-3) / 1e9
     peak, peak_kind = load_peaks()
 
-    # bytes each kernel must move (as built).  Large tensors take the split
-    # path: the quantize pass (reported as k_quant_zre) also writes the
-    # quartic bytes, which k_zre_encode reads back.
-    split = kern.get("k_zre_encode", (0, 0.0))[0] > 0
-    qbytes = (n + 639) // 640 * 128
+    # bytes each kernel must move: read x and err (8n); read x, err and
+    # write err and the stream (12n + L); read the stream and write y
+    # (L + 4n); read the stream and read-modify-write acc at non-zeros
     algo = {
         "k_absmax": 8 * n,
-        "k_quant_zre": 12 * n + (qbytes if split else L),
-        "k_zre_encode": qbytes + L,
+        "k_quant_zre": 12 * n + L,
         "k_decode_write": L + 4 * n,
         "k_decode_accumulate": L + 8 * nnz,
     }
@@ -260,13 +257,11 @@ def run_ours(args, rank, world, local):
         per = ms / launches
         gbs = algo[name] / (per * 1e-3) / 1e9
         kernels[name] = {"launches": launches, "avg_ms": round(per, 5),
-                         "kernel": ("k_quant_pack (split path)" if name == "k_quant_zre" and split
-                                    else name),
                          "algo_bytes_per_launch": algo[name], "achieved_gbs": round(gbs, 1),
                          "frac": round(gbs / peak, 4)}
     dom = max(kernels, key=lambda k: kern[k][1])
     c_ms, d_ms, a_ms = (v / args.steps for v in legs)
-    compress_bytes = algo["k_absmax"] + algo["k_quant_zre"] + (algo["k_zre_encode"] if split else 0)
+    compress_bytes = algo["k_absmax"] + algo["k_quant_zre"]
     decompress_bytes = algo["k_decode_write"]
     result = {
         "metric": METRIC,

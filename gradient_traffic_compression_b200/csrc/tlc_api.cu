@@ -35,7 +35,6 @@ void init_device(int d) {
     di.occ_decode_write = tlc::occupancy_decode(false);
     di.occ_decode_acc = tlc::occupancy_decode(true);
     di.occ_quant_batch = tlc::occupancy_quant_batch();
-    tlc::occupancy_split(di.occ_pack_vec, di.occ_pack_scalar, di.occ_encode);
     di.occ_decode_batch_write = tlc::occupancy_decode_batch(false);
     di.occ_decode_batch_acc = tlc::occupancy_decode_batch(true);
     cudaMemPoolProps props;
@@ -111,7 +110,7 @@ struct Timing {
 Timing g_timing;
 
 const char *const kKindNames[tlc::kKindCount] = {"k_absmax", "k_quant_zre", "k_decode_write",
-                                                 "k_decode_accumulate", "k_zre_encode"};
+                                                 "k_decode_accumulate"};
 
 }  // namespace
 
@@ -214,13 +213,13 @@ tlc_status tlc_compress(const float *x, size_t n, float s, float *err, uint8_t *
   if (!dev) return TLC_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   void *scratch = nullptr;
-  const size_t bytes = tlc::compress_scratch_bytes_for(*dev, n, true);
+  const size_t bytes = tlc::compress_scratch_bytes_for(*dev, n);
   if (scratch_alloc(*dev, bytes + 256, &scratch, st) != cudaSuccess) return TLC_ERR_CUDA;
   // a status word for calls without one, past everything the kernels use
   int32_t *status_ptr =
       dev_status ? dev_status : reinterpret_cast<int32_t *>(static_cast<char *>(scratch) + bytes);
   ce = tlc::launch_compress(*dev, x, n, s, err, out, out_cap, out_len, status_ptr, wait_limit(),
-                            scratch, st, true);
+                            scratch, st);
   const cudaError_t fe = cudaFreeAsync(scratch, st);
   return (ce == cudaSuccess && fe == cudaSuccess) ? TLC_OK : TLC_ERR_CUDA;
 }
@@ -363,7 +362,8 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   const size_t sz_M = tlc::align_up(4 * (size_t)count + 8, 256);      // mbits, q_ticket
   const size_t sz_QS = tlc::align_up(8 * qtt.size(), 256);
   const size_t sz_DS = tlc::align_up(8 * (dtt.size() + 1), 256);     // d_ticket, d_status
-  const size_t total = sz_T + sz_C + sz_Q + sz_D + sz_M + sz_QS + sz_DS + 256;
+  const size_t sz_P = tlc::align_up(sizeof(tlc::BatchPrep) * count + 8, 256);  // prep, total
+  const size_t total = sz_T + sz_C + sz_Q + sz_D + sz_M + sz_QS + sz_DS + sz_P + 256;
   tlc_plan_s *P = new tlc_plan_s();
   P->device = dev->device;
   P->count = count;
@@ -395,7 +395,9 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   D.d_status = reinterpret_cast<uint64_t *>(zd + 8);
   D.d_zero_base = zd;
   D.d_zero_bytes = 8 * (dtt.size() + 1);
-  P->spare_status = reinterpret_cast<int32_t *>(zd + sz_DS);
+  D.d_prep = reinterpret_cast<tlc::BatchPrep *>(zd + sz_DS);
+  D.d_total = reinterpret_cast<uint32_t *>(zd + sz_DS + sizeof(tlc::BatchPrep) * count);
+  P->spare_status = reinterpret_cast<int32_t *>(zd + sz_DS + sz_P);
   ce = cudaMemcpy(b, T.data(), sizeof(tlc::BatchTensor) * count, cudaMemcpyHostToDevice);
   if (ce == cudaSuccess && !chunks.empty())
     ce = cudaMemcpy(b + sz_T, chunks.data(), sizeof(tlc::BatchChunk) * chunks.size(),

@@ -647,139 +647,6 @@ __global__ void TLC_Q_BOUNDS k_quant_zre(const QuantArgs a) {
   }
 }
 
-// ------------------------------------- split path for large tensors ------
-// For large tensors the fused kernel's per-tile encode phase (block scans and
-// the look-back) stalls each block's memory stream.  The split path runs
-// quantization as a pure streaming kernel that also writes the quartic
-// bytes (n/5 bytes) to scratch, then zero-run encodes them in large tiles.
-constexpr int kEncBytesPerThread = 64;
-// Encode tiles are light, so the prefix frontier of the look-back is what
-// limits them: read 8 words per lane (256 tiles) per round trip.
-#ifndef TLC_ENC_LOOKV
-#define TLC_ENC_LOOKV 8
-#endif
-constexpr int kEncLookV = TLC_ENC_LOOKV;
-constexpr uint32_t kEncTileGroups = kQThreads * kEncBytesPerThread;  // 16384
-static_assert(kEncTileGroups < 65536, "aggregate fields are 16 bits");
-
-struct PackArgs {
-  const float *x;
-  float *err;
-  uint64_t n;
-  float s;
-  const uint32_t *partial;
-  uint32_t n_partial;
-  uint8_t *qbytes;        // ceil(n/640) * 128 bytes
-};
-
-// Every warp takes 640-value steps, grid-stride; no block synchronisation.
-template <bool kVec>
-__global__ void TLC_Q_BOUNDS k_quant_pack(const PackArgs a) {
-  __shared__ __align__(16) uint32_t dig_s[kQWarps][kChunkElems / 4];
-  __shared__ float scale_s, thr_s;
-  __shared__ int ok_s;
-  if (threadIdx.x < kWarp) {
-    uint32_t mb = 0;
-    for (uint32_t i = threadIdx.x; i < a.n_partial; i += kWarp) mb = max(mb, a.partial[i]);
-    mb = __reduce_max_sync(0xffffffffu, mb);
-    if (threadIdx.x == 0) {
-      float scale = 0.0f, thr = 0.0f;
-      ok_s = scale_from_max(mb, a.s, scale, thr) ? 1 : 0;
-      scale_s = scale;
-      thr_s = thr;
-    }
-  }
-  __syncthreads();
-  if (!ok_s) return;  // non-finite: err stays untouched; k_zre_encode reports it
-  const float scale = scale_s, thr = thr_s;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint64_t steps = (a.n + kChunkElems - 1) / kChunkElems;
-  const uint64_t nwarps = (uint64_t)gridDim.x * kQWarps;
-  for (uint64_t c = (uint64_t)blockIdx.x * kQWarps + warp; c < steps; c += nwarps) {
-    const uint64_t e0 = c * kChunkElems;
-    const bool full = kVec && e0 + kChunkElems <= a.n;
-    const uint32_t packed = quant_chunk(a.x, a.err, a.n, e0, full, scale, thr, dig_s[warp]);
-    reinterpret_cast<uint32_t *>(a.qbytes)[c * (kChunkGroups / 4) + lane] = packed;
-  }
-}
-
-struct EncodeArgs {
-  const uint8_t *qbytes;
-  uint64_t qbytes_len;    // readable bytes of qbytes
-  uint64_t groups;
-  float s;
-  const uint32_t *partial;
-  uint32_t n_partial;
-  uint8_t *out;
-  uint64_t out_cap;
-  uint64_t *out_len;
-  uint64_t *status;
-  uint32_t *ticket;
-  uint32_t n_tiles;
-  int32_t *dev_status;
-  uint32_t max_polls;
-};
-
-__global__ void __launch_bounds__(kQThreads, 2) k_zre_encode(const EncodeArgs a) {
-  __shared__ QuantSmem sm;
-  __shared__ uint32_t tile_id_s;
-  __shared__ float scale_s;
-  __shared__ int ok_s;
-  if (threadIdx.x < kWarp) {
-    uint32_t mb = 0;
-    for (uint32_t i = threadIdx.x; i < a.n_partial; i += kWarp) mb = max(mb, a.partial[i]);
-    mb = __reduce_max_sync(0xffffffffu, mb);
-    if (threadIdx.x == 0) {
-      float scale = 0.0f, thr = 0.0f;
-      ok_s = scale_from_max(mb, a.s, scale, thr) ? 1 : 0;
-      scale_s = scale;
-    }
-  }
-  __syncthreads();
-  if (!ok_s) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-      report(a.dev_status, TLC_ERR_NONFINITE);
-      *a.out_len = 0;
-    }
-    return;
-  }
-  const float scale = scale_s;
-  const TileJob job = {nullptr, nullptr, 0, a.groups, a.out, a.out_cap, a.out_len,
-                       a.status, a.n_tiles, true};
-  constexpr int kZW = kEncBytesPerThread / 4;
-  for (;;) {
-    if (threadIdx.x == 0) {
-      tile_id_s = atomicAdd(a.ticket, 1u);
-      sm.A = 0xffffffffu;
-    }
-    __syncthreads();
-    const uint32_t t = tile_id_s;
-    if (t >= a.n_tiles) break;
-    const uint64_t g0 = (uint64_t)t * kEncTileGroups;
-    const uint32_t tgv = (uint32_t)umin64(kEncTileGroups, a.groups - g0);
-    const uint64_t p = g0 + (uint64_t)threadIdx.x * kEncBytesPerThread;
-    uint32_t qw[kZW];
-#pragma unroll
-    for (int v = 0; v < kZW / 4; ++v) {
-      uint4 q4 = make_uint4(0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u);
-      if (p + 16 * (v + 1) <= a.qbytes_len)
-        q4 = __ldg(reinterpret_cast<const uint4 *>(a.qbytes + p) + v);
-      qw[4 * v] = q4.x;
-      qw[4 * v + 1] = q4.y;
-      qw[4 * v + 2] = q4.z;
-      qw[4 * v + 3] = q4.w;
-    }
-    // bytes past the tensor's groups read as all-zero groups
-#pragma unroll
-    for (int k = 0; k < kEncBytesPerThread; ++k) {
-      if (p + k >= a.groups)
-        qw[k >> 2] = (qw[k >> 2] & ~(0xffu << (8 * (k & 3)))) | (121u << (8 * (k & 3)));
-    }
-    zre_encode_tile<kEncBytesPerThread, kEncLookV>(job, t, tgv, qw, scale, sm, a.dev_status,
-                                                   a.max_polls);
-  }
-}
-
 // ------------------------------------------------- batched (tensor lists) --
 // Magnitude pass over a list of tensors: one block per chunk of up to
 // kBatchChunk values of one tensor, one atomic maximum per tensor.
@@ -888,33 +755,15 @@ uint32_t compress_partials(const DeviceInfo &dev, uint64_t n) {
   return (uint32_t)want;
 }
 
-// Large tensors take the split path (streaming quantize + separate encode).
-#ifndef TLC_SPLIT_MIN_N
-#define TLC_SPLIT_MIN_N (1ull << 22)
-#endif
-static bool use_split(uint64_t n, bool allow_split) {
-  return allow_split && n >= TLC_SPLIT_MIN_N;
-}
-static uint64_t qbytes_len(uint64_t n) {
-  return (n + kChunkElems - 1) / kChunkElems * kChunkGroups;
-}
-static uint32_t encode_tiles(uint64_t n) {
-  const uint64_t g = (n + 4) / 5;
-  return (uint32_t)((g + kEncTileGroups - 1) / kEncTileGroups);
-}
-
-size_t compress_scratch_bytes_for(const DeviceInfo &dev, uint64_t n, bool allow_split) {
-  const uint32_t n_part = compress_partials(dev, n);
-  if (!use_split(n, allow_split)) return compress_scratch_bytes(n_part, compress_tiles(n));
-  return compress_scratch_bytes(n_part, encode_tiles(n)) + align_up(qbytes_len(n), 256);
+size_t compress_scratch_bytes_for(const DeviceInfo &dev, uint64_t n) {
+  return compress_scratch_bytes(compress_partials(dev, n), compress_tiles(n));
 }
 
 cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, float s,
                             float *err, uint8_t *out, uint64_t out_cap, uint64_t *out_len,
                             int32_t *dev_status, uint32_t max_polls, void *scratch,
-                            cudaStream_t stream, bool allow_split) {
-  const bool split = use_split(n, allow_split);
-  const uint32_t n_tiles = split ? encode_tiles(n) : compress_tiles(n);
+                            cudaStream_t stream) {
+  const uint32_t n_tiles = compress_tiles(n);
   const uint32_t n_part = compress_partials(dev, n);
   CompressScratch sc = compress_scratch_layout(scratch, n_part, n_tiles);
   const bool vec = ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(err)) & 15) == 0;
@@ -931,52 +780,6 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
   timing_end(kKindAbsmax, stream);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-
-  if (split) {
-    uint8_t *qb = static_cast<uint8_t *>(scratch) + compress_scratch_bytes(n_part, n_tiles);
-    PackArgs pa;
-    pa.x = x;
-    pa.err = err;
-    pa.n = n;
-    pa.s = s;
-    pa.partial = sc.partial;
-    pa.n_partial = n_part;
-    pa.qbytes = qb;
-    const uint64_t steps = (n + kChunkElems - 1) / kChunkElems;
-    const int occ = vec ? dev.occ_pack_vec : dev.occ_pack_scalar;
-    uint64_t grid = (uint64_t)dev.sm_count * (uint64_t)(occ > 0 ? occ : 1);
-    const uint64_t need = (steps + kQWarps - 1) / kQWarps;
-    if (grid > need) grid = need;
-    timing_begin(kKindQuantZre, stream);
-    if (vec)
-      k_quant_pack<true><<<(uint32_t)grid, kQThreads, 0, stream>>>(pa);
-    else
-      k_quant_pack<false><<<(uint32_t)grid, kQThreads, 0, stream>>>(pa);
-    timing_end(kKindQuantZre, stream);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    EncodeArgs ea;
-    ea.qbytes = qb;
-    ea.qbytes_len = qbytes_len(n);
-    ea.groups = (n + 4) / 5;
-    ea.s = s;
-    ea.partial = sc.partial;
-    ea.n_partial = n_part;
-    ea.out = out;
-    ea.out_cap = out_cap;
-    ea.out_len = out_len;
-    ea.status = sc.status;
-    ea.ticket = sc.ticket;
-    ea.n_tiles = n_tiles;
-    ea.dev_status = dev_status;
-    ea.max_polls = max_polls;
-    uint32_t egrid = (uint32_t)dev.sm_count * (uint32_t)(dev.occ_encode > 0 ? dev.occ_encode : 1);
-    if (egrid > n_tiles) egrid = n_tiles;
-    timing_begin(kKindZreEncode, stream);
-    k_zre_encode<<<egrid, kQThreads, 0, stream>>>(ea);
-    timing_end(kKindZreEncode, stream);
-    return cudaGetLastError();
-  }
 
   QuantArgs qa;
   qa.x = x;
@@ -1042,12 +845,6 @@ int occupancy_quant_batch() {
   int occ = 0;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_quant_zre_batch, kQThreads, 0);
   return occ;
-}
-
-void occupancy_split(int &pack_vec, int &pack_scalar, int &encode) {
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&pack_vec, k_quant_pack<true>, kQThreads, 0);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&pack_scalar, k_quant_pack<false>, kQThreads, 0);
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&encode, k_zre_encode, kQThreads, 0);
 }
 
 int occupancy_quant(bool vec) {

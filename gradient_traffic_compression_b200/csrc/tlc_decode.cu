@@ -380,69 +380,100 @@ k_decode(const DecodeArgs a) {
 
 struct BatchDecodeArgs {
   const BatchTensor *tensors;
-  const uint32_t *tile_tensor;  // tensor of each global (upper-bound) tile
+  uint32_t count;
+  const BatchPrep *prep;        // per-tensor payload length, scale, first tile
+  const uint32_t *total;        // tiles in the compact numbering
+  uint32_t n_tiles;             // upper bound of total (sizes the grid)
   const uint8_t *arena;
-  const uint64_t *in_lens;      // per-tensor stream lengths
   uint64_t *status;
   uint32_t *ticket;
-  uint32_t n_tiles;             // upper bound over all tensors
   int32_t *dev_status;
   uint32_t max_polls;
 };
 
-// Decode the streams of a list of tensors from their arena slots: tiles of
-// all tensors in one ticket order, each look-back confined to its stream;
-// tiles past a stream's actual length do nothing.
+constexpr int kPrepThreads = 1024;
+constexpr uint32_t kSmemSearch = 2048;  // tensors whose first tiles fit in shared memory
+
+// One block: validate every tensor's stream once, and number the tiles that
+// actually exist (ceil(m / tile) per stream, 0 for a corrupt one)
+// consecutively, tensor by tensor.
+__global__ void __launch_bounds__(kPrepThreads)
+k_decode_batch_prepare(const BatchTensor *__restrict__ tensors, uint32_t count,
+                       const uint8_t *__restrict__ arena, const uint64_t *__restrict__ in_lens,
+                       uint32_t tile_bytes, BatchPrep *__restrict__ prep,
+                       uint32_t *__restrict__ total, int32_t *dev_status) {
+  __shared__ uint32_t scan_s[kPrepThreads / kWarp + 1];
+  uint32_t base = 0;
+  for (uint32_t c0 = 0; c0 < count; c0 += kPrepThreads) {
+    const uint32_t i = c0 + threadIdx.x;
+    uint64_t m = 0;
+    float scale = 0.0f;
+    uint32_t tiles = 0;
+    if (i < count) {
+      const BatchTensor &T = tensors[i];
+      if (read_stream_header(arena + T.arena_off, in_lens + i, T.cap, T.groups, m, scale)) {
+        tiles = (uint32_t)((m + tile_bytes - 1) / tile_bytes);
+      } else {
+        m = 0;
+        report(dev_status, TLC_ERR_CORRUPT);
+      }
+    }
+    uint32_t sum;
+    const uint32_t off = block_exclusive_sum<kPrepThreads>(tiles, scan_s, sum);
+    if (i < count) {
+      BatchPrep p;
+      p.m = m;
+      p.scale = scale;
+      p.act_begin = base + off;
+      prep[i] = p;
+    }
+    base += sum;
+  }
+  if (threadIdx.x == 0) *total = base;
+}
+
+// Decode the streams of a list of tensors from their arena slots: the tiles
+// that exist, numbered tensor by tensor, taken in ticket order; each
+// look-back is confined to its stream.  A tile's tensor is found by binary
+// search over the tensors' first tiles.
 template <int kMode>
 __global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArgs a) {
   constexpr int kDTile = DecodeShape<kMode>::kTile;
   extern __shared__ __align__(16) uint8_t grp_s[];
   __shared__ DecodeSmem sm;
-  __shared__ uint64_t m_s;
+  __shared__ uint32_t begin_s[kSmemSearch];
   __shared__ uint32_t tile_s;
-  __shared__ float scale_s;
-  __shared__ int ok_s;
   for (int v = threadIdx.x; v < 256; v += kDThreads) sm.lut[v] = v < 243 ? digits_of(v) : 0;
+  const bool in_smem = a.count <= kSmemSearch;
+  if (in_smem)
+    for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads) begin_s[i] = a.prep[i].act_begin;
+  const uint32_t total = *a.total;
   for (;;) {
-    if (threadIdx.x == 0) {
-      const uint32_t u = atomicAdd(a.ticket, 1u);
-      tile_s = u;
-      if (u < a.n_tiles) {
-        const BatchTensor &T = a.tensors[a.tile_tensor[u]];
-        uint64_t m = 0;
-        float scale = 0.0f;
-        ok_s = read_stream_header(a.arena + T.arena_off, a.in_lens + a.tile_tensor[u], T.cap,
-                                  T.groups, m, scale) ? 1 : 0;
-        m_s = m;
-        scale_s = scale;
-      }
-    }
+    if (threadIdx.x == 0) tile_s = atomicAdd(a.ticket, 1u);
     __syncthreads();
     const uint32_t u = tile_s;
-    if (u >= a.n_tiles) break;
-    const uint32_t id = a.tile_tensor[u];
-    const BatchTensor &T = a.tensors[id];
-    const uint32_t t = u - T.d_tile_begin;
-    if (!ok_s) {
-      if (t == 0 && threadIdx.x == 0) report(a.dev_status, TLC_ERR_CORRUPT);
-      __syncthreads();
-      continue;
+    if (u >= total) break;
+    // last tensor whose first tile is <= u (tensors without tiles are skipped
+    // naturally: they share their first tile with the next tensor)
+    uint32_t lo = 0, hi = a.count - 1;
+    while (lo < hi) {
+      const uint32_t mid = (lo + hi + 1) >> 1;
+      const uint32_t b = in_smem ? begin_s[mid] : a.prep[mid].act_begin;
+      if (b <= u) lo = mid; else hi = mid - 1;
     }
+    const BatchTensor &T = a.tensors[lo];
+    const BatchPrep &P = a.prep[lo];
     DecodeJob job;
     job.payload = a.arena + T.arena_off + 4;
-    job.m = m_s;
+    job.m = P.m;
     job.n = T.n;
     job.groups = T.groups;
-    job.scale = scale_s;
+    job.scale = P.scale;
     job.y = T.y;
     job.status = a.status + T.d_tile_begin;
     job.n_tiles = (uint32_t)((job.m + kDTile - 1) / kDTile);
     job.vec = T.vec_y != 0;
-    if (t >= job.n_tiles) {  // this stream is shorter than its slot
-      __syncthreads();
-      continue;
-    }
-    decode_tile<kMode>(job, t, sm, grp_s, a.dev_status, a.max_polls);
+    decode_tile<kMode>(job, u - P.act_begin, sm, grp_s, a.dev_status, a.max_polls);
   }
 }
 
@@ -531,11 +562,17 @@ cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
                                 int32_t *dev_status, uint32_t max_polls, cudaStream_t stream) {
   cudaError_t e = cudaMemsetAsync(p.d_zero_base, 0, p.d_zero_bytes, stream);
   if (e != cudaSuccess) return e;
+  k_decode_batch_prepare<<<1, kPrepThreads, 0, stream>>>(
+      p.tensors, p.count, arena, in_lens, decode_tile_payload_bytes(accumulate), p.d_prep,
+      p.d_total, dev_status);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   BatchDecodeArgs a;
   a.tensors = p.tensors;
-  a.tile_tensor = p.d_tile_tensor;
+  a.count = p.count;
+  a.prep = p.d_prep;
+  a.total = p.d_total;
   a.arena = arena;
-  a.in_lens = in_lens;
   a.status = p.d_status;
   a.ticket = p.d_ticket;
   a.n_tiles = p.n_d_tiles;

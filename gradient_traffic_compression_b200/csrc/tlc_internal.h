@@ -17,9 +17,6 @@ struct DeviceInfo {
   int occ_decode_write = 0;
   int occ_decode_acc = 0;
   int occ_quant_batch = 0;
-  int occ_pack_vec = 0;
-  int occ_pack_scalar = 0;
-  int occ_encode = 0;
   int occ_decode_batch_write = 0;
   int occ_decode_batch_acc = 0;
   cudaMemPool_t pool = nullptr;
@@ -68,6 +65,13 @@ struct BatchTensor {
   uint32_t vec_y;        // y 16-byte aligned
 };
 
+// Per-tensor facts of one batched decode, written by the prepare kernel.
+struct BatchPrep {
+  uint64_t m;            // payload length (0 when the stream is corrupt)
+  float scale;
+  uint32_t act_begin;    // first tile in the compact numbering
+};
+
 struct BatchChunk {
   uint32_t tensor;
   uint32_t pad;
@@ -93,6 +97,8 @@ struct BatchPlanDev {
   uint64_t *d_status;
   void *d_zero_base;      // d_ticket and d_status, contiguous
   size_t d_zero_bytes;
+  BatchPrep *d_prep;      // count entries, rewritten by every decode call
+  uint32_t *d_total;      // compact tile count of the current decode call
 };
 
 cudaError_t launch_compress_batch(const DeviceInfo &dev, const BatchPlanDev &p, float s,
@@ -111,24 +117,20 @@ const DeviceInfo *device_info(int d);
 uint32_t wait_limit();
 
 // Kernel kinds for the optional per-launch timing (see tlc_kernel_timing).
-// k_quant_zre and the split path's k_quant_pack share a kind (the quantize
-// pass); k_zre_encode is the split path's separate encode pass.
 enum KernelKind { kKindAbsmax = 0, kKindQuantZre, kKindDecodeWrite, kKindDecodeAccumulate,
-                  kKindZreEncode, kKindCount };
+                  kKindCount };
 void timing_begin(int kind, cudaStream_t stream);
 void timing_end(int kind, cudaStream_t stream);
 
 uint32_t compress_tiles(uint64_t n);
 uint32_t compress_partials(const DeviceInfo &dev, uint64_t n);
-// Scratch bytes of one compress call (the split path for large n adds the
-// quartic bytes); allow_split = false keeps every size on the fused kernel.
-size_t compress_scratch_bytes_for(const DeviceInfo &dev, uint64_t n, bool allow_split);
+// Scratch bytes of one compress call.
+size_t compress_scratch_bytes_for(const DeviceInfo &dev, uint64_t n);
 cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, float s, float *err,
                             uint8_t *out, uint64_t out_cap, uint64_t *out_len,
                             int32_t *dev_status, uint32_t max_polls, void *scratch,
-                            cudaStream_t stream, bool allow_split);
+                            cudaStream_t stream);
 int occupancy_quant(bool vec);
-void occupancy_split(int &pack_vec, int &pack_scalar, int &encode);
 
 // Decode scratch per stream: status[tiles] (u64) then the ticket (u64 slot);
 // both must be zero before the launch.

@@ -160,3 +160,24 @@ def test_batch_isolates_a_corrupt_stream(g):
     _, st, _ = oracle.compress(xs[1], 1.5, errs[1])
     _, y = oracle.decompress(st, sizes[1])
     assert np.array_equal(bits(b.ys[1].cpu().numpy()), bits(y))
+
+
+def test_batch_rejects_a_bad_length_and_decodes_the_rest(g):
+    sizes = [777, 5000, 20481]
+    xs, errs = zip(*[mixed(97 + i, n) for i, n in enumerate(sizes)])
+    b = Batch(g, list(xs), list(errs))
+    b.plan.compress(1.5, b.arena, b.lens, b.status)
+    torch.cuda.synchronize()
+    for bad in (0, 3, 10 ** 9):
+        lens = b.lens.clone()
+        lens[1] = bad                                   # no header / beyond the slot
+        st = torch.zeros(1, dtype=torch.int32, device="cuda")
+        for y in b.ys:
+            y.fill_(7.0)
+        b.plan.decompress(b.arena, lens, dev_status=st)
+        torch.cuda.synchronize()
+        assert int(st.item()) == 3
+        for i in (0, 2):
+            _, stream, _ = oracle.compress(xs[i], 1.5, errs[i])
+            _, y = oracle.decompress(stream, sizes[i])
+            assert np.array_equal(bits(b.ys[i].cpu().numpy()), bits(y))

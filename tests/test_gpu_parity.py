@@ -443,16 +443,15 @@ def test_bounded_wait_reports_timeout(g):
     assert_compress_parity(g, x, s, err)
 
 
-# ---- large tensors: streaming quantize + separate zero-run encode ---------
+# ---- large tensors: sizes, alignments and runs over many tiles -----------
 
-SPLIT_MIN = 1 << 22            # sizes from here on take the split path
-ENC_TILE_VALUES = 5 * 16384    # values per encode tile (16384 groups)
+SPLIT_MIN = 1 << 22
 
 
 @pytest.mark.parametrize("n,offset", [(SPLIT_MIN, 0), (SPLIT_MIN + 1, 0),
                                       (SPLIT_MIN + 12345, 0), (SPLIT_MIN + 7, 1),
                                       (SPLIT_MIN + 640 * 3 + 9, 3)])
-def test_split_path_sizes(g, n, offset):
+def test_large_sizes(g, n, offset):
     x, err, s = mixed_case(3000 + n % 997, n, zero_frac=0.7)
     st, _ = assert_compress_parity(g, x, s, err, offset=offset)
     assert_roundtrip_parity(g, st, n, offset=offset)
@@ -469,14 +468,14 @@ SPLIT_RUNS = {
 
 
 @pytest.mark.parametrize("name", list(SPLIT_RUNS))
-def test_split_runs_across_encode_tiles(g, name):
+def test_large_runs_across_tiles(g, name):
     n = SPLIT_MIN + 3
     x = _literal_groups_case(n, SPLIT_RUNS[name])
     st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
     assert_roundtrip_parity(g, st, n)
 
 
-def test_split_path_nonfinite_and_zero(g):
+def test_large_nonfinite_and_zero(g):
     n = SPLIT_MIN + 5
     x, err, s = mixed_case(4, n)
     x[n - 3] = np.inf
