@@ -253,101 +253,114 @@ __device__ __forceinline__ void put_out(const TileJob &j, uint64_t pos, uint8_t 
   if (4 + pos < j.out_cap) j.out[4 + pos] = v;
 }
 
-// Decoupled look-back for tile t (whole block calls; warp 0 works): publish
-// the tile's aggregate, combine earlier tiles' words until an inclusive
-// prefix is found, publish this tile's inclusive prefix, and return the
-// exclusive prefix (emitted count, incoming run length mod 14) to all threads.
-// Each round trip reads 32 * kLookV earlier words: every lane first folds
-// its kLookV words (oldest to nearest), then lane 0 folds the lanes.
+// Decoupled look-back for tile t, by one whole warp: publish the tile's
+// aggregate, combine earlier tiles' words until an inclusive prefix is
+// found, publish this tile's inclusive prefix, and return the exclusive
+// prefix (emitted count, incoming run length mod 14) to every lane.  Each
+// round trip reads 32 * kV earlier words: every lane first folds its kV
+// words (oldest to nearest), then the lanes are folded in order.
+template <int kV>
+__device__ __forceinline__ void lookback_warp(const TileJob &j, uint32_t t, const ZAgg &agg,
+                                              uint32_t &cin, uint32_t &tin, int32_t *dev_status,
+                                              uint32_t max_polls) {
+  constexpr int kLookV = kV;
+  const int lane = threadIdx.x & 31;
+  if (t == 0) {
+    if (lane == 0) {
+      uint32_t C = 0, tt = 0;
+      eval_agg(C, tt, agg);
+      st_relaxed_u64(j.status, pack_prefix(C, tt));
+    }
+    cin = 0;
+    tin = 0;
+    return;
+  }
+  if (lane == 0) st_relaxed_u64(j.status + t, pack_agg(agg));
+  bool timed_out = false;
+  bool have_suffix = false;
+  ZAgg suffix = {0, 0, 0, 0};
+  int64_t end = (int64_t)t - 1;
+  uint32_t C = 0, tt = 0;
+  for (;;) {
+    uint64_t w[kLookV];
+    load_window(j.status, end, pack_prefix(0, 0), max_polls, timed_out, w);
+    int jp = kLookV;
+    uint64_t wp = 0;
+#pragma unroll
+    for (int k = 0; k < kLookV; ++k)
+      if (jp == kLookV && (w[k] >> kFlagShift) == 2) {
+        jp = k;
+        wp = w[k];
+      }
+    // this lane's words nearer than its prefix (or all of them), folded
+    // from the oldest to the nearest
+    ZAgg lagg = {1u, 0u, 0u, 0u};
+    bool have = false;
+#pragma unroll
+    for (int k = kLookV - 1; k >= 0; --k) {
+      if (k < jp) {
+        const ZAgg ak = unpack_agg(w[k]);
+        lagg = have ? compose(lagg, ak) : ak;
+        have = true;
+      }
+    }
+    uint32_t lC = 0, lt = 0;  // this lane's state after its prefix
+    if (jp < kLookV) {
+      lC = (uint32_t)(wp & 0xffffffffu);
+      lt = (uint32_t)((wp >> 32) & 0xfu);
+      if (have) eval_agg(lC, lt, lagg);
+    }
+    const uint32_t pmask = __ballot_sync(0xffffffffu, jp < kLookV);
+    const int pl = pmask ? __ffs(pmask) - 1 : kWarp;
+    if (pmask) {
+      C = __shfl_sync(0xffffffffu, lC, pl);
+      tt = __shfl_sync(0xffffffffu, lt, pl);
+    }
+    // lanes pl-1 .. 0 (or 31 .. 0 without a prefix), oldest first
+    ZAgg acc = {1u, 0u, 0u, 0u};
+    bool acc_have = false;
+    for (int l = pl - 1; l >= 0; --l) {
+      ZAgg al;
+      al.all = __shfl_sync(0xffffffffu, lagg.all, l);
+      al.A = __shfl_sync(0xffffffffu, lagg.A, l);
+      al.R = __shfl_sync(0xffffffffu, lagg.R, l);
+      al.tc = __shfl_sync(0xffffffffu, lagg.tc, l);
+      if (pmask) {
+        eval_agg(C, tt, al);
+      } else {
+        acc = acc_have ? compose(acc, al) : al;
+        acc_have = true;
+      }
+    }
+    if (pmask) {
+      if (have_suffix) eval_agg(C, tt, suffix);
+      break;
+    }
+    suffix = have_suffix ? compose(acc, suffix) : acc;
+    have_suffix = true;
+    end -= kWarp * kLookV;
+  }
+  if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(dev_status, TLC_ERR_TIMEOUT);
+  if (lane == 0) {
+    uint32_t Ci = C, ti = tt;
+    eval_agg(Ci, ti, agg);
+    st_relaxed_u64(j.status + t, pack_prefix(Ci, ti));
+  }
+  cin = C;
+  tin = tt;
+}
+
+// The same, called by the whole block (warp 0 works); ends synchronised.
 template <int kV>
 __device__ __forceinline__ void lookback_tile(const TileJob &j, uint32_t t, const ZAgg &agg,
                                               uint32_t &cin, uint32_t &tin, QuantSmem &sm,
                                               int32_t *dev_status, uint32_t max_polls) {
-  constexpr int kLookV = kV;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  if (warp == 0) {
-    if (t == 0) {
-      if (lane == 0) {
-        uint32_t C = 0, tt = 0;
-        eval_agg(C, tt, agg);
-        st_relaxed_u64(j.status, pack_prefix(C, tt));
-        sm.cin = 0;
-        sm.tin = 0;
-      }
-    } else {
-      if (lane == 0) st_relaxed_u64(j.status + t, pack_agg(agg));
-      bool timed_out = false;
-      bool have_suffix = false;
-      ZAgg suffix = {0, 0, 0, 0};
-      int64_t end = (int64_t)t - 1;
-      uint32_t C = 0, tt = 0;
-      for (;;) {
-        uint64_t w[kLookV];
-        load_window(j.status, end, pack_prefix(0, 0), max_polls, timed_out, w);
-        int jp = kLookV;
-        uint64_t wp = 0;
-#pragma unroll
-        for (int k = 0; k < kLookV; ++k)
-          if (jp == kLookV && (w[k] >> kFlagShift) == 2) {
-            jp = k;
-            wp = w[k];
-          }
-        // this lane's words nearer than its prefix (or all of them), folded
-        // from the oldest to the nearest
-        ZAgg lagg = {1u, 0u, 0u, 0u};
-        bool have = false;
-#pragma unroll
-        for (int k = kLookV - 1; k >= 0; --k) {
-          if (k < jp) {
-            const ZAgg ak = unpack_agg(w[k]);
-            lagg = have ? compose(lagg, ak) : ak;
-            have = true;
-          }
-        }
-        uint32_t lC = 0, lt = 0;  // this lane's state after its prefix
-        if (jp < kLookV) {
-          lC = (uint32_t)(wp & 0xffffffffu);
-          lt = (uint32_t)((wp >> 32) & 0xfu);
-          if (have) eval_agg(lC, lt, lagg);
-        }
-        const uint32_t pmask = __ballot_sync(0xffffffffu, jp < kLookV);
-        const int pl = pmask ? __ffs(pmask) - 1 : kWarp;
-        if (pmask) {
-          C = __shfl_sync(0xffffffffu, lC, pl);
-          tt = __shfl_sync(0xffffffffu, lt, pl);
-        }
-        // lanes pl-1 .. 0 (or 31 .. 0 without a prefix), oldest first
-        ZAgg acc = {1u, 0u, 0u, 0u};
-        bool acc_have = false;
-        for (int l = pl - 1; l >= 0; --l) {
-          ZAgg al;
-          al.all = __shfl_sync(0xffffffffu, lagg.all, l);
-          al.A = __shfl_sync(0xffffffffu, lagg.A, l);
-          al.R = __shfl_sync(0xffffffffu, lagg.R, l);
-          al.tc = __shfl_sync(0xffffffffu, lagg.tc, l);
-          if (pmask) {
-            eval_agg(C, tt, al);
-          } else {
-            acc = acc_have ? compose(acc, al) : al;
-            acc_have = true;
-          }
-        }
-        if (pmask) {
-          if (have_suffix) eval_agg(C, tt, suffix);
-          break;
-        }
-        suffix = have_suffix ? compose(acc, suffix) : acc;
-        have_suffix = true;
-        end -= kWarp * kLookV;
-      }
-      if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(dev_status, TLC_ERR_TIMEOUT);
-      if (lane == 0) {
-        sm.cin = C;
-        sm.tin = tt;
-        uint32_t Ci = C, ti = tt;
-        eval_agg(Ci, ti, agg);
-        st_relaxed_u64(j.status + t, pack_prefix(Ci, ti));
-      }
+  if ((threadIdx.x >> 5) == 0) {
+    uint32_t c, ti;
+    lookback_warp<kV>(j, t, agg, c, ti, dev_status, max_polls);
+    if ((threadIdx.x & 31) == 0) {
+      sm.cin = c;
+      sm.tin = ti;
     }
   }
   __syncthreads();
