@@ -26,11 +26,11 @@
 
 namespace tlc {
 
-// Payload bytes per thread (multiple of 4): small tiles balance the dense
+// Payload bytes per thread (1, 2 or a multiple of 4): small tiles balance the dense
 // write mode best; the accumulate mode touches little memory per tile and
 // prefers fewer, larger tiles.
 #ifndef TLC_D_BYTES_WRITE
-#define TLC_D_BYTES_WRITE 4
+#define TLC_D_BYTES_WRITE 2
 #endif
 #ifndef TLC_D_BYTES_ACC
 #define TLC_D_BYTES_ACC 8
@@ -167,11 +167,12 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
 
   // ---- load the tile's payload bytes, expansion counts, block scan -------
   const uint64_t b0 = (uint64_t)u * kDTile + (uint64_t)threadIdx.x * kDBytes;
-  uint32_t bw[kDBytes / 4];
+  uint32_t bw[(kDBytes + 3) / 4];
 #pragma unroll
-  for (int k = 0; k < kDBytes / 4; ++k) bw[k] = 0x79797979u;
+  for (int k = 0; k < (kDBytes + 3) / 4; ++k) bw[k] = 0x79797979u;
   int nvalid = 0;
-  if (b0 + kDBytes <= j.m && ((reinterpret_cast<uintptr_t>(j.payload + b0) & 3) == 0)) {
+  if (kDBytes % 4 == 0 && b0 + kDBytes <= j.m &&
+      ((reinterpret_cast<uintptr_t>(j.payload + b0) & 3) == 0)) {
     const uint32_t *p32 = reinterpret_cast<const uint32_t *>(j.payload + b0);
 #pragma unroll
     for (int k = 0; k < kDBytes / 4; ++k) bw[k] = __ldg(p32 + k);
@@ -187,18 +188,25 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
     }
   }
   uint32_t esum = 0;
+  bool mine_lit = false;  // a literal group other than the all-zero 121
 #pragma unroll
   for (int k = 0; k < kDBytes; ++k) {
     const uint32_t b = (bw[k >> 2] >> (8 * (k & 3))) & 0xffu;
-    if (k < nvalid) esum += b >= 243u ? b - 241u : 1u;
+    if (k < nvalid) {
+      esum += b >= 243u ? b - 241u : 1u;
+      mine_lit = mine_lit || (b < 243u && b != 121u);
+    }
   }
   uint32_t E;
   const uint32_t off = block_exclusive_sum<kDThreads>(esum, sm.scan, E);
-  // Dense output always expands the tile's groups in shared memory.  The
-  // accumulate mode does so too when the tile is mostly literals (then a
-  // coalesced float4 pass over acc is cheapest); for escape-heavy tiles it
-  // visits only the literal groups.
-  const bool expand = kMode == kWrite || E <= 4u * (uint32_t)kDTile;
+  // A tile without non-zero literals decodes to zeros only: plain zero
+  // stores (dense output) or nothing at all (accumulate).  Otherwise dense
+  // output expands the tile's groups in shared memory; so does the
+  // accumulate mode when the tile is mostly literals (then a coalesced
+  // float4 pass over acc is cheapest), while for escape-heavy tiles it visits
+  // only the literal groups.
+  const bool any_lit = __syncthreads_or(mine_lit) != 0;
+  const bool expand = any_lit && (kMode == kWrite || E <= 4u * (uint32_t)kDTile);
 
   // ---- look-back (warp 0); the other warps pre-fill zero groups ----------
   if (warp == 0) {
@@ -220,7 +228,29 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
   }
   const uint64_t Ec = O >= j.groups ? 0 : umin64(E, j.groups - O);
 
-  if (expand) {
+  if (!any_lit) {
+    if (kMode == kWrite) {
+      const uint64_t e_begin = 5 * O;
+      const uint64_t e_end = umin64(5 * (O + Ec), j.n);
+      const uint64_t v0 = (e_begin + 3) / 4, v1 = e_end / 4;
+      if (e_end > e_begin) {
+        if (!j.vec || v1 <= v0) {
+          for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) j.y[e] = 0.0f;
+        } else {
+          float4 *y4 = reinterpret_cast<float4 *>(j.y);
+          for (uint64_t v = v0 + threadIdx.x; v < v1; v += kDThreads)
+            y4[v] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          if (threadIdx.x < 4) {
+            const uint64_t e = e_begin + threadIdx.x;
+            if (e < 4 * v0) j.y[e] = 0.0f;
+          } else if (threadIdx.x < 8) {
+            const uint64_t e = 4 * v1 + (threadIdx.x - 4);
+            if (e < e_end) j.y[e] = 0.0f;
+          }
+        }
+      }
+    }
+  } else if (expand) {
     // literal bytes into the expanded group buffer
     uint32_t pos = off;
 #pragma unroll
