@@ -243,10 +243,14 @@ def run_ours(args, rank, world, local):
 
     # bytes each kernel must move: read x and err (8n); read x, err and
     # write err and the stream (12n + L); read the stream and write y
-    # (L + 4n); read the stream and read-modify-write acc at non-zeros
+    # (L + 4n); read the stream and read-modify-write acc at non-zeros.
+    # On the deferred-placement path (large n) k_quant_zre stages the
+    # encoded bytes and k_zre_place writes the stream (L).
+    deferred = kern.get("k_zre_place", (0, 0.0))[0] > 0
     algo = {
         "k_absmax": 8 * n,
-        "k_quant_zre": 12 * n + L,
+        "k_quant_zre": 12 * n + (0 if deferred else L),
+        "k_zre_place": L,
         "k_decode_write": L + 4 * n,
         "k_decode_accumulate": L + 8 * nnz,
     }
@@ -261,7 +265,7 @@ def run_ours(args, rank, world, local):
                          "frac": round(gbs / peak, 4)}
     dom = max(kernels, key=lambda k: kern[k][1])
     c_ms, d_ms, a_ms = (v / args.steps for v in legs)
-    compress_bytes = algo["k_absmax"] + algo["k_quant_zre"]
+    compress_bytes = algo["k_absmax"] + algo["k_quant_zre"] + (L if deferred else 0)
     decompress_bytes = algo["k_decode_write"]
     result = {
         "metric": METRIC,

@@ -66,10 +66,11 @@ def build_library(verbose: bool = False, ptxas_info: bool = False) -> str:
 
 
 KERNEL_SOURCES = {
-    "k_absmax": ["tlc_compress.cu", "tlc_device.cuh"],
-    "k_quant_zre": ["tlc_compress.cu", "tlc_device.cuh"],
-    "k_decode_write": ["tlc_decode.cu", "tlc_device.cuh"],
-    "k_decode_accumulate": ["tlc_decode.cu", "tlc_device.cuh"],
+    "k_absmax": ["tlc_compress.cu", "tlc_device.cuh", "tlc_internal.h"],
+    "k_quant_zre": ["tlc_compress.cu", "tlc_device.cuh", "tlc_internal.h"],
+    "k_zre_place": ["tlc_compress.cu", "tlc_device.cuh", "tlc_internal.h"],
+    "k_decode_write": ["tlc_decode.cu", "tlc_device.cuh", "tlc_internal.h"],
+    "k_decode_accumulate": ["tlc_decode.cu", "tlc_device.cuh", "tlc_internal.h"],
 }
 
 

@@ -110,7 +110,7 @@ struct Timing {
 Timing g_timing;
 
 const char *const kKindNames[tlc::kKindCount] = {"k_absmax", "k_quant_zre", "k_decode_write",
-                                                 "k_decode_accumulate"};
+                                                  "k_decode_accumulate", "k_zre_place"};
 
 }  // namespace
 
@@ -213,13 +213,14 @@ tlc_status tlc_compress(const float *x, size_t n, float s, float *err, uint8_t *
   if (!dev) return TLC_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   void *scratch = nullptr;
-  const size_t bytes = tlc::compress_scratch_bytes_for(*dev, n);
+  const bool deferred = tlc::compress_deferred(n);
+  const size_t bytes = tlc::compress_scratch_bytes_for(*dev, n, deferred);
   if (scratch_alloc(*dev, bytes + 256, &scratch, st) != cudaSuccess) return TLC_ERR_CUDA;
   // a status word for calls without one, past everything the kernels use
   int32_t *status_ptr =
       dev_status ? dev_status : reinterpret_cast<int32_t *>(static_cast<char *>(scratch) + bytes);
   ce = tlc::launch_compress(*dev, x, n, s, err, out, out_cap, out_len, status_ptr, wait_limit(),
-                            scratch, st);
+                            scratch, st, deferred);
   const cudaError_t fe = cudaFreeAsync(scratch, st);
   return (ce == cudaSuccess && fe == cudaSuccess) ? TLC_OK : TLC_ERR_CUDA;
 }

@@ -47,6 +47,39 @@ inline CompressScratch compress_scratch_layout(void *base, uint32_t n_part, uint
   return s;
 }
 
+// The deferred-placement path appends, after the look-back layout (whose
+// status words hold the tiles' summaries and the chunk counters there): the
+// placement chunks' summaries (compress_place_chunks u64), a finite-step
+// word, and a staging slot of compress_stage_bytes_per_tile() bytes per tile.
+struct DeferredScratch {
+  uint64_t *cagg;
+  uint32_t *ok;
+  uint8_t *stage;
+};
+
+// Staging bytes per tile of the deferred-placement path (one tile's groups).
+uint32_t compress_stage_bytes_per_tile();
+// Placement chunks of the deferred path for n_tiles tiles.
+uint32_t compress_place_chunks(uint32_t n_tiles);
+
+inline size_t deferred_head_bytes(uint32_t n_tiles) {
+  return align_up(8 * (size_t)compress_place_chunks(n_tiles) + 4, 256);
+}
+
+inline size_t deferred_scratch_bytes(uint32_t n_part, uint32_t n_tiles) {
+  return compress_scratch_bytes(n_part, n_tiles) + deferred_head_bytes(n_tiles) +
+         (size_t)n_tiles * compress_stage_bytes_per_tile();
+}
+
+inline DeferredScratch deferred_scratch_layout(void *base, uint32_t n_part, uint32_t n_tiles) {
+  DeferredScratch d;
+  char *p = static_cast<char *>(base) + compress_scratch_bytes(n_part, n_tiles);
+  d.cagg = reinterpret_cast<uint64_t *>(p);
+  d.ok = reinterpret_cast<uint32_t *>(d.cagg + compress_place_chunks(n_tiles));
+  d.stage = reinterpret_cast<uint8_t *>(p + deferred_head_bytes(n_tiles));
+  return d;
+}
+
 // ---- tensor lists (plans) ---------------------------------------------------
 // Values per block of the batched magnitude pass (a multiple of 4 * 512).
 constexpr uint32_t kBatchChunk = 8192;
@@ -118,18 +151,23 @@ uint32_t wait_limit();
 
 // Kernel kinds for the optional per-launch timing (see tlc_kernel_timing).
 enum KernelKind { kKindAbsmax = 0, kKindQuantZre, kKindDecodeWrite, kKindDecodeAccumulate,
-                  kKindCount };
+                  kKindZrePlace, kKindCount };
 void timing_begin(int kind, cudaStream_t stream);
 void timing_end(int kind, cudaStream_t stream);
 
 uint32_t compress_tiles(uint64_t n);
 uint32_t compress_partials(const DeviceInfo &dev, uint64_t n);
+// Whether tlc_compress takes the deferred-placement path for n values.
+bool compress_deferred(uint64_t n);
 // Scratch bytes of one compress call.
-size_t compress_scratch_bytes_for(const DeviceInfo &dev, uint64_t n);
+size_t compress_scratch_bytes_for(const DeviceInfo &dev, uint64_t n, bool deferred);
+// deferred: tiles stage their bytes and two small kernels place them (the
+// scratch must then be compress_scratch_bytes_for(.., true) bytes); else
+// tiles place their bytes themselves with a look-back over earlier tiles.
 cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, float s, float *err,
                             uint8_t *out, uint64_t out_cap, uint64_t *out_len,
                             int32_t *dev_status, uint32_t max_polls, void *scratch,
-                            cudaStream_t stream);
+                            cudaStream_t stream, bool deferred);
 int occupancy_quant(bool vec);
 
 // Decode scratch per stream: status[tiles] (u64) then the ticket (u64 slot);

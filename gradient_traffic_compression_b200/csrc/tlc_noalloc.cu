@@ -67,8 +67,9 @@ extern "C" tlc_status tlc_compress_noalloc(const float *x, size_t n, float s, fl
   // left from an earlier call is used.
   int32_t *status_ptr =
       dev_status ? dev_status : tlc::compress_scratch_layout(scratch, n_part, n_tiles).spare_status;
+  // the static scratch holds the look-back layout only, at any size
   const cudaError_t ce = tlc::launch_compress(*dev, x, n, s, err, out, out_cap, out_len,
                                               status_ptr, tlc::wait_limit(), scratch,
-                                              reinterpret_cast<cudaStream_t>(stream));
+                                              reinterpret_cast<cudaStream_t>(stream), false);
   return ce == cudaSuccess ? TLC_OK : TLC_ERR_CUDA;
 }

@@ -94,7 +94,10 @@ size_t tlc_compress_bound(size_t n);
  * *dev_status gets TLC_ERR_NONFINITE, *out_len gets 0, err is left
  * unchanged and out holds no stream.
  * Host errors: TLC_ERR_INVALID_ARG if a pointer is NULL, n is out of range,
- * s is outside [1, 2) or NaN, out_cap is too small, or x/err/out overlap. */
+ * s is outside [1, 2) or NaN, out_cap is too small, or x/err/out overlap.
+ * Scratch: about 8 bytes per 20480 values; from 384 * 20480 values on, also
+ * a staging area of about n/5 bytes (the placement of the zero-run encoded
+ * bytes then runs as a separate kernel). */
 tlc_status tlc_compress(const float *x, size_t n, float s, float *err,
                         uint8_t *out, size_t out_cap, uint64_t *out_len,
                         int32_t *dev_status, tlc_stream_t stream);

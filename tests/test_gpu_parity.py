@@ -445,19 +445,19 @@ def test_bounded_wait_reports_timeout(g):
 
 # ---- large tensors: sizes, alignments and runs over many tiles -----------
 
-SPLIT_MIN = 1 << 22
+LARGE_MIN = 1 << 22
 
 
-@pytest.mark.parametrize("n,offset", [(SPLIT_MIN, 0), (SPLIT_MIN + 1, 0),
-                                      (SPLIT_MIN + 12345, 0), (SPLIT_MIN + 7, 1),
-                                      (SPLIT_MIN + 640 * 3 + 9, 3)])
+@pytest.mark.parametrize("n,offset", [(LARGE_MIN, 0), (LARGE_MIN + 1, 0),
+                                      (LARGE_MIN + 12345, 0), (LARGE_MIN + 7, 1),
+                                      (LARGE_MIN + 640 * 3 + 9, 3)])
 def test_large_sizes(g, n, offset):
     x, err, s = mixed_case(3000 + n % 997, n, zero_frac=0.7)
     st, _ = assert_compress_parity(g, x, s, err, offset=offset)
     assert_roundtrip_parity(g, st, n, offset=offset)
 
 
-SPLIT_RUNS = {
+LARGE_RUNS = {
     "enc_edge_mod0": [16384 - 15, 16384 + 13],
     "enc_edge_mod1": [16384 - 16, 16384 + 14],
     "enc_edge_mod13": [2 * 16384 - 14, 2 * 16384 + 12],
@@ -467,19 +467,75 @@ SPLIT_RUNS = {
 }
 
 
-@pytest.mark.parametrize("name", list(SPLIT_RUNS))
+@pytest.mark.parametrize("name", list(LARGE_RUNS))
 def test_large_runs_across_tiles(g, name):
-    n = SPLIT_MIN + 3
-    x = _literal_groups_case(n, SPLIT_RUNS[name])
+    n = LARGE_MIN + 3
+    x = _literal_groups_case(n, LARGE_RUNS[name])
     st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
     assert_roundtrip_parity(g, st, n)
 
 
 def test_large_nonfinite_and_zero(g):
-    n = SPLIT_MIN + 5
+    n = LARGE_MIN + 5
     x, err, s = mixed_case(4, n)
     x[n - 3] = np.inf
     rc, st, e, L = gpu_compress(g, x, s, err)
     assert rc == 2 and L == 0 and np.array_equal(bits(e), bits(err))
     st, _ = assert_compress_parity(g, np.zeros(n, np.float32), 1.5, np.zeros(n, np.float32))
     assert_roundtrip_parity(g, st, n)
+
+
+# ---- the deferred-placement path (tensors of 384 tiles and more) ---------
+# Tiles there stage their bytes and a second kernel places them; below 384
+# tiles the tiles place their own bytes.  Both must give the same streams.
+
+DEFER_TILES = 384
+
+
+@pytest.mark.parametrize("n", [(DEFER_TILES - 1) * TILE_VALUES, (DEFER_TILES - 1) * TILE_VALUES + 1,
+                               DEFER_TILES * TILE_VALUES - 1, DEFER_TILES * TILE_VALUES,
+                               DEFER_TILES * TILE_VALUES + 4, (DEFER_TILES + 3) * TILE_VALUES + 641])
+def test_deferred_threshold_sizes(g, n):
+    x, err, s = mixed_case(5000 + n % 991, n, zero_frac=0.8)
+    st, _ = assert_compress_parity(g, x, s, err)
+    assert_roundtrip_parity(g, st, n)
+
+
+@pytest.mark.parametrize("name", list(RUN_CASES))
+def test_deferred_runs_across_tiles(g, name):
+    # the run cases of the look-back path, in a tensor that takes the deferred one
+    n = 5 * 4096 * (DEFER_TILES + 2) + 3
+    x = _literal_groups_case(n, RUN_CASES[name])
+    st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
+    assert_roundtrip_parity(g, st, n)
+
+
+@pytest.mark.parametrize("tail", [0, 1, 13, 14, 15, 27, 28, 4096 * 3 + 5])
+def test_deferred_run_lengths_at_stream_end(g, tail):
+    gtot = 4096 * DEFER_TILES + tail + 1
+    n = 5 * gtot
+    x = _literal_groups_case(n, [gtot - tail - 1])
+    st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
+    assert_roundtrip_parity(g, st, n)
+
+
+def test_deferred_sparse_literals_every_tile(g):
+    # one literal per tile at a drifting position: every tile has a leading
+    # run whose remainder byte depends on the tiles before it
+    n = 5 * 4096 * (DEFER_TILES + 5)
+    groups = [t * 4096 + (t * 977) % 4096 for t in range(DEFER_TILES + 5)]
+    x = _literal_groups_case(n, groups)
+    st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
+    assert_roundtrip_parity(g, st, n)
+
+
+def test_deferred_dense_and_nonfinite(g):
+    n = DEFER_TILES * TILE_VALUES + 77
+    x = (synth.uniforms(synth.key_for(7, 5), n) * 2 - 1).astype(np.float32)
+    st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
+    assert st.size - 4 > 0.9 * ((n + 4) // 5)
+    assert_roundtrip_parity(g, st, n)
+    x[n // 2] = np.nan
+    err = np.zeros(n, np.float32)
+    rc, _, e, L = gpu_compress(g, x, 1.0, err)
+    assert rc == 2 and L == 0 and np.array_equal(bits(e), bits(err))
