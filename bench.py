@@ -246,11 +246,14 @@ def run_ours(args, rank, world, local):
     # (L + 4n); read the stream and read-modify-write acc at non-zeros.
     # On the deferred-placement path (large n) k_quant_zre stages the
     # encoded bytes and k_zre_place writes the stream (L).
+    # Large streams get a counting pass over the stream (L) before each
+    # decode kernel.
     deferred = kern.get("k_zre_place", (0, 0.0))[0] > 0
     algo = {
         "k_absmax": 8 * n,
         "k_quant_zre": 12 * n + (0 if deferred else L),
         "k_zre_place": L,
+        "k_decode_count": L,
         "k_decode_write": L + 4 * n,
         "k_decode_accumulate": L + 8 * nnz,
     }

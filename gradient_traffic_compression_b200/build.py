@@ -71,6 +71,7 @@ KERNEL_SOURCES = {
     "k_zre_place": ["tlc_compress.cu", "tlc_device.cuh", "tlc_internal.h"],
     "k_decode_write": ["tlc_decode.cu", "tlc_device.cuh", "tlc_internal.h"],
     "k_decode_accumulate": ["tlc_decode.cu", "tlc_device.cuh", "tlc_internal.h"],
+    "k_decode_count": ["tlc_decode.cu", "tlc_device.cuh", "tlc_internal.h"],
 }
 
 

@@ -109,8 +109,9 @@ struct Timing {
 };
 Timing g_timing;
 
-const char *const kKindNames[tlc::kKindCount] = {"k_absmax", "k_quant_zre", "k_decode_write",
-                                                  "k_decode_accumulate", "k_zre_place"};
+const char *const kKindNames[tlc::kKindCount] = {"k_absmax",      "k_quant_zre",
+                                                  "k_decode_write", "k_decode_accumulate",
+                                                  "k_zre_place",    "k_decode_count"};
 
 }  // namespace
 
@@ -249,10 +250,10 @@ tlc_status tlc_decompress(const uint8_t *in, const uint64_t *in_len, size_t in_c
   if (scratch_alloc(*dev, bytes, &scratch, st) != cudaSuccess) return TLC_ERR_CUDA;
   uint64_t *status = static_cast<uint64_t *>(scratch);
   int32_t *status_ptr = dev_status ? dev_status : reinterpret_cast<int32_t *>(status + words);
-  ce = cudaMemsetAsync(scratch, 0, 8 * words, st);
+  ce = tlc::decode_deferred(tiles) ? cudaSuccess : cudaMemsetAsync(scratch, 0, 8 * words, st);
   if (ce == cudaSuccess)
     ce = tlc::launch_decode(*dev, in, in_len, in_cap, n, y, false, status_ptr, wait_limit(),
-                            status, reinterpret_cast<uint32_t *>(status + tiles), st);
+                            status, st);
   const cudaError_t fe = cudaFreeAsync(scratch, st);
   return (ce == cudaSuccess && fe == cudaSuccess) ? TLC_OK : TLC_ERR_CUDA;
 }
@@ -272,21 +273,23 @@ tlc_status tlc_decompress_accumulate(const uint8_t *const *ins, const uint64_t *
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t g = groups_of(n);
   size_t total_words = 0;
-  for (int w = 0; w < k; ++w)
-    total_words += tlc::decode_scratch_words(tlc::decode_tiles_max(in_caps[w], g));
+  bool zero = false;  // some stream takes the look-back path
+  for (int w = 0; w < k; ++w) {
+    const uint32_t tiles = tlc::decode_tiles_max(in_caps[w], g);
+    total_words += tlc::decode_scratch_words(tiles);
+    zero = zero || !tlc::decode_deferred(tiles);
+  }
   const size_t bytes = tlc::align_up(8 * total_words + 8, 256);
   void *scratch = nullptr;
   if (scratch_alloc(*dev, bytes, &scratch, st) != cudaSuccess) return TLC_ERR_CUDA;
   uint64_t *base = static_cast<uint64_t *>(scratch);
   int32_t *status_ptr = dev_status ? dev_status : reinterpret_cast<int32_t *>(base + total_words);
-  ce = cudaMemsetAsync(scratch, 0, 8 * total_words, st);
+  ce = zero ? cudaMemsetAsync(scratch, 0, 8 * total_words, st) : cudaSuccess;
   size_t at = 0;
   for (int w = 0; w < k && ce == cudaSuccess; ++w) {
     const uint32_t tiles = tlc::decode_tiles_max(in_caps[w], g);
-    uint64_t *status = base + at;
     ce = tlc::launch_decode(*dev, ins[w], in_lens ? in_lens + w : nullptr, in_caps[w], n, acc,
-                            true, status_ptr, wait_limit(), status,
-                            reinterpret_cast<uint32_t *>(status + tiles), st);
+                            true, status_ptr, wait_limit(), base + at, st);
     at += tlc::decode_scratch_words(tiles);
   }
   const cudaError_t fe = cudaFreeAsync(scratch, st);

@@ -151,7 +151,7 @@ uint32_t wait_limit();
 
 // Kernel kinds for the optional per-launch timing (see tlc_kernel_timing).
 enum KernelKind { kKindAbsmax = 0, kKindQuantZre, kKindDecodeWrite, kKindDecodeAccumulate,
-                  kKindZrePlace, kKindCount };
+                  kKindZrePlace, kKindDecodeCount, kKindCount };
 void timing_begin(int kind, cudaStream_t stream);
 void timing_end(int kind, cudaStream_t stream);
 
@@ -170,14 +170,45 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
                             cudaStream_t stream, bool deferred);
 int occupancy_quant(bool vec);
 
-// Decode scratch per stream: status[tiles] (u64) then the ticket (u64 slot);
-// both must be zero before the launch.
+// Decode scratch per stream: decode_scratch_words(tiles) u64 words, where
+// tiles = decode_tiles_max counts 512-byte payload units (the smallest tile).
+// Look-back path: status[tiles] (u64) then the ticket (u64 slot); both must
+// be zero before the launch.  Deferred-prefix path (decode_deferred): the
+// units' group counts (u32), the 32-unit chunks' counts (u64), then the
+// ticket; the counting kernel writes all of them, so nothing needs clearing.
+constexpr uint32_t kDecodeUnit = 512;
+constexpr uint32_t kDecodeChunkUnits = 32;
 uint32_t decode_tiles_max(uint64_t cap, uint64_t groups);
+bool decode_deferred(uint32_t tiles);
 inline size_t decode_scratch_words(uint32_t tiles) { return (size_t)tiles + 1; }
+
+struct DecodeScratch {
+  uint64_t *status;   // look-back path
+  uint32_t *ticket;
+  uint32_t *ecount;   // deferred-prefix path
+  uint64_t *csum;
+};
+
+inline DecodeScratch decode_scratch_layout(uint64_t *base, uint32_t tiles, bool deferred) {
+  DecodeScratch d = {};
+  if (deferred) {
+    d.ecount = reinterpret_cast<uint32_t *>(base);
+    d.csum = base + (tiles + 1) / 2;
+    d.ticket = reinterpret_cast<uint32_t *>(d.csum + (tiles + kDecodeChunkUnits - 1) /
+                                                         kDecodeChunkUnits);
+  } else {
+    d.status = base;
+    d.ticket = reinterpret_cast<uint32_t *>(base + tiles);
+  }
+  return d;
+}
+
+// scratch: decode_scratch_words(decode_tiles_max(cap, groups)) words, zero
+// unless decode_deferred(...) of that tile count.
 cudaError_t launch_decode(const DeviceInfo &dev, const uint8_t *in, const uint64_t *len_dev,
                           uint64_t cap, uint64_t n, float *y, bool accumulate,
-                          int32_t *dev_status, uint32_t max_polls, uint64_t *status,
-                          uint32_t *ticket, cudaStream_t stream);
+                          int32_t *dev_status, uint32_t max_polls, uint64_t *scratch,
+                          cudaStream_t stream);
 cudaError_t launch_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_status,
                              cudaStream_t stream);
 int occupancy_decode(bool accumulate);

@@ -116,7 +116,10 @@ tlc_status tlc_compress(const float *x, size_t n, float s, float *err,
  * TLC_ERR_CORRUPT in *dev_status when the length read from in_len is below
  * 4 or above in_cap, the header is negative or not finite, or the payload
  * does not expand to exactly ceil(n/5) groups.  Then y holds unspecified
- * values, but nothing outside y is written. */
+ * values, but nothing outside y is written.
+ * When min(in_cap - 4, ceil(n/5)) spans 16384 or more 512-byte units
+ * (about 8 MiB; per stream in tlc_decompress_accumulate), a counting kernel
+ * runs before the decode kernel; the result is the same. */
 tlc_status tlc_decompress(const uint8_t *in, const uint64_t *in_len,
                           size_t in_cap, size_t n, float *y,
                           int32_t *dev_status, tlc_stream_t stream);

@@ -539,3 +539,72 @@ def test_deferred_dense_and_nonfinite(g):
     err = np.zeros(n, np.float32)
     rc, _, e, L = gpu_compress(g, x, 1.0, err)
     assert rc == 2 and L == 0 and np.array_equal(bits(e), bits(err))
+
+
+# ---- decode with a counting pass (capacities of 8 MiB and more) ----------
+# When the stream's capacity allows 16384 or more 512-byte units, each
+# tile's first group index comes from a counting kernel instead of a
+# look-back; the outputs must be the same.
+
+DECODE_DEFER_BYTES = 16384 * 512
+
+
+def _dense_stream(seed, payload_bytes):
+    """A stream whose payload is (almost) all literals: uniform values, s = 1."""
+    n = 5 * payload_bytes - (seed % 4)
+    x = (synth.uniforms(synth.key_for(seed, 5), n) * 2 - 1).astype(np.float32)
+    rc, st, _ = oracle.compress(x, 1.0, np.zeros(n, np.float32))
+    assert rc == 0
+    return st, n
+
+
+@pytest.mark.parametrize("payload", [DECODE_DEFER_BYTES - 513, DECODE_DEFER_BYTES,
+                                     DECODE_DEFER_BYTES + 4 * 2048 + 77])
+def test_decode_counting_pass_dense(g, payload):
+    st, n = _dense_stream(payload % 1000, payload)
+    assert_roundtrip_parity(g, st, n)
+    for offset in (0, 1):
+        rc_o, y_o = oracle.decompress(st, n)
+        rc_g, y_g = gpu_decompress(g, st, n, offset=offset)
+        assert rc_g == rc_o == 0 and np.array_equal(bits(y_g), bits(y_o))
+    acc0 = synth.normal(synth.key_for(payload, 6), n, 1.0)
+    rc_o, a_o = oracle.decompress_accumulate([st, st], n, acc0)
+    rc_g, a_g = gpu_accumulate(g, [st, st], n, acc0)
+    assert rc_g == rc_o == 0 and np.array_equal(bits(a_g), bits(a_o))
+
+
+def test_decode_counting_pass_large_capacity_small_stream(g):
+    # a short stream in a buffer sized for the worst case: the capacity picks
+    # the counting pass, the length on the device decides the tiles
+    n = 5 * DECODE_DEFER_BYTES + 12345
+    x, err, s = mixed_case(41, n, zero_frac=0.97)
+    rc, st, _ = oracle.compress(x, s, err)
+    cap = g.tlc_compress_bound(n)
+    rc_o, y_o = oracle.decompress(st, n)
+    rc_g, y_g = gpu_decompress(g, st, n, in_len=st.size, cap=cap)
+    assert rc_g == rc_o == 0 and np.array_equal(bits(y_g), bits(y_o))
+    acc0 = synth.normal(synth.key_for(42, 6), n, 1.0)
+    rc_o, a_o = oracle.decompress_accumulate([st, st, st], n, acc0)
+    rc_g, a_g = gpu_accumulate(g, [st, st, st], n, acc0, device_lens=True)
+    assert rc_g == rc_o == 0 and np.array_equal(bits(a_g), bits(a_o))
+
+
+def test_decode_counting_pass_corrupt(g):
+    st, n = _dense_stream(7, DECODE_DEFER_BYTES + 999)
+    # one byte short: the groups no longer add up to ceil(n/5)
+    rc, _ = gpu_decompress(g, st[:-1], n)
+    assert rc == 3
+    # a length above the capacity, and a negative header
+    rc, _ = gpu_decompress(g, st, n, in_len=st.size + 1, cap=st.size)
+    assert rc == 3
+    bad = st.copy()
+    bad[3] |= 0x80
+    rc, _ = gpu_decompress(g, bad, n)
+    assert rc == 3
+    # an escape that runs past the tensor's groups
+    bad = st.copy()
+    bad[4 + 1000] = 255
+    rc, _ = gpu_decompress(g, bad, n)
+    assert rc == 3
+    # the context is still usable, and a good stream still decodes
+    assert_roundtrip_parity(g, st, n)
