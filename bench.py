@@ -85,7 +85,68 @@ def workload_config(n, log2n):
 
 # ----------------------------------------------------------- clock sampler --
 
-class ClockSampler:
+class NvmlClockSampler:
+    """SM clock and clock-event reasons read through NVML (read-only queries)
+    every `period` seconds on a background thread; only samples between
+    mark("start") and mark("end") are summarised."""
+
+    NAMES = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+             ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+             ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+             ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, bus_id=None, period=0.01):
+        import threading
+
+        import pynvml
+        pynvml.nvmlInit()
+        self.nv = pynvml
+        self.h = (pynvml.nvmlDeviceGetHandleByPciBusId(bus_id) if bus_id
+                  else pynvml.nvmlDeviceGetHandleByIndex(0))
+        self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        self.samples = []
+        self.period = period
+        self.halt = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _run(self):
+        nv, h = self.nv, self.h
+        while not self.halt.is_set():
+            try:
+                self.samples.append((time.time(), nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+            except Exception:
+                pass
+            self.halt.wait(self.period)
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self):
+        self.halt.set()
+        self.thread.join(5)
+        t0, t1 = getattr(self, "start", None), getattr(self, "end", None)
+        rows = [r for r in self.samples if t0 is None or t1 is None or t0 <= r[0] <= t1]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["no samples"],
+                    "samples": 0, "source": "nvml"}
+        reasons = sorted({name for _, _, bits in rows for name, attr in self.NAMES
+                          if bits & getattr(self.nv, attr)})
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": self.max_mhz,
+                "sm_min_mhz": min(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows), "source": "nvml"}
+
+
+def ClockSampler(bus_id=None):
+    """NVML sampler when pynvml works, else nvidia-smi -lms."""
+    try:
+        return NvmlClockSampler(bus_id)
+    except Exception:
+        return SmiClockSampler(bus_id)
+
+
+class SmiClockSampler:
     FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
