@@ -257,29 +257,33 @@ def run_ours(args, rank, world, local):
     except Exception:
         bus = None
 
-    # per-leg events (compress | decompress | accumulate) and library kernel timing
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # The dominant kernel kind, from a pass with every kind timed (part of
+    # the warm-up, untimed).
+    tlc.tlc_kernel_timing_kinds(None)
+    tlc.tlc_kernel_timing(True)
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    tlc.tlc_kernel_timing(False)
+    pre = tlc.tlc_kernel_timing_read()
+    dom = max((k for k in pre if pre[k][0]), key=lambda k: pre[k][1])
+
+    # Timed region: K steps between two events, with an event pair around
+    # each launch of the dominant kernel only (each pair costs a few
+    # microseconds of device time).  Every launch is counted.
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(bus)
     time.sleep(0.2)
+    tlc.tlc_kernel_timing_kinds([dom])
     tlc.tlc_kernel_timing(True)
     sampler.mark("start")
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for k in range(args.steps):
-        e = ev[k]
-        e[0].record(stream)
-        tlc.tlc_compress(x, S_PARAM, err, out, out_len, status, stream)
-        e[1].record(stream)
-        tlc.tlc_decompress(out, n, y, in_len=out_len, in_cap=cap, dev_status=status,
-                           stream=stream)
-        e[2].record(stream)
-        tlc.tlc_decompress_accumulate([out], n, acc, in_lens=out_len, in_caps=[cap],
-                                      dev_status=status, stream=stream)
-        e[3].record(stream)
+    for _ in range(args.steps):
+        step()
     t_end.record(stream)
     torch.cuda.synchronize()
     sampler.mark("end")
@@ -290,10 +294,33 @@ def run_ours(args, rank, world, local):
     kern = tlc.tlc_kernel_timing_read()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the timed region")
-
     total_ms = t_start.elapsed_time(t_end)
-    legs = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)) for i in range(3)]
-    total_ms, *legs = max_over_ranks([total_ms] + legs, device=dev)
+    dom_ms = kern[dom][1] / max(kern[dom][0], 1)
+    total_ms, dom_ms = max_over_ranks([total_ms, dom_ms], device=dev)
+
+    # Breakdown pass after the timed region (not part of `value`): every
+    # kind timed, and events between the three calls of each step.
+    steps2 = max(1, min(args.steps, 100))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps2)]
+    tlc.tlc_kernel_timing_kinds(None)
+    tlc.tlc_kernel_timing(True)
+    for k in range(steps2):
+        e = ev[k]
+        e[0].record(stream)
+        tlc.tlc_compress(x, S_PARAM, err, out, out_len, status, stream)
+        e[1].record(stream)
+        tlc.tlc_decompress(out, n, y, in_len=out_len, in_cap=cap, dev_status=status,
+                           stream=stream)
+        e[2].record(stream)
+        tlc.tlc_decompress_accumulate([out], n, acc, in_lens=out_len, in_caps=[cap],
+                                      dev_status=status, stream=stream)
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    tlc.tlc_kernel_timing(False)
+    kern2 = tlc.tlc_kernel_timing_read()
+    legs = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps2)) / steps2
+            for i in range(3)]
+    legs = max_over_ranks(legs, device=dev)
 
     L = int(out_len.item())
     nnz = int(torch.count_nonzero(y).item())
@@ -319,7 +346,7 @@ def run_ours(args, rank, world, local):
         "k_decode_accumulate": L + 8 * nnz,
     }
     kernels = {}
-    for name, (launches, ms) in kern.items():
+    for name, (launches, ms) in kern2.items():
         if launches == 0:
             continue
         per = ms / launches
@@ -327,8 +354,8 @@ def run_ours(args, rank, world, local):
         kernels[name] = {"launches": launches, "avg_ms": round(per, 5),
                          "algo_bytes_per_launch": algo[name], "achieved_gbs": round(gbs, 1),
                          "frac": round(gbs / peak, 4)}
-    dom = max(kernels, key=lambda k: kern[k][1])
-    c_ms, d_ms, a_ms = (v / args.steps for v in legs)
+    dom_gbs = algo[dom] / (dom_ms * 1e-3) / 1e9
+    c_ms, d_ms, a_ms = legs
     compress_bytes = algo["k_absmax"] + algo["k_quant_zre"] + (L if deferred else 0)
     decompress_bytes = algo["k_decode_write"]
     result = {
@@ -352,12 +379,13 @@ def run_ours(args, rank, world, local):
         "roofline": {
             "bound": "hbm",
             "kernel": dom,
-            "achieved": kernels[dom]["achieved_gbs"],
+            "achieved": round(dom_gbs, 1),
             "peak": peak,
             "peak_source": f"{peak_kind} hbm_gbs",
             "unit": "GB/s",
-            "frac": kernels[dom]["frac"],
+            "frac": round(dom_gbs / peak, 4),
             "traffic": traffic_for(dom, n),
+            "timing": f"CUDA events around every {dom} launch in the timed region",
         },
         "legs": {
             "compress_gbs": round(in_bytes / (c_ms * 1e-3) / 1e9, 1),
@@ -373,6 +401,8 @@ def run_ours(args, rank, world, local):
             "nonzero_values": nnz,
         },
         "kernels": kernels,
+        "breakdown": (f"legs and kernels: a separate pass of {steps2} steps after the timed "
+                      "region, with events between the calls and around every kernel"),
     }
 
     if not args.no_e2e:
@@ -447,6 +477,7 @@ def run_config_set(args, rank, world, local):
 
     import gradient_traffic_compression_b200 as tlc
     import synth
+    from gradient_traffic_compression_b200.exchange import max_over_ranks
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -510,10 +541,29 @@ def run_config_set(args, rank, world, local):
             pass
     torch.cuda.synchronize()
     steps = max(1, min(args.steps, 50))
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    # timed region: whole steps between two events; launches counted, no
+    # per-kernel events
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
+    tlc.tlc_kernel_timing_kinds([])
+    tlc.tlc_kernel_timing(True)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        for _ in legs():
+            pass
+    t1.record(stream)
+    torch.cuda.synchronize()
+    tlc.tlc_kernel_timing(False)
+    launches = tlc.tlc_kernel_timing_read()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())}")
+    step_ms = max_over_ranks([t0.elapsed_time(t1) / steps], device=dev)[0]
+    # breakdown pass: events between the legs and around every kernel
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    tlc.tlc_kernel_timing_kinds(None)
     tlc.tlc_kernel_timing(True)
     for k in range(steps):
         ev[k][0].record(stream)
@@ -522,11 +572,8 @@ def run_config_set(args, rank, world, local):
     torch.cuda.synchronize()
     tlc.tlc_kernel_timing(False)
     kern = tlc.tlc_kernel_timing_read()
-    if int(status.item()) != 0:
-        raise RuntimeError(f"device status {int(status.item())}")
     legs_ms = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)) / steps
                for i in range(3)]
-    step_ms = sum(legs_ms)
     L = int(lens.sum().item())
     in_bytes = 4 * total
     peak, _ = load_peaks()
@@ -544,7 +591,9 @@ def run_config_set(args, rank, world, local):
                  "stream_bytes": L, "bits_per_value": round(8 * L / total, 5)},
         "kernels": {k: {"launches": v[0], "avg_ms": round(v[1] / max(v[0], 1), 5)}
                     for k, v in kern.items() if v[0]},
-        "gpu_launches": int(sum(v[0] for v in kern.values())),
+        "gpu_launches": int(sum(v[0] for v in launches.values())),
+        "breakdown": ("legs and kernels: a separate pass of the same steps after the timed "
+                      "region, with events between the legs and around every kernel"),
     }
     if args.config == 5:
         res["legs"]["accumulate_ms"] = round(legs_ms[2], 4)

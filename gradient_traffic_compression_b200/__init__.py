@@ -26,6 +26,7 @@ from .tlc import (  # noqa: F401
     tlc_decompress_batch,
     tlc_decompress_accumulate,
     tlc_kernel_timing,
+    tlc_kernel_timing_kinds,
     tlc_plan_arena_bytes,
     tlc_plan_create,
     tlc_plan_destroy,

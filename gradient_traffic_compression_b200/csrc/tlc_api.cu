@@ -86,6 +86,7 @@ cudaError_t scratch_alloc(const tlc::DeviceInfo &dev, size_t bytes, void **p, cu
 struct Timing {
   std::mutex mu;
   std::atomic<bool> on{false};
+  uint32_t kinds = ~0u;  // kinds that get an event pair
   struct Pending {
     int kind;
     cudaEvent_t b, e;
@@ -93,7 +94,7 @@ struct Timing {
   std::vector<Pending> pending;
   std::vector<cudaEvent_t> spare;
   cudaEvent_t open_begin[tlc::kKindCount] = {};
-  uint64_t launches[tlc::kKindCount] = {};
+  uint64_t launches[tlc::kKindCount] = {};  // every launch while on
   double ms[tlc::kKindCount] = {};
 
   cudaEvent_t get() {
@@ -109,9 +110,9 @@ struct Timing {
 };
 Timing g_timing;
 
-const char *const kKindNames[tlc::kKindCount] = {"k_absmax",      "k_quant_zre",
-                                                  "k_decode_write", "k_decode_accumulate",
-                                                  "k_zre_place",    "k_decode_count"};
+const char *const kKindNames[tlc::kKindCount] = {
+    "k_absmax",    "k_quant_zre",    "k_decode_write",        "k_decode_accumulate",
+    "k_zre_place", "k_decode_count", "k_decode_batch_prepare"};
 
 }  // namespace
 
@@ -126,6 +127,8 @@ uint32_t wait_limit() { return ::wait_limit(); }
 void timing_begin(int kind, cudaStream_t stream) {
   if (!g_timing.on.load(std::memory_order_relaxed)) return;
   std::lock_guard<std::mutex> lk(g_timing.mu);
+  g_timing.launches[kind] += 1;
+  if (!((g_timing.kinds >> kind) & 1u)) return;
   cudaEvent_t ev = g_timing.get();
   cudaEventRecord(ev, stream);
   g_timing.open_begin[kind] = ev;
@@ -144,6 +147,11 @@ void timing_end(int kind, cudaStream_t stream) {
 
 extern "C" {
 
+void tlc_kernel_timing_kinds(uint32_t mask) {
+  std::lock_guard<std::mutex> lk(g_timing.mu);
+  g_timing.kinds = mask;
+}
+
 void tlc_kernel_timing(int enable) {
   std::lock_guard<std::mutex> lk(g_timing.mu);
   if (enable) {
@@ -159,10 +167,8 @@ int tlc_kernel_timing_read(uint64_t *launches, double *total_ms, int max_kinds) 
   std::lock_guard<std::mutex> lk(g_timing.mu);
   for (auto &p : g_timing.pending) {
     float ms = 0.0f;
-    if (cudaEventSynchronize(p.e) == cudaSuccess && cudaEventElapsedTime(&ms, p.b, p.e) == cudaSuccess) {
-      g_timing.launches[p.kind] += 1;
+    if (cudaEventSynchronize(p.e) == cudaSuccess && cudaEventElapsedTime(&ms, p.b, p.e) == cudaSuccess)
       g_timing.ms[p.kind] += ms;
-    }
     g_timing.spare.push_back(p.b);
     g_timing.spare.push_back(p.e);
   }

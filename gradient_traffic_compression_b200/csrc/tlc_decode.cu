@@ -732,9 +732,11 @@ cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
                                 int32_t *dev_status, uint32_t max_polls, cudaStream_t stream) {
   cudaError_t e = cudaMemsetAsync(p.d_zero_base, 0, p.d_zero_bytes, stream);
   if (e != cudaSuccess) return e;
+  timing_begin(kKindDecodePrepare, stream);
   k_decode_batch_prepare<<<1, kPrepThreads, 0, stream>>>(
       p.tensors, p.count, arena, in_lens, decode_tile_payload_bytes(accumulate), p.d_prep,
       p.d_total, dev_status);
+  timing_end(kKindDecodePrepare, stream);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   BatchDecodeArgs a;

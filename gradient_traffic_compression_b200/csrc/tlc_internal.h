@@ -151,7 +151,7 @@ uint32_t wait_limit();
 
 // Kernel kinds for the optional per-launch timing (see tlc_kernel_timing).
 enum KernelKind { kKindAbsmax = 0, kKindQuantZre, kKindDecodeWrite, kKindDecodeAccumulate,
-                  kKindZrePlace, kKindDecodeCount, kKindCount };
+                  kKindZrePlace, kKindDecodeCount, kKindDecodePrepare, kKindCount };
 void timing_begin(int kind, cudaStream_t stream);
 void timing_end(int kind, cudaStream_t stream);
 

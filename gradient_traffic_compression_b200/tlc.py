@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
     L.tlc_kernel_timing.restype = None
     L.tlc_kernel_timing_read.argtypes = [P, P, ctypes.c_int]
     L.tlc_kernel_timing_read.restype = ctypes.c_int
+    L.tlc_kernel_timing_kinds.argtypes = [ctypes.c_uint32]
+    L.tlc_kernel_timing_kinds.restype = None
     L.tlc_kernel_name.argtypes = [ctypes.c_int]
     L.tlc_kernel_name.restype = ctypes.c_char_p
     _ = U64
@@ -298,13 +300,33 @@ def tlc_kernel_timing(enable: bool) -> None:
     lib().tlc_kernel_timing(1 if enable else 0)
 
 
+def tlc_kernel_timing_kinds(names=None) -> None:
+    """Give event pairs to the named kernel kinds only (None: all kinds)."""
+    L = lib()
+    if names is None:
+        L.tlc_kernel_timing_kinds(0xFFFFFFFF)
+        return
+    index = {}
+    k = 0
+    while True:
+        nm = L.tlc_kernel_name(k)
+        if nm is None:
+            break
+        index[nm.decode()] = k
+        k += 1
+    mask = 0
+    for nm in names:
+        mask |= 1 << index[nm]
+    L.tlc_kernel_timing_kinds(mask)
+
+
 def tlc_kernel_timing_read() -> dict:
     """{kernel name: (launches, total device ms)} since timing was enabled."""
     L = lib()
-    k = 8
+    k = 32
     launches = (ctypes.c_uint64 * k)()
     ms = (ctypes.c_double * k)()
-    nk = L.tlc_kernel_timing_read(launches, ms, k)
+    nk = min(L.tlc_kernel_timing_read(launches, ms, k), k)
     return {L.tlc_kernel_name(i).decode(): (int(launches[i]), float(ms[i])) for i in range(nk)}
 
 

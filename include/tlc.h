@@ -247,14 +247,20 @@ void tlc_set_wait_limit(uint32_t max_polls);
 tlc_status tlc_test_wait_timeout(uint32_t max_polls, int32_t *dev_status,
                                  tlc_stream_t stream);
 
-/* Per-kernel timing, for benchmarks.  While enabled, the library records a
- * CUDA event pair on the caller's stream around every kernel it launches.
- * tlc_kernel_timing(1) clears the totals and starts recording; (0) stops.
+/* Per-kernel timing, for benchmarks.  While enabled, the library counts
+ * every kernel it launches, by kind, and records a CUDA event pair on the
+ * caller's stream around each launch of the selected kinds.
+ * tlc_kernel_timing(1) clears the totals and starts; (0) stops.
+ * tlc_kernel_timing_kinds(mask) selects the kinds that get event pairs (bit
+ * k = kind k; all kinds at load time); an event pair costs a few
+ * microseconds of device time, so a benchmark may time one kind only.
  * tlc_kernel_timing_read waits for the recorded events and, for each kernel
  * kind k < max_kinds, stores the number of launches in launches[k] and the
- * summed device time in total_ms[k]; it returns the number of kinds.
+ * summed device time of its timed launches in total_ms[k] (0 for a kind
+ * that was not selected); it returns the number of kinds.
  * tlc_kernel_name(k) names kind k (NULL past the last one). */
 void tlc_kernel_timing(int enable);
+void tlc_kernel_timing_kinds(uint32_t mask);
 int tlc_kernel_timing_read(uint64_t *launches, double *total_ms, int max_kinds);
 const char *tlc_kernel_name(int kind);
 

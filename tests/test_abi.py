@@ -130,3 +130,27 @@ def test_plan_create_rejects_bad_arguments_on_the_host(L):
     assert L.tlc_compress_batch(None, 1.0, None, None, None, None) == INV
     assert L.tlc_decompress_batch(None, None, None, 0, None, None) == INV
     assert L.tlc_plan_arena_bytes(None) == 0
+
+
+def test_kernel_timing_names_and_kind_mask(L):
+    # host-side bookkeeping only: nothing is launched, so no event is recorded
+    import gradient_traffic_compression_b200 as g
+    names = []
+    while True:
+        nm = L.tlc_kernel_name(len(names))
+        if nm is None:
+            break
+        names.append(nm.decode())
+    for kind in ("k_absmax", "k_quant_zre", "k_zre_place", "k_decode_count", "k_decode_write",
+                 "k_decode_accumulate", "k_decode_batch_prepare"):
+        assert kind in names
+    assert len(set(names)) == len(names)
+    g.tlc_kernel_timing_kinds(["k_quant_zre"])
+    g.tlc_kernel_timing(True)
+    got = g.tlc_kernel_timing_read()
+    g.tlc_kernel_timing(False)
+    g.tlc_kernel_timing_kinds(None)
+    assert set(got) == set(names)
+    assert all(v == (0, 0.0) for v in got.values())
+    with pytest.raises(KeyError):
+        g.tlc_kernel_timing_kinds(["no_such_kernel"])
