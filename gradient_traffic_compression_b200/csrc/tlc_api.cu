@@ -339,6 +339,7 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   std::vector<tlc::BatchChunk> chunks;
   std::vector<uint32_t> qtt, dtt;
   std::vector<uint64_t> offsets(count + 1, 0);
+  uint64_t n_dchunks = 0;
   const uint32_t dtile = tlc::decode_tile_payload_bytes(false);
   for (int i = 0; i < count; ++i) {
     tlc::BatchTensor &t = T[i];
@@ -356,6 +357,9 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
     t.d_tile_begin = (uint32_t)dtt.size();
     t.d_tiles = (uint32_t)((t.groups + dtile - 1) / dtile);
     for (uint32_t k = 0; k < t.d_tiles; ++k) dtt.push_back((uint32_t)i);
+    t.d_chunk_begin = (uint32_t)n_dchunks;
+    t.d_chunks = (t.d_tiles + tlc::kDecodeChunkUnits - 1) / tlc::kDecodeChunkUnits;
+    n_dchunks += t.d_chunks;
     t.vec_q = xs && (((reinterpret_cast<uintptr_t>(t.x) | reinterpret_cast<uintptr_t>(t.err)) &
                       15) == 0);
     t.vec_y = ys && ((reinterpret_cast<uintptr_t>(t.y) & 15) == 0);
@@ -373,7 +377,9 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   const size_t sz_QS = tlc::align_up(8 * qtt.size(), 256);
   const size_t sz_DS = tlc::align_up(8 * (dtt.size() + 1), 256);     // d_ticket, d_status
   const size_t sz_P = tlc::align_up(sizeof(tlc::BatchPrep) * count + 8, 256);  // prep, total
-  const size_t total = sz_T + sz_C + sz_Q + sz_D + sz_M + sz_QS + sz_DS + sz_P + 256;
+  const size_t sz_E = tlc::align_up(4 * dtt.size(), 256);            // counting pass
+  const size_t sz_S = tlc::align_up(8 * n_dchunks, 256);
+  const size_t total = sz_T + sz_C + sz_Q + sz_D + sz_M + sz_QS + sz_DS + sz_P + 256 + sz_E + sz_S;
   tlc_plan_s *P = new tlc_plan_s();
   P->device = dev->device;
   P->count = count;
@@ -408,6 +414,9 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   D.d_prep = reinterpret_cast<tlc::BatchPrep *>(zd + sz_DS);
   D.d_total = reinterpret_cast<uint32_t *>(zd + sz_DS + sizeof(tlc::BatchPrep) * count);
   P->spare_status = reinterpret_cast<int32_t *>(zd + sz_DS + sz_P);
+  D.d_ecount = reinterpret_cast<uint32_t *>(zd + sz_DS + sz_P + 256);
+  D.d_csum = reinterpret_cast<uint64_t *>(zd + sz_DS + sz_P + 256 + sz_E);
+  D.n_d_chunks = (uint32_t)n_dchunks;
   ce = cudaMemcpy(b, T.data(), sizeof(tlc::BatchTensor) * count, cudaMemcpyHostToDevice);
   if (ce == cudaSuccess && !chunks.empty())
     ce = cudaMemcpy(b + sz_T, chunks.data(), sizeof(tlc::BatchChunk) * chunks.size(),

@@ -453,13 +453,67 @@ k_decode(const DecodeArgs a) {
   }
 }
 
-// Deferred prefixes, first pass: the group count of every 512-byte payload
-// unit (one warp per unit, one 32-bit word per lane) and of every chunk of
-// kDecodeChunkUnits units (one block per chunk, blocks striding over the
-// chunks that exist).  Block 0 also clears k_decode's ticket.  A stream whose
-// length or header is invalid is left to k_decode to report.
+// Deferred prefixes, first pass, for chunk c of one stream: the group count
+// of each of its 512-byte payload units (one warp per unit, one 32-bit word
+// per lane, every word loaded before any is counted) and of the chunk.
+// Whole block; ends synchronised.
 constexpr int kUnitsPerWarp = kDecodeChunkUnits / (kDThreads / kWarp);
 static_assert(kDecodeUnit == 4 * kWarp * 4, "four words per lane per unit");
+__device__ __forceinline__ void count_chunk(const uint8_t *payload, uint64_t m, uint32_t c,
+                                            uint32_t *ecount, uint64_t *csum, uint32_t *wsum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t n_units = (uint32_t)((m + kDecodeUnit - 1) / kDecodeUnit);
+  const bool al4 = (reinterpret_cast<uintptr_t>(payload) & 3) == 0;
+  constexpr int kW = kUnitsPerWarp * (kDecodeUnit / (4 * kWarp));
+  uint32_t w[kW];
+  int nb[kW];
+#pragma unroll
+  for (int k = 0; k < kW; ++k) {
+    const uint32_t unit = c * kDecodeChunkUnits + warp * kUnitsPerWarp + k / 4;
+    const uint64_t p = (uint64_t)unit * kDecodeUnit + 4 * (uint64_t)(lane + kWarp * (k % 4));
+    w[k] = 0;
+    nb[k] = 0;
+    if (al4 && p + 4 <= m) {
+      w[k] = __ldg(reinterpret_cast<const uint32_t *>(payload + p));
+      nb[k] = 4;
+    } else {
+      for (int q = 0; q < 4; ++q)
+        if (p + q < m) {
+          w[k] |= (uint32_t)__ldg(payload + p + q) << (8 * q);
+          nb[k] = q + 1;
+        }
+    }
+  }
+  uint32_t wtot = 0;
+#pragma unroll
+  for (int i = 0; i < kUnitsPerWarp; ++i) {
+    uint32_t e = 0;
+#pragma unroll
+    for (int k = 4 * i; k < 4 * i + 4; ++k)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t b = (w[k] >> (8 * q)) & 0xffu;
+        if (q < nb[k]) e += b >= 243u ? b - 241u : 1u;
+      }
+    e = __reduce_add_sync(0xffffffffu, e);
+    const uint32_t unit = c * kDecodeChunkUnits + warp * kUnitsPerWarp + i;
+    if (lane == 0 && unit < n_units) ecount[unit] = e;
+    wtot += e;
+  }
+  if (lane == 0) wsum[warp] = wtot;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint64_t sum = 0;
+#pragma unroll
+    for (int v = 0; v < kDThreads / kWarp; ++v) sum += wsum[v];
+    csum[c] = sum;
+  }
+  __syncthreads();
+}
+
+// Counting pass of one stream: blocks stride over the chunks that exist.
+// Block 0 also clears k_decode's ticket.  A stream whose length or header is
+// invalid is left to k_decode to report.
 __global__ void __launch_bounds__(kDThreads) k_decode_count(const DecodeArgs a) {
   __shared__ uint64_t m_s;
   __shared__ int ok_s;
@@ -476,57 +530,8 @@ __global__ void __launch_bounds__(kDThreads) k_decode_count(const DecodeArgs a) 
   const uint64_t m = m_s;
   const uint32_t n_units = (uint32_t)((m + kDecodeUnit - 1) / kDecodeUnit);
   const uint32_t n_chunks = (n_units + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint8_t *payload = a.in + 4;
-  const bool al4 = (reinterpret_cast<uintptr_t>(payload) & 3) == 0;
-  for (uint32_t c = blockIdx.x; c < n_chunks; c += gridDim.x) {
-    // this warp's units, every word loaded before any is counted
-    constexpr int kW = kUnitsPerWarp * (kDecodeUnit / (4 * kWarp));
-    uint32_t w[kW];
-    int nb[kW];
-#pragma unroll
-    for (int k = 0; k < kW; ++k) {
-      const uint32_t unit = c * kDecodeChunkUnits + warp * kUnitsPerWarp + k / 4;
-      const uint64_t p = (uint64_t)unit * kDecodeUnit + 4 * (uint64_t)(lane + kWarp * (k % 4));
-      w[k] = 0;
-      nb[k] = 0;
-      if (al4 && p + 4 <= m) {
-        w[k] = __ldg(reinterpret_cast<const uint32_t *>(payload + p));
-        nb[k] = 4;
-      } else {
-        for (int q = 0; q < 4; ++q)
-          if (p + q < m) {
-            w[k] |= (uint32_t)__ldg(payload + p + q) << (8 * q);
-            nb[k] = q + 1;
-          }
-      }
-    }
-    uint32_t wtot = 0;
-#pragma unroll
-    for (int i = 0; i < kUnitsPerWarp; ++i) {
-      uint32_t e = 0;
-#pragma unroll
-      for (int k = 4 * i; k < 4 * i + 4; ++k)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t b = (w[k] >> (8 * q)) & 0xffu;
-          if (q < nb[k]) e += b >= 243u ? b - 241u : 1u;
-        }
-      e = __reduce_add_sync(0xffffffffu, e);
-      const uint32_t unit = c * kDecodeChunkUnits + warp * kUnitsPerWarp + i;
-      if (lane == 0 && unit < n_units) a.ecount[unit] = e;
-      wtot += e;
-    }
-    if (lane == 0) wsum[warp] = wtot;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      uint64_t sum = 0;
-#pragma unroll
-      for (int v = 0; v < kDThreads / kWarp; ++v) sum += wsum[v];
-      a.csum[c] = sum;
-    }
-    __syncthreads();
-  }
+  for (uint32_t c = blockIdx.x; c < n_chunks; c += gridDim.x)
+    count_chunk(a.in + 4, m, c, a.ecount, a.csum, wsum);
 }
 
 struct BatchDecodeArgs {
@@ -540,6 +545,9 @@ struct BatchDecodeArgs {
   uint32_t *ticket;
   int32_t *dev_status;
   uint32_t max_polls;
+  uint32_t *ecount;             // counting pass (plans of 16384 units and more)
+  uint64_t *csum;
+  uint32_t n_chunks;            // chunks of all tensors (upper bound)
 };
 
 constexpr int kPrepThreads = 1024;
@@ -587,7 +595,7 @@ k_decode_batch_prepare(const BatchTensor *__restrict__ tensors, uint32_t count,
 // that exist, numbered tensor by tensor, taken in ticket order; each
 // look-back is confined to its stream.  A tile's tensor is found by binary
 // search over the tensors' first tiles.
-template <int kMode>
+template <int kMode, bool kDeferred>
 __global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArgs a) {
   constexpr int kDTile = DecodeShape<kMode>::kTile;
   extern __shared__ __align__(16) uint8_t grp_s[];
@@ -624,7 +632,39 @@ __global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArg
     job.status = a.status + T.d_tile_begin;
     job.n_tiles = (uint32_t)((job.m + kDTile - 1) / kDTile);
     job.vec = T.vec_y != 0;
-    decode_tile<kMode>(job, u - P.act_begin, sm, grp_s, a.dev_status, a.max_polls);
+    job.ecount = kDeferred ? a.ecount + T.d_tile_begin : nullptr;
+    job.csum = kDeferred ? a.csum + T.d_chunk_begin : nullptr;
+    decode_tile<kMode, kDeferred>(job, u - P.act_begin, sm, grp_s, a.dev_status, a.max_polls);
+  }
+}
+
+// Counting pass of a plan's streams: blocks stride over every tensor's
+// chunks (numbered tensor by tensor, up to each tensor's bound) and count
+// those inside the tensor's stream.  A tensor's chunks start at
+// d_chunk_begin; it is found by binary search.  Block 0 also clears the
+// decode ticket.
+__global__ void __launch_bounds__(kDThreads) k_decode_batch_count(const BatchDecodeArgs a) {
+  __shared__ uint32_t begin_s[kSmemSearch];
+  __shared__ uint32_t wsum[kDThreads / kWarp];
+  const bool in_smem = a.count <= kSmemSearch;
+  if (in_smem)
+    for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads)
+      begin_s[i] = a.tensors[i].d_chunk_begin;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket = 0;
+  __syncthreads();
+  for (uint32_t g = blockIdx.x; g < a.n_chunks; g += gridDim.x) {
+    uint32_t lo = 0, hi = a.count - 1;
+    while (lo < hi) {
+      const uint32_t mid = (lo + hi + 1) >> 1;
+      const uint32_t b = in_smem ? begin_s[mid] : a.tensors[mid].d_chunk_begin;
+      if (b <= g) lo = mid; else hi = mid - 1;
+    }
+    const BatchTensor &T = a.tensors[lo];
+    const uint32_t c = g - T.d_chunk_begin;
+    const uint64_t m = a.prep[lo].m;  // 0 for a corrupt stream
+    if ((uint64_t)c * kDecodeChunkUnits * kDecodeUnit >= m) continue;  // block-uniform
+    count_chunk(a.arena + T.arena_off + 4, m, c, a.ecount + T.d_tile_begin,
+                a.csum + T.d_chunk_begin, wsum);
   }
 }
 
@@ -715,14 +755,24 @@ uint32_t decode_tile_payload_bytes(bool accumulate) {
 
 template <int kMode>
 static cudaError_t launch_batch_one(const DeviceInfo &dev, const BatchDecodeArgs &a,
-                                    cudaStream_t stream) {
+                                    bool deferred, cudaStream_t stream) {
   const size_t smem = decode_smem_bytes(kMode == kAccumulate);
   const int occ = kMode == kWrite ? dev.occ_decode_batch_write : dev.occ_decode_batch_acc;
   uint32_t grid = (uint32_t)dev.sm_count * (uint32_t)(occ > 0 ? occ : 1);
   if (grid > a.n_tiles) grid = a.n_tiles;
+  if (deferred) {
+    uint32_t cgrid = a.n_chunks;
+    if (cgrid > (uint32_t)dev.sm_count * 8) cgrid = (uint32_t)dev.sm_count * 8;
+    timing_begin(kKindDecodeCount, stream);
+    k_decode_batch_count<<<cgrid, kDThreads, 0, stream>>>(a);
+    timing_end(kKindDecodeCount, stream);
+  }
   const int kind = kMode == kWrite ? kKindDecodeWrite : kKindDecodeAccumulate;
   timing_begin(kind, stream);
-  k_decode_batch<kMode><<<grid, kDThreads, smem, stream>>>(a);
+  if (deferred)
+    k_decode_batch<kMode, true><<<grid, kDThreads, smem, stream>>>(a);
+  else
+    k_decode_batch<kMode, false><<<grid, kDThreads, smem, stream>>>(a);
   timing_end(kind, stream);
   return cudaGetLastError();
 }
@@ -750,22 +800,31 @@ cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
   a.n_tiles = p.n_d_tiles;
   a.dev_status = dev_status;
   a.max_polls = max_polls;
-  return accumulate ? launch_batch_one<kAccumulate>(dev, a, stream)
-                    : launch_batch_one<kWrite>(dev, a, stream);
+  a.ecount = p.d_ecount;
+  a.csum = p.d_csum;
+  a.n_chunks = p.n_d_chunks;
+  const bool deferred = decode_deferred(p.n_d_tiles);
+  return accumulate ? launch_batch_one<kAccumulate>(dev, a, deferred, stream)
+                    : launch_batch_one<kWrite>(dev, a, deferred, stream);
 }
 
 int occupancy_decode_batch(bool accumulate) {
   int occ = 0;
   const size_t smem = decode_smem_bytes(accumulate);
   if (accumulate) {
-    cudaFuncSetAttribute(k_decode_batch<kAccumulate>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_batch<kAccumulate>, kDThreads,
-                                                  smem);
+    cudaFuncSetAttribute(k_decode_batch<kAccumulate, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(k_decode_batch<kAccumulate, true>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_batch<kAccumulate, false>,
+                                                  kDThreads, smem);
   } else {
-    cudaFuncSetAttribute(k_decode_batch<kWrite>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_batch<kWrite>, kDThreads, smem);
+    cudaFuncSetAttribute(k_decode_batch<kWrite, false>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(k_decode_batch<kWrite, true>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_batch<kWrite, false>, kDThreads,
+                                                  smem);
   }
   return occ;
 }

@@ -94,6 +94,7 @@ struct BatchTensor {
   uint64_t cap;          // slot size = 4 + ceil(n/5)
   uint32_t q_tile_begin, q_tiles;  // compress tiles (global numbering)
   uint32_t d_tile_begin, d_tiles;  // decode tiles (global numbering, upper bound)
+  uint32_t d_chunk_begin, d_chunks;  // 32-unit chunks of the counting pass (same)
   uint32_t vec_q;        // x and err 16-byte aligned
   uint32_t vec_y;        // y 16-byte aligned
 };
@@ -132,6 +133,9 @@ struct BatchPlanDev {
   size_t d_zero_bytes;
   BatchPrep *d_prep;      // count entries, rewritten by every decode call
   uint32_t *d_total;      // compact tile count of the current decode call
+  uint32_t *d_ecount;     // counting pass: group count per 512-byte unit (n_d_tiles)
+  uint64_t *d_csum;       // and per 32-unit chunk (n_d_chunks)
+  uint32_t n_d_chunks;
 };
 
 cudaError_t launch_compress_batch(const DeviceInfo &dev, const BatchPlanDev &p, float s,

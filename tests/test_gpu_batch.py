@@ -181,3 +181,46 @@ def test_batch_rejects_a_bad_length_and_decodes_the_rest(g):
             _, stream, _ = oracle.compress(xs[i], 1.5, errs[i])
             _, y = oracle.decompress(stream, sizes[i])
             assert np.array_equal(bits(b.ys[i].cpu().numpy()), bits(y))
+
+
+def test_batch_counting_pass_large_plan(g):
+    # 8.4 M groups or more in total: the plan's decodes take the counting
+    # pass (a unit count per 512 payload bytes) instead of the look-back
+    sizes = [5 * 16384 * 512 - 3, 777, 3_000_001, 250_000]
+    xs, errs = [], []
+    for i, n in enumerate(sizes):
+        x, e = mixed(120 + i, n, zero_frac=0.3 if i != 2 else 0.95, sigma=1e-3)
+        xs.append(x)
+        errs.append(e)
+    b = Batch(g, xs, errs)
+    b.plan.compress(1.25, b.arena, b.lens, b.status)
+    b.plan.decompress(b.arena, b.lens, accumulate=False, dev_status=b.status)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    streams = []
+    for i, x in enumerate(xs):
+        rc, st, _ = oracle.compress(x, 1.25, errs[i])
+        assert rc == 0
+        assert b.stream(i).tolist() == st.tolist(), f"tensor {i}"
+        _, y = oracle.decompress(st, x.size)
+        assert np.array_equal(bits(b.ys[i].cpu().numpy()), bits(y)), f"y {i}"
+        streams.append(st)
+    accs0 = [synth.normal(synth.key_for(130 + i, 2), n, 1.0) for i, n in enumerate(sizes)]
+    for t, a in zip(b.ys, accs0):
+        t.copy_(torch.from_numpy(a))
+    b.plan.decompress(b.arena, b.lens, accumulate=True, dev_status=b.status)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    for i, x in enumerate(xs):
+        _, want = oracle.decompress_accumulate([streams[i]], x.size, accs0[i])
+        assert np.array_equal(bits(b.ys[i].cpu().numpy()), bits(want)), f"acc {i}"
+    # a corrupt stream among them is reported and the others still decode
+    lens = b.lens.clone()
+    lens[2] -= 1
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    b.plan.decompress(b.arena, lens, dev_status=st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 3
+    for i in (0, 1, 3):
+        _, y = oracle.decompress(streams[i], sizes[i])
+        assert np.array_equal(bits(b.ys[i].cpu().numpy()), bits(y)), f"y {i} after corrupt"
