@@ -339,7 +339,7 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   std::vector<tlc::BatchChunk> chunks;
   std::vector<uint32_t> qtt, dtt;
   std::vector<uint64_t> offsets(count + 1, 0);
-  uint64_t n_dchunks = 0;
+  uint64_t n_dchunks = 0, n_qchunks = 0;
   const uint32_t dtile = tlc::decode_tile_payload_bytes(false);
   for (int i = 0; i < count; ++i) {
     tlc::BatchTensor &t = T[i];
@@ -354,6 +354,8 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
     t.q_tile_begin = (uint32_t)qtt.size();
     t.q_tiles = tlc::compress_tiles(t.n);
     for (uint32_t k = 0; k < t.q_tiles; ++k) qtt.push_back((uint32_t)i);
+    t.q_chunk_begin = (uint32_t)n_qchunks;
+    n_qchunks += tlc::compress_place_chunks(t.q_tiles);
     t.d_tile_begin = (uint32_t)dtt.size();
     t.d_tiles = (uint32_t)((t.groups + dtile - 1) / dtile);
     for (uint32_t k = 0; k < t.d_tiles; ++k) dtt.push_back((uint32_t)i);
@@ -379,7 +381,12 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   const size_t sz_P = tlc::align_up(sizeof(tlc::BatchPrep) * count + 8, 256);  // prep, total
   const size_t sz_E = tlc::align_up(4 * dtt.size(), 256);            // counting pass
   const size_t sz_S = tlc::align_up(8 * n_dchunks, 256);
-  const size_t total = sz_T + sz_C + sz_Q + sz_D + sz_M + sz_QS + sz_DS + sz_P + 256 + sz_E + sz_S;
+  // deferred placement of the compress side: chunk summaries, staging
+  const bool q_def = xs && tlc::compress_deferred_tiles(qtt.size());
+  const size_t sz_QC = q_def ? tlc::align_up(8 * n_qchunks, 256) : 0;
+  const size_t sz_QT = q_def ? (size_t)tlc::compress_stage_bytes_per_tile() * qtt.size() : 0;
+  const size_t total = sz_T + sz_C + sz_Q + sz_D + sz_M + sz_QS + sz_DS + sz_P + 256 + sz_E +
+                       sz_S + sz_QC + sz_QT;
   tlc_plan_s *P = new tlc_plan_s();
   P->device = dev->device;
   P->count = count;
@@ -417,6 +424,11 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   D.d_ecount = reinterpret_cast<uint32_t *>(zd + sz_DS + sz_P + 256);
   D.d_csum = reinterpret_cast<uint64_t *>(zd + sz_DS + sz_P + 256 + sz_E);
   D.n_d_chunks = (uint32_t)n_dchunks;
+  D.q_deferred = q_def;
+  D.q_cagg = q_def ? reinterpret_cast<uint64_t *>(zd + sz_DS + sz_P + 256 + sz_E + sz_S) : nullptr;
+  D.q_stage = q_def ? reinterpret_cast<uint8_t *>(zd + sz_DS + sz_P + 256 + sz_E + sz_S + sz_QC)
+                    : nullptr;
+  D.n_q_chunks = (uint32_t)n_qchunks;
   ce = cudaMemcpy(b, T.data(), sizeof(tlc::BatchTensor) * count, cudaMemcpyHostToDevice);
   if (ce == cudaSuccess && !chunks.empty())
     ce = cudaMemcpy(b + sz_T, chunks.data(), sizeof(tlc::BatchChunk) * chunks.size(),

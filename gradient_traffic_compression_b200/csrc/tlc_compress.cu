@@ -1022,10 +1022,19 @@ struct BatchQuantArgs {
   uint32_t n_tiles;             // over all tensors
   int32_t *dev_status;
   uint32_t max_polls;
+  // deferred placement: tile summaries and chunk counters (in status),
+  // chunk summaries, staging
+  uint32_t *aggs;
+  uint32_t *ccount;
+  uint64_t *cagg;
+  uint8_t *stage;
 };
 
 // Quantize + encode over a list of tensors: tiles of all tensors in one
-// ticket order (tensor by tensor), each look-back confined to its tensor.
+// ticket order (tensor by tensor), each look-back confined to its tensor;
+// with kDeferred, each tensor's tiles stage their bytes for
+// k_zre_place_batch instead.
+template <bool kDeferred>
 __global__ void TLC_Q_BOUNDS k_quant_zre_batch(const BatchQuantArgs a) {
   __shared__ QuantSmem sm;
   __shared__ uint32_t tile_id_s;
@@ -1048,8 +1057,95 @@ __global__ void TLC_Q_BOUNDS k_quant_zre_batch(const BatchQuantArgs a) {
     }
     const TileJob job = {T.x,   T.err, T.n, T.groups, a.arena + T.arena_off, T.cap,
                          a.out_lens + id, a.status + T.q_tile_begin, T.q_tiles, T.vec_q != 0};
-    quant_tile(job, DeferJob{}, t, scale, thr, sm, a.dev_status, a.max_polls);
+    if (kDeferred) {
+      const DeferJob dj = {a.aggs + T.q_tile_begin,
+                           a.stage + (uint64_t)T.q_tile_begin * kTileGroups,
+                           a.ccount + T.q_chunk_begin, a.cagg + T.q_chunk_begin};
+      quant_tile<true>(job, dj, t, scale, thr, sm, a.dev_status, a.max_polls);
+    } else {
+      quant_tile<false>(job, DeferJob{}, t, scale, thr, sm, a.dev_status, a.max_polls);
+    }
   }
+}
+
+// Deferred placement over a list of tensors, one warp per tile (global
+// numbering): the warp finds its tensor, composes the summaries of the
+// tensor's earlier 32-tile chunks, scans its own chunk, and writes its
+// tile's leading run and staged bytes; the warp of a tensor's last tile
+// writes the closing remainder byte and the length.  Tensors whose step is
+// non-finite are skipped (k_quant_zre_batch set their length to 0).
+__global__ void __launch_bounds__(kPlaceThreads) k_zre_place_batch(const BatchQuantArgs a) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t u = blockIdx.x * (kPlaceThreads / kWarp) + (threadIdx.x >> 5);
+  if (u >= a.n_tiles) return;  // whole warp
+  const uint32_t id = a.tile_tensor[u];
+  const BatchTensor &T = a.tensors[id];
+  float scale = 0.0f, thr = 0.0f;
+  if (!scale_from_max(a.mbits[id], a.s, scale, thr)) return;
+  const uint32_t t = u - T.q_tile_begin;
+  const uint32_t c = t / kPlaceTiles;
+  const uint32_t t0 = c * kPlaceTiles;
+  const uint32_t nv = (uint32_t)umin64(kPlaceTiles, T.q_tiles - t0);
+  const uint32_t *aggs = a.aggs + T.q_tile_begin;
+  const uint64_t *cagg = a.cagg + T.q_chunk_begin;
+  // chunks [0, c) of this tensor: lane l folds [l * per, (l + 1) * per)
+  const uint32_t per = (c + kWarp - 1) / kWarp;
+  ZScan p = {0u, {0u, 0u, 0u, 0u}};
+  const uint32_t pe = (uint32_t)umin64((uint64_t)(lane + 1) * per, c);
+  for (uint32_t i = lane * per; i < pe; ++i) p = zcombine(p, {1u, ChunkCodec::unpack(cagg[i])});
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const ZScan o = zshfl_up(p, d);
+    if (lane >= d) p = zcombine(o, p);
+  }
+  uint32_t C = 0, tt = 0;
+  if (__shfl_sync(0xffffffffu, p.valid, 31)) {
+    ZAgg pa;
+    pa.all = __shfl_sync(0xffffffffu, p.a.all, 31);
+    pa.A = __shfl_sync(0xffffffffu, p.a.A, 31);
+    pa.R = __shfl_sync(0xffffffffu, p.a.R, 31);
+    pa.tc = __shfl_sync(0xffffffffu, p.a.tc, 31);
+    eval_agg(C, tt, pa);
+  }
+  // the chunk's tiles, one per lane; this tile is lane t - t0
+  uint32_t w = 0;
+  ZScan v = {0u, {0u, 0u, 0u, 0u}};
+  if ((uint32_t)lane < nv) {
+    w = aggs[t0 + lane];
+    v = {1u, unpack_agg32(w)};
+  }
+  ZScan inc = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const ZScan o = zshfl_up(inc, d);
+    if (lane >= d) inc = zcombine(o, inc);
+  }
+  ZScan exc = zshfl_up(inc, 1);
+  if (lane == 0) exc.valid = 0;
+  if (exc.valid) eval_agg(C, tt, exc.a);
+  const int me = (int)(t - t0);
+  C = __shfl_sync(0xffffffffu, C, me);
+  tt = __shfl_sync(0xffffffffu, tt, me);
+  w = __shfl_sync(0xffffffffu, w, me);
+  const ZAgg ag = unpack_agg32(w);
+  uint8_t *out = a.arena + T.arena_off;
+  const uint64_t out_cap = T.cap;
+  if (t == T.q_tiles - 1 && lane == 0) {
+    uint32_t Ce = C, te = tt;
+    eval_agg(Ce, te, ag);
+    if (te && 4ull + Ce < out_cap) out[4 + Ce] = remainder_byte(te);
+    a.out_lens[id] = 4ull + Ce + (te ? 1u : 0u);
+  }
+  const uint32_t lead = lead_count(ag, tt);
+  const uint32_t r = (tt + ag.A) % 14u;
+  const bool rem = !ag.all && r;
+  uint8_t *o = out + 4ull + C;
+  const uint64_t room = out_cap > 4ull + C ? out_cap - 4ull - C : 0;
+  warp_fill_255(o, (uint32_t)umin64(lead - (rem ? 1u : 0u), room), lane);
+  if (rem && lane == 0 && lead - 1 < room) o[lead - 1] = remainder_byte(r);
+  if (lead < room)
+    warp_copy(o + lead, a.stage + (uint64_t)u * kTileGroups, (uint32_t)umin64(ag.R, room - lead),
+              lane);
 }
 
 // ------------------------------------------------------------- launcher ---
@@ -1073,6 +1169,8 @@ size_t compress_scratch_bytes_for(const DeviceInfo &dev, uint64_t n, bool deferr
 }
 
 bool compress_deferred(uint64_t n) { return compress_tiles(n) >= kDeferMinTiles; }
+
+bool compress_deferred_tiles(uint64_t n_tiles) { return n_tiles >= kDeferMinTiles; }
 
 uint32_t compress_stage_bytes_per_tile() { return kTileGroups; }
 
@@ -1183,17 +1281,31 @@ cudaError_t launch_compress_batch(const DeviceInfo &dev, const BatchPlanDev &p, 
   qa.n_tiles = p.n_q_tiles;
   qa.dev_status = dev_status;
   qa.max_polls = max_polls;
+  qa.aggs = reinterpret_cast<uint32_t *>(p.q_status);  // cleared with the status words
+  qa.ccount = qa.aggs + p.n_q_tiles;
+  qa.cagg = p.q_cagg;
+  qa.stage = p.q_stage;
   uint32_t grid = (uint32_t)dev.sm_count * (uint32_t)(dev.occ_quant_batch > 0 ? dev.occ_quant_batch : 1);
   if (grid > p.n_q_tiles) grid = p.n_q_tiles;
   timing_begin(kKindQuantZre, stream);
-  k_quant_zre_batch<<<grid, kQThreads, 0, stream>>>(qa);
+  if (p.q_deferred)
+    k_quant_zre_batch<true><<<grid, kQThreads, 0, stream>>>(qa);
+  else
+    k_quant_zre_batch<false><<<grid, kQThreads, 0, stream>>>(qa);
   timing_end(kKindQuantZre, stream);
+  if (p.q_deferred) {
+    const uint32_t per_block = kPlaceThreads / kWarp;
+    timing_begin(kKindZrePlace, stream);
+    k_zre_place_batch<<<(p.n_q_tiles + per_block - 1) / per_block, kPlaceThreads, 0, stream>>>(
+        qa);
+    timing_end(kKindZrePlace, stream);
+  }
   return cudaGetLastError();
 }
 
 int occupancy_quant_batch() {
   int occ = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_quant_zre_batch, kQThreads, 0);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_quant_zre_batch<false>, kQThreads, 0);
   return occ;
 }
 

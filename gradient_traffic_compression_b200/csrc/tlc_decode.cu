@@ -555,40 +555,50 @@ constexpr uint32_t kSmemSearch = 2048;  // tensors whose first tiles fit in shar
 
 // One block: validate every tensor's stream once, and number the tiles that
 // actually exist (ceil(m / tile) per stream, 0 for a corrupt one)
-// consecutively, tensor by tensor.
+// consecutively, tensor by tensor; the same for the counting pass's 32-unit
+// chunks.  total[0] = tiles, total[1] = chunks.
 __global__ void __launch_bounds__(kPrepThreads)
 k_decode_batch_prepare(const BatchTensor *__restrict__ tensors, uint32_t count,
                        const uint8_t *__restrict__ arena, const uint64_t *__restrict__ in_lens,
                        uint32_t tile_bytes, BatchPrep *__restrict__ prep,
                        uint32_t *__restrict__ total, int32_t *dev_status) {
   __shared__ uint32_t scan_s[kPrepThreads / kWarp + 1];
-  uint32_t base = 0;
+  uint32_t base = 0, cbase = 0;
   for (uint32_t c0 = 0; c0 < count; c0 += kPrepThreads) {
     const uint32_t i = c0 + threadIdx.x;
     uint64_t m = 0;
     float scale = 0.0f;
-    uint32_t tiles = 0;
+    uint32_t tiles = 0, chunks = 0;
     if (i < count) {
       const BatchTensor &T = tensors[i];
       if (read_stream_header(arena + T.arena_off, in_lens + i, T.cap, T.groups, m, scale)) {
         tiles = (uint32_t)((m + tile_bytes - 1) / tile_bytes);
+        const uint64_t units = (m + kDecodeUnit - 1) / kDecodeUnit;
+        chunks = (uint32_t)((units + kDecodeChunkUnits - 1) / kDecodeChunkUnits);
       } else {
         m = 0;
         report(dev_status, TLC_ERR_CORRUPT);
       }
     }
-    uint32_t sum;
+    uint32_t sum, csum_all;
     const uint32_t off = block_exclusive_sum<kPrepThreads>(tiles, scan_s, sum);
+    const uint32_t coff = block_exclusive_sum<kPrepThreads>(chunks, scan_s, csum_all);
     if (i < count) {
       BatchPrep p;
       p.m = m;
       p.scale = scale;
       p.act_begin = base + off;
+      p.cact_begin = cbase + coff;
+      p.pad = 0;
       prep[i] = p;
     }
     base += sum;
+    cbase += csum_all;
   }
-  if (threadIdx.x == 0) *total = base;
+  if (threadIdx.x == 0) {
+    total[0] = base;
+    total[1] = cbase;
+  }
 }
 
 // Decode the streams of a list of tensors from their arena slots: the tiles
@@ -638,32 +648,30 @@ __global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArg
   }
 }
 
-// Counting pass of a plan's streams: blocks stride over every tensor's
-// chunks (numbered tensor by tensor, up to each tensor's bound) and count
-// those inside the tensor's stream.  A tensor's chunks start at
-// d_chunk_begin; it is found by binary search.  Block 0 also clears the
-// decode ticket.
+// Counting pass of a plan's streams: blocks stride over the chunks that
+// exist, numbered tensor by tensor by the prepare kernel (a tensor's first
+// chunk is found by binary search).  Block 0 also clears the decode ticket.
 __global__ void __launch_bounds__(kDThreads) k_decode_batch_count(const BatchDecodeArgs a) {
   __shared__ uint32_t begin_s[kSmemSearch];
   __shared__ uint32_t wsum[kDThreads / kWarp];
   const bool in_smem = a.count <= kSmemSearch;
   if (in_smem)
-    for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads)
-      begin_s[i] = a.tensors[i].d_chunk_begin;
+    for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads) begin_s[i] = a.prep[i].cact_begin;
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket = 0;
   __syncthreads();
-  for (uint32_t g = blockIdx.x; g < a.n_chunks; g += gridDim.x) {
+  const uint32_t total = a.total[1];
+  for (uint32_t g = blockIdx.x; g < total; g += gridDim.x) {
+    // last tensor whose first chunk is <= g (tensors without chunks share
+    // their first chunk with the next tensor)
     uint32_t lo = 0, hi = a.count - 1;
     while (lo < hi) {
       const uint32_t mid = (lo + hi + 1) >> 1;
-      const uint32_t b = in_smem ? begin_s[mid] : a.tensors[mid].d_chunk_begin;
+      const uint32_t b = in_smem ? begin_s[mid] : a.prep[mid].cact_begin;
       if (b <= g) lo = mid; else hi = mid - 1;
     }
     const BatchTensor &T = a.tensors[lo];
-    const uint32_t c = g - T.d_chunk_begin;
-    const uint64_t m = a.prep[lo].m;  // 0 for a corrupt stream
-    if ((uint64_t)c * kDecodeChunkUnits * kDecodeUnit >= m) continue;  // block-uniform
-    count_chunk(a.arena + T.arena_off + 4, m, c, a.ecount + T.d_tile_begin,
+    const BatchPrep &P = a.prep[lo];
+    count_chunk(a.arena + T.arena_off + 4, P.m, g - P.cact_begin, a.ecount + T.d_tile_begin,
                 a.csum + T.d_chunk_begin, wsum);
   }
 }

@@ -93,6 +93,7 @@ struct BatchTensor {
   uint64_t arena_off;    // the tensor's stream slot in the arena
   uint64_t cap;          // slot size = 4 + ceil(n/5)
   uint32_t q_tile_begin, q_tiles;  // compress tiles (global numbering)
+  uint32_t q_chunk_begin;          // 32-tile chunks of the deferred placement
   uint32_t d_tile_begin, d_tiles;  // decode tiles (global numbering, upper bound)
   uint32_t d_chunk_begin, d_chunks;  // 32-unit chunks of the counting pass (same)
   uint32_t vec_q;        // x and err 16-byte aligned
@@ -104,6 +105,8 @@ struct BatchPrep {
   uint64_t m;            // payload length (0 when the stream is corrupt)
   float scale;
   uint32_t act_begin;    // first tile in the compact numbering
+  uint32_t cact_begin;   // first counting-pass chunk in the compact numbering
+  uint32_t pad;
 };
 
 struct BatchChunk {
@@ -132,7 +135,11 @@ struct BatchPlanDev {
   void *d_zero_base;      // d_ticket and d_status, contiguous
   size_t d_zero_bytes;
   BatchPrep *d_prep;      // count entries, rewritten by every decode call
-  uint32_t *d_total;      // compact tile count of the current decode call
+  uint32_t *d_total;      // compact tile and chunk counts of the current decode call
+  bool q_deferred;        // compress with deferred placement (n_q_tiles >= threshold)
+  uint64_t *q_cagg;       // deferred placement: per 32-tile chunk summaries,
+  uint8_t *q_stage;       // and the staged bytes, compress_stage_bytes_per_tile() per tile;
+  uint32_t n_q_chunks;    // tile summaries and chunk counters sit in q_status
   uint32_t *d_ecount;     // counting pass: group count per 512-byte unit (n_d_tiles)
   uint64_t *d_csum;       // and per 32-unit chunk (n_d_chunks)
   uint32_t n_d_chunks;
@@ -161,8 +168,10 @@ void timing_end(int kind, cudaStream_t stream);
 
 uint32_t compress_tiles(uint64_t n);
 uint32_t compress_partials(const DeviceInfo &dev, uint64_t n);
-// Whether tlc_compress takes the deferred-placement path for n values.
+// Whether tlc_compress takes the deferred-placement path for n values, and
+// whether a plan does, for its total tile count.
 bool compress_deferred(uint64_t n);
+bool compress_deferred_tiles(uint64_t n_tiles);
 // Scratch bytes of one compress call.
 size_t compress_scratch_bytes_for(const DeviceInfo &dev, uint64_t n, bool deferred);
 // deferred: tiles stage their bytes and two small kernels place them (the

@@ -224,3 +224,33 @@ def test_batch_counting_pass_large_plan(g):
     for i in (0, 1, 3):
         _, y = oracle.decompress(streams[i], sizes[i])
         assert np.array_equal(bits(b.ys[i].cpu().numpy()), bits(y)), f"y {i} after corrupt"
+
+
+def test_batch_deferred_placement_many_tensors(g):
+    # 384 compress tiles or more in total: every tensor's tiles stage their
+    # bytes and a placement kernel writes the streams; small tensors of one
+    # tile sit beside a large one, one of them non-finite
+    rng_sizes = (synth.uniforms(synth.key_for(140, 0), 150) * 60_000).astype(np.int64) + 1
+    sizes = [int(v) for v in rng_sizes] + [384 * 20480 + 12345]
+    xs, errs = [], []
+    for i, n in enumerate(sizes):
+        x, e = mixed(150 + i, n, zero_frac=(0.5 + 0.45 * (i % 3) / 2), sigma=1e-3)
+        xs.append(x)
+        errs.append(e)
+    xs[7] = xs[7].copy()
+    xs[7][xs[7].size // 2] = np.inf
+    b = Batch(g, xs, errs, with_y=False)
+    for step in range(2):
+        b.plan.compress(1.5, b.arena, b.lens, b.status)
+        torch.cuda.synchronize()
+        assert int(b.status.item()) == 2
+        b.status.zero_()
+        for i, x in enumerate(xs):
+            rc, st, e2 = oracle.compress(x, 1.5, errs[i])
+            if i == 7:
+                assert rc == 2 and int(b.lens[i].item()) == 0
+                assert np.array_equal(bits(b.errs[i].cpu().numpy()), bits(errs[i]))
+                continue
+            assert b.stream(i).tolist() == st.tolist(), f"step {step} tensor {i} (n={x.size})"
+            assert np.array_equal(bits(b.errs[i].cpu().numpy()), bits(e2)), f"err {i}"
+            errs[i] = e2
