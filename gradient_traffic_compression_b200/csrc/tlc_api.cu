@@ -340,7 +340,6 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   std::vector<uint32_t> qtt, dtt;
   std::vector<uint64_t> offsets(count + 1, 0);
   uint64_t n_dchunks = 0, n_qchunks = 0;
-  const uint32_t dtile = tlc::decode_tile_payload_bytes(false);
   for (int i = 0; i < count; ++i) {
     tlc::BatchTensor &t = T[i];
     t.x = xs ? xs[i] : nullptr;
@@ -357,7 +356,7 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
     t.q_chunk_begin = (uint32_t)n_qchunks;
     n_qchunks += tlc::compress_place_chunks(t.q_tiles);
     t.d_tile_begin = (uint32_t)dtt.size();
-    t.d_tiles = (uint32_t)((t.groups + dtile - 1) / dtile);
+    t.d_tiles = tlc::decode_tiles_max(t.cap, t.groups);  // 512-byte units
     for (uint32_t k = 0; k < t.d_tiles; ++k) dtt.push_back((uint32_t)i);
     t.d_chunk_begin = (uint32_t)n_dchunks;
     t.d_chunks = (t.d_tiles + tlc::kDecodeChunkUnits - 1) / tlc::kDecodeChunkUnits;

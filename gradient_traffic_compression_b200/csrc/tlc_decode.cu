@@ -685,14 +685,14 @@ __global__ void k_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_s
 
 // ------------------------------------------------------------- launchers --
 uint32_t decode_tiles_max(uint64_t cap, uint64_t groups) {
-  // sized for the smaller of the two tile shapes, so it covers both modes
-  constexpr int kSmallest = DecodeShape<kWrite>::kTile < DecodeShape<kAccumulate>::kTile
-                                ? DecodeShape<kWrite>::kTile
-                                : DecodeShape<kAccumulate>::kTile;
+  // 512-byte units: at least as many as the tiles of either mode (tiles are
+  // whole units), and the counting pass's unit count
+  static_assert(DecodeShape<kWrite>::kTile % kDecodeUnit == 0 &&
+                    DecodeShape<kAccumulate>::kTile % kDecodeUnit == 0,
+                "tiles are whole units");
   uint64_t m = cap >= 4 ? cap - 4 : 0;
   if (m > groups) m = groups;
-  static_assert(kSmallest == kDecodeUnit, "tiles_max also counts the counting pass's units");
-  uint64_t t = (m + kSmallest - 1) / kSmallest;
+  uint64_t t = (m + kDecodeUnit - 1) / kDecodeUnit;
   return (uint32_t)(t < 1 ? 1 : t);
 }
 

@@ -94,7 +94,8 @@ struct BatchTensor {
   uint64_t cap;          // slot size = 4 + ceil(n/5)
   uint32_t q_tile_begin, q_tiles;  // compress tiles (global numbering)
   uint32_t q_chunk_begin;          // 32-tile chunks of the deferred placement
-  uint32_t d_tile_begin, d_tiles;  // decode tiles (global numbering, upper bound)
+  uint32_t d_tile_begin, d_tiles;  // decode 512-byte units (global numbering, upper
+                                   // bound of the tiles of either mode)
   uint32_t d_chunk_begin, d_chunks;  // 32-unit chunks of the counting pass (same)
   uint32_t vec_q;        // x and err 16-byte aligned
   uint32_t vec_y;        // y 16-byte aligned
@@ -184,7 +185,8 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
 int occupancy_quant(bool vec);
 
 // Decode scratch per stream: decode_scratch_words(tiles) u64 words, where
-// tiles = decode_tiles_max counts 512-byte payload units (the smallest tile).
+// tiles = decode_tiles_max counts 512-byte payload units (every tile is a
+// whole number of units).
 // Look-back path: status[tiles] (u64) then the ticket (u64 slot); both must
 // be zero before the launch.  Deferred-prefix path (decode_deferred): the
 // units' group counts (u32), the 32-unit chunks' counts (u64), then the
