@@ -42,7 +42,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--log2n", type=int, default=28, help="tensor size 2^k (default 28)")
-    p.add_argument("--e2e-steps", type=int, default=3)
+    p.add_argument("--e2e-steps", type=int, default=8)
     p.add_argument("--cpu-baseline-log2n", type=int, default=26)
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -413,57 +413,85 @@ def run_ours(args, rank, world, local):
 
 
 def run_e2e(args, tlc, torch, dev, x_h, n, cap, world):
-    """Same step through the public API with host buffers: pinned host x and
-    err copied in, stream, err and y copied out, every step."""
+    """The step through the public API with host buffers.  Every step copies
+    its gradient x in from pinned host memory, compresses it (the error
+    buffer stays on the device: it is the codec's state, like a model's
+    weights), decompresses and accumulates, and copies the stream buffer
+    (its capacity and the length word) and the decoded y out to pinned host
+    memory.  Two buffer sets and three streams (copy-in, compute, copy-out)
+    let step i's copy-out overlap step i+1's copy-in; a step's compute waits
+    for its own copy-in, and a buffer is refilled only after its last
+    reader is done."""
     import torch.distributed as dist
 
     from gradient_traffic_compression_b200.exchange import max_over_ranks
     xh = torch.from_numpy(x_h).pin_memory()
-    eh = torch.zeros(n, dtype=torch.float32).pin_memory()
-    yh = torch.empty(n, dtype=torch.float32).pin_memory()
-    sh = torch.empty(cap, dtype=torch.uint8).pin_memory()
-    x = torch.empty(n, dtype=torch.float32, device=dev)
-    err = torch.empty(n, dtype=torch.float32, device=dev)
-    out = torch.empty(cap, dtype=torch.uint8, device=dev)
-    out_len = torch.zeros(1, dtype=torch.int64, device=dev)
-    y = torch.empty(n, dtype=torch.float32, device=dev)
+    yh = [torch.empty(n, dtype=torch.float32).pin_memory() for _ in range(2)]
+    sh = [torch.empty(cap, dtype=torch.uint8).pin_memory() for _ in range(2)]
+    lh = [torch.empty(1, dtype=torch.int64).pin_memory() for _ in range(2)]
+    xd = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(2)]
+    yd = [torch.empty(n, dtype=torch.float32, device=dev) for _ in range(2)]
+    od = [torch.empty(cap, dtype=torch.uint8, device=dev) for _ in range(2)]
+    ld = [torch.zeros(1, dtype=torch.int64, device=dev) for _ in range(2)]
+    err = torch.zeros(n, dtype=torch.float32, device=dev)
     acc = torch.zeros(n, dtype=torch.float32, device=dev)
     st = torch.zeros(1, dtype=torch.int32, device=dev)
-    d2h = [0]
+    s_c = torch.cuda.current_stream(dev)
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_c = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def step():
-        x.copy_(xh, non_blocking=True)
-        err.copy_(eh, non_blocking=True)
-        tlc.tlc_compress(x, S_PARAM, err, out, out_len, st)
-        L = int(out_len.item())
-        sh[:L].copy_(out[:L], non_blocking=True)
-        eh.copy_(err, non_blocking=True)
-        tlc.tlc_decompress(out, n, y, in_len=out_len, in_cap=cap, dev_status=st)
-        tlc.tlc_decompress_accumulate([out], n, acc, in_lens=out_len, in_caps=[cap],
-                                      dev_status=st)
-        yh.copy_(y, non_blocking=True)
-        torch.cuda.synchronize()
-        d2h[0] = L + 8 * n
+    def step(i):
+        b = i % 2
+        s_in.wait_event(ev_c[b])            # step i-2 no longer reads xd[b]
+        with torch.cuda.stream(s_in):
+            xd[b].copy_(xh, non_blocking=True)
+        ev_in[b].record(s_in)
+        s_c.wait_event(ev_in[b])
+        s_c.wait_event(ev_out[b])           # step i-2's outputs are out
+        tlc.tlc_compress(xd[b], S_PARAM, err, od[b], ld[b], st, s_c)
+        tlc.tlc_decompress(od[b], n, yd[b], in_len=ld[b], in_cap=cap, dev_status=st, stream=s_c)
+        tlc.tlc_decompress_accumulate([od[b]], n, acc, in_lens=ld[b], in_caps=[cap],
+                                      dev_status=st, stream=s_c)
+        ev_c[b].record(s_c)
+        s_out.wait_event(ev_c[b])
+        with torch.cuda.stream(s_out):
+            sh[b].copy_(od[b], non_blocking=True)
+            lh[b].copy_(ld[b], non_blocking=True)
+            yh[b].copy_(yd[b], non_blocking=True)
+        ev_out[b].record(s_out)
 
-    step()
+    for i in range(2):
+        step(i)
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    t0.record()
-    for _ in range(args.e2e_steps):
-        step()
-    t1.record()
+    t0.record(s_c)
+    s_in.wait_stream(s_c)
+    s_out.wait_stream(s_c)
+    for i in range(args.e2e_steps):
+        step(i)
+    s_c.wait_stream(s_in)
+    s_c.wait_stream(s_out)
+    t1.record(s_c)
     torch.cuda.synchronize()
     ms = max_over_ranks([t0.elapsed_time(t1) / args.e2e_steps], device=dev)[0]
     if int(st.item()) != 0:
         raise RuntimeError(f"device status {int(st.item())} in the e2e run")
+    L = int(lh[(args.e2e_steps - 1) % 2].item())
+    if L < 4 or L > cap:
+        raise RuntimeError(f"e2e stream length {L} out of range")
     return {"value": round(world * 4 * n / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
             "ms_per_step": round(ms, 3), "steps": args.e2e_steps,
-            "h2d_bytes_per_step": 8 * n, "d2h_bytes_per_step": d2h[0],
-            "path": "pinned host x, err -> device; tlc_compress; stream + err -> host; "
-                    "tlc_decompress; tlc_decompress_accumulate; y -> host"}
+            "h2d_bytes_per_step": 4 * n, "d2h_bytes_per_step": cap + 8 + 4 * n,
+            "path": "pinned host x -> device; tlc_compress (error buffer resident); "
+                    "tlc_decompress; tlc_decompress_accumulate; stream buffer, length and "
+                    "y -> pinned host; copy-in, compute and copy-out on three streams, "
+                    "two buffer sets"}
 
 
 # ------------------------------------------- tensor sets and K streams ----

@@ -14,6 +14,25 @@ node of B200s this is:
    aggregation buffer (``tlc_decompress_accumulate``, K = world), so all
    ranks hold bit-identical sums.
 
+The page's workers push compressed gradients to parameter servers, which
+aggregate them and send back the compressed model delta ("Proposed method":
+3LC compresses both gradients and model deltas).  ``exchange_step_sharded``
+is that two-sided form over NCCL with no server processes: rank r serves
+shard r of every tensor.
+
+1. every rank compresses each shard of its gradient with its own error
+   buffer (one stream per shard);
+2. all-to-all of those streams (lengths first, then slots as long as the
+   longest), so rank r receives every rank's stream for shard r;
+3. rank r adds them in rank order (``tlc_decompress_accumulate``), then
+   compresses that aggregate, the shard's model delta, with its own
+   server-side error buffer;
+4. the delta streams are all-gathered and every rank decodes all shards,
+   so every rank holds the same model delta.
+
+About 2 * n / 5 stream bytes per rank cross NVLink at most, against
+world * n / 5 for the all-gather form.
+
 The transport is torch.distributed (NCCL on GPUs; gloo works for host
 tensors).  The codec steps run in libtlc.so; nothing here computes on the
 values.
@@ -76,3 +95,104 @@ def exchange_step(x, s, err, acc, group=None, dev_status=None):
     rows = [slots[r].contiguous() for r in range(slots.shape[0])]
     tlc.tlc_decompress_accumulate(rows, n, acc, in_caps=lengths, dev_status=st)
     return lengths, st
+
+
+def shard_bounds(n, world):
+    """Contiguous shards of n values over world ranks: rank r serves values
+    [b[r], b[r+1]); the first n % world shards hold one value more."""
+    base, extra = divmod(int(n), int(world))
+    b = [0]
+    for r in range(world):
+        b.append(b[-1] + base + (1 if r < extra else 0))
+    return b
+
+
+def alltoall_streams(streams, lengths, group=None):
+    """All-to-all of variable-length byte streams.
+
+    streams[d] holds, in its first lengths[d] bytes, the stream this rank
+    sends to rank d (uint8 tensors on the backend's device).  Returns
+    (slots, lengths_in): slots is a [world, width] uint8 tensor whose row s
+    holds rank s's stream for this rank in its first lengths_in[s] bytes.
+    Three collectives: the lengths (all-to-all), the common slot width (the
+    longest stream anywhere, an all-reduce), then the slots (all-to-all)."""
+    world = dist.get_world_size(group)
+    dev = streams[0].device
+    mine = torch.tensor([int(v) for v in lengths], dtype=torch.int64, device=dev)
+    lens_in = torch.empty_like(mine)
+    dist.all_to_all_single(lens_in, mine, group=group)
+    width_t = torch.tensor([max(int(mine.max().item()), 1)], dtype=torch.int64, device=dev)
+    dist.all_reduce(width_t, op=dist.ReduceOp.MAX, group=group)
+    width = int(width_t.item())
+    send = torch.zeros(world * width, dtype=torch.uint8, device=dev)
+    for d in range(world):
+        L = int(lengths[d])
+        send[d * width: d * width + L].copy_(streams[d][:L])
+    recv = torch.empty_like(send)
+    dist.all_to_all_single(recv, send, group=group)
+    return recv.view(world, width), [int(v) for v in lens_in.tolist()]
+
+
+class CudaCodec:
+    """The codec steps of the sharded exchange through libtlc.so (CUDA
+    tensors).  Each method enqueues work on the current stream; a length is
+    read back to the host only where the transport needs it."""
+
+    def __init__(self):
+        from . import tlc
+        self.tlc = tlc
+
+    def compress(self, x, s, err, dev_status):
+        t = self.tlc
+        out = torch.empty(t.tlc_compress_bound(x.numel()), dtype=torch.uint8, device=x.device)
+        out_len = torch.zeros(1, dtype=torch.int64, device=x.device)
+        t.tlc_compress(x, s, err, out, out_len, dev_status)
+        length = int(out_len.item())
+        if length == 0:
+            raise RuntimeError(f"compression failed (status {int(dev_status.item())})")
+        return out, length
+
+    def accumulate(self, streams, lengths, n, acc, dev_status):
+        rows = [st.contiguous() for st in streams]
+        self.tlc.tlc_decompress_accumulate(rows, n, acc, in_caps=[int(v) for v in lengths],
+                                           dev_status=dev_status)
+
+    def decompress(self, stream, length, n, y, dev_status):
+        self.tlc.tlc_decompress(stream.contiguous(), n, y, in_cap=int(length),
+                                dev_status=dev_status)
+
+
+def exchange_step_sharded(x, s, err, server_err, y, group=None, codec=None, dev_status=None):
+    """One two-sided step (see the module docstring).
+
+    x: this rank's gradient (n values); err: its worker-side error buffer
+    (n values, updated); server_err: the error buffer of the shard this rank
+    serves (shard_bounds(n, world)[r + 1] - [r] values, updated); y: receives
+    the model delta (n values, the same on every rank).  codec defaults to
+    CudaCodec.  Returns (lengths sent per shard, delta stream lengths)."""
+    codec = codec if codec is not None else CudaCodec()
+    world = dist.get_world_size(group)
+    rank = dist.get_rank(group)
+    n = x.numel()
+    if n < world:
+        raise ValueError(f"{n} values cannot be shared among {world} ranks")
+    b = shard_bounds(n, world)
+    if server_err.numel() != b[rank + 1] - b[rank]:
+        raise ValueError("server_err must hold this rank's shard")
+    st = dev_status if dev_status is not None else torch.zeros(
+        1, dtype=torch.int32, device=x.device)
+    # 1. worker side: one stream per shard
+    ups = [codec.compress(x[b[d]:b[d + 1]], s, err[b[d]:b[d + 1]], st) for d in range(world)]
+    # 2. to the shard's server
+    slots, lens_in = alltoall_streams([u[0] for u in ups], [u[1] for u in ups], group)
+    # 3. server side: aggregate in rank order, compress the model delta
+    m = b[rank + 1] - b[rank]
+    agg = torch.zeros(m, dtype=torch.float32, device=x.device)
+    codec.accumulate([slots[r, :lens_in[r]] for r in range(world)], lens_in, m, agg, st)
+    down, down_len = codec.compress(agg, s, server_err, st)
+    # 4. every shard's delta to every rank
+    rows, lens_down = allgather_streams(down, down_len, group)
+    for d in range(world):
+        codec.decompress(rows[d, :lens_down[d]], lens_down[d], b[d + 1] - b[d],
+                         y[b[d]:b[d + 1]], st)
+    return [u[1] for u in ups], lens_down

@@ -93,3 +93,122 @@ def test_two_gloo_ranks_exchange_and_time():
         x[synth.bernoulli(synth.key_for(600 + rank, 3), n, 0.5 + 0.2 * rank)] = 0.0
         _, st, _ = oracle.compress(x, 1.75, np.zeros(n, np.float32))
         assert r0[3][rank] == st.tolist()
+
+
+class _OracleCodec:
+    """The codec steps of exchange_step_sharded on host tensors through the
+    CPU oracle (test code only; on GPUs the CUDA codec runs them)."""
+
+    def compress(self, x, s, err, dev_status):
+        import torch
+
+        import oracle
+        rc, st, e2 = oracle.compress(x.numpy(), s, err.numpy())
+        assert rc == 0
+        err.copy_(torch.from_numpy(e2))
+        return torch.from_numpy(st), int(st.size)
+
+    def accumulate(self, streams, lengths, n, acc, dev_status):
+        import torch
+
+        import oracle
+        rc, a = oracle.decompress_accumulate([t[:L].numpy() for t, L in zip(streams, lengths)],
+                                             n, acc.numpy())
+        assert rc == 0
+        acc.copy_(torch.from_numpy(a))
+
+    def decompress(self, stream, length, n, y, dev_status):
+        import torch
+
+        import oracle
+        rc, v = oracle.decompress(stream[:length].numpy(), n)
+        assert rc == 0
+        y.copy_(torch.from_numpy(v))
+
+
+def _sharded_inputs(rank, n):
+    import synth
+    x = synth.normal(synth.key_for(700 + rank, 0), n, 1e-3)
+    x[synth.bernoulli(synth.key_for(700 + rank, 3), n, 0.4 + 0.2 * rank)] = 0.0
+    return x
+
+
+def _sharded_worker(rank, world, port, n, steps, q):
+    try:
+        sys.path.insert(0, ROOT)
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        from gradient_traffic_compression_b200.exchange import (exchange_step_sharded,
+                                                                shard_bounds)
+        dist.init_process_group("gloo", rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=60))
+        b = shard_bounds(n, world)
+        x = torch.from_numpy(_sharded_inputs(rank, n))
+        err = torch.zeros(n, dtype=torch.float32)
+        server_err = torch.zeros(b[rank + 1] - b[rank], dtype=torch.float32)
+        ys = []
+        for _ in range(steps):
+            y = torch.zeros(n, dtype=torch.float32)
+            up, down = exchange_step_sharded(x, 1.5, err, server_err, y, codec=_OracleCodec(),
+                                             dev_status=torch.zeros(1, dtype=torch.int32))
+            ys.append(y.numpy().tobytes())
+        q.put((rank, ys, up, down))
+        dist.barrier()
+        dist.destroy_process_group()
+    except Exception as e:  # report to the parent instead of hanging it
+        q.put((rank, "error", repr(e)))
+
+
+@pytest.mark.timeout(240)
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_exchange_matches_a_single_process_model(world):
+    n, steps = 20_011, 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sharded_worker, args=(r, world, port, n, steps, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    results = {}
+    for _ in range(world):
+        item = q.get(timeout=200)
+        assert item[1] != "error", item
+        results[item[0]] = item
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # every rank holds the same model delta at every step
+    for r in range(1, world):
+        assert results[r][1] == results[0][1]
+    # the same computation in one process: per shard, every worker's stream,
+    # their rank-ordered sum, the server's compression of it, its decoding
+    sys.path.insert(0, ROOT)
+    import oracle
+    from gradient_traffic_compression_b200.exchange import shard_bounds
+    b = shard_bounds(n, world)
+    xs = [_sharded_inputs(r, n) for r in range(world)]
+    errs = [np.zeros(n, np.float32) for _ in range(world)]
+    serrs = [np.zeros(b[d + 1] - b[d], np.float32) for d in range(world)]
+    for k in range(steps):
+        y = np.zeros(n, np.float32)
+        for d in range(world):
+            lo, hi = b[d], b[d + 1]
+            streams = []
+            for r in range(world):
+                rc, st, e2 = oracle.compress(xs[r][lo:hi], 1.5, errs[r][lo:hi])
+                errs[r][lo:hi] = e2
+                streams.append(st)
+                if k == steps - 1:
+                    assert results[r][2][d] == st.size       # bytes sent for shard d
+            _, agg = oracle.decompress_accumulate(streams, hi - lo, np.zeros(hi - lo, np.float32))
+            rc, sd, serrs[d] = oracle.compress(agg, 1.5, serrs[d])
+            _, y[lo:hi] = oracle.decompress(sd, hi - lo)
+            if k == steps - 1:
+                assert results[0][3][d] == sd.size
+        assert results[0][1][k] == y.tobytes(), f"step {k}"
