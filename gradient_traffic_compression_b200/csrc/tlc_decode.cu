@@ -152,17 +152,17 @@ struct DecodeJob {
 };
 
 // Deferred prefixes: the first group index of the tile that starts at
-// payload unit `unit`, from the counts that k_decode_count wrote (the chunks
-// before the unit's chunk, then the units before it in its chunk), by one
-// whole warp.  No wait.
-__device__ __forceinline__ uint64_t prefix_from_counts(const uint32_t *ecount,
-                                                       const uint64_t *csum, uint32_t unit) {
-  const int lane = threadIdx.x & 31;
+// payload unit `unit` is the sum of the counts that k_decode_count wrote for
+// the chunks before the unit's chunk and for the units before it in its
+// chunk.  Every thread of the block sums a strided share; the result is this
+// warp's partial sum (in every lane).  No wait.
+__device__ __forceinline__ uint64_t prefix_share(const uint32_t *ecount, const uint64_t *csum,
+                                                 uint32_t unit) {
   const uint32_t c = unit / kDecodeChunkUnits;
   uint64_t s = 0;
-  for (uint32_t i = lane; i < c; i += kWarp) s += csum[i];
+  for (uint32_t i = threadIdx.x; i < c; i += kDThreads) s += csum[i];
   const uint32_t t0 = c * kDecodeChunkUnits;
-  if (t0 + lane < unit) s += ecount[t0 + lane];
+  if (threadIdx.x < kDecodeChunkUnits && t0 + threadIdx.x < unit) s += ecount[t0 + threadIdx.x];
   return warp_sum_u64(s);
 }
 
@@ -170,6 +170,7 @@ struct DecodeSmem {
   uint16_t lut[256];       // base-3 digits of every quartic byte
   uint32_t scan[kDThreads / kWarp + 1];
   uint64_t o;
+  uint64_t part[kDThreads / kWarp];  // per-warp partial prefixes (counting pass)
 };
 
 // Validate a stream (length and header) and return its payload length and
@@ -244,18 +245,25 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
   const bool any_lit = __syncthreads_or(mine_lit) != 0;
   const bool expand = any_lit && (kMode == kWrite || E <= 4u * (uint32_t)kDTile);
 
-  // ---- look-back (warp 0); the other warps pre-fill zero groups ----------
-  if (warp == 0) {
-    uint64_t O;
-    if (kDeferred) {
-      static_assert(kDTile % kDecodeUnit == 0 && kDecodeChunkUnits % (kDTile / kDecodeUnit) == 0,
-                    "tiles are whole units and never straddle a chunk");
-      O = prefix_from_counts(j.ecount, j.csum, u * (uint32_t)(kDTile / kDecodeUnit));
-    } else {
-      bool timed_out = false;
-      O = lookback_sum(j.status, u, E, max_polls, timed_out);
-      if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(dev_status, TLC_ERR_TIMEOUT);
+  // ---- the tile's first group index ---------------------------------------
+  // Counting pass: every thread sums a strided share of the counts before
+  // the tile, then all threads pre-fill the zero groups.  Look-back: warp 0
+  // looks back while the other warps pre-fill.
+  if (kDeferred) {
+    static_assert(kDTile % kDecodeUnit == 0 && kDecodeChunkUnits % (kDTile / kDecodeUnit) == 0,
+                  "tiles are whole units and never straddle a chunk");
+    const uint64_t p = prefix_share(j.ecount, j.csum, u * (uint32_t)(kDTile / kDecodeUnit));
+    if (lane == 0) sm.part[warp] = p;
+    if (expand) {
+      const uint32_t words = (E + 15) / 16;
+      for (uint32_t w = threadIdx.x; w < words; w += kDThreads)
+        reinterpret_cast<uint4 *>(grp_s)[w] =
+            make_uint4(0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u);
     }
+  } else if (warp == 0) {
+    bool timed_out = false;
+    const uint64_t O = lookback_sum(j.status, u, E, max_polls, timed_out);
+    if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(dev_status, TLC_ERR_TIMEOUT);
     if (lane == 0) sm.o = O;
   } else if (expand) {
     const uint32_t words = (E + 15) / 16;
@@ -264,7 +272,14 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
           make_uint4(0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u);
   }
   __syncthreads();
-  const uint64_t O = sm.o;
+  uint64_t O;
+  if (kDeferred) {
+    O = 0;
+#pragma unroll
+    for (int w = 0; w < kDThreads / kWarp; ++w) O += sm.part[w];
+  } else {
+    O = sm.o;
+  }
   if (threadIdx.x == 0) {
     const bool last = (u == j.n_tiles - 1);
     if (O + E > j.groups || (last && O + E != j.groups)) report(dev_status, TLC_ERR_CORRUPT);
