@@ -239,7 +239,9 @@ def test_batch_deferred_placement_many_tensors(g):
         errs.append(e)
     xs[7] = xs[7].copy()
     xs[7][xs[7].size // 2] = np.inf
-    b = Batch(g, xs, errs, with_y=False)
+    # every third tensor 4- but not 16-byte aligned (the scalar quantize path)
+    b = Batch(g, xs, errs, offsets=[(i % 3 == 1) * (1 + i % 2) for i in range(len(xs))],
+              with_y=False)
     for step in range(2):
         b.plan.compress(1.5, b.arena, b.lens, b.status)
         torch.cuda.synchronize()

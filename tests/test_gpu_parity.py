@@ -56,12 +56,14 @@ def _check_f32_guards(buf, n, offset=0):
     assert np.all(raw[GUARD + offset + n:] == 0x7FA5A5A5)
 
 
-def gpu_compress(g, x, s, err, offset=0):
-    """(status, stream, err', out_len) through tlc_compress."""
+def gpu_compress(g, x, s, err, offset=0, out_offset=0):
+    """(status, stream, err', out_len) through tlc_compress; out_offset > 0
+    shifts the stream buffer by that many bytes (any alignment)."""
     n = x.size
     xt, et = _dev_f32(x, offset), _dev_f32(err, offset)
     cap = g.tlc_compress_bound(n)
-    obuf = torch.full((cap + 2 * GUARD,), CANARY, dtype=torch.uint8, device="cuda")
+    obuf = torch.full((cap + 2 * GUARD + out_offset,), CANARY, dtype=torch.uint8, device="cuda")
+    obuf = obuf[out_offset:]
     out = obuf[GUARD:GUARD + cap]
     out_len = torch.zeros(1, dtype=torch.int64, device="cuda")
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -75,11 +77,12 @@ def gpu_compress(g, x, s, err, offset=0):
     return int(st.item()), ob[GUARD:GUARD + L].copy(), et.cpu().numpy(), L
 
 
-def gpu_decompress(g, stream, n, offset=0, in_len=None, cap=None):
+def gpu_decompress(g, stream, n, offset=0, in_len=None, cap=None, in_offset=0):
     buf, y = _guarded_f32(n, offset)
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
     cap = stream.size if cap is None else cap
-    sb = torch.full((max(cap, 1),), CANARY, dtype=torch.uint8, device="cuda")
+    sb = torch.full((max(cap, 1) + in_offset,), CANARY, dtype=torch.uint8, device="cuda")
+    sb = sb[in_offset:]
     if stream.size:
         sb[:stream.size].copy_(torch.from_numpy(stream))
     lt = None
@@ -109,9 +112,9 @@ def gpu_accumulate(g, streams, n, acc0, offset=0, device_lens=False):
     return int(st.item()), acc.cpu().numpy()
 
 
-def assert_compress_parity(g, x, s, err, offset=0):
+def assert_compress_parity(g, x, s, err, offset=0, out_offset=0):
     rc_o, st_o, e_o = oracle.compress(x, s, err)
-    rc_g, st_g, e_g, L = gpu_compress(g, x, s, err, offset)
+    rc_g, st_g, e_g, L = gpu_compress(g, x, s, err, offset, out_offset)
     assert rc_g == rc_o
     assert L == st_o.size
     if not np.array_equal(st_g, st_o):
@@ -123,9 +126,9 @@ def assert_compress_parity(g, x, s, err, offset=0):
     return st_o, e_o
 
 
-def assert_roundtrip_parity(g, stream, n, offset=0):
+def assert_roundtrip_parity(g, stream, n, offset=0, in_offset=0, cap=None, in_len=None):
     rc_o, y_o = oracle.decompress(stream, n)
-    rc_g, y_g = gpu_decompress(g, stream, n, offset)
+    rc_g, y_g = gpu_decompress(g, stream, n, offset, in_len=in_len, cap=cap, in_offset=in_offset)
     assert rc_g == rc_o
     d = np.flatnonzero(bits(y_g) != bits(y_o))
     assert d.size == 0, f"y differs at {d[:8]}"
@@ -608,3 +611,29 @@ def test_decode_counting_pass_corrupt(g):
     assert rc == 3
     # the context is still usable, and a good stream still decodes
     assert_roundtrip_parity(g, st, n)
+
+
+# ---- alignment on the wait-free paths ------------------------------------
+
+@pytest.mark.parametrize("offset,out_offset", [(1, 0), (3, 5), (0, 1), (0, 7), (2, 13)])
+def test_deferred_placement_any_alignment(g, offset, out_offset):
+    # unaligned x / err (the scalar quantize path) and stream buffers at odd
+    # byte offsets (the placement kernel's head, 16-byte body and tail)
+    n = DEFER_TILES * TILE_VALUES + 3 * 641
+    x, err, s = mixed_case(6000 + 7 * offset + out_offset, n, zero_frac=0.6)
+    st, _ = assert_compress_parity(g, x, s, err, offset=offset, out_offset=out_offset)
+    assert_roundtrip_parity(g, st, n, offset=offset)
+
+
+@pytest.mark.parametrize("in_offset", [1, 2, 3, 6])
+def test_decode_counting_pass_unaligned_payload(g, in_offset):
+    # a payload that does not start on a 4-byte boundary (the counting pass's
+    # byte-wise loads) in a buffer large enough for the counting pass
+    n = 5 * DECODE_DEFER_BYTES + 4321
+    x, err, s = mixed_case(6100 + in_offset, n, zero_frac=0.8)
+    rc, st, _ = oracle.compress(x, s, err)
+    assert rc == 0
+    cap = g.tlc_compress_bound(n)
+    assert_roundtrip_parity(g, st, n, in_offset=in_offset, cap=cap, in_len=st.size)
+    dense, nd = _dense_stream(in_offset, DECODE_DEFER_BYTES + 999)
+    assert_roundtrip_parity(g, dense, nd, offset=1, in_offset=in_offset)
