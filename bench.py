@@ -47,6 +47,8 @@ def parse_args():
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--graph", action="store_true",
+                   help="configs 2, 4, 5: replay each step from a CUDA graph of its calls")
     p.add_argument("--per-tensor", action="store_true",
                    help="configs 2/4: one C-ABI call per tensor instead of a plan")
     p.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4, 5],
@@ -523,7 +525,8 @@ def run_config_set(args, rank, world, local):
     outs = [torch.empty(c, dtype=torch.uint8, device=dev) for c in caps]
     lens = torch.zeros(len(ns), dtype=torch.int64, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    stream = torch.cuda.current_stream()
+    strm = [torch.cuda.current_stream()]   # the stream the legs run on
+    stream = strm[0]
     if args.config == 5:
         acc = torch.zeros(ns[0], dtype=torch.float32, device=dev)
         ys, accs = None, None
@@ -539,29 +542,29 @@ def run_config_set(args, rank, world, local):
 
     def legs():
         if use_plan:
-            plan.compress(s, arena, lens, status, stream)
+            plan.compress(s, arena, lens, status, strm[0])
             yield
-            plan.decompress(arena, lens, accumulate=False, dev_status=status, stream=stream)
+            plan.decompress(arena, lens, accumulate=False, dev_status=status, stream=strm[0])
             yield
-            acc_plan.decompress(arena, lens, accumulate=True, dev_status=status, stream=stream)
+            acc_plan.decompress(arena, lens, accumulate=True, dev_status=status, stream=strm[0])
             yield
             return
         for i in range(len(ns)):
-            tlc.tlc_compress(xs[i], s, errs[i], outs[i], lens[i:i + 1], status, stream)
+            tlc.tlc_compress(xs[i], s, errs[i], outs[i], lens[i:i + 1], status, strm[0])
         yield
         if args.config == 5:
             yield
             tlc.tlc_decompress_accumulate(outs, ns[0], acc, in_lens=lens, in_caps=caps,
-                                          dev_status=status, stream=stream)
+                                          dev_status=status, stream=strm[0])
         else:
             for i in range(len(ns)):
                 tlc.tlc_decompress(outs[i], ns[i], ys[i], in_len=lens[i:i + 1], in_cap=caps[i],
-                                   dev_status=status, stream=stream)
+                                   dev_status=status, stream=strm[0])
             yield
             for i in range(len(ns)):
                 tlc.tlc_decompress_accumulate([outs[i]], ns[i], accs[i], in_lens=lens[i:i + 1],
                                               in_caps=[caps[i]], dev_status=status,
-                                              stream=stream)
+                                              stream=strm[0])
         yield
 
     for _ in range(max(3, args.warmup)):
@@ -569,6 +572,24 @@ def run_config_set(args, rank, world, local):
             pass
     torch.cuda.synchronize()
     steps = max(1, min(args.steps, 50))
+    graph = None
+    if args.graph:
+        # one step captured as a CUDA graph, replayed in the timed region;
+        # its launches are counted while it is captured
+        tlc.tlc_kernel_timing_kinds([])
+        tlc.tlc_kernel_timing(True)
+        graph = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(dev)
+        cs.wait_stream(stream)
+        strm[0] = cs
+        with torch.cuda.graph(graph, stream=cs):
+            for _ in legs():
+                pass
+        strm[0] = stream
+        tlc.tlc_kernel_timing(False)
+        per_step = tlc.tlc_kernel_timing_read()
+        graph.replay()
+        torch.cuda.synchronize()
     # timed region: whole steps between two events; launches counted, no
     # per-kernel events
     if world > 1:
@@ -580,12 +601,17 @@ def run_config_set(args, rank, world, local):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for _ in range(steps):
-        for _ in legs():
-            pass
+        if graph is not None:
+            graph.replay()
+        else:
+            for _ in legs():
+                pass
     t1.record(stream)
     torch.cuda.synchronize()
     tlc.tlc_kernel_timing(False)
     launches = tlc.tlc_kernel_timing_read()
+    if graph is not None:
+        launches = {k: (v[0] * steps, 0.0) for k, v in per_step.items()}
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())}")
     step_ms = max_over_ranks([t0.elapsed_time(t1) / steps], device=dev)[0]
@@ -613,7 +639,9 @@ def run_config_set(args, rank, world, local):
         "config": {"workload": cfg["name"], "tensors": len(ns), "values": total, "s": s,
                    "calls": ("one plan call per leg (tlc_compress_batch / "
                              "tlc_decompress_batch)" if use_plan else
-                             "one C-ABI call per tensor and leg")},
+                             "one C-ABI call per tensor and leg")
+                   + ("; each step replayed from a CUDA graph of those calls" if args.graph
+                      else "")},
         "legs": {"compress_ms": round(legs_ms[0], 4),
                  "compress_gbs": round(in_bytes / (legs_ms[0] * 1e-3) / 1e9, 1),
                  "stream_bytes": L, "bits_per_value": round(8 * L / total, 5)},
