@@ -754,7 +754,9 @@ def traffic_for(kernel, n):
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
-    from gradient_traffic_compression_b200.build import source_digest
+    from gradient_traffic_compression_b200.build import KERNEL_SOURCES, source_digest
+    if kernel not in KERNEL_SOURCES:
+        return None
     digest = source_digest(kernel)
     with open(path) as f:
         for line in f:
