@@ -645,6 +645,7 @@ def run_config_set(args, rank, world, local):
         "legs": {"compress_ms": round(legs_ms[0], 4),
                  "compress_gbs": round(in_bytes / (legs_ms[0] * 1e-3) / 1e9, 1),
                  "stream_bytes": L, "bits_per_value": round(8 * L / total, 5)},
+        "per_tensor_us": round(1e3 * step_ms / len(ns), 3),
         "kernels": {k: {"launches": v[0], "avg_ms": round(v[1] / max(v[0], 1), 5)}
                     for k, v in kern.items() if v[0]},
         "gpu_launches": int(sum(v[0] for v in launches.values())),
