@@ -278,12 +278,13 @@ __device__ __forceinline__ ZScan zshfl_up(const ZScan &v, int d) {
   return r;
 }
 
-// Summary of a chunk of kPlaceTiles tiles in a status word (A, R < 2^20).
+// The summary of a chunk of kPlaceTiles tiles in 64 bits (A, R < 2^20), as
+// the deferred path stores it per chunk.
 constexpr int kPlaceTiles = 32;
 static_assert((uint64_t)kPlaceTiles * kTileGroups < (1u << 20), "chunk A and R fit in 20 bits");
 struct ChunkCodec {
   __device__ static uint64_t pack(const ZAgg &a) {
-    return kFlagAgg | (uint64_t)a.A | ((uint64_t)a.R << 20) | ((uint64_t)a.tc << 40) |
+    return (uint64_t)a.A | ((uint64_t)a.R << 20) | ((uint64_t)a.tc << 40) |
            ((uint64_t)a.all << 44);
   }
   __device__ static ZAgg unpack(uint64_t w) {

@@ -22,11 +22,12 @@
 // For streams whose capacity holds 16384 or more 512-byte units (8 MiB), a
 // counting kernel, k_decode_count, first writes the group count of every
 // unit and of every 32-unit chunk; each tile then sums the counts before it
-// instead of looking back.  No tile waits on another, which measured
-// 0.789 -> 0.480 ms (dense output) and 0.629 -> 0.592 ms (accumulate) on a
-// dense 2^28-value stream, and 0.189 -> 0.178 / 0.040 -> 0.026 ms on the
-// sparse config-3 stream, for about 0.010 ms per counting launch.  Below
-// that size the extra launch costs more than the look-back on sparse streams.
+// (every thread a strided share) instead of looking back.  No tile waits on
+// another, which measured 0.789 -> 0.459 ms (dense output) and 0.629 ->
+// 0.505 ms (accumulate) on a dense 2^28-value stream, and 0.189 -> 0.178 /
+// 0.040 -> 0.026 ms on the sparse config-3 stream, for about 0.011 ms per
+// counting launch.  Below that size the extra launch costs more than the
+// look-back on sparse streams.
 // Every write is clamped to the ceil(n/5) groups of the tensor; a stream that
 // does not expand to exactly that many groups is reported as corrupt.
 #include "tlc_device.cuh"
