@@ -10,6 +10,7 @@
 
 #include "../../include/tlc.h"
 #include "tlc_internal.h"
+#include <nvtx3/nvToolsExt.h>
 
 namespace {
 
@@ -76,6 +77,15 @@ bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
 bool n_ok(size_t n) { return n >= 1 && n < (size_t(1) << 32); }
 
 size_t groups_of(size_t n) { return (n + 4) / 5; }
+
+// A named NVTX range around each call that enqueues work, so profilers and
+// timeline tools show the calls around their kernels (no cost without one).
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange &) = delete;
+  NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // Stream-ordered scratch from the library's pool.
 cudaError_t scratch_alloc(const tlc::DeviceInfo &dev, size_t bytes, void **p, cudaStream_t st) {
@@ -208,6 +218,7 @@ void tlc_set_wait_limit(uint32_t max_polls) {
 tlc_status tlc_compress(const float *x, size_t n, float s, float *err, uint8_t *out,
                         size_t out_cap, uint64_t *out_len, int32_t *dev_status,
                         tlc_stream_t stream) {
+  NvtxRange nvtx("tlc_compress");
   if (!x || !err || !out || !out_len || !n_ok(n)) return TLC_ERR_INVALID_ARG;
   if (!(s >= 1.0f && s < 2.0f)) return TLC_ERR_INVALID_ARG;  // also rejects NaN
   if (out_cap < tlc_compress_bound(n)) return TLC_ERR_INVALID_ARG;
@@ -240,6 +251,7 @@ static tlc_status check_stream_arg(const uint8_t *in, size_t cap, bool len_on_de
 
 tlc_status tlc_decompress(const uint8_t *in, const uint64_t *in_len, size_t in_cap, size_t n,
                           float *y, int32_t *dev_status, tlc_stream_t stream) {
+  NvtxRange nvtx("tlc_decompress");
   if (!y) return TLC_ERR_INVALID_ARG;
   tlc_status v = check_stream_arg(in, in_cap, in_len != nullptr, n);
   if (v != TLC_OK) return v;
@@ -267,6 +279,7 @@ tlc_status tlc_decompress(const uint8_t *in, const uint64_t *in_len, size_t in_c
 tlc_status tlc_decompress_accumulate(const uint8_t *const *ins, const uint64_t *in_lens,
                                      const size_t *in_caps, int k, size_t n, float *acc,
                                      int32_t *dev_status, tlc_stream_t stream) {
+  NvtxRange nvtx("tlc_decompress_accumulate");
   if (!ins || !in_caps || !acc || k < 1 || !n_ok(n)) return TLC_ERR_INVALID_ARG;
   for (int w = 0; w < k; ++w) {
     tlc_status v = check_stream_arg(ins[w], in_caps[w], in_lens != nullptr, n);
@@ -470,6 +483,7 @@ static const tlc::DeviceInfo *plan_device(tlc_plan plan) {
 
 tlc_status tlc_compress_batch(tlc_plan plan, float s, uint8_t *arena, uint64_t *out_lens,
                               int32_t *dev_status, tlc_stream_t stream) {
+  NvtxRange nvtx("tlc_compress_batch");
   if (!plan || !plan->has_inputs || !arena || !out_lens) return TLC_ERR_INVALID_ARG;
   if (!(s >= 1.0f && s < 2.0f)) return TLC_ERR_INVALID_ARG;
   const tlc::DeviceInfo *dev = plan_device(plan);
@@ -482,6 +496,7 @@ tlc_status tlc_compress_batch(tlc_plan plan, float s, uint8_t *arena, uint64_t *
 
 tlc_status tlc_decompress_batch(tlc_plan plan, const uint8_t *arena, const uint64_t *in_lens,
                                 int accumulate, int32_t *dev_status, tlc_stream_t stream) {
+  NvtxRange nvtx("tlc_decompress_batch");
   if (!plan || !plan->has_outputs || !arena || !in_lens) return TLC_ERR_INVALID_ARG;
   const tlc::DeviceInfo *dev = plan_device(plan);
   if (!dev) return TLC_ERR_INVALID_ARG;
