@@ -46,6 +46,9 @@ def parse_args():
     p.add_argument("--cpu-baseline-log2n", type=int, default=26)
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sweep", action="store_true",
+                   help="--impl reference: also time the oracle per direction over the "
+                        "config-3 sweep 2^20..2^24 and configs 1 and 5")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--graph", action="store_true",
                    help="configs 2, 4, 5: replay each step from a CUDA graph of its calls")
@@ -677,6 +680,38 @@ def oracle_step(oracle, x, n, acc):
     return st.size, acc
 
 
+def cpu_sweep():
+    """The CPU oracle per direction (median of 3 runs each, one core) over
+    the config-3 sweep 2^20..2^24 and on configs 1 and 5 (one of config 5's
+    streams, which is what one compress and one decompress see)."""
+    import numpy as np
+    import oracle
+    import synth
+    cases = [("config 3", 1 << k, 3, 1.9) for k in range(20, 25)]
+    cases += [("config 1", synth.CONFIGS[1]["n"], 1, synth.CONFIGS[1]["s"]),
+              ("config 5 (one stream)", synth.CONFIGS[5]["n"], 5, synth.CONFIGS[5]["s"])]
+    out = []
+    for name, n, cfg, s in cases:
+        x = synth.flat_tensor(cfg, n=n)
+        err = np.zeros(n, np.float32)
+        tc, td = [], []
+        for _ in range(3):
+            t0 = time.perf_counter()
+            rc, st, _ = oracle.compress(x, s, err)
+            t1 = time.perf_counter()
+            rc2, _ = oracle.decompress(st, n)
+            t2 = time.perf_counter()
+            if rc or rc2:
+                raise RuntimeError(f"oracle status {rc}/{rc2}")
+            tc.append(t1 - t0)
+            td.append(t2 - t1)
+        out.append({"workload": name, "n": int(n),
+                    "compress_gbs": round(4 * n / statistics.median(tc) / 1e9, 4),
+                    "decompress_gbs": round(4 * n / statistics.median(td) / 1e9, 4),
+                    "bits_per_value": round(8 * st.size / n, 4)})
+    return out
+
+
 def cpu_baseline(args):
     """The CPU oracle (single-threaded C, as it stands) on a bounded sample of
     the same workload: repeated compress + decompress + accumulate steps."""
@@ -743,7 +778,7 @@ def run_reference(args, rank, world):
                          "cpu": cpu_model()},
         "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "bits_per_value": round(8 * L / ns, 5),
-    }
+    } | ({"cpu_sweep": cpu_sweep()} if args.cpu_sweep else {})
 
 
 # ---------------------------------------------------------------- traffic ---
