@@ -637,3 +637,31 @@ def test_decode_counting_pass_unaligned_payload(g, in_offset):
     assert_roundtrip_parity(g, st, n, in_offset=in_offset, cap=cap, in_len=st.size)
     dense, nd = _dense_stream(in_offset, DECODE_DEFER_BYTES + 999)
     assert_roundtrip_parity(g, dense, nd, offset=1, in_offset=in_offset)
+
+
+def test_accumulate_mixes_look_back_and_counting_streams(g):
+    # one call whose streams take different decode paths: an exact-size
+    # buffer (look-back) and a worst-case buffer (counting pass), in order
+    n = 5 * DECODE_DEFER_BYTES + 777
+    x, err, s = mixed_case(6200, n, zero_frac=0.9)
+    rc, st, _ = oracle.compress(x, s, err)
+    x2, err2, _ = mixed_case(6201, n, zero_frac=0.5)
+    rc2, st2, _ = oracle.compress(x2, s, err2)
+    assert rc == rc2 == 0
+    cap_big = g.tlc_compress_bound(n)
+    acc0 = synth.normal(synth.key_for(6202, 6), n, 1.0)
+    buf, acc = _guarded_f32(n)
+    acc.copy_(torch.from_numpy(acc0))
+    small = torch.from_numpy(st).cuda()
+    big = torch.full((cap_big,), CANARY, dtype=torch.uint8, device="cuda")
+    big[:st2.size].copy_(torch.from_numpy(st2))
+    small2 = torch.from_numpy(st).cuda()
+    lens = torch.tensor([st.size, st2.size, st.size], dtype=torch.int64, device="cuda")
+    dev_st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g.tlc_decompress_accumulate([small, big, small2], n, acc, in_lens=lens,
+                                in_caps=[st.size, cap_big, st.size], dev_status=dev_st)
+    torch.cuda.synchronize()
+    _check_f32_guards(buf, n)
+    rc_o, a_o = oracle.decompress_accumulate([st, st2, st], n, acc0)
+    assert int(dev_st.item()) == rc_o == 0
+    assert np.array_equal(bits(acc.cpu().numpy()), bits(a_o))
