@@ -665,3 +665,62 @@ def test_accumulate_mixes_look_back_and_counting_streams(g):
     rc_o, a_o = oracle.decompress_accumulate([st, st2, st], n, acc0)
     assert int(dev_st.item()) == rc_o == 0
     assert np.array_equal(bits(acc.cpu().numpy()), bits(a_o))
+
+
+# ---- the largest tensors: 32-bit index limits ------------------------------
+
+def test_near_maximum_size_properties(g):
+    # n just below 2^32 (the largest the calls accept): +-1 planted at chosen
+    # positions in zeros, M = 1, s = 1, so q = x exactly.  Every expectation
+    # follows from the format's definition: the decoded values and the error
+    # buffer, the stream length from the zero runs between the literal
+    # groups, and the literal bytes in order.
+    n = (1 << 32) - 7
+    G = (n + 4) // 5
+    planted = sorted({0, 1, 4, 5, 20479, 20480, 5 * 4096 * 384 - 1,
+                      (1 << 31) - 1, 1 << 31, (1 << 31) + 1, (1 << 31) + 5 * 14 * 3,
+                      (1 << 32) - 5 * 4096 - 3, n - 6, n - 1})
+    signs = [1 if i % 3 else -1 for i in range(len(planted))]
+    try:
+        x = torch.zeros(n, dtype=torch.float32, device="cuda")
+        err = torch.zeros(n, dtype=torch.float32, device="cuda")
+        y = torch.empty(n, dtype=torch.float32, device="cuda")
+    except torch.cuda.OutOfMemoryError:
+        pytest.skip("not enough device memory for 3 x 17 GB")
+    idx = torch.tensor(planted, dtype=torch.int64, device="cuda")
+    x[idx] = torch.tensor(signs, dtype=torch.float32, device="cuda")
+    cap = g.tlc_compress_bound(n)
+    out = torch.empty(cap, dtype=torch.uint8, device="cuda")
+    out_len = torch.zeros(1, dtype=torch.int64, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g.tlc_compress(x, 1.0, err, out, out_len, st)
+    g.tlc_decompress(out, n, y, in_len=out_len, in_cap=cap, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    # x' = x, |x'| = M = scale: every planted value is kept whole, err' = 0
+    assert int(torch.count_nonzero(err).item()) == 0
+    assert int(torch.count_nonzero(y).item()) == len(planted)
+    assert y[idx].cpu().tolist() == [float(v) for v in signs]
+    # the stream: header 1.0f, then literal groups and zero runs
+    groups = {}
+    for p, v in zip(planted, signs):
+        gi, j = divmod(p, 5)
+        digits = groups.setdefault(gi, [1, 1, 1, 1, 1])
+        digits[j] = v + 1
+    lits = sorted(groups)
+    runs = [lits[0]] + [b - a - 1 for a, b in zip(lits, lits[1:])] + [G - 1 - lits[-1]]
+    want_len = 4 + len(lits) + sum((r + 13) // 14 for r in runs if r > 0)
+    L = int(out_len.item())
+    assert L == want_len
+    s = out[:L].cpu().numpy()
+    assert s[:4].tolist() == list(np.float32(1.0).tobytes())
+    lit_bytes = [int(b) for b in s[4:] if b < 243 and b != 121]
+    want = []
+    for gi in lits:
+        v = 0
+        for d in groups[gi]:
+            v = 3 * v + d
+        want.append(v)
+    assert lit_bytes == want
+    # single zero groups between literals stay 121; all longer runs are escapes
+    assert int((s[4:] == 121).sum()) == sum(1 for r in runs if r % 14 == 1)
