@@ -724,3 +724,10 @@ def test_near_maximum_size_properties(g):
     assert lit_bytes == want
     # single zero groups between literals stay 121; all longer runs are escapes
     assert int((s[4:] == 121).sum()) == sum(1 for r in runs if r % 14 == 1)
+    # accumulate into zeros: the same values, and +0.0 everywhere else
+    del err
+    acc = torch.zeros(n, dtype=torch.float32, device="cuda")
+    g.tlc_decompress_accumulate([out], n, acc, in_lens=out_len, in_caps=[cap], dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert bool(torch.equal(acc.view(torch.int32), y.view(torch.int32)))
