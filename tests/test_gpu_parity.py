@@ -731,3 +731,43 @@ def test_near_maximum_size_properties(g):
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert bool(torch.equal(acc.view(torch.int32), y.view(torch.int32)))
+
+
+def test_decode_fuzz_random_payloads(g):
+    # random payload bytes behind a valid header: the decoder must agree with
+    # the oracle on CORRUPT or OK, match it bit for bit when OK, and never
+    # write outside y (the guards) -- for dense output and for accumulate
+    u = synth.uniforms(synth.key_for(7000, 0), 3 * 300)
+    agree = ok_cases = 0
+    for i in range(300):
+        n = 1 + int(u[3 * i] * 60_000)
+        groups = (n + 4) // 5
+        m = 1 + int(u[3 * i + 1] * (groups - 1))
+        kind = int(u[3 * i + 2] * 3)
+        raw = (synth.uniforms(synth.key_for(7001 + i, 1), m) * 256).astype(np.uint8)
+        if kind == 1:      # mostly escapes: expands fast, often too far
+            raw = np.where(raw < 200, 243 + raw % 13, raw).astype(np.uint8)
+        elif kind == 2:    # mostly single groups: expands slowly, often too short
+            raw = np.where(raw >= 243, 121, raw).astype(np.uint8)
+        if i % 2 == 0:     # cut and finish the random bytes to expand exactly
+            exp = np.where(raw >= 243, raw.astype(np.int64) - 241, 1)
+            cum = np.cumsum(exp)
+            keep = int(np.searchsorted(cum, groups, side="right"))
+            raw = raw[:keep]
+            left = groups - (int(cum[keep - 1]) if keep else 0)
+            tail = [255] * (left // 14) + ([] if left % 14 == 0 else
+                                           [121] if left % 14 == 1 else [241 + left % 14])
+            raw = np.concatenate([raw, np.array(tail, np.uint8)]).astype(np.uint8)
+        stream = np.concatenate([np.frombuffer(np.float32(0.5).tobytes(), np.uint8), raw])
+        rc_o, y_o = oracle.decompress(stream, n)
+        rc_g, y_g = gpu_decompress(g, stream, n)
+        assert rc_g == rc_o, f"case {i}: n={n} m={m} kind={kind}"
+        if rc_o == 0:
+            ok_cases += 1
+            assert np.array_equal(bits(y_g), bits(y_o)), f"case {i}"
+            acc0 = synth.normal(synth.key_for(7001 + i, 2), n, 1.0)
+            rc_oa, a_o = oracle.decompress_accumulate([stream], n, acc0)
+            rc_ga, a_g = gpu_accumulate(g, [stream], n, acc0)
+            assert rc_ga == rc_oa == 0 and np.array_equal(bits(a_g), bits(a_o))
+        agree += 1
+    assert agree == 300 and ok_cases >= 100
