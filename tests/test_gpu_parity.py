@@ -771,3 +771,29 @@ def test_decode_fuzz_random_payloads(g):
             assert rc_ga == rc_oa == 0 and np.array_equal(bits(a_g), bits(a_o))
         agree += 1
     assert agree == 300 and ok_cases >= 100
+
+
+def test_compress_fuzz_magnitudes_and_special_values(g):
+    # random scales from subnormal to near FLT_MAX, signed zeros, subnormals,
+    # exact ties of the rounding, random s: stream, length, status and error
+    # buffer must match the oracle bit for bit
+    u = synth.uniforms(synth.key_for(7100, 0), 6 * 200)
+    for i in range(200):
+        n = 1 + int(u[6 * i] * 30_000)
+        scale_exp = -45 + u[6 * i + 1] * 83          # 1e-45 .. 1e38
+        s = float(np.float32(1.0 + 0.999999 * u[6 * i + 2]))
+        x = (synth.normal(synth.key_for(7101 + i, 0), n, 1.0) * np.float32(10.0 ** scale_exp))
+        x = x.astype(np.float32)
+        err = (synth.laplace(synth.key_for(7101 + i, 1), n, 1.0) *
+               np.float32(10.0 ** (scale_exp - 1))).astype(np.float32)
+        pick = synth.uniforms(synth.key_for(7101 + i, 2), n)
+        x[pick < 0.2] = 0.0
+        x[(pick >= 0.2) & (pick < 0.25)] = -0.0
+        sub = (pick >= 0.25) & (pick < 0.3)
+        x[sub] = np.float32(1e-40) * np.sign(x[sub] + np.float32(1e-45))
+        if u[6 * i + 3] < 0.3:                       # plant exact ties at M * s / 2
+            mx = np.max(np.abs(x + err))
+            if np.isfinite(mx) and mx > 0:
+                k = int(u[6 * i + 4] * n)
+                x[k] = np.float32(np.float32(mx) * np.float32(s) / np.float32(2.0)) - err[k]
+        assert_compress_parity(g, x, s, err)
