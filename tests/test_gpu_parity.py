@@ -731,6 +731,8 @@ def test_near_maximum_size_properties(g):
     torch.cuda.synchronize()
     assert int(st.item()) == 0
     assert bool(torch.equal(acc.view(torch.int32), y.view(torch.int32)))
+    del x, y, acc, out
+    torch.cuda.empty_cache()   # hand the 50 GB back before the next tests
 
 
 def test_decode_fuzz_random_payloads(g):
