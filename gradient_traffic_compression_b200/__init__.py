@@ -18,6 +18,7 @@ from .tlc import (  # noqa: F401
     decompress,
     lib,
     status_string,
+    stream_info,
     tlc_compress,
     tlc_compress_batch,
     tlc_compress_bound,

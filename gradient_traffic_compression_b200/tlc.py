@@ -344,6 +344,28 @@ def compress(x, s: float, err, stream=None):
     return out, out_len, st
 
 
+def stream_info(stream_buf, length, n: int, s: float | None = None) -> dict:
+    """Host-side facts of one stream, for logging: its length, bits per value
+    (header included), the scale M*s from the 4-byte little-endian header,
+    and M when s is given.  stream_buf: uint8 tensor (any device) or bytes-like
+    holding at least the header; length: int or one-element tensor.  Reads
+    the 4 header bytes only (a device-to-host copy and synchronisation for
+    CUDA tensors)."""
+    import struct
+    L = int(length.item()) if hasattr(length, "item") else int(length)
+    if hasattr(stream_buf, "cpu"):
+        head = bytes(stream_buf[:4].cpu().numpy().tobytes())
+    else:
+        head = bytes(stream_buf[:4])
+    if L < 4 or len(head) < 4:
+        raise ValueError("a stream holds at least its 4-byte header")
+    scale = struct.unpack("<f", head)[0]
+    info = {"length": L, "bits_per_value": 8.0 * L / int(n), "scale": scale}
+    if s is not None:
+        info["M"] = scale / float(s)
+    return info
+
+
 def decompress(stream_buf, n: int, in_len=None, stream=None):
     """Allocate y and decompress: returns (y, dev_status)."""
     import torch

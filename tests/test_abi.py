@@ -154,3 +154,16 @@ def test_kernel_timing_names_and_kind_mask(L):
     assert all(v == (0, 0.0) for v in got.values())
     with pytest.raises(KeyError):
         g.tlc_kernel_timing_kinds(["no_such_kernel"])
+
+
+def test_stream_info_reads_the_header():
+    import numpy as np
+
+    import gradient_traffic_compression_b200 as g
+    import oracle
+    x = np.zeros(1000, np.float32)
+    x[10] = 3.0
+    rc, st, _ = oracle.compress(x, 1.5, np.zeros(1000, np.float32))
+    info = g.stream_info(st.tobytes(), st.size, 1000, 1.5)
+    assert info["length"] == st.size and info["scale"] == np.float32(4.5)
+    assert abs(info["M"] - 3.0) < 1e-6 and info["bits_per_value"] == 8.0 * st.size / 1000
