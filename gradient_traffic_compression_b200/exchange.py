@@ -77,23 +77,18 @@ def allgather_streams(stream, length, group=None):
     return torch.stack(rows), lengths
 
 
-def exchange_step(x, s, err, acc, group=None, dev_status=None):
-    """One data-parallel step on CUDA tensors: compress x (err updated in
-    place), all-gather the streams, add all ranks' decoded values into acc
-    (rank order).  Returns (lengths, dev_status tensor)."""
-    from . import tlc
+def exchange_step(x, s, err, acc, group=None, dev_status=None, codec=None):
+    """One data-parallel step: compress x (err updated in place), all-gather
+    the streams, add all ranks' decoded values into acc (rank order).
+    codec defaults to CudaCodec (CUDA tensors).  Returns (lengths, dev_status
+    tensor)."""
+    codec = codec if codec is not None else CudaCodec()
     n = x.numel()
-    out = torch.empty(tlc.tlc_compress_bound(n), dtype=torch.uint8, device=x.device)
-    out_len = torch.zeros(1, dtype=torch.int64, device=x.device)
     st = dev_status if dev_status is not None else torch.zeros(
         1, dtype=torch.int32, device=x.device)
-    tlc.tlc_compress(x, s, err, out, out_len, st)
-    length = int(out_len.item())
-    if length == 0:
-        raise RuntimeError(f"compression failed on this rank (status {int(st.item())})")
+    out, length = codec.compress(x, s, err, st)
     slots, lengths = allgather_streams(out, length, group)
-    rows = [slots[r].contiguous() for r in range(slots.shape[0])]
-    tlc.tlc_decompress_accumulate(rows, n, acc, in_caps=lengths, dev_status=st)
+    codec.accumulate([slots[r, :lengths[r]] for r in range(slots.shape[0])], lengths, n, acc, st)
     return lengths, st
 
 
@@ -134,7 +129,7 @@ def alltoall_streams(streams, lengths, group=None):
 
 
 class CudaCodec:
-    """The codec steps of the sharded exchange through libtlc.so (CUDA
+    """The codec steps of both exchange forms through libtlc.so (CUDA
     tensors).  Each method enqueues work on the current stream; a length is
     read back to the host only where the transport needs it."""
 

@@ -212,3 +212,61 @@ def test_sharded_exchange_matches_a_single_process_model(world):
             if k == steps - 1:
                 assert results[0][3][d] == sd.size
         assert results[0][1][k] == y.tobytes(), f"step {k}"
+
+
+def _allgather_worker(rank, world, port, n, q):
+    try:
+        sys.path.insert(0, ROOT)
+        os.environ["MASTER_ADDR"] = "127.0.0.1"
+        os.environ["MASTER_PORT"] = str(port)
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        from gradient_traffic_compression_b200.exchange import exchange_step
+        dist.init_process_group("gloo", rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=60))
+        x = torch.from_numpy(_sharded_inputs(rank, n))
+        err = torch.zeros(n, dtype=torch.float32)
+        acc = torch.zeros(n, dtype=torch.float32)
+        lengths, _ = exchange_step(x, 1.5, err, acc, codec=_OracleCodec(),
+                                   dev_status=torch.zeros(1, dtype=torch.int32))
+        q.put((rank, acc.numpy().tobytes(), lengths, err.numpy().tobytes()))
+        dist.barrier()
+        dist.destroy_process_group()
+    except Exception as e:  # report to the parent instead of hanging it
+        q.put((rank, "error", repr(e)))
+
+
+@pytest.mark.timeout(240)
+@pytest.mark.parametrize("world", [2, 3])
+def test_allgather_exchange_step_matches_a_single_process_model(world):
+    n = 30_001
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_allgather_worker, args=(r, world, port, n, q))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(world):
+        item = q.get(timeout=200)
+        assert item[1] != "error", item
+        res[item[0]] = item
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    sys.path.insert(0, ROOT)
+    import oracle
+    streams, errs = [], []
+    for r in range(world):
+        rc, st, e2 = oracle.compress(_sharded_inputs(r, n), 1.5, np.zeros(n, np.float32))
+        streams.append(st)
+        errs.append(e2)
+    _, want = oracle.decompress_accumulate(streams, n, np.zeros(n, np.float32))
+    for r in range(world):
+        assert res[r][1] == want.tobytes()                   # the same sum everywhere
+        assert res[r][2] == [st.size for st in streams]      # every rank's length
+        assert res[r][3] == errs[r].tobytes()                # each rank's own error buffer
