@@ -34,6 +34,7 @@ from .tlc import (  # noqa: F401
     tlc_plan_stream_offset,
     tlc_kernel_timing_read,
     tlc_set_wait_limit,
+    tlc_test_compress_wait_timeout,
     tlc_test_wait_timeout,
     version,
 )

@@ -507,7 +507,8 @@ tlc_status tlc_decompress_batch(tlc_plan plan, const uint8_t *arena, const uint6
   return ce == cudaSuccess ? TLC_OK : TLC_ERR_CUDA;
 }
 
-tlc_status tlc_test_wait_timeout(uint32_t max_polls, int32_t *dev_status, tlc_stream_t stream) {
+static tlc_status run_wait_test(bool compress_side, uint32_t max_polls, int32_t *dev_status,
+                                tlc_stream_t stream) {
   if (!max_polls || !dev_status) return TLC_ERR_INVALID_ARG;
   cudaError_t ce;
   const tlc::DeviceInfo *dev = current_device(ce);
@@ -517,9 +518,21 @@ tlc_status tlc_test_wait_timeout(uint32_t max_polls, int32_t *dev_status, tlc_st
   if (scratch_alloc(*dev, 256, &scratch, st) != cudaSuccess) return TLC_ERR_CUDA;
   ce = cudaMemsetAsync(scratch, 0, 256, st);
   if (ce == cudaSuccess)
-    ce = tlc::launch_wait_test(static_cast<uint64_t *>(scratch), max_polls, dev_status, st);
+    ce = compress_side
+             ? tlc::launch_compress_wait_test(static_cast<uint64_t *>(scratch), max_polls,
+                                              dev_status, st)
+             : tlc::launch_wait_test(static_cast<uint64_t *>(scratch), max_polls, dev_status, st);
   const cudaError_t fe = cudaFreeAsync(scratch, st);
   return (ce == cudaSuccess && fe == cudaSuccess) ? TLC_OK : TLC_ERR_CUDA;
+}
+
+tlc_status tlc_test_wait_timeout(uint32_t max_polls, int32_t *dev_status, tlc_stream_t stream) {
+  return run_wait_test(false, max_polls, dev_status, stream);
+}
+
+tlc_status tlc_test_compress_wait_timeout(uint32_t max_polls, int32_t *dev_status,
+                                          tlc_stream_t stream) {
+  return run_wait_test(true, max_polls, dev_status, stream);
 }
 
 }  // extern "C"

@@ -1149,6 +1149,21 @@ __global__ void __launch_bounds__(kPlaceThreads) k_zre_place_batch(const BatchQu
               lane);
 }
 
+// Wait-limit check of the compress look-back: tile 1 looks back at a tile 0
+// that never publishes (its status word stays 0); lookback_words reports
+// TLC_ERR_TIMEOUT once the polls run out and returns a zero prefix.
+__global__ void k_compress_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_status) {
+  const ZAgg agg = {0u, 0u, 1u, 0u};
+  uint32_t cin = 0, tin = 0;
+  lookback_words<kLookV, TileCodec>(status, 1, agg, cin, tin, dev_status, max_polls);
+}
+
+cudaError_t launch_compress_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_status,
+                                      cudaStream_t stream) {
+  k_compress_wait_test<<<1, kWarp, 0, stream>>>(status, max_polls, dev_status);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------- launcher ---
 uint32_t compress_tiles(uint64_t n) {
   const uint64_t g = (n + 4) / 5;

@@ -226,6 +226,8 @@ cudaError_t launch_decode(const DeviceInfo &dev, const uint8_t *in, const uint64
                           cudaStream_t stream);
 cudaError_t launch_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_status,
                              cudaStream_t stream);
+cudaError_t launch_compress_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_status,
+                                      cudaStream_t stream);
 int occupancy_decode(bool accumulate);
 
 }  // namespace tlc

@@ -5,6 +5,7 @@
 // tile of 4096 byte groups, a tile ticket, and one partial maximum per block
 // of the magnitude pass.  Here that scratch is a fixed array in the
 // library's own device memory instead of a stream-ordered allocation.
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -20,18 +21,27 @@ constexpr size_t kScratchBytes = 256 * 1024;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void *g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::mutex g_mu;
+std::atomic<void *> g_scratch_ptr[kMaxDevices];
 
 // Host code may not use g_noalloc_scratch as an address (on the host it only
-// names the symbol); ask the runtime for the device address, once per device,
-// while that device is current.
-void resolve_scratch(int d) {
-  void *p = nullptr;
-  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-  g_scratch_ptr[d] = (e == cudaSuccess) ? p : nullptr;
-  g_scratch_err[d] = e;
+// names the symbol); ask the runtime for the device address while that
+// device is current.  The address is kept only once it has been obtained: a
+// failed attempt (for example before the device has a context) returns
+// nullptr, clears the runtime's last-error slot, and the next call tries
+// again.
+void *scratch_for_device(int d) {
+  void *p = g_scratch_ptr[d].load(std::memory_order_acquire);
+  if (p) return p;
+  std::lock_guard<std::mutex> lk(g_mu);
+  p = g_scratch_ptr[d].load(std::memory_order_relaxed);
+  if (p) return p;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  g_scratch_ptr[d].store(p, std::memory_order_release);
+  return p;
 }
 
 }  // namespace
@@ -55,13 +65,12 @@ extern "C" tlc_status tlc_compress_noalloc(const float *x, size_t n, float s, fl
   if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxDevices) return TLC_ERR_CUDA;
   const tlc::DeviceInfo *dev = tlc::device_info(d);
   if (!dev) return TLC_ERR_CUDA;
-  std::call_once(g_once[d], resolve_scratch, d);
-  if (g_scratch_err[d] != cudaSuccess || !g_scratch_ptr[d]) return TLC_ERR_CUDA;
+  void *scratch = scratch_for_device(d);
+  if (!scratch) return TLC_ERR_CUDA;
 
   const uint32_t n_tiles = tlc::compress_tiles(n);
   const uint32_t n_part = tlc::compress_partials(*dev, n);
   if (tlc::compress_scratch_bytes(n_part, n_tiles) > kScratchBytes) return TLC_ERR_INVALID_ARG;
-  void *scratch = g_scratch_ptr[d];
   // k_absmax clears the status words and the ticket before k_quant_zre reads
   // them, and writes every partial maximum that k_quant_zre reads, so nothing
   // left from an earlier call is used.

@@ -52,6 +52,8 @@ def lib() -> ctypes.CDLL:
     L.tlc_set_wait_limit.restype = None
     L.tlc_test_wait_timeout.argtypes = [ctypes.c_uint32, P, P]
     L.tlc_test_wait_timeout.restype = ctypes.c_int
+    L.tlc_test_compress_wait_timeout.argtypes = [ctypes.c_uint32, P, P]
+    L.tlc_test_compress_wait_timeout.restype = ctypes.c_int
     L.tlc_compress_noalloc.argtypes = [P, S, ctypes.c_float, P, P, S, P, P, P]
     L.tlc_compress_noalloc.restype = ctypes.c_int
     L.tlc_plan_create.argtypes = [ctypes.c_int, P, P, P, P, P]
@@ -296,6 +298,13 @@ def tlc_test_wait_timeout(max_polls: int, dev_status, stream=None) -> int:
     return _check("tlc_test_wait_timeout", code)
 
 
+def tlc_test_compress_wait_timeout(max_polls: int, dev_status, stream=None) -> int:
+    import torch
+    code = lib().tlc_test_compress_wait_timeout(
+        int(max_polls), _dev_ptr(dev_status, "dev_status", torch.int32), _stream(stream))
+    return _check("tlc_test_compress_wait_timeout", code)
+
+
 def tlc_kernel_timing(enable: bool) -> None:
     lib().tlc_kernel_timing(1 if enable else 0)
 
@@ -344,13 +353,14 @@ def compress(x, s: float, err, stream=None):
     return out, out_len, st
 
 
-def stream_info(stream_buf, length, n: int, s: float | None = None) -> dict:
-    """Host-side facts of one stream, for logging: its length, bits per value
-    (header included), the scale M*s from the 4-byte little-endian header,
-    and M when s is given.  stream_buf: uint8 tensor (any device) or bytes-like
-    holding at least the header; length: int or one-element tensor.  Reads
-    the 4 header bytes only (a device-to-host copy and synchronisation for
-    CUDA tensors)."""
+def stream_info(stream_buf, length, n: int) -> dict:
+    """Host-side facts of one stream, for logging: what its header and length
+    hold, and nothing derived from the codec's arithmetic.  Returns its length
+    in bytes, bits per value (header included) and the scale M*s from the
+    4-byte little-endian header.  stream_buf: uint8 tensor (any device) or
+    bytes-like holding at least the header; length: int or one-element
+    tensor.  Reads the 4 header bytes only (a device-to-host copy and
+    synchronisation for CUDA tensors)."""
     import struct
     L = int(length.item()) if hasattr(length, "item") else int(length)
     if hasattr(stream_buf, "cpu"):
@@ -360,10 +370,7 @@ def stream_info(stream_buf, length, n: int, s: float | None = None) -> dict:
     if L < 4 or len(head) < 4:
         raise ValueError("a stream holds at least its 4-byte header")
     scale = struct.unpack("<f", head)[0]
-    info = {"length": L, "bits_per_value": 8.0 * L / int(n), "scale": scale}
-    if s is not None:
-        info["M"] = scale / float(s)
-    return info
+    return {"length": L, "bits_per_value": 8.0 * L / int(n), "scale": scale}
 
 
 def decompress(stream_buf, n: int, in_len=None, stream=None):

@@ -214,6 +214,8 @@ tlc_status tlc_decompress_batch(tlc_plan plan, const uint8_t *arena, const uint6
  * else TLC_ERR_INVALID_ARG and nothing is enqueued.
  * - The first call on a device resolves the array's device address (with
  *   that device current); make that first call before any stream capture.
+ *   If resolving fails, that call returns TLC_ERR_CUDA without enqueuing
+ *   anything, and the next call on the device tries again.
  * - Every call on a device shares the one array.  Calls whose work overlaps
  *   on the GPU (different streams, or different host threads without
  *   ordering between their streams) race on it and give wrong results;
@@ -246,6 +248,12 @@ void tlc_set_wait_limit(uint32_t max_polls);
  * NULL dev_status. */
 tlc_status tlc_test_wait_timeout(uint32_t max_polls, int32_t *dev_status,
                                  tlc_stream_t stream);
+
+/* The same check for the compress kernel's cross-block wait (the look-back
+ * that places a tile's zero-run encoded bytes): one tile waits for a
+ * predecessor that never publishes.  Same arguments and results. */
+tlc_status tlc_test_compress_wait_timeout(uint32_t max_polls, int32_t *dev_status,
+                                          tlc_stream_t stream);
 
 /* Per-kernel timing, for benchmarks.  While enabled, the library counts
  * every kernel it launches, by kind, and records a CUDA event pair on the

@@ -446,6 +446,17 @@ def test_bounded_wait_reports_timeout(g):
     assert_compress_parity(g, x, s, err)
 
 
+def test_compress_bounded_wait_reports_timeout(g):
+    # the compress kernel's look-back, waiting on a tile that never publishes
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    g.tlc_test_compress_wait_timeout(64, st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 4
+    # the context is still usable afterwards
+    x, err, s = mixed_case(2, 30000)
+    assert_compress_parity(g, x, s, err)
+
+
 # ---- large tensors: sizes, alignments and runs over many tiles -----------
 
 LARGE_MIN = 1 << 22
