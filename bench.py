@@ -7,8 +7,9 @@ multiplication, quartic packing, zero-run encoding), tlc_decompress (dense
 fp32 output) and tlc_decompress_accumulate (the stream added into a dense
 fp32 aggregation buffer).  The workload is the flat 2^28-value fp32 tensor,
 Laplace(0, 1e-4) with 90% exact zeros in geometric runs (mean 64), s = 1.9,
-with the error buffer carried from step to step.  Inputs (2 GiB of x + err)
-exceed the 126 MB L2, so every step streams from HBM.
+with the error buffer carried from step to step and a fresh gradient every
+step (a few seeded gradients resident on the device, taken in turn).  Inputs
+(2 GiB of x + err) exceed the 126 MB L2, so every step streams from HBM.
 
 value = 4n bytes of fp32 input per step and GPU / device time per step.
 Under torchrun each rank compresses its own tensor (replicas, weak scaling);
@@ -43,6 +44,11 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--log2n", type=int, default=28, help="tensor size 2^k (default 28)")
     p.add_argument("--e2e-steps", type=int, default=8)
+    p.add_argument("--dense", action="store_true",
+                   help="config 3 shape with uniform values and s = 1: a dense stream "
+                        "(the decoder's weak case), an extra line, not the headline")
+    p.add_argument("--grads", type=int, default=4,
+                   help="seeded gradients kept on the device and taken in turn, one per step")
     p.add_argument("--cpu-baseline-log2n", type=int, default=26)
     p.add_argument("--cpu-baseline-seconds", type=float, default=10.0)
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -54,6 +60,9 @@ def parse_args():
                    help="configs 2, 4, 5: replay each step from a CUDA graph of its calls")
     p.add_argument("--per-tensor", action="store_true",
                    help="configs 2/4: one C-ABI call per tensor instead of a plan")
+    p.add_argument("--exchange", choices=["allgather", "sharded"], default=None,
+                   help="time the data-parallel exchange step (NCCL, every rank) on the "
+                        "headline workload instead of the single-GPU codec step")
     p.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4, 5],
                    help="workload: 3 (default, the headline) or another of the five "
                         "parity configs, measured the same way (extra lines)")
@@ -76,11 +85,34 @@ def load_peaks():
     return 6650.0, "fallback"
 
 
-def workload_config(n, log2n):
+def gradient(args, n, step):
+    """The gradient of one step: the workload's seeded tensor, or with
+    --dense uniform values in [-1, 1) (with s = 1 a large share of the values
+    quantize to +-1, so nearly every group is a literal byte of the stream)."""
+    import numpy as np
+
+    import synth
+    if args.dense:
+        return (synth.uniforms(synth.key_for(step, 5), n) * 2 - 1).astype(np.float32)
+    return synth.flat_tensor(args.config, n=n, step=step)
+
+
+def workload_config(n, log2n, dense=False):
+    if dense:
+        return {
+            "workload": (f"flat fp32 tensor of 2^{log2n} values, uniform in [-1, 1), s=1.0 "
+                         "(a dense stream, about one byte per five values); step = compress "
+                         "+ decompress + decompress-accumulate (K=1), error buffer carried, a "
+                         "fresh gradient each step"),
+            "n": n, "s": 1.0, "input_bytes_per_step": 4 * n,
+            "l2": "inputs (x + err = 8n bytes) larger than the 126 MB L2; no flush"
+            if n >= 1 << 24 else "inputs partly L2-resident"}
     return {
         "workload": (f"flat fp32 tensor of 2^{log2n} values, Laplace(0,1e-4) with 90% exact "
                      f"zeros in geometric runs (mean 64), s={S_PARAM}; step = compress + "
-                     "decompress + decompress-accumulate (K=1), error buffer carried"),
+                     "decompress + decompress-accumulate (K=1), error buffer carried, a "
+                     "fresh gradient each step (seeded gradients resident on the device, "
+                     "taken in turn)"),
         "n": n,
         "s": S_PARAM,
         "input_bytes_per_step": 4 * n,
@@ -228,10 +260,16 @@ def run_ours(args, rank, world, local):
         args.log2n = 20
         args.no_e2e = True
         args.no_cpu_baseline = True
+    if args.dense:
+        S_PARAM = 1.0
+        args.no_cpu_baseline = True
     n = 1 << args.log2n
-    x_h = synth.flat_tensor(args.config, n=n, step=rank)   # each rank: its own gradient
-
-    x = torch.from_numpy(x_h).to(dev)
+    # A fresh gradient every step: a few seeded gradients of the workload,
+    # resident on the device, taken in turn (each rank its own), while the
+    # error buffer carries over from step to step.
+    xs = []
+    for k in range(args.grads):
+        xs.append(torch.from_numpy(gradient(args, n, 1000 * rank + k)).to(dev))
     err = torch.zeros(n, dtype=torch.float32, device=dev)
     cap = tlc.tlc_compress_bound(n)
     out = torch.empty(cap, dtype=torch.uint8, device=dev)
@@ -240,8 +278,11 @@ def run_ours(args, rank, world, local):
     acc = torch.zeros(n, dtype=torch.float32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     stream = torch.cuda.current_stream()
+    turn = [0]
 
     def step():
+        x = xs[turn[0] % len(xs)]
+        turn[0] += 1
         tlc.tlc_compress(x, S_PARAM, err, out, out_len, status, stream)
         tlc.tlc_decompress(out, n, y, in_len=out_len, in_cap=cap, dev_status=status,
                            stream=stream)
@@ -273,6 +314,33 @@ def run_ours(args, rank, world, local):
     pre = tlc.tlc_kernel_timing_read()
     dom = max((k for k in pre if pre[k][0]), key=lambda k: pre[k][1])
 
+    # --graph: one CUDA graph per resident gradient, each holding one whole
+    # step (the three calls, with their scratch allocations); the timed
+    # region replays them in turn.  Small tensors are bound by the host's
+    # enqueue cost otherwise.
+    graphs = []
+    graph_launches = None
+    if args.graph:
+        tlc.tlc_kernel_timing_kinds([])
+        tlc.tlc_kernel_timing(True)
+        cs = torch.cuda.Stream(dev)
+        cs.wait_stream(stream)
+        for k in range(len(xs)):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cs):
+                tlc.tlc_compress(xs[k], S_PARAM, err, out, out_len, status, cs)
+                tlc.tlc_decompress(out, n, y, in_len=out_len, in_cap=cap, dev_status=status,
+                                   stream=cs)
+                tlc.tlc_decompress_accumulate([out], n, acc, in_lens=out_len, in_caps=[cap],
+                                              dev_status=status, stream=cs)
+            graphs.append(gr)
+        tlc.tlc_kernel_timing(False)
+        per_graph = tlc.tlc_kernel_timing_read()
+        graph_launches = sum(v[0] for v in per_graph.values()) / len(graphs)
+        for gr in graphs:
+            gr.replay()
+        torch.cuda.synchronize()
+
     # Timed region: K steps between two events, with an event pair around
     # each launch of the dominant kernel only (each pair costs a few
     # microseconds of device time).  Every launch is counted.
@@ -287,8 +355,11 @@ def run_ours(args, rank, world, local):
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for _ in range(args.steps):
-        step()
+    for i in range(args.steps):
+        if graphs:
+            graphs[i % len(graphs)].replay()
+        else:
+            step()
     t_end.record(stream)
     torch.cuda.synchronize()
     sampler.mark("end")
@@ -300,7 +371,14 @@ def run_ours(args, rank, world, local):
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} in the timed region")
     total_ms = t_start.elapsed_time(t_end)
-    dom_ms = kern[dom][1] / max(kern[dom][0], 1)
+    if graphs:
+        # replays do not pass through the library: the dominant kernel's
+        # launch time comes from the timed pre-pass, launches from the capture
+        dom_ms = pre[dom][1] / max(pre[dom][0], 1)
+        kern = {k: (int(graph_launches * args.steps) if k == dom else 0, 0.0) for k in kern}
+        kern[dom] = (int(graph_launches * args.steps), 0.0)
+    else:
+        dom_ms = kern[dom][1] / max(kern[dom][0], 1)
     total_ms, dom_ms = max_over_ranks([total_ms, dom_ms], device=dev)
 
     # Breakdown pass after the timed region (not part of `value`): every
@@ -312,7 +390,7 @@ def run_ours(args, rank, world, local):
     for k in range(steps2):
         e = ev[k]
         e[0].record(stream)
-        tlc.tlc_compress(x, S_PARAM, err, out, out_len, status, stream)
+        tlc.tlc_compress(xs[k % len(xs)], S_PARAM, err, out, out_len, status, stream)
         e[1].record(stream)
         tlc.tlc_decompress(out, n, y, in_len=out_len, in_cap=cap, dev_status=status,
                            stream=stream)
@@ -376,9 +454,11 @@ def run_ours(args, rank, world, local):
         "vs_baseline": None,
         "dtype": "f32",
         "data": "synthetic",
-        "config": (workload_config(n, args.log2n) if args.config == 3 else
+        "config": (workload_config(n, args.log2n, args.dense) if args.config == 3 else
                    {"workload": synth.CONFIGS[args.config]["name"], "n": n, "s": S_PARAM,
-                    "l2": "L2-resident (x + err = 8 MiB)"}) | {"parallelism": f"replicas x{world}"},
+                    "l2": "L2-resident (x + err = 8 MiB)"}) | {"parallelism": f"replicas x{world}"}
+                  | ({"calls": "each step replayed from a CUDA graph of its three calls"}
+                     if graphs else {}),
         "clocks": clocks,
         "gpu_launches": int(sum(v[0] for v in kern.values())),
         "roofline": {
@@ -390,7 +470,10 @@ def run_ours(args, rank, world, local):
             "unit": "GB/s",
             "frac": round(dom_gbs / peak, 4),
             "traffic": traffic_for(dom, n),
-            "timing": f"CUDA events around every {dom} launch in the timed region",
+            "timing": (f"CUDA events around every {dom} launch in the timed region"
+                       if not graphs else
+                       f"CUDA events around each {dom} launch of a pre-pass (the timed "
+                       "region replays CUDA graphs)"),
         },
         "legs": {
             "compress_gbs": round(in_bytes / (c_ms * 1e-3) / 1e9, 1),
@@ -411,15 +494,19 @@ def run_ours(args, rank, world, local):
     }
 
     if not args.no_e2e:
-        result["e2e"] = run_e2e(args, tlc, torch, dev, x_h, n, cap, world)
+        del xs
+        torch.cuda.empty_cache()
+        xs_h = [gradient(args, n, 1000 * rank + k) for k in range(2)]
+        result["e2e"] = run_e2e(args, tlc, torch, dev, xs_h, n, cap, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args)
     return result
 
 
-def run_e2e(args, tlc, torch, dev, x_h, n, cap, world):
+def run_e2e(args, tlc, torch, dev, xs_h, n, cap, world):
     """The step through the public API with host buffers.  Every step copies
-    its gradient x in from pinned host memory, compresses it (the error
+    its gradient x in from pinned host memory (two seeded gradients, taken in
+    turn), compresses it (the error
     buffer stays on the device: it is the codec's state, like a model's
     weights), decompresses and accumulates, and copies the stream buffer
     (its capacity and the length word) and the decoded y out to pinned host
@@ -430,7 +517,7 @@ def run_e2e(args, tlc, torch, dev, x_h, n, cap, world):
     import torch.distributed as dist
 
     from gradient_traffic_compression_b200.exchange import max_over_ranks
-    xh = torch.from_numpy(x_h).pin_memory()
+    xh = [torch.from_numpy(a).pin_memory() for a in xs_h]
     yh = [torch.empty(n, dtype=torch.float32).pin_memory() for _ in range(2)]
     sh = [torch.empty(cap, dtype=torch.uint8).pin_memory() for _ in range(2)]
     lh = [torch.empty(1, dtype=torch.int64).pin_memory() for _ in range(2)]
@@ -452,7 +539,7 @@ def run_e2e(args, tlc, torch, dev, x_h, n, cap, world):
         b = i % 2
         s_in.wait_event(ev_c[b])            # step i-2 no longer reads xd[b]
         with torch.cuda.stream(s_in):
-            xd[b].copy_(xh, non_blocking=True)
+            xd[b].copy_(xh[i % len(xh)], non_blocking=True)
         ev_in[b].record(s_in)
         s_c.wait_event(ev_in[b])
         s_c.wait_event(ev_out[b])           # step i-2's outputs are out
@@ -668,6 +755,101 @@ def run_config_set(args, rank, world, local):
     return res
 
 
+# ------------------------------------------------------ multi-rank exchange --
+
+def run_exchange(args, rank, world, local):
+    """The data-parallel exchange step itself (--exchange): every rank
+    compresses its own gradient of the headline workload, the compressed
+    streams cross the ranks over NCCL, and every rank decodes them.
+    allgather: exchange_step (all-gather of the streams, K = world
+    decompress-accumulate); sharded: exchange_step_sharded (all-to-all of
+    per-shard streams, server-side aggregate and delta compression,
+    all-gather of the delta streams, decode).  Timed with CUDA events on
+    the step's stream, the maximum over ranks; one JSON line (rank 0)."""
+    import torch
+
+    import gradient_traffic_compression_b200 as tlc
+    import synth
+    from gradient_traffic_compression_b200.exchange import (exchange_step,
+                                                            exchange_step_sharded,
+                                                            max_over_ranks, shard_bounds)
+    dev = torch.device("cuda", local)
+    n = 1 << args.log2n
+    xs = [torch.from_numpy(synth.flat_tensor(3, n=n, step=1000 * rank + k)).to(dev)
+          for k in range(args.grads)]
+    err = torch.zeros(n, dtype=torch.float32, device=dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+    if args.exchange == "allgather":
+        acc = torch.zeros(n, dtype=torch.float32, device=dev)
+    else:
+        b = shard_bounds(n, world)
+        server_err = torch.zeros(b[rank + 1] - b[rank], dtype=torch.float32, device=dev)
+        y = torch.zeros(n, dtype=torch.float32, device=dev)
+    turn = [0]
+    last = {}
+
+    def step():
+        x = xs[turn[0] % len(xs)]
+        turn[0] += 1
+        if args.exchange == "allgather":
+            lens, _ = exchange_step(x, S_PARAM, err, acc, dev_status=st)
+            last["widths"] = [lens]
+        else:
+            up, down = exchange_step_sharded(x, S_PARAM, err, server_err, y, dev_status=st)
+            last["widths"] = [up, down]
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    tlc.tlc_kernel_timing_kinds(["k_quant_zre"])
+    tlc.tlc_kernel_timing(True)
+    import torch.distributed as dist
+    dist.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    tlc.tlc_kernel_timing(False)
+    kern = tlc.tlc_kernel_timing_read()
+    if int(st.item()) != 0:
+        raise RuntimeError(f"device status {int(st.item())} in the exchange")
+    ms = t0.elapsed_time(t1) / args.steps
+    dom = kern.get("k_quant_zre", (0, 0.0))
+    dom_ms = dom[1] / max(dom[0], 1)
+    ms, dom_ms = max_over_ranks([ms, dom_ms], device=dev)
+    widths = [int(t.max().item()) for t in last["widths"]]
+    sent = sum((world - 1) * w for w in widths)
+    peak, peak_kind = load_peaks()
+    dom_gbs = 12 * n / (dom_ms * 1e-3) / 1e9 if dom_ms else None
+    return {
+        "metric": METRIC, "value": round(world * 4 * n / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": workload_config(n, args.log2n) | {
+            "parallelism": f"data-parallel exchange over {world} rank(s), NCCL",
+            "step": ("exchange_step: compress, all-gather of the streams, K = world "
+                     "decompress-accumulate" if args.exchange == "allgather" else
+                     "exchange_step_sharded: per-shard compress, all-to-all, aggregate, "
+                     "delta compress, all-gather, decode")},
+        "exchange": {"form": args.exchange, "slot_widths": widths,
+                     "stream_bytes_sent_per_rank_per_step": sent,
+                     "bits_per_value_on_the_wire": round(8 * sum(widths) / n, 5)},
+        "gpu_launches": int(sum(v[0] for v in kern.values())),
+        "roofline": {"bound": "hbm", "kernel": "k_quant_zre",
+                     "achieved": round(dom_gbs, 1) if dom_gbs else None, "peak": peak,
+                     "peak_source": f"{peak_kind} hbm_gbs", "unit": "GB/s",
+                     "frac": round(dom_gbs / peak, 4) if dom_gbs else None,
+                     "traffic": traffic_for("k_quant_zre", n)},
+    }
+
+
 # ------------------------------------------------------- CPU oracle timing --
 
 def oracle_step(oracle, x, n, acc):
@@ -813,22 +995,30 @@ def main():
         if res is not None:
             print(json.dumps(res), flush=True)
         return
-    if world > 1:
+    grouped = world > 1 or args.exchange is not None
+    if grouped:
         import datetime
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(local)
+        if world == 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(29500 + os.getpid() % 1000))
+            os.environ.setdefault("RANK", "0")
+            os.environ.setdefault("WORLD_SIZE", "1")
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                 device_id=torch.device("cuda", local))
     try:
-        if args.config in (1, 3):
+        if args.exchange is not None:
+            res = run_exchange(args, rank, world, local)
+        elif args.config in (1, 3):
             res = run_ours(args, rank, world, local)
         else:
             res = run_config_set(args, rank, world, local)
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
-        if world > 1:
+        if grouped:
             import torch.distributed as dist
             dist.destroy_process_group()
 

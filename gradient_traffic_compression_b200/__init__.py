@@ -23,8 +23,12 @@ from .tlc import (  # noqa: F401
     tlc_compress_batch,
     tlc_compress_bound,
     tlc_compress_noalloc,
+    tlc_compress_recorded,
+    record_fields,
     tlc_decompress,
     tlc_decompress_batch,
+    tlc_debug_build,
+    tlc_debug_fault,
     tlc_decompress_accumulate,
     tlc_kernel_timing,
     tlc_kernel_timing_kinds,

@@ -17,6 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 SOURCES = ["tlc_api.cu", "tlc_compress.cu", "tlc_decode.cu", "tlc_noalloc.cu"]
 HEADERS = ["tlc_device.cuh", "tlc_internal.h"]
 LIB_NAME = "libtlc.so"
+DEBUG_LIB_NAME = "libtlc_debug.so"   # -DTLC_DEBUG: recording bounds checks, canaries
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -26,8 +27,8 @@ NVCC_FLAGS = [
 ]
 
 
-def library_path() -> str:
-    return os.path.join(PKG, LIB_NAME)
+def library_path(debug: bool = False) -> str:
+    return os.path.join(PKG, DEBUG_LIB_NAME if debug else LIB_NAME)
 
 
 def _nvcc() -> str:
@@ -43,19 +44,21 @@ def _inputs():
         yield os.path.join(CSRC, f)
 
 
-def is_stale() -> bool:
-    lib = library_path()
+def is_stale(debug: bool = False) -> bool:
+    lib = library_path(debug)
     if not os.path.exists(lib):
         return True
     t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _inputs())
 
 
-def build_library(verbose: bool = False, ptxas_info: bool = False) -> str:
-    """Compile every CUDA source into libtlc.so next to this file."""
-    out = library_path()
+def build_library(verbose: bool = False, ptxas_info: bool = False, debug: bool = False) -> str:
+    """Compile every CUDA source into libtlc.so next to this file (debug:
+    libtlc_debug.so, with -DTLC_DEBUG)."""
+    out = library_path(debug)
     tmp = out + f".tmp{os.getpid()}"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-o", tmp, *[os.path.join(CSRC, f) for f in SOURCES]]
+    cmd = [_nvcc(), *NVCC_FLAGS, *(["-DTLC_DEBUG"] if debug else []), "-o", tmp,
+           *[os.path.join(CSRC, f) for f in SOURCES]]
     if ptxas_info:
         cmd.insert(1, "-Xptxas=-v")
     if verbose:
@@ -89,11 +92,11 @@ def source_digest(kernel: str | None = None) -> str:
     return h.hexdigest()[:12]
 
 
-def ensure_built() -> str:
-    if is_stale():
-        build_library()
-    return library_path()
+def ensure_built(debug: bool = False) -> str:
+    if is_stale(debug):
+        build_library(debug=debug)
+    return library_path(debug)
 
 
 if __name__ == "__main__":
-    print(build_library(verbose=True, ptxas_info="-v" in sys.argv))
+    print(build_library(verbose=True, ptxas_info="-v" in sys.argv, debug="--debug" in sys.argv))

@@ -2,15 +2,37 @@
 // allocation from a per-device stream-ordered pool, and kernel launches.
 // No host synchronisation happens here; all data-dependent checks run on the
 // device and report through *dev_status.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <cstddef>
 #include <cstring>
 #include <mutex>
 #include <vector>
 
 #include "../../include/tlc.h"
+#define TLC_TU 3
+#include "tlc_device.cuh"
 #include "tlc_internal.h"
 #include <nvtx3/nvToolsExt.h>
+
+namespace tlc {
+TLC_DEFINE_DEBUG_READER(debug_fault_api)
+uint32_t debug_fault_compress(bool reset);
+uint32_t debug_fault_decode(bool reset);
+
+#ifdef TLC_DEBUG
+// Debug build: every scratch allocation gets kCanary bytes of 0xA5 on both
+// sides; after the call's kernels, this kernel checks them.
+constexpr size_t kCanary = 256;
+__global__ void k_check_canaries(const uint8_t *base, size_t bytes) {
+  for (size_t i = threadIdx.x; i < kCanary; i += blockDim.x) {
+    (void)TLC_CHECK(base[i] == 0xA5);
+    (void)TLC_CHECK(base[kCanary + bytes + i] == 0xA5);
+  }
+}
+#endif
+}  // namespace tlc
 
 namespace {
 
@@ -36,8 +58,11 @@ void init_device(int d) {
     di.occ_decode_write = tlc::occupancy_decode(false);
     di.occ_decode_acc = tlc::occupancy_decode(true);
     di.occ_quant_batch = tlc::occupancy_quant_batch();
-    di.occ_decode_batch_write = tlc::occupancy_decode_batch(false);
-    di.occ_decode_batch_acc = tlc::occupancy_decode_batch(true);
+    di.occ_decode_batch_write = tlc::occupancy_decode_batch(false, false);
+    di.occ_decode_batch_acc = tlc::occupancy_decode_batch(true, false);
+    di.occ_decode_batch_ix_write = tlc::occupancy_decode_batch(false, true);
+    di.occ_decode_batch_ix_acc = tlc::occupancy_decode_batch(true, true);
+    tlc::occupancy_decode_ix(di.occ_decode_ix);
     cudaMemPoolProps props;
     std::memset(&props, 0, sizeof(props));
     props.allocType = cudaMemAllocationTypePinned;
@@ -87,9 +112,39 @@ struct NvtxRange {
   NvtxRange &operator=(const NvtxRange &) = delete;
 };
 
-// Stream-ordered scratch from the library's pool.
-cudaError_t scratch_alloc(const tlc::DeviceInfo &dev, size_t bytes, void **p, cudaStream_t st) {
-  return cudaMallocFromPoolAsync(p, bytes, dev.pool, st);
+// Stream-ordered scratch from the library's pool.  (The debug build adds
+// canaries on both sides and checks them when the scratch is freed.)
+struct Scratch {
+  void *base = nullptr;
+  size_t bytes = 0;
+};
+
+cudaError_t scratch_alloc(const tlc::DeviceInfo &dev, size_t bytes, void **p, cudaStream_t st,
+                          Scratch &sc) {
+  sc.bytes = bytes;
+#ifdef TLC_DEBUG
+  cudaError_t e = cudaMallocFromPoolAsync(&sc.base, bytes + 2 * tlc::kCanary, dev.pool, st);
+  if (e != cudaSuccess) return e;
+  char *b = static_cast<char *>(sc.base);
+  e = cudaMemsetAsync(b, 0xA5, tlc::kCanary, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(b + tlc::kCanary + bytes, 0xA5, tlc::kCanary, st);
+  *p = b + tlc::kCanary;
+  return e;
+#else
+  cudaError_t e = cudaMallocFromPoolAsync(&sc.base, bytes, dev.pool, st);
+  *p = sc.base;
+  return e;
+#endif
+}
+
+cudaError_t scratch_free(Scratch &sc, cudaStream_t st) {
+  if (!sc.base) return cudaSuccess;
+#ifdef TLC_DEBUG
+  tlc::k_check_canaries<<<1, 256, 0, st>>>(static_cast<const uint8_t *>(sc.base), sc.bytes);
+#endif
+  const cudaError_t e = cudaFreeAsync(sc.base, st);
+  sc.base = nullptr;
+  return e;
 }
 
 // ---- optional per-kernel timing -------------------------------------------
@@ -209,16 +264,37 @@ const char *tlc_status_string(tlc_status s) {
   return "unknown status";
 }
 
-const char *tlc_version(void) { return "0.1.0"; }
+const char *tlc_version(void) { return "0.2.0"; }
+
+int tlc_debug_build(void) {
+#ifdef TLC_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+uint32_t tlc_debug_fault(int reset) {
+  const uint32_t f[3] = {tlc::debug_fault_api(reset != 0), tlc::debug_fault_compress(reset != 0),
+                         tlc::debug_fault_decode(reset != 0)};
+  for (uint32_t v : f)
+    if (v) return v;
+  return 0;
+}
 
 void tlc_set_wait_limit(uint32_t max_polls) {
   g_wait_limit.store(max_polls, std::memory_order_relaxed);
 }
 
-tlc_status tlc_compress(const float *x, size_t n, float s, float *err, uint8_t *out,
-                        size_t out_cap, uint64_t *out_len, int32_t *dev_status,
-                        tlc_stream_t stream) {
-  NvtxRange nvtx("tlc_compress");
+static_assert(sizeof(tlc_compress_record) == sizeof(tlc::CompressRecord) &&
+                  offsetof(tlc_compress_record, nonzeros) ==
+                      offsetof(tlc::CompressRecord, nonzeros) &&
+                  offsetof(tlc_compress_record, length) == offsetof(tlc::CompressRecord, length),
+              "the public record and the kernels' record share one layout");
+
+static tlc_status compress_call(const float *x, size_t n, float s, float *err, uint8_t *out,
+                                size_t out_cap, uint64_t *out_len, int32_t *dev_status,
+                                tlc::CompressRecord *rec, tlc_stream_t stream) {
   if (!x || !err || !out || !out_len || !n_ok(n)) return TLC_ERR_INVALID_ARG;
   if (!(s >= 1.0f && s < 2.0f)) return TLC_ERR_INVALID_ARG;  // also rejects NaN
   if (out_cap < tlc_compress_bound(n)) return TLC_ERR_INVALID_ARG;
@@ -231,16 +307,33 @@ tlc_status tlc_compress(const float *x, size_t n, float s, float *err, uint8_t *
   if (!dev) return TLC_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   void *scratch = nullptr;
+  Scratch sc;
   const bool deferred = tlc::compress_deferred(n);
   const size_t bytes = tlc::compress_scratch_bytes_for(*dev, n, deferred);
-  if (scratch_alloc(*dev, bytes + 256, &scratch, st) != cudaSuccess) return TLC_ERR_CUDA;
+  if (scratch_alloc(*dev, bytes + 256, &scratch, st, sc) != cudaSuccess) return TLC_ERR_CUDA;
   // a status word for calls without one, past everything the kernels use
   int32_t *status_ptr =
       dev_status ? dev_status : reinterpret_cast<int32_t *>(static_cast<char *>(scratch) + bytes);
   ce = tlc::launch_compress(*dev, x, n, s, err, out, out_cap, out_len, status_ptr, wait_limit(),
-                            scratch, st, deferred);
-  const cudaError_t fe = cudaFreeAsync(scratch, st);
+                            scratch, st, deferred, rec);
+  const cudaError_t fe = scratch_free(sc, st);
   return (ce == cudaSuccess && fe == cudaSuccess) ? TLC_OK : TLC_ERR_CUDA;
+}
+
+tlc_status tlc_compress(const float *x, size_t n, float s, float *err, uint8_t *out,
+                        size_t out_cap, uint64_t *out_len, int32_t *dev_status,
+                        tlc_stream_t stream) {
+  NvtxRange nvtx("tlc_compress");
+  return compress_call(x, n, s, err, out, out_cap, out_len, dev_status, nullptr, stream);
+}
+
+tlc_status tlc_compress_recorded(const float *x, size_t n, float s, float *err, uint8_t *out,
+                                 size_t out_cap, uint64_t *out_len, int32_t *dev_status,
+                                 tlc_compress_record *record, tlc_stream_t stream) {
+  NvtxRange nvtx("tlc_compress_recorded");
+  if (!record) return TLC_ERR_INVALID_ARG;
+  return compress_call(x, n, s, err, out, out_cap, out_len, dev_status,
+                       reinterpret_cast<tlc::CompressRecord *>(record), stream);
 }
 
 static tlc_status check_stream_arg(const uint8_t *in, size_t cap, bool len_on_device, size_t n) {
@@ -262,17 +355,30 @@ tlc_status tlc_decompress(const uint8_t *in, const uint64_t *in_len, size_t in_c
   if (!dev) return TLC_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const uint32_t tiles = tlc::decode_tiles_max(in_cap, groups_of(n));
-  const size_t words = tlc::decode_scratch_words(tiles);
-  const size_t bytes = tlc::align_up(8 * words + 8, 256);
   void *scratch = nullptr;
-  if (scratch_alloc(*dev, bytes, &scratch, st) != cudaSuccess) return TLC_ERR_CUDA;
-  uint64_t *status = static_cast<uint64_t *>(scratch);
-  int32_t *status_ptr = dev_status ? dev_status : reinterpret_cast<int32_t *>(status + words);
-  ce = tlc::decode_deferred(tiles) ? cudaSuccess : cudaMemsetAsync(scratch, 0, 8 * words, st);
-  if (ce == cudaSuccess)
-    ce = tlc::launch_decode(*dev, in, in_len, in_cap, n, y, false, status_ptr, wait_limit(),
-                            status, st);
-  const cudaError_t fe = cudaFreeAsync(scratch, st);
+  Scratch sc;
+  if (tlc::decode_deferred(tiles)) {
+    // large stream: index, then decode
+    const tlc::IndexedStream is = {in, in_len, in_cap};
+    const size_t bytes = tlc::indexed_layout(&is, 1, n).total_bytes;
+    if (scratch_alloc(*dev, bytes + 256, &scratch, st, sc) != cudaSuccess) return TLC_ERR_CUDA;
+    int32_t *status_ptr =
+        dev_status ? dev_status : reinterpret_cast<int32_t *>(static_cast<char *>(scratch) + bytes);
+    ce = tlc::launch_decode_indexed(*dev, &is, 1, n, y, false, status_ptr, wait_limit(), scratch,
+                                    st);
+  } else {
+    // small stream: one launch, tiles find their place by a look-back
+    const size_t words = tlc::decode_scratch_words(tiles);
+    const size_t bytes = tlc::align_up(8 * words + 8, 256);
+    if (scratch_alloc(*dev, bytes, &scratch, st, sc) != cudaSuccess) return TLC_ERR_CUDA;
+    uint64_t *status = static_cast<uint64_t *>(scratch);
+    int32_t *status_ptr = dev_status ? dev_status : reinterpret_cast<int32_t *>(status + words);
+    ce = cudaMemsetAsync(scratch, 0, 8 * words, st);
+    if (ce == cudaSuccess)
+      ce = tlc::launch_decode(*dev, in, in_len, in_cap, n, y, false, status_ptr, wait_limit(),
+                              status, st);
+  }
+  const cudaError_t fe = scratch_free(sc, st);
   return (ce == cudaSuccess && fe == cudaSuccess) ? TLC_OK : TLC_ERR_CUDA;
 }
 
@@ -291,27 +397,43 @@ tlc_status tlc_decompress_accumulate(const uint8_t *const *ins, const uint64_t *
   if (!dev) return TLC_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const size_t g = groups_of(n);
-  size_t total_words = 0;
-  bool zero = false;  // some stream takes the look-back path
-  for (int w = 0; w < k; ++w) {
-    const uint32_t tiles = tlc::decode_tiles_max(in_caps[w], g);
-    total_words += tlc::decode_scratch_words(tiles);
-    zero = zero || !tlc::decode_deferred(tiles);
-  }
-  const size_t bytes = tlc::align_up(8 * total_words + 8, 256);
   void *scratch = nullptr;
-  if (scratch_alloc(*dev, bytes, &scratch, st) != cudaSuccess) return TLC_ERR_CUDA;
-  uint64_t *base = static_cast<uint64_t *>(scratch);
-  int32_t *status_ptr = dev_status ? dev_status : reinterpret_cast<int32_t *>(base + total_words);
-  ce = zero ? cudaMemsetAsync(scratch, 0, 8 * total_words, st) : cudaSuccess;
-  size_t at = 0;
-  for (int w = 0; w < k && ce == cudaSuccess; ++w) {
-    const uint32_t tiles = tlc::decode_tiles_max(in_caps[w], g);
-    ce = tlc::launch_decode(*dev, ins[w], in_lens ? in_lens + w : nullptr, in_caps[w], n, acc,
-                            true, status_ptr, wait_limit(), base + at, st);
-    at += tlc::decode_scratch_words(tiles);
+  Scratch sc;
+  const uint32_t tiles0 = tlc::decode_tiles_max(in_caps[0], g);
+  if (k == 1 && !tlc::decode_deferred(tiles0)) {
+    // one small stream: one launch with a look-back
+    const size_t words = tlc::decode_scratch_words(tiles0);
+    const size_t bytes = tlc::align_up(8 * words + 8, 256);
+    if (scratch_alloc(*dev, bytes, &scratch, st, sc) != cudaSuccess) return TLC_ERR_CUDA;
+    uint64_t *base = static_cast<uint64_t *>(scratch);
+    int32_t *status_ptr = dev_status ? dev_status : reinterpret_cast<int32_t *>(base + words);
+    ce = cudaMemsetAsync(scratch, 0, 8 * words, st);
+    if (ce == cudaSuccess)
+      ce = tlc::launch_decode(*dev, ins[0], in_lens, in_caps[0], n, acc, true, status_ptr,
+                              wait_limit(), base, st);
+  } else {
+    // index + one read-modify-write of acc per pass of up to kIndexPass
+    // streams; passes run in stream order on `stream`, so the sum keeps
+    // the worker order
+    const int passes = (k + tlc::kIndexPass - 1) / tlc::kIndexPass;
+    std::vector<tlc::IndexedStream> is(k);
+    for (int w = 0; w < k; ++w) is[w] = {ins[w], in_lens ? in_lens + w : nullptr, in_caps[w]};
+    size_t bytes = 0;
+    for (int p = 0; p < passes; ++p) {
+      const int kp = std::min(tlc::kIndexPass, k - p * tlc::kIndexPass);
+      bytes = std::max(bytes, tlc::indexed_layout(&is[p * tlc::kIndexPass], kp, n).total_bytes);
+    }
+    if (scratch_alloc(*dev, bytes + 256, &scratch, st, sc) != cudaSuccess) return TLC_ERR_CUDA;
+    int32_t *status_ptr =
+        dev_status ? dev_status : reinterpret_cast<int32_t *>(static_cast<char *>(scratch) + bytes);
+    ce = cudaSuccess;
+    for (int p = 0; p < passes && ce == cudaSuccess; ++p) {
+      const int kp = std::min(tlc::kIndexPass, k - p * tlc::kIndexPass);
+      ce = tlc::launch_decode_indexed(*dev, &is[p * tlc::kIndexPass], kp, n, acc, true,
+                                      status_ptr, wait_limit(), scratch, st);
+    }
   }
-  const cudaError_t fe = cudaFreeAsync(scratch, st);
+  const cudaError_t fe = scratch_free(sc, st);
   return (ce == cudaSuccess && fe == cudaSuccess) ? TLC_OK : TLC_ERR_CUDA;
 }
 
@@ -352,7 +474,7 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   std::vector<tlc::BatchChunk> chunks;
   std::vector<uint32_t> qtt, dtt;
   std::vector<uint64_t> offsets(count + 1, 0);
-  uint64_t n_dchunks = 0, n_qchunks = 0;
+  uint64_t n_dchunks = 0, n_qchunks = 0, n_off = 0, n_pages = 0;
   for (int i = 0; i < count; ++i) {
     tlc::BatchTensor &t = T[i];
     t.x = xs ? xs[i] : nullptr;
@@ -374,12 +496,16 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
     t.d_chunk_begin = (uint32_t)n_dchunks;
     t.d_chunks = (t.d_tiles + tlc::kDecodeChunkUnits - 1) / tlc::kDecodeChunkUnits;
     n_dchunks += t.d_chunks;
+    t.d_off_begin = (uint32_t)n_off;
+    n_off += (uint64_t)t.d_tiles + 1;
+    t.d_page_begin = (uint32_t)n_pages;
+    n_pages += tlc::decode_pages(t.groups);
     t.vec_q = xs && (((reinterpret_cast<uintptr_t>(t.x) | reinterpret_cast<uintptr_t>(t.err)) &
                       15) == 0);
     t.vec_y = ys && ((reinterpret_cast<uintptr_t>(t.y) & 15) == 0);
     for (uint64_t b = 0; b < t.n; b += tlc::kBatchChunk) chunks.push_back({(uint32_t)i, 0u, b});
     if (qtt.size() >= (1ull << 31) || dtt.size() >= (1ull << 31) ||
-        chunks.size() >= (1ull << 31))
+        chunks.size() >= (1ull << 31) || n_off >= (1ull << 31) || n_pages >= (1ull << 31))
       return TLC_ERR_INVALID_ARG;
   }
   // device layout: tables, then the zeroed-per-call scratch of each direction
@@ -389,10 +515,14 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   const size_t sz_D = tlc::align_up(4 * dtt.size(), 256);
   const size_t sz_M = tlc::align_up(4 * (size_t)count + 8, 256);      // mbits, q_ticket
   const size_t sz_QS = tlc::align_up(8 * qtt.size(), 256);
-  const size_t sz_DS = tlc::align_up(8 * (dtt.size() + 1), 256);     // d_ticket, d_status
+  // decode: tickets, per-tensor valid flags, look-back words (per unit for
+  // small plans, per index chunk for indexed ones), zeroed per call
+  const bool d_ix = tlc::decode_deferred((uint32_t)dtt.size());
+  const size_t d_head = tlc::align_up(8 + 4 * (size_t)count, 8);
+  const size_t sz_DS = tlc::align_up(d_head + 8 * dtt.size(), 256);
   const size_t sz_P = tlc::align_up(sizeof(tlc::BatchPrep) * count + 8, 256);  // prep, total
-  const size_t sz_E = tlc::align_up(4 * dtt.size(), 256);            // counting pass
-  const size_t sz_S = tlc::align_up(8 * n_dchunks, 256);
+  const size_t sz_E = d_ix ? tlc::align_up(4 * n_off, 256) : 0;      // index: units' first groups
+  const size_t sz_S = d_ix ? tlc::align_up(4 * n_pages, 256) : 0;    // index: page tables
   // deferred placement of the compress side: chunk summaries, staging
   const bool q_def = xs && tlc::compress_deferred_tiles(qtt.size());
   const size_t sz_QC = q_def ? tlc::align_up(8 * n_qchunks, 256) : 0;
@@ -427,14 +557,16 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   D.q_zero_bytes = sz_M + 8 * qtt.size();
   char *zd = zq + sz_M + sz_QS;
   D.d_ticket = reinterpret_cast<uint32_t *>(zd);
-  D.d_status = reinterpret_cast<uint64_t *>(zd + 8);
+  D.d_ticket2 = reinterpret_cast<uint32_t *>(zd + 4);
+  D.d_ok = reinterpret_cast<uint32_t *>(zd + 8);
+  D.d_status = reinterpret_cast<uint64_t *>(zd + d_head);
   D.d_zero_base = zd;
-  D.d_zero_bytes = 8 * (dtt.size() + 1);
+  D.d_zero_bytes = d_head + 8 * (d_ix ? n_dchunks : dtt.size());
   D.d_prep = reinterpret_cast<tlc::BatchPrep *>(zd + sz_DS);
   D.d_total = reinterpret_cast<uint32_t *>(zd + sz_DS + sizeof(tlc::BatchPrep) * count);
   P->spare_status = reinterpret_cast<int32_t *>(zd + sz_DS + sz_P);
-  D.d_ecount = reinterpret_cast<uint32_t *>(zd + sz_DS + sz_P + 256);
-  D.d_csum = reinterpret_cast<uint64_t *>(zd + sz_DS + sz_P + 256 + sz_E);
+  D.d_off = d_ix ? reinterpret_cast<uint32_t *>(zd + sz_DS + sz_P + 256) : nullptr;
+  D.d_page = d_ix ? reinterpret_cast<uint32_t *>(zd + sz_DS + sz_P + 256 + sz_E) : nullptr;
   D.n_d_chunks = (uint32_t)n_dchunks;
   D.q_deferred = q_def;
   D.q_cagg = q_def ? reinterpret_cast<uint64_t *>(zd + sz_DS + sz_P + 256 + sz_E + sz_S) : nullptr;
@@ -515,14 +647,15 @@ static tlc_status run_wait_test(bool compress_side, uint32_t max_polls, int32_t 
   if (!dev) return TLC_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   void *scratch = nullptr;
-  if (scratch_alloc(*dev, 256, &scratch, st) != cudaSuccess) return TLC_ERR_CUDA;
+  Scratch sc;
+  if (scratch_alloc(*dev, 256, &scratch, st, sc) != cudaSuccess) return TLC_ERR_CUDA;
   ce = cudaMemsetAsync(scratch, 0, 256, st);
   if (ce == cudaSuccess)
     ce = compress_side
              ? tlc::launch_compress_wait_test(static_cast<uint64_t *>(scratch), max_polls,
                                               dev_status, st)
              : tlc::launch_wait_test(static_cast<uint64_t *>(scratch), max_polls, dev_status, st);
-  const cudaError_t fe = cudaFreeAsync(scratch, st);
+  const cudaError_t fe = scratch_free(sc, st);
   return (ce == cudaSuccess && fe == cudaSuccess) ? TLC_OK : TLC_ERR_CUDA;
 }
 

@@ -49,10 +49,13 @@
 // emitted(t) = (all ? floor : ceil)((t + A) / 14) + R
 // t_out(t)   = all ? (t + A) mod 14 : tc
 // Two segments compose associatively (see compose()).
+#define TLC_TU 1
 #include "tlc_device.cuh"
 #include "tlc_internal.h"
 
 namespace tlc {
+
+TLC_DEFINE_DEBUG_READER(debug_fault_compress)
 
 // ------------------------------------------------------------ k_absmax ----
 constexpr int kAbsThreads = 512;
@@ -66,7 +69,8 @@ template <bool kVec>
 __global__ void __launch_bounds__(kAbsThreads)
 k_absmax(const float *__restrict__ x, const float *__restrict__ err, uint64_t n,
          uint32_t *__restrict__ partial, uint64_t *__restrict__ zero_words,
-         uint32_t n_zero) {
+         uint32_t n_zero, CompressRecord *rec) {
+  if (rec && blockIdx.x == 0 && threadIdx.x == 0) rec->nonzeros = 0;
   uint32_t m = 0;
   const uint64_t gtid = (uint64_t)blockIdx.x * kAbsThreads + threadIdx.x;
   const uint64_t nth = (uint64_t)gridDim.x * kAbsThreads;
@@ -309,6 +313,7 @@ struct TileJob {
   uint64_t *status;   // this tensor's tile status words
   uint32_t n_tiles;
   bool vec;           // x and err are 16-byte aligned
+  CompressRecord *rec;  // or nullptr: the call's record (non-zero count, length)
 };
 
 // The deferred-placement path's buffers for one tensor.
@@ -325,10 +330,11 @@ struct QuantSmem {
   __align__(16) uint32_t tile[kTileGroups / 4];          // the tile's quartic bytes
   uint32_t scan[kQWarps + 1];
   uint32_t A, cin, tin, last;
+  uint32_t nzw[kQWarps];  // per-warp non-zero counts of a tile (recording calls)
 };
 
 __device__ __forceinline__ void put_out(const TileJob &j, uint64_t pos, uint8_t v) {
-  if (4 + pos < j.out_cap) j.out[4 + pos] = v;
+  if (TLC_BOUND(4 + pos < j.out_cap)) j.out[4 + pos] = v;
 }
 
 // Decoupled look-back for item t of a single-pass scan over status words,
@@ -475,6 +481,7 @@ __device__ __forceinline__ void finish_tile(const TileJob &j, uint32_t t, const 
     eval_agg(C, tt, agg);
     if (tt) put_out(j, C, remainder_byte(tt));
     *j.out_len = 4ull + C + (tt ? 1u : 0u);
+    if (j.rec) j.rec->length = 4ull + C + (tt ? 1u : 0u);
   }
 }
 
@@ -482,9 +489,17 @@ __device__ __forceinline__ void finish_tile(const TileJob &j, uint32_t t, const 
 // the 128 quartic bytes of these values, four per lane, returned packed
 // (lane L holds groups 4L..4L+3 of the step).  `dig` is this warp's 640-byte
 // shared buffer of digits.  Values past n count as zero (digit 1).
+// Values with a non-zero digit among four digits (one per byte, 0..2, 1 is zero).
+__device__ __forceinline__ uint32_t nonzero_digits(uint32_t dw) {
+  const uint32_t x = dw ^ 0x01010101u;
+  return __popc((x | (x >> 1)) & 0x01010101u);
+}
+
+// kCount: also add the number of non-zero q of the step's values to nz.
+template <bool kCount>
 __device__ __forceinline__ uint32_t quant_chunk(const float *x, float *err, uint64_t n,
                                                 uint64_t e0, bool vec_full, float scale,
-                                                float thr, uint32_t *dig) {
+                                                float thr, uint32_t *dig, uint32_t &nz) {
   const int lane = threadIdx.x & 31;
   if (vec_full) {
     const float4 *x4 = reinterpret_cast<const float4 *>(x + e0);
@@ -505,6 +520,7 @@ __device__ __forceinline__ uint32_t quant_chunk(const float *x, float *err, uint
       dw |= quant_digit(__fadd_rn(xv[k].w, ev[k].w), scale, thr, o.w) << 24;
       err4[lane + 32 * k] = o;
       dig[lane + 32 * k] = dw;
+      if (kCount) nz += nonzero_digits(dw);
     }
   } else if (e0 < n) {
     // tail or unaligned step: scalar and bounds-checked
@@ -523,6 +539,7 @@ __device__ __forceinline__ uint32_t quant_chunk(const float *x, float *err, uint
         dw |= d << (8 * q);
       }
       dig[lane + 32 * k] = dw;
+      if (kCount) nz += nonzero_digits(dw);
     }
   } else {
     // step entirely past the end: all-zero groups
@@ -620,6 +637,11 @@ __device__ __forceinline__ void zre_encode_tile(const TileJob &j, const DeferJob
     if (threadIdx.x == 0) dj.aggs[t] = pack_agg32(agg);
     uint8_t *st = dj.stage + (uint64_t)t * kTileGroups;
     uint32_t k_out = off;
+    // a tile emits at most one byte per group after its leading run
+    auto stage = [&](uint8_t v) {
+      if (TLC_CHECK(k_out < (uint32_t)kTileGroups)) st[k_out] = v;
+      ++k_out;
+    };
     int prev = prev_in;
 #pragma unroll
     for (int k = 0; k < kZB; ++k) {
@@ -628,15 +650,15 @@ __device__ __forceinline__ void zre_encode_tile(const TileJob &j, const DeferJob
       if (p >= (int)tgv) break;
       if (prev < 0) {
         if (b != 121u) {  // the tile's first literal; the run before it is placed later
-          st[k_out++] = (uint8_t)b;
+          stage((uint8_t)b);
           prev = p;
         }
       } else if (b == 121u) {
-        if ((p - prev - 1) % 14 == 13) st[k_out++] = 255;
+        if ((p - prev - 1) % 14 == 13) stage(255);
       } else {
         const uint32_t r = (uint32_t)(p - 1 - prev) % 14u;
-        if (r) st[k_out++] = remainder_byte(r);
-        st[k_out++] = (uint8_t)b;
+        if (r) stage(remainder_byte(r));
+        stage((uint8_t)b);
         prev = p;
       }
     }
@@ -680,7 +702,8 @@ __device__ __forceinline__ void zre_encode_tile(const TileJob &j, const DeferJob
 // One tile of 4096 byte groups (20480 values) of one tensor, fused: quantize
 // and update the error buffer, pack the quartic bytes into shared memory,
 // then zero-run encode them.  Whole block; ends synchronised.
-template <bool kDeferred = false>
+// kCount: the tile's non-zero values are added to the call's record.
+template <bool kDeferred = false, bool kCount = false>
 __device__ __forceinline__ void quant_tile(const TileJob &j, const DeferJob &dj, uint32_t t,
                                            float scale, float thr,
                                            QuantSmem &sm, int32_t *dev_status,
@@ -691,14 +714,26 @@ __device__ __forceinline__ void quant_tile(const TileJob &j, const DeferJob &dj,
   const uint32_t tgv = (uint32_t)umin64(kTileGroups, j.groups - g0);
   const uint64_t e_tile = g0 * 5;
   const bool full = j.vec && (e_tile + kTileElems <= j.n);
+  uint32_t nz = 0;
 #pragma unroll 1
   for (int it = 0; it < kQIters; ++it) {
     const int c = it * kQWarps + warp;
     const uint64_t e0 = e_tile + (uint64_t)c * kChunkElems;
     sm.tile[c * (kChunkGroups / 4) + lane] =
-        quant_chunk(j.x, j.err, j.n, e0, full, scale, thr, sm.dig[warp]);
+        quant_chunk<kCount>(j.x, j.err, j.n, e0, full, scale, thr, sm.dig[warp], nz);
+  }
+  if (kCount) {
+    nz = __reduce_add_sync(0xffffffffu, nz);
+    if (lane == 0) sm.nzw[warp] = nz;
   }
   __syncthreads();
+  if (kCount && threadIdx.x == 0) {
+    uint32_t tot = 0;
+#pragma unroll
+    for (int w = 0; w < kQWarps; ++w) tot += sm.nzw[w];
+    if (tot) atomicAdd(reinterpret_cast<unsigned long long *>(&j.rec->nonzeros),
+                       (unsigned long long)tot);
+  }
   uint32_t qw[kZWords];
   if constexpr (kZWords == 2) {
     const uint2 q2 = reinterpret_cast<const uint2 *>(sm.tile)[threadIdx.x];
@@ -780,6 +815,7 @@ struct QuantArgs {
   uint32_t n_tiles;
   int32_t *dev_status;
   uint32_t max_polls;
+  CompressRecord *rec;  // or nullptr
 };
 
 #if TLC_Q_MINB > 1
@@ -788,7 +824,8 @@ struct QuantArgs {
 #define TLC_Q_BOUNDS __launch_bounds__(kQThreads)
 #endif
 
-template <bool kVec, bool kDeferred>
+// kRecord: the call asked for a record (M, scale, non-zero count, length).
+template <bool kVec, bool kDeferred, bool kRecord = false>
 __global__ void TLC_Q_BOUNDS k_quant_zre(const QuantArgs a) {
   __shared__ QuantSmem sm;
   __shared__ uint32_t tile_id_s;
@@ -805,6 +842,10 @@ __global__ void TLC_Q_BOUNDS k_quant_zre(const QuantArgs a) {
       ok_s = scale_from_max(mb, a.s, scale, thr) ? 1 : 0;
       scale_s = scale;
       thr_s = thr;
+      if (kRecord && blockIdx.x == 0) {
+        a.rec->m_bits = mb;
+        a.rec->scale = ok_s ? scale : 0.0f;
+      }
     }
   }
   __syncthreads();
@@ -813,19 +854,20 @@ __global__ void TLC_Q_BOUNDS k_quant_zre(const QuantArgs a) {
     if (blockIdx.x == 0 && threadIdx.x == 0) {
       report(a.dev_status, TLC_ERR_NONFINITE);
       *a.out_len = 0;
+      if (kRecord) a.rec->length = 0;
     }
     return;
   }
   const float scale = scale_s, thr = thr_s;
   const TileJob job = {a.x, a.err, a.n, a.groups, a.out, a.out_cap, a.out_len,
-                       a.status, a.n_tiles, kVec};
+                       a.status, a.n_tiles, kVec, kRecord ? a.rec : nullptr};
   const DeferJob djob = {a.aggs, a.stage, a.ccount, a.cagg};
   for (;;) {
     if (threadIdx.x == 0) tile_id_s = atomicAdd(a.ticket, 1u);
     __syncthreads();
     const uint32_t t = tile_id_s;
     if (t >= a.n_tiles) break;
-    quant_tile<kDeferred>(job, djob, t, scale, thr, sm, a.dev_status, a.max_polls);
+    quant_tile<kDeferred, kRecord>(job, djob, t, scale, thr, sm, a.dev_status, a.max_polls);
   }
 }
 
@@ -879,7 +921,7 @@ static_assert(kPlaceTiles % kPlaceBlockTiles == 0, "blocks do not straddle chunk
 __global__ void __launch_bounds__(kPlaceThreads)
 k_zre_place(const uint32_t *__restrict__ aggs, const uint64_t *__restrict__ cagg,
             uint32_t n_tiles, const uint32_t *ok, const uint8_t *__restrict__ stage, uint8_t *out,
-            uint64_t out_cap, uint64_t *out_len) {
+            uint64_t out_cap, uint64_t *out_len, CompressRecord *rec) {
   __shared__ uint32_t tC[kPlaceBlockTiles], tT[kPlaceBlockTiles], tA[kPlaceBlockTiles];
   if (!*ok) return;  // non-finite step: nothing was encoded
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -939,8 +981,9 @@ k_zre_place(const uint32_t *__restrict__ aggs, const uint64_t *__restrict__ cagg
     if (t0 + nv == n_tiles && (uint32_t)lane == nv - 1 && k < kPlaceBlockTiles) {
       // the stream's end: state after the last tile
       eval_agg(C, tt, v.a);
-      if (tt && 4ull + C < out_cap) out[4 + C] = remainder_byte(tt);
+      if (tt && TLC_BOUND(4ull + C < out_cap)) out[4 + C] = remainder_byte(tt);
       *out_len = 4ull + C + (tt ? 1u : 0u);
+      if (rec) rec->length = 4ull + C + (tt ? 1u : 0u);
     }
   }
   __syncthreads();
@@ -953,8 +996,9 @@ k_zre_place(const uint32_t *__restrict__ aggs, const uint64_t *__restrict__ cagg
   const bool rem = !a.all && r;  // the run ends in the tile with a remainder
   uint8_t *o = out + 4ull + C;
   const uint64_t room = out_cap > 4ull + C ? out_cap - 4ull - C : 0;
+  (void)TLC_CHECK((uint64_t)lead + a.R <= room);  // the tile's bytes fit the stream
   warp_fill_255(o, (uint32_t)umin64(lead - (rem ? 1u : 0u), room), lane);
-  if (rem && lane == 0 && lead - 1 < room) o[lead - 1] = remainder_byte(r);
+  if (rem && lane == 0 && TLC_BOUND(lead - 1 < room)) o[lead - 1] = remainder_byte(r);
   if (lead < room)
     warp_copy(o + lead, stage + (uint64_t)t * kTileGroups, (uint32_t)umin64(a.R, room - lead),
               lane);
@@ -1057,7 +1101,8 @@ __global__ void TLC_Q_BOUNDS k_quant_zre_batch(const BatchQuantArgs a) {
       continue;
     }
     const TileJob job = {T.x,   T.err, T.n, T.groups, a.arena + T.arena_off, T.cap,
-                         a.out_lens + id, a.status + T.q_tile_begin, T.q_tiles, T.vec_q != 0};
+                         a.out_lens + id, a.status + T.q_tile_begin, T.q_tiles, T.vec_q != 0,
+                         nullptr};
     if (kDeferred) {
       const DeferJob dj = {a.aggs + T.q_tile_begin,
                            a.stage + (uint64_t)T.q_tile_begin * kTileGroups,
@@ -1134,7 +1179,7 @@ __global__ void __launch_bounds__(kPlaceThreads) k_zre_place_batch(const BatchQu
   if (t == T.q_tiles - 1 && lane == 0) {
     uint32_t Ce = C, te = tt;
     eval_agg(Ce, te, ag);
-    if (te && 4ull + Ce < out_cap) out[4 + Ce] = remainder_byte(te);
+    if (te && TLC_BOUND(4ull + Ce < out_cap)) out[4 + Ce] = remainder_byte(te);
     a.out_lens[id] = 4ull + Ce + (te ? 1u : 0u);
   }
   const uint32_t lead = lead_count(ag, tt);
@@ -1142,8 +1187,9 @@ __global__ void __launch_bounds__(kPlaceThreads) k_zre_place_batch(const BatchQu
   const bool rem = !ag.all && r;
   uint8_t *o = out + 4ull + C;
   const uint64_t room = out_cap > 4ull + C ? out_cap - 4ull - C : 0;
+  (void)TLC_CHECK((uint64_t)lead + ag.R <= room);  // the tile's bytes fit the stream
   warp_fill_255(o, (uint32_t)umin64(lead - (rem ? 1u : 0u), room), lane);
-  if (rem && lane == 0 && lead - 1 < room) o[lead - 1] = remainder_byte(r);
+  if (rem && lane == 0 && TLC_BOUND(lead - 1 < room)) o[lead - 1] = remainder_byte(r);
   if (lead < room)
     warp_copy(o + lead, a.stage + (uint64_t)u * kTileGroups, (uint32_t)umin64(ag.R, room - lead),
               lane);
@@ -1195,7 +1241,7 @@ uint32_t compress_place_chunks(uint32_t n_tiles) { return (n_tiles + kPlaceTiles
 cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, float s,
                             float *err, uint8_t *out, uint64_t out_cap, uint64_t *out_len,
                             int32_t *dev_status, uint32_t max_polls, void *scratch,
-                            cudaStream_t stream, bool deferred) {
+                            cudaStream_t stream, bool deferred, CompressRecord *rec) {
   const uint32_t n_tiles = compress_tiles(n);
   const uint32_t n_part = compress_partials(dev, n);
   CompressScratch sc = compress_scratch_layout(scratch, n_part, n_tiles);
@@ -1206,10 +1252,10 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
   timing_begin(kKindAbsmax, stream);
   if (vec)
     k_absmax<true><<<n_part, kAbsThreads, 0, stream>>>(x, err, n, sc.partial, sc.status,
-                                                        n_tiles + 1);
+                                                        n_tiles + 1, rec);
   else
     k_absmax<false><<<n_part, kAbsThreads, 0, stream>>>(x, err, n, sc.partial, sc.status,
-                                                         n_tiles + 1);
+                                                         n_tiles + 1, rec);
   timing_end(kKindAbsmax, stream);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1230,6 +1276,7 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
   qa.n_tiles = n_tiles;
   qa.dev_status = dev_status;
   qa.max_polls = max_polls;
+  qa.rec = rec;
 
   // the deferred path keeps its tile summaries (u32 each) and then its
   // chunk counters where the look-back words would be: k_absmax clears
@@ -1254,7 +1301,10 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
   if (grid > n_tiles) grid = n_tiles;
   timing_begin(kKindQuantZre, stream);
   if (deferred) {
-    if (vec)
+    if (rec)
+      (vec ? k_quant_zre<true, true, true> : k_quant_zre<false, true, true>)
+          <<<grid, kQThreads, 0, stream>>>(qa);
+    else if (vec)
       k_quant_zre<true, true><<<grid, kQThreads, 0, stream>>>(qa);
     else
       k_quant_zre<false, true><<<grid, kQThreads, 0, stream>>>(qa);
@@ -1262,10 +1312,13 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
     timing_begin(kKindZrePlace, stream);
     const uint32_t n_blocks = (n_tiles + kPlaceBlockTiles - 1) / kPlaceBlockTiles;
     k_zre_place<<<n_blocks, kPlaceThreads, 0, stream>>>(qa.aggs, ds.cagg, n_tiles, ds.ok,
-                                                         ds.stage, out, out_cap, out_len);
+                                                         ds.stage, out, out_cap, out_len, rec);
     timing_end(kKindZrePlace, stream);
   } else {
-    if (vec)
+    if (rec)
+      (vec ? k_quant_zre<true, false, true> : k_quant_zre<false, false, true>)
+          <<<grid, kQThreads, 0, stream>>>(qa);
+    else if (vec)
       k_quant_zre<true, false><<<grid, kQThreads, 0, stream>>>(qa);
     else
       k_quant_zre<false, false><<<grid, kQThreads, 0, stream>>>(qa);

@@ -6,34 +6,51 @@
 // q * M * s); the Abstract's exchange of state changes between nodes is the
 // receive side, where several workers' streams are summed.
 //
-// One kernel, k_decode, in two modes:
+// Two modes:
 //   kWrite       dense output: y_i = +scale, -scale or +0.0
 //   kAccumulate  acc_i += y_i only where q_i != 0 (acc keeps its bits at
-//                zeros), one launch per worker stream, in worker order
-// A tile is 1024 (kWrite) or 2048 (kAccumulate) payload bytes.  Per tile:
-// expansion counts e_k (an escape byte b >= 243 stands for b - 241 groups of
-// 121, any other byte for itself), a block scan, and a decoupled look-back
-// over earlier tiles for the tile's first group index O.  The tile's groups
-// are then expanded in shared memory (at most 14 bytes per payload byte) and
-// walked as float4 columns with coalesced 128-bit accesses: written in kWrite
-// mode, read-modify-written (all-zero columns skipped) in kAccumulate mode.
-// An accumulate tile made mostly of escapes instead visits only its literal
-// groups, so there work and traffic follow the non-zeros.
-// For streams whose capacity holds 16384 or more 512-byte units (8 MiB), a
-// counting kernel, k_decode_count, first writes the group count of every
-// unit and of every 32-unit chunk; each tile then sums the counts before it
-// (every thread a strided share) instead of looking back.  No tile waits on
-// another, which measured 0.789 -> 0.459 ms (dense output) and 0.629 ->
-// 0.505 ms (accumulate) on a dense 2^28-value stream, and 0.189 -> 0.178 /
-// 0.040 -> 0.026 ms on the sparse config-3 stream, for about 0.011 ms per
-// counting launch.  Below that size the extra launch costs more than the
-// look-back on sparse streams.
-// Every write is clamped to the ceil(n/5) groups of the tensor; a stream that
-// does not expand to exactly that many groups is reported as corrupt.
+//                zeros), streams in worker order
+//
+// Small streams (capacity below 8 MiB), one stream at a time: k_decode, one
+// launch.  A tile is 512 (kWrite) or 2048 (kAccumulate) payload bytes: per
+// tile, expansion counts e_k (an escape byte b >= 243 stands for b - 241
+// groups of 121, any other byte for itself), a block scan, and a decoupled
+// look-back over earlier tiles for the tile's first group index.
+//
+// Large streams, and several streams summed in one pass: an index, then the
+// decode.
+//   k_decode_index  per 32-unit chunk of 512-byte payload units: the units'
+//                   group counts, a decoupled look-back over the chunks for
+//                   the chunk's first group, then every unit's first group
+//                   (off[u]) and, for every 1024th group, the unit that holds
+//                   it (page[p]).  The last chunk checks that the stream
+//                   expands to exactly ceil(n/5) groups and marks it valid.
+//   k_decode_ix     no cross-block wait.  Each stream is decoded in one of
+//                   two tilings, chosen on the device from its density:
+//     payload tiles  (sparse streams, more than 4 groups per payload byte on
+//                    average): a tile is a fixed run of payload bytes whose
+//                    first group is off[] of its first unit; an accumulate
+//                    tile made mostly of escapes visits only its literal
+//                    groups, so the work follows the non-zeros.
+//     gather tiles   (denser streams, and always when several streams are
+//                    summed): a tile is a fixed run of output groups.  Its
+//                    first unit comes from page[]; one warp per unit scans
+//                    the unit's bytes and places its literal groups into
+//                    shared memory (pre-filled with the zero group), then the
+//                    values are written (or read-modify-written once for all
+//                    streams, added in stream order) as coalesced float4s.
+//                    Every tile writes the same amount, however the stream's
+//                    bytes expand.
+// The quartic bytes live only in shared memory.  Every write is clamped to
+// the ceil(n/5) groups of the tensor; a stream that does not expand to
+// exactly that many groups is reported as corrupt and left out.
+#define TLC_TU 2
 #include "tlc_device.cuh"
 #include "tlc_internal.h"
 
 namespace tlc {
+
+TLC_DEFINE_DEBUG_READER(debug_fault_decode)
 
 // Payload bytes per thread (1, 2 or a multiple of 4): small tiles balance the dense
 // write mode best; the accumulate mode touches little memory per tile and
@@ -45,6 +62,7 @@ namespace tlc {
 #define TLC_D_BYTES_ACC 8
 #endif
 constexpr int kDThreads = 256;
+constexpr int kDWarps = kDThreads / kWarp;
 constexpr int kWrite = 0, kAccumulate = 1;
 template <int kMode>
 struct DecodeShape {
@@ -56,19 +74,24 @@ struct DecodeShape {
 #define TLC_D_LOOKV 1
 #endif
 constexpr int kLookV = TLC_D_LOOKV;   // look-back words per lane per round trip
-// Streams whose capacity allows this many 512-byte units or more get their
-// tile prefixes from a counting pass (k_decode_count) instead of a look-back.
+// Streams whose capacity allows this many 512-byte units or more are
+// decoded through the index.
 #ifndef TLC_DEFER_DECODE_MIN_TILES
 #define TLC_DEFER_DECODE_MIN_TILES 16384
 #endif
 constexpr uint32_t kDecodeDeferMinTiles = TLC_DEFER_DECODE_MIN_TILES;
-static_assert(kDecodeDeferMinTiles >= 4, "the deferred layout fits in tiles + 1 words");
+// Output groups per gather tile, summed over its streams (a tile of k
+// streams covers TLC_GT_ACC / k' groups, k' = k rounded up to 2, 4 or 8).
+#ifndef TLC_GT_ACC
+#define TLC_GT_ACC 16384
+#endif
+constexpr uint32_t kPage = 1024;  // groups per page-table entry
+static_assert(TLC_GT_ACC % (8 * kPage) == 0, "tiles are whole pages");
+static_assert(kDecodeUnit == 4 * kWarp * 4, "a unit is 16 bytes per lane of a warp");
 
 size_t decode_smem_bytes(bool accumulate);
 
 struct DecodeArgs {
-  uint32_t *ecount;        // deferred prefixes only: each 512-byte unit's group count
-  uint64_t *csum;          // and each 32-unit chunk's
   const uint8_t *in;
   const uint64_t *len_dev;
   uint64_t cap;
@@ -87,11 +110,21 @@ __device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
   return v;
 }
 
-// Exclusive prefix (in groups) of tile u, by warp 0.  Publishes the tile's
-// aggregate first and its inclusive prefix last.  Each round trip reads
-// 32 * kLookV earlier tiles' words.
+// Look-back words per lane per round trip of the index's chunk scan: the
+// index's blocks all start at once, so the first prefix spreads forward by
+// 32 * V chunks per round trip.
+#ifndef TLC_IX_LOOKV
+#define TLC_IX_LOOKV 8
+#endif
+
+// Exclusive prefix (a sum) of item u of a single-pass scan, by one warp.
+// Publishes the item's aggregate first and its inclusive prefix last.  Each
+// round trip reads 32 * V earlier items' words.  Every lane gets the
+// result.
+template <int V = kLookV>
 __device__ uint64_t lookback_sum(uint64_t *status, uint32_t u, uint64_t E, uint32_t max_polls,
                                  bool &timed_out) {
+  constexpr int kLookV = V;
   const int lane = threadIdx.x & 31;
   if (u == 0) {
     if (lane == 0) st_relaxed_u64(status, kFlagPrefix | E);
@@ -138,46 +171,35 @@ __device__ __forceinline__ float dequant(uint32_t dig, float scale) {
   return dig == 1u ? 0.0f : (dig == 2u ? scale : -scale);
 }
 
-// One stream's decode job, as the tile function sees it.
+__device__ __forceinline__ uint32_t expansion(uint32_t b) { return b >= 243u ? b - 241u : 1u; }
+
+// One stream's decode job, as the payload-tile function sees it.
 struct DecodeJob {
   const uint8_t *payload;  // stream bytes after the 4-byte header
   uint64_t m;              // payload length
   uint64_t n, groups;
   float scale;
   float *y;                // output (kWrite) or accumulation buffer
-  uint64_t *status;        // this stream's tile status words
+  uint64_t *status;        // look-back path: this stream's tile status words
   uint32_t n_tiles;        // tiles actually present: ceil(m / tile)
   bool vec;                // y is 16-byte aligned
-  const uint32_t *ecount;  // deferred prefixes: group count per 512-byte unit
-  const uint64_t *csum;    // and per chunk of kDecodeChunkUnits units
+  const uint32_t *off;     // indexed path: first group of every 512-byte unit
 };
-
-// Deferred prefixes: the first group index of the tile that starts at
-// payload unit `unit` is the sum of the counts that k_decode_count wrote for
-// the chunks before the unit's chunk and for the units before it in its
-// chunk.  Every thread of the block sums a strided share; the result is this
-// warp's partial sum (in every lane).  No wait.
-__device__ __forceinline__ uint64_t prefix_share(const uint32_t *ecount, const uint64_t *csum,
-                                                 uint32_t unit) {
-  const uint32_t c = unit / kDecodeChunkUnits;
-  uint64_t s = 0;
-  for (uint32_t i = threadIdx.x; i < c; i += kDThreads) s += csum[i];
-  const uint32_t t0 = c * kDecodeChunkUnits;
-  if (threadIdx.x < kDecodeChunkUnits && t0 + threadIdx.x < unit) s += ecount[t0 + threadIdx.x];
-  return warp_sum_u64(s);
-}
 
 struct DecodeSmem {
   uint16_t lut[256];       // base-3 digits of every quartic byte
   uint32_t scan[kDThreads / kWarp + 1];
   uint64_t o;
-  uint64_t part[kDThreads / kWarp];  // per-warp partial prefixes (counting pass)
 };
+
+__device__ __forceinline__ void fill_lut(uint16_t *lut) {
+  for (int v = threadIdx.x; v < 256; v += blockDim.x) lut[v] = v < 243 ? digits_of(v) : 0;
+}
 
 // Validate a stream (length and header) and return its payload length and
 // scale.  Corrupt when the length is below 4 or above the readable capacity,
 // the payload would be longer than the tensor's groups or empty, or the
-// header is negative or not finite.
+// header is negative or not finite (the encoder never writes such a header).
 __device__ __forceinline__ bool read_stream_header(const uint8_t *in, const uint64_t *len_dev,
                                                    uint64_t cap, uint64_t groups, uint64_t &m,
                                                    float &scale) {
@@ -191,16 +213,108 @@ __device__ __forceinline__ bool read_stream_header(const uint8_t *in, const uint
   return true;
 }
 
-// One tile of one stream; the whole block calls it and it ends synchronised.
-// kDeferred: the tile's first group index comes from k_decode_count's
-// counts instead of a look-back.
-template <int kMode, bool kDeferred = false>
+// Write values [e_begin, e_end) of groups whose quartic bytes sit in grp
+// (grp[0] is group g_first), or add their non-zero values in accumulate
+// mode.  Float4 columns with coalesced 128-bit accesses when y is 16-byte
+// aligned, single values at the edges.  Values 4v..4v+3 lie in group g =
+// 4v/5 (digits d0..) and, when d0 >= 2, spill into group g+1; both groups'
+// digit words are joined so one shift lines the four digits up.
+// The calling group of threads is a whole block (tid = threadIdx.x, nth =
+// blockDim.x) or a whole warp (tid = lane, nth = 32).
+template <int kMode>
+__device__ __forceinline__ void emit_values(const uint8_t *grp, uint64_t g_first,
+                                            uint64_t e_begin, uint64_t e_end, float *y, bool vec,
+                                            float scale, const uint16_t *lut,
+                                            uint32_t tid, uint32_t nth) {
+  if (e_end <= e_begin) return;
+  const uint32_t o32 = (uint32_t)g_first;
+  auto put = [&](uint64_t e) {
+    const uint32_t e32 = (uint32_t)e;
+    const uint32_t g = e32 / 5u;
+    const uint32_t dig = (lut[grp[g - o32]] >> (2 * (e32 - 5u * g))) & 3u;
+    if (kMode == kWrite)
+      y[e] = dequant(dig, scale);
+    else if (dig != 1u)
+      y[e] = __fadd_rn(y[e], dequant(dig, scale));
+  };
+  const uint64_t v0 = (e_begin + 3) / 4, v1 = e_end / 4;
+  if (!vec || v1 <= v0) {
+    for (uint64_t e = e_begin + tid; e < e_end; e += nth) put(e);
+    return;
+  }
+  float4 *y4 = reinterpret_cast<float4 *>(y);
+  for (uint64_t v = v0 + tid; v < v1; v += nth) {
+    const uint32_t e0 = (uint32_t)(4 * v);
+    const uint32_t g = e0 / 5u;
+    const uint32_t d0 = e0 - 5u * g;
+    const uint32_t li = g - o32;
+    const uint32_t c0 = grp[li];
+    const uint32_t c1 = d0 >= 2u ? (uint32_t)grp[li + 1] : 121u;
+    if (kMode == kWrite) {
+      float4 o;
+      if (c0 == 121u && c1 == 121u) {
+        o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      } else {
+        const uint32_t w = ((uint32_t)lut[c0] | ((uint32_t)lut[c1] << 10)) >> (2u * d0);
+        o.x = dequant(w & 3u, scale);
+        o.y = dequant((w >> 2) & 3u, scale);
+        o.z = dequant((w >> 4) & 3u, scale);
+        o.w = dequant((w >> 6) & 3u, scale);
+      }
+      y4[v] = o;
+    } else if (c0 != 121u || c1 != 121u) {
+      const uint32_t w = ((uint32_t)lut[c0] | ((uint32_t)lut[c1] << 10)) >> (2u * d0);
+      if ((w & 0xffu) != 0x55u) {  // some of the four digits is not zero
+        float4 o = y4[v];
+        if ((w & 3u) != 1u) o.x = __fadd_rn(o.x, dequant(w & 3u, scale));
+        if (((w >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, dequant((w >> 2) & 3u, scale));
+        if (((w >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, dequant((w >> 4) & 3u, scale));
+        if (((w >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, dequant((w >> 6) & 3u, scale));
+        y4[v] = o;
+      }
+    }
+  }
+  if (tid < 4) {
+    const uint64_t e = e_begin + tid;
+    if (e < 4 * v0) put(e);
+  } else if (tid < 8) {
+    const uint64_t e = 4 * v1 + (tid - 4);
+    if (e < e_end) put(e);
+  }
+}
+
+// Zeros over values [e_begin, e_end) (dense output of all-zero groups), by
+// a block or a warp as emit_values.
+__device__ __forceinline__ void emit_zeros(uint64_t e_begin, uint64_t e_end, float *y, bool vec,
+                                           uint32_t tid, uint32_t nth) {
+  if (e_end <= e_begin) return;
+  const uint64_t v0 = (e_begin + 3) / 4, v1 = e_end / 4;
+  if (!vec || v1 <= v0) {
+    for (uint64_t e = e_begin + tid; e < e_end; e += nth) y[e] = 0.0f;
+    return;
+  }
+  float4 *y4 = reinterpret_cast<float4 *>(y);
+  for (uint64_t v = v0 + tid; v < v1; v += nth) y4[v] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  if (tid < 4) {
+    const uint64_t e = e_begin + tid;
+    if (e < 4 * v0) y[e] = 0.0f;
+  } else if (tid < 8) {
+    const uint64_t e = 4 * v1 + (tid - 4);
+    if (e < e_end) y[e] = 0.0f;
+  }
+}
+
+// One payload tile of one stream; the whole block calls it and it ends
+// synchronised.  kIndexed: the tile's first group index is off[] of its first
+// unit (written by k_decode_index) instead of a look-back.
+template <int kMode, bool kIndexed>
 __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, DecodeSmem &sm,
                                             uint8_t *grp_s, int32_t *dev_status,
                                             uint32_t max_polls) {
   constexpr int kDBytes = DecodeShape<kMode>::kBytes;
   constexpr int kDTile = DecodeShape<kMode>::kTile;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  static_assert(kDTile % kDecodeUnit == 0, "tiles are whole units");
+  const int warp = threadIdx.x >> 5;
   const float scale = j.scale;
 
   // ---- load the tile's payload bytes, expansion counts, block scan -------
@@ -231,7 +345,7 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
   for (int k = 0; k < kDBytes; ++k) {
     const uint32_t b = (bw[k >> 2] >> (8 * (k & 3))) & 0xffu;
     if (k < nvalid) {
-      esum += b >= 243u ? b - 241u : 1u;
+      esum += expansion(b);
       mine_lit = mine_lit || (b < 243u && b != 121u);
     }
   }
@@ -247,14 +361,10 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
   const bool expand = any_lit && (kMode == kWrite || E <= 4u * (uint32_t)kDTile);
 
   // ---- the tile's first group index ---------------------------------------
-  // Counting pass: every thread sums a strided share of the counts before
-  // the tile, then all threads pre-fill the zero groups.  Look-back: warp 0
-  // looks back while the other warps pre-fill.
-  if (kDeferred) {
-    static_assert(kDTile % kDecodeUnit == 0 && kDecodeChunkUnits % (kDTile / kDecodeUnit) == 0,
-                  "tiles are whole units and never straddle a chunk");
-    const uint64_t p = prefix_share(j.ecount, j.csum, u * (uint32_t)(kDTile / kDecodeUnit));
-    if (lane == 0) sm.part[warp] = p;
+  // Indexed: one load, while every thread pre-fills the zero groups.
+  // Look-back: warp 0 looks back while the other warps pre-fill.
+  if (kIndexed) {
+    if (threadIdx.x == 0) sm.o = __ldg(j.off + (uint64_t)u * (kDTile / kDecodeUnit));
     if (expand) {
       const uint32_t words = (E + 15) / 16;
       for (uint32_t w = threadIdx.x; w < words; w += kDThreads)
@@ -264,8 +374,8 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
   } else if (warp == 0) {
     bool timed_out = false;
     const uint64_t O = lookback_sum(j.status, u, E, max_polls, timed_out);
-    if (__any_sync(0xffffffffu, timed_out) && lane == 0) report(dev_status, TLC_ERR_TIMEOUT);
-    if (lane == 0) sm.o = O;
+    if (__any_sync(0xffffffffu, timed_out) && threadIdx.x == 0) report(dev_status, TLC_ERR_TIMEOUT);
+    if (threadIdx.x == 0) sm.o = O;
   } else if (expand) {
     const uint32_t words = (E + 15) / 16;
     for (uint32_t w = threadIdx.x - kWarp; w < words; w += kDThreads - kWarp)
@@ -273,42 +383,17 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
           make_uint4(0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u);
   }
   __syncthreads();
-  uint64_t O;
-  if (kDeferred) {
-    O = 0;
-#pragma unroll
-    for (int w = 0; w < kDThreads / kWarp; ++w) O += sm.part[w];
-  } else {
-    O = sm.o;
-  }
-  if (threadIdx.x == 0) {
+  const uint64_t O = sm.o;
+  if (!kIndexed && threadIdx.x == 0) {
+    // (the index already checked the indexed path's total)
     const bool last = (u == j.n_tiles - 1);
     if (O + E > j.groups || (last && O + E != j.groups)) report(dev_status, TLC_ERR_CORRUPT);
   }
   const uint64_t Ec = O >= j.groups ? 0 : umin64(E, j.groups - O);
 
   if (!any_lit) {
-    if (kMode == kWrite) {
-      const uint64_t e_begin = 5 * O;
-      const uint64_t e_end = umin64(5 * (O + Ec), j.n);
-      const uint64_t v0 = (e_begin + 3) / 4, v1 = e_end / 4;
-      if (e_end > e_begin) {
-        if (!j.vec || v1 <= v0) {
-          for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) j.y[e] = 0.0f;
-        } else {
-          float4 *y4 = reinterpret_cast<float4 *>(j.y);
-          for (uint64_t v = v0 + threadIdx.x; v < v1; v += kDThreads)
-            y4[v] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          if (threadIdx.x < 4) {
-            const uint64_t e = e_begin + threadIdx.x;
-            if (e < 4 * v0) j.y[e] = 0.0f;
-          } else if (threadIdx.x < 8) {
-            const uint64_t e = 4 * v1 + (threadIdx.x - 4);
-            if (e < e_end) j.y[e] = 0.0f;
-          }
-        }
-      }
-    }
+    if (kMode == kWrite)
+      emit_zeros(5 * O, umin64(5 * (O + Ec), j.n), j.y, j.vec, threadIdx.x, kDThreads);
   } else if (expand) {
     // literal bytes into the expanded group buffer
     uint32_t pos = off;
@@ -319,76 +404,15 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
         if (b >= 243u) {
           pos += b - 241u;
         } else {
-          grp_s[pos] = (uint8_t)b;
+          if (TLC_CHECK(pos < (uint32_t)DecodeShape<kMode>::kMaxGroups)) grp_s[pos] = (uint8_t)b;
           ++pos;
         }
       }
     }
     __syncthreads();
     // groups [O, O+Ec) -> values [5 O, min(5 (O+Ec), n))
-    const uint64_t e_begin = 5 * O;
-    const uint64_t e_end = umin64(5 * (O + Ec), j.n);
-    if (e_end > e_begin) {
-      const uint32_t o32 = (uint32_t)O;
-      // one value: written (dense output) or added where non-zero (accumulate)
-      auto put = [&](uint64_t e) {
-        const uint32_t e32 = (uint32_t)e;
-        const uint32_t g = e32 / 5u;
-        const uint32_t dig = (sm.lut[grp_s[g - o32]] >> (2 * (e32 - 5u * g))) & 3u;
-        if (kMode == kWrite)
-          j.y[e] = dequant(dig, scale);
-        else if (dig != 1u)
-          j.y[e] = __fadd_rn(j.y[e], dequant(dig, scale));
-      };
-      const uint64_t v0 = (e_begin + 3) / 4, v1 = e_end / 4;
-      if (!j.vec || v1 <= v0) {
-        for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) put(e);
-      } else {
-        // Values 4v..4v+3 lie in group g = 4v/5 (digits d0..) and, when
-        // d0 >= 2, spill into group g+1; both groups' digit words are joined
-        // so one shift lines the four digits up.
-        float4 *y4 = reinterpret_cast<float4 *>(j.y);
-        for (uint64_t v = v0 + threadIdx.x; v < v1; v += kDThreads) {
-          const uint32_t e0 = (uint32_t)(4 * v);
-          const uint32_t g = e0 / 5u;
-          const uint32_t d0 = e0 - 5u * g;
-          const uint32_t li = g - o32;
-          const uint32_t c0 = grp_s[li];
-          const uint32_t c1 = d0 >= 2u ? (uint32_t)grp_s[li + 1] : 121u;
-          if (kMode == kWrite) {
-            float4 o;
-            if (c0 == 121u && c1 == 121u) {
-              o = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            } else {
-              const uint32_t w =
-                  ((uint32_t)sm.lut[c0] | ((uint32_t)sm.lut[c1] << 10)) >> (2u * d0);
-              o.x = dequant(w & 3u, scale);
-              o.y = dequant((w >> 2) & 3u, scale);
-              o.z = dequant((w >> 4) & 3u, scale);
-              o.w = dequant((w >> 6) & 3u, scale);
-            }
-            y4[v] = o;
-          } else if (c0 != 121u || c1 != 121u) {
-            const uint32_t w = ((uint32_t)sm.lut[c0] | ((uint32_t)sm.lut[c1] << 10)) >> (2u * d0);
-            if ((w & 0xffu) != 0x55u) {  // some of the four digits is not zero
-              float4 o = y4[v];
-              if ((w & 3u) != 1u) o.x = __fadd_rn(o.x, dequant(w & 3u, scale));
-              if (((w >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, dequant((w >> 2) & 3u, scale));
-              if (((w >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, dequant((w >> 4) & 3u, scale));
-              if (((w >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, dequant((w >> 6) & 3u, scale));
-              y4[v] = o;
-            }
-          }
-        }
-        if (threadIdx.x < 4) {
-          const uint64_t e = e_begin + threadIdx.x;
-          if (e < 4 * v0) put(e);
-        } else if (threadIdx.x < 8) {
-          const uint64_t e = 4 * v1 + (threadIdx.x - 4);
-          if (e < e_end) put(e);
-        }
-      }
-    }
+    emit_values<kMode>(grp_s, O, 5 * O, umin64(5 * (O + Ec), j.n), j.y, j.vec, scale, sm.lut,
+                       threadIdx.x, kDThreads);
   } else {
     // accumulate, escape-heavy tile: visit only literal groups other than
     // the all-zero 121; each group's (up to five) acc values are loaded
@@ -424,7 +448,9 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
   __syncthreads();
 }
 
-template <int kMode, bool kVec, bool kDeferred>
+// Small streams: payload tiles in ticket order, each finding its first group
+// by a decoupled look-back over the tiles before it.
+template <int kMode, bool kVec>
 __global__ void __launch_bounds__(kDThreads)
 k_decode(const DecodeArgs a) {
   constexpr int kDTile = DecodeShape<kMode>::kTile;
@@ -442,7 +468,7 @@ k_decode(const DecodeArgs a) {
     m_s = m;
     scale_s = scale;
   }
-  for (int v = threadIdx.x; v < 256; v += kDThreads) sm.lut[v] = v < 243 ? digits_of(v) : 0;
+  fill_lut(sm.lut);
   __syncthreads();
   if (!ok_s) {
     if (blockIdx.x == 0 && threadIdx.x == 0) report(a.dev_status, TLC_ERR_CORRUPT);
@@ -458,111 +484,594 @@ k_decode(const DecodeArgs a) {
   job.status = a.status;
   job.n_tiles = (uint32_t)((job.m + kDTile - 1) / kDTile);
   job.vec = kVec;
-  job.ecount = a.ecount;
-  job.csum = a.csum;
+  job.off = nullptr;
   for (;;) {
     if (threadIdx.x == 0) tile_s = atomicAdd(a.ticket, 1u);
     __syncthreads();
     const uint32_t u = tile_s;
     if (u >= job.n_tiles) break;
-    decode_tile<kMode, kDeferred>(job, u, sm, grp_s, a.dev_status, a.max_polls);
+    decode_tile<kMode, false>(job, u, sm, grp_s, a.dev_status, a.max_polls);
   }
 }
 
-// Deferred prefixes, first pass, for chunk c of one stream: the group count
-// of each of its 512-byte payload units (one warp per unit, one 32-bit word
-// per lane, every word loaded before any is counted) and of the chunk.
-// Whole block; ends synchronised.
-constexpr int kUnitsPerWarp = kDecodeChunkUnits / (kDThreads / kWarp);
-static_assert(kDecodeUnit == 4 * kWarp * 4, "four words per lane per unit");
-__device__ __forceinline__ void count_chunk(const uint8_t *payload, uint64_t m, uint32_t c,
-                                            uint32_t *ecount, uint64_t *csum, uint32_t *wsum) {
+// ===================================================================== index
+// The index of one stream, as k_decode_index writes it.
+struct IndexOut {
+  const uint8_t *payload;
+  uint64_t m;          // payload length (valid header)
+  uint64_t groups;
+  uint64_t *status;    // look-back words, one per 32-unit chunk (zero at launch)
+  uint32_t *off;       // first group of every unit, plus the total after the last
+  uint32_t *page;      // unit holding group p * kPage, for every page p
+  uint32_t *ok;        // set to 1 when the stream expands to exactly `groups`
+};
+
+// Chunk c (32 units of 512 payload bytes) of one stream.  Whole block; ends
+// synchronised.  ucnt: 32 words of shared memory.
+constexpr int kUnitsPerWarp = kDecodeChunkUnits / kDWarps;
+__device__ __forceinline__ void index_chunk(const IndexOut &s, uint32_t c, uint32_t *ucnt,
+                                            int32_t *dev_status, uint32_t max_polls) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t n_units = (uint32_t)((m + kDecodeUnit - 1) / kDecodeUnit);
-  const bool al4 = (reinterpret_cast<uintptr_t>(payload) & 3) == 0;
+  const uint64_t n_units = (s.m + kDecodeUnit - 1) / kDecodeUnit;
+  const bool al4 = (reinterpret_cast<uintptr_t>(s.payload) & 3) == 0;
+  // the warp's units: each lane one 32-bit word per quarter unit, words
+  // interleaved across lanes so every load is coalesced; all loads first
   constexpr int kW = kUnitsPerWarp * (kDecodeUnit / (4 * kWarp));
   uint32_t w[kW];
   int nb[kW];
 #pragma unroll
   for (int k = 0; k < kW; ++k) {
-    const uint32_t unit = c * kDecodeChunkUnits + warp * kUnitsPerWarp + k / 4;
-    const uint64_t p = (uint64_t)unit * kDecodeUnit + 4 * (uint64_t)(lane + kWarp * (k % 4));
+    const uint64_t unit = (uint64_t)c * kDecodeChunkUnits + warp * kUnitsPerWarp + k / 4;
+    const uint64_t p = unit * kDecodeUnit + 4 * (uint64_t)(lane + kWarp * (k % 4));
     w[k] = 0;
     nb[k] = 0;
-    if (al4 && p + 4 <= m) {
-      w[k] = __ldg(reinterpret_cast<const uint32_t *>(payload + p));
+    if (al4 && p + 4 <= s.m) {
+      w[k] = __ldg(reinterpret_cast<const uint32_t *>(s.payload + p));
       nb[k] = 4;
     } else {
       for (int q = 0; q < 4; ++q)
-        if (p + q < m) {
-          w[k] |= (uint32_t)__ldg(payload + p + q) << (8 * q);
+        if (p + q < s.m) {
+          w[k] |= (uint32_t)__ldg(s.payload + p + q) << (8 * q);
           nb[k] = q + 1;
         }
     }
   }
-  uint32_t wtot = 0;
 #pragma unroll
   for (int i = 0; i < kUnitsPerWarp; ++i) {
     uint32_t e = 0;
 #pragma unroll
     for (int k = 4 * i; k < 4 * i + 4; ++k)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint32_t b = (w[k] >> (8 * q)) & 0xffu;
-        if (q < nb[k]) e += b >= 243u ? b - 241u : 1u;
-      }
+      for (int q = 0; q < 4; ++q)
+        if (q < nb[k]) e += expansion((w[k] >> (8 * q)) & 0xffu);
     e = __reduce_add_sync(0xffffffffu, e);
-    const uint32_t unit = c * kDecodeChunkUnits + warp * kUnitsPerWarp + i;
-    if (lane == 0 && unit < n_units) ecount[unit] = e;
-    wtot += e;
+    if (lane == 0) ucnt[warp * kUnitsPerWarp + i] = e;
   }
-  if (lane == 0) wsum[warp] = wtot;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    uint64_t sum = 0;
+  if (warp == 0) {
+    const uint32_t v = ucnt[lane];
+    uint32_t inc = v;
 #pragma unroll
-    for (int v = 0; v < kDThreads / kWarp; ++v) sum += wsum[v];
-    csum[c] = sum;
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
+      if (lane >= d) inc += t;
+    }
+    const uint32_t E = __shfl_sync(0xffffffffu, inc, 31);
+    bool timed_out = false;
+    const uint64_t P = lookback_sum<TLC_IX_LOOKV>(s.status, c, E, max_polls, timed_out);
+    timed_out = __any_sync(0xffffffffu, timed_out);
+    if (timed_out && lane == 0) report(dev_status, TLC_ERR_TIMEOUT);
+    const uint64_t u = (uint64_t)c * kDecodeChunkUnits + lane;
+    if (u < n_units) {
+      const uint64_t o = P + (inc - v);
+      s.off[u] = (uint32_t)umin64(o, 0xffffffffull);
+      // the pages whose first group lies in this unit
+      const uint64_t pend = umin64(o + v, s.groups);
+      for (uint64_t p = (o + kPage - 1) / kPage; p * kPage < pend; ++p)
+        if (TLC_CHECK(p < (s.groups + kPage - 1) / kPage)) s.page[p] = (uint32_t)u;
+      if (u == n_units - 1) {
+        s.off[u + 1] = (uint32_t)umin64(o + v, 0xffffffffull);
+        if (o + v == s.groups && !timed_out) *s.ok = 1u;
+        else report(dev_status, TLC_ERR_CORRUPT);
+      }
+    }
   }
   __syncthreads();
 }
 
-// Counting pass of one stream: blocks stride over the chunks that exist.
-// Block 0 also clears k_decode's ticket.  A stream whose length or header is
-// invalid is left to k_decode to report.
-__global__ void __launch_bounds__(kDThreads) k_decode_count(const DecodeArgs a) {
-  __shared__ uint64_t m_s;
-  __shared__ int ok_s;
-  __shared__ uint32_t wsum[kDThreads / kWarp];
-  if (threadIdx.x == 0) {
+// Up to kIndexPass streams of n values each, decoded in one launch pair.
+struct IxStream {
+  const uint8_t *in;
+  const uint64_t *len_dev;
+  uint64_t cap;
+  uint64_t *status;
+  uint32_t *off;
+  uint32_t *page;
+};
+struct IxArgs {
+  IxStream s[kIndexPass];
+  int k;
+  uint64_t n, groups;
+  uint32_t *ticket;    // index chunks (zero at launch)
+  uint32_t *ticket2;   // decode tiles (cleared by k_decode_index)
+  uint32_t *ok;        // per stream (zero at launch)
+  float *y;
+  bool vec;
+  int32_t *dev_status;
+  uint32_t max_polls;
+};
+
+// Index of every stream: the chunks that exist (from each stream's length),
+// numbered stream by stream, taken in ticket order.
+__global__ void __launch_bounds__(kDThreads) k_decode_index(const IxArgs a) {
+  __shared__ uint64_t m_s[kIndexPass];
+  __shared__ uint32_t pre_s[kIndexPass + 1];
+  __shared__ uint32_t ucnt[kDecodeChunkUnits];
+  __shared__ uint32_t tile_s;
+  if (threadIdx.x < (unsigned)a.k) {
+    const IxStream &S = a.s[threadIdx.x];
     uint64_t m = 0;
     float scale = 0.0f;
-    ok_s = read_stream_header(a.in, a.len_dev, a.cap, a.groups, m, scale) ? 1 : 0;
-    m_s = m;
-    if (blockIdx.x == 0) *a.ticket = 0;
+    const bool valid = read_stream_header(S.in, S.len_dev, S.cap, a.groups, m, scale);
+    m_s[threadIdx.x] = valid ? m : 0;
+    if (!valid && blockIdx.x == 0) report(a.dev_status, TLC_ERR_CORRUPT);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket2 = 0;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    pre_s[0] = 0;
+    for (int s = 0; s < a.k; ++s)
+      pre_s[s + 1] = pre_s[s] +
+          (uint32_t)((m_s[s] + (uint64_t)kDecodeUnit * kDecodeChunkUnits - 1) /
+                     ((uint64_t)kDecodeUnit * kDecodeChunkUnits));
+  }
+  __syncthreads();
+  const uint32_t total = pre_s[a.k];
+  for (;;) {
+    if (threadIdx.x == 0) tile_s = atomicAdd(a.ticket, 1u);
+    __syncthreads();
+    const uint32_t t = tile_s;
+    if (t >= total) break;
+    int s = 0;
+    while (s + 1 < a.k && pre_s[s + 1] <= t) ++s;
+    const IxStream &S = a.s[s];
+    const IndexOut io = {S.in + 4, m_s[s], a.groups, S.status, S.off, S.page, a.ok + s};
+    index_chunk(io, t - pre_s[s], ucnt, a.dev_status, a.max_polls);
+  }
+}
+
+// ============================================================= warp units
+// One 512-byte payload unit of an indexed stream, by one warp.  The unit's
+// first group is off[u]; its groups are expanded into the warp's own shared
+// memory (up to kWarpGroups) and written (or added) as coalesced float4s,
+// the float4s that straddle the next unit as single values.  A unit without
+// non-zero literals is plain zeros (dense output) or nothing (accumulate);
+// a unit that expands past kWarpGroups, or (accumulate) whose literals are
+// few, writes its zeros and then visits only its literal groups.  No warp
+// waits on another.
+#ifndef TLC_WARP_GROUPS
+#define TLC_WARP_GROUPS 2048
+#endif
+constexpr uint32_t kWarpGroups = TLC_WARP_GROUPS;
+static_assert(kWarpGroups % 16 == 0, "whole 16-byte words");
+
+template <int kMode>
+__device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, const uint16_t *lut,
+                                            uint8_t *ws) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t base = (uint64_t)u * kDecodeUnit + 16ull * lane;
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  int nb = 0;
+  if (base < j.m) {
+    const uint64_t left = j.m - base;
+    const uint8_t *p = j.payload + base;
+    if (left >= 16 && (reinterpret_cast<uintptr_t>(p) & 3) == 0) {
+      const uint32_t *p32 = reinterpret_cast<const uint32_t *>(p);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) w[k] = __ldg(p32 + k);
+      nb = 16;
+    } else {
+      nb = (int)umin64(left, 16);
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        if (k < nb) w[k >> 2] |= (uint32_t)__ldg(p + k) << (8 * (k & 3));
+    }
+  }
+  uint32_t e = 0, lits = 0;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    if (k < nb) {
+      const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
+      e += expansion(b);
+      lits += (b < 243u && b != 121u) ? 1u : 0u;
+    }
+  }
+  uint32_t inc = e;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc += t;
+  }
+  const uint32_t E = __shfl_sync(0xffffffffu, inc, 31);
+  const uint32_t L = __reduce_add_sync(0xffffffffu, lits);
+  const uint32_t excl = inc - e;
+  const uint64_t O = __ldg(j.off + u);
+  const uint64_t Ec = O >= j.groups ? 0 : umin64(E, j.groups - O);
+  const uint64_t e_begin = 5 * O, e_end = umin64(5 * (O + Ec), j.n);
+  if (L == 0) {
+    if (kMode == kWrite) emit_zeros(e_begin, e_end, j.y, j.vec, lane, kWarp);
+    return;
+  }
+  if (E <= kWarpGroups && (kMode == kWrite || 16 * L >= E)) {
+    for (uint32_t q = lane; q < (E + 15) / 16; q += kWarp)
+      reinterpret_cast<uint4 *>(ws)[q] =
+          make_uint4(0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u);
+    __syncwarp();
+    uint32_t pos = excl;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if (k < nb) {
+        const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
+        if (b >= 243u) {
+          pos += b - 241u;
+        } else {
+          if (TLC_CHECK(pos < kWarpGroups)) ws[pos] = (uint8_t)b;
+          ++pos;
+        }
+      }
+    }
+    __syncwarp();
+    emit_values<kMode>(ws, O, e_begin, e_end, j.y, j.vec, j.scale, lut, lane, kWarp);
+    __syncwarp();
+    return;
+  }
+  // long zero runs around a few literals: zeros first (dense output), then
+  // the literal groups (each group's values loaded before any is added)
+  if (kMode == kWrite) {
+    emit_zeros(e_begin, e_end, j.y, j.vec, lane, kWarp);
+    __syncwarp();
+  }
+  uint64_t g = O + excl;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    if (k < nb) {
+      const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
+      if (b >= 243u) {
+        g += b - 241u;
+      } else {
+        if (b != 121u && g < j.groups) {
+          const uint32_t dg = lut[b];
+          if (kMode == kWrite) {
+#pragma unroll
+            for (int d = 0; d < 5; ++d) {
+              const uint64_t ei = 5 * g + d;
+              if (ei < j.n) j.y[ei] = dequant((dg >> (2 * d)) & 3u, j.scale);
+            }
+          } else {
+            float v[5];
+#pragma unroll
+            for (int d = 0; d < 5; ++d) {
+              const uint64_t ei = 5 * g + d;
+              v[d] = (((dg >> (2 * d)) & 3u) != 1u && ei < j.n) ? j.y[ei] : 0.0f;
+            }
+#pragma unroll
+            for (int d = 0; d < 5; ++d) {
+              const uint32_t dig = (dg >> (2 * d)) & 3u;
+              const uint64_t ei = 5 * g + d;
+              if (dig != 1u && ei < j.n) j.y[ei] = __fadd_rn(v[d], dequant(dig, j.scale));
+            }
+          }
+        }
+        ++g;
+      }
+    }
+  }
+  __syncwarp();
+}
+
+// Shared memory of a block of warp-unit decoders.
+struct UnitSmem {
+  uint16_t lut[256];
+  __align__(16) uint8_t ws[kDWarps][kWarpGroups + 16];
+};
+
+// One indexed stream (dense output, or added into acc): every warp takes
+// units blockIdx.x * warps + warp, then every (grid's warps)-th unit.
+template <int kMode>
+__global__ void __launch_bounds__(kDThreads, 8) k_decode_units(const IxArgs a) {
+  __shared__ UnitSmem sm;
+  __shared__ DecodeJob job_s;
+  __shared__ int ok_s;
+  fill_lut(sm.lut);
+  if (threadIdx.x == 0) {
+    const IxStream &S = a.s[0];
+    uint64_t m = 0;
+    float scale = 0.0f;
+    ok_s = a.ok[0] && read_stream_header(S.in, S.len_dev, S.cap, a.groups, m, scale);
+    DecodeJob j;
+    j.payload = S.in + 4;
+    j.m = m;
+    j.n = a.n;
+    j.groups = a.groups;
+    j.scale = scale;
+    j.y = a.y;
+    j.status = nullptr;
+    j.n_tiles = (uint32_t)((m + kDecodeUnit - 1) / kDecodeUnit);
+    j.vec = a.vec;
+    j.off = S.off;
+    job_s = j;
   }
   __syncthreads();
   if (!ok_s) return;
-  const uint64_t m = m_s;
-  const uint32_t n_units = (uint32_t)((m + kDecodeUnit - 1) / kDecodeUnit);
-  const uint32_t n_chunks = (n_units + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
-  for (uint32_t c = blockIdx.x; c < n_chunks; c += gridDim.x)
-    count_chunk(a.in + 4, m, c, a.ecount, a.csum, wsum);
+  const DecodeJob j = job_s;
+  const int warp = threadIdx.x >> 5;
+  const uint32_t nw = gridDim.x * kDWarps;
+  for (uint32_t u = blockIdx.x * kDWarps + warp; u < j.n_tiles; u += nw)
+    decode_unit<kMode>(j, u, sm.lut, sm.ws[warp]);
 }
 
+// ==================================================================== gather
+// A stream as the gather tiles read it.
+struct GStream {
+  const uint8_t *payload;
+  const uint32_t *off;
+  const uint32_t *page;
+  uint64_t m;
+  float scale;
+  uint32_t n_units;
+};
+
+template <int kK>
+struct GatherSmem {
+  uint32_t uf[kK], nu[kK];  // first unit and unit count of each stream in the tile
+  uint32_t lit[kK];         // the stream has a non-zero literal in the tile
+};
+
+// One warp: unit u of stream S.  Each lane takes 16 consecutive payload
+// bytes; a warp scan of their expansion counts gives each lane's first
+// group; literal groups that fall in [g0, g0 + gn) go to grp.  Sets *lit
+// when a literal other than the zero group 121 was placed.
+__device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t g0, uint32_t gn,
+                                          uint8_t *grp, uint32_t *lit) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t base = (uint64_t)u * kDecodeUnit + 16ull * lane;
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  int nb = 0;
+  if (base < S.m) {
+    const uint64_t left = S.m - base;
+    const uint8_t *p = S.payload + base;
+    if (left >= 16 && (reinterpret_cast<uintptr_t>(p) & 3) == 0) {
+      const uint32_t *p32 = reinterpret_cast<const uint32_t *>(p);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) w[k] = __ldg(p32 + k);
+      nb = 16;
+    } else {
+      nb = (int)umin64(left, 16);
+#pragma unroll
+      for (int k = 0; k < 16; ++k)
+        if (k < nb) w[k >> 2] |= (uint32_t)__ldg(p + k) << (8 * (k & 3));
+    }
+  }
+  uint32_t e = 0;
+#pragma unroll
+  for (int k = 0; k < 16; ++k)
+    if (k < nb) e += expansion((w[k >> 2] >> (8 * (k & 3))) & 0xffu);
+  uint32_t inc = e;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc += t;
+  }
+  uint64_t g = (uint64_t)__ldg(S.off + u) + (inc - e);
+  const uint64_t ge = g0 + gn;
+  bool mine = false;
+  if (nb > 0 && g < ge && g + e > g0) {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if (k < nb) {
+        const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
+        if (b < 243u) {
+          if (g >= g0 && g < ge && TLC_CHECK(g - g0 < (uint64_t)gn)) {
+            grp[g - g0] = (uint8_t)b;
+            mine = mine || b != 121u;
+          }
+          ++g;
+        } else {
+          g += b - 241u;
+        }
+      }
+    }
+  }
+  if (__any_sync(0xffffffffu, mine) && lane == 0) *lit = 1u;
+}
+
+// One gather tile: output groups [g0, g0 + gn) of k streams (k <= kK, all
+// valid, in stream order).  Whole block; ends synchronised.  grp holds
+// kK * kGt bytes.
+template <int kMode, int kGt, int kK>
+__device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g0,
+                                            uint64_t groups, uint64_t n, float *y, bool vec,
+                                            const uint16_t *lut, uint8_t *grp,
+                                            GatherSmem<kK> &sm) {
+  static_assert(kGt % kPage == 0 && kGt % 16 == 0, "tile shape");
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t gn = (uint32_t)umin64(kGt, groups - g0);
+  // pre-fill with the zero group; each stream's unit range from the pages
+  for (int s = 0; s < k; ++s)
+    for (uint32_t w = threadIdx.x; w < (gn + 15) / 16; w += kDThreads)
+      reinterpret_cast<uint4 *>(grp + s * kGt)[w] =
+          make_uint4(0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u);
+  if (warp == 0 && lane < k) {
+    const GStream &S = gs[lane];
+    const uint32_t last = S.n_units - 1;
+    uint32_t uf = umin64(__ldg(S.page + g0 / kPage), last);
+    uint32_t ul = g0 + gn < groups ? (uint32_t)umin64(__ldg(S.page + (g0 + gn) / kPage), last)
+                                   : last;
+    if (ul < uf) ul = uf;
+    sm.uf[lane] = uf;
+    sm.nu[lane] = ul - uf + 1;
+    sm.lit[lane] = 0u;
+  }
+  __syncthreads();
+  for (int s = 0; s < k; ++s)
+    for (uint32_t i = warp; i < sm.nu[s]; i += kDWarps)
+      walk_unit(gs[s], sm.uf[s] + i, g0, gn, grp + s * kGt, &sm.lit[s]);
+  __syncthreads();
+  const uint64_t e_begin = 5 * g0, e_end = umin64(5 * (g0 + gn), n);
+  if (kMode == kWrite) {
+    if (sm.lit[0])
+      emit_values<kWrite>(grp, g0, e_begin, e_end, y, vec, gs[0].scale, lut, threadIdx.x,
+                          kDThreads);
+    else
+      emit_zeros(e_begin, e_end, y, vec, threadIdx.x, kDThreads);
+  } else if (kK == 1) {
+    if (sm.lit[0])
+      emit_values<kAccumulate>(grp, g0, e_begin, e_end, y, vec, gs[0].scale, lut, threadIdx.x,
+                               kDThreads);
+  } else {
+    // several streams: one read-modify-write of each float4 of acc, the
+    // streams' non-zero values added in stream order
+    uint32_t act = 0;  // bit s: stream s has a non-zero value in the tile
+#pragma unroll
+    for (int s = 0; s < kK; ++s)
+      if (s < k && sm.lit[s]) act |= 1u << s;
+    if (act) {
+      const uint32_t o32 = (uint32_t)g0;
+      const uint64_t v0 = vec ? (e_begin + 3) / 4 : e_end, v1 = vec ? e_end / 4 : e_end;
+      float4 *y4 = reinterpret_cast<float4 *>(y);
+      for (uint64_t v = v0 + threadIdx.x; v < v1; v += kDThreads) {
+        const uint32_t e0 = (uint32_t)(4 * v);
+        const uint32_t g = e0 / 5u;
+        const uint32_t d0 = e0 - 5u * g;
+        const uint32_t li = g - o32;
+        float4 o;
+        bool loaded = false;
+#pragma unroll
+        for (int i = 0; i < kK; ++i) {
+          if ((act >> i) & 1u) {
+            const uint8_t *gb = grp + i * kGt;
+            const uint32_t c0 = gb[li];
+            const uint32_t c1 = d0 >= 2u ? (uint32_t)gb[li + 1] : 121u;
+            if (c0 == 121u && c1 == 121u) continue;
+            const uint32_t w = ((uint32_t)lut[c0] | ((uint32_t)lut[c1] << 10)) >> (2u * d0);
+            if ((w & 0xffu) == 0x55u) continue;
+            if (!loaded) {
+              o = y4[v];
+              loaded = true;
+            }
+            const float sc = gs[i].scale;
+            if ((w & 3u) != 1u) o.x = __fadd_rn(o.x, dequant(w & 3u, sc));
+            if (((w >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, dequant((w >> 2) & 3u, sc));
+            if (((w >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, dequant((w >> 4) & 3u, sc));
+            if (((w >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, dequant((w >> 6) & 3u, sc));
+          }
+        }
+        if (loaded) y4[v] = o;
+      }
+      // single values: the edges of the float4 range, or every value when
+      // acc is not 16-byte aligned
+      auto put = [&](uint64_t e) {
+        const uint32_t e32 = (uint32_t)e;
+        const uint32_t g = e32 / 5u;
+        const uint32_t sh = 2 * (e32 - 5u * g);
+        float v = 0.0f;
+        bool loaded = false;
+#pragma unroll
+        for (int i = 0; i < kK; ++i) {
+          if ((act >> i) & 1u) {
+            const uint32_t dig = (lut[grp[i * kGt + (g - o32)]] >> sh) & 3u;
+            if (dig == 1u) continue;
+            if (!loaded) {
+              v = y[e];
+              loaded = true;
+            }
+            v = __fadd_rn(v, dequant(dig, gs[i].scale));
+          }
+        }
+        if (loaded) y[e] = v;
+      };
+      if (!vec || v1 <= v0) {
+        for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) put(e);
+      } else if (threadIdx.x < 4) {
+        const uint64_t e = e_begin + threadIdx.x;
+        if (e < 4 * v0) put(e);
+      } else if (threadIdx.x < 8) {
+        const uint64_t e = 4 * v1 + (threadIdx.x - 4);
+        if (e < e_end) put(e);
+      }
+    }
+  }
+  __syncthreads();
+}
+
+// Shared memory (dynamic part) of k_decode_ix: the gather tile's group bytes.
+template <int kGt, int kK>
+constexpr size_t ix_smem_bytes() {
+  return (size_t)kK * kGt + 16;
+}
+
+// Add k <= kK indexed streams (in stream order) into acc, by gather tiles.
+// Streams the index did not mark valid are left out.  Tiles in ticket
+// order; no tile waits on another.
+template <int kGt, int kK>
+__global__ void __launch_bounds__(kDThreads, 6) k_decode_ix(const IxArgs a) {
+  extern __shared__ __align__(16) uint8_t dyn_s[];
+  __shared__ uint16_t lut[256];
+  __shared__ GatherSmem<kK> gsm;
+  __shared__ GStream gs[kK];
+  __shared__ int na_s;
+  __shared__ uint32_t tile_s;
+  fill_lut(lut);
+  if (threadIdx.x == 0) {
+    // the valid streams, in stream order
+    int na = 0;
+    for (int s = 0; s < a.k && s < kK; ++s) {
+      if (!a.ok[s]) continue;
+      const IxStream &S = a.s[s];
+      uint64_t m = 0;
+      float scale = 0.0f;
+      if (!read_stream_header(S.in, S.len_dev, S.cap, a.groups, m, scale)) continue;
+      GStream g;
+      g.payload = S.in + 4;
+      g.off = S.off;
+      g.page = S.page;
+      g.m = m;
+      g.scale = scale;
+      g.n_units = (uint32_t)((m + kDecodeUnit - 1) / kDecodeUnit);
+      gs[na++] = g;
+    }
+    na_s = na;
+  }
+  __syncthreads();
+  const int na = na_s;
+  if (na == 0) return;
+  const uint64_t n_tiles = (a.groups + kGt - 1) / kGt;
+  for (;;) {
+    if (threadIdx.x == 0) tile_s = atomicAdd(a.ticket2, 1u);
+    __syncthreads();
+    const uint32_t t = tile_s;
+    if (t >= n_tiles) break;
+    gather_tile<kAccumulate, kGt, kK>(gs, na, (uint64_t)t * kGt, a.groups, a.n, a.y, a.vec, lut,
+                                      dyn_s, gsm);
+  }
+}
+
+// ================================================================= batches
 struct BatchDecodeArgs {
   const BatchTensor *tensors;
   uint32_t count;
-  const BatchPrep *prep;        // per-tensor payload length, scale, first tile
-  const uint32_t *total;        // tiles in the compact numbering
-  uint32_t n_tiles;             // upper bound of total (sizes the grid)
+  const BatchPrep *prep;        // per-tensor payload length, scale, tiling, first tile
+  const uint32_t *total;        // tiles and chunks in the compact numbering
+  uint32_t n_tiles;             // upper bound of total[0] (sizes the grid)
   const uint8_t *arena;
   uint64_t *status;
   uint32_t *ticket;
+  uint32_t *ticket2;            // indexed plans: the decode kernel's ticket
   int32_t *dev_status;
   uint32_t max_polls;
-  uint32_t *ecount;             // counting pass (plans of 16384 units and more)
-  uint64_t *csum;
+  uint32_t *off;                // indexed plans: units' first groups,
+  uint32_t *page;               // page tables,
+  uint32_t *ok;                 // per-tensor valid flags
   uint32_t n_chunks;            // chunks of all tensors (upper bound)
 };
 
@@ -570,9 +1079,9 @@ constexpr int kPrepThreads = 1024;
 constexpr uint32_t kSmemSearch = 2048;  // tensors whose first tiles fit in shared memory
 
 // One block: validate every tensor's stream once, and number the tiles that
-// actually exist (ceil(m / tile) per stream, 0 for a corrupt one)
-// consecutively, tensor by tensor; the same for the counting pass's 32-unit
-// chunks.  total[0] = tiles, total[1] = chunks.
+// actually exist (ceil(m / tile_bytes) per stream, none for a corrupt one)
+// consecutively, tensor by tensor; the same for the index's 32-unit chunks.
+// total[0] = tiles, total[1] = chunks.
 __global__ void __launch_bounds__(kPrepThreads)
 k_decode_batch_prepare(const BatchTensor *__restrict__ tensors, uint32_t count,
                        const uint8_t *__restrict__ arena, const uint64_t *__restrict__ in_lens,
@@ -617,18 +1126,31 @@ k_decode_batch_prepare(const BatchTensor *__restrict__ tensors, uint32_t count,
   }
 }
 
-// Decode the streams of a list of tensors from their arena slots: the tiles
-// that exist, numbered tensor by tensor, taken in ticket order; each
-// look-back is confined to its stream.  A tile's tensor is found by binary
-// search over the tensors' first tiles.
-template <int kMode, bool kDeferred>
+// Last tensor whose first numbered item (begin) is <= u; tensors without
+// items share their first item with the next tensor and are skipped.
+__device__ __forceinline__ uint32_t find_tensor(const uint32_t *begin_s, bool in_smem,
+                                                const BatchPrep *prep, uint32_t count, uint32_t u,
+                                                bool chunks) {
+  uint32_t lo = 0, hi = count - 1;
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi + 1) >> 1;
+    const uint32_t b = in_smem ? begin_s[mid] : (chunks ? prep[mid].cact_begin
+                                                          : prep[mid].act_begin);
+    if (b <= u) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+// Small plans: the payload tiles of every tensor in one ticket order, each
+// look-back confined to its stream.
+template <int kMode>
 __global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArgs a) {
   constexpr int kDTile = DecodeShape<kMode>::kTile;
   extern __shared__ __align__(16) uint8_t grp_s[];
   __shared__ DecodeSmem sm;
   __shared__ uint32_t begin_s[kSmemSearch];
   __shared__ uint32_t tile_s;
-  for (int v = threadIdx.x; v < 256; v += kDThreads) sm.lut[v] = v < 243 ? digits_of(v) : 0;
+  fill_lut(sm.lut);
   const bool in_smem = a.count <= kSmemSearch;
   if (in_smem)
     for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads) begin_s[i] = a.prep[i].act_begin;
@@ -638,16 +1160,9 @@ __global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArg
     __syncthreads();
     const uint32_t u = tile_s;
     if (u >= total) break;
-    // last tensor whose first tile is <= u (tensors without tiles are skipped
-    // naturally: they share their first tile with the next tensor)
-    uint32_t lo = 0, hi = a.count - 1;
-    while (lo < hi) {
-      const uint32_t mid = (lo + hi + 1) >> 1;
-      const uint32_t b = in_smem ? begin_s[mid] : a.prep[mid].act_begin;
-      if (b <= u) lo = mid; else hi = mid - 1;
-    }
-    const BatchTensor &T = a.tensors[lo];
-    const BatchPrep &P = a.prep[lo];
+    const uint32_t id = find_tensor(begin_s, in_smem, a.prep, a.count, u, false);
+    const BatchTensor &T = a.tensors[id];
+    const BatchPrep &P = a.prep[id];
     DecodeJob job;
     job.payload = a.arena + T.arena_off + 4;
     job.m = P.m;
@@ -658,37 +1173,70 @@ __global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArg
     job.status = a.status + T.d_tile_begin;
     job.n_tiles = (uint32_t)((job.m + kDTile - 1) / kDTile);
     job.vec = T.vec_y != 0;
-    job.ecount = kDeferred ? a.ecount + T.d_tile_begin : nullptr;
-    job.csum = kDeferred ? a.csum + T.d_chunk_begin : nullptr;
-    decode_tile<kMode, kDeferred>(job, u - P.act_begin, sm, grp_s, a.dev_status, a.max_polls);
+    job.off = nullptr;
+    decode_tile<kMode, false>(job, u - P.act_begin, sm, grp_s, a.dev_status, a.max_polls);
   }
 }
 
-// Counting pass of a plan's streams: blocks stride over the chunks that
-// exist, numbered tensor by tensor by the prepare kernel (a tensor's first
-// chunk is found by binary search).  Block 0 also clears the decode ticket.
-__global__ void __launch_bounds__(kDThreads) k_decode_batch_count(const BatchDecodeArgs a) {
+// Index of a plan's streams: the chunks that exist, numbered tensor by
+// tensor by the prepare kernel, in ticket order.  Block 0 also clears the
+// decode kernel's ticket.
+__global__ void __launch_bounds__(kDThreads) k_decode_batch_index(const BatchDecodeArgs a) {
   __shared__ uint32_t begin_s[kSmemSearch];
-  __shared__ uint32_t wsum[kDThreads / kWarp];
+  __shared__ uint32_t ucnt[kDecodeChunkUnits];
+  __shared__ uint32_t tile_s;
   const bool in_smem = a.count <= kSmemSearch;
   if (in_smem)
     for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads) begin_s[i] = a.prep[i].cact_begin;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket = 0;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket2 = 0;
   __syncthreads();
   const uint32_t total = a.total[1];
-  for (uint32_t g = blockIdx.x; g < total; g += gridDim.x) {
-    // last tensor whose first chunk is <= g (tensors without chunks share
-    // their first chunk with the next tensor)
-    uint32_t lo = 0, hi = a.count - 1;
-    while (lo < hi) {
-      const uint32_t mid = (lo + hi + 1) >> 1;
-      const uint32_t b = in_smem ? begin_s[mid] : a.prep[mid].cact_begin;
-      if (b <= g) lo = mid; else hi = mid - 1;
-    }
-    const BatchTensor &T = a.tensors[lo];
-    const BatchPrep &P = a.prep[lo];
-    count_chunk(a.arena + T.arena_off + 4, P.m, g - P.cact_begin, a.ecount + T.d_tile_begin,
-                a.csum + T.d_chunk_begin, wsum);
+  for (;;) {
+    if (threadIdx.x == 0) tile_s = atomicAdd(a.ticket, 1u);
+    __syncthreads();
+    const uint32_t g = tile_s;
+    if (g >= total) break;
+    const uint32_t id = find_tensor(begin_s, in_smem, a.prep, a.count, g, true);
+    const BatchTensor &T = a.tensors[id];
+    const BatchPrep &P = a.prep[id];
+    const IndexOut io = {a.arena + T.arena_off + 4, P.m, T.groups, a.status + T.d_chunk_begin,
+                         a.off + T.d_off_begin, a.page + T.d_page_begin, a.ok + id};
+    index_chunk(io, g - P.cact_begin, ucnt, a.dev_status, a.max_polls);
+  }
+}
+
+// Large plans: every tensor's 512-byte units (numbered tensor by tensor by
+// the prepare kernel), one warp per unit as in k_decode_units; a tensor the
+// index did not mark valid is left out.
+template <int kMode>
+__global__ void __launch_bounds__(kDThreads, 8) k_decode_batch_units(const BatchDecodeArgs a) {
+  __shared__ UnitSmem sm;
+  __shared__ uint32_t begin_s[kSmemSearch];
+  fill_lut(sm.lut);
+  const bool in_smem = a.count <= kSmemSearch;
+  if (in_smem)
+    for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads) begin_s[i] = a.prep[i].act_begin;
+  __syncthreads();
+  const uint32_t total = *a.total;
+  const int warp = threadIdx.x >> 5;
+  const uint32_t nw = gridDim.x * kDWarps;
+  for (uint32_t gu = blockIdx.x * kDWarps + warp; gu < total; gu += nw) {
+    const uint32_t id = find_tensor(begin_s, in_smem, a.prep, a.count, gu, false);
+    if (!a.ok[id]) continue;  // uniform in the warp
+    const BatchTensor &T = a.tensors[id];
+    const BatchPrep &P = a.prep[id];
+    DecodeJob j;
+    j.payload = a.arena + T.arena_off + 4;
+    j.m = P.m;
+    j.n = T.n;
+    j.groups = T.groups;
+    j.scale = P.scale;
+    j.y = T.y;
+    j.status = nullptr;
+    j.n_tiles = (uint32_t)((P.m + kDecodeUnit - 1) / kDecodeUnit);
+    j.vec = T.vec_y != 0;
+    j.off = a.off + T.d_off_begin;
+    decode_unit<kMode>(j, gu - P.act_begin, sm.lut, sm.ws[warp]);
   }
 }
 
@@ -702,7 +1250,7 @@ __global__ void k_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_s
 // ------------------------------------------------------------- launchers --
 uint32_t decode_tiles_max(uint64_t cap, uint64_t groups) {
   // 512-byte units: at least as many as the tiles of either mode (tiles are
-  // whole units), and the counting pass's unit count
+  // whole units), and the index's unit count
   static_assert(DecodeShape<kWrite>::kTile % kDecodeUnit == 0 &&
                     DecodeShape<kAccumulate>::kTile % kDecodeUnit == 0,
                 "tiles are whole units");
@@ -717,27 +1265,24 @@ size_t decode_smem_bytes(bool accumulate) {
                              : DecodeShape<kWrite>::kMaxGroups) + 16;
 }
 
+bool decode_deferred(uint32_t tiles) { return tiles >= kDecodeDeferMinTiles; }
+
+uint32_t decode_tile_payload_bytes(bool accumulate) {
+  return accumulate ? DecodeShape<kAccumulate>::kTile : DecodeShape<kWrite>::kTile;
+}
+
+uint32_t decode_pages(uint64_t groups) { return (uint32_t)((groups + kPage - 1) / kPage); }
+
 template <int kMode, bool kVec>
 static cudaError_t launch_one(const DeviceInfo &dev, const DecodeArgs &a, uint32_t tiles,
-                              bool deferred, cudaStream_t stream) {
+                              cudaStream_t stream) {
   const size_t smem = decode_smem_bytes(kMode == kAccumulate);
   const int occ = kMode == kWrite ? dev.occ_decode_write : dev.occ_decode_acc;
   uint32_t grid = (uint32_t)dev.sm_count * (uint32_t)(occ > 0 ? occ : 1);
   if (grid > tiles) grid = tiles;
-  if (deferred) {
-    // tiles (the capacity's 512-byte units) bound the units that exist
-    uint32_t cgrid = (tiles + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
-    if (cgrid > (uint32_t)dev.sm_count * 8) cgrid = (uint32_t)dev.sm_count * 8;
-    timing_begin(kKindDecodeCount, stream);
-    k_decode_count<<<cgrid, kDThreads, 0, stream>>>(a);
-    timing_end(kKindDecodeCount, stream);
-  }
   const int kind = kMode == kWrite ? kKindDecodeWrite : kKindDecodeAccumulate;
   timing_begin(kind, stream);
-  if (deferred)
-    k_decode<kMode, kVec, true><<<grid, kDThreads, smem, stream>>>(a);
-  else
-    k_decode<kMode, kVec, false><<<grid, kDThreads, smem, stream>>>(a);
+  k_decode<kMode, kVec><<<grid, kDThreads, smem, stream>>>(a);
   timing_end(kind, stream);
   return cudaGetLastError();
 }
@@ -748,55 +1293,173 @@ cudaError_t launch_decode(const DeviceInfo &dev, const uint8_t *in, const uint64
                           cudaStream_t stream) {
   const uint64_t groups = (n + 4) / 5;
   const uint32_t tiles = decode_tiles_max(cap, groups);
-  const bool deferred = decode_deferred(tiles);
-  const DecodeScratch ds = decode_scratch_layout(scratch, tiles, deferred);
   DecodeArgs a;
-  a.ecount = ds.ecount;
-  a.csum = ds.csum;
   a.in = in;
   a.len_dev = len_dev;
   a.cap = cap;
   a.n = n;
   a.groups = groups;
   a.y = y;
-  a.status = ds.status;
-  a.ticket = ds.ticket;
+  a.status = scratch;
+  a.ticket = reinterpret_cast<uint32_t *>(scratch + tiles);
   a.dev_status = dev_status;
   a.max_polls = max_polls;
   const bool vec = (reinterpret_cast<uintptr_t>(y) & 15) == 0;
   if (accumulate)
-    return vec ? launch_one<kAccumulate, true>(dev, a, tiles, deferred, stream)
-               : launch_one<kAccumulate, false>(dev, a, tiles, deferred, stream);
-  return vec ? launch_one<kWrite, true>(dev, a, tiles, deferred, stream)
-             : launch_one<kWrite, false>(dev, a, tiles, deferred, stream);
+    return vec ? launch_one<kAccumulate, true>(dev, a, tiles, stream)
+               : launch_one<kAccumulate, false>(dev, a, tiles, stream);
+  return vec ? launch_one<kWrite, true>(dev, a, tiles, stream)
+             : launch_one<kWrite, false>(dev, a, tiles, stream);
 }
 
-bool decode_deferred(uint32_t tiles) { return tiles >= kDecodeDeferMinTiles; }
+// ---- indexed decode of up to kIndexPass streams --------------------------
+// Scratch: [ticket, ticket2, ok[kIndexPass]] and every stream's chunk status
+// words (zeroed before each launch pair), then each stream's off[] and
+// page[] arrays.
+static size_t ix_head_bytes() { return align_up(8 + 4 * kIndexPass, 64); }
 
-uint32_t decode_tile_payload_bytes(bool accumulate) {
-  return accumulate ? DecodeShape<kAccumulate>::kTile : DecodeShape<kWrite>::kTile;
+IndexedLayout indexed_layout(const IndexedStream *s, int k, uint64_t n) {
+  IndexedLayout L = {};
+  const uint64_t groups = (n + 4) / 5;
+  size_t at = ix_head_bytes();
+  for (int i = 0; i < k; ++i) {
+    const uint32_t units = decode_tiles_max(s[i].cap, groups);
+    L.status_off[i] = at;
+    at += 8 * (size_t)((units + kDecodeChunkUnits - 1) / kDecodeChunkUnits);
+  }
+  L.zero_bytes = align_up(at, 256);
+  at = L.zero_bytes;
+  for (int i = 0; i < k; ++i) {
+    const uint32_t units = decode_tiles_max(s[i].cap, groups);
+    L.off_off[i] = at;
+    at = align_up(at + 4 * ((size_t)units + 1), 16);
+    L.page_off[i] = at;
+    at = align_up(at + 4 * (size_t)decode_pages(groups), 16);
+  }
+  L.total_bytes = align_up(at, 256);
+  return L;
 }
 
+// Blocks per SM: the warp-unit kernels (slots 0 dense output, 1
+// accumulate) and each k_decode_ix instantiation (slots 2, 3, 4: up to 2, 4
+// and 8 streams), with their shared memory.
+template <int kGt, int kK>
+static int ix_occupancy() {
+  constexpr size_t smem = ix_smem_bytes<kGt, kK>();
+  cudaFuncSetAttribute(k_decode_ix<kGt, kK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)smem);
+  int occ = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_ix<kGt, kK>, kDThreads, smem);
+  return occ;
+}
+
+void occupancy_decode_ix(int occ[5]) {
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ[0], k_decode_units<kWrite>, kDThreads, 0);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ[1], k_decode_units<kAccumulate>, kDThreads,
+                                                0);
+  occ[2] = ix_occupancy<TLC_GT_ACC / 2, 2>();
+  occ[3] = ix_occupancy<TLC_GT_ACC / 4, 4>();
+  occ[4] = ix_occupancy<TLC_GT_ACC / 8, 8>();
+}
+
+static uint32_t persistent_grid(const DeviceInfo &dev, int occ, uint64_t work_blocks) {
+  uint64_t grid = (uint64_t)dev.sm_count * (uint64_t)(occ > 0 ? occ : 1);
+  if (grid > work_blocks) grid = work_blocks;
+  return (uint32_t)(grid < 1 ? 1 : grid);
+}
+
+template <int kGt, int kK>
+static cudaError_t launch_ix(const DeviceInfo &dev, const IxArgs &a, int occ_slot,
+                             cudaStream_t stream) {
+  constexpr size_t smem = ix_smem_bytes<kGt, kK>();
+  const uint32_t grid =
+      persistent_grid(dev, dev.occ_decode_ix[occ_slot], (a.groups + kGt - 1) / kGt);
+  timing_begin(kKindDecodeAccumulate, stream);
+  k_decode_ix<kGt, kK><<<grid, kDThreads, smem, stream>>>(a);
+  timing_end(kKindDecodeAccumulate, stream);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s, int k, uint64_t n,
+                                  float *y, bool accumulate, int32_t *dev_status,
+                                  uint32_t max_polls, void *scratch, cudaStream_t stream) {
+  if (k < 1 || k > kIndexPass || (!accumulate && k != 1)) return cudaErrorInvalidValue;
+  const IndexedLayout L = indexed_layout(s, k, n);
+  char *base = static_cast<char *>(scratch);
+  cudaError_t e = cudaMemsetAsync(scratch, 0, L.zero_bytes, stream);
+  if (e != cudaSuccess) return e;
+  IxArgs a;
+  a.k = k;
+  a.n = n;
+  a.groups = (n + 4) / 5;
+  a.ticket = reinterpret_cast<uint32_t *>(base);
+  a.ticket2 = reinterpret_cast<uint32_t *>(base + 4);
+  a.ok = reinterpret_cast<uint32_t *>(base + 8);
+  a.y = y;
+  a.vec = (reinterpret_cast<uintptr_t>(y) & 15) == 0;
+  a.dev_status = dev_status;
+  a.max_polls = max_polls;
+  uint64_t chunks = 0, units_max = 0;
+  for (int i = 0; i < kIndexPass; ++i) {
+    IxStream &S = a.s[i];
+    if (i < k) {
+      S.in = s[i].in;
+      S.len_dev = s[i].len_dev;
+      S.cap = s[i].cap;
+      S.status = reinterpret_cast<uint64_t *>(base + L.status_off[i]);
+      S.off = reinterpret_cast<uint32_t *>(base + L.off_off[i]);
+      S.page = reinterpret_cast<uint32_t *>(base + L.page_off[i]);
+      const uint32_t units = decode_tiles_max(s[i].cap, a.groups);
+      chunks += (units + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
+      if (units > units_max) units_max = units;
+    } else {
+      S = IxStream{};
+    }
+  }
+  timing_begin(kKindDecodeCount, stream);
+  k_decode_index<<<persistent_grid(dev, 8, chunks), kDThreads, 0, stream>>>(a);
+  timing_end(kKindDecodeCount, stream);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (k == 1) {
+    // one warp per 512-byte unit
+    const int kind = accumulate ? kKindDecodeAccumulate : kKindDecodeWrite;
+    const uint32_t grid = persistent_grid(dev, dev.occ_decode_ix[accumulate ? 1 : 0],
+                                          (units_max + kDWarps - 1) / kDWarps);
+    timing_begin(kind, stream);
+    if (accumulate)
+      k_decode_units<kAccumulate><<<grid, kDThreads, 0, stream>>>(a);
+    else
+      k_decode_units<kWrite><<<grid, kDThreads, 0, stream>>>(a);
+    timing_end(kind, stream);
+    return cudaGetLastError();
+  }
+  if (k == 2) return launch_ix<TLC_GT_ACC / 2, 2>(dev, a, 2, stream);
+  if (k <= 4) return launch_ix<TLC_GT_ACC / 4, 4>(dev, a, 3, stream);
+  return launch_ix<TLC_GT_ACC / 8, 8>(dev, a, 4, stream);
+}
+
+// ---- plans ----------------------------------------------------------------
 template <int kMode>
 static cudaError_t launch_batch_one(const DeviceInfo &dev, const BatchDecodeArgs &a,
-                                    bool deferred, cudaStream_t stream) {
-  const size_t smem = decode_smem_bytes(kMode == kAccumulate);
-  const int occ = kMode == kWrite ? dev.occ_decode_batch_write : dev.occ_decode_batch_acc;
-  uint32_t grid = (uint32_t)dev.sm_count * (uint32_t)(occ > 0 ? occ : 1);
-  if (grid > a.n_tiles) grid = a.n_tiles;
-  if (deferred) {
-    uint32_t cgrid = a.n_chunks;
-    if (cgrid > (uint32_t)dev.sm_count * 8) cgrid = (uint32_t)dev.sm_count * 8;
-    timing_begin(kKindDecodeCount, stream);
-    k_decode_batch_count<<<cgrid, kDThreads, 0, stream>>>(a);
-    timing_end(kKindDecodeCount, stream);
-  }
+                                    bool indexed, cudaStream_t stream) {
   const int kind = kMode == kWrite ? kKindDecodeWrite : kKindDecodeAccumulate;
+  if (!indexed) {
+    const size_t smem = decode_smem_bytes(kMode == kAccumulate);
+    const int occ = kMode == kWrite ? dev.occ_decode_batch_write : dev.occ_decode_batch_acc;
+    timing_begin(kind, stream);
+    k_decode_batch<kMode><<<persistent_grid(dev, occ, a.n_tiles), kDThreads, smem, stream>>>(a);
+    timing_end(kind, stream);
+    return cudaGetLastError();
+  }
+  timing_begin(kKindDecodeCount, stream);
+  k_decode_batch_index<<<persistent_grid(dev, 8, a.n_chunks), kDThreads, 0, stream>>>(a);
+  timing_end(kKindDecodeCount, stream);
+  const int occ = kMode == kWrite ? dev.occ_decode_batch_ix_write : dev.occ_decode_batch_ix_acc;
   timing_begin(kind, stream);
-  if (deferred)
-    k_decode_batch<kMode, true><<<grid, kDThreads, smem, stream>>>(a);
-  else
-    k_decode_batch<kMode, false><<<grid, kDThreads, smem, stream>>>(a);
+  k_decode_batch_units<kMode>
+      <<<persistent_grid(dev, occ, (a.n_tiles + kDWarps - 1) / kDWarps), kDThreads, 0, stream>>>(
+          a);
   timing_end(kind, stream);
   return cudaGetLastError();
 }
@@ -804,12 +1467,14 @@ static cudaError_t launch_batch_one(const DeviceInfo &dev, const BatchDecodeArgs
 cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
                                 const uint8_t *arena, const uint64_t *in_lens, bool accumulate,
                                 int32_t *dev_status, uint32_t max_polls, cudaStream_t stream) {
+  const bool indexed = decode_deferred(p.n_d_tiles);
   cudaError_t e = cudaMemsetAsync(p.d_zero_base, 0, p.d_zero_bytes, stream);
   if (e != cudaSuccess) return e;
   timing_begin(kKindDecodePrepare, stream);
   k_decode_batch_prepare<<<1, kPrepThreads, 0, stream>>>(
-      p.tensors, p.count, arena, in_lens, decode_tile_payload_bytes(accumulate), p.d_prep,
-      p.d_total, dev_status);
+      p.tensors, p.count, arena, in_lens,
+      indexed ? kDecodeUnit : decode_tile_payload_bytes(accumulate), p.d_prep, p.d_total,
+      dev_status);
   timing_end(kKindDecodePrepare, stream);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -821,36 +1486,35 @@ cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
   a.arena = arena;
   a.status = p.d_status;
   a.ticket = p.d_ticket;
-  a.n_tiles = p.n_d_tiles;
+  a.ticket2 = p.d_ticket2;
+  a.n_tiles = p.n_d_tiles;   // units (indexed) or an upper bound of the payload tiles
   a.dev_status = dev_status;
   a.max_polls = max_polls;
-  a.ecount = p.d_ecount;
-  a.csum = p.d_csum;
+  a.off = p.d_off;
+  a.page = p.d_page;
+  a.ok = p.d_ok;
   a.n_chunks = p.n_d_chunks;
-  const bool deferred = decode_deferred(p.n_d_tiles);
-  return accumulate ? launch_batch_one<kAccumulate>(dev, a, deferred, stream)
-                    : launch_batch_one<kWrite>(dev, a, deferred, stream);
+  return accumulate ? launch_batch_one<kAccumulate>(dev, a, indexed, stream)
+                    : launch_batch_one<kWrite>(dev, a, indexed, stream);
 }
 
-int occupancy_decode_batch(bool accumulate) {
+template <int kMode>
+static int batch_occupancy(bool indexed) {
   int occ = 0;
-  const size_t smem = decode_smem_bytes(accumulate);
-  if (accumulate) {
-    cudaFuncSetAttribute(k_decode_batch<kAccumulate, false>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(k_decode_batch<kAccumulate, true>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_batch<kAccumulate, false>,
-                                                  kDThreads, smem);
+  if (indexed) {
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_batch_units<kMode>, kDThreads,
+                                                  0);
   } else {
-    cudaFuncSetAttribute(k_decode_batch<kWrite, false>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(k_decode_batch<kWrite, true>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_batch<kWrite, false>, kDThreads,
-                                                  smem);
+    const size_t smem = decode_smem_bytes(kMode == kAccumulate);
+    cudaFuncSetAttribute(k_decode_batch<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_batch<kMode>, kDThreads, smem);
   }
   return occ;
+}
+
+int occupancy_decode_batch(bool accumulate, bool indexed) {
+  return accumulate ? batch_occupancy<kAccumulate>(indexed) : batch_occupancy<kWrite>(indexed);
 }
 
 cudaError_t launch_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_status,
@@ -863,27 +1527,18 @@ int occupancy_decode(bool accumulate) {
   int occ = 0;
   const size_t smem = decode_smem_bytes(accumulate);
   if (accumulate) {
-    cudaFuncSetAttribute(k_decode<kAccumulate, true, false>,
+    cudaFuncSetAttribute(k_decode<kAccumulate, true>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(k_decode<kAccumulate, false, false>,
+    cudaFuncSetAttribute(k_decode<kAccumulate, false>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(k_decode<kAccumulate, true, true>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(k_decode<kAccumulate, false, true>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode<kAccumulate, true, false>,
-                                                  kDThreads, smem);
-  } else {
-    cudaFuncSetAttribute(k_decode<kWrite, true, false>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(k_decode<kWrite, false, false>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(k_decode<kWrite, true, true>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(k_decode<kWrite, false, true>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode<kWrite, true, false>, kDThreads,
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode<kAccumulate, true>, kDThreads,
                                                   smem);
+  } else {
+    cudaFuncSetAttribute(k_decode<kWrite, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    cudaFuncSetAttribute(k_decode<kWrite, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode<kWrite, true>, kDThreads, smem);
   }
   return occ;
 }

@@ -36,6 +36,47 @@ __device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
   asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
+// ---------------------------------------------------------------------------
+// Debug build (compiled with -DTLC_DEBUG; build.py --debug makes
+// libtlc_debug.so).  Bounds checks that never fault: a failing check records
+// its location (source line | translation unit << 16) in this translation
+// unit's device word, first failure kept, and the access it guards is
+// skipped.  TLC_BOUND(c) guards a clamp that every build needs (c is always
+// evaluated; valid inputs never fail it, so the debug build records when it
+// does); TLC_CHECK(c) guards an index the code keeps in bounds by
+// construction (evaluated in the debug build only).  The host reads the
+// words through tlc_debug_fault().
+// ---------------------------------------------------------------------------
+#ifndef TLC_TU
+#define TLC_TU 0
+#endif
+#ifdef TLC_DEBUG
+static __device__ uint32_t g_tlc_debug_fault;  // one per translation unit
+__device__ __forceinline__ bool debug_check(bool ok, uint32_t where) {
+  if (!ok) atomicCAS(&g_tlc_debug_fault, 0u, where);
+  return ok;
+}
+#define TLC_BOUND(c) (::tlc::debug_check((c), (uint32_t)__LINE__ | ((uint32_t)TLC_TU << 16)))
+#define TLC_CHECK(c) (::tlc::debug_check((c), (uint32_t)__LINE__ | ((uint32_t)TLC_TU << 16)))
+// Host side: this translation unit's word, optionally cleared.
+#define TLC_DEFINE_DEBUG_READER(fn)                                  \
+  uint32_t fn(bool reset) {                                          \
+    uint32_t v = 0;                                                  \
+    if (cudaMemcpyFromSymbol(&v, g_tlc_debug_fault, 4) != cudaSuccess) \
+      v = 0xffffffffu;                                               \
+    if (reset) {                                                     \
+      const uint32_t z = 0;                                          \
+      (void)cudaMemcpyToSymbol(g_tlc_debug_fault, &z, 4);            \
+    }                                                                \
+    return v;                                                        \
+  }
+#else
+#define TLC_BOUND(c) (c)
+#define TLC_CHECK(c) (true)
+#define TLC_DEFINE_DEBUG_READER(fn) \
+  uint32_t fn(bool) { return 0u; }
+#endif
+
 // Record a data-dependent failure; the first error wins, zero is never written.
 __device__ __forceinline__ void report(int32_t *dev_status, int code) {
   if (dev_status) atomicCAS(reinterpret_cast<int *>(dev_status), 0, code);

@@ -8,6 +8,15 @@
 
 namespace tlc {
 
+// The per-call record of a compression (same layout as the public
+// tlc_compress_record): written by the kernels, on the device.
+struct CompressRecord {
+  uint32_t m_bits;
+  float scale;
+  uint64_t nonzeros;
+  uint64_t length;
+};
+
 // Per-device facts, queried once per device and cached for the process.
 struct DeviceInfo {
   int device = -1;
@@ -19,6 +28,9 @@ struct DeviceInfo {
   int occ_quant_batch = 0;
   int occ_decode_batch_write = 0;
   int occ_decode_batch_acc = 0;
+  int occ_decode_batch_ix_write = 0;
+  int occ_decode_batch_ix_acc = 0;
+  int occ_decode_ix[5] = {};  // warp units (write, accumulate); sums of 2, 4, 8 streams
   cudaMemPool_t pool = nullptr;
 };
 
@@ -96,9 +108,11 @@ struct BatchTensor {
   uint32_t q_chunk_begin;          // 32-tile chunks of the deferred placement
   uint32_t d_tile_begin, d_tiles;  // decode 512-byte units (global numbering, upper
                                    // bound of the tiles of either mode)
-  uint32_t d_chunk_begin, d_chunks;  // 32-unit chunks of the counting pass (same)
+  uint32_t d_chunk_begin, d_chunks;  // 32-unit chunks of the index (same)
   uint32_t vec_q;        // x and err 16-byte aligned
   uint32_t vec_y;        // y 16-byte aligned
+  uint32_t d_off_begin;  // indexed plans: the tensor's units' first groups (d_tiles + 1)
+  uint32_t d_page_begin; // and its page table (ceil(groups / 1024) entries)
 };
 
 // Per-tensor facts of one batched decode, written by the prepare kernel.
@@ -106,7 +120,7 @@ struct BatchPrep {
   uint64_t m;            // payload length (0 when the stream is corrupt)
   float scale;
   uint32_t act_begin;    // first tile in the compact numbering
-  uint32_t cact_begin;   // first counting-pass chunk in the compact numbering
+  uint32_t cact_begin;   // first index chunk in the compact numbering
   uint32_t pad;
 };
 
@@ -132,8 +146,10 @@ struct BatchPlanDev {
   void *q_zero_base;      // mbits, q_ticket and q_status, contiguous
   size_t q_zero_bytes;
   uint32_t *d_ticket;
-  uint64_t *d_status;
-  void *d_zero_base;      // d_ticket and d_status, contiguous
+  uint32_t *d_ticket2;    // indexed plans: the decode kernel's ticket
+  uint32_t *d_ok;         // indexed plans: per-tensor valid flags
+  uint64_t *d_status;     // look-back words (per unit, or per index chunk)
+  void *d_zero_base;      // d_ticket, d_ticket2, d_ok and d_status, contiguous
   size_t d_zero_bytes;
   BatchPrep *d_prep;      // count entries, rewritten by every decode call
   uint32_t *d_total;      // compact tile and chunk counts of the current decode call
@@ -141,8 +157,8 @@ struct BatchPlanDev {
   uint64_t *q_cagg;       // deferred placement: per 32-tile chunk summaries,
   uint8_t *q_stage;       // and the staged bytes, compress_stage_bytes_per_tile() per tile;
   uint32_t n_q_chunks;    // tile summaries and chunk counters sit in q_status
-  uint32_t *d_ecount;     // counting pass: group count per 512-byte unit (n_d_tiles)
-  uint64_t *d_csum;       // and per 32-unit chunk (n_d_chunks)
+  uint32_t *d_off;        // indexed plans: units' first groups, all tensors
+  uint32_t *d_page;       // and page tables
   uint32_t n_d_chunks;
 };
 
@@ -153,8 +169,9 @@ cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
                                 const uint8_t *arena, const uint64_t *in_lens, bool accumulate,
                                 int32_t *dev_status, uint32_t max_polls, cudaStream_t stream);
 int occupancy_quant_batch();
-int occupancy_decode_batch(bool accumulate);
+int occupancy_decode_batch(bool accumulate, bool indexed);
 uint32_t decode_tile_payload_bytes(bool accumulate);
+uint32_t decode_pages(uint64_t groups);
 
 // Per-device facts for device d (initialised on first use); nullptr on error.
 const DeviceInfo *device_info(int d);
@@ -178,52 +195,51 @@ size_t compress_scratch_bytes_for(const DeviceInfo &dev, uint64_t n, bool deferr
 // deferred: tiles stage their bytes and two small kernels place them (the
 // scratch must then be compress_scratch_bytes_for(.., true) bytes); else
 // tiles place their bytes themselves with a look-back over earlier tiles.
+// rec: nullptr, or the call's record (device-writable).
 cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, float s, float *err,
                             uint8_t *out, uint64_t out_cap, uint64_t *out_len,
                             int32_t *dev_status, uint32_t max_polls, void *scratch,
-                            cudaStream_t stream, bool deferred);
+                            cudaStream_t stream, bool deferred, CompressRecord *rec = nullptr);
 int occupancy_quant(bool vec);
 
-// Decode scratch per stream: decode_scratch_words(tiles) u64 words, where
-// tiles = decode_tiles_max counts 512-byte payload units (every tile is a
-// whole number of units).
-// Look-back path: status[tiles] (u64) then the ticket (u64 slot); both must
-// be zero before the launch.  Deferred-prefix path (decode_deferred): the
-// units' group counts (u32), the 32-unit chunks' counts (u64), then the
-// ticket; the counting kernel writes all of them, so nothing needs clearing.
+// Decode of one small stream (look-back): scratch of decode_scratch_words(
+// tiles) u64 words, tiles = decode_tiles_max(cap, groups) 512-byte payload
+// units (every tile is a whole number of units): status[tiles] then the
+// ticket; all zero before the launch.
+// Streams whose capacity spans decode_deferred(tiles) units or more, and
+// sums of several streams, go through the index instead
+// (launch_decode_indexed).
 constexpr uint32_t kDecodeUnit = 512;
 constexpr uint32_t kDecodeChunkUnits = 32;
 uint32_t decode_tiles_max(uint64_t cap, uint64_t groups);
 bool decode_deferred(uint32_t tiles);
 inline size_t decode_scratch_words(uint32_t tiles) { return (size_t)tiles + 1; }
 
-struct DecodeScratch {
-  uint64_t *status;   // look-back path
-  uint32_t *ticket;
-  uint32_t *ecount;   // deferred-prefix path
-  uint64_t *csum;
-};
-
-inline DecodeScratch decode_scratch_layout(uint64_t *base, uint32_t tiles, bool deferred) {
-  DecodeScratch d = {};
-  if (deferred) {
-    d.ecount = reinterpret_cast<uint32_t *>(base);
-    d.csum = base + (tiles + 1) / 2;
-    d.ticket = reinterpret_cast<uint32_t *>(d.csum + (tiles + kDecodeChunkUnits - 1) /
-                                                         kDecodeChunkUnits);
-  } else {
-    d.status = base;
-    d.ticket = reinterpret_cast<uint32_t *>(base + tiles);
-  }
-  return d;
-}
-
-// scratch: decode_scratch_words(decode_tiles_max(cap, groups)) words, zero
-// unless decode_deferred(...) of that tile count.
 cudaError_t launch_decode(const DeviceInfo &dev, const uint8_t *in, const uint64_t *len_dev,
                           uint64_t cap, uint64_t n, float *y, bool accumulate,
                           int32_t *dev_status, uint32_t max_polls, uint64_t *scratch,
                           cudaStream_t stream);
+
+// Indexed decode of up to kIndexPass streams of n values each: one index
+// launch and one decode launch (dense output: exactly one stream;
+// accumulate: the streams added in order).  The scratch is
+// indexed_layout(..).total_bytes bytes; the launcher clears its first
+// zero_bytes itself.
+constexpr int kIndexPass = 8;
+struct IndexedStream {
+  const uint8_t *in;
+  const uint64_t *len_dev;  // or nullptr: cap is the exact length
+  uint64_t cap;
+};
+struct IndexedLayout {
+  size_t status_off[kIndexPass], off_off[kIndexPass], page_off[kIndexPass];
+  size_t zero_bytes, total_bytes;
+};
+IndexedLayout indexed_layout(const IndexedStream *s, int k, uint64_t n);
+cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s, int k, uint64_t n,
+                                  float *y, bool accumulate, int32_t *dev_status,
+                                  uint32_t max_polls, void *scratch, cudaStream_t stream);
+void occupancy_decode_ix(int occ[5]);
 cudaError_t launch_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_status,
                              cudaStream_t stream);
 cudaError_t launch_compress_wait_test(uint64_t *status, uint32_t max_polls, int32_t *dev_status,

@@ -8,8 +8,9 @@ node of B200s this is:
 1. every rank compresses its own gradient with its own error buffer
    (``tlc_compress``, or ``tlc_compress_batch`` for a tensor list);
 2. the variable-length streams are all-gathered: first the lengths (one
-   int64 per rank), then every rank's stream in a slot as long as the
-   longest one, so only about world * max(length) bytes cross NVLink;
+   int64 per rank, kept on the device), then every rank's stream in a slot
+   as long as the longest one, so only about world * max(length) bytes
+   cross NVLink; the slot width is the one number read back to the host;
 3. every rank adds all ranks' decoded streams, in rank order, into its
    aggregation buffer (``tlc_decompress_accumulate``, K = world), so all
    ranks hold bit-identical sums.
@@ -53,42 +54,52 @@ def max_over_ranks(values, device=None, group=None):
     return [float(v) for v in t.tolist()]
 
 
+def _length_tensor(length, device):
+    if isinstance(length, torch.Tensor):
+        return length.reshape(1).to(torch.int64)
+    return torch.tensor([int(length)], dtype=torch.int64, device=device)
+
+
 def allgather_streams(stream, length, group=None):
     """All-gather one variable-length byte stream per rank.
 
     stream: uint8 tensor holding this rank's stream in its first `length`
-    bytes (device or host, as the backend needs); length: int.  Returns
-    (slots, lengths): slots is a [world, max_length] uint8 tensor on the
-    stream's device whose row r holds rank r's stream in its first
-    lengths[r] bytes; lengths is a list of ints.  Two collectives: the
-    lengths, then the slots (every rank sends exactly max_length bytes).
-    """
+    bytes (device or host, as the backend needs); length: a one-element
+    int64 tensor on the same device (or an int).  Returns (slots, lengths):
+    slots is a [world, width] uint8 tensor whose row r holds rank r's stream
+    in its first lengths[r] bytes, width the longest length; lengths is an
+    int64 tensor [world] on the stream's device.  Two collectives (the
+    lengths, then the slots) and one host read, of the width, which the
+    second collective's size needs."""
     world = dist.get_world_size(group)
     dev = stream.device
-    mine = torch.tensor([int(length)], dtype=torch.int64, device=dev)
-    lens = [torch.empty_like(mine) for _ in range(world)]
-    dist.all_gather(lens, mine, group=group)
-    lengths = [int(t.item()) for t in lens]
-    width = max(max(lengths), 1)
-    slot = torch.zeros(width, dtype=torch.uint8, device=dev)
-    slot[: int(length)].copy_(stream[: int(length)])
-    rows = [torch.empty_like(slot) for _ in range(world)]
-    dist.all_gather(rows, slot, group=group)
-    return torch.stack(rows), lengths
+    mine = _length_tensor(length, dev)
+    lens = torch.empty(world, dtype=torch.int64, device=dev)
+    dist.all_gather_into_tensor(lens, mine, group=group)
+    width = max(int(lens.max().item()), 1)
+    if stream.numel() >= width:
+        slot = stream[:width].contiguous()
+    else:
+        slot = torch.zeros(width, dtype=torch.uint8, device=dev)
+        slot[: stream.numel()].copy_(stream)
+    rows = torch.empty(world, width, dtype=torch.uint8, device=dev)
+    dist.all_gather_into_tensor(rows.view(-1), slot, group=group)
+    return rows, lens
 
 
 def exchange_step(x, s, err, acc, group=None, dev_status=None, codec=None):
     """One data-parallel step: compress x (err updated in place), all-gather
     the streams, add all ranks' decoded values into acc (rank order).
-    codec defaults to CudaCodec (CUDA tensors).  Returns (lengths, dev_status
-    tensor)."""
+    codec defaults to CudaCodec (CUDA tensors).  Returns (lengths, dev_status):
+    lengths is an int64 tensor [world] on x's device.  The step reads one
+    number back to the host (the slot width of the all-gather)."""
     codec = codec if codec is not None else CudaCodec()
     n = x.numel()
     st = dev_status if dev_status is not None else torch.zeros(
         1, dtype=torch.int32, device=x.device)
     out, length = codec.compress(x, s, err, st)
     slots, lengths = allgather_streams(out, length, group)
-    codec.accumulate([slots[r, :lengths[r]] for r in range(slots.shape[0])], lengths, n, acc, st)
+    codec.accumulate(slots, lengths, n, acc, st)
     return lengths, st
 
 
@@ -106,55 +117,60 @@ def alltoall_streams(streams, lengths, group=None):
     """All-to-all of variable-length byte streams.
 
     streams[d] holds, in its first lengths[d] bytes, the stream this rank
-    sends to rank d (uint8 tensors on the backend's device).  Returns
-    (slots, lengths_in): slots is a [world, width] uint8 tensor whose row s
-    holds rank s's stream for this rank in its first lengths_in[s] bytes.
-    Three collectives: the lengths (all-to-all), the common slot width (the
-    longest stream anywhere, an all-reduce), then the slots (all-to-all)."""
+    sends to rank d (uint8 tensors on the backend's device); lengths[d] is a
+    one-element int64 tensor on that device (or an int).  Returns (slots,
+    lengths_in): slots is a [world, width] uint8 tensor whose row s holds
+    rank s's stream for this rank in its first lengths_in[s] bytes;
+    lengths_in is an int64 tensor [world].  Three collectives (the lengths,
+    the common slot width as a maximum over ranks, the slots) and one host
+    read, of the width."""
     world = dist.get_world_size(group)
     dev = streams[0].device
-    mine = torch.tensor([int(v) for v in lengths], dtype=torch.int64, device=dev)
+    mine = torch.cat([_length_tensor(v, dev) for v in lengths])
     lens_in = torch.empty_like(mine)
     dist.all_to_all_single(lens_in, mine, group=group)
-    width_t = torch.tensor([max(int(mine.max().item()), 1)], dtype=torch.int64, device=dev)
+    width_t = mine.max().reshape(1).clone()
     dist.all_reduce(width_t, op=dist.ReduceOp.MAX, group=group)
-    width = int(width_t.item())
-    send = torch.zeros(world * width, dtype=torch.uint8, device=dev)
+    width = max(int(width_t.item()), 1)
+    send = torch.zeros(world, width, dtype=torch.uint8, device=dev)
     for d in range(world):
-        L = int(lengths[d])
-        send[d * width: d * width + L].copy_(streams[d][:L])
+        L = min(width, streams[d].numel())
+        send[d, :L].copy_(streams[d][:L])
     recv = torch.empty_like(send)
-    dist.all_to_all_single(recv, send, group=group)
-    return recv.view(world, width), [int(v) for v in lens_in.tolist()]
+    dist.all_to_all_single(recv.view(-1), send.view(-1), group=group)
+    return recv, lens_in
 
 
 class CudaCodec:
     """The codec steps of both exchange forms through libtlc.so (CUDA
-    tensors).  Each method enqueues work on the current stream; a length is
-    read back to the host only where the transport needs it."""
+    tensors).  Each method only enqueues work on the current stream; the
+    lengths stay on the device (the decoders read them there)."""
 
     def __init__(self):
         from . import tlc
         self.tlc = tlc
 
     def compress(self, x, s, err, dev_status):
+        """(stream buffer of tlc_compress_bound(n) bytes, length as a
+        one-element int64 device tensor)."""
         t = self.tlc
         out = torch.empty(t.tlc_compress_bound(x.numel()), dtype=torch.uint8, device=x.device)
         out_len = torch.zeros(1, dtype=torch.int64, device=x.device)
         t.tlc_compress(x, s, err, out, out_len, dev_status)
-        length = int(out_len.item())
-        if length == 0:
-            raise RuntimeError(f"compression failed (status {int(dev_status.item())})")
-        return out, length
+        return out, out_len
 
-    def accumulate(self, streams, lengths, n, acc, dev_status):
-        rows = [st.contiguous() for st in streams]
-        self.tlc.tlc_decompress_accumulate(rows, n, acc, in_caps=[int(v) for v in lengths],
+    def accumulate(self, rows, lengths, n, acc, dev_status):
+        """acc += the decoded rows, in row order; rows: [k, width] uint8,
+        lengths: int64 [k] on the device."""
+        k, width = rows.shape
+        self.tlc.tlc_decompress_accumulate([rows[r] for r in range(k)], n, acc,
+                                           in_lens=lengths.contiguous(), in_caps=[width] * k,
                                            dev_status=dev_status)
 
-    def decompress(self, stream, length, n, y, dev_status):
-        self.tlc.tlc_decompress(stream.contiguous(), n, y, in_cap=int(length),
-                                dev_status=dev_status)
+    def decompress(self, row, length, n, y, dev_status):
+        """y = the decoded row (uint8 [width]); length: one-element int64."""
+        self.tlc.tlc_decompress(row, n, y, in_len=length.reshape(1).contiguous(),
+                                in_cap=row.numel(), dev_status=dev_status)
 
 
 def exchange_step_sharded(x, s, err, server_err, y, group=None, codec=None, dev_status=None):
@@ -164,7 +180,10 @@ def exchange_step_sharded(x, s, err, server_err, y, group=None, codec=None, dev_
     (n values, updated); server_err: the error buffer of the shard this rank
     serves (shard_bounds(n, world)[r + 1] - [r] values, updated); y: receives
     the model delta (n values, the same on every rank).  codec defaults to
-    CudaCodec.  Returns (lengths sent per shard, delta stream lengths)."""
+    CudaCodec.  Returns (lengths this rank sent per shard, delta stream
+    lengths per shard), int64 tensors [world] on x's device.  The step reads
+    two numbers back to the host (the slot widths of its two variable-size
+    collectives)."""
     codec = codec if codec is not None else CudaCodec()
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
@@ -183,11 +202,11 @@ def exchange_step_sharded(x, s, err, server_err, y, group=None, codec=None, dev_
     # 3. server side: aggregate in rank order, compress the model delta
     m = b[rank + 1] - b[rank]
     agg = torch.zeros(m, dtype=torch.float32, device=x.device)
-    codec.accumulate([slots[r, :lens_in[r]] for r in range(world)], lens_in, m, agg, st)
+    codec.accumulate(slots, lens_in, m, agg, st)
     down, down_len = codec.compress(agg, s, server_err, st)
     # 4. every shard's delta to every rank
     rows, lens_down = allgather_streams(down, down_len, group)
     for d in range(world):
-        codec.decompress(rows[d, :lens_down[d]], lens_down[d], b[d + 1] - b[d],
-                         y[b[d]:b[d + 1]], st)
-    return [u[1] for u in ups], lens_down
+        codec.decompress(rows[d], lens_down[d:d + 1], b[d + 1] - b[d], y[b[d]:b[d + 1]], st)
+    ups_len = torch.cat([_length_tensor(u[1], x.device) for u in ups])
+    return ups_len, lens_down

@@ -27,13 +27,17 @@ class TLCError(RuntimeError):
 
 
 def lib() -> ctypes.CDLL:
-    """Load libtlc.so (building it with nvcc first if it does not exist)."""
+    """Load libtlc.so (building it with nvcc first if it does not exist).
+    With TLC_LIB=debug in the environment, load the debug build,
+    libtlc_debug.so, instead (recording bounds checks and scratch canaries;
+    see tlc_debug_fault)."""
     global _lib
     if _lib is not None:
         return _lib
-    path = _build.library_path()
+    debug = os.environ.get("TLC_LIB", "") == "debug"
+    path = _build.library_path(debug)
     if not os.path.exists(path):
-        _build.build_library()
+        _build.build_library(debug=debug)
     L = ctypes.CDLL(path)
     P, S, U64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint64
     L.tlc_compress_bound.argtypes = [S]
@@ -54,6 +58,8 @@ def lib() -> ctypes.CDLL:
     L.tlc_test_wait_timeout.restype = ctypes.c_int
     L.tlc_test_compress_wait_timeout.argtypes = [ctypes.c_uint32, P, P]
     L.tlc_test_compress_wait_timeout.restype = ctypes.c_int
+    L.tlc_compress_recorded.argtypes = [P, S, ctypes.c_float, P, P, S, P, P, P, P]
+    L.tlc_compress_recorded.restype = ctypes.c_int
     L.tlc_compress_noalloc.argtypes = [P, S, ctypes.c_float, P, P, S, P, P, P]
     L.tlc_compress_noalloc.restype = ctypes.c_int
     L.tlc_plan_create.argtypes = [ctypes.c_int, P, P, P, P, P]
@@ -76,6 +82,10 @@ def lib() -> ctypes.CDLL:
     L.tlc_kernel_timing_kinds.restype = None
     L.tlc_kernel_name.argtypes = [ctypes.c_int]
     L.tlc_kernel_name.restype = ctypes.c_char_p
+    L.tlc_debug_build.argtypes = []
+    L.tlc_debug_build.restype = ctypes.c_int
+    L.tlc_debug_fault.argtypes = [ctypes.c_int]
+    L.tlc_debug_fault.restype = ctypes.c_uint32
     _ = U64
     _lib = L
     return L
@@ -141,6 +151,37 @@ def tlc_compress(x, s: float, err, out, out_len, dev_status=None, stream=None) -
         _dev_ptr(out, "out", torch.uint8), out.numel(), _dev_ptr(out_len, "out_len"),
         _dev_ptr(dev_status, "dev_status", torch.int32), _stream(stream))
     return _check("tlc_compress", code)
+
+
+RECORD_BYTES = 24   # sizeof(tlc_compress_record)
+
+
+def tlc_compress_recorded(x, s: float, err, out, out_len, record, dev_status=None,
+                          stream=None) -> int:
+    """tlc_compress that also fills `record`: a CUDA tensor of at least 24
+    bytes (e.g. torch.empty(24, dtype=torch.uint8, device=...)) that
+    receives the call's tlc_compress_record; read it with record_fields."""
+    import torch
+    if record.numel() * record.element_size() < RECORD_BYTES:
+        raise ValueError("record needs 24 bytes")
+    n = x.numel()
+    code = lib().tlc_compress_recorded(
+        _dev_ptr(x, "x", torch.float32), n, float(s), _dev_ptr(err, "err", torch.float32),
+        _dev_ptr(out, "out", torch.uint8), out.numel(), _dev_ptr(out_len, "out_len"),
+        _dev_ptr(dev_status, "dev_status", torch.int32), _dev_ptr(record, "record"),
+        _stream(stream))
+    return _check("tlc_compress_recorded", code)
+
+
+def record_fields(record) -> dict:
+    """The fields of a tlc_compress_record as the device wrote them (copies
+    the 24 bytes to the host, which waits for the call): m_bits, scale,
+    nonzeros, length."""
+    import struct
+    raw = bytes(record.reshape(-1).view(__import__("torch").uint8)[:RECORD_BYTES].cpu()
+                .numpy().tobytes())
+    m_bits, scale, nonzeros, length = struct.unpack("<IfQQ", raw)
+    return {"m_bits": m_bits, "scale": scale, "nonzeros": nonzeros, "length": length}
 
 
 NOALLOC_MAX_N = 1 << 29
@@ -303,6 +344,17 @@ def tlc_test_compress_wait_timeout(max_polls: int, dev_status, stream=None) -> i
     code = lib().tlc_test_compress_wait_timeout(
         int(max_polls), _dev_ptr(dev_status, "dev_status", torch.int32), _stream(stream))
     return _check("tlc_test_compress_wait_timeout", code)
+
+
+def tlc_debug_build() -> bool:
+    """True when the loaded library is the debug build."""
+    return bool(lib().tlc_debug_build())
+
+
+def tlc_debug_fault(reset: bool = True) -> int:
+    """First failed debug check (source line | file id << 16), 0 if none; always
+    0 outside the debug build.  Waits for the device's queued work."""
+    return int(lib().tlc_debug_fault(1 if reset else 0))
 
 
 def tlc_kernel_timing(enable: bool) -> None:

@@ -102,6 +102,31 @@ tlc_status tlc_compress(const float *x, size_t n, float s, float *err,
                         uint8_t *out, size_t out_cap, uint64_t *out_len,
                         int32_t *dev_status, tlc_stream_t stream);
 
+/* What one compression did, written by the device ("Findings" bullet 1
+ * quotes the method's effect as bits per value and compression ratio):
+ *   m_bits    IEEE-754 bits of M = max_i |x_i + err_i| (0x7f800000 or more:
+ *             the step was non-finite)
+ *   scale     M * s, the value in the stream header (0 when non-finite)
+ *   nonzeros  number of values with q != 0
+ *   length    stream length 4 + m in bytes (0 when non-finite), the same
+ *             value as *out_len; bits per value = 8 * length / n. */
+typedef struct {
+    uint32_t m_bits;
+    float scale;
+    uint64_t nonzeros;
+    uint64_t length;
+} tlc_compress_record;
+
+/* tlc_compress that also fills *record (device-writable memory: device or
+ * mapped pinned host memory), in the same stream order as the stream
+ * itself.  Arguments, results and errors otherwise those of tlc_compress;
+ * record == NULL is TLC_ERR_INVALID_ARG.  The stream and error buffer are
+ * bit-identical to tlc_compress's. */
+tlc_status tlc_compress_recorded(const float *x, size_t n, float s, float *err,
+                                 uint8_t *out, size_t out_cap, uint64_t *out_len,
+                                 int32_t *dev_status, tlc_compress_record *record,
+                                 tlc_stream_t stream);
+
 /* Decompress one stream into a dense fp32 tensor (inverse of bullets 1-3):
  * y_i = +scale, -scale or +0.0 for q_i = 1, -1, 0.
  *
@@ -225,6 +250,20 @@ tlc_status tlc_decompress_batch(tlc_plan plan, const uint8_t *arena, const uint6
 tlc_status tlc_compress_noalloc(const float *x, size_t n, float s, float *err,
                                 uint8_t *out, size_t out_cap, uint64_t *out_len,
                                 int32_t *dev_status, tlc_stream_t stream);
+
+/* Debug build.  libtlc_debug.so (the same sources compiled with
+ * -DTLC_DEBUG) checks every index of its shared-memory staging, stream
+ * placement and page tables before the access, and puts 256-byte canaries of
+ * 0xA5 on both sides of every scratch allocation, checked by a small kernel
+ * when the scratch is freed.  A failing check never faults: it records its
+ * location (source line | file id << 16; file ids 1 compress, 2 decode,
+ * 3 API) and skips the access.
+ * tlc_debug_build() is 1 in that library and 0 in libtlc.so.
+ * tlc_debug_fault(reset) returns the first recorded location, or 0 (always
+ * 0 in libtlc.so), and clears it when reset is non-zero.  It reads device
+ * memory, so it waits for the device's queued work. */
+int tlc_debug_build(void);
+uint32_t tlc_debug_fault(int reset);
 
 /* Human-readable name of a status code (static string). */
 const char *tlc_status_string(tlc_status status);

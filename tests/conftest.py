@@ -77,6 +77,22 @@ def load_quartic_anchors():
     return out
 
 
+@pytest.fixture(autouse=True)
+def _debug_build_checks(request):
+    """Under TLC_LIB=debug (the debug build of the library), every GPU test
+    also requires that no bounds check or scratch canary failed."""
+    yield
+    if os.environ.get("TLC_LIB") != "debug" or request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import gradient_traffic_compression_b200 as g
+    assert g.tlc_debug_build(), "TLC_LIB=debug but the release library is loaded"
+    fault = g.tlc_debug_fault(reset=True)
+    assert fault == 0, f"debug check failed at line {fault & 0xFFFF} of file id {fault >> 16}"
+
+
 @pytest.fixture(scope="session")
 def orc():
     import oracle

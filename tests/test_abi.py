@@ -170,3 +170,19 @@ def test_stream_info_reads_the_header():
     assert info["length"] == st.size and info["scale"] == np.float32(4.5)
     assert info["bits_per_value"] == 8.0 * st.size / 1000
     assert set(info) == {"length", "bits_per_value", "scale"}   # header facts only
+
+
+def test_debug_build_compiles_and_says_so(L):
+    # the debug build (recording bounds checks, scratch canaries) is the
+    # same sources with -DTLC_DEBUG; it exports the same symbols
+    import ctypes
+
+    from gradient_traffic_compression_b200 import build
+    path = build.ensure_built(debug=True)
+    D = ctypes.CDLL(path)
+    missing = [fn for fn in declared_functions() if not hasattr(D, fn)]
+    assert not missing
+    D.tlc_debug_build.restype = ctypes.c_int
+    assert D.tlc_debug_build() == 1
+    assert L.tlc_debug_build() == 0
+    assert L.tlc_debug_fault(1) == 0      # nothing to record in the release build

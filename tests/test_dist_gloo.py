@@ -49,7 +49,8 @@ def _worker(rank, world, port, q):
         rc, st, _ = oracle.compress(x, 1.75, np.zeros(n, np.float32))
         buf = torch.zeros(st.size + 17, dtype=torch.uint8)
         buf[: st.size] = torch.from_numpy(st)
-        slots, lengths = allgather_streams(buf, st.size)
+        slots, lengths = allgather_streams(buf, torch.tensor([st.size]))
+        lengths = lengths.tolist()
         streams = [slots[r, : lengths[r]].numpy().copy() for r in range(world)]
         rc2, acc = oracle.decompress_accumulate(streams, n, np.zeros(n, np.float32))
         q.put((rank, mx, lengths, [s_.tolist() for s_ in streams], acc.tobytes(), rc, rc2))
@@ -96,8 +97,9 @@ def test_two_gloo_ranks_exchange_and_time():
 
 
 class _OracleCodec:
-    """The codec steps of exchange_step_sharded on host tensors through the
-    CPU oracle (test code only; on GPUs the CUDA codec runs them)."""
+    """The codec steps of both exchange forms on host tensors through the
+    CPU oracle (test code only; on GPUs the CUDA codec runs them), with the
+    codec interface of CudaCodec: lengths travel as int64 tensors."""
 
     def compress(self, x, s, err, dev_status):
         import torch
@@ -106,22 +108,22 @@ class _OracleCodec:
         rc, st, e2 = oracle.compress(x.numpy(), s, err.numpy())
         assert rc == 0
         err.copy_(torch.from_numpy(e2))
-        return torch.from_numpy(st), int(st.size)
+        return torch.from_numpy(st), torch.tensor([st.size], dtype=torch.int64)
 
-    def accumulate(self, streams, lengths, n, acc, dev_status):
+    def accumulate(self, rows, lengths, n, acc, dev_status):
         import torch
 
         import oracle
-        rc, a = oracle.decompress_accumulate([t[:L].numpy() for t, L in zip(streams, lengths)],
-                                             n, acc.numpy())
+        rc, a = oracle.decompress_accumulate(
+            [rows[r, :L].numpy() for r, L in enumerate(lengths.tolist())], n, acc.numpy())
         assert rc == 0
         acc.copy_(torch.from_numpy(a))
 
-    def decompress(self, stream, length, n, y, dev_status):
+    def decompress(self, row, length, n, y, dev_status):
         import torch
 
         import oracle
-        rc, v = oracle.decompress(stream[:length].numpy(), n)
+        rc, v = oracle.decompress(row[:int(length.reshape(-1)[0])].numpy(), n)
         assert rc == 0
         y.copy_(torch.from_numpy(v))
 
@@ -157,7 +159,7 @@ def _sharded_worker(rank, world, port, n, steps, q):
             up, down = exchange_step_sharded(x, 1.5, err, server_err, y, codec=_OracleCodec(),
                                              dev_status=torch.zeros(1, dtype=torch.int32))
             ys.append(y.numpy().tobytes())
-        q.put((rank, ys, up, down))
+        q.put((rank, ys, up.tolist(), down.tolist()))
         dist.barrier()
         dist.destroy_process_group()
     except Exception as e:  # report to the parent instead of hanging it
@@ -232,7 +234,7 @@ def _allgather_worker(rank, world, port, n, q):
         acc = torch.zeros(n, dtype=torch.float32)
         lengths, _ = exchange_step(x, 1.5, err, acc, codec=_OracleCodec(),
                                    dev_status=torch.zeros(1, dtype=torch.int32))
-        q.put((rank, acc.numpy().tobytes(), lengths, err.numpy().tobytes()))
+        q.put((rank, acc.numpy().tobytes(), lengths.tolist(), err.numpy().tobytes()))
         dist.barrier()
         dist.destroy_process_group()
     except Exception as e:  # report to the parent instead of hanging it

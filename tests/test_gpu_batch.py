@@ -256,3 +256,56 @@ def test_batch_deferred_placement_many_tensors(g):
             assert b.stream(i).tolist() == st.tolist(), f"step {step} tensor {i} (n={x.size})"
             assert np.array_equal(bits(b.errs[i].cpu().numpy()), bits(e2)), f"err {i}"
             errs[i] = e2
+
+
+def test_batch_indexed_plan_mixes_gather_and_payload_tiles(g):
+    # an indexed plan (8.4 M groups or more) whose tensors take different
+    # tilings: dense streams (uniform values, about one group per payload
+    # byte) take output tiles, sparse ones payload tiles; one y off 16-byte
+    # alignment, and a corrupt stream among them
+    sizes = [5 * 16384 * 512 + 11, 333_333, 4_000_003, 1_500_000, 77]
+    xs, errs = [], []
+    for i, n in enumerate(sizes):
+        if i in (0, 3, 4):
+            x = (synth.uniforms(synth.key_for(160 + i, 0), n) * 2 - 1).astype(np.float32)
+            e = np.zeros(n, np.float32)
+        else:
+            x, e = mixed(160 + i, n, zero_frac=0.97, sigma=1e-3)
+        xs.append(x)
+        errs.append(e)
+    b = Batch(g, xs, errs, offsets=[0, 0, 0, 1, 0])
+    b.plan.compress(1.25, b.arena, b.lens, b.status)
+    b.plan.decompress(b.arena, b.lens, accumulate=False, dev_status=b.status)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    streams = []
+    for i, x in enumerate(xs):
+        rc, st, _ = oracle.compress(x, 1.25, errs[i])
+        assert rc == 0
+        assert b.stream(i).tolist() == st.tolist(), f"tensor {i}"
+        groups = (x.size + 4) // 5
+        if i in (0, 3):
+            assert groups <= 4 * (st.size - 4), "a dense stream"
+        if i in (1, 2):
+            assert groups > 4 * (st.size - 4), "a sparse stream"
+        _, y = oracle.decompress(st, x.size)
+        assert np.array_equal(bits(b.ys[i].cpu().numpy()), bits(y)), f"y {i}"
+        streams.append(st)
+    accs0 = [synth.normal(synth.key_for(170 + i, 2), n, 1.0) for i, n in enumerate(sizes)]
+    for t, a in zip(b.ys, accs0):
+        t.copy_(torch.from_numpy(a))
+    b.plan.decompress(b.arena, b.lens, accumulate=True, dev_status=b.status)
+    torch.cuda.synchronize()
+    assert int(b.status.item()) == 0
+    for i, x in enumerate(xs):
+        _, want = oracle.decompress_accumulate([streams[i]], x.size, accs0[i])
+        assert np.array_equal(bits(b.ys[i].cpu().numpy()), bits(want)), f"acc {i}"
+    lens = b.lens.clone()
+    lens[0] -= 1
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    b.plan.decompress(b.arena, lens, dev_status=st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) == 3
+    for i in (1, 2, 3, 4):
+        _, y = oracle.decompress(streams[i], sizes[i])
+        assert np.array_equal(bits(b.ys[i].cpu().numpy()), bits(y)), f"y {i} after corrupt"

@@ -54,7 +54,7 @@ def test_exchange_step_one_rank():
         torch.cuda.synchronize()
         assert int(st.item()) == 0
         rc, stream, err_o = oracle.compress(x_h, 1.75, e_h)
-        assert lengths == [stream.size]
+        assert lengths.tolist() == [stream.size]
         _, acc_o = oracle.decompress_accumulate([stream], n, acc0)
         assert np.array_equal(acc.cpu().numpy().view(np.uint32), acc_o.view(np.uint32))
         assert np.array_equal(err.cpu().numpy().view(np.uint32), err_o.view(np.uint32))
@@ -90,7 +90,7 @@ def test_exchange_step_sharded_one_rank():
         _, agg = oracle.decompress_accumulate([s_up], n, np.zeros(n, np.float32))
         rc2, s_down, serr_o = oracle.compress(agg, 1.5, se_h)
         _, y_o = oracle.decompress(s_down, n)
-        assert rc == rc2 == 0 and up == [s_up.size] and down == [s_down.size]
+        assert rc == rc2 == 0 and up.tolist() == [s_up.size] and down.tolist() == [s_down.size]
         bits = lambda a: np.ascontiguousarray(a).view(np.uint32)  # noqa: E731
         assert np.array_equal(bits(err.cpu().numpy()), bits(err_o))
         assert np.array_equal(bits(server_err.cpu().numpy()), bits(serr_o))
