@@ -474,7 +474,7 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   std::vector<tlc::BatchChunk> chunks;
   std::vector<uint32_t> qtt, dtt;
   std::vector<uint64_t> offsets(count + 1, 0);
-  uint64_t n_dchunks = 0, n_qchunks = 0, n_off = 0, n_pages = 0;
+  uint64_t n_dchunks = 0, n_qchunks = 0;
   for (int i = 0; i < count; ++i) {
     tlc::BatchTensor &t = T[i];
     t.x = xs ? xs[i] : nullptr;
@@ -496,16 +496,12 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
     t.d_chunk_begin = (uint32_t)n_dchunks;
     t.d_chunks = (t.d_tiles + tlc::kDecodeChunkUnits - 1) / tlc::kDecodeChunkUnits;
     n_dchunks += t.d_chunks;
-    t.d_off_begin = (uint32_t)n_off;
-    n_off += (uint64_t)t.d_tiles + 1;
-    t.d_page_begin = (uint32_t)n_pages;
-    n_pages += tlc::decode_pages(t.groups);
     t.vec_q = xs && (((reinterpret_cast<uintptr_t>(t.x) | reinterpret_cast<uintptr_t>(t.err)) &
                       15) == 0);
     t.vec_y = ys && ((reinterpret_cast<uintptr_t>(t.y) & 15) == 0);
     for (uint64_t b = 0; b < t.n; b += tlc::kBatchChunk) chunks.push_back({(uint32_t)i, 0u, b});
     if (qtt.size() >= (1ull << 31) || dtt.size() >= (1ull << 31) ||
-        chunks.size() >= (1ull << 31) || n_off >= (1ull << 31) || n_pages >= (1ull << 31))
+        chunks.size() >= (1ull << 31) || n_dchunks + count >= (1ull << 31))
       return TLC_ERR_INVALID_ARG;
   }
   // device layout: tables, then the zeroed-per-call scratch of each direction
@@ -515,14 +511,16 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   const size_t sz_D = tlc::align_up(4 * dtt.size(), 256);
   const size_t sz_M = tlc::align_up(4 * (size_t)count + 8, 256);      // mbits, q_ticket
   const size_t sz_QS = tlc::align_up(8 * qtt.size(), 256);
-  // decode: tickets, per-tensor valid flags, look-back words (per unit for
-  // small plans, per index chunk for indexed ones), zeroed per call
+  // decode, zeroed per call: the ticket, per-tensor valid flags and
+  // finished-chunk counters, and (small plans) one look-back word per unit
   const bool d_ix = tlc::decode_deferred((uint32_t)dtt.size());
-  const size_t d_head = tlc::align_up(8 + 4 * (size_t)count, 8);
-  const size_t sz_DS = tlc::align_up(d_head + 8 * dtt.size(), 256);
+  const size_t d_head = tlc::align_up(4 + 8 * (size_t)count, 8);
+  const size_t sz_DS = tlc::align_up(d_head + (d_ix ? 0 : 8 * dtt.size()), 256);
   const size_t sz_P = tlc::align_up(sizeof(tlc::BatchPrep) * count + 8, 256);  // prep, total
-  const size_t sz_E = d_ix ? tlc::align_up(4 * n_off, 256) : 0;      // index: units' first groups
-  const size_t sz_S = d_ix ? tlc::align_up(4 * n_pages, 256) : 0;    // index: page tables
+  // the index of indexed plans: units' first groups in their chunk, chunks'
+  // first groups
+  const size_t sz_E = d_ix ? tlc::align_up(4 * dtt.size(), 256) : 0;
+  const size_t sz_S = d_ix ? tlc::align_up(4 * (n_dchunks + count), 256) : 0;
   // deferred placement of the compress side: chunk summaries, staging
   const bool q_def = xs && tlc::compress_deferred_tiles(qtt.size());
   const size_t sz_QC = q_def ? tlc::align_up(8 * n_qchunks, 256) : 0;
@@ -557,16 +555,16 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   D.q_zero_bytes = sz_M + 8 * qtt.size();
   char *zd = zq + sz_M + sz_QS;
   D.d_ticket = reinterpret_cast<uint32_t *>(zd);
-  D.d_ticket2 = reinterpret_cast<uint32_t *>(zd + 4);
-  D.d_ok = reinterpret_cast<uint32_t *>(zd + 8);
-  D.d_status = reinterpret_cast<uint64_t *>(zd + d_head);
+  D.d_ok = reinterpret_cast<uint32_t *>(zd + 4);
+  D.d_done = reinterpret_cast<uint32_t *>(zd + 4 + 4 * (size_t)count);
+  D.d_status = d_ix ? nullptr : reinterpret_cast<uint64_t *>(zd + d_head);
   D.d_zero_base = zd;
-  D.d_zero_bytes = d_head + 8 * (d_ix ? n_dchunks : dtt.size());
+  D.d_zero_bytes = d_head + (d_ix ? 0 : 8 * dtt.size());
   D.d_prep = reinterpret_cast<tlc::BatchPrep *>(zd + sz_DS);
   D.d_total = reinterpret_cast<uint32_t *>(zd + sz_DS + sizeof(tlc::BatchPrep) * count);
   P->spare_status = reinterpret_cast<int32_t *>(zd + sz_DS + sz_P);
-  D.d_off = d_ix ? reinterpret_cast<uint32_t *>(zd + sz_DS + sz_P + 256) : nullptr;
-  D.d_page = d_ix ? reinterpret_cast<uint32_t *>(zd + sz_DS + sz_P + 256 + sz_E) : nullptr;
+  D.d_loc = d_ix ? reinterpret_cast<uint32_t *>(zd + sz_DS + sz_P + 256) : nullptr;
+  D.d_cpre = d_ix ? reinterpret_cast<uint32_t *>(zd + sz_DS + sz_P + 256 + sz_E) : nullptr;
   D.n_d_chunks = (uint32_t)n_dchunks;
   D.q_deferred = q_def;
   D.q_cagg = q_def ? reinterpret_cast<uint64_t *>(zd + sz_DS + sz_P + 256 + sz_E + sz_S) : nullptr;

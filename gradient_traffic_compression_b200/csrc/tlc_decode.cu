@@ -11,36 +11,33 @@
 //   kAccumulate  acc_i += y_i only where q_i != 0 (acc keeps its bits at
 //                zeros), streams in worker order
 //
-// Small streams (capacity below 8 MiB), one stream at a time: k_decode, one
-// launch.  A tile is 512 (kWrite) or 2048 (kAccumulate) payload bytes: per
-// tile, expansion counts e_k (an escape byte b >= 243 stands for b - 241
-// groups of 121, any other byte for itself), a block scan, and a decoupled
-// look-back over earlier tiles for the tile's first group index.
+// Small streams (capacity below 8 MiB), one at a time: k_decode, one launch.
+// A tile is 512 (kWrite) or 2048 (kAccumulate) payload bytes: per tile,
+// expansion counts e_k (an escape byte b >= 243 stands for b - 241 groups of
+// 121, any other byte for itself), a block scan, and a decoupled look-back
+// over earlier tiles for the tile's first group index.
 //
 // Large streams, and several streams summed in one pass: an index, then the
-// decode.
-//   k_decode_index  per 32-unit chunk of 512-byte payload units: the units'
-//                   group counts, a decoupled look-back over the chunks for
-//                   the chunk's first group, then every unit's first group
-//                   (off[u]) and, for every 1024th group, the unit that holds
-//                   it (page[p]).  The last chunk checks that the stream
-//                   expands to exactly ceil(n/5) groups and marks it valid.
-//   k_decode_ix     no cross-block wait.  Each stream is decoded in one of
-//                   two tilings, chosen on the device from its density:
-//     payload tiles  (sparse streams, more than 4 groups per payload byte on
-//                    average): a tile is a fixed run of payload bytes whose
-//                    first group is off[] of its first unit; an accumulate
-//                    tile made mostly of escapes visits only its literal
-//                    groups, so the work follows the non-zeros.
-//     gather tiles   (denser streams, and always when several streams are
-//                    summed): a tile is a fixed run of output groups.  Its
-//                    first unit comes from page[]; one warp per unit scans
-//                    the unit's bytes and places its literal groups into
-//                    shared memory (pre-filled with the zero group), then the
-//                    values are written (or read-modify-written once for all
-//                    streams, added in stream order) as coalesced float4s.
-//                    Every tile writes the same amount, however the stream's
-//                    bytes expand.
+// decode; no block of either kernel waits on another.
+//   k_decode_index  one block per 32-unit chunk of 512-byte payload units:
+//                   each unit's first group relative to its chunk (loc[u])
+//                   and the chunk's group count; the last block of a stream
+//                   to finish (an atomic counter) scans the chunk counts into
+//                   each chunk's first group (cpre[c]), checks that the stream
+//                   expands to exactly ceil(n/5) groups, marks it valid, and,
+//                   for sums of several streams, records for every 1024th
+//                   group the chunk that holds it (page[p]).
+//   k_decode_units  one stream: one warp per 512-byte unit, first group
+//                   cpre[u / 32] + loc[u]; the unit's groups are expanded in
+//                   the warp's shared memory and written (or added) as
+//                   coalesced float4s, each from a table of the 81 sign
+//                   patterns of four digits times the scale.
+//   k_decode_ix     2..8 streams: output tiles of a fixed number of groups;
+//                   per stream, the tile's first unit from page[] and loc[],
+//                   one warp per unit places the literal groups in shared
+//                   memory, then each float4 of acc is read once, the
+//                   streams' non-zero values added in stream order, and
+//                   written once.
 // The quartic bytes live only in shared memory.  Every write is clamped to
 // the ceil(n/5) groups of the tensor; a stream that does not expand to
 // exactly that many groups is reported as corrupt and left out.
@@ -52,9 +49,9 @@ namespace tlc {
 
 TLC_DEFINE_DEBUG_READER(debug_fault_decode)
 
-// Payload bytes per thread (1, 2 or a multiple of 4): small tiles balance the dense
-// write mode best; the accumulate mode touches little memory per tile and
-// prefers fewer, larger tiles.
+// Payload bytes per thread (1, 2 or a multiple of 4) of the small-stream
+// tiles: small tiles balance the dense write mode best; the accumulate mode
+// touches little memory per tile and prefers fewer, larger tiles.
 #ifndef TLC_D_BYTES_WRITE
 #define TLC_D_BYTES_WRITE 2
 #endif
@@ -88,6 +85,7 @@ constexpr uint32_t kDecodeDeferMinTiles = TLC_DEFER_DECODE_MIN_TILES;
 constexpr uint32_t kPage = 1024;  // groups per page-table entry
 static_assert(TLC_GT_ACC % (8 * kPage) == 0, "tiles are whole pages");
 static_assert(kDecodeUnit == 4 * kWarp * 4, "a unit is 16 bytes per lane of a warp");
+static_assert(kDecodeChunkUnits == kWarp, "a chunk's units are one per lane of a warp");
 
 size_t decode_smem_bytes(bool accumulate);
 
@@ -110,21 +108,12 @@ __device__ __forceinline__ uint64_t warp_sum_u64(uint64_t v) {
   return v;
 }
 
-// Look-back words per lane per round trip of the index's chunk scan: the
-// index's blocks all start at once, so the first prefix spreads forward by
-// 32 * V chunks per round trip.
-#ifndef TLC_IX_LOOKV
-#define TLC_IX_LOOKV 8
-#endif
-
-// Exclusive prefix (a sum) of item u of a single-pass scan, by one warp.
-// Publishes the item's aggregate first and its inclusive prefix last.  Each
-// round trip reads 32 * V earlier items' words.  Every lane gets the
+// Exclusive prefix (a sum) of tile u of a single-pass scan, by one warp.
+// Publishes the tile's aggregate first and its inclusive prefix last.  Each
+// round trip reads 32 * kLookV earlier tiles' words.  Every lane gets the
 // result.
-template <int V = kLookV>
 __device__ uint64_t lookback_sum(uint64_t *status, uint32_t u, uint64_t E, uint32_t max_polls,
                                  bool &timed_out) {
-  constexpr int kLookV = V;
   const int lane = threadIdx.x & 31;
   if (u == 0) {
     if (lane == 0) st_relaxed_u64(status, kFlagPrefix | E);
@@ -173,17 +162,18 @@ __device__ __forceinline__ float dequant(uint32_t dig, float scale) {
 
 __device__ __forceinline__ uint32_t expansion(uint32_t b) { return b >= 243u ? b - 241u : 1u; }
 
-// One stream's decode job, as the payload-tile function sees it.
+// One stream's decode job.
 struct DecodeJob {
   const uint8_t *payload;  // stream bytes after the 4-byte header
   uint64_t m;              // payload length
   uint64_t n, groups;
   float scale;
   float *y;                // output (kWrite) or accumulation buffer
-  uint64_t *status;        // look-back path: this stream's tile status words
-  uint32_t n_tiles;        // tiles actually present: ceil(m / tile)
+  uint64_t *status;        // small streams: this stream's tile status words
+  uint32_t n_tiles;        // tiles (or units) actually present
   bool vec;                // y is 16-byte aligned
-  const uint32_t *off;     // indexed path: first group of every 512-byte unit
+  const uint32_t *loc;     // indexed streams: units' first groups within their chunk
+  const uint32_t *cpre;    // and chunks' first groups
 };
 
 struct DecodeSmem {
@@ -194,6 +184,16 @@ struct DecodeSmem {
 
 __device__ __forceinline__ void fill_lut(uint16_t *lut) {
   for (int v = threadIdx.x; v < 256; v += blockDim.x) lut[v] = v < 243 ? digits_of(v) : 0;
+}
+
+// For every 8-bit word of four digits (2 bits each, first value lowest), the
+// four quantized values q in {-1, 0, +1} as floats; a value is q * scale,
+// which is exact (and +0.0 for q = 0).  Digit 3 never occurs.
+__device__ __forceinline__ void fill_patterns(float4 *pat) {
+  for (int v = threadIdx.x; v < 256; v += blockDim.x) {
+    auto q = [](uint32_t d) { return d == 0u ? -1.0f : (d == 2u ? 1.0f : 0.0f); };
+    pat[v] = make_float4(q(v & 3u), q((v >> 2) & 3u), q((v >> 4) & 3u), q((v >> 6) & 3u));
+  }
 }
 
 // Validate a stream (length and header) and return its payload length and
@@ -305,9 +305,10 @@ __device__ __forceinline__ void emit_zeros(uint64_t e_begin, uint64_t e_end, flo
 }
 
 // One payload tile of one stream; the whole block calls it and it ends
-// synchronised.  kIndexed: the tile's first group index is off[] of its first
-// unit (written by k_decode_index) instead of a look-back.
-template <int kMode, bool kIndexed>
+// synchronised.  The tile's first group index comes from a decoupled
+// look-back over the tiles before it (small streams) or, kIndexed, from the
+// index (cpre and loc of its first unit; the index has checked the total).
+template <int kMode, bool kIndexed = false>
 __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, DecodeSmem &sm,
                                             uint8_t *grp_s, int32_t *dev_status,
                                             uint32_t max_polls) {
@@ -361,10 +362,13 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
   const bool expand = any_lit && (kMode == kWrite || E <= 4u * (uint32_t)kDTile);
 
   // ---- the tile's first group index ---------------------------------------
-  // Indexed: one load, while every thread pre-fills the zero groups.
+  // Indexed: one lookup while every thread pre-fills the zero groups.
   // Look-back: warp 0 looks back while the other warps pre-fill.
   if (kIndexed) {
-    if (threadIdx.x == 0) sm.o = __ldg(j.off + (uint64_t)u * (kDTile / kDecodeUnit));
+    constexpr uint32_t kTileUnits = kDTile / kDecodeUnit;
+    if (threadIdx.x == 0)
+      sm.o = (uint64_t)__ldg(j.cpre + (u * kTileUnits) / kDecodeChunkUnits) +
+             __ldg(j.loc + u * kTileUnits);
     if (expand) {
       const uint32_t words = (E + 15) / 16;
       for (uint32_t w = threadIdx.x; w < words; w += kDThreads)
@@ -385,7 +389,6 @@ __device__ __forceinline__ void decode_tile(const DecodeJob &j, uint32_t u, Deco
   __syncthreads();
   const uint64_t O = sm.o;
   if (!kIndexed && threadIdx.x == 0) {
-    // (the index already checked the indexed path's total)
     const bool last = (u == j.n_tiles - 1);
     if (O + E > j.groups || (last && O + E != j.groups)) report(dev_status, TLC_ERR_CORRUPT);
   }
@@ -484,14 +487,66 @@ k_decode(const DecodeArgs a) {
   job.status = a.status;
   job.n_tiles = (uint32_t)((job.m + kDTile - 1) / kDTile);
   job.vec = kVec;
-  job.off = nullptr;
   for (;;) {
     if (threadIdx.x == 0) tile_s = atomicAdd(a.ticket, 1u);
     __syncthreads();
     const uint32_t u = tile_s;
     if (u >= job.n_tiles) break;
-    decode_tile<kMode, false>(job, u, sm, grp_s, a.dev_status, a.max_polls);
+    decode_tile<kMode>(job, u, sm, grp_s, a.dev_status, a.max_polls);
   }
+}
+
+// Values [e_begin, e_end) of the groups whose digit words (lut[] of their
+// quartic bytes) sit in wd (wd[0] is group g_first), by one warp: each
+// aligned float4 is the sign pattern of its four digits times the scale
+// (dense output) or added to acc where a digit is not zero (accumulate);
+// single values at the ends, and everywhere when y is not 16-byte aligned.
+// Values 4v..4v+3 lie in group g = 4v/5 (digits d0..) and, when d0 >= 2,
+// spill into group g+1; both groups' digit words are joined so one shift
+// lines the four digits up.
+template <int kMode>
+__device__ __forceinline__ void warp_emit(const uint16_t *wd, uint64_t g_first, uint64_t e_begin,
+                                          uint64_t e_end, float *y, bool vec, float scale,
+                                          const float4 *pat, int lane) {
+  if (e_end <= e_begin) return;
+  const uint32_t gf = (uint32_t)g_first;
+  // n < 2^32, so value and float4 indices fit 32 bits
+  auto put = [&](uint32_t e) {
+    const uint32_t g = e / 5u;
+    const uint32_t dig = (wd[g - gf] >> (2 * (e - 5u * g))) & 3u;
+    if (kMode == kWrite)
+      y[e] = dequant(dig, scale);
+    else if (dig != 1u)
+      y[e] = __fadd_rn(y[e], dequant(dig, scale));
+  };
+  const uint32_t v0 = (uint32_t)((e_begin + 3) / 4), v1 = (uint32_t)(e_end / 4);
+  if (!vec || v1 <= v0) {
+    for (uint32_t e = (uint32_t)e_begin + lane; e < (uint32_t)e_end; e += kWarp) put(e);
+    return;
+  }
+  float4 *y4 = reinterpret_cast<float4 *>(y);
+  for (uint32_t v = v0 + lane; v < v1; v += kWarp) {
+    const uint32_t e0 = v << 2;
+    const uint32_t g = e0 / 5u;
+    const uint32_t d0 = e0 - 5u * g;
+    const uint32_t li = g - gf;
+    const uint32_t p8 = (((uint32_t)wd[li] | ((uint32_t)wd[li + 1] << 10)) >> (2u * d0)) & 0xffu;
+    const float4 p = pat[p8];
+    if (kMode == kWrite) {
+      y4[v] = make_float4(__fmul_rn(p.x, scale), __fmul_rn(p.y, scale), __fmul_rn(p.z, scale),
+                          __fmul_rn(p.w, scale));
+    } else if (p8 != 0x55u) {  // some of the four digits is not zero
+      float4 o = y4[v];
+      if ((p8 & 3u) != 1u) o.x = __fadd_rn(o.x, __fmul_rn(p.x, scale));
+      if (((p8 >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, __fmul_rn(p.y, scale));
+      if (((p8 >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, __fmul_rn(p.z, scale));
+      if (((p8 >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, __fmul_rn(p.w, scale));
+      y4[v] = o;
+    }
+  }
+  // the partial float4s at both ends, one value per lane
+  const uint32_t h = 4 * v0 - (uint32_t)e_begin, t = (uint32_t)e_end - 4 * v1;  // each < 4
+  if ((uint32_t)lane < h + t) put((uint32_t)lane < h ? (uint32_t)e_begin + lane : 4 * v1 + (lane - h));
 }
 
 // ===================================================================== index
@@ -500,82 +555,152 @@ struct IndexOut {
   const uint8_t *payload;
   uint64_t m;          // payload length (valid header)
   uint64_t groups;
-  uint64_t *status;    // look-back words, one per 32-unit chunk (zero at launch)
-  uint32_t *off;       // first group of every unit, plus the total after the last
-  uint32_t *page;      // unit holding group p * kPage, for every page p
+  uint32_t *loc;       // per unit: its first group, counted from its chunk's first
+  uint32_t *cpre;      // per chunk: its group count, then (scanned by the stream's last
+                       // chunk to finish) its first group; cpre[n_chunks]: the total
+  uint32_t *page;      // or nullptr: per page, the chunk holding group p * kPage
+  uint32_t *done;      // the stream's finished chunks (zero at launch)
   uint32_t *ok;        // set to 1 when the stream expands to exactly `groups`
 };
 
-// Chunk c (32 units of 512 payload bytes) of one stream.  Whole block; ends
-// synchronised.  ucnt: 32 words of shared memory.
+struct IndexSmem {
+  uint32_t ucnt[kDecodeChunkUnits];
+  uint64_t wsum[kDWarps + 1];
+  uint32_t last;
+};
+
+__device__ __forceinline__ uint32_t sat32(uint64_t v) { return (uint32_t)umin64(v, 0xffffffffull); }
+
+// The stream's chunk counts, scanned by one block into each chunk's first
+// group, the total checked against the tensor's groups, and the page table.
+// In passes of kScanPer chunks per thread: each thread loads its contiguous
+// share into registers (all loads issued first), then a block scan of the
+// shares (64-bit: a corrupt stream's counts may add up past 2^32).
+constexpr int kScanPer = 8;
+__device__ void scan_chunks(const IndexOut &s, uint32_t n_chunks, IndexSmem &sm,
+                            int32_t *dev_status) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint64_t carry = 0;
+  for (uint32_t base = 0; base < n_chunks; base += kDThreads * kScanPer) {
+    const uint32_t c0 = base + threadIdx.x * kScanPer;
+    uint32_t v[kScanPer];
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) v[i] = c0 + i < n_chunks ? __ldcg(s.cpre + c0 + i) : 0u;
+    uint64_t sum = 0;
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) sum += v[i];
+    uint64_t inc = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint64_t t = __shfl_up_sync(0xffffffffu, inc, d);
+      if (lane >= d) inc += t;
+    }
+    if (lane == 31) sm.wsum[warp] = inc;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint64_t run = 0;
+      for (int w = 0; w < kDWarps; ++w) {
+        const uint64_t t = sm.wsum[w];
+        sm.wsum[w] = run;
+        run += t;
+      }
+      sm.wsum[kDWarps] = run;
+    }
+    __syncthreads();
+    uint64_t run = carry + sm.wsum[warp] + inc - sum;
+    carry += sm.wsum[kDWarps];
+#pragma unroll
+    for (int i = 0; i < kScanPer; ++i) {
+      const uint32_t c = c0 + i;
+      if (c < n_chunks) {
+        s.cpre[c] = sat32(run);
+        if (s.page) {
+          const uint64_t pend = umin64(run + v[i], s.groups);
+          for (uint64_t p = (run + kPage - 1) / kPage; p * kPage < pend; ++p)
+            if (TLC_CHECK(p < (s.groups + kPage - 1) / kPage)) s.page[p] = c;
+        }
+        run += v[i];
+      }
+    }
+    __syncthreads();  // sm.wsum is rewritten by the next pass
+  }
+  if (threadIdx.x == 0) {
+    s.cpre[n_chunks] = sat32(carry);
+    if (carry == s.groups) *s.ok = 1u;
+    else report(dev_status, TLC_ERR_CORRUPT);
+  }
+}
+
+// Atomic add with acquire-release ordering at GPU scope: this thread's
+// earlier writes are visible to whichever thread's add comes later, and
+// that thread sees them.
+__device__ __forceinline__ uint32_t atomic_add_acq_rel(uint32_t *p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
+               : "memory");
+  return old;
+}
+
+// Chunk c (32 units of 512 payload bytes) of one stream of n_chunks: the
+// units' group counts (one warp per 4 units, one 32-bit word per lane per
+// quarter unit, all loads first), loc[] and the chunk's count; the stream's
+// last chunk to finish then scans the counts.  Whole block; ends
+// synchronised.
 constexpr int kUnitsPerWarp = kDecodeChunkUnits / kDWarps;
-__device__ __forceinline__ void index_chunk(const IndexOut &s, uint32_t c, uint32_t *ucnt,
-                                            int32_t *dev_status, uint32_t max_polls) {
+__device__ __forceinline__ void index_chunk(const IndexOut &s, uint32_t c, uint32_t n_chunks,
+                                            IndexSmem &sm, int32_t *dev_status) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint64_t n_units = (s.m + kDecodeUnit - 1) / kDecodeUnit;
-  const bool al4 = (reinterpret_cast<uintptr_t>(s.payload) & 3) == 0;
-  // the warp's units: each lane one 32-bit word per quarter unit, words
-  // interleaved across lanes so every load is coalesced; all loads first
+  const uint64_t u0 = (uint64_t)c * kDecodeChunkUnits + warp * kUnitsPerWarp;
   constexpr int kW = kUnitsPerWarp * (kDecodeUnit / (4 * kWarp));
-  uint32_t w[kW];
-  int nb[kW];
+  if ((reinterpret_cast<uintptr_t>(s.payload) & 3) == 0 && (u0 + kUnitsPerWarp) * kDecodeUnit <= s.m) {
+    // the warp's units lie inside the payload: one 32-bit word per lane per
+    // quarter unit, words interleaved across lanes so every load is
+    // coalesced, all loads issued first
+    uint32_t w[kW];
 #pragma unroll
-  for (int k = 0; k < kW; ++k) {
-    const uint64_t unit = (uint64_t)c * kDecodeChunkUnits + warp * kUnitsPerWarp + k / 4;
-    const uint64_t p = unit * kDecodeUnit + 4 * (uint64_t)(lane + kWarp * (k % 4));
-    w[k] = 0;
-    nb[k] = 0;
-    if (al4 && p + 4 <= s.m) {
-      w[k] = __ldg(reinterpret_cast<const uint32_t *>(s.payload + p));
-      nb[k] = 4;
-    } else {
-      for (int q = 0; q < 4; ++q)
-        if (p + q < s.m) {
-          w[k] |= (uint32_t)__ldg(s.payload + p + q) << (8 * q);
-          nb[k] = q + 1;
-        }
+    for (int k = 0; k < kW; ++k)
+      w[k] = __ldg(reinterpret_cast<const uint32_t *>(
+          s.payload + (u0 + k / 4) * kDecodeUnit + 4 * (uint64_t)(lane + kWarp * (k % 4))));
+#pragma unroll
+    for (int i = 0; i < kUnitsPerWarp; ++i) {
+      uint32_t e = 0;
+#pragma unroll
+      for (int k = 4 * i; k < 4 * i + 4; ++k)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) e += expansion((w[k] >> (8 * q)) & 0xffu);
+      e = __reduce_add_sync(0xffffffffu, e);
+      if (lane == 0) sm.ucnt[warp * kUnitsPerWarp + i] = e;
     }
-  }
-#pragma unroll
-  for (int i = 0; i < kUnitsPerWarp; ++i) {
-    uint32_t e = 0;
-#pragma unroll
-    for (int k = 4 * i; k < 4 * i + 4; ++k)
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        if (q < nb[k]) e += expansion((w[k] >> (8 * q)) & 0xffu);
-    e = __reduce_add_sync(0xffffffffu, e);
-    if (lane == 0) ucnt[warp * kUnitsPerWarp + i] = e;
+  } else {
+    // the stream's last units, or an unaligned payload: byte loads
+    for (int i = 0; i < kUnitsPerWarp; ++i) {
+      uint32_t e = 0;
+      const uint64_t b0 = (u0 + i) * kDecodeUnit;
+      for (uint64_t p = b0 + lane; p < b0 + kDecodeUnit && p < s.m; p += kWarp)
+        e += expansion(__ldg(s.payload + p));
+      e = __reduce_add_sync(0xffffffffu, e);
+      if (lane == 0) sm.ucnt[warp * kUnitsPerWarp + i] = e;
+    }
   }
   __syncthreads();
   if (warp == 0) {
-    const uint32_t v = ucnt[lane];
+    const uint32_t v = sm.ucnt[lane];
     uint32_t inc = v;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
       const uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
       if (lane >= d) inc += t;
     }
-    const uint32_t E = __shfl_sync(0xffffffffu, inc, 31);
-    bool timed_out = false;
-    const uint64_t P = lookback_sum<TLC_IX_LOOKV>(s.status, c, E, max_polls, timed_out);
-    timed_out = __any_sync(0xffffffffu, timed_out);
-    if (timed_out && lane == 0) report(dev_status, TLC_ERR_TIMEOUT);
     const uint64_t u = (uint64_t)c * kDecodeChunkUnits + lane;
-    if (u < n_units) {
-      const uint64_t o = P + (inc - v);
-      s.off[u] = (uint32_t)umin64(o, 0xffffffffull);
-      // the pages whose first group lies in this unit
-      const uint64_t pend = umin64(o + v, s.groups);
-      for (uint64_t p = (o + kPage - 1) / kPage; p * kPage < pend; ++p)
-        if (TLC_CHECK(p < (s.groups + kPage - 1) / kPage)) s.page[p] = (uint32_t)u;
-      if (u == n_units - 1) {
-        s.off[u + 1] = (uint32_t)umin64(o + v, 0xffffffffull);
-        if (o + v == s.groups && !timed_out) *s.ok = 1u;
-        else report(dev_status, TLC_ERR_CORRUPT);
-      }
+    if (u < n_units) s.loc[u] = inc - v;
+    if (lane == 31) {
+      s.cpre[c] = inc;  // the chunk's count (at most 32 * 512 * 14), released by the add
+      sm.last = atomic_add_acq_rel(s.done, 1u) == n_chunks - 1 ? 1u : 0u;
     }
   }
+  __syncthreads();
+  if (sm.last) scan_chunks(s, n_chunks, sm, dev_status);
   __syncthreads();
 }
 
@@ -584,30 +709,33 @@ struct IxStream {
   const uint8_t *in;
   const uint64_t *len_dev;
   uint64_t cap;
-  uint64_t *status;
-  uint32_t *off;
-  uint32_t *page;
+  uint32_t *loc;
+  uint32_t *cpre;
+  uint32_t *page;      // nullptr for a single stream
 };
 struct IxArgs {
   IxStream s[kIndexPass];
   int k;
   uint64_t n, groups;
-  uint32_t *ticket;    // index chunks (zero at launch)
   uint32_t *ticket2;   // decode tiles (cleared by k_decode_index)
   uint32_t *ok;        // per stream (zero at launch)
+  uint32_t *done;      // per stream (zero at launch)
   float *y;
   bool vec;
   int32_t *dev_status;
-  uint32_t max_polls;
 };
 
+__device__ __forceinline__ uint32_t chunks_of(uint64_t m) {
+  return (uint32_t)((m + (uint64_t)kDecodeUnit * kDecodeChunkUnits - 1) /
+                    ((uint64_t)kDecodeUnit * kDecodeChunkUnits));
+}
+
 // Index of every stream: the chunks that exist (from each stream's length),
-// numbered stream by stream, taken in ticket order.
-__global__ void __launch_bounds__(kDThreads) k_decode_index(const IxArgs a) {
+// numbered stream by stream; block b takes chunks b, b + grid, ...
+__global__ void __launch_bounds__(kDThreads, 6) k_decode_index(const IxArgs a) {
   __shared__ uint64_t m_s[kIndexPass];
   __shared__ uint32_t pre_s[kIndexPass + 1];
-  __shared__ uint32_t ucnt[kDecodeChunkUnits];
-  __shared__ uint32_t tile_s;
+  __shared__ IndexSmem sm;
   if (threadIdx.x < (unsigned)a.k) {
     const IxStream &S = a.s[threadIdx.x];
     uint64_t m = 0;
@@ -620,44 +748,46 @@ __global__ void __launch_bounds__(kDThreads) k_decode_index(const IxArgs a) {
   __syncthreads();
   if (threadIdx.x == 0) {
     pre_s[0] = 0;
-    for (int s = 0; s < a.k; ++s)
-      pre_s[s + 1] = pre_s[s] +
-          (uint32_t)((m_s[s] + (uint64_t)kDecodeUnit * kDecodeChunkUnits - 1) /
-                     ((uint64_t)kDecodeUnit * kDecodeChunkUnits));
+    for (int s = 0; s < a.k; ++s) pre_s[s + 1] = pre_s[s] + chunks_of(m_s[s]);
   }
   __syncthreads();
   const uint32_t total = pre_s[a.k];
-  for (;;) {
-    if (threadIdx.x == 0) tile_s = atomicAdd(a.ticket, 1u);
-    __syncthreads();
-    const uint32_t t = tile_s;
-    if (t >= total) break;
+  for (uint32_t t = blockIdx.x; t < total; t += gridDim.x) {
     int s = 0;
     while (s + 1 < a.k && pre_s[s + 1] <= t) ++s;
     const IxStream &S = a.s[s];
-    const IndexOut io = {S.in + 4, m_s[s], a.groups, S.status, S.off, S.page, a.ok + s};
-    index_chunk(io, t - pre_s[s], ucnt, a.dev_status, a.max_polls);
+    const IndexOut io = {S.in + 4, m_s[s], a.groups, S.loc, S.cpre, S.page, a.done + s,
+                         a.ok + s};
+    index_chunk(io, t - pre_s[s], pre_s[s + 1] - pre_s[s], sm, a.dev_status);
   }
 }
 
 // ============================================================= warp units
 // One 512-byte payload unit of an indexed stream, by one warp.  The unit's
-// first group is off[u]; its groups are expanded into the warp's own shared
-// memory (up to kWarpGroups) and written (or added) as coalesced float4s,
-// the float4s that straddle the next unit as single values.  A unit without
-// non-zero literals is plain zeros (dense output) or nothing (accumulate);
-// a unit that expands past kWarpGroups, or (accumulate) whose literals are
-// few, writes its zeros and then visits only its literal groups.  No warp
-// waits on another.
+// first group is cpre[u / 32] + loc[u].  Its groups are decoded in windows
+// of kWarpGroups: the window is pre-filled with the zero group's digit word,
+// the unit's literal groups in the window are placed as their digit words
+// (lut[] of the byte) in the warp's own shared memory, and warp_emit writes
+// (or adds) the window's values; the float4s that straddle a window's or the
+// unit's end become single values.  A unit without non-zero literals is
+// plain zeros (dense output) or nothing (accumulate); an accumulate unit
+// whose literals are few visits only its literal groups.  No warp waits on
+// another.
 #ifndef TLC_WARP_GROUPS
-#define TLC_WARP_GROUPS 2048
+#define TLC_WARP_GROUPS 1024
 #endif
 constexpr uint32_t kWarpGroups = TLC_WARP_GROUPS;
-static_assert(kWarpGroups % 16 == 0, "whole 16-byte words");
+static_assert(kWarpGroups % 8 == 0, "whole 16-byte words of digit words");
+constexpr uint16_t kZeroDigits = 0x155;  // digit word of the zero group 121 (five 1s)
+
+__device__ __forceinline__ uint64_t unit_first_group(const uint32_t *cpre, const uint32_t *loc,
+                                                     uint32_t u) {
+  return (uint64_t)__ldg(cpre + (u / kDecodeChunkUnits)) + __ldg(loc + u);
+}
 
 template <int kMode>
 __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, const uint16_t *lut,
-                                            uint8_t *ws) {
+                                            const float4 *pat, uint16_t *wd) {
   const int lane = threadIdx.x & 31;
   const uint64_t base = (uint64_t)u * kDecodeUnit + 16ull * lane;
   uint32_t w[4] = {0u, 0u, 0u, 0u};
@@ -695,59 +825,25 @@ __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, cons
   const uint32_t E = __shfl_sync(0xffffffffu, inc, 31);
   const uint32_t L = __reduce_add_sync(0xffffffffu, lits);
   const uint32_t excl = inc - e;
-  const uint64_t O = __ldg(j.off + u);
-  const uint64_t Ec = O >= j.groups ? 0 : umin64(E, j.groups - O);
-  const uint64_t e_begin = 5 * O, e_end = umin64(5 * (O + Ec), j.n);
+  const uint64_t O = unit_first_group(j.cpre, j.loc, u);
+  const uint32_t Ec = O >= j.groups ? 0u : (uint32_t)umin64(E, j.groups - O);
   if (L == 0) {
-    if (kMode == kWrite) emit_zeros(e_begin, e_end, j.y, j.vec, lane, kWarp);
+    if (kMode == kWrite) emit_zeros(5 * O, umin64(5 * (O + Ec), j.n), j.y, j.vec, lane, kWarp);
     return;
   }
-  if (E <= kWarpGroups && (kMode == kWrite || 16 * L >= E)) {
-    for (uint32_t q = lane; q < (E + 15) / 16; q += kWarp)
-      reinterpret_cast<uint4 *>(ws)[q] =
-          make_uint4(0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u);
-    __syncwarp();
-    uint32_t pos = excl;
+  if (kMode == kAccumulate && 16 * L < E) {
+    // long zero runs around a few literals: visit the literal groups only
+    // (each group's values loaded before any is added)
+    uint64_t g = O + excl;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       if (k < nb) {
         const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
         if (b >= 243u) {
-          pos += b - 241u;
+          g += b - 241u;
         } else {
-          if (TLC_CHECK(pos < kWarpGroups)) ws[pos] = (uint8_t)b;
-          ++pos;
-        }
-      }
-    }
-    __syncwarp();
-    emit_values<kMode>(ws, O, e_begin, e_end, j.y, j.vec, j.scale, lut, lane, kWarp);
-    __syncwarp();
-    return;
-  }
-  // long zero runs around a few literals: zeros first (dense output), then
-  // the literal groups (each group's values loaded before any is added)
-  if (kMode == kWrite) {
-    emit_zeros(e_begin, e_end, j.y, j.vec, lane, kWarp);
-    __syncwarp();
-  }
-  uint64_t g = O + excl;
-#pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    if (k < nb) {
-      const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
-      if (b >= 243u) {
-        g += b - 241u;
-      } else {
-        if (b != 121u && g < j.groups) {
-          const uint32_t dg = lut[b];
-          if (kMode == kWrite) {
-#pragma unroll
-            for (int d = 0; d < 5; ++d) {
-              const uint64_t ei = 5 * g + d;
-              if (ei < j.n) j.y[ei] = dequant((dg >> (2 * d)) & 3u, j.scale);
-            }
-          } else {
+          if (b != 121u && g < j.groups) {
+            const uint32_t dg = lut[b];
             float v[5];
 #pragma unroll
             for (int d = 0; d < 5; ++d) {
@@ -761,28 +857,70 @@ __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, cons
               if (dig != 1u && ei < j.n) j.y[ei] = __fadd_rn(v[d], dequant(dig, j.scale));
             }
           }
+          ++g;
         }
-        ++g;
       }
     }
+    return;
   }
-  __syncwarp();
+  for (uint32_t w0 = 0; w0 < Ec; w0 += kWarpGroups) {
+    const uint32_t wn = min(kWarpGroups, Ec - w0);
+    for (uint32_t q = lane; q < (wn + 7) / 8; q += kWarp)
+      reinterpret_cast<uint4 *>(wd)[q] =
+          make_uint4(0x01550155u, 0x01550155u, 0x01550155u, 0x01550155u);
+    __syncwarp();
+    uint32_t pos = excl;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if (k < nb) {
+        const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
+        if (b >= 243u) {
+          pos += b - 241u;
+        } else {
+          if (pos - w0 < wn) wd[pos - w0] = lut[b];  // unsigned: pos in [w0, w0 + wn)
+          ++pos;
+        }
+      }
+    }
+    __syncwarp();
+    const uint64_t gb = O + w0;
+    warp_emit<kMode>(wd, gb, 5 * gb, umin64(5 * (gb + wn), j.n), j.y, j.vec, j.scale, pat, lane);
+    __syncwarp();
+  }
 }
+
+// Streams that expand to more than this many groups per payload byte on
+// average are written by block-wide payload tiles instead of warp units.
+#ifndef TLC_SPARSE_EXPANSION
+#define TLC_SPARSE_EXPANSION 4
+#endif
 
 // Shared memory of a block of warp-unit decoders.
 struct UnitSmem {
-  uint16_t lut[256];
-  __align__(16) uint8_t ws[kDWarps][kWarpGroups + 16];
+  DecodeSmem d;   // digit table, block scan, a tile's first group
+  float4 pat[256];
+  __align__(16) uint16_t wd[kDWarps][kWarpGroups + 8];
 };
+static_assert(sizeof(UnitSmem::wd) >= DecodeShape<kWrite>::kMaxGroups + 16,
+              "a dense-output payload tile's groups fit the warps' windows");
 
-// One indexed stream (dense output, or added into acc): every warp takes
-// units blockIdx.x * warps + warp, then every (grid's warps)-th unit.
+__device__ __forceinline__ void fill_unit_tables(UnitSmem &sm) {
+  fill_lut(sm.d.lut);
+  fill_patterns(sm.pat);
+}
+
+// One indexed stream (dense output, or added into acc): warp w of block b
+// takes units b * warps + w, then every (grid's warps)-th unit.  A sparse
+// stream's dense output is written by whole blocks instead, one 512-byte
+// payload tile (unit) per block in ticket order: its all-zero tiles are each
+// one long run of zero stores, which a block writes faster than a warp.
 template <int kMode>
 __global__ void __launch_bounds__(kDThreads, 8) k_decode_units(const IxArgs a) {
   __shared__ UnitSmem sm;
   __shared__ DecodeJob job_s;
   __shared__ int ok_s;
-  fill_lut(sm.lut);
+  __shared__ uint32_t tile_s;
+  fill_unit_tables(sm);
   if (threadIdx.x == 0) {
     const IxStream &S = a.s[0];
     uint64_t m = 0;
@@ -798,23 +936,37 @@ __global__ void __launch_bounds__(kDThreads, 8) k_decode_units(const IxArgs a) {
     j.status = nullptr;
     j.n_tiles = (uint32_t)((m + kDecodeUnit - 1) / kDecodeUnit);
     j.vec = a.vec;
-    j.off = S.off;
+    j.loc = S.loc;
+    j.cpre = S.cpre;
     job_s = j;
   }
   __syncthreads();
   if (!ok_s) return;
-  const DecodeJob j = job_s;
+  if (kMode == kWrite && job_s.groups > (uint64_t)TLC_SPARSE_EXPANSION * job_s.m) {
+    static_assert(DecodeShape<kWrite>::kTile == kDecodeUnit, "dense-output tiles are units");
+    uint8_t *grp = reinterpret_cast<uint8_t *>(&sm.wd[0][0]);
+    for (;;) {
+      if (threadIdx.x == 0) tile_s = atomicAdd(a.ticket2, 1u);
+      __syncthreads();
+      const uint32_t t = tile_s;
+      if (t >= job_s.n_tiles) break;
+      decode_tile<kWrite, true>(job_s, t, sm.d, grp, a.dev_status, 0u);
+    }
+    return;
+  }
+  // the job stays in shared memory: its fields are read where they are used
   const int warp = threadIdx.x >> 5;
   const uint32_t nw = gridDim.x * kDWarps;
-  for (uint32_t u = blockIdx.x * kDWarps + warp; u < j.n_tiles; u += nw)
-    decode_unit<kMode>(j, u, sm.lut, sm.ws[warp]);
+  for (uint32_t u = blockIdx.x * kDWarps + warp; u < job_s.n_tiles; u += nw)
+    decode_unit<kMode>(job_s, u, sm.d.lut, sm.pat, sm.wd[warp]);
 }
 
 // ==================================================================== gather
 // A stream as the gather tiles read it.
 struct GStream {
   const uint8_t *payload;
-  const uint32_t *off;
+  const uint32_t *loc;
+  const uint32_t *cpre;
   const uint32_t *page;
   uint64_t m;
   float scale;
@@ -826,6 +978,19 @@ struct GatherSmem {
   uint32_t uf[kK], nu[kK];  // first unit and unit count of each stream in the tile
   uint32_t lit[kK];         // the stream has a non-zero literal in the tile
 };
+
+// The unit of stream S that holds group g (< the stream's groups), by one
+// warp: the page gives the chunk, the chunk's 32 loc[] entries the unit.
+// Every lane gets the result.
+__device__ __forceinline__ uint32_t unit_of_group(const GStream &S, uint64_t g) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t n_chunks = (S.n_units + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
+  const uint32_t c = (uint32_t)umin64(__ldg(S.page + g / kPage), n_chunks - 1);
+  const uint64_t u = (uint64_t)c * kDecodeChunkUnits + lane;
+  const bool in = u < S.n_units && (uint64_t)__ldg(S.cpre + c) + __ldg(S.loc + u) <= g;
+  const uint32_t mask = __ballot_sync(0xffffffffu, in);
+  return c * kDecodeChunkUnits + (mask ? 31 - __clz(mask) : 0);
+}
 
 // One warp: unit u of stream S.  Each lane takes 16 consecutive payload
 // bytes; a warp scan of their expansion counts gives each lane's first
@@ -862,7 +1027,7 @@ __device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t
     const uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
     if (lane >= d) inc += t;
   }
-  uint64_t g = (uint64_t)__ldg(S.off + u) + (inc - e);
+  uint64_t g = unit_first_group(S.cpre, S.loc, u) + (inc - e);
   const uint64_t ge = g0 + gn;
   bool mine = false;
   if (nb > 0 && g < ge && g + e > g0) {
@@ -885,120 +1050,107 @@ __device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t
   if (__any_sync(0xffffffffu, mine) && lane == 0) *lit = 1u;
 }
 
-// One gather tile: output groups [g0, g0 + gn) of k streams (k <= kK, all
-// valid, in stream order).  Whole block; ends synchronised.  grp holds
-// kK * kGt bytes.
-template <int kMode, int kGt, int kK>
+// One gather tile: output groups [g0, g0 + gn) of k streams (2 <= k <= kK,
+// all valid, in stream order) added into acc.  Whole block; ends
+// synchronised.  grp holds kK * kGt bytes.
+template <int kGt, int kK>
 __device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g0,
                                             uint64_t groups, uint64_t n, float *y, bool vec,
-                                            const uint16_t *lut, uint8_t *grp,
+                                            const uint16_t *lut, const float4 *pat, uint8_t *grp,
                                             GatherSmem<kK> &sm) {
-  static_assert(kGt % kPage == 0 && kGt % 16 == 0, "tile shape");
+  static_assert(kGt % kPage == 0 && kGt % 16 == 0 && kK <= kDWarps, "tile shape");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t gn = (uint32_t)umin64(kGt, groups - g0);
-  // pre-fill with the zero group; each stream's unit range from the pages
+  // pre-fill with the zero group; warp s finds stream s's unit range
   for (int s = 0; s < k; ++s)
     for (uint32_t w = threadIdx.x; w < (gn + 15) / 16; w += kDThreads)
       reinterpret_cast<uint4 *>(grp + s * kGt)[w] =
           make_uint4(0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u);
-  if (warp == 0 && lane < k) {
-    const GStream &S = gs[lane];
-    const uint32_t last = S.n_units - 1;
-    uint32_t uf = umin64(__ldg(S.page + g0 / kPage), last);
-    uint32_t ul = g0 + gn < groups ? (uint32_t)umin64(__ldg(S.page + (g0 + gn) / kPage), last)
-                                   : last;
+  if (warp < k) {
+    const GStream &S = gs[warp];
+    const uint32_t uf = unit_of_group(S, g0);
+    uint32_t ul = g0 + gn < groups ? unit_of_group(S, g0 + gn) : S.n_units - 1;
     if (ul < uf) ul = uf;
-    sm.uf[lane] = uf;
-    sm.nu[lane] = ul - uf + 1;
-    sm.lit[lane] = 0u;
+    if (lane == 0) {
+      sm.uf[warp] = uf;
+      sm.nu[warp] = ul - uf + 1;
+      sm.lit[warp] = 0u;
+    }
   }
   __syncthreads();
   for (int s = 0; s < k; ++s)
     for (uint32_t i = warp; i < sm.nu[s]; i += kDWarps)
       walk_unit(gs[s], sm.uf[s] + i, g0, gn, grp + s * kGt, &sm.lit[s]);
   __syncthreads();
-  const uint64_t e_begin = 5 * g0, e_end = umin64(5 * (g0 + gn), n);
-  if (kMode == kWrite) {
-    if (sm.lit[0])
-      emit_values<kWrite>(grp, g0, e_begin, e_end, y, vec, gs[0].scale, lut, threadIdx.x,
-                          kDThreads);
-    else
-      emit_zeros(e_begin, e_end, y, vec, threadIdx.x, kDThreads);
-  } else if (kK == 1) {
-    if (sm.lit[0])
-      emit_values<kAccumulate>(grp, g0, e_begin, e_end, y, vec, gs[0].scale, lut, threadIdx.x,
-                               kDThreads);
-  } else {
-    // several streams: one read-modify-write of each float4 of acc, the
-    // streams' non-zero values added in stream order
-    uint32_t act = 0;  // bit s: stream s has a non-zero value in the tile
+  // one read-modify-write of each float4 of acc: the streams' non-zero
+  // values added in stream order
+  uint32_t act = 0;  // bit s: stream s has a non-zero value in the tile
 #pragma unroll
-    for (int s = 0; s < kK; ++s)
-      if (s < k && sm.lit[s]) act |= 1u << s;
-    if (act) {
-      const uint32_t o32 = (uint32_t)g0;
-      const uint64_t v0 = vec ? (e_begin + 3) / 4 : e_end, v1 = vec ? e_end / 4 : e_end;
-      float4 *y4 = reinterpret_cast<float4 *>(y);
-      for (uint64_t v = v0 + threadIdx.x; v < v1; v += kDThreads) {
-        const uint32_t e0 = (uint32_t)(4 * v);
-        const uint32_t g = e0 / 5u;
-        const uint32_t d0 = e0 - 5u * g;
-        const uint32_t li = g - o32;
-        float4 o;
-        bool loaded = false;
+  for (int s = 0; s < kK; ++s)
+    if (s < k && sm.lit[s]) act |= 1u << s;
+  if (act) {
+    const uint64_t e_begin = 5 * g0, e_end = umin64(5 * (g0 + gn), n);
+    const uint32_t o32 = (uint32_t)g0;
+    const uint64_t v0 = vec ? (e_begin + 3) / 4 : e_end, v1 = vec ? e_end / 4 : e_end;
+    float4 *y4 = reinterpret_cast<float4 *>(y);
+    for (uint32_t v = (uint32_t)v0 + threadIdx.x; v < (uint32_t)v1; v += kDThreads) {
+      const uint32_t e0 = v << 2;
+      const uint32_t g = e0 / 5u;
+      const uint32_t d0 = e0 - 5u * g;
+      const uint32_t li = g - o32;
+      float4 o;
+      bool loaded = false;
 #pragma unroll
-        for (int i = 0; i < kK; ++i) {
-          if ((act >> i) & 1u) {
-            const uint8_t *gb = grp + i * kGt;
-            const uint32_t c0 = gb[li];
-            const uint32_t c1 = d0 >= 2u ? (uint32_t)gb[li + 1] : 121u;
-            if (c0 == 121u && c1 == 121u) continue;
-            const uint32_t w = ((uint32_t)lut[c0] | ((uint32_t)lut[c1] << 10)) >> (2u * d0);
-            if ((w & 0xffu) == 0x55u) continue;
-            if (!loaded) {
-              o = y4[v];
-              loaded = true;
-            }
-            const float sc = gs[i].scale;
-            if ((w & 3u) != 1u) o.x = __fadd_rn(o.x, dequant(w & 3u, sc));
-            if (((w >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, dequant((w >> 2) & 3u, sc));
-            if (((w >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, dequant((w >> 4) & 3u, sc));
-            if (((w >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, dequant((w >> 6) & 3u, sc));
+      for (int i = 0; i < kK; ++i) {
+        if ((act >> i) & 1u) {
+          const uint8_t *gb = grp + i * kGt;
+          const uint32_t c0 = gb[li], c1 = gb[li + 1];
+          const uint32_t p8 = (((uint32_t)lut[c0] | ((uint32_t)lut[c1] << 10)) >> (2u * d0)) & 0xffu;
+          if (p8 == 0x55u) continue;
+          if (!loaded) {
+            o = y4[v];
+            loaded = true;
           }
+          const float4 p = pat[p8];
+          const float sc = gs[i].scale;
+          if ((p8 & 3u) != 1u) o.x = __fadd_rn(o.x, __fmul_rn(p.x, sc));
+          if (((p8 >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, __fmul_rn(p.y, sc));
+          if (((p8 >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, __fmul_rn(p.z, sc));
+          if (((p8 >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, __fmul_rn(p.w, sc));
         }
-        if (loaded) y4[v] = o;
       }
-      // single values: the edges of the float4 range, or every value when
-      // acc is not 16-byte aligned
-      auto put = [&](uint64_t e) {
-        const uint32_t e32 = (uint32_t)e;
-        const uint32_t g = e32 / 5u;
-        const uint32_t sh = 2 * (e32 - 5u * g);
-        float v = 0.0f;
-        bool loaded = false;
+      if (loaded) y4[v] = o;
+    }
+    // single values: the edges of the float4 range, or every value when
+    // acc is not 16-byte aligned
+    auto put = [&](uint64_t e) {
+      const uint32_t e32 = (uint32_t)e;
+      const uint32_t g = e32 / 5u;
+      const uint32_t sh = 2 * (e32 - 5u * g);
+      float v = 0.0f;
+      bool loaded = false;
 #pragma unroll
-        for (int i = 0; i < kK; ++i) {
-          if ((act >> i) & 1u) {
-            const uint32_t dig = (lut[grp[i * kGt + (g - o32)]] >> sh) & 3u;
-            if (dig == 1u) continue;
-            if (!loaded) {
-              v = y[e];
-              loaded = true;
-            }
-            v = __fadd_rn(v, dequant(dig, gs[i].scale));
+      for (int i = 0; i < kK; ++i) {
+        if ((act >> i) & 1u) {
+          const uint32_t dig = (lut[grp[i * kGt + (g - o32)]] >> sh) & 3u;
+          if (dig == 1u) continue;
+          if (!loaded) {
+            v = y[e];
+            loaded = true;
           }
+          v = __fadd_rn(v, dequant(dig, gs[i].scale));
         }
-        if (loaded) y[e] = v;
-      };
-      if (!vec || v1 <= v0) {
-        for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) put(e);
-      } else if (threadIdx.x < 4) {
-        const uint64_t e = e_begin + threadIdx.x;
-        if (e < 4 * v0) put(e);
-      } else if (threadIdx.x < 8) {
-        const uint64_t e = 4 * v1 + (threadIdx.x - 4);
-        if (e < e_end) put(e);
       }
+      if (loaded) y[e] = v;
+    };
+    if (!vec || v1 <= v0) {
+      for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) put(e);
+    } else if (threadIdx.x < 4) {
+      const uint64_t e = e_begin + threadIdx.x;
+      if (e < 4 * v0) put(e);
+    } else if (threadIdx.x < 8) {
+      const uint64_t e = 4 * v1 + (threadIdx.x - 4);
+      if (e < e_end) put(e);
     }
   }
   __syncthreads();
@@ -1010,18 +1162,20 @@ constexpr size_t ix_smem_bytes() {
   return (size_t)kK * kGt + 16;
 }
 
-// Add k <= kK indexed streams (in stream order) into acc, by gather tiles.
-// Streams the index did not mark valid are left out.  Tiles in ticket
-// order; no tile waits on another.
+// Add k (2 <= k <= kK) indexed streams, in stream order, into acc by gather
+// tiles.  Streams the index did not mark valid are left out.  Tiles in
+// ticket order; no tile waits on another.
 template <int kGt, int kK>
 __global__ void __launch_bounds__(kDThreads, 6) k_decode_ix(const IxArgs a) {
   extern __shared__ __align__(16) uint8_t dyn_s[];
+  __shared__ float4 pat[256];
   __shared__ uint16_t lut[256];
   __shared__ GatherSmem<kK> gsm;
   __shared__ GStream gs[kK];
   __shared__ int na_s;
   __shared__ uint32_t tile_s;
   fill_lut(lut);
+  fill_patterns(pat);
   if (threadIdx.x == 0) {
     // the valid streams, in stream order
     int na = 0;
@@ -1033,7 +1187,8 @@ __global__ void __launch_bounds__(kDThreads, 6) k_decode_ix(const IxArgs a) {
       if (!read_stream_header(S.in, S.len_dev, S.cap, a.groups, m, scale)) continue;
       GStream g;
       g.payload = S.in + 4;
-      g.off = S.off;
+      g.loc = S.loc;
+      g.cpre = S.cpre;
       g.page = S.page;
       g.m = m;
       g.scale = scale;
@@ -1051,8 +1206,8 @@ __global__ void __launch_bounds__(kDThreads, 6) k_decode_ix(const IxArgs a) {
     __syncthreads();
     const uint32_t t = tile_s;
     if (t >= n_tiles) break;
-    gather_tile<kAccumulate, kGt, kK>(gs, na, (uint64_t)t * kGt, a.groups, a.n, a.y, a.vec, lut,
-                                      dyn_s, gsm);
+    gather_tile<kGt, kK>(gs, na, (uint64_t)t * kGt, a.groups, a.n, a.y, a.vec, lut, pat, dyn_s,
+                         gsm);
   }
 }
 
@@ -1066,12 +1221,12 @@ struct BatchDecodeArgs {
   const uint8_t *arena;
   uint64_t *status;
   uint32_t *ticket;
-  uint32_t *ticket2;            // indexed plans: the decode kernel's ticket
   int32_t *dev_status;
   uint32_t max_polls;
-  uint32_t *off;                // indexed plans: units' first groups,
-  uint32_t *page;               // page tables,
-  uint32_t *ok;                 // per-tensor valid flags
+  uint32_t *loc;                // indexed plans: units' first groups in their chunk,
+  uint32_t *cpre;               // chunks' first groups (d_chunks + 1 per tensor),
+  uint32_t *done;               // per-tensor finished chunks and
+  uint32_t *ok;                 // valid flags (both zero at launch)
   uint32_t n_chunks;            // chunks of all tensors (upper bound)
 };
 
@@ -1173,35 +1328,28 @@ __global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArg
     job.status = a.status + T.d_tile_begin;
     job.n_tiles = (uint32_t)((job.m + kDTile - 1) / kDTile);
     job.vec = T.vec_y != 0;
-    job.off = nullptr;
-    decode_tile<kMode, false>(job, u - P.act_begin, sm, grp_s, a.dev_status, a.max_polls);
+    decode_tile<kMode>(job, u - P.act_begin, sm, grp_s, a.dev_status, a.max_polls);
   }
 }
 
 // Index of a plan's streams: the chunks that exist, numbered tensor by
-// tensor by the prepare kernel, in ticket order.  Block 0 also clears the
-// decode kernel's ticket.
-__global__ void __launch_bounds__(kDThreads) k_decode_batch_index(const BatchDecodeArgs a) {
+// tensor by the prepare kernel; block b takes chunks b, b + grid, ...
+__global__ void __launch_bounds__(kDThreads, 8) k_decode_batch_index(const BatchDecodeArgs a) {
   __shared__ uint32_t begin_s[kSmemSearch];
-  __shared__ uint32_t ucnt[kDecodeChunkUnits];
-  __shared__ uint32_t tile_s;
+  __shared__ IndexSmem sm;
   const bool in_smem = a.count <= kSmemSearch;
   if (in_smem)
     for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads) begin_s[i] = a.prep[i].cact_begin;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket2 = 0;
   __syncthreads();
   const uint32_t total = a.total[1];
-  for (;;) {
-    if (threadIdx.x == 0) tile_s = atomicAdd(a.ticket, 1u);
-    __syncthreads();
-    const uint32_t g = tile_s;
-    if (g >= total) break;
+  for (uint32_t g = blockIdx.x; g < total; g += gridDim.x) {
     const uint32_t id = find_tensor(begin_s, in_smem, a.prep, a.count, g, true);
     const BatchTensor &T = a.tensors[id];
     const BatchPrep &P = a.prep[id];
-    const IndexOut io = {a.arena + T.arena_off + 4, P.m, T.groups, a.status + T.d_chunk_begin,
-                         a.off + T.d_off_begin, a.page + T.d_page_begin, a.ok + id};
-    index_chunk(io, g - P.cact_begin, ucnt, a.dev_status, a.max_polls);
+    const uint32_t n_chunks = chunks_of(P.m);
+    const IndexOut io = {a.arena + T.arena_off + 4, P.m, T.groups, a.loc + T.d_tile_begin,
+                         a.cpre + T.d_chunk_begin + id, nullptr, a.done + id, a.ok + id};
+    index_chunk(io, g - P.cact_begin, n_chunks, sm, a.dev_status);
   }
 }
 
@@ -1212,31 +1360,42 @@ template <int kMode>
 __global__ void __launch_bounds__(kDThreads, 8) k_decode_batch_units(const BatchDecodeArgs a) {
   __shared__ UnitSmem sm;
   __shared__ uint32_t begin_s[kSmemSearch];
-  fill_lut(sm.lut);
+  __shared__ DecodeJob jobs[kDWarps];  // each warp's current tensor
+  fill_unit_tables(sm);
   const bool in_smem = a.count <= kSmemSearch;
   if (in_smem)
     for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads) begin_s[i] = a.prep[i].act_begin;
   __syncthreads();
   const uint32_t total = *a.total;
-  const int warp = threadIdx.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t nw = gridDim.x * kDWarps;
+  DecodeJob &j = jobs[warp];
+  uint32_t cur = 0xffffffffu;
   for (uint32_t gu = blockIdx.x * kDWarps + warp; gu < total; gu += nw) {
     const uint32_t id = find_tensor(begin_s, in_smem, a.prep, a.count, gu, false);
     if (!a.ok[id]) continue;  // uniform in the warp
-    const BatchTensor &T = a.tensors[id];
-    const BatchPrep &P = a.prep[id];
-    DecodeJob j;
-    j.payload = a.arena + T.arena_off + 4;
-    j.m = P.m;
-    j.n = T.n;
-    j.groups = T.groups;
-    j.scale = P.scale;
-    j.y = T.y;
-    j.status = nullptr;
-    j.n_tiles = (uint32_t)((P.m + kDecodeUnit - 1) / kDecodeUnit);
-    j.vec = T.vec_y != 0;
-    j.off = a.off + T.d_off_begin;
-    decode_unit<kMode>(j, gu - P.act_begin, sm.lut, sm.ws[warp]);
+    const uint32_t first = in_smem ? begin_s[id] : a.prep[id].act_begin;
+    if (id != cur) {
+      __syncwarp();
+      if (lane == 0) {
+        const BatchTensor &T = a.tensors[id];
+        const BatchPrep &P = a.prep[id];
+        j.payload = a.arena + T.arena_off + 4;
+        j.m = P.m;
+        j.n = T.n;
+        j.groups = T.groups;
+        j.scale = P.scale;
+        j.y = T.y;
+        j.status = nullptr;
+        j.n_tiles = (uint32_t)((P.m + kDecodeUnit - 1) / kDecodeUnit);
+        j.vec = T.vec_y != 0;
+        j.loc = a.loc + T.d_tile_begin;
+        j.cpre = a.cpre + T.d_chunk_begin + id;
+      }
+      __syncwarp();
+      cur = id;
+    }
+    decode_unit<kMode>(j, gu - first, sm.d.lut, sm.pat, sm.wd[warp]);
   }
 }
 
@@ -1273,16 +1432,20 @@ uint32_t decode_tile_payload_bytes(bool accumulate) {
 
 uint32_t decode_pages(uint64_t groups) { return (uint32_t)((groups + kPage - 1) / kPage); }
 
+static uint32_t persistent_grid(const DeviceInfo &dev, int occ, uint64_t work_blocks) {
+  uint64_t grid = (uint64_t)dev.sm_count * (uint64_t)(occ > 0 ? occ : 1);
+  if (grid > work_blocks) grid = work_blocks;
+  return (uint32_t)(grid < 1 ? 1 : grid);
+}
+
 template <int kMode, bool kVec>
 static cudaError_t launch_one(const DeviceInfo &dev, const DecodeArgs &a, uint32_t tiles,
                               cudaStream_t stream) {
   const size_t smem = decode_smem_bytes(kMode == kAccumulate);
   const int occ = kMode == kWrite ? dev.occ_decode_write : dev.occ_decode_acc;
-  uint32_t grid = (uint32_t)dev.sm_count * (uint32_t)(occ > 0 ? occ : 1);
-  if (grid > tiles) grid = tiles;
   const int kind = kMode == kWrite ? kKindDecodeWrite : kKindDecodeAccumulate;
   timing_begin(kind, stream);
-  k_decode<kMode, kVec><<<grid, kDThreads, smem, stream>>>(a);
+  k_decode<kMode, kVec><<<persistent_grid(dev, occ, tiles), kDThreads, smem, stream>>>(a);
   timing_end(kind, stream);
   return cudaGetLastError();
 }
@@ -1313,28 +1476,26 @@ cudaError_t launch_decode(const DeviceInfo &dev, const uint8_t *in, const uint64
 }
 
 // ---- indexed decode of up to kIndexPass streams --------------------------
-// Scratch: [ticket, ticket2, ok[kIndexPass]] and every stream's chunk status
-// words (zeroed before each launch pair), then each stream's off[] and
-// page[] arrays.
-static size_t ix_head_bytes() { return align_up(8 + 4 * kIndexPass, 64); }
+// Scratch: [ticket2, ok[kIndexPass], done[kIndexPass]] (cleared before each
+// launch pair), then each stream's loc[] (one word per unit of its
+// capacity), cpre[] (one per chunk, plus the total) and, for two streams or
+// more, page[] (one per 1024 groups).
+static size_t ix_head_bytes() { return align_up(4 + 8 * kIndexPass, 256); }
 
 IndexedLayout indexed_layout(const IndexedStream *s, int k, uint64_t n) {
   IndexedLayout L = {};
   const uint64_t groups = (n + 4) / 5;
-  size_t at = ix_head_bytes();
+  L.zero_bytes = ix_head_bytes();
+  size_t at = L.zero_bytes;
   for (int i = 0; i < k; ++i) {
     const uint32_t units = decode_tiles_max(s[i].cap, groups);
-    L.status_off[i] = at;
-    at += 8 * (size_t)((units + kDecodeChunkUnits - 1) / kDecodeChunkUnits);
-  }
-  L.zero_bytes = align_up(at, 256);
-  at = L.zero_bytes;
-  for (int i = 0; i < k; ++i) {
-    const uint32_t units = decode_tiles_max(s[i].cap, groups);
-    L.off_off[i] = at;
-    at = align_up(at + 4 * ((size_t)units + 1), 16);
+    const uint32_t chunks = (units + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
+    L.loc_off[i] = at;
+    at = align_up(at + 4 * (size_t)units, 16);
+    L.cpre_off[i] = at;
+    at = align_up(at + 4 * ((size_t)chunks + 1), 16);
     L.page_off[i] = at;
-    at = align_up(at + 4 * (size_t)decode_pages(groups), 16);
+    if (k > 1) at = align_up(at + 4 * (size_t)decode_pages(groups), 16);
   }
   L.total_bytes = align_up(at, 256);
   return L;
@@ -1362,12 +1523,6 @@ void occupancy_decode_ix(int occ[5]) {
   occ[4] = ix_occupancy<TLC_GT_ACC / 8, 8>();
 }
 
-static uint32_t persistent_grid(const DeviceInfo &dev, int occ, uint64_t work_blocks) {
-  uint64_t grid = (uint64_t)dev.sm_count * (uint64_t)(occ > 0 ? occ : 1);
-  if (grid > work_blocks) grid = work_blocks;
-  return (uint32_t)(grid < 1 ? 1 : grid);
-}
-
 template <int kGt, int kK>
 static cudaError_t launch_ix(const DeviceInfo &dev, const IxArgs &a, int occ_slot,
                              cudaStream_t stream) {
@@ -1383,6 +1538,7 @@ static cudaError_t launch_ix(const DeviceInfo &dev, const IxArgs &a, int occ_slo
 cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s, int k, uint64_t n,
                                   float *y, bool accumulate, int32_t *dev_status,
                                   uint32_t max_polls, void *scratch, cudaStream_t stream) {
+  (void)max_polls;  // nothing in the indexed decode waits on another block
   if (k < 1 || k > kIndexPass || (!accumulate && k != 1)) return cudaErrorInvalidValue;
   const IndexedLayout L = indexed_layout(s, k, n);
   char *base = static_cast<char *>(scratch);
@@ -1392,13 +1548,12 @@ cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s,
   a.k = k;
   a.n = n;
   a.groups = (n + 4) / 5;
-  a.ticket = reinterpret_cast<uint32_t *>(base);
-  a.ticket2 = reinterpret_cast<uint32_t *>(base + 4);
-  a.ok = reinterpret_cast<uint32_t *>(base + 8);
+  a.ticket2 = reinterpret_cast<uint32_t *>(base);
+  a.ok = reinterpret_cast<uint32_t *>(base + 4);
+  a.done = reinterpret_cast<uint32_t *>(base + 4 + 4 * kIndexPass);
   a.y = y;
   a.vec = (reinterpret_cast<uintptr_t>(y) & 15) == 0;
   a.dev_status = dev_status;
-  a.max_polls = max_polls;
   uint64_t chunks = 0, units_max = 0;
   for (int i = 0; i < kIndexPass; ++i) {
     IxStream &S = a.s[i];
@@ -1406,9 +1561,9 @@ cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s,
       S.in = s[i].in;
       S.len_dev = s[i].len_dev;
       S.cap = s[i].cap;
-      S.status = reinterpret_cast<uint64_t *>(base + L.status_off[i]);
-      S.off = reinterpret_cast<uint32_t *>(base + L.off_off[i]);
-      S.page = reinterpret_cast<uint32_t *>(base + L.page_off[i]);
+      S.loc = reinterpret_cast<uint32_t *>(base + L.loc_off[i]);
+      S.cpre = reinterpret_cast<uint32_t *>(base + L.cpre_off[i]);
+      S.page = k > 1 ? reinterpret_cast<uint32_t *>(base + L.page_off[i]) : nullptr;
       const uint32_t units = decode_tiles_max(s[i].cap, a.groups);
       chunks += (units + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
       if (units > units_max) units_max = units;
@@ -1417,7 +1572,7 @@ cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s,
     }
   }
   timing_begin(kKindDecodeCount, stream);
-  k_decode_index<<<persistent_grid(dev, 8, chunks), kDThreads, 0, stream>>>(a);
+  k_decode_index<<<persistent_grid(dev, 6, chunks), kDThreads, 0, stream>>>(a);
   timing_end(kKindDecodeCount, stream);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1486,12 +1641,12 @@ cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
   a.arena = arena;
   a.status = p.d_status;
   a.ticket = p.d_ticket;
-  a.ticket2 = p.d_ticket2;
   a.n_tiles = p.n_d_tiles;   // units (indexed) or an upper bound of the payload tiles
   a.dev_status = dev_status;
   a.max_polls = max_polls;
-  a.off = p.d_off;
-  a.page = p.d_page;
+  a.loc = p.d_loc;
+  a.cpre = p.d_cpre;
+  a.done = p.d_done;
   a.ok = p.d_ok;
   a.n_chunks = p.n_d_chunks;
   return accumulate ? launch_batch_one<kAccumulate>(dev, a, indexed, stream)

@@ -111,8 +111,6 @@ struct BatchTensor {
   uint32_t d_chunk_begin, d_chunks;  // 32-unit chunks of the index (same)
   uint32_t vec_q;        // x and err 16-byte aligned
   uint32_t vec_y;        // y 16-byte aligned
-  uint32_t d_off_begin;  // indexed plans: the tensor's units' first groups (d_tiles + 1)
-  uint32_t d_page_begin; // and its page table (ceil(groups / 1024) entries)
 };
 
 // Per-tensor facts of one batched decode, written by the prepare kernel.
@@ -146,10 +144,10 @@ struct BatchPlanDev {
   void *q_zero_base;      // mbits, q_ticket and q_status, contiguous
   size_t q_zero_bytes;
   uint32_t *d_ticket;
-  uint32_t *d_ticket2;    // indexed plans: the decode kernel's ticket
   uint32_t *d_ok;         // indexed plans: per-tensor valid flags
-  uint64_t *d_status;     // look-back words (per unit, or per index chunk)
-  void *d_zero_base;      // d_ticket, d_ticket2, d_ok and d_status, contiguous
+  uint32_t *d_done;       // indexed plans: per-tensor finished index chunks
+  uint64_t *d_status;     // small plans: look-back words, one per unit
+  void *d_zero_base;      // d_ticket, d_ok, d_done and d_status, contiguous
   size_t d_zero_bytes;
   BatchPrep *d_prep;      // count entries, rewritten by every decode call
   uint32_t *d_total;      // compact tile and chunk counts of the current decode call
@@ -157,8 +155,10 @@ struct BatchPlanDev {
   uint64_t *q_cagg;       // deferred placement: per 32-tile chunk summaries,
   uint8_t *q_stage;       // and the staged bytes, compress_stage_bytes_per_tile() per tile;
   uint32_t n_q_chunks;    // tile summaries and chunk counters sit in q_status
-  uint32_t *d_off;        // indexed plans: units' first groups, all tensors
-  uint32_t *d_page;       // and page tables
+  uint32_t *d_loc;        // indexed plans: units' first groups within their chunk (per
+                          // tensor d_tiles words from d_tile_begin)
+  uint32_t *d_cpre;       // and chunks' first groups (per tensor d_chunks + 1 words from
+                          // d_chunk_begin + tensor index)
   uint32_t n_d_chunks;
 };
 
@@ -232,7 +232,7 @@ struct IndexedStream {
   uint64_t cap;
 };
 struct IndexedLayout {
-  size_t status_off[kIndexPass], off_off[kIndexPass], page_off[kIndexPass];
+  size_t loc_off[kIndexPass], cpre_off[kIndexPass], page_off[kIndexPass];
   size_t zero_bytes, total_bytes;
 };
 IndexedLayout indexed_layout(const IndexedStream *s, int k, uint64_t n);

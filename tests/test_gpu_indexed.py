@@ -2,13 +2,14 @@
 
 Streams whose buffer spans 8 MiB or more, and every sum of two or more
 streams, are decoded through an index (each 512-byte payload unit's first
-group, and the unit that holds every 1024th group).  A single stream then
-takes payload tiles when it expands to more than 4 groups per payload byte on
-average and output (gather) tiles otherwise; several streams are summed in
-one pass of gather tiles.  These tests build streams of chosen density
-directly (any split of the zero runs is a valid stream), decode them on both
-sides of that switch, and sum mixes of dense, sparse, corrupt and unaligned
-streams, bit for bit against the oracle.
+group, and the chunk that holds every 1024th group).  A single stream is then
+decoded by one warp per unit: a unit that expands to at most 2048 groups
+(4 groups per payload byte on average) is expanded in shared memory and
+written as float4s, a longer one is written as zeros and then its literal
+groups; several streams are summed in one pass of output tiles.  These tests
+build streams of chosen density directly (any split of the zero runs is a
+valid stream), decode them on both sides of that switch, and sum mixes of
+dense, sparse, corrupt and unaligned streams, bit for bit against the oracle.
 """
 from __future__ import annotations
 
@@ -24,7 +25,7 @@ pytestmark = pytest.mark.gpu
 GUARD = 256
 CANARY = 0xA5
 INDEX_MIN_GROUPS = 16384 * 512     # 8 MiB of payload units: the indexed path
-GATHER_MAX_EXPANSION = 4           # gather tiles up to this many groups per byte
+GATHER_MAX_EXPANSION = 4           # units expanded in shared memory up to this many groups per byte
 
 
 @pytest.fixture(scope="module")
