@@ -314,12 +314,14 @@ def run_ours(args, rank, world, local):
     pre = tlc.tlc_kernel_timing_read()
     dom = max((k for k in pre if pre[k][0]), key=lambda k: pre[k][1])
 
-    # --graph: one CUDA graph per resident gradient, each holding one whole
-    # step (the three calls, with their scratch allocations); the timed
-    # region replays them in turn.  Small tensors are bound by the host's
-    # enqueue cost otherwise.
-    graphs = []        # per resident gradient: one graph per call of the step
+    # --graph: CUDA graphs of the calls, so that small tensors are timed on
+    # the GPU rather than at the host's launch rate.  Per resident gradient:
+    # one graph of `reps` whole steps (the timed region) and one graph of
+    # `reps` calls of each leg (the breakdown pass); reps shrinks as the
+    # tensor grows, to 1 from 2^26 values on.
+    graphs, leg_graphs = [], []
     graph_launches = None
+    reps = max(1, min(32, 1 << max(0, 26 - args.log2n))) if args.graph else 1
     if args.graph:
         tlc.tlc_kernel_timing_kinds([])
         tlc.tlc_kernel_timing(True)
@@ -333,20 +335,31 @@ def run_ours(args, rank, world, local):
                                                     in_caps=[cap], dev_status=status, stream=cs),
         ]
         for k in range(len(xs)):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cs):
+                for _ in range(reps):
+                    for call in calls:
+                        call(k)
+            graphs.append(gr)
+        tlc.tlc_kernel_timing(False)
+        per_graph = tlc.tlc_kernel_timing_read()
+        graph_launches = sum(v[0] for v in per_graph.values()) / len(graphs) / reps
+        for k in range(len(xs)):
             trio = []
             for call in calls:
                 gr = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(gr, stream=cs):
-                    call(k)
+                    for _ in range(reps):
+                        call(k)
                 trio.append(gr)
-            graphs.append(trio)
-        tlc.tlc_kernel_timing(False)
-        per_graph = tlc.tlc_kernel_timing_read()
-        graph_launches = sum(v[0] for v in per_graph.values()) / len(graphs)
-        for trio in graphs:
+            leg_graphs.append(trio)
+        for gr in graphs:
+            gr.replay()
+        for trio in leg_graphs:
             for gr in trio:
                 gr.replay()
         torch.cuda.synchronize()
+        args.steps = max(reps, args.steps // reps * reps)
 
     # Timed region: K steps between two events, with an event pair around
     # each launch of the dominant kernel only (each pair costs a few
@@ -362,11 +375,11 @@ def run_ours(args, rank, world, local):
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for i in range(args.steps):
-        if graphs:
-            for gr in graphs[i % len(graphs)]:
-                gr.replay()
-        else:
+    if graphs:
+        for i in range(args.steps // reps):
+            graphs[i % len(graphs)].replay()
+    else:
+        for i in range(args.steps):
             step()
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -399,8 +412,8 @@ def run_ours(args, rank, world, local):
         e = ev[k]
         e[0].record(stream)
         if graphs:
-            # each call replayed from its graph, events between the replays
-            for i, gr in enumerate(graphs[k % len(graphs)]):
+            # each leg replayed from its graph of `reps` calls, events between
+            for i, gr in enumerate(leg_graphs[k % len(leg_graphs)]):
                 gr.replay()
                 e[i + 1].record(stream)
             continue
@@ -415,7 +428,7 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
     tlc.tlc_kernel_timing(False)
     kern2 = tlc.tlc_kernel_timing_read()
-    legs = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps2)) / steps2
+    legs = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps2)) / steps2 / reps
             for i in range(3)]
     legs = max_over_ranks(legs, device=dev)
 
@@ -471,7 +484,7 @@ def run_ours(args, rank, world, local):
         "config": (workload_config(n, args.log2n, args.dense) if args.config == 3 else
                    {"workload": synth.CONFIGS[args.config]["name"], "n": n, "s": S_PARAM,
                     "l2": "L2-resident (x + err = 8 MiB)"}) | {"parallelism": f"replicas x{world}"}
-                  | ({"calls": "each step replayed from a CUDA graph of its three calls"}
+                  | ({"calls": f"CUDA graphs of {reps} whole steps, replayed"}
                      if graphs else {}),
         "clocks": clocks,
         "gpu_launches": int(sum(v[0] for v in kern.values())),
@@ -506,8 +519,8 @@ def run_ours(args, rank, world, local):
         "breakdown": (f"legs and kernels: a separate pass of {steps2} steps after the timed "
                       "region, with events between the calls and around every kernel"
                       if not graphs else
-                      f"legs: a separate pass of {steps2} steps after the timed region, each "
-                      "call replayed from its own CUDA graph with events between the "
+                      f"legs: a separate pass of {steps2} replays after the timed region, "
+                      f"each leg from its own CUDA graph of {reps} calls, events between the "
                       "replays (per-kernel times are not taken inside graphs)"),
     }
 
@@ -648,32 +661,39 @@ def run_config_set(args, rank, world, local):
         arena = torch.empty(plan.arena_bytes, dtype=torch.uint8, device=dev)
         acc_plan = tlc.Plan(ys=accs)
 
-    def legs():
+    def leg_compress():
         if use_plan:
             plan.compress(s, arena, lens, status, strm[0])
-            yield
-            plan.decompress(arena, lens, accumulate=False, dev_status=status, stream=strm[0])
-            yield
-            acc_plan.decompress(arena, lens, accumulate=True, dev_status=status, stream=strm[0])
-            yield
             return
         for i in range(len(ns)):
             tlc.tlc_compress(xs[i], s, errs[i], outs[i], lens[i:i + 1], status, strm[0])
-        yield
-        if args.config == 5:
-            yield
+
+    def leg_decompress():
+        if use_plan:
+            plan.decompress(arena, lens, accumulate=False, dev_status=status, stream=strm[0])
+        elif args.config != 5:
+            for i in range(len(ns)):
+                tlc.tlc_decompress(outs[i], ns[i], ys[i], in_len=lens[i:i + 1], in_cap=caps[i],
+                                   dev_status=status, stream=strm[0])
+
+    def leg_accumulate():
+        if use_plan:
+            acc_plan.decompress(arena, lens, accumulate=True, dev_status=status, stream=strm[0])
+        elif args.config == 5:
             tlc.tlc_decompress_accumulate(outs, ns[0], acc, in_lens=lens, in_caps=caps,
                                           dev_status=status, stream=strm[0])
         else:
             for i in range(len(ns)):
-                tlc.tlc_decompress(outs[i], ns[i], ys[i], in_len=lens[i:i + 1], in_cap=caps[i],
-                                   dev_status=status, stream=strm[0])
-            yield
-            for i in range(len(ns)):
                 tlc.tlc_decompress_accumulate([outs[i]], ns[i], accs[i], in_lens=lens[i:i + 1],
                                               in_caps=[caps[i]], dev_status=status,
                                               stream=strm[0])
-        yield
+
+    leg_fns = [leg_compress, leg_decompress, leg_accumulate]
+
+    def legs():
+        for fn in leg_fns:
+            fn()
+            yield
 
     for _ in range(max(3, args.warmup)):
         for _ in legs():
@@ -681,9 +701,12 @@ def run_config_set(args, rank, world, local):
     torch.cuda.synchronize()
     steps = max(1, min(args.steps, 50))
     graph = None
+    # --graph: `reps` whole steps captured as one CUDA graph (several for a
+    # small tensor set, so that the GPU, not the host's launch rate, sets the
+    # time), replayed in the timed region; launches counted while captured
+    reps = (16 if total < (1 << 24) else 1) if args.graph else 1
+    leg_graphs = []
     if args.graph:
-        # one step captured as a CUDA graph, replayed in the timed region;
-        # its launches are counted while it is captured
         tlc.tlc_kernel_timing_kinds([])
         tlc.tlc_kernel_timing(True)
         graph = torch.cuda.CUDAGraph()
@@ -691,13 +714,22 @@ def run_config_set(args, rank, world, local):
         cs.wait_stream(stream)
         strm[0] = cs
         with torch.cuda.graph(graph, stream=cs):
-            for _ in legs():
-                pass
-        strm[0] = stream
+            for _ in range(reps):
+                for _ in legs():
+                    pass
         tlc.tlc_kernel_timing(False)
-        per_step = tlc.tlc_kernel_timing_read()
+        per_step = {k: (v[0] // reps, v[1]) for k, v in tlc.tlc_kernel_timing_read().items()}
+        # one graph of `reps` calls per leg, for the breakdown pass
+        for fn in leg_fns:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=cs):
+                for _ in range(reps):
+                    fn()
+            leg_graphs.append(gr)
+        strm[0] = stream
         graph.replay()
         torch.cuda.synchronize()
+        steps = max(reps, steps // reps * reps)
     # timed region: whole steps between two events; launches counted, no
     # per-kernel events
     if world > 1:
@@ -708,7 +740,7 @@ def run_config_set(args, rank, world, local):
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for _ in range(steps):
+    for _ in range(steps // reps):
         if graph is not None:
             graph.replay()
         else:
@@ -729,12 +761,17 @@ def run_config_set(args, rank, world, local):
     tlc.tlc_kernel_timing(True)
     for k in range(steps):
         ev[k][0].record(stream)
+        if leg_graphs:
+            for j, gr in enumerate(leg_graphs):
+                gr.replay()
+                ev[k][j + 1].record(stream)
+            continue
         for j, _ in enumerate(legs()):
             ev[k][j + 1].record(stream)
     torch.cuda.synchronize()
     tlc.tlc_kernel_timing(False)
     kern = tlc.tlc_kernel_timing_read()
-    legs_ms = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)) / steps
+    legs_ms = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps)) / steps / reps
                for i in range(3)]
     L = int(lens.sum().item())
     in_bytes = 4 * total
@@ -748,8 +785,8 @@ def run_config_set(args, rank, world, local):
                    "calls": ("one plan call per leg (tlc_compress_batch / "
                              "tlc_decompress_batch)" if use_plan else
                              "one C-ABI call per tensor and leg")
-                   + ("; each step replayed from a CUDA graph of those calls" if args.graph
-                      else "")},
+                   + (f"; replayed from CUDA graphs of {reps} steps (the breakdown: of "
+                      f"{reps} calls of each leg)" if args.graph else "")},
         "legs": {"compress_ms": round(legs_ms[0], 4),
                  "compress_gbs": round(in_bytes / (legs_ms[0] * 1e-3) / 1e9, 1),
                  "stream_bytes": L, "bits_per_value": round(8 * L / total, 5)},

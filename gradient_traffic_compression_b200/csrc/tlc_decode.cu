@@ -525,6 +525,8 @@ __device__ __forceinline__ void warp_emit(const uint16_t *wd, uint64_t g_first, 
     return;
   }
   float4 *y4 = reinterpret_cast<float4 *>(y);
+  // (dense output: four float4s per lane in flight)
+#pragma unroll(kMode == kWrite ? 4 : 1)
   for (uint32_t v = v0 + lane; v < v1; v += kWarp) {
     const uint32_t e0 = v << 2;
     const uint32_t g = e0 / 5u;
@@ -581,11 +583,16 @@ __device__ void scan_chunks(const IndexOut &s, uint32_t n_chunks, IndexSmem &sm,
                             int32_t *dev_status) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint64_t carry = 0;
-  for (uint32_t base = 0; base < n_chunks; base += kDThreads * kScanPer) {
-    const uint32_t c0 = base + threadIdx.x * kScanPer;
+  // each thread a contiguous share of at most kScanPer chunks, as small as
+  // the pass allows (the page-table writes of a share are one thread's)
+  for (uint32_t base = 0; base < n_chunks;) {
+    const uint32_t per = min((uint32_t)kScanPer, (n_chunks - base + kDThreads - 1) / kDThreads);
+    const uint32_t c0 = base + threadIdx.x * per;
+    const uint32_t cend = min(c0 + per, n_chunks);
+    base += kDThreads * per;
     uint32_t v[kScanPer];
 #pragma unroll
-    for (int i = 0; i < kScanPer; ++i) v[i] = c0 + i < n_chunks ? __ldcg(s.cpre + c0 + i) : 0u;
+    for (int i = 0; i < kScanPer; ++i) v[i] = c0 + i < cend ? __ldcg(s.cpre + c0 + i) : 0u;
     uint64_t sum = 0;
 #pragma unroll
     for (int i = 0; i < kScanPer; ++i) sum += v[i];
@@ -612,7 +619,7 @@ __device__ void scan_chunks(const IndexOut &s, uint32_t n_chunks, IndexSmem &sm,
 #pragma unroll
     for (int i = 0; i < kScanPer; ++i) {
       const uint32_t c = c0 + i;
-      if (c < n_chunks) {
+      if (c < cend) {
         s.cpre[c] = sat32(run);
         if (s.page) {
           const uint64_t pend = umin64(run + v[i], s.groups);
@@ -979,25 +986,35 @@ struct GatherSmem {
   uint32_t lit[kK];         // the stream has a non-zero literal in the tile
 };
 
-// The unit of stream S that holds group g (< the stream's groups), by one
-// warp: the page gives the chunk, the chunk's 32 loc[] entries the unit.
-// Every lane gets the result.
-__device__ __forceinline__ uint32_t unit_of_group(const GStream &S, uint64_t g) {
+// The units of stream S that hold groups ga and gb (each below the
+// stream's groups, or gb = ~0 for the stream's last unit), by one warp: the
+// page gives a group's chunk, the chunk's 32 loc[] entries its unit; both
+// lookups' loads are issued together.  Every lane gets the results.
+__device__ __forceinline__ void units_of_groups(const GStream &S, uint64_t ga, uint64_t gb,
+                                                uint32_t &ua, uint32_t &ub) {
   const int lane = threadIdx.x & 31;
   const uint32_t n_chunks = (S.n_units + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
-  const uint32_t c = (uint32_t)umin64(__ldg(S.page + g / kPage), n_chunks - 1);
-  const uint64_t u = (uint64_t)c * kDecodeChunkUnits + lane;
-  const bool in = u < S.n_units && (uint64_t)__ldg(S.cpre + c) + __ldg(S.loc + u) <= g;
-  const uint32_t mask = __ballot_sync(0xffffffffu, in);
-  return c * kDecodeChunkUnits + (mask ? 31 - __clz(mask) : 0);
+  const bool last = gb == ~0ull;
+  const uint32_t ca = (uint32_t)umin64(__ldg(S.page + ga / kPage), n_chunks - 1);
+  const uint32_t cb = last ? 0u : (uint32_t)umin64(__ldg(S.page + gb / kPage), n_chunks - 1);
+  const uint64_t va = (uint64_t)ca * kDecodeChunkUnits + lane;
+  const uint64_t vb = (uint64_t)cb * kDecodeChunkUnits + lane;
+  const uint64_t pa = __ldg(S.cpre + ca), pb = last ? 0 : __ldg(S.cpre + cb);
+  const uint32_t la = va < S.n_units ? __ldg(S.loc + va) : 0xffffffffu;
+  const uint32_t lb = (!last && vb < S.n_units) ? __ldg(S.loc + vb) : 0xffffffffu;
+  const uint32_t ma = __ballot_sync(0xffffffffu, va < S.n_units && pa + la <= ga);
+  const uint32_t mb = __ballot_sync(0xffffffffu, !last && vb < S.n_units && pb + lb <= gb);
+  ua = ca * kDecodeChunkUnits + (ma ? 31 - __clz(ma) : 0);
+  ub = last ? S.n_units - 1 : cb * kDecodeChunkUnits + (mb ? 31 - __clz(mb) : 0);
 }
 
 // One warp: unit u of stream S.  Each lane takes 16 consecutive payload
 // bytes; a warp scan of their expansion counts gives each lane's first
-// group; literal groups that fall in [g0, g0 + gn) go to grp.  Sets *lit
-// when a literal other than the zero group 121 was placed.
+// group; literal groups that fall in [g0, g0 + gn) go to wd as their digit
+// words (lut[] of the byte).  Sets *lit when a literal other than the zero
+// group 121 was placed.
 __device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t g0, uint32_t gn,
-                                          uint8_t *grp, uint32_t *lit) {
+                                          uint16_t *wd, const uint16_t *lut, uint32_t *lit) {
   const int lane = threadIdx.x & 31;
   const uint64_t base = (uint64_t)u * kDecodeUnit + 16ull * lane;
   uint32_t w[4] = {0u, 0u, 0u, 0u};
@@ -1037,7 +1054,7 @@ __device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t
         const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
         if (b < 243u) {
           if (g >= g0 && g < ge && TLC_CHECK(g - g0 < (uint64_t)gn)) {
-            grp[g - g0] = (uint8_t)b;
+            wd[g - g0] = lut[b];
             mine = mine || b != 121u;
           }
           ++g;
@@ -1050,26 +1067,27 @@ __device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t
   if (__any_sync(0xffffffffu, mine) && lane == 0) *lit = 1u;
 }
 
-// One gather tile: output groups [g0, g0 + gn) of k streams (2 <= k <= kK,
-// all valid, in stream order) added into acc.  Whole block; ends
-// synchronised.  grp holds kK * kGt bytes.
+// One gather tile: output groups [g0, g0 + gn) of k streams (k <= kK, all
+// valid, in stream order) added into acc.  Whole block; ends synchronised.
+// wd holds kK * (kGt + 8) digit words.
 template <int kGt, int kK>
 __device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g0,
                                             uint64_t groups, uint64_t n, float *y, bool vec,
-                                            const uint16_t *lut, const float4 *pat, uint8_t *grp,
+                                            const uint16_t *lut, const float4 *pat, uint16_t *wd,
                                             GatherSmem<kK> &sm) {
-  static_assert(kGt % kPage == 0 && kGt % 16 == 0 && kK <= kDWarps, "tile shape");
+  static_assert(kGt % kPage == 0 && kGt % 8 == 0 && kK <= kDWarps, "tile shape");
+  constexpr uint32_t kStride = kGt + 8;  // digit words per stream (one spare word)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t gn = (uint32_t)umin64(kGt, groups - g0);
-  // pre-fill with the zero group; warp s finds stream s's unit range
+  // pre-fill with the zero group's digit word; warp s finds stream s's units
   for (int s = 0; s < k; ++s)
-    for (uint32_t w = threadIdx.x; w < (gn + 15) / 16; w += kDThreads)
-      reinterpret_cast<uint4 *>(grp + s * kGt)[w] =
-          make_uint4(0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u);
+    for (uint32_t w = threadIdx.x; w < (gn + 7) / 8; w += kDThreads)
+      reinterpret_cast<uint4 *>(wd + s * kStride)[w] =
+          make_uint4(0x01550155u, 0x01550155u, 0x01550155u, 0x01550155u);
   if (warp < k) {
     const GStream &S = gs[warp];
-    const uint32_t uf = unit_of_group(S, g0);
-    uint32_t ul = g0 + gn < groups ? unit_of_group(S, g0 + gn) : S.n_units - 1;
+    uint32_t uf, ul;
+    units_of_groups(S, g0, g0 + gn < groups ? g0 + gn : ~0ull, uf, ul);
     if (ul < uf) ul = uf;
     if (lane == 0) {
       sm.uf[warp] = uf;
@@ -1078,9 +1096,15 @@ __device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g
     }
   }
   __syncthreads();
-  for (int s = 0; s < k; ++s)
-    for (uint32_t i = warp; i < sm.nu[s]; i += kDWarps)
-      walk_unit(gs[s], sm.uf[s] + i, g0, gn, grp + s * kGt, &sm.lit[s]);
+  // every (stream, unit) pair of the tile, spread over the warps
+  uint32_t items = 0;
+  for (int s = 0; s < k; ++s) items += sm.nu[s];
+  for (uint32_t i = warp; i < items; i += kDWarps) {
+    int s = 0;
+    uint32_t r = i;
+    while (r >= sm.nu[s]) r -= sm.nu[s++];
+    walk_unit(gs[s], sm.uf[s] + r, g0, gn, wd + s * kStride, lut, &sm.lit[s]);
+  }
   __syncthreads();
   // one read-modify-write of each float4 of acc: the streams' non-zero
   // values added in stream order
@@ -1103,9 +1127,8 @@ __device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g
 #pragma unroll
       for (int i = 0; i < kK; ++i) {
         if ((act >> i) & 1u) {
-          const uint8_t *gb = grp + i * kGt;
-          const uint32_t c0 = gb[li], c1 = gb[li + 1];
-          const uint32_t p8 = (((uint32_t)lut[c0] | ((uint32_t)lut[c1] << 10)) >> (2u * d0)) & 0xffu;
+          const uint16_t *ws = wd + i * kStride;
+          const uint32_t p8 = (((uint32_t)ws[li] | ((uint32_t)ws[li + 1] << 10)) >> (2u * d0)) & 0xffu;
           if (p8 == 0x55u) continue;
           if (!loaded) {
             o = y4[v];
@@ -1132,7 +1155,7 @@ __device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g
 #pragma unroll
       for (int i = 0; i < kK; ++i) {
         if ((act >> i) & 1u) {
-          const uint32_t dig = (lut[grp[i * kGt + (g - o32)]] >> sh) & 3u;
+          const uint32_t dig = (wd[i * kStride + (g - o32)] >> sh) & 3u;
           if (dig == 1u) continue;
           if (!loaded) {
             v = y[e];
@@ -1156,10 +1179,11 @@ __device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g
   __syncthreads();
 }
 
-// Shared memory (dynamic part) of k_decode_ix: the gather tile's group bytes.
+// Shared memory (dynamic part) of k_decode_ix: the gather tile's digit
+// words, kGt + 8 per stream.
 template <int kGt, int kK>
 constexpr size_t ix_smem_bytes() {
-  return (size_t)kK * kGt + 16;
+  return (size_t)kK * (kGt + 8) * sizeof(uint16_t);
 }
 
 // Add k (2 <= k <= kK) indexed streams, in stream order, into acc by gather
@@ -1206,8 +1230,8 @@ __global__ void __launch_bounds__(kDThreads, 6) k_decode_ix(const IxArgs a) {
     __syncthreads();
     const uint32_t t = tile_s;
     if (t >= n_tiles) break;
-    gather_tile<kGt, kK>(gs, na, (uint64_t)t * kGt, a.groups, a.n, a.y, a.vec, lut, pat, dyn_s,
-                         gsm);
+    gather_tile<kGt, kK>(gs, na, (uint64_t)t * kGt, a.groups, a.n, a.y, a.vec, lut, pat,
+                         reinterpret_cast<uint16_t *>(dyn_s), gsm);
   }
 }
 
