@@ -68,7 +68,7 @@ struct DecodeShape {
   static constexpr int kMaxGroups = kTile * 14;      // largest expansion of a tile
 };
 #ifndef TLC_D_LOOKV
-#define TLC_D_LOOKV 1
+#define TLC_D_LOOKV 4
 #endif
 constexpr int kLookV = TLC_D_LOOKV;   // look-back words per lane per round trip
 // Streams whose capacity allows this many 512-byte units or more are
@@ -161,6 +161,18 @@ __device__ __forceinline__ float dequant(uint32_t dig, float scale) {
 }
 
 __device__ __forceinline__ uint32_t expansion(uint32_t b) { return b >= 243u ? b - 241u : 1u; }
+
+// The same for the four bytes of a word at once: each byte stands for
+// 1 + max(b - 242, 0) groups, so the word for 4 + the byte sum of the
+// saturated differences.
+__device__ __forceinline__ uint32_t word_expansion(uint32_t w) {
+  return 4u + __vsadu4(__vsubus4(w, 0xF2F2F2F2u), 0u);
+}
+
+// Literal bytes other than the zero group 121 among the four bytes of a word.
+__device__ __forceinline__ uint32_t word_literals(uint32_t w) {
+  return __popc(__vcmpltu4(w, 0xF3F3F3F3u) & __vcmpne4(w, 0x79797979u)) >> 3;
+}
 
 // One stream's decode job.
 struct DecodeJob {
@@ -673,9 +685,7 @@ __device__ __forceinline__ void index_chunk(const IndexOut &s, uint32_t c, uint3
     for (int i = 0; i < kUnitsPerWarp; ++i) {
       uint32_t e = 0;
 #pragma unroll
-      for (int k = 4 * i; k < 4 * i + 4; ++k)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) e += expansion((w[k] >> (8 * q)) & 0xffu);
+      for (int k = 4 * i; k < 4 * i + 4; ++k) e += word_expansion(w[k]);
       e = __reduce_add_sync(0xffffffffu, e);
       if (lane == 0) sm.ucnt[warp * kUnitsPerWarp + i] = e;
     }
@@ -815,12 +825,20 @@ __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, cons
     }
   }
   uint32_t e = 0, lits = 0;
+  if (nb == 16) {
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    if (k < nb) {
-      const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
-      e += expansion(b);
-      lits += (b < 243u && b != 121u) ? 1u : 0u;
+    for (int k = 0; k < 4; ++k) {
+      e += word_expansion(w[k]);
+      lits += word_literals(w[k]);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if (k < nb) {
+        const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
+        e += expansion(b);
+        lits += (b < 243u && b != 121u) ? 1u : 0u;
+      }
     }
   }
   uint32_t inc = e;
@@ -1035,9 +1053,14 @@ __device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t
     }
   }
   uint32_t e = 0;
+  if (nb == 16) {
 #pragma unroll
-  for (int k = 0; k < 16; ++k)
-    if (k < nb) e += expansion((w[k >> 2] >> (8 * (k & 3))) & 0xffu);
+    for (int k = 0; k < 4; ++k) e += word_expansion(w[k]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 16; ++k)
+      if (k < nb) e += expansion((w[k >> 2] >> (8 * (k & 3))) & 0xffu);
+  }
   uint32_t inc = e;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
