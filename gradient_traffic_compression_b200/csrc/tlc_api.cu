@@ -511,10 +511,10 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   const size_t sz_D = tlc::align_up(4 * dtt.size(), 256);
   const size_t sz_M = tlc::align_up(4 * (size_t)count + 8, 256);      // mbits, q_ticket
   const size_t sz_QS = tlc::align_up(8 * qtt.size(), 256);
-  // decode, zeroed per call: the ticket, per-tensor valid flags and
-  // finished-chunk counters, and (small plans) one look-back word per unit
+  // decode: the ticket, per-tensor valid flags and (small plans, zeroed per
+  // call) one look-back word per unit
   const bool d_ix = tlc::decode_deferred((uint32_t)dtt.size());
-  const size_t d_head = tlc::align_up(4 + 8 * (size_t)count, 8);
+  const size_t d_head = tlc::align_up(4 + 4 * (size_t)count, 8);
   const size_t sz_DS = tlc::align_up(d_head + (d_ix ? 0 : 8 * dtt.size()), 256);
   const size_t sz_P = tlc::align_up(sizeof(tlc::BatchPrep) * count + 8, 256);  // prep, total
   // the index of indexed plans: units' first groups in their chunk, chunks'
@@ -556,7 +556,6 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   char *zd = zq + sz_M + sz_QS;
   D.d_ticket = reinterpret_cast<uint32_t *>(zd);
   D.d_ok = reinterpret_cast<uint32_t *>(zd + 4);
-  D.d_done = reinterpret_cast<uint32_t *>(zd + 4 + 4 * (size_t)count);
   D.d_status = d_ix ? nullptr : reinterpret_cast<uint64_t *>(zd + d_head);
   D.d_zero_base = zd;
   D.d_zero_bytes = d_head + (d_ix ? 0 : 8 * dtt.size());

@@ -70,6 +70,7 @@ __global__ void __launch_bounds__(kAbsThreads)
 k_absmax(const float *__restrict__ x, const float *__restrict__ err, uint64_t n,
          uint32_t *__restrict__ partial, uint64_t *__restrict__ zero_words,
          uint32_t n_zero, CompressRecord *rec) {
+  pdl_enter();
   if (rec && blockIdx.x == 0 && threadIdx.x == 0) rec->nonzeros = 0;
   uint32_t m = 0;
   const uint64_t gtid = (uint64_t)blockIdx.x * kAbsThreads + threadIdx.x;
@@ -831,6 +832,7 @@ __global__ void TLC_Q_BOUNDS k_quant_zre(const QuantArgs a) {
   __shared__ uint32_t tile_id_s;
   __shared__ float scale_s, thr_s;
   __shared__ int ok_s;
+  pdl_enter();
 
   // M from the per-block partial maxima of k_absmax.
   if (threadIdx.x < kWarp) {
@@ -923,6 +925,7 @@ k_zre_place(const uint32_t *__restrict__ aggs, const uint64_t *__restrict__ cagg
             uint32_t n_tiles, const uint32_t *ok, const uint8_t *__restrict__ stage, uint8_t *out,
             uint64_t out_cap, uint64_t *out_len, CompressRecord *rec) {
   __shared__ uint32_t tC[kPlaceBlockTiles], tT[kPlaceBlockTiles], tA[kPlaceBlockTiles];
+  pdl_enter();
   if (!*ok) return;  // non-finite step: nothing was encoded
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t b0 = blockIdx.x * kPlaceBlockTiles;  // the block's first tile
@@ -1010,6 +1013,7 @@ k_zre_place(const uint32_t *__restrict__ aggs, const uint64_t *__restrict__ cagg
 __global__ void __launch_bounds__(kAbsThreads)
 k_absmax_batch(const BatchTensor *__restrict__ tensors, const BatchChunk *__restrict__ chunks,
                uint32_t *__restrict__ mbits) {
+  pdl_enter();
   const BatchChunk ch = chunks[blockIdx.x];
   const BatchTensor &T = tensors[ch.tensor];
   const uint64_t b = ch.start, e = umin64(ch.start + kBatchChunk, T.n);
@@ -1083,6 +1087,7 @@ template <bool kDeferred>
 __global__ void TLC_Q_BOUNDS k_quant_zre_batch(const BatchQuantArgs a) {
   __shared__ QuantSmem sm;
   __shared__ uint32_t tile_id_s;
+  pdl_enter();
   for (;;) {
     if (threadIdx.x == 0) tile_id_s = atomicAdd(a.ticket, 1u);
     __syncthreads();
@@ -1121,6 +1126,7 @@ __global__ void TLC_Q_BOUNDS k_quant_zre_batch(const BatchQuantArgs a) {
 // writes the closing remainder byte and the length.  Tensors whose step is
 // non-finite are skipped (k_quant_zre_batch set their length to 0).
 __global__ void __launch_bounds__(kPlaceThreads) k_zre_place_batch(const BatchQuantArgs a) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const uint32_t u = blockIdx.x * (kPlaceThreads / kWarp) + (threadIdx.x >> 5);
   if (u >= a.n_tiles) return;  // whole warp
@@ -1251,11 +1257,11 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
   // the word right after the status array).
   timing_begin(kKindAbsmax, stream);
   if (vec)
-    k_absmax<true><<<n_part, kAbsThreads, 0, stream>>>(x, err, n, sc.partial, sc.status,
-                                                        n_tiles + 1, rec);
+    launch_k(k_absmax<true>, n_part, kAbsThreads, 0, stream, x, err, n, sc.partial, sc.status,
+             n_tiles + 1, rec);
   else
-    k_absmax<false><<<n_part, kAbsThreads, 0, stream>>>(x, err, n, sc.partial, sc.status,
-                                                         n_tiles + 1, rec);
+    launch_k(k_absmax<false>, n_part, kAbsThreads, 0, stream, x, err, n, sc.partial, sc.status,
+             n_tiles + 1, rec);
   timing_end(kKindAbsmax, stream);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1302,26 +1308,26 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
   timing_begin(kKindQuantZre, stream);
   if (deferred) {
     if (rec)
-      (vec ? k_quant_zre<true, true, true> : k_quant_zre<false, true, true>)
-          <<<grid, kQThreads, 0, stream>>>(qa);
+      launch_k(vec ? k_quant_zre<true, true, true> : k_quant_zre<false, true, true>, grid,
+               kQThreads, 0, stream, qa);
     else if (vec)
-      k_quant_zre<true, true><<<grid, kQThreads, 0, stream>>>(qa);
+      launch_k(k_quant_zre<true, true>, grid, kQThreads, 0, stream, qa);
     else
-      k_quant_zre<false, true><<<grid, kQThreads, 0, stream>>>(qa);
+      launch_k(k_quant_zre<false, true>, grid, kQThreads, 0, stream, qa);
     timing_end(kKindQuantZre, stream);
     timing_begin(kKindZrePlace, stream);
     const uint32_t n_blocks = (n_tiles + kPlaceBlockTiles - 1) / kPlaceBlockTiles;
-    k_zre_place<<<n_blocks, kPlaceThreads, 0, stream>>>(qa.aggs, ds.cagg, n_tiles, ds.ok,
-                                                         ds.stage, out, out_cap, out_len, rec);
+    launch_k(k_zre_place, n_blocks, kPlaceThreads, 0, stream, qa.aggs, ds.cagg, n_tiles, ds.ok,
+             ds.stage, out, out_cap, out_len, rec);
     timing_end(kKindZrePlace, stream);
   } else {
     if (rec)
-      (vec ? k_quant_zre<true, false, true> : k_quant_zre<false, false, true>)
-          <<<grid, kQThreads, 0, stream>>>(qa);
+      launch_k(vec ? k_quant_zre<true, false, true> : k_quant_zre<false, false, true>, grid,
+               kQThreads, 0, stream, qa);
     else if (vec)
-      k_quant_zre<true, false><<<grid, kQThreads, 0, stream>>>(qa);
+      launch_k(k_quant_zre<true, false>, grid, kQThreads, 0, stream, qa);
     else
-      k_quant_zre<false, false><<<grid, kQThreads, 0, stream>>>(qa);
+      launch_k(k_quant_zre<false, false>, grid, kQThreads, 0, stream, qa);
     timing_end(kKindQuantZre, stream);
   }
   return cudaGetLastError();
@@ -1334,7 +1340,7 @@ cudaError_t launch_compress_batch(const DeviceInfo &dev, const BatchPlanDev &p, 
   cudaError_t e = cudaMemsetAsync(p.q_zero_base, 0, p.q_zero_bytes, stream);
   if (e != cudaSuccess) return e;
   timing_begin(kKindAbsmax, stream);
-  k_absmax_batch<<<p.n_chunks, kAbsThreads, 0, stream>>>(p.tensors, p.chunks, p.mbits);
+  launch_k(k_absmax_batch, p.n_chunks, kAbsThreads, 0, stream, p.tensors, p.chunks, p.mbits);
   timing_end(kKindAbsmax, stream);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1358,15 +1364,15 @@ cudaError_t launch_compress_batch(const DeviceInfo &dev, const BatchPlanDev &p, 
   if (grid > p.n_q_tiles) grid = p.n_q_tiles;
   timing_begin(kKindQuantZre, stream);
   if (p.q_deferred)
-    k_quant_zre_batch<true><<<grid, kQThreads, 0, stream>>>(qa);
+    launch_k(k_quant_zre_batch<true>, grid, kQThreads, 0, stream, qa);
   else
-    k_quant_zre_batch<false><<<grid, kQThreads, 0, stream>>>(qa);
+    launch_k(k_quant_zre_batch<false>, grid, kQThreads, 0, stream, qa);
   timing_end(kKindQuantZre, stream);
   if (p.q_deferred) {
     const uint32_t per_block = kPlaceThreads / kWarp;
     timing_begin(kKindZrePlace, stream);
-    k_zre_place_batch<<<(p.n_q_tiles + per_block - 1) / per_block, kPlaceThreads, 0, stream>>>(
-        qa);
+    launch_k(k_zre_place_batch, (p.n_q_tiles + per_block - 1) / per_block, kPlaceThreads, 0,
+             stream, qa);
     timing_end(kKindZrePlace, stream);
   }
   return cudaGetLastError();

@@ -19,14 +19,14 @@
 //
 // Large streams, and several streams summed in one pass: an index, then the
 // decode; no block of either kernel waits on another.
-//   k_decode_index  one block per 32-unit chunk of 512-byte payload units:
+//   k_index_count   one block per 64-unit chunk of 512-byte payload units:
 //                   each unit's first group relative to its chunk (loc[u])
-//                   and the chunk's group count; the last block of a stream
-//                   to finish (an atomic counter) scans the chunk counts into
-//                   each chunk's first group (cpre[c]), checks that the stream
-//                   expands to exactly ceil(n/5) groups, marks it valid, and,
-//                   for sums of several streams, records for every 1024th
-//                   group the chunk that holds it (page[p]).
+//                   and the chunk's group count.
+//   k_index_scan    one block per stream: the chunk counts scanned into each
+//                   chunk's first group (cpre[c]), the check that the stream
+//                   expands to exactly ceil(n/5) groups (its valid flag),
+//                   and, for sums of several streams, for every 1024th group
+//                   the chunk that holds it (page[p]).
 //   k_decode_units  one stream: one warp per 512-byte unit, first group
 //                   cpre[u / 32] + loc[u]; the unit's groups are expanded in
 //                   the warp's shared memory and written (or added) as
@@ -85,7 +85,7 @@ constexpr uint32_t kDecodeDeferMinTiles = TLC_DEFER_DECODE_MIN_TILES;
 constexpr uint32_t kPage = 1024;  // groups per page-table entry
 static_assert(TLC_GT_ACC % (8 * kPage) == 0, "tiles are whole pages");
 static_assert(kDecodeUnit == 4 * kWarp * 4, "a unit is 16 bytes per lane of a warp");
-static_assert(kDecodeChunkUnits == kWarp, "a chunk's units are one per lane of a warp");
+static_assert(kDecodeChunkUnits == 2 * kWarp, "a chunk's units are two per lane of a warp");
 
 size_t decode_smem_bytes(bool accumulate);
 
@@ -162,16 +162,40 @@ __device__ __forceinline__ float dequant(uint32_t dig, float scale) {
 
 __device__ __forceinline__ uint32_t expansion(uint32_t b) { return b >= 243u ? b - 241u : 1u; }
 
-// The same for the four bytes of a word at once: each byte stands for
-// 1 + max(b - 242, 0) groups, so the word for 4 + the byte sum of the
-// saturated differences.
-__device__ __forceinline__ uint32_t word_expansion(uint32_t w) {
-  return 4u + __vsadu4(__vsubus4(w, 0xF2F2F2F2u), 0u);
+// The same for 16 bytes (four words) at once.  An escape byte 243..255
+// (0xF3..0xFF: high nibble F, low nibble at least 3) stands for its low
+// nibble - 1 groups, so 16 bytes expand to 16 + (the escapes' low nibbles)
+// - 2 (the escapes).  esc_bits(w) has bit 7 of each escape byte of w set:
+// the per-byte sums of its one add cannot carry.  Per byte lane the low
+// nibbles add up to at most 60 and the escape counts to 4, so one multiply
+// sums the four byte lanes.
+__device__ __forceinline__ uint32_t esc_bits(uint32_t w) {
+  return w & ((w & 0x7F7F7F7Fu) + 0x0D0D0D0Du) & 0x80808080u;
+}
+__device__ __forceinline__ uint32_t byte_lane_sum(uint32_t x) { return (x * 0x01010101u) >> 24; }
+__device__ __forceinline__ uint32_t expansion16(const uint32_t (&w)[4]) {
+  uint32_t lo = 0, cnt = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t e = esc_bits(w[k]) >> 7;  // 1 in each escape byte
+    lo += w[k] & 0x0F0F0F0Fu & (e * 0x0Fu);
+    cnt += e;
+  }
+  return 16u + byte_lane_sum(lo) - 2u * byte_lane_sum(cnt);
 }
 
-// Literal bytes other than the zero group 121 among the four bytes of a word.
-__device__ __forceinline__ uint32_t word_literals(uint32_t w) {
-  return __popc(__vcmpltu4(w, 0xF3F3F3F3u) & __vcmpne4(w, 0x79797979u)) >> 3;
+// Literal bytes other than the zero group 121 among 16 bytes: those that
+// are neither escapes nor 121 (a zero byte of w ^ 0x79.., found without
+// carries between bytes).
+__device__ __forceinline__ uint32_t literals16(const uint32_t (&w)[4]) {
+  uint32_t cnt = 0;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t x = w[k] ^ 0x79797979u;
+    const uint32_t nz = ((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x;  // bit 7: byte of x not zero
+    cnt += ((~nz & 0x80808080u) | esc_bits(w[k])) >> 7;
+  }
+  return 16u - byte_lane_sum(cnt);
 }
 
 // One stream's decode job.
@@ -198,15 +222,40 @@ __device__ __forceinline__ void fill_lut(uint16_t *lut) {
   for (int v = threadIdx.x; v < 256; v += blockDim.x) lut[v] = v < 243 ? digits_of(v) : 0;
 }
 
-// For every 8-bit word of four digits (2 bits each, first value lowest), the
-// four quantized values q in {-1, 0, +1} as floats; a value is q * scale,
-// which is exact (and +0.0 for q = 0).  Digit 3 never occurs.
-__device__ __forceinline__ void fill_patterns(float4 *pat) {
-  for (int v = threadIdx.x; v < 256; v += blockDim.x) {
+// For every 4-bit word of two digits (2 bits each, first value lowest), the
+// two quantized values q in {-1, 0, +1} as floats; a value is q * scale,
+// which is exact (and +0.0 for q = 0).  Digit 3 never occurs.  The 16
+// entries of 8 bytes fill the 32 banks once, so no pattern of lookups has a
+// bank conflict.
+__device__ __forceinline__ void fill_pairs(float2 *pair) {
+  for (int v = threadIdx.x; v < 16; v += blockDim.x) {
     auto q = [](uint32_t d) { return d == 0u ? -1.0f : (d == 2u ? 1.0f : 0.0f); };
-    pat[v] = make_float4(q(v & 3u), q((v >> 2) & 3u), q((v >> 4) & 3u), q((v >> 6) & 3u));
+    pair[v] = make_float2(q(v & 3u), q((v >> 2) & 3u));
   }
 }
+
+// Four values from the 8-bit word p8 of their four digits: the pair table's
+// products with the scale, written or added where the digit is not zero.
+__device__ __forceinline__ float4 pattern4(const float2 *pair, uint32_t p8, float scale) {
+  const float2 a = pair[p8 & 15u], b = pair[p8 >> 4];
+  return make_float4(__fmul_rn(a.x, scale), __fmul_rn(a.y, scale), __fmul_rn(b.x, scale),
+                     __fmul_rn(b.y, scale));
+}
+__device__ __forceinline__ void add_pattern4(float4 &o, const float2 *pair, uint32_t p8,
+                                             float scale) {
+  const float4 p = pattern4(pair, p8, scale);
+  if ((p8 & 3u) != 1u) o.x = __fadd_rn(o.x, p.x);
+  if (((p8 >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, p.y);
+  if (((p8 >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, p.z);
+  if (((p8 >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, p.w);
+}
+
+// Digit words in shared memory windows sit at swizzled positions: position
+// p at p ^ (((p >> 6) & 7) << 1).  Lanes placing literals about 16
+// positions apart then hit distinct banks, and the 26 consecutive positions
+// a row of 32 float4s reads still do.  The swizzle stays inside each
+// aligned block of 16 positions, so a window is filled in whole blocks.
+__device__ __forceinline__ uint32_t wsw(uint32_t p) { return p ^ (((p >> 6) & 7u) << 1); }
 
 // Validate a stream (length and header) and return its payload length and
 // scale.  Corrupt when the length is below 4 or above the readable capacity,
@@ -475,6 +524,7 @@ k_decode(const DecodeArgs a) {
   __shared__ uint32_t tile_s;
   __shared__ float scale_s;
   __shared__ int ok_s;
+  pdl_enter();
 
   if (threadIdx.x == 0) {
     uint64_t m = 0;
@@ -509,27 +559,35 @@ k_decode(const DecodeArgs a) {
 }
 
 // Values [e_begin, e_end) of the groups whose digit words (lut[] of their
-// quartic bytes) sit in wd (wd[0] is group g_first), by one warp: each
-// aligned float4 is the sign pattern of its four digits times the scale
-// (dense output) or added to acc where a digit is not zero (accumulate);
-// single values at the ends, and everywhere when y is not 16-byte aligned.
-// Values 4v..4v+3 lie in group g = 4v/5 (digits d0..) and, when d0 >= 2,
-// spill into group g+1; both groups' digit words are joined so one shift
-// lines the four digits up.
+// quartic bytes) sit in wd at swizzled positions (position 0 is group
+// g_first), by one warp: each aligned float4 is its four digits' pair-table
+// entries times the scale (dense output) or added to acc where a digit is
+// not zero (accumulate, two float4s per lane loaded before either is
+// added); single values at the ends, and everywhere when y is not 16-byte
+// aligned.  Values 4v..4v+3 lie in group g = 4v/5 (digits d0..) and, when
+// d0 >= 2, spill into group g+1; both groups' digit words are joined so one
+// shift lines the four digits up.
 template <int kMode>
 __device__ __forceinline__ void warp_emit(const uint16_t *wd, uint64_t g_first, uint64_t e_begin,
                                           uint64_t e_end, float *y, bool vec, float scale,
-                                          const float4 *pat, int lane) {
+                                          const float2 *pair, int lane) {
   if (e_end <= e_begin) return;
   const uint32_t gf = (uint32_t)g_first;
   // n < 2^32, so value and float4 indices fit 32 bits
   auto put = [&](uint32_t e) {
     const uint32_t g = e / 5u;
-    const uint32_t dig = (wd[g - gf] >> (2 * (e - 5u * g))) & 3u;
+    const uint32_t dig = (wd[wsw(g - gf)] >> (2 * (e - 5u * g))) & 3u;
     if (kMode == kWrite)
       y[e] = dequant(dig, scale);
     else if (dig != 1u)
       y[e] = __fadd_rn(y[e], dequant(dig, scale));
+  };
+  auto digits8 = [&](uint32_t v) -> uint32_t {
+    const uint32_t e0 = v << 2;
+    const uint32_t g = e0 / 5u;
+    const uint32_t d0 = e0 - 5u * g;
+    const uint32_t li = g - gf;
+    return (((uint32_t)wd[wsw(li)] | ((uint32_t)wd[wsw(li + 1)] << 10)) >> (2u * d0)) & 0xffu;
   };
   const uint32_t v0 = (uint32_t)((e_begin + 3) / 4), v1 = (uint32_t)(e_end / 4);
   if (!vec || v1 <= v0) {
@@ -537,71 +595,163 @@ __device__ __forceinline__ void warp_emit(const uint16_t *wd, uint64_t g_first, 
     return;
   }
   float4 *y4 = reinterpret_cast<float4 *>(y);
-  // (dense output: four float4s per lane in flight)
-#pragma unroll(kMode == kWrite ? 4 : 1)
-  for (uint32_t v = v0 + lane; v < v1; v += kWarp) {
-    const uint32_t e0 = v << 2;
-    const uint32_t g = e0 / 5u;
-    const uint32_t d0 = e0 - 5u * g;
-    const uint32_t li = g - gf;
-    const uint32_t p8 = (((uint32_t)wd[li] | ((uint32_t)wd[li + 1] << 10)) >> (2u * d0)) & 0xffu;
-    const float4 p = pat[p8];
-    if (kMode == kWrite) {
-      y4[v] = make_float4(__fmul_rn(p.x, scale), __fmul_rn(p.y, scale), __fmul_rn(p.z, scale),
-                          __fmul_rn(p.w, scale));
-    } else if (p8 != 0x55u) {  // some of the four digits is not zero
-      float4 o = y4[v];
-      if ((p8 & 3u) != 1u) o.x = __fadd_rn(o.x, __fmul_rn(p.x, scale));
-      if (((p8 >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, __fmul_rn(p.y, scale));
-      if (((p8 >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, __fmul_rn(p.z, scale));
-      if (((p8 >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, __fmul_rn(p.w, scale));
-      y4[v] = o;
+  if (kMode == kWrite) {
+    // four float4s per lane in flight
+#pragma unroll 4
+    for (uint32_t v = v0 + lane; v < v1; v += kWarp) y4[v] = pattern4(pair, digits8(v), scale);
+  } else {
+    for (uint32_t v = v0 + lane; v < v1; v += 2 * kWarp) {
+      const uint32_t vb = v + kWarp;
+      const uint32_t pa = digits8(v);
+      const uint32_t pb = vb < v1 ? digits8(vb) : 0x55u;
+      float4 oa = make_float4(0.0f, 0.0f, 0.0f, 0.0f), ob = oa;
+      if (pa != 0x55u) oa = y4[v];  // 0x55: four zero digits
+      if (pb != 0x55u) ob = y4[vb];
+      if (pa != 0x55u) {
+        add_pattern4(oa, pair, pa, scale);
+        y4[v] = oa;
+      }
+      if (pb != 0x55u) {
+        add_pattern4(ob, pair, pb, scale);
+        y4[vb] = ob;
+      }
     }
   }
   // the partial float4s at both ends, one value per lane
   const uint32_t h = 4 * v0 - (uint32_t)e_begin, t = (uint32_t)e_end - 4 * v1;  // each < 4
-  if ((uint32_t)lane < h + t) put((uint32_t)lane < h ? (uint32_t)e_begin + lane : 4 * v1 + (lane - h));
+  if ((uint32_t)lane < h + t)
+    put((uint32_t)lane < h ? (uint32_t)e_begin + lane : 4 * v1 + (lane - h));
 }
 
 // ===================================================================== index
-// The index of one stream, as k_decode_index writes it.
-struct IndexOut {
-  const uint8_t *payload;
-  uint64_t m;          // payload length (valid header)
-  uint64_t groups;
-  uint32_t *loc;       // per unit: its first group, counted from its chunk's first
-  uint32_t *cpre;      // per chunk: its group count, then (scanned by the stream's last
-                       // chunk to finish) its first group; cpre[n_chunks]: the total
-  uint32_t *page;      // or nullptr: per page, the chunk holding group p * kPage
-  uint32_t *done;      // the stream's finished chunks (zero at launch)
-  uint32_t *ok;        // set to 1 when the stream expands to exactly `groups`
-};
+// The index of one stream: per 512-byte payload unit its first group,
+// counted from the first group of its 64-unit chunk (loc); per chunk its
+// group count, which the scan turns into the chunk's first group (cpre;
+// cpre[n_chunks] is then the stream's total); and, for sums of several
+// streams, per page of kPage groups the chunk holding the page's first
+// group.  Two kernels: the count (one block per chunk, eight units per
+// warp; no block waits on another) and the scan (one block per stream).
 
-struct IndexSmem {
-  uint32_t ucnt[kDecodeChunkUnits];
-  uint64_t wsum[kDWarps + 1];
-  uint32_t last;
+static_assert(kDecodeUnit == 4 * 4 * kWarp, "a unit is four 32-bit words per lane");
+constexpr uint32_t kWarpUnits = 8;  // units one warp of the count takes
+static_assert(kDecodeChunkUnits == kDWarps * kWarpUnits, "a chunk is one count block's units");
+
+// Units u0 .. u0 + 7 of a payload of m bytes, by one warp (every load of
+// the eight units issued before any count): lane i < 8 gets the group count
+// of unit u0 + i, every other lane 0; bytes past the payload count 0.
+// A unit wholly inside a 4-byte aligned payload is read as word lane + 32k
+// (k < 4) of the unit, so every load is one coalesced 128-byte line; the
+// payload's last unit, and every unit of an unaligned payload, byte by byte
+// (lane L: bytes 16L .. 16L + 15).
+__device__ __forceinline__ uint32_t count_units8(const uint8_t *payload, uint64_t m, uint64_t u0) {
+  const uint32_t lane = threadIdx.x & 31;
+  if (u0 * kDecodeUnit >= m) return 0u;
+  const uint64_t whole = m / kDecodeUnit - u0;  // units of this warp wholly inside (>= 0)
+  const uint32_t n_word = (reinterpret_cast<uintptr_t>(payload) & 3) == 0
+                              ? (uint32_t)umin64(whole, kWarpUnits) : 0u;
+  const uint32_t *p32 = reinterpret_cast<const uint32_t *>(payload + u0 * kDecodeUnit) + lane;
+  uint32_t w[kWarpUnits][4];
+  if (n_word == kWarpUnits) {
+#pragma unroll
+    for (uint32_t i = 0; i < kWarpUnits; ++i)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) w[i][k] = __ldg(p32 + i * (kDecodeUnit / 4) + k * kWarp);
+  } else {
+    // byte loads where needed; a byte past the payload is read as a
+    // literal 121 and its count taken off below
+#pragma unroll
+    for (uint32_t i = 0; i < kWarpUnits; ++i) {
+      if (i < n_word) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) w[i][k] = __ldg(p32 + i * (kDecodeUnit / 4) + k * kWarp);
+      } else {
+        const uint64_t b0 = (u0 + i) * kDecodeUnit + 16ull * lane;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t x = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t p = b0 + 4 * k + j;
+            x |= (p < m ? (uint32_t)__ldg(payload + p) : 121u) << (8 * j);
+          }
+          w[i][k] = x;
+        }
+      }
+    }
+  }
+  // a unit expands to at most 512 * 14 < 2^16 groups: two units per word
+  uint32_t pk[kWarpUnits / 2];
+#pragma unroll
+  for (uint32_t i = 0; i < kWarpUnits / 2; ++i)
+    pk[i] = __reduce_add_sync(0xffffffffu,
+                              expansion16(w[2 * i]) | (expansion16(w[2 * i + 1]) << 16));
+  const uint32_t h = (lane >> 1) & 3u;
+  const uint32_t v = h == 0 ? pk[0] : (h == 1 ? pk[1] : (h == 2 ? pk[2] : pk[3]));
+  uint32_t mine = lane < kWarpUnits ? ((lane & 1u) ? v >> 16 : v & 0xffffu) : 0u;
+  // the padding bytes past the payload counted one group each
+  if (lane < kWarpUnits) {
+    const uint64_t ub = (u0 + lane) * kDecodeUnit;
+    mine -= (uint32_t)(ub >= m ? kDecodeUnit : (ub + kDecodeUnit > m ? ub + kDecodeUnit - m : 0));
+  }
+  return mine;
+}
+
+// Chunk c (64 units) of a stream's payload of m bytes, by one block: warp w
+// counts units 8w .. 8w + 7; loc[u] = the unit's first group counted from
+// the chunk's first, cnt[c] = the chunk's group count (at most
+// 64 * 512 * 14).  wtot_s holds kDWarps words.  Ends synchronised.
+__device__ __forceinline__ void count_chunk(const uint8_t *payload, uint64_t m, uint32_t c,
+                                            uint32_t *loc, uint32_t *cnt, uint32_t *wtot_s) {
+  const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint64_t n_units = (m + kDecodeUnit - 1) / kDecodeUnit;
+  const uint64_t u0 = (uint64_t)c * kDecodeChunkUnits + warp * kWarpUnits;
+  const uint32_t mine = count_units8(payload, m, u0);
+  uint32_t inc = mine;
+#pragma unroll
+  for (uint32_t d = 1; d < kWarpUnits; d <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc += t;
+  }
+  if (lane == kWarpUnits - 1) wtot_s[warp] = inc;
+  __syncthreads();
+  uint32_t off = 0;
+  for (uint32_t w = 0; w < warp; ++w) off += wtot_s[w];
+  if (lane < kWarpUnits && u0 + lane < n_units) loc[u0 + lane] = off + inc - mine;
+  if (warp == kDWarps - 1 && lane == kWarpUnits - 1) cnt[c] = off + inc;
+  __syncthreads();  // wtot_s is rewritten by the next chunk
+}
+
+// What the scan of one stream writes.
+struct IndexOut {
+  uint32_t *cpre;      // chunk counts in, first groups out, then the total
+  uint32_t *page;      // or nullptr: per page, the chunk holding group p * kPage
+  uint32_t *ok;        // 1 when the stream expands to exactly `groups`, else 0
+  uint64_t groups;
 };
 
 __device__ __forceinline__ uint32_t sat32(uint64_t v) { return (uint32_t)umin64(v, 0xffffffffull); }
 
-// The stream's chunk counts, scanned by one block into each chunk's first
-// group, the total checked against the tensor's groups, and the page table.
-// In passes of kScanPer chunks per thread: each thread loads its contiguous
-// share into registers (all loads issued first), then a block scan of the
-// shares (64-bit: a corrupt stream's counts may add up past 2^32).
+// The stream's chunk counts, scanned by one block of kThreads into each
+// chunk's first group, the total checked against the tensor's groups, and
+// the page table.  In passes of up to kScanPer chunks per thread: each
+// thread loads its contiguous share into registers (all loads issued
+// first), then a block scan of the shares (64-bit: a corrupt stream's
+// counts may add up past 2^32).  wsum holds kThreads / 32 + 1 words.
 constexpr int kScanPer = 8;
-__device__ void scan_chunks(const IndexOut &s, uint32_t n_chunks, IndexSmem &sm,
+template <int kThreads>
+__device__ void scan_chunks(const IndexOut &s, uint32_t n_chunks, uint64_t *wsum,
                             int32_t *dev_status) {
+  constexpr int kWarps = kThreads / kWarp;
+  static_assert(kWarps <= kWarp, "one warp scans the warp sums");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint64_t carry = 0;
   // each thread a contiguous share of at most kScanPer chunks, as small as
   // the pass allows (the page-table writes of a share are one thread's)
   for (uint32_t base = 0; base < n_chunks;) {
-    const uint32_t per = min((uint32_t)kScanPer, (n_chunks - base + kDThreads - 1) / kDThreads);
+    const uint32_t per = min((uint32_t)kScanPer, (n_chunks - base + kThreads - 1) / kThreads);
     const uint32_t c0 = base + threadIdx.x * per;
     const uint32_t cend = min(c0 + per, n_chunks);
-    base += kDThreads * per;
+    base += kThreads * per;
     uint32_t v[kScanPer];
 #pragma unroll
     for (int i = 0; i < kScanPer; ++i) v[i] = c0 + i < cend ? __ldcg(s.cpre + c0 + i) : 0u;
@@ -614,20 +764,22 @@ __device__ void scan_chunks(const IndexOut &s, uint32_t n_chunks, IndexSmem &sm,
       const uint64_t t = __shfl_up_sync(0xffffffffu, inc, d);
       if (lane >= d) inc += t;
     }
-    if (lane == 31) sm.wsum[warp] = inc;
+    if (lane == 31) wsum[warp] = inc;
     __syncthreads();
-    if (threadIdx.x == 0) {
-      uint64_t run = 0;
-      for (int w = 0; w < kDWarps; ++w) {
-        const uint64_t t = sm.wsum[w];
-        sm.wsum[w] = run;
-        run += t;
+    if (warp == 0) {
+      const uint64_t x = lane < kWarps ? wsum[lane] : 0;
+      uint64_t y = x;
+#pragma unroll
+      for (int d = 1; d < 32; d <<= 1) {
+        const uint64_t t = __shfl_up_sync(0xffffffffu, y, d);
+        if (lane >= d) y += t;
       }
-      sm.wsum[kDWarps] = run;
+      if (lane < kWarps) wsum[lane] = y - x;
+      if (lane == 31) wsum[kWarps] = y;
     }
     __syncthreads();
-    uint64_t run = carry + sm.wsum[warp] + inc - sum;
-    carry += sm.wsum[kDWarps];
+    uint64_t run = carry + wsum[warp] + inc - sum;
+    carry += wsum[kWarps];
 #pragma unroll
     for (int i = 0; i < kScanPer; ++i) {
       const uint32_t c = c0 + i;
@@ -641,87 +793,18 @@ __device__ void scan_chunks(const IndexOut &s, uint32_t n_chunks, IndexSmem &sm,
         run += v[i];
       }
     }
-    __syncthreads();  // sm.wsum is rewritten by the next pass
+    __syncthreads();  // wsum is rewritten by the next pass
   }
   if (threadIdx.x == 0) {
     s.cpre[n_chunks] = sat32(carry);
-    if (carry == s.groups) *s.ok = 1u;
-    else report(dev_status, TLC_ERR_CORRUPT);
+    const bool ok = carry == s.groups;
+    *s.ok = ok ? 1u : 0u;
+    if (!ok) report(dev_status, TLC_ERR_CORRUPT);
   }
 }
 
-// Atomic add with acquire-release ordering at GPU scope: this thread's
-// earlier writes are visible to whichever thread's add comes later, and
-// that thread sees them.
-__device__ __forceinline__ uint32_t atomic_add_acq_rel(uint32_t *p, uint32_t v) {
-  uint32_t old;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v)
-               : "memory");
-  return old;
-}
-
-// Chunk c (32 units of 512 payload bytes) of one stream of n_chunks: the
-// units' group counts (one warp per 4 units, one 32-bit word per lane per
-// quarter unit, all loads first), loc[] and the chunk's count; the stream's
-// last chunk to finish then scans the counts.  Whole block; ends
-// synchronised.
-constexpr int kUnitsPerWarp = kDecodeChunkUnits / kDWarps;
-__device__ __forceinline__ void index_chunk(const IndexOut &s, uint32_t c, uint32_t n_chunks,
-                                            IndexSmem &sm, int32_t *dev_status) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint64_t n_units = (s.m + kDecodeUnit - 1) / kDecodeUnit;
-  const uint64_t u0 = (uint64_t)c * kDecodeChunkUnits + warp * kUnitsPerWarp;
-  constexpr int kW = kUnitsPerWarp * (kDecodeUnit / (4 * kWarp));
-  if ((reinterpret_cast<uintptr_t>(s.payload) & 3) == 0 && (u0 + kUnitsPerWarp) * kDecodeUnit <= s.m) {
-    // the warp's units lie inside the payload: one 32-bit word per lane per
-    // quarter unit, words interleaved across lanes so every load is
-    // coalesced, all loads issued first
-    uint32_t w[kW];
-#pragma unroll
-    for (int k = 0; k < kW; ++k)
-      w[k] = __ldg(reinterpret_cast<const uint32_t *>(
-          s.payload + (u0 + k / 4) * kDecodeUnit + 4 * (uint64_t)(lane + kWarp * (k % 4))));
-#pragma unroll
-    for (int i = 0; i < kUnitsPerWarp; ++i) {
-      uint32_t e = 0;
-#pragma unroll
-      for (int k = 4 * i; k < 4 * i + 4; ++k) e += word_expansion(w[k]);
-      e = __reduce_add_sync(0xffffffffu, e);
-      if (lane == 0) sm.ucnt[warp * kUnitsPerWarp + i] = e;
-    }
-  } else {
-    // the stream's last units, or an unaligned payload: byte loads
-    for (int i = 0; i < kUnitsPerWarp; ++i) {
-      uint32_t e = 0;
-      const uint64_t b0 = (u0 + i) * kDecodeUnit;
-      for (uint64_t p = b0 + lane; p < b0 + kDecodeUnit && p < s.m; p += kWarp)
-        e += expansion(__ldg(s.payload + p));
-      e = __reduce_add_sync(0xffffffffu, e);
-      if (lane == 0) sm.ucnt[warp * kUnitsPerWarp + i] = e;
-    }
-  }
-  __syncthreads();
-  if (warp == 0) {
-    const uint32_t v = sm.ucnt[lane];
-    uint32_t inc = v;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
-      if (lane >= d) inc += t;
-    }
-    const uint64_t u = (uint64_t)c * kDecodeChunkUnits + lane;
-    if (u < n_units) s.loc[u] = inc - v;
-    if (lane == 31) {
-      s.cpre[c] = inc;  // the chunk's count (at most 32 * 512 * 14), released by the add
-      sm.last = atomic_add_acq_rel(s.done, 1u) == n_chunks - 1 ? 1u : 0u;
-    }
-  }
-  __syncthreads();
-  if (sm.last) scan_chunks(s, n_chunks, sm, dev_status);
-  __syncthreads();
-}
-
-// Up to kIndexPass streams of n values each, decoded in one launch pair.
+// Up to kIndexPass streams of n values each, indexed and decoded by one
+// launch sequence.
 struct IxStream {
   const uint8_t *in;
   const uint64_t *len_dev;
@@ -734,9 +817,8 @@ struct IxArgs {
   IxStream s[kIndexPass];
   int k;
   uint64_t n, groups;
-  uint32_t *ticket2;   // decode tiles (cleared by k_decode_index)
-  uint32_t *ok;        // per stream (zero at launch)
-  uint32_t *done;      // per stream (zero at launch)
+  uint32_t *ticket2;   // decode tiles (cleared by the scan)
+  uint32_t *ok;        // per stream (written by the scan)
   float *y;
   bool vec;
   int32_t *dev_status;
@@ -747,21 +829,20 @@ __device__ __forceinline__ uint32_t chunks_of(uint64_t m) {
                     ((uint64_t)kDecodeUnit * kDecodeChunkUnits));
 }
 
-// Index of every stream: the chunks that exist (from each stream's length),
-// numbered stream by stream; block b takes chunks b, b + grid, ...
-__global__ void __launch_bounds__(kDThreads, 6) k_decode_index(const IxArgs a) {
+// Count of every stream: the chunks that exist (from each stream's length;
+// none for a corrupt one), numbered stream by stream; block b takes chunks
+// b, b + grid, ...
+__global__ void __launch_bounds__(kDThreads, 4) k_index_count(const IxArgs a) {
   __shared__ uint64_t m_s[kIndexPass];
   __shared__ uint32_t pre_s[kIndexPass + 1];
-  __shared__ IndexSmem sm;
+  __shared__ uint32_t wtot_s[kDWarps];
+  pdl_enter();
   if (threadIdx.x < (unsigned)a.k) {
     const IxStream &S = a.s[threadIdx.x];
     uint64_t m = 0;
     float scale = 0.0f;
-    const bool valid = read_stream_header(S.in, S.len_dev, S.cap, a.groups, m, scale);
-    m_s[threadIdx.x] = valid ? m : 0;
-    if (!valid && blockIdx.x == 0) report(a.dev_status, TLC_ERR_CORRUPT);
+    m_s[threadIdx.x] = read_stream_header(S.in, S.len_dev, S.cap, a.groups, m, scale) ? m : 0;
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) *a.ticket2 = 0;
   __syncthreads();
   if (threadIdx.x == 0) {
     pre_s[0] = 0;
@@ -773,10 +854,37 @@ __global__ void __launch_bounds__(kDThreads, 6) k_decode_index(const IxArgs a) {
     int s = 0;
     while (s + 1 < a.k && pre_s[s + 1] <= t) ++s;
     const IxStream &S = a.s[s];
-    const IndexOut io = {S.in + 4, m_s[s], a.groups, S.loc, S.cpre, S.page, a.done + s,
-                         a.ok + s};
-    index_chunk(io, t - pre_s[s], pre_s[s + 1] - pre_s[s], sm, a.dev_status);
+    count_chunk(S.in + 4, m_s[s], t - pre_s[s], S.loc, S.cpre, wtot_s);
   }
+}
+
+// Scan of every stream, block s for stream s (a corrupt stream gets ok = 0
+// and a report); block 0 also clears the decode ticket.
+constexpr int kScanThreads = 1024;
+__global__ void __launch_bounds__(kScanThreads) k_index_scan(const IxArgs a) {
+  __shared__ uint64_t wsum[kScanThreads / kWarp + 1];
+  __shared__ uint64_t m_s;
+  __shared__ int valid_s;
+  pdl_enter();
+  const int s = blockIdx.x;
+  const IxStream &S = a.s[s];
+  if (threadIdx.x == 0) {
+    uint64_t m = 0;
+    float scale = 0.0f;
+    valid_s = read_stream_header(S.in, S.len_dev, S.cap, a.groups, m, scale) ? 1 : 0;
+    m_s = m;
+    if (s == 0) *a.ticket2 = 0u;
+  }
+  __syncthreads();
+  if (!valid_s) {
+    if (threadIdx.x == 0) {
+      a.ok[s] = 0u;
+      report(a.dev_status, TLC_ERR_CORRUPT);
+    }
+    return;
+  }
+  const IndexOut io = {S.cpre, S.page, a.ok + s, a.groups};
+  scan_chunks<kScanThreads>(io, chunks_of(m_s), wsum, a.dev_status);
 }
 
 // ============================================================= warp units
@@ -794,8 +902,8 @@ __global__ void __launch_bounds__(kDThreads, 6) k_decode_index(const IxArgs a) {
 #define TLC_WARP_GROUPS 1024
 #endif
 constexpr uint32_t kWarpGroups = TLC_WARP_GROUPS;
-static_assert(kWarpGroups % 8 == 0, "whole 16-byte words of digit words");
-constexpr uint16_t kZeroDigits = 0x155;  // digit word of the zero group 121 (five 1s)
+static_assert(kWarpGroups % 16 == 0, "whole swizzle blocks of digit words");
+constexpr uint32_t kZeroDigits2 = 0x01550155u;  // two digit words of the zero group 121
 
 __device__ __forceinline__ uint64_t unit_first_group(const uint32_t *cpre, const uint32_t *loc,
                                                      uint32_t u) {
@@ -804,7 +912,7 @@ __device__ __forceinline__ uint64_t unit_first_group(const uint32_t *cpre, const
 
 template <int kMode>
 __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, const uint16_t *lut,
-                                            const float4 *pat, uint16_t *wd) {
+                                            const float2 *pair, uint16_t *wd) {
   const int lane = threadIdx.x & 31;
   const uint64_t base = (uint64_t)u * kDecodeUnit + 16ull * lane;
   uint32_t w[4] = {0u, 0u, 0u, 0u};
@@ -826,11 +934,8 @@ __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, cons
   }
   uint32_t e = 0, lits = 0;
   if (nb == 16) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      e += word_expansion(w[k]);
-      lits += word_literals(w[k]);
-    }
+    e = expansion16(w);
+    lits = literals16(w);
   } else {
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
@@ -890,9 +995,11 @@ __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, cons
   }
   for (uint32_t w0 = 0; w0 < Ec; w0 += kWarpGroups) {
     const uint32_t wn = min(kWarpGroups, Ec - w0);
-    for (uint32_t q = lane; q < (wn + 7) / 8; q += kWarp)
-      reinterpret_cast<uint4 *>(wd)[q] =
-          make_uint4(0x01550155u, 0x01550155u, 0x01550155u, 0x01550155u);
+    // positions 0..wn (the last one read by a float4 that spills), in whole
+    // swizzle blocks of 16
+    for (uint32_t q = lane; q < 2 * (wn / 16 + 1); q += kWarp)
+      reinterpret_cast<uint4 *>(wd)[q] = make_uint4(kZeroDigits2, kZeroDigits2, kZeroDigits2,
+                                                    kZeroDigits2);
     __syncwarp();
     uint32_t pos = excl;
 #pragma unroll
@@ -902,14 +1009,14 @@ __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, cons
         if (b >= 243u) {
           pos += b - 241u;
         } else {
-          if (pos - w0 < wn) wd[pos - w0] = lut[b];  // unsigned: pos in [w0, w0 + wn)
+          if (pos - w0 < wn) wd[wsw(pos - w0)] = lut[b];  // unsigned: pos in [w0, w0 + wn)
           ++pos;
         }
       }
     }
     __syncwarp();
     const uint64_t gb = O + w0;
-    warp_emit<kMode>(wd, gb, 5 * gb, umin64(5 * (gb + wn), j.n), j.y, j.vec, j.scale, pat, lane);
+    warp_emit<kMode>(wd, gb, 5 * gb, umin64(5 * (gb + wn), j.n), j.y, j.vec, j.scale, pair, lane);
     __syncwarp();
   }
 }
@@ -923,15 +1030,15 @@ __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, cons
 // Shared memory of a block of warp-unit decoders.
 struct UnitSmem {
   DecodeSmem d;   // digit table, block scan, a tile's first group
-  float4 pat[256];
-  __align__(16) uint16_t wd[kDWarps][kWarpGroups + 8];
+  float2 pair[16];
+  __align__(16) uint16_t wd[kDWarps][kWarpGroups + 16];
 };
 static_assert(sizeof(UnitSmem::wd) >= DecodeShape<kWrite>::kMaxGroups + 16,
               "a dense-output payload tile's groups fit the warps' windows");
 
 __device__ __forceinline__ void fill_unit_tables(UnitSmem &sm) {
   fill_lut(sm.d.lut);
-  fill_patterns(sm.pat);
+  fill_pairs(sm.pair);
 }
 
 // One indexed stream (dense output, or added into acc): warp w of block b
@@ -939,13 +1046,23 @@ __device__ __forceinline__ void fill_unit_tables(UnitSmem &sm) {
 // stream's dense output is written by whole blocks instead, one 512-byte
 // payload tile (unit) per block in ticket order: its all-zero tiles are each
 // one long run of zero stores, which a block writes faster than a warp.
+// Blocks per SM the warp-unit kernels are compiled for: the accumulate
+// emit keeps two float4s of acc per lane in flight, and the plan kernel
+// tracks its tensor: both need the registers of 6 blocks.
 template <int kMode>
-__global__ void __launch_bounds__(kDThreads, 8) k_decode_units(const IxArgs a) {
+constexpr int units_min_blocks(bool batch) {
+  return kMode == kWrite && !batch ? 8 : 6;
+}
+
+template <int kMode>
+__global__ void __launch_bounds__(kDThreads, units_min_blocks<kMode>(false))
+    k_decode_units(const IxArgs a) {
   __shared__ UnitSmem sm;
   __shared__ DecodeJob job_s;
   __shared__ int ok_s;
   __shared__ uint32_t tile_s;
   fill_unit_tables(sm);
+  pdl_enter();
   if (threadIdx.x == 0) {
     const IxStream &S = a.s[0];
     uint64_t m = 0;
@@ -983,7 +1100,7 @@ __global__ void __launch_bounds__(kDThreads, 8) k_decode_units(const IxArgs a) {
   const int warp = threadIdx.x >> 5;
   const uint32_t nw = gridDim.x * kDWarps;
   for (uint32_t u = blockIdx.x * kDWarps + warp; u < job_s.n_tiles; u += nw)
-    decode_unit<kMode>(job_s, u, sm.d.lut, sm.pat, sm.wd[warp]);
+    decode_unit<kMode>(job_s, u, sm.d.lut, sm.pair, sm.wd[warp]);
 }
 
 // ==================================================================== gather
@@ -1006,8 +1123,9 @@ struct GatherSmem {
 
 // The units of stream S that hold groups ga and gb (each below the
 // stream's groups, or gb = ~0 for the stream's last unit), by one warp: the
-// page gives a group's chunk, the chunk's 32 loc[] entries its unit; both
-// lookups' loads are issued together.  Every lane gets the results.
+// page gives a group's chunk, the chunk's 64 loc[] entries (two per lane)
+// its unit; both lookups' loads are issued together.  Every lane gets the
+// results.
 __device__ __forceinline__ void units_of_groups(const GStream &S, uint64_t ga, uint64_t gb,
                                                 uint32_t &ua, uint32_t &ub) {
   const int lane = threadIdx.x & 31;
@@ -1015,21 +1133,26 @@ __device__ __forceinline__ void units_of_groups(const GStream &S, uint64_t ga, u
   const bool last = gb == ~0ull;
   const uint32_t ca = (uint32_t)umin64(__ldg(S.page + ga / kPage), n_chunks - 1);
   const uint32_t cb = last ? 0u : (uint32_t)umin64(__ldg(S.page + gb / kPage), n_chunks - 1);
-  const uint64_t va = (uint64_t)ca * kDecodeChunkUnits + lane;
-  const uint64_t vb = (uint64_t)cb * kDecodeChunkUnits + lane;
   const uint64_t pa = __ldg(S.cpre + ca), pb = last ? 0 : __ldg(S.cpre + cb);
-  const uint32_t la = va < S.n_units ? __ldg(S.loc + va) : 0xffffffffu;
-  const uint32_t lb = (!last && vb < S.n_units) ? __ldg(S.loc + vb) : 0xffffffffu;
-  const uint32_t ma = __ballot_sync(0xffffffffu, va < S.n_units && pa + la <= ga);
-  const uint32_t mb = __ballot_sync(0xffffffffu, !last && vb < S.n_units && pb + lb <= gb);
-  ua = ca * kDecodeChunkUnits + (ma ? 31 - __clz(ma) : 0);
-  ub = last ? S.n_units - 1 : cb * kDecodeChunkUnits + (mb ? 31 - __clz(mb) : 0);
+  // the last unit of the chunk whose first group is at most g (loc[] does
+  // not decrease within a chunk)
+  auto find = [&](uint32_t c, uint64_t p, uint64_t g, bool use) -> uint32_t {
+    const uint64_t v0 = (uint64_t)c * kDecodeChunkUnits + lane, v1 = v0 + kWarp;
+    const bool ok0 = use && v0 < S.n_units, ok1 = use && v1 < S.n_units;
+    const uint32_t l0 = ok0 ? __ldg(S.loc + v0) : 0u, l1 = ok1 ? __ldg(S.loc + v1) : 0u;
+    const uint32_t m0 = __ballot_sync(0xffffffffu, ok0 && p + l0 <= g);
+    const uint32_t m1 = __ballot_sync(0xffffffffu, ok1 && p + l1 <= g);
+    return c * kDecodeChunkUnits + (m1 ? kWarp + 31 - __clz(m1) : (m0 ? 31 - __clz(m0) : 0));
+  };
+  ua = find(ca, pa, ga, true);
+  const uint32_t fb = find(cb, pb, gb, !last);
+  ub = last ? S.n_units - 1 : fb;
 }
 
 // One warp: unit u of stream S.  Each lane takes 16 consecutive payload
 // bytes; a warp scan of their expansion counts gives each lane's first
 // group; literal groups that fall in [g0, g0 + gn) go to wd as their digit
-// words (lut[] of the byte).  Sets *lit when a literal other than the zero
+// words (lut[] of the byte), at swizzled positions.  Sets *lit when a literal other than the zero
 // group 121 was placed.
 __device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t g0, uint32_t gn,
                                           uint16_t *wd, const uint16_t *lut, uint32_t *lit) {
@@ -1052,10 +1175,10 @@ __device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t
         if (k < nb) w[k >> 2] |= (uint32_t)__ldg(p + k) << (8 * (k & 3));
     }
   }
+  const uint64_t first = unit_first_group(S.cpre, S.loc, u);  // loaded with the bytes
   uint32_t e = 0;
   if (nb == 16) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) e += word_expansion(w[k]);
+    e = expansion16(w);
   } else {
 #pragma unroll
     for (int k = 0; k < 16; ++k)
@@ -1067,7 +1190,7 @@ __device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t
     const uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
     if (lane >= d) inc += t;
   }
-  uint64_t g = unit_first_group(S.cpre, S.loc, u) + (inc - e);
+  uint64_t g = first + (inc - e);
   const uint64_t ge = g0 + gn;
   bool mine = false;
   if (nb > 0 && g < ge && g + e > g0) {
@@ -1077,7 +1200,7 @@ __device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t
         const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
         if (b < 243u) {
           if (g >= g0 && g < ge && TLC_CHECK(g - g0 < (uint64_t)gn)) {
-            wd[g - g0] = lut[b];
+            wd[wsw((uint32_t)(g - g0))] = lut[b];
             mine = mine || b != 121u;
           }
           ++g;
@@ -1092,21 +1215,23 @@ __device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t
 
 // One gather tile: output groups [g0, g0 + gn) of k streams (k <= kK, all
 // valid, in stream order) added into acc.  Whole block; ends synchronised.
-// wd holds kK * (kGt + 8) digit words.
+// wd holds kK * (kGt + 16) digit words.
 template <int kGt, int kK>
 __device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g0,
                                             uint64_t groups, uint64_t n, float *y, bool vec,
-                                            const uint16_t *lut, const float4 *pat, uint16_t *wd,
+                                            const uint16_t *lut, const float2 *pair, uint16_t *wd,
                                             GatherSmem<kK> &sm) {
-  static_assert(kGt % kPage == 0 && kGt % 8 == 0 && kK <= kDWarps, "tile shape");
-  constexpr uint32_t kStride = kGt + 8;  // digit words per stream (one spare word)
+  static_assert(kGt % kPage == 0 && kGt % 16 == 0 && kK <= kDWarps && kK <= 8, "tile shape");
+  constexpr uint32_t kStride = kGt + 16;  // digit words per stream (one spare swizzle block)
+  constexpr int kPk = (kK + 3) / 4;       // words of four streams' 8-bit digit words
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t gn = (uint32_t)umin64(kGt, groups - g0);
-  // pre-fill with the zero group's digit word; warp s finds stream s's units
+  // pre-fill positions 0..gn (in whole swizzle blocks) with the zero group's
+  // digit word; warp s finds stream s's units
   for (int s = 0; s < k; ++s)
-    for (uint32_t w = threadIdx.x; w < (gn + 7) / 8; w += kDThreads)
+    for (uint32_t w = threadIdx.x; w < 2 * (gn / 16 + 1); w += kDThreads)
       reinterpret_cast<uint4 *>(wd + s * kStride)[w] =
-          make_uint4(0x01550155u, 0x01550155u, 0x01550155u, 0x01550155u);
+          make_uint4(kZeroDigits2, kZeroDigits2, kZeroDigits2, kZeroDigits2);
   if (warp < k) {
     const GStream &S = gs[warp];
     uint32_t uf, ul;
@@ -1140,32 +1265,50 @@ __device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g
     const uint32_t o32 = (uint32_t)g0;
     const uint64_t v0 = vec ? (e_begin + 3) / 4 : e_end, v1 = vec ? e_end / 4 : e_end;
     float4 *y4 = reinterpret_cast<float4 *>(y);
-    for (uint32_t v = (uint32_t)v0 + threadIdx.x; v < (uint32_t)v1; v += kDThreads) {
+    // the active streams' four digits of float4 v, eight bits per stream
+    // packed into pk; returns the streams with a non-zero digit
+    auto digits = [&](uint32_t v, uint32_t(&pk)[kPk]) -> uint32_t {
       const uint32_t e0 = v << 2;
       const uint32_t g = e0 / 5u;
       const uint32_t d0 = e0 - 5u * g;
-      const uint32_t li = g - o32;
-      float4 o;
-      bool loaded = false;
+      const uint32_t ia = wsw(g - o32), ib = wsw(g - o32 + 1);
+      uint32_t nz = 0;
+#pragma unroll
+      for (int i = 0; i < kPk; ++i) pk[i] = 0x55555555u;
 #pragma unroll
       for (int i = 0; i < kK; ++i) {
         if ((act >> i) & 1u) {
           const uint16_t *ws = wd + i * kStride;
-          const uint32_t p8 = (((uint32_t)ws[li] | ((uint32_t)ws[li + 1] << 10)) >> (2u * d0)) & 0xffu;
-          if (p8 == 0x55u) continue;
-          if (!loaded) {
-            o = y4[v];
-            loaded = true;
-          }
-          const float4 p = pat[p8];
-          const float sc = gs[i].scale;
-          if ((p8 & 3u) != 1u) o.x = __fadd_rn(o.x, __fmul_rn(p.x, sc));
-          if (((p8 >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, __fmul_rn(p.y, sc));
-          if (((p8 >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, __fmul_rn(p.z, sc));
-          if (((p8 >> 6) & 3u) != 1u) o.w = __fadd_rn(o.w, __fmul_rn(p.w, sc));
+          const uint32_t p8 = (((uint32_t)ws[ia] | ((uint32_t)ws[ib] << 10)) >> (2u * d0)) & 0xffu;
+          pk[i / 4] ^= (p8 ^ 0x55u) << (8 * (i % 4));
+          if (p8 != 0x55u) nz |= 1u << i;
         }
       }
-      if (loaded) y4[v] = o;
+      return nz;
+    };
+    auto add_streams = [&](float4 &o, uint32_t nz, const uint32_t(&pk)[kPk]) {
+#pragma unroll
+      for (int i = 0; i < kK; ++i)
+        if ((nz >> i) & 1u)
+          add_pattern4(o, pair, (pk[i / 4] >> (8 * (i % 4))) & 0xffu, gs[i].scale);
+    };
+    // two float4s per thread, both loaded before either is added
+    for (uint32_t v = (uint32_t)v0 + threadIdx.x; v < (uint32_t)v1; v += 2 * kDThreads) {
+      const uint32_t vb = v + kDThreads;
+      uint32_t pka[kPk], pkb[kPk];
+      const uint32_t nza = digits(v, pka);
+      const uint32_t nzb = vb < (uint32_t)v1 ? digits(vb, pkb) : 0u;
+      float4 oa = make_float4(0.0f, 0.0f, 0.0f, 0.0f), ob = oa;
+      if (nza) oa = y4[v];
+      if (nzb) ob = y4[vb];
+      if (nza) {
+        add_streams(oa, nza, pka);
+        y4[v] = oa;
+      }
+      if (nzb) {
+        add_streams(ob, nzb, pkb);
+        y4[vb] = ob;
+      }
     }
     // single values: the edges of the float4 range, or every value when
     // acc is not 16-byte aligned
@@ -1178,7 +1321,7 @@ __device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g
 #pragma unroll
       for (int i = 0; i < kK; ++i) {
         if ((act >> i) & 1u) {
-          const uint32_t dig = (wd[i * kStride + (g - o32)] >> sh) & 3u;
+          const uint32_t dig = (wd[i * kStride + wsw(g - o32)] >> sh) & 3u;
           if (dig == 1u) continue;
           if (!loaded) {
             v = y[e];
@@ -1203,10 +1346,10 @@ __device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g
 }
 
 // Shared memory (dynamic part) of k_decode_ix: the gather tile's digit
-// words, kGt + 8 per stream.
+// words, kGt + 16 per stream.
 template <int kGt, int kK>
 constexpr size_t ix_smem_bytes() {
-  return (size_t)kK * (kGt + 8) * sizeof(uint16_t);
+  return (size_t)kK * (kGt + 16) * sizeof(uint16_t);
 }
 
 // Add k (2 <= k <= kK) indexed streams, in stream order, into acc by gather
@@ -1215,14 +1358,15 @@ constexpr size_t ix_smem_bytes() {
 template <int kGt, int kK>
 __global__ void __launch_bounds__(kDThreads, 6) k_decode_ix(const IxArgs a) {
   extern __shared__ __align__(16) uint8_t dyn_s[];
-  __shared__ float4 pat[256];
+  __shared__ float2 pair[16];
   __shared__ uint16_t lut[256];
   __shared__ GatherSmem<kK> gsm;
   __shared__ GStream gs[kK];
   __shared__ int na_s;
   __shared__ uint32_t tile_s;
   fill_lut(lut);
-  fill_patterns(pat);
+  fill_pairs(pair);
+  pdl_enter();
   if (threadIdx.x == 0) {
     // the valid streams, in stream order
     int na = 0;
@@ -1253,7 +1397,7 @@ __global__ void __launch_bounds__(kDThreads, 6) k_decode_ix(const IxArgs a) {
     __syncthreads();
     const uint32_t t = tile_s;
     if (t >= n_tiles) break;
-    gather_tile<kGt, kK>(gs, na, (uint64_t)t * kGt, a.groups, a.n, a.y, a.vec, lut, pat,
+    gather_tile<kGt, kK>(gs, na, (uint64_t)t * kGt, a.groups, a.n, a.y, a.vec, lut, pair,
                          reinterpret_cast<uint16_t *>(dyn_s), gsm);
   }
 }
@@ -1272,8 +1416,7 @@ struct BatchDecodeArgs {
   uint32_t max_polls;
   uint32_t *loc;                // indexed plans: units' first groups in their chunk,
   uint32_t *cpre;               // chunks' first groups (d_chunks + 1 per tensor),
-  uint32_t *done;               // per-tensor finished chunks and
-  uint32_t *ok;                 // valid flags (both zero at launch)
+  uint32_t *ok;                 // valid flags (written by the scan)
   uint32_t n_chunks;            // chunks of all tensors (upper bound)
 };
 
@@ -1282,7 +1425,7 @@ constexpr uint32_t kSmemSearch = 2048;  // tensors whose first tiles fit in shar
 
 // One block: validate every tensor's stream once, and number the tiles that
 // actually exist (ceil(m / tile_bytes) per stream, none for a corrupt one)
-// consecutively, tensor by tensor; the same for the index's 32-unit chunks.
+// consecutively, tensor by tensor; the same for the index's 64-unit chunks.
 // total[0] = tiles, total[1] = chunks.
 __global__ void __launch_bounds__(kPrepThreads)
 k_decode_batch_prepare(const BatchTensor *__restrict__ tensors, uint32_t count,
@@ -1290,6 +1433,7 @@ k_decode_batch_prepare(const BatchTensor *__restrict__ tensors, uint32_t count,
                        uint32_t tile_bytes, BatchPrep *__restrict__ prep,
                        uint32_t *__restrict__ total, int32_t *dev_status) {
   __shared__ uint32_t scan_s[kPrepThreads / kWarp + 1];
+  pdl_enter();
   uint32_t base = 0, cbase = 0;
   for (uint32_t c0 = 0; c0 < count; c0 += kPrepThreads) {
     const uint32_t i = c0 + threadIdx.x;
@@ -1316,7 +1460,7 @@ k_decode_batch_prepare(const BatchTensor *__restrict__ tensors, uint32_t count,
       p.scale = scale;
       p.act_begin = base + off;
       p.cact_begin = cbase + coff;
-      p.pad = 0;
+      p.valid = m > 0 ? 1u : 0u;
       prep[i] = p;
     }
     base += sum;
@@ -1353,6 +1497,7 @@ __global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArg
   __shared__ uint32_t begin_s[kSmemSearch];
   __shared__ uint32_t tile_s;
   fill_lut(sm.lut);
+  pdl_enter();
   const bool in_smem = a.count <= kSmemSearch;
   if (in_smem)
     for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads) begin_s[i] = a.prep[i].act_begin;
@@ -1379,11 +1524,12 @@ __global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArg
   }
 }
 
-// Index of a plan's streams: the chunks that exist, numbered tensor by
+// Count of a plan's streams: the chunks that exist, numbered tensor by
 // tensor by the prepare kernel; block b takes chunks b, b + grid, ...
-__global__ void __launch_bounds__(kDThreads, 8) k_decode_batch_index(const BatchDecodeArgs a) {
+__global__ void __launch_bounds__(kDThreads, 4) k_index_count_batch(const BatchDecodeArgs a) {
   __shared__ uint32_t begin_s[kSmemSearch];
-  __shared__ IndexSmem sm;
+  __shared__ uint32_t wtot_s[kDWarps];
+  pdl_enter();
   const bool in_smem = a.count <= kSmemSearch;
   if (in_smem)
     for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads) begin_s[i] = a.prep[i].cact_begin;
@@ -1393,10 +1539,25 @@ __global__ void __launch_bounds__(kDThreads, 8) k_decode_batch_index(const Batch
     const uint32_t id = find_tensor(begin_s, in_smem, a.prep, a.count, g, true);
     const BatchTensor &T = a.tensors[id];
     const BatchPrep &P = a.prep[id];
-    const uint32_t n_chunks = chunks_of(P.m);
-    const IndexOut io = {a.arena + T.arena_off + 4, P.m, T.groups, a.loc + T.d_tile_begin,
-                         a.cpre + T.d_chunk_begin + id, nullptr, a.done + id, a.ok + id};
-    index_chunk(io, g - P.cact_begin, n_chunks, sm, a.dev_status);
+    count_chunk(a.arena + T.arena_off + 4, P.m, g - P.cact_begin, a.loc + T.d_tile_begin,
+                a.cpre + T.d_chunk_begin + id, wtot_s);
+  }
+}
+
+// Scan of a plan's streams: block b takes tensors b, b + grid, ...; a
+// tensor whose stream the prepare kernel found corrupt gets ok = 0.
+__global__ void __launch_bounds__(kDThreads) k_index_scan_batch(const BatchDecodeArgs a) {
+  __shared__ uint64_t wsum[kDWarps + 1];
+  pdl_enter();
+  for (uint32_t id = blockIdx.x; id < a.count; id += gridDim.x) {
+    const BatchTensor &T = a.tensors[id];
+    const BatchPrep &P = a.prep[id];
+    if (!P.valid) {
+      if (threadIdx.x == 0) a.ok[id] = 0u;
+      continue;
+    }
+    const IndexOut io = {a.cpre + T.d_chunk_begin + id, nullptr, a.ok + id, T.groups};
+    scan_chunks<kDThreads>(io, chunks_of(P.m), wsum, a.dev_status);
   }
 }
 
@@ -1404,11 +1565,13 @@ __global__ void __launch_bounds__(kDThreads, 8) k_decode_batch_index(const Batch
 // the prepare kernel), one warp per unit as in k_decode_units; a tensor the
 // index did not mark valid is left out.
 template <int kMode>
-__global__ void __launch_bounds__(kDThreads, 8) k_decode_batch_units(const BatchDecodeArgs a) {
+__global__ void __launch_bounds__(kDThreads, units_min_blocks<kMode>(true))
+    k_decode_batch_units(const BatchDecodeArgs a) {
   __shared__ UnitSmem sm;
   __shared__ uint32_t begin_s[kSmemSearch];
   __shared__ DecodeJob jobs[kDWarps];  // each warp's current tensor
   fill_unit_tables(sm);
+  pdl_enter();
   const bool in_smem = a.count <= kSmemSearch;
   if (in_smem)
     for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads) begin_s[i] = a.prep[i].act_begin;
@@ -1442,7 +1605,7 @@ __global__ void __launch_bounds__(kDThreads, 8) k_decode_batch_units(const Batch
       __syncwarp();
       cur = id;
     }
-    decode_unit<kMode>(j, gu - first, sm.d.lut, sm.pat, sm.wd[warp]);
+    decode_unit<kMode>(j, gu - first, sm.d.lut, sm.pair, sm.wd[warp]);
   }
 }
 
@@ -1492,7 +1655,7 @@ static cudaError_t launch_one(const DeviceInfo &dev, const DecodeArgs &a, uint32
   const int occ = kMode == kWrite ? dev.occ_decode_write : dev.occ_decode_acc;
   const int kind = kMode == kWrite ? kKindDecodeWrite : kKindDecodeAccumulate;
   timing_begin(kind, stream);
-  k_decode<kMode, kVec><<<persistent_grid(dev, occ, tiles), kDThreads, smem, stream>>>(a);
+  launch_k(k_decode<kMode, kVec>, persistent_grid(dev, occ, tiles), kDThreads, smem, stream, a);
   timing_end(kind, stream);
   return cudaGetLastError();
 }
@@ -1523,17 +1686,16 @@ cudaError_t launch_decode(const DeviceInfo &dev, const uint8_t *in, const uint64
 }
 
 // ---- indexed decode of up to kIndexPass streams --------------------------
-// Scratch: [ticket2, ok[kIndexPass], done[kIndexPass]] (cleared before each
-// launch pair), then each stream's loc[] (one word per unit of its
-// capacity), cpre[] (one per chunk, plus the total) and, for two streams or
-// more, page[] (one per 1024 groups).
-static size_t ix_head_bytes() { return align_up(4 + 8 * kIndexPass, 256); }
+// Scratch: [ticket2, ok[kIndexPass]] (written by the scan), then each
+// stream's loc[] (one word per unit of its capacity), cpre[] (one per chunk,
+// plus the total) and, for two streams or more, page[] (one per 1024
+// groups).
+static size_t ix_head_bytes() { return align_up(4 + 4 * kIndexPass, 256); }
 
 IndexedLayout indexed_layout(const IndexedStream *s, int k, uint64_t n) {
   IndexedLayout L = {};
   const uint64_t groups = (n + 4) / 5;
-  L.zero_bytes = ix_head_bytes();
-  size_t at = L.zero_bytes;
+  size_t at = ix_head_bytes();
   for (int i = 0; i < k; ++i) {
     const uint32_t units = decode_tiles_max(s[i].cap, groups);
     const uint32_t chunks = (units + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
@@ -1577,7 +1739,7 @@ static cudaError_t launch_ix(const DeviceInfo &dev, const IxArgs &a, int occ_slo
   const uint32_t grid =
       persistent_grid(dev, dev.occ_decode_ix[occ_slot], (a.groups + kGt - 1) / kGt);
   timing_begin(kKindDecodeAccumulate, stream);
-  k_decode_ix<kGt, kK><<<grid, kDThreads, smem, stream>>>(a);
+  launch_k(k_decode_ix<kGt, kK>, grid, kDThreads, smem, stream, a);
   timing_end(kKindDecodeAccumulate, stream);
   return cudaGetLastError();
 }
@@ -1589,15 +1751,12 @@ cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s,
   if (k < 1 || k > kIndexPass || (!accumulate && k != 1)) return cudaErrorInvalidValue;
   const IndexedLayout L = indexed_layout(s, k, n);
   char *base = static_cast<char *>(scratch);
-  cudaError_t e = cudaMemsetAsync(scratch, 0, L.zero_bytes, stream);
-  if (e != cudaSuccess) return e;
   IxArgs a;
   a.k = k;
   a.n = n;
   a.groups = (n + 4) / 5;
   a.ticket2 = reinterpret_cast<uint32_t *>(base);
   a.ok = reinterpret_cast<uint32_t *>(base + 4);
-  a.done = reinterpret_cast<uint32_t *>(base + 4 + 4 * kIndexPass);
   a.y = y;
   a.vec = (reinterpret_cast<uintptr_t>(y) & 15) == 0;
   a.dev_status = dev_status;
@@ -1619,9 +1778,10 @@ cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s,
     }
   }
   timing_begin(kKindDecodeCount, stream);
-  k_decode_index<<<persistent_grid(dev, 6, chunks), kDThreads, 0, stream>>>(a);
+  launch_k(k_index_count, persistent_grid(dev, 4, chunks), kDThreads, 0, stream, a);
+  launch_k(k_index_scan, k, kScanThreads, 0, stream, a);
   timing_end(kKindDecodeCount, stream);
-  e = cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (k == 1) {
     // one warp per 512-byte unit
@@ -1630,9 +1790,9 @@ cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s,
                                           (units_max + kDWarps - 1) / kDWarps);
     timing_begin(kind, stream);
     if (accumulate)
-      k_decode_units<kAccumulate><<<grid, kDThreads, 0, stream>>>(a);
+      launch_k(k_decode_units<kAccumulate>, grid, kDThreads, 0, stream, a);
     else
-      k_decode_units<kWrite><<<grid, kDThreads, 0, stream>>>(a);
+      launch_k(k_decode_units<kWrite>, grid, kDThreads, 0, stream, a);
     timing_end(kind, stream);
     return cudaGetLastError();
   }
@@ -1650,18 +1810,19 @@ static cudaError_t launch_batch_one(const DeviceInfo &dev, const BatchDecodeArgs
     const size_t smem = decode_smem_bytes(kMode == kAccumulate);
     const int occ = kMode == kWrite ? dev.occ_decode_batch_write : dev.occ_decode_batch_acc;
     timing_begin(kind, stream);
-    k_decode_batch<kMode><<<persistent_grid(dev, occ, a.n_tiles), kDThreads, smem, stream>>>(a);
+    launch_k(k_decode_batch<kMode>, persistent_grid(dev, occ, a.n_tiles), kDThreads, smem, stream,
+             a);
     timing_end(kind, stream);
     return cudaGetLastError();
   }
   timing_begin(kKindDecodeCount, stream);
-  k_decode_batch_index<<<persistent_grid(dev, 8, a.n_chunks), kDThreads, 0, stream>>>(a);
+  launch_k(k_index_count_batch, persistent_grid(dev, 4, a.n_chunks), kDThreads, 0, stream, a);
+  launch_k(k_index_scan_batch, persistent_grid(dev, 8, a.count), kDThreads, 0, stream, a);
   timing_end(kKindDecodeCount, stream);
   const int occ = kMode == kWrite ? dev.occ_decode_batch_ix_write : dev.occ_decode_batch_ix_acc;
   timing_begin(kind, stream);
-  k_decode_batch_units<kMode>
-      <<<persistent_grid(dev, occ, (a.n_tiles + kDWarps - 1) / kDWarps), kDThreads, 0, stream>>>(
-          a);
+  launch_k(k_decode_batch_units<kMode>,
+           persistent_grid(dev, occ, (a.n_tiles + kDWarps - 1) / kDWarps), kDThreads, 0, stream, a);
   timing_end(kind, stream);
   return cudaGetLastError();
 }
@@ -1670,13 +1831,17 @@ cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
                                 const uint8_t *arena, const uint64_t *in_lens, bool accumulate,
                                 int32_t *dev_status, uint32_t max_polls, cudaStream_t stream) {
   const bool indexed = decode_deferred(p.n_d_tiles);
-  cudaError_t e = cudaMemsetAsync(p.d_zero_base, 0, p.d_zero_bytes, stream);
-  if (e != cudaSuccess) return e;
+  cudaError_t e = cudaSuccess;
+  if (!indexed) {
+    // the ticket and the look-back words (an indexed plan's scan writes
+    // its valid flags, and its units need no ticket)
+    e = cudaMemsetAsync(p.d_zero_base, 0, p.d_zero_bytes, stream);
+    if (e != cudaSuccess) return e;
+  }
   timing_begin(kKindDecodePrepare, stream);
-  k_decode_batch_prepare<<<1, kPrepThreads, 0, stream>>>(
-      p.tensors, p.count, arena, in_lens,
-      indexed ? kDecodeUnit : decode_tile_payload_bytes(accumulate), p.d_prep, p.d_total,
-      dev_status);
+  launch_k(k_decode_batch_prepare, 1, kPrepThreads, 0, stream, p.tensors, p.count, arena, in_lens,
+           indexed ? kDecodeUnit : decode_tile_payload_bytes(accumulate), p.d_prep, p.d_total,
+           dev_status);
   timing_end(kKindDecodePrepare, stream);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1693,7 +1858,6 @@ cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
   a.max_polls = max_polls;
   a.loc = p.d_loc;
   a.cpre = p.d_cpre;
-  a.done = p.d_done;
   a.ok = p.d_ok;
   a.n_chunks = p.n_d_chunks;
   return accumulate ? launch_batch_one<kAccumulate>(dev, a, indexed, stream)

@@ -37,6 +37,25 @@ __device__ __forceinline__ void st_relaxed_u64(uint64_t *p, uint64_t v) {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the library is launched
+// (launch_k) so that it may begin while the kernel before it on the stream
+// is finishing.  Each kernel therefore calls pdl_wait() in every block
+// before its first access to global memory (it returns once the previous
+// grid has completed and its writes are visible; a kernel that ran without
+// the overlap returns at once), and then pdl_trigger() to let the next
+// kernel's blocks be placed as soon as all of its own blocks have started.
+// Only shared memory may be touched before pdl_wait().
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_trigger();
+}
+
+// ---------------------------------------------------------------------------
 // Debug build (compiled with -DTLC_DEBUG; build.py --debug makes
 // libtlc_debug.so).  Bounds checks that never fault: a failing check records
 // its location (source line | translation unit << 16) in this translation

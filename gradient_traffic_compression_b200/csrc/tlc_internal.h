@@ -5,6 +5,7 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <utility>
 
 namespace tlc {
 
@@ -108,7 +109,7 @@ struct BatchTensor {
   uint32_t q_chunk_begin;          // 32-tile chunks of the deferred placement
   uint32_t d_tile_begin, d_tiles;  // decode 512-byte units (global numbering, upper
                                    // bound of the tiles of either mode)
-  uint32_t d_chunk_begin, d_chunks;  // 32-unit chunks of the index (same)
+  uint32_t d_chunk_begin, d_chunks;  // 64-unit chunks of the index (same)
   uint32_t vec_q;        // x and err 16-byte aligned
   uint32_t vec_y;        // y 16-byte aligned
 };
@@ -119,7 +120,7 @@ struct BatchPrep {
   float scale;
   uint32_t act_begin;    // first tile in the compact numbering
   uint32_t cact_begin;   // first index chunk in the compact numbering
-  uint32_t pad;
+  uint32_t valid;        // the stream's length and header are valid
 };
 
 struct BatchChunk {
@@ -145,9 +146,9 @@ struct BatchPlanDev {
   size_t q_zero_bytes;
   uint32_t *d_ticket;
   uint32_t *d_ok;         // indexed plans: per-tensor valid flags
-  uint32_t *d_done;       // indexed plans: per-tensor finished index chunks
   uint64_t *d_status;     // small plans: look-back words, one per unit
-  void *d_zero_base;      // d_ticket, d_ok, d_done and d_status, contiguous
+  void *d_zero_base;      // d_ticket, d_ok and d_status, contiguous (small plans
+                          // clear them before each decode)
   size_t d_zero_bytes;
   BatchPrep *d_prep;      // count entries, rewritten by every decode call
   uint32_t *d_total;      // compact tile and chunk counts of the current decode call
@@ -181,6 +182,25 @@ uint32_t wait_limit();
 // Kernel kinds for the optional per-launch timing (see tlc_kernel_timing).
 enum KernelKind { kKindAbsmax = 0, kKindQuantZre, kKindDecodeWrite, kKindDecodeAccumulate,
                   kKindZrePlace, kKindDecodeCount, kKindDecodePrepare, kKindCount };
+// Launch a kernel that may overlap the end of the kernel before it on the
+// stream (programmatic stream serialization); the kernel waits for that
+// kernel's completion itself (pdl_wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                            cudaStream_t stream, Args &&...args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 void timing_begin(int kind, cudaStream_t stream);
 void timing_end(int kind, cudaStream_t stream);
 
@@ -210,7 +230,7 @@ int occupancy_quant(bool vec);
 // sums of several streams, go through the index instead
 // (launch_decode_indexed).
 constexpr uint32_t kDecodeUnit = 512;
-constexpr uint32_t kDecodeChunkUnits = 32;
+constexpr uint32_t kDecodeChunkUnits = 64;
 uint32_t decode_tiles_max(uint64_t cap, uint64_t groups);
 bool decode_deferred(uint32_t tiles);
 inline size_t decode_scratch_words(uint32_t tiles) { return (size_t)tiles + 1; }
@@ -220,11 +240,10 @@ cudaError_t launch_decode(const DeviceInfo &dev, const uint8_t *in, const uint64
                           int32_t *dev_status, uint32_t max_polls, uint64_t *scratch,
                           cudaStream_t stream);
 
-// Indexed decode of up to kIndexPass streams of n values each: one index
-// launch and one decode launch (dense output: exactly one stream;
-// accumulate: the streams added in order).  The scratch is
-// indexed_layout(..).total_bytes bytes; the launcher clears its first
-// zero_bytes itself.
+// Indexed decode of up to kIndexPass streams of n values each: the index
+// (a count and a scan launch) and one decode launch (dense output: exactly
+// one stream; accumulate: the streams added in order).  The scratch is
+// indexed_layout(..).total_bytes bytes; nothing in it needs clearing.
 constexpr int kIndexPass = 8;
 struct IndexedStream {
   const uint8_t *in;
@@ -233,7 +252,7 @@ struct IndexedStream {
 };
 struct IndexedLayout {
   size_t loc_off[kIndexPass], cpre_off[kIndexPass], page_off[kIndexPass];
-  size_t zero_bytes, total_bytes;
+  size_t total_bytes;
 };
 IndexedLayout indexed_layout(const IndexedStream *s, int k, uint64_t n);
 cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s, int k, uint64_t n,

@@ -165,6 +165,27 @@ def test_indexed_decode_tile_edges(g, extra_groups):
         assert rc_o == rc_g == 0 and np.array_equal(bits(a_g), bits(a_o))
 
 
+CHUNK_BYTES = 64 * 512   # payload bytes of one index chunk (64 units)
+
+
+@pytest.mark.parametrize("extra_bytes", [0, 1, 511, 512, CHUNK_BYTES - 1, CHUNK_BYTES + 513])
+def test_indexed_decode_whole_chunks(g, extra_bytes):
+    # all-literal payloads (one group per byte) of a whole number of index
+    # chunks (INDEX_MIN_GROUPS bytes is 256 of them), and just past one
+    groups = INDEX_MIN_GROUPS + extra_bytes
+    n = 5 * groups
+    st = synth_stream(950 + extra_bytes, n, 1.0)
+    assert st.size - 4 == groups
+    rc_o, y_o = oracle.decompress(st, n)
+    rc_g, y_g = decompress(g, st, n, cap=g.tlc_compress_bound(n))
+    assert rc_o == rc_g == 0 and np.array_equal(bits(y_g), bits(y_o))
+    acc0 = synth.normal(synth.key_for(951, extra_bytes), n, 1.0)
+    st2 = synth_stream(952 + extra_bytes, n, 6.0)
+    rc_o, a_o = oracle.decompress_accumulate([st, st2], n, acc0)
+    rc_g, a_g = accumulate(g, [st, st2], n, acc0)
+    assert rc_o == rc_g == 0 and np.array_equal(bits(a_g), bits(a_o))
+
+
 @pytest.mark.parametrize("in_offset", [1, 3, 12])
 def test_indexed_decode_unaligned_payload(g, in_offset):
     n = LARGE_N + 77
