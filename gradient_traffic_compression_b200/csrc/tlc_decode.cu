@@ -23,21 +23,22 @@
 //                   each unit's first group relative to its chunk (loc[u])
 //                   and the chunk's group count.
 //   k_index_scan    one block per stream: the chunk counts scanned into each
-//                   chunk's first group (cpre[c]), the check that the stream
-//                   expands to exactly ceil(n/5) groups (its valid flag),
-//                   and, for sums of several streams, for every 1024th group
-//                   the chunk that holds it (page[p]).
+//                   chunk's first group (cpre[c]) and the check that the
+//                   stream expands to exactly ceil(n/5) groups (its valid
+//                   flag); for sums of several streams the same for the
+//                   non-zero literal groups ("entries").
 //   k_decode_units  one stream: one warp per 512-byte unit, first group
-//                   cpre[u / 32] + loc[u]; the unit's groups are expanded in
+//                   cpre[u / 64] + loc[u]; the unit's groups are expanded in
 //                   the warp's shared memory and written (or added) as
-//                   coalesced float4s, each from a table of the 81 sign
-//                   patterns of four digits times the scale.
-//   k_decode_ix     2..8 streams: output tiles of a fixed number of groups;
-//                   per stream, the tile's first unit from page[] and loc[],
-//                   one warp per unit places the literal groups in shared
-//                   memory, then each float4 of acc is read once, the
-//                   streams' non-zero values added in stream order, and
-//                   written once.
+//                   coalesced float4s from a table of two-digit value pairs.
+//   k_index_entries 2..8 streams: one warp per unit writes the unit's entries
+//                   (tile position and digit word) to the stream's list, in
+//                   group order, and the first entry of every sum tile.
+//   k_apply_entries 2..8 streams: tiles of 4096 groups; each stream's entries
+//                   of the tile go to shared memory with a per-group stream
+//                   mask, then each thread reads a marked group's acc values
+//                   once, adds the streams' values in stream order and
+//                   writes them once.
 // The quartic bytes live only in shared memory.  Every write is clamped to
 // the ceil(n/5) groups of the tensor; a stream that does not expand to
 // exactly that many groups is reported as corrupt and left out.
@@ -77,13 +78,6 @@ constexpr int kLookV = TLC_D_LOOKV;   // look-back words per lane per round trip
 #define TLC_DEFER_DECODE_MIN_TILES 16384
 #endif
 constexpr uint32_t kDecodeDeferMinTiles = TLC_DEFER_DECODE_MIN_TILES;
-// Output groups per gather tile, summed over its streams (a tile of k
-// streams covers TLC_GT_ACC / k' groups, k' = k rounded up to 2, 4 or 8).
-#ifndef TLC_GT_ACC
-#define TLC_GT_ACC 16384
-#endif
-constexpr uint32_t kPage = 1024;  // groups per page-table entry
-static_assert(TLC_GT_ACC % (8 * kPage) == 0, "tiles are whole pages");
 static_assert(kDecodeUnit == 4 * kWarp * 4, "a unit is 16 bytes per lane of a warp");
 static_assert(kDecodeChunkUnits == 2 * kWarp, "a chunk's units are two per lane of a warp");
 
@@ -222,28 +216,24 @@ __device__ __forceinline__ void fill_lut(uint16_t *lut) {
   for (int v = threadIdx.x; v < 256; v += blockDim.x) lut[v] = v < 243 ? digits_of(v) : 0;
 }
 
-// For every 4-bit word of two digits (2 bits each, first value lowest), the
-// two quantized values q in {-1, 0, +1} as floats; a value is q * scale,
-// which is exact (and +0.0 for q = 0).  Digit 3 never occurs.  The 16
-// entries of 8 bytes fill the 32 banks once, so no pattern of lookups has a
-// bank conflict.
-__device__ __forceinline__ void fill_pairs(float2 *pair) {
-  for (int v = threadIdx.x; v < 16; v += blockDim.x) {
+// A warp's scaled pair table: for every 4-bit word of two digits (2 bits
+// each, first value lowest) the two values q * scale, q in {-1, 0, +1} (each
+// product exact, +0.0 for q = 0; digit 3 never occurs), filled by lanes
+// 0..15.  The 16 entries of 8 bytes fill the 32 banks once, so no pattern
+// of lookups has a bank conflict.
+__device__ __forceinline__ void fill_scaled_pairs(float2 *sp, float scale, int lane) {
+  if (lane < 16) {
     auto q = [](uint32_t d) { return d == 0u ? -1.0f : (d == 2u ? 1.0f : 0.0f); };
-    pair[v] = make_float2(q(v & 3u), q((v >> 2) & 3u));
+    sp[lane] = make_float2(__fmul_rn(q(lane & 3u), scale), __fmul_rn(q((lane >> 2) & 3u), scale));
   }
+  __syncwarp();
 }
-
-// Four values from the 8-bit word p8 of their four digits: the pair table's
-// products with the scale, written or added where the digit is not zero.
-__device__ __forceinline__ float4 pattern4(const float2 *pair, uint32_t p8, float scale) {
-  const float2 a = pair[p8 & 15u], b = pair[p8 >> 4];
-  return make_float4(__fmul_rn(a.x, scale), __fmul_rn(a.y, scale), __fmul_rn(b.x, scale),
-                     __fmul_rn(b.y, scale));
+__device__ __forceinline__ float4 quad(const float2 *sp, uint32_t p8) {
+  const float2 a = sp[p8 & 15u], b = sp[p8 >> 4];
+  return make_float4(a.x, a.y, b.x, b.y);
 }
-__device__ __forceinline__ void add_pattern4(float4 &o, const float2 *pair, uint32_t p8,
-                                             float scale) {
-  const float4 p = pattern4(pair, p8, scale);
+__device__ __forceinline__ void add_quad(float4 &o, const float2 *sp, uint32_t p8) {
+  const float4 p = quad(sp, p8);
   if ((p8 & 3u) != 1u) o.x = __fadd_rn(o.x, p.x);
   if (((p8 >> 2) & 3u) != 1u) o.y = __fadd_rn(o.y, p.y);
   if (((p8 >> 4) & 3u) != 1u) o.z = __fadd_rn(o.z, p.z);
@@ -558,29 +548,25 @@ k_decode(const DecodeArgs a) {
   }
 }
 
-// Values [e_begin, e_end) of the groups whose digit words (lut[] of their
-// quartic bytes) sit in wd at swizzled positions (position 0 is group
-// g_first), by one warp: each aligned float4 is its four digits' pair-table
-// entries times the scale (dense output) or added to acc where a digit is
-// not zero (accumulate, two float4s per lane loaded before either is
-// added); single values at the ends, and everywhere when y is not 16-byte
-// aligned.  Values 4v..4v+3 lie in group g = 4v/5 (digits d0..) and, when
-// d0 >= 2, spill into group g+1; both groups' digit words are joined so one
-// shift lines the four digits up.
-template <int kMode>
-__device__ __forceinline__ void warp_emit(const uint16_t *wd, uint64_t g_first, uint64_t e_begin,
-                                          uint64_t e_end, float *y, bool vec, float scale,
-                                          const float2 *pair, int lane) {
+// Accumulate mode: values [e_begin, e_end) of the groups whose digit words
+// (lut[] of their quartic bytes) sit in wd at swizzled positions counted
+// from group g_first, added into acc by one warp where a digit is not zero:
+// aligned float4s, two per lane loaded before either is added, each from
+// the warp's scaled pair table (sp); single values at the ends, and
+// everywhere when acc is not 16-byte aligned.  Values 4v..4v+3 lie in group
+// g = 4v/5 (digits d0..) and, when d0 >= 2, spill into group g+1; both
+// groups' digit words are joined so one shift lines the four digits up.
+__device__ __forceinline__ void warp_accumulate(const uint16_t *wd, uint64_t g_first,
+                                                uint64_t e_begin, uint64_t e_end, float *y,
+                                                bool vec, float scale, const float2 *sp,
+                                                int lane) {
   if (e_end <= e_begin) return;
   const uint32_t gf = (uint32_t)g_first;
   // n < 2^32, so value and float4 indices fit 32 bits
   auto put = [&](uint32_t e) {
     const uint32_t g = e / 5u;
     const uint32_t dig = (wd[wsw(g - gf)] >> (2 * (e - 5u * g))) & 3u;
-    if (kMode == kWrite)
-      y[e] = dequant(dig, scale);
-    else if (dig != 1u)
-      y[e] = __fadd_rn(y[e], dequant(dig, scale));
+    if (dig != 1u) y[e] = __fadd_rn(y[e], dequant(dig, scale));
   };
   auto digits8 = [&](uint32_t v) -> uint32_t {
     const uint32_t e0 = v << 2;
@@ -595,26 +581,20 @@ __device__ __forceinline__ void warp_emit(const uint16_t *wd, uint64_t g_first, 
     return;
   }
   float4 *y4 = reinterpret_cast<float4 *>(y);
-  if (kMode == kWrite) {
-    // four float4s per lane in flight
-#pragma unroll 4
-    for (uint32_t v = v0 + lane; v < v1; v += kWarp) y4[v] = pattern4(pair, digits8(v), scale);
-  } else {
-    for (uint32_t v = v0 + lane; v < v1; v += 2 * kWarp) {
-      const uint32_t vb = v + kWarp;
-      const uint32_t pa = digits8(v);
-      const uint32_t pb = vb < v1 ? digits8(vb) : 0x55u;
-      float4 oa = make_float4(0.0f, 0.0f, 0.0f, 0.0f), ob = oa;
-      if (pa != 0x55u) oa = y4[v];  // 0x55: four zero digits
-      if (pb != 0x55u) ob = y4[vb];
-      if (pa != 0x55u) {
-        add_pattern4(oa, pair, pa, scale);
-        y4[v] = oa;
-      }
-      if (pb != 0x55u) {
-        add_pattern4(ob, pair, pb, scale);
-        y4[vb] = ob;
-      }
+  for (uint32_t v = v0 + lane; v < v1; v += 2 * kWarp) {
+    const uint32_t vb = v + kWarp;
+    const uint32_t pa = digits8(v);
+    const uint32_t pb = vb < v1 ? digits8(vb) : 0x55u;
+    float4 oa = make_float4(0.0f, 0.0f, 0.0f, 0.0f), ob = oa;
+    if (pa != 0x55u) oa = y4[v];  // 0x55: four zero digits
+    if (pb != 0x55u) ob = y4[vb];
+    if (pa != 0x55u) {
+      add_quad(oa, sp, pa);
+      y4[v] = oa;
+    }
+    if (pb != 0x55u) {
+      add_quad(ob, sp, pb);
+      y4[vb] = ob;
     }
   }
   // the partial float4s at both ends, one value per lane
@@ -623,14 +603,70 @@ __device__ __forceinline__ void warp_emit(const uint16_t *wd, uint64_t g_first, 
     put((uint32_t)lane < h ? (uint32_t)e_begin + lane : 4 * v1 + (lane - h));
 }
 
+// Dense output: the values [5 gb, min(5 (gb + wn), n)) of the groups
+// [gb, gb + wn) whose digit words sit in wd at swizzled positions counted
+// from gb & ~3, by one warp.  Each lane expands one whole batch of four
+// groups 4a .. 4a + 3 (values 20a .. 20a + 19, float4s 5a .. 5a + 4) from one
+// 8-byte read of their digit words (a multiple-of-4 position, so the four
+// words share one aligned block that the swizzle at most swaps by halves)
+// and the warp's scaled pair table, into `stage` (5 * 32 float4s); the warp
+// then writes the staged float4s coalesced.  The values of partial batches
+// at both ends, and every value when y is not 16-byte aligned, go singly.
+constexpr int kStageQuads = 5 * kWarp;
+__device__ __forceinline__ void warp_write(const uint16_t *wd, uint64_t gb, uint32_t wn,
+                                           uint64_t n, float *y, bool vec, float scale,
+                                           const float2 *sp, float4 *stage, int lane) {
+  const uint64_t gal = gb & ~3ull;
+  const uint64_t e_begin = 5 * gb, e_end = umin64(5 * (gb + wn), n);
+  if (e_end <= e_begin) return;
+  auto put = [&](uint64_t e) {
+    const uint64_t g = e / 5;
+    const uint32_t dig = (wd[wsw((uint32_t)(g - gal))] >> (2 * (uint32_t)(e - 5 * g))) & 3u;
+    y[e] = dequant(dig, scale);
+  };
+  const uint64_t a_lo = (gb + 3) / 4, a_hi = umin64((gb + wn) / 4, n / 20);
+  if (!vec || a_hi <= a_lo) {
+    for (uint64_t e = e_begin + lane; e < e_end; e += kWarp) put(e);
+    return;
+  }
+  // the partial batches' values: at most 15 at the start and 19 at the end
+  const uint32_t h = (uint32_t)(20 * a_lo - e_begin), t = (uint32_t)(e_end - 20 * a_hi);
+  for (uint32_t i = lane; i < h + t; i += kWarp) put(i < h ? e_begin + i : 20 * a_hi + (i - h));
+  float4 *y4 = reinterpret_cast<float4 *>(y);
+  const uint32_t p_lo = (uint32_t)(4 * a_lo - gal);  // window position of batch a_lo
+  for (uint64_t a = a_lo; a < a_hi; a += kWarp) {
+    const uint32_t nb = (uint32_t)umin64(kWarp, a_hi - a);
+    if ((uint32_t)lane < nb) {
+      const uint32_t q = wsw(p_lo + 4 * (uint32_t)(a - a_lo) + 4 * lane);
+      const uint2 dw = *reinterpret_cast<const uint2 *>(wd + (q & ~3u));
+      const uint32_t h0 = (q & 2u) ? dw.y : dw.x;  // words of groups 4a, 4a + 1
+      const uint32_t h1 = (q & 2u) ? dw.x : dw.y;  // and 4a + 2, 4a + 3
+      // the batch's 20 digits, two bits each: 16 in lo, 4 in hi
+      const uint32_t w3 = h1 >> 16;
+      const uint32_t lo = (h0 & 0x3ffu) | ((h0 >> 16) << 10) | ((h1 & 0x3ffu) << 20) | (w3 << 30);
+      const uint32_t hi = w3 >> 2;
+      float4 *sl = stage + 5 * lane;
+      sl[0] = quad(sp, lo & 0xffu);
+      sl[1] = quad(sp, (lo >> 8) & 0xffu);
+      sl[2] = quad(sp, (lo >> 16) & 0xffu);
+      sl[3] = quad(sp, lo >> 24);
+      sl[4] = quad(sp, hi);
+    }
+    __syncwarp();
+    float4 *dst = y4 + 5 * a;
+    for (uint32_t i = lane; i < 5 * nb; i += kWarp) dst[i] = stage[i];
+    __syncwarp();
+  }
+}
+
 // ===================================================================== index
 // The index of one stream: per 512-byte payload unit its first group,
 // counted from the first group of its 64-unit chunk (loc); per chunk its
 // group count, which the scan turns into the chunk's first group (cpre;
-// cpre[n_chunks] is then the stream's total); and, for sums of several
-// streams, per page of kPage groups the chunk holding the page's first
-// group.  Two kernels: the count (one block per chunk, eight units per
-// warp; no block waits on another) and the scan (one block per stream).
+// cpre[n_chunks] is then the stream's total).  For sums of several streams
+// the same for the non-zero literal groups ("entries": eloc, ecpre).  Two
+// kernels: the count (one block per chunk, eight units per warp; no block
+// waits on another) and the scan (one block per stream).
 
 static_assert(kDecodeUnit == 4 * 4 * kWarp, "a unit is four 32-bit words per lane");
 constexpr uint32_t kWarpUnits = 8;  // units one warp of the count takes
@@ -643,8 +679,12 @@ static_assert(kDecodeChunkUnits == kDWarps * kWarpUnits, "a chunk is one count b
 // (k < 4) of the unit, so every load is one coalesced 128-byte line; the
 // payload's last unit, and every unit of an unaligned payload, byte by byte
 // (lane L: bytes 16L .. 16L + 15).
-__device__ __forceinline__ uint32_t count_units8(const uint8_t *payload, uint64_t m, uint64_t u0) {
+// With kEnt, ent_out gets the same for the unit's non-zero literal groups.
+template <bool kEnt>
+__device__ __forceinline__ uint32_t count_units8(const uint8_t *payload, uint64_t m, uint64_t u0,
+                                                 uint32_t &ent_out) {
   const uint32_t lane = threadIdx.x & 31;
+  ent_out = 0u;
   if (u0 * kDecodeUnit >= m) return 0u;
   const uint64_t whole = m / kDecodeUnit - u0;  // units of this warp wholly inside (>= 0)
   const uint32_t n_word = (reinterpret_cast<uintptr_t>(payload) & 3) == 0
@@ -679,19 +719,31 @@ __device__ __forceinline__ uint32_t count_units8(const uint8_t *payload, uint64_
       }
     }
   }
-  // a unit expands to at most 512 * 14 < 2^16 groups: two units per word
-  uint32_t pk[kWarpUnits / 2];
+  // a unit expands to at most 512 * 14 < 2^16 groups and has at most 512
+  // entries: two units per word, both counts from one pass over the words
+  uint32_t pk[kWarpUnits / 2], pe[kWarpUnits / 2];
 #pragma unroll
-  for (uint32_t i = 0; i < kWarpUnits / 2; ++i)
-    pk[i] = __reduce_add_sync(0xffffffffu,
-                              expansion16(w[2 * i]) | (expansion16(w[2 * i + 1]) << 16));
+  for (uint32_t i = 0; i < kWarpUnits / 2; ++i) {
+    pk[i] = expansion16(w[2 * i]) | (expansion16(w[2 * i + 1]) << 16);
+    if (kEnt) pe[i] = literals16(w[2 * i]) | (literals16(w[2 * i + 1]) << 16);
+  }
+#pragma unroll
+  for (uint32_t i = 0; i < kWarpUnits / 2; ++i) {
+    pk[i] = __reduce_add_sync(0xffffffffu, pk[i]);
+    if (kEnt) pe[i] = __reduce_add_sync(0xffffffffu, pe[i]);
+  }
   const uint32_t h = (lane >> 1) & 3u;
   const uint32_t v = h == 0 ? pk[0] : (h == 1 ? pk[1] : (h == 2 ? pk[2] : pk[3]));
   uint32_t mine = lane < kWarpUnits ? ((lane & 1u) ? v >> 16 : v & 0xffffu) : 0u;
-  // the padding bytes past the payload counted one group each
+  // the padding bytes past the payload counted one group each (and, being
+  // 121, no entry)
   if (lane < kWarpUnits) {
     const uint64_t ub = (u0 + lane) * kDecodeUnit;
     mine -= (uint32_t)(ub >= m ? kDecodeUnit : (ub + kDecodeUnit > m ? ub + kDecodeUnit - m : 0));
+  }
+  if (kEnt) {
+    const uint32_t ve = h == 0 ? pe[0] : (h == 1 ? pe[1] : (h == 2 ? pe[2] : pe[3]));
+    ent_out = lane < kWarpUnits ? ((lane & 1u) ? ve >> 16 : ve & 0xffffu) : 0u;
   }
   return mine;
 }
@@ -699,44 +751,64 @@ __device__ __forceinline__ uint32_t count_units8(const uint8_t *payload, uint64_
 // Chunk c (64 units) of a stream's payload of m bytes, by one block: warp w
 // counts units 8w .. 8w + 7; loc[u] = the unit's first group counted from
 // the chunk's first, cnt[c] = the chunk's group count (at most
-// 64 * 512 * 14).  wtot_s holds kDWarps words.  Ends synchronised.
+// 64 * 512 * 14); with kEnt the same for entries in eloc and ecnt.
+// wtot_s holds 2 * kDWarps words.  Ends synchronised.
+__device__ __forceinline__ uint32_t scan8(uint32_t x, uint32_t lane) {
+#pragma unroll
+  for (uint32_t d = 1; d < kWarpUnits; d <<= 1) {
+    const uint32_t t = __shfl_up_sync(0xffffffffu, x, d);
+    if (lane >= d) x += t;
+  }
+  return x;
+}
+template <bool kEnt>
 __device__ __forceinline__ void count_chunk(const uint8_t *payload, uint64_t m, uint32_t c,
-                                            uint32_t *loc, uint32_t *cnt, uint32_t *wtot_s) {
+                                            uint32_t *loc, uint32_t *cnt, uint32_t *eloc,
+                                            uint32_t *ecnt, uint32_t *wtot_s) {
   const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint64_t n_units = (m + kDecodeUnit - 1) / kDecodeUnit;
   const uint64_t u0 = (uint64_t)c * kDecodeChunkUnits + warp * kWarpUnits;
-  const uint32_t mine = count_units8(payload, m, u0);
-  uint32_t inc = mine;
-#pragma unroll
-  for (uint32_t d = 1; d < kWarpUnits; d <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
-    if (lane >= d) inc += t;
+  uint32_t ent = 0;
+  const uint32_t mine = count_units8<kEnt>(payload, m, u0, ent);
+  const uint32_t inc = scan8(mine, lane), einc = scan8(ent, lane);
+  if (lane == kWarpUnits - 1) {
+    wtot_s[warp] = inc;
+    wtot_s[kDWarps + warp] = einc;
   }
-  if (lane == kWarpUnits - 1) wtot_s[warp] = inc;
   __syncthreads();
-  uint32_t off = 0;
-  for (uint32_t w = 0; w < warp; ++w) off += wtot_s[w];
-  if (lane < kWarpUnits && u0 + lane < n_units) loc[u0 + lane] = off + inc - mine;
-  if (warp == kDWarps - 1 && lane == kWarpUnits - 1) cnt[c] = off + inc;
+  uint32_t off = 0, eoff = 0;
+  for (uint32_t w = 0; w < warp; ++w) {
+    off += wtot_s[w];
+    eoff += wtot_s[kDWarps + w];
+  }
+  if (lane < kWarpUnits && u0 + lane < n_units) {
+    loc[u0 + lane] = off + inc - mine;
+    if (kEnt) eloc[u0 + lane] = eoff + einc - ent;
+  }
+  if (warp == kDWarps - 1 && lane == kWarpUnits - 1) {
+    cnt[c] = off + inc;
+    if (kEnt) ecnt[c] = eoff + einc;
+  }
   __syncthreads();  // wtot_s is rewritten by the next chunk
 }
 
-// What the scan of one stream writes.
+// What the scan of one array of one stream writes.
 struct IndexOut {
-  uint32_t *cpre;      // chunk counts in, first groups out, then the total
-  uint32_t *page;      // or nullptr: per page, the chunk holding group p * kPage
-  uint32_t *ok;        // 1 when the stream expands to exactly `groups`, else 0
+  uint32_t *cpre;      // chunk counts in, first groups (or entries) out, then the total
+  uint32_t *ok;        // or nullptr: 1 when the stream expands to exactly `groups`, else 0
   uint64_t groups;
+  uint32_t *tail;      // or nullptr: also gets the total
 };
 
 __device__ __forceinline__ uint32_t sat32(uint64_t v) { return (uint32_t)umin64(v, 0xffffffffull); }
 
 // The stream's chunk counts, scanned by one block of kThreads into each
-// chunk's first group, the total checked against the tensor's groups, and
-// the page table.  In passes of up to kScanPer chunks per thread: each
-// thread loads its contiguous share into registers (all loads issued
-// first), then a block scan of the shares (64-bit: a corrupt stream's
-// counts may add up past 2^32).  wsum holds kThreads / 32 + 1 words.
+// chunk's first group (or entry) and the total, checked against the
+// tensor's groups when s.ok is set.  In passes of up to kScanPer chunks per
+// thread: each thread loads its contiguous share into registers (all loads
+// issued first), then a block scan of the shares (64-bit: a corrupt
+// stream's counts may add up past 2^32).  wsum holds kThreads / 32 + 1
+// words.
 constexpr int kScanPer = 8;
 template <int kThreads>
 __device__ void scan_chunks(const IndexOut &s, uint32_t n_chunks, uint64_t *wsum,
@@ -745,8 +817,6 @@ __device__ void scan_chunks(const IndexOut &s, uint32_t n_chunks, uint64_t *wsum
   static_assert(kWarps <= kWarp, "one warp scans the warp sums");
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   uint64_t carry = 0;
-  // each thread a contiguous share of at most kScanPer chunks, as small as
-  // the pass allows (the page-table writes of a share are one thread's)
   for (uint32_t base = 0; base < n_chunks;) {
     const uint32_t per = min((uint32_t)kScanPer, (n_chunks - base + kThreads - 1) / kThreads);
     const uint32_t c0 = base + threadIdx.x * per;
@@ -785,11 +855,6 @@ __device__ void scan_chunks(const IndexOut &s, uint32_t n_chunks, uint64_t *wsum
       const uint32_t c = c0 + i;
       if (c < cend) {
         s.cpre[c] = sat32(run);
-        if (s.page) {
-          const uint64_t pend = umin64(run + v[i], s.groups);
-          for (uint64_t p = (run + kPage - 1) / kPage; p * kPage < pend; ++p)
-            if (TLC_CHECK(p < (s.groups + kPage - 1) / kPage)) s.page[p] = c;
-        }
         run += v[i];
       }
     }
@@ -797,21 +862,27 @@ __device__ void scan_chunks(const IndexOut &s, uint32_t n_chunks, uint64_t *wsum
   }
   if (threadIdx.x == 0) {
     s.cpre[n_chunks] = sat32(carry);
-    const bool ok = carry == s.groups;
-    *s.ok = ok ? 1u : 0u;
-    if (!ok) report(dev_status, TLC_ERR_CORRUPT);
+    if (s.tail) *s.tail = sat32(carry);
+    if (s.ok) {
+      const bool ok = carry == s.groups;
+      *s.ok = ok ? 1u : 0u;
+      if (!ok) report(dev_status, TLC_ERR_CORRUPT);
+    }
   }
 }
 
 // Up to kIndexPass streams of n values each, indexed and decoded by one
-// launch sequence.
+// launch sequence.  The entry arrays are set for sums of several streams.
 struct IxStream {
   const uint8_t *in;
   const uint64_t *len_dev;
   uint64_t cap;
   uint32_t *loc;
   uint32_t *cpre;
-  uint32_t *page;      // nullptr for a single stream
+  uint32_t *eloc;      // or nullptr: units' first entries within their chunk
+  uint32_t *ecpre;     // chunks' first entries, then the total
+  uint32_t *list;      // entries: (group - tile's first) << 16 | digit word, in group order
+  uint32_t *tfe;       // per sum tile: its first entry; tfe[n_tiles] = the total
 };
 struct IxArgs {
   IxStream s[kIndexPass];
@@ -829,14 +900,22 @@ __device__ __forceinline__ uint32_t chunks_of(uint64_t m) {
                     ((uint64_t)kDecodeUnit * kDecodeChunkUnits));
 }
 
-// Count of every stream: the chunks that exist (from each stream's length;
-// none for a corrupt one), numbered stream by stream; block b takes chunks
-// b, b + grid, ...
-__global__ void __launch_bounds__(kDThreads, 4) k_index_count(const IxArgs a) {
-  __shared__ uint64_t m_s[kIndexPass];
-  __shared__ uint32_t pre_s[kIndexPass + 1];
-  __shared__ uint32_t wtot_s[kDWarps];
-  pdl_enter();
+// Groups per tile of a sum of several streams.
+#ifndef TLC_SUM_TILE
+#define TLC_SUM_TILE 4096
+#endif
+constexpr uint32_t kSumTile = TLC_SUM_TILE;
+static_assert(kSumTile % 16 == 0 && kSumTile <= 65536, "a tile position fits 16 bits");
+__host__ __device__ __forceinline__ uint32_t sum_tiles(uint64_t groups) {
+  return (uint32_t)((groups + kSumTile - 1) / kSumTile);
+}
+
+// Valid streams' payload lengths (0 for a corrupt one) into m_s and the
+// running count of their `per(m)` items into pre_s (k + 1 words); whole
+// block, ends synchronised.
+template <typename F>
+__device__ __forceinline__ void stream_prefix(const IxArgs &a, uint64_t *m_s, uint32_t *pre_s,
+                                              F per) {
   if (threadIdx.x < (unsigned)a.k) {
     const IxStream &S = a.s[threadIdx.x];
     uint64_t m = 0;
@@ -846,15 +925,27 @@ __global__ void __launch_bounds__(kDThreads, 4) k_index_count(const IxArgs a) {
   __syncthreads();
   if (threadIdx.x == 0) {
     pre_s[0] = 0;
-    for (int s = 0; s < a.k; ++s) pre_s[s + 1] = pre_s[s] + chunks_of(m_s[s]);
+    for (int s = 0; s < a.k; ++s) pre_s[s + 1] = pre_s[s] + per(m_s[s]);
   }
   __syncthreads();
+}
+
+// Count of every stream: the chunks that exist (from each stream's length;
+// none for a corrupt one), numbered stream by stream; block b takes chunks
+// b, b + grid, ...
+template <bool kEnt>
+__global__ void __launch_bounds__(kDThreads, 4) k_index_count(const IxArgs a) {
+  __shared__ uint64_t m_s[kIndexPass];
+  __shared__ uint32_t pre_s[kIndexPass + 1];
+  __shared__ uint32_t wtot_s[2 * kDWarps];
+  pdl_enter();
+  stream_prefix(a, m_s, pre_s, [](uint64_t m) { return chunks_of(m); });
   const uint32_t total = pre_s[a.k];
   for (uint32_t t = blockIdx.x; t < total; t += gridDim.x) {
     int s = 0;
     while (s + 1 < a.k && pre_s[s + 1] <= t) ++s;
     const IxStream &S = a.s[s];
-    count_chunk(S.in + 4, m_s[s], t - pre_s[s], S.loc, S.cpre, wtot_s);
+    count_chunk<kEnt>(S.in + 4, m_s[s], t - pre_s[s], S.loc, S.cpre, S.eloc, S.ecpre, wtot_s);
   }
 }
 
@@ -883,8 +974,13 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const IxArgs a) {
     }
     return;
   }
-  const IndexOut io = {S.cpre, S.page, a.ok + s, a.groups};
-  scan_chunks<kScanThreads>(io, chunks_of(m_s), wsum, a.dev_status);
+  const uint32_t nc = chunks_of(m_s);
+  const IndexOut io = {S.cpre, a.ok + s, a.groups, nullptr};
+  scan_chunks<kScanThreads>(io, nc, wsum, a.dev_status);
+  if (S.ecpre) {
+    const IndexOut eo = {S.ecpre, nullptr, 0, S.tfe + sum_tiles(a.groups)};
+    scan_chunks<kScanThreads>(eo, nc, wsum, a.dev_status);
+  }
 }
 
 // ============================================================= warp units
@@ -892,7 +988,7 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const IxArgs a) {
 // first group is cpre[u / 32] + loc[u].  Its groups are decoded in windows
 // of kWarpGroups: the window is pre-filled with the zero group's digit word,
 // the unit's literal groups in the window are placed as their digit words
-// (lut[] of the byte) in the warp's own shared memory, and warp_emit writes
+// (lut[] of the byte) in the warp's own shared memory, and warp_write writes
 // (or adds) the window's values; the float4s that straddle a window's or the
 // unit's end become single values.  A unit without non-zero literals is
 // plain zeros (dense output) or nothing (accumulate); an accumulate unit
@@ -910,9 +1006,11 @@ __device__ __forceinline__ uint64_t unit_first_group(const uint32_t *cpre, const
   return (uint64_t)__ldg(cpre + (u / kDecodeChunkUnits)) + __ldg(loc + u);
 }
 
+// One unit by one warp; sp is the warp's scaled pair table (for j's scale),
+// wd its window of digit words, stage its staging for dense output.
 template <int kMode>
 __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, const uint16_t *lut,
-                                            const float2 *pair, uint16_t *wd) {
+                                            const float2 *sp, uint16_t *wd, float4 *stage) {
   const int lane = threadIdx.x & 31;
   const uint64_t base = (uint64_t)u * kDecodeUnit + 16ull * lane;
   uint32_t w[4] = {0u, 0u, 0u, 0u};
@@ -995,9 +1093,13 @@ __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, cons
   }
   for (uint32_t w0 = 0; w0 < Ec; w0 += kWarpGroups) {
     const uint32_t wn = min(kWarpGroups, Ec - w0);
-    // positions 0..wn (the last one read by a float4 that spills), in whole
-    // swizzle blocks of 16
-    for (uint32_t q = lane; q < 2 * (wn / 16 + 1); q += kWarp)
+    // window positions count from the window's first group rounded down to
+    // a multiple of 4: groups at off .. off + wn - 1
+    const uint64_t gb = O + w0;
+    const uint32_t off = (uint32_t)(gb & 3u);
+    // positions 0 .. off + wn (the last one read by a float4 that spills),
+    // in whole swizzle blocks of 16
+    for (uint32_t q = lane; q < 2 * ((off + wn) / 16 + 1); q += kWarp)
       reinterpret_cast<uint4 *>(wd)[q] = make_uint4(kZeroDigits2, kZeroDigits2, kZeroDigits2,
                                                     kZeroDigits2);
     __syncwarp();
@@ -1009,14 +1111,17 @@ __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, cons
         if (b >= 243u) {
           pos += b - 241u;
         } else {
-          if (pos - w0 < wn) wd[wsw(pos - w0)] = lut[b];  // unsigned: pos in [w0, w0 + wn)
+          if (pos - w0 < wn) wd[wsw(pos - w0 + off)] = lut[b];  // unsigned: pos in [w0, w0 + wn)
           ++pos;
         }
       }
     }
     __syncwarp();
-    const uint64_t gb = O + w0;
-    warp_emit<kMode>(wd, gb, 5 * gb, umin64(5 * (gb + wn), j.n), j.y, j.vec, j.scale, pair, lane);
+    if (kMode == kWrite)
+      warp_write(wd, gb, wn, j.n, j.y, j.vec, j.scale, sp, stage, lane);
+    else
+      warp_accumulate(wd, gb - off, 5 * gb, umin64(5 * (gb + wn), j.n), j.y, j.vec, j.scale, sp,
+                      lane);
     __syncwarp();
   }
 }
@@ -1027,18 +1132,22 @@ __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, cons
 #define TLC_SPARSE_EXPANSION 4
 #endif
 
-// Shared memory of a block of warp-unit decoders.
+// Shared memory of a block of warp-unit decoders: per warp its scaled pair
+// table, its window of digit words (positions up to kWarpGroups + 3, filled
+// in whole swizzle blocks) and, for dense output, its staging.
+template <int kMode>
 struct UnitSmem {
   DecodeSmem d;   // digit table, block scan, a tile's first group
-  float2 pair[16];
+  float2 sp[kDWarps][16];
   __align__(16) uint16_t wd[kDWarps][kWarpGroups + 16];
+  __align__(16) float4 stage[kMode == kWrite ? kDWarps : 1][kStageQuads];
 };
-static_assert(sizeof(UnitSmem::wd) >= DecodeShape<kWrite>::kMaxGroups + 16,
+static_assert(sizeof(UnitSmem<kWrite>::wd) >= DecodeShape<kWrite>::kMaxGroups + 16,
               "a dense-output payload tile's groups fit the warps' windows");
 
-__device__ __forceinline__ void fill_unit_tables(UnitSmem &sm) {
-  fill_lut(sm.d.lut);
-  fill_pairs(sm.pair);
+template <int kMode>
+__device__ __forceinline__ float4 *unit_stage(UnitSmem<kMode> &sm, int warp) {
+  return sm.stage[kMode == kWrite ? warp : 0];
 }
 
 // One indexed stream (dense output, or added into acc): warp w of block b
@@ -1048,20 +1157,21 @@ __device__ __forceinline__ void fill_unit_tables(UnitSmem &sm) {
 // one long run of zero stores, which a block writes faster than a warp.
 // Blocks per SM the warp-unit kernels are compiled for: the accumulate
 // emit keeps two float4s of acc per lane in flight, and the plan kernel
-// tracks its tensor: both need the registers of 6 blocks.
+// tracks its tensor: both need the registers of 6 blocks.  Dense output
+// runs 5 (its staging's shared memory).
 template <int kMode>
 constexpr int units_min_blocks(bool batch) {
-  return kMode == kWrite && !batch ? 8 : 6;
+  return kMode == kWrite ? 5 : 6;  // dense output: its staging allows 5 blocks
 }
 
 template <int kMode>
 __global__ void __launch_bounds__(kDThreads, units_min_blocks<kMode>(false))
     k_decode_units(const IxArgs a) {
-  __shared__ UnitSmem sm;
+  __shared__ UnitSmem<kMode> sm;
   __shared__ DecodeJob job_s;
   __shared__ int ok_s;
   __shared__ uint32_t tile_s;
-  fill_unit_tables(sm);
+  fill_lut(sm.d.lut);
   pdl_enter();
   if (threadIdx.x == 0) {
     const IxStream &S = a.s[0];
@@ -1099,307 +1209,241 @@ __global__ void __launch_bounds__(kDThreads, units_min_blocks<kMode>(false))
   // the job stays in shared memory: its fields are read where they are used
   const int warp = threadIdx.x >> 5;
   const uint32_t nw = gridDim.x * kDWarps;
+  fill_scaled_pairs(sm.sp[warp], job_s.scale, threadIdx.x & 31);
   for (uint32_t u = blockIdx.x * kDWarps + warp; u < job_s.n_tiles; u += nw)
-    decode_unit<kMode>(job_s, u, sm.d.lut, sm.pair, sm.wd[warp]);
+    decode_unit<kMode>(job_s, u, sm.d.lut, sm.sp[warp], sm.wd[warp], unit_stage(sm, warp));
 }
 
-// ==================================================================== gather
-// A stream as the gather tiles read it.
-struct GStream {
-  const uint8_t *payload;
-  const uint32_t *loc;
-  const uint32_t *cpre;
-  const uint32_t *page;
-  uint64_t m;
-  float scale;
-  uint32_t n_units;
-};
-
-template <int kK>
-struct GatherSmem {
-  uint32_t uf[kK], nu[kK];  // first unit and unit count of each stream in the tile
-  uint32_t lit[kK];         // the stream has a non-zero literal in the tile
-};
-
-// The units of stream S that hold groups ga and gb (each below the
-// stream's groups, or gb = ~0 for the stream's last unit), by one warp: the
-// page gives a group's chunk, the chunk's 64 loc[] entries (two per lane)
-// its unit; both lookups' loads are issued together.  Every lane gets the
-// results.
-__device__ __forceinline__ void units_of_groups(const GStream &S, uint64_t ga, uint64_t gb,
-                                                uint32_t &ua, uint32_t &ub) {
+// ======================================================= sums of streams
+// Entries: one warp per unit of every valid stream (numbered stream by
+// stream).  Lane L takes the unit's bytes 16L .. 16L + 15; warp scans give
+// its first group (cpre + loc) and first entry (ecpre + eloc).  Each
+// non-zero literal group g becomes entry list[e] = (g mod kSumTile) << 16 |
+// its digit word, and every tile boundary b * kSumTile that falls in the
+// lane's groups gets tfe[b] = the index of the first entry at or after it.
+// Units are disjoint runs of groups, so every entry and boundary is written
+// once, and the list is in group order.
+__global__ void __launch_bounds__(kDThreads) k_index_entries(const IxArgs a) {
+  __shared__ uint64_t m_s[kIndexPass];
+  __shared__ uint32_t pre_s[kIndexPass + 1];
+  __shared__ uint16_t lut[256];
+  fill_lut(lut);
+  pdl_enter();
+  stream_prefix(a, m_s, pre_s, [](uint64_t m) {
+    return (uint32_t)((m + kDecodeUnit - 1) / kDecodeUnit);
+  });
+  const uint32_t total = pre_s[a.k];
   const int lane = threadIdx.x & 31;
-  const uint32_t n_chunks = (S.n_units + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
-  const bool last = gb == ~0ull;
-  const uint32_t ca = (uint32_t)umin64(__ldg(S.page + ga / kPage), n_chunks - 1);
-  const uint32_t cb = last ? 0u : (uint32_t)umin64(__ldg(S.page + gb / kPage), n_chunks - 1);
-  const uint64_t pa = __ldg(S.cpre + ca), pb = last ? 0 : __ldg(S.cpre + cb);
-  // the last unit of the chunk whose first group is at most g (loc[] does
-  // not decrease within a chunk)
-  auto find = [&](uint32_t c, uint64_t p, uint64_t g, bool use) -> uint32_t {
-    const uint64_t v0 = (uint64_t)c * kDecodeChunkUnits + lane, v1 = v0 + kWarp;
-    const bool ok0 = use && v0 < S.n_units, ok1 = use && v1 < S.n_units;
-    const uint32_t l0 = ok0 ? __ldg(S.loc + v0) : 0u, l1 = ok1 ? __ldg(S.loc + v1) : 0u;
-    const uint32_t m0 = __ballot_sync(0xffffffffu, ok0 && p + l0 <= g);
-    const uint32_t m1 = __ballot_sync(0xffffffffu, ok1 && p + l1 <= g);
-    return c * kDecodeChunkUnits + (m1 ? kWarp + 31 - __clz(m1) : (m0 ? 31 - __clz(m0) : 0));
-  };
-  ua = find(ca, pa, ga, true);
-  const uint32_t fb = find(cb, pb, gb, !last);
-  ub = last ? S.n_units - 1 : fb;
-}
-
-// One warp: unit u of stream S.  Each lane takes 16 consecutive payload
-// bytes; a warp scan of their expansion counts gives each lane's first
-// group; literal groups that fall in [g0, g0 + gn) go to wd as their digit
-// words (lut[] of the byte), at swizzled positions.  Sets *lit when a literal other than the zero
-// group 121 was placed.
-__device__ __forceinline__ void walk_unit(const GStream &S, uint32_t u, uint64_t g0, uint32_t gn,
-                                          uint16_t *wd, const uint16_t *lut, uint32_t *lit) {
-  const int lane = threadIdx.x & 31;
-  const uint64_t base = (uint64_t)u * kDecodeUnit + 16ull * lane;
-  uint32_t w[4] = {0u, 0u, 0u, 0u};
-  int nb = 0;
-  if (base < S.m) {
-    const uint64_t left = S.m - base;
-    const uint8_t *p = S.payload + base;
-    if (left >= 16 && (reinterpret_cast<uintptr_t>(p) & 3) == 0) {
-      const uint32_t *p32 = reinterpret_cast<const uint32_t *>(p);
+  const uint32_t nw = gridDim.x * kDWarps;
+  for (uint32_t t = blockIdx.x * kDWarps + (threadIdx.x >> 5); t < total; t += nw) {
+    int s = 0;
+    while (s + 1 < a.k && pre_s[s + 1] <= t) ++s;
+    if (!a.ok[s]) continue;  // uniform in the warp
+    const IxStream &S = a.s[s];
+    const uint32_t u = t - pre_s[s];
+    const uint64_t m = m_s[s];
+    const uint8_t *payload = S.in + 4;
+    const uint64_t base = (uint64_t)u * kDecodeUnit + 16ull * lane;
+    uint32_t w[4] = {0x79797979u, 0x79797979u, 0x79797979u, 0x79797979u};
+    int nb = 0;
+    if (base < m) {
+      const uint64_t left = m - base;
+      const uint8_t *p = payload + base;
+      if (left >= 16 && (reinterpret_cast<uintptr_t>(p) & 3) == 0) {
+        const uint32_t *p32 = reinterpret_cast<const uint32_t *>(p);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) w[k] = __ldg(p32 + k);
-      nb = 16;
-    } else {
-      nb = (int)umin64(left, 16);
+        for (int k = 0; k < 4; ++k) w[k] = __ldg(p32 + k);
+        nb = 16;
+      } else {
+        nb = (int)umin64(left, 16);
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        if (k < nb) w[k >> 2] |= (uint32_t)__ldg(p + k) << (8 * (k & 3));
+        for (int k = 0; k < 16; ++k)
+          if (k < nb)
+            w[k >> 2] = (w[k >> 2] & ~(0xffu << (8 * (k & 3)))) |
+                        ((uint32_t)__ldg(p + k) << (8 * (k & 3)));
+      }
     }
-  }
-  const uint64_t first = unit_first_group(S.cpre, S.loc, u);  // loaded with the bytes
-  uint32_t e = 0;
-  if (nb == 16) {
-    e = expansion16(w);
-  } else {
+    const uint32_t c0 = u / kDecodeChunkUnits;
+    const uint64_t g_unit = (uint64_t)__ldg(S.cpre + c0) + __ldg(S.loc + u);
+    const uint64_t e_unit = (uint64_t)__ldg(S.ecpre + c0) + __ldg(S.eloc + u);
+    // padding bytes (past the payload) are literal 121s: one group, no entry
+    const uint32_t eg = nb > 0 ? expansion16(w) - (16u - (uint32_t)nb) : 0u;
+    const uint32_t ee = nb > 0 ? literals16(w) : 0u;
+    uint32_t ig = eg, ie = ee;
 #pragma unroll
-    for (int k = 0; k < 16; ++k)
-      if (k < nb) e += expansion((w[k >> 2] >> (8 * (k & 3))) & 0xffu);
-  }
-  uint32_t inc = e;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const uint32_t t = __shfl_up_sync(0xffffffffu, inc, d);
-    if (lane >= d) inc += t;
-  }
-  uint64_t g = first + (inc - e);
-  const uint64_t ge = g0 + gn;
-  bool mine = false;
-  if (nb > 0 && g < ge && g + e > g0) {
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t tg = __shfl_up_sync(0xffffffffu, ig, d);
+      const uint32_t te = __shfl_up_sync(0xffffffffu, ie, d);
+      if (lane >= d) {
+        ig += tg;
+        ie += te;
+      }
+    }
+    uint64_t g = g_unit + ig - eg;
+    uint32_t e = (uint32_t)(e_unit + ie - ee);
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       if (k < nb) {
         const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
-        if (b < 243u) {
-          if (g >= g0 && g < ge && TLC_CHECK(g - g0 < (uint64_t)gn)) {
-            wd[wsw((uint32_t)(g - g0))] = lut[b];
-            mine = mine || b != 121u;
-          }
-          ++g;
-        } else {
-          g += b - 241u;
+        const uint32_t run = b >= 243u ? b - 241u : 1u;
+        // a tile boundary among this byte's groups [g, g + run) (run < kSumTile)
+        const uint64_t bnd = (g + kSumTile - 1) / kSumTile;
+        if (bnd * kSumTile < g + run && TLC_CHECK(bnd <= sum_tiles(a.groups)))
+          S.tfe[bnd] = e;
+        if (b < 243u && b != 121u) {
+          if (TLC_CHECK(e < m)) S.list[e] = ((uint32_t)(g % kSumTile) << 16) | lut[b];
+          ++e;
         }
+        g += run;
       }
     }
   }
-  if (__any_sync(0xffffffffu, mine) && lane == 0) *lit = 1u;
 }
 
-// One gather tile: output groups [g0, g0 + gn) of k streams (k <= kK, all
-// valid, in stream order) added into acc.  Whole block; ends synchronised.
-// wd holds kK * (kGt + 16) digit words.
-template <int kGt, int kK>
-__device__ __forceinline__ void gather_tile(const GStream *gs, int k, uint64_t g0,
-                                            uint64_t groups, uint64_t n, float *y, bool vec,
-                                            const uint16_t *lut, const float2 *pair, uint16_t *wd,
-                                            GatherSmem<kK> &sm) {
-  static_assert(kGt % kPage == 0 && kGt % 16 == 0 && kK <= kDWarps && kK <= 8, "tile shape");
-  constexpr uint32_t kStride = kGt + 16;  // digit words per stream (one spare swizzle block)
-  constexpr int kPk = (kK + 3) / 4;       // words of four streams' 8-bit digit words
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t gn = (uint32_t)umin64(kGt, groups - g0);
-  // pre-fill positions 0..gn (in whole swizzle blocks) with the zero group's
-  // digit word; warp s finds stream s's units
-  for (int s = 0; s < k; ++s)
-    for (uint32_t w = threadIdx.x; w < 2 * (gn / 16 + 1); w += kDThreads)
-      reinterpret_cast<uint4 *>(wd + s * kStride)[w] =
-          make_uint4(kZeroDigits2, kZeroDigits2, kZeroDigits2, kZeroDigits2);
-  if (warp < k) {
-    const GStream &S = gs[warp];
-    uint32_t uf, ul;
-    units_of_groups(S, g0, g0 + gn < groups ? g0 + gn : ~0ull, uf, ul);
-    if (ul < uf) ul = uf;
-    if (lane == 0) {
-      sm.uf[warp] = uf;
-      sm.nu[warp] = ul - uf + 1;
-      sm.lit[warp] = 0u;
-    }
-  }
-  __syncthreads();
-  // every (stream, unit) pair of the tile, spread over the warps
-  uint32_t items = 0;
-  for (int s = 0; s < k; ++s) items += sm.nu[s];
-  for (uint32_t i = warp; i < items; i += kDWarps) {
-    int s = 0;
-    uint32_t r = i;
-    while (r >= sm.nu[s]) r -= sm.nu[s++];
-    walk_unit(gs[s], sm.uf[s] + r, g0, gn, wd + s * kStride, lut, &sm.lit[s]);
-  }
-  __syncthreads();
-  // one read-modify-write of each float4 of acc: the streams' non-zero
-  // values added in stream order
-  uint32_t act = 0;  // bit s: stream s has a non-zero value in the tile
-#pragma unroll
-  for (int s = 0; s < kK; ++s)
-    if (s < k && sm.lit[s]) act |= 1u << s;
-  if (act) {
-    const uint64_t e_begin = 5 * g0, e_end = umin64(5 * (g0 + gn), n);
-    const uint32_t o32 = (uint32_t)g0;
-    const uint64_t v0 = vec ? (e_begin + 3) / 4 : e_end, v1 = vec ? e_end / 4 : e_end;
-    float4 *y4 = reinterpret_cast<float4 *>(y);
-    // the active streams' four digits of float4 v, eight bits per stream
-    // packed into pk; returns the streams with a non-zero digit
-    auto digits = [&](uint32_t v, uint32_t(&pk)[kPk]) -> uint32_t {
-      const uint32_t e0 = v << 2;
-      const uint32_t g = e0 / 5u;
-      const uint32_t d0 = e0 - 5u * g;
-      const uint32_t ia = wsw(g - o32), ib = wsw(g - o32 + 1);
-      uint32_t nz = 0;
-#pragma unroll
-      for (int i = 0; i < kPk; ++i) pk[i] = 0x55555555u;
-#pragma unroll
-      for (int i = 0; i < kK; ++i) {
-        if ((act >> i) & 1u) {
-          const uint16_t *ws = wd + i * kStride;
-          const uint32_t p8 = (((uint32_t)ws[ia] | ((uint32_t)ws[ib] << 10)) >> (2u * d0)) & 0xffu;
-          pk[i / 4] ^= (p8 ^ 0x55u) << (8 * (i % 4));
-          if (p8 != 0x55u) nz |= 1u << i;
-        }
-      }
-      return nz;
-    };
-    auto add_streams = [&](float4 &o, uint32_t nz, const uint32_t(&pk)[kPk]) {
-#pragma unroll
-      for (int i = 0; i < kK; ++i)
-        if ((nz >> i) & 1u)
-          add_pattern4(o, pair, (pk[i / 4] >> (8 * (i % 4))) & 0xffu, gs[i].scale);
-    };
-    // two float4s per thread, both loaded before either is added
-    for (uint32_t v = (uint32_t)v0 + threadIdx.x; v < (uint32_t)v1; v += 2 * kDThreads) {
-      const uint32_t vb = v + kDThreads;
-      uint32_t pka[kPk], pkb[kPk];
-      const uint32_t nza = digits(v, pka);
-      const uint32_t nzb = vb < (uint32_t)v1 ? digits(vb, pkb) : 0u;
-      float4 oa = make_float4(0.0f, 0.0f, 0.0f, 0.0f), ob = oa;
-      if (nza) oa = y4[v];
-      if (nzb) ob = y4[vb];
-      if (nza) {
-        add_streams(oa, nza, pka);
-        y4[v] = oa;
-      }
-      if (nzb) {
-        add_streams(ob, nzb, pkb);
-        y4[vb] = ob;
-      }
-    }
-    // single values: the edges of the float4 range, or every value when
-    // acc is not 16-byte aligned
-    auto put = [&](uint64_t e) {
-      const uint32_t e32 = (uint32_t)e;
-      const uint32_t g = e32 / 5u;
-      const uint32_t sh = 2 * (e32 - 5u * g);
-      float v = 0.0f;
-      bool loaded = false;
-#pragma unroll
-      for (int i = 0; i < kK; ++i) {
-        if ((act >> i) & 1u) {
-          const uint32_t dig = (wd[i * kStride + wsw(g - o32)] >> sh) & 3u;
-          if (dig == 1u) continue;
-          if (!loaded) {
-            v = y[e];
-            loaded = true;
-          }
-          v = __fadd_rn(v, dequant(dig, gs[i].scale));
-        }
-      }
-      if (loaded) y[e] = v;
-    };
-    if (!vec || v1 <= v0) {
-      for (uint64_t e = e_begin + threadIdx.x; e < e_end; e += kDThreads) put(e);
-    } else if (threadIdx.x < 4) {
-      const uint64_t e = e_begin + threadIdx.x;
-      if (e < 4 * v0) put(e);
-    } else if (threadIdx.x < 8) {
-      const uint64_t e = 4 * v1 + (threadIdx.x - 4);
-      if (e < e_end) put(e);
-    }
-  }
-  __syncthreads();
-}
-
-// Shared memory (dynamic part) of k_decode_ix: the gather tile's digit
-// words, kGt + 16 per stream.
-template <int kGt, int kK>
-constexpr size_t ix_smem_bytes() {
-  return (size_t)kK * (kGt + 16) * sizeof(uint16_t);
-}
-
-// Add k (2 <= k <= kK) indexed streams, in stream order, into acc by gather
-// tiles.  Streams the index did not mark valid are left out.  Tiles in
-// ticket order; no tile waits on another.
-template <int kGt, int kK>
-__global__ void __launch_bounds__(kDThreads, 6) k_decode_ix(const IxArgs a) {
-  extern __shared__ __align__(16) uint8_t dyn_s[];
-  __shared__ float2 pair[16];
-  __shared__ uint16_t lut[256];
-  __shared__ GatherSmem<kK> gsm;
-  __shared__ GStream gs[kK];
-  __shared__ int na_s;
-  __shared__ uint32_t tile_s;
-  fill_lut(lut);
-  fill_pairs(pair);
+// Sum tiles: kSumTile groups of acc, one block each (block b takes tiles
+// b, b + grid, ...).  Every valid stream's entries of the tile
+// [tfe[t], tfe[t + 1]) go to the tile's digit words in shared memory (kK *
+// kSumTile words) and set the stream's bit in their group's mask byte.
+// Then each thread takes whole groups: it reads the values of a marked
+// group that some stream changes once, adds the marking streams' values in
+// stream order and writes them once.  No value is touched by two threads,
+// so the streams need no barrier between them.
+template <int kK>
+__global__ void __launch_bounds__(kDThreads, 3) k_apply_entries(const IxArgs a) {
+  extern __shared__ __align__(16) uint8_t dyn_s[];  // mask bytes, then digit words
+  __shared__ float scale_s[kK];
+  __shared__ const uint32_t *list_s[kK];  // per-lane stream choice: read from shared memory
+  __shared__ uint32_t lo_s[kK], cnt_s[kK + 1];
+  uint32_t *mask = reinterpret_cast<uint32_t *>(dyn_s);
+  uint16_t *wd = reinterpret_cast<uint16_t *>(dyn_s + kSumTile);
   pdl_enter();
-  if (threadIdx.x == 0) {
-    // the valid streams, in stream order
-    int na = 0;
-    for (int s = 0; s < a.k && s < kK; ++s) {
-      if (!a.ok[s]) continue;
-      const IxStream &S = a.s[s];
+  if (threadIdx.x < (unsigned)kK) {
+    float scale = 0.0f;
+    const uint32_t *list = nullptr;
+    if ((int)threadIdx.x < a.k) {
+      const IxStream &S = a.s[threadIdx.x];
       uint64_t m = 0;
-      float scale = 0.0f;
-      if (!read_stream_header(S.in, S.len_dev, S.cap, a.groups, m, scale)) continue;
-      GStream g;
-      g.payload = S.in + 4;
-      g.loc = S.loc;
-      g.cpre = S.cpre;
-      g.page = S.page;
-      g.m = m;
-      g.scale = scale;
-      g.n_units = (uint32_t)((m + kDecodeUnit - 1) / kDecodeUnit);
-      gs[na++] = g;
+      list = S.list;
+      if (!a.ok[threadIdx.x] || !read_stream_header(S.in, S.len_dev, S.cap, a.groups, m, scale))
+        scale = -1.0f;  // left out
     }
-    na_s = na;
+    scale_s[threadIdx.x] = scale;
+    list_s[threadIdx.x] = list;
   }
   __syncthreads();
-  const int na = na_s;
-  if (na == 0) return;
-  const uint64_t n_tiles = (a.groups + kGt - 1) / kGt;
-  for (;;) {
-    if (threadIdx.x == 0) tile_s = atomicAdd(a.ticket2, 1u);
+  const uint32_t n_tiles = sum_tiles(a.groups);
+  for (uint32_t t = blockIdx.x; t < n_tiles; t += gridDim.x) {
+    const uint64_t g0 = (uint64_t)t * kSumTile;
+    const uint32_t gn = (uint32_t)umin64(kSumTile, a.groups - g0);
+    for (uint32_t i = threadIdx.x; i < kSumTile / 16; i += kDThreads)
+      reinterpret_cast<uint4 *>(mask)[i] = make_uint4(0u, 0u, 0u, 0u);
+    if (threadIdx.x < (unsigned)kK) {
+      uint32_t lo = 0, hi = 0;
+      if ((int)threadIdx.x < a.k && scale_s[threadIdx.x] >= 0.0f) {
+        lo = __ldg(a.s[threadIdx.x].tfe + t);
+        hi = __ldg(a.s[threadIdx.x].tfe + t + 1);
+        if (hi < lo) hi = lo;
+      }
+      lo_s[threadIdx.x] = lo;
+      cnt_s[threadIdx.x] = hi - lo;
+    }
     __syncthreads();
-    const uint32_t t = tile_s;
-    if (t >= n_tiles) break;
-    gather_tile<kGt, kK>(gs, na, (uint64_t)t * kGt, a.groups, a.n, a.y, a.vec, lut, pair,
-                         reinterpret_cast<uint16_t *>(dyn_s), gsm);
+    if (threadIdx.x == 0) {
+      uint32_t run = 0;
+      for (int s = 0; s < kK; ++s) {
+        const uint32_t c = cnt_s[s];
+        cnt_s[s] = run;
+        run += c;
+      }
+      cnt_s[kK] = run;
+    }
+    __syncthreads();
+    const uint32_t all = cnt_s[kK];
+    if (all == 0) continue;  // uniform; nothing here reads the tile's shared memory
+    // the tile's entries of every stream, flattened
+    for (uint32_t i = threadIdx.x; i < all; i += kDThreads) {
+      int s = 0;
+      while (s + 1 < kK && cnt_s[s + 1] <= i) ++s;
+      const uint32_t ent = __ldg(list_s[s] + lo_s[s] + (i - cnt_s[s]));
+      const uint32_t p = ent >> 16;
+      if (TLC_CHECK(p < gn)) {
+        wd[s * kSumTile + p] = (uint16_t)(ent & 0x3ffu);
+        atomicOr(mask + (p >> 2), 1u << (8 * (p & 3) + s));
+      }
+    }
+    __syncthreads();
+    // this thread's groups are i = threadIdx.x + kDThreads * j; the marked
+    // ones four at a time: first, from shared memory alone, which of their
+    // values some stream changes, then those values loaded (all before any
+    // add), the streams' values added in stream order, and written
+    static_assert(kSumTile / kDThreads <= 32, "a thread's groups fit one word of bits");
+    const uint8_t *mb = reinterpret_cast<const uint8_t *>(mask);
+    uint32_t todo = 0;
+#pragma unroll
+    for (uint32_t j = 0; j < kSumTile / kDThreads; ++j) {
+      const uint32_t i = threadIdx.x + kDThreads * j;
+      if (i < gn && mb[i]) todo |= 1u << j;
+    }
+    while (todo) {
+      constexpr int kAt = 4;
+      uint32_t gi[kAt], tch[kAt];
+#pragma unroll
+      for (int q = 0; q < kAt; ++q) {
+        gi[q] = 0u;
+        tch[q] = 0u;
+        if (todo) {
+          const uint32_t i = threadIdx.x + kDThreads * (uint32_t)(__ffs(todo) - 1);
+          todo &= todo - 1;
+          gi[q] = i;
+          uint32_t mk = mb[i], t = 0;
+          while (mk) {
+            const int st = __ffs(mk) - 1;
+            mk &= mk - 1;
+            const uint32_t dw = wd[st * kSumTile + i];
+            // digit d is not zero (not 1): bit 2d of dw clear
+#pragma unroll
+            for (int d = 0; d < 5; ++d) t |= (((dw >> (2 * d)) & 1u) ^ 1u) << d;
+          }
+          const uint64_t e0 = 5 * (g0 + i);
+          tch[q] = t & ((1u << (uint32_t)umin64(5, a.n - e0)) - 1u);  // the last group may be short
+        }
+      }
+      float v[kAt][5];
+#pragma unroll
+      for (int q = 0; q < kAt; ++q) {
+        const uint64_t e0 = 5 * (g0 + gi[q]);
+#pragma unroll
+        for (int d = 0; d < 5; ++d) v[q][d] = ((tch[q] >> d) & 1u) ? a.y[e0 + d] : 0.0f;
+      }
+#pragma unroll
+      for (int q = 0; q < kAt; ++q) {
+        if (!tch[q]) continue;
+        const uint32_t i = gi[q];
+        const uint64_t e0 = 5 * (g0 + i);
+        uint32_t mk = mb[i];
+        while (mk) {
+          const int st = __ffs(mk) - 1;
+          mk &= mk - 1;
+          const uint32_t dw = wd[st * kSumTile + i];
+          const float sc = scale_s[st];
+#pragma unroll
+          for (int d = 0; d < 5; ++d) {
+            const uint32_t dig = (dw >> (2 * d)) & 3u;
+            if (dig != 1u) v[q][d] = __fadd_rn(v[q][d], dequant(dig, sc));
+          }
+        }
+#pragma unroll
+        for (int d = 0; d < 5; ++d)
+          if ((tch[q] >> d) & 1u) a.y[e0 + d] = v[q][d];
+      }
+    }
+    __syncthreads();  // the tile's shared memory is rewritten by the next tile
   }
+}
+
+template <int kK>
+constexpr size_t apply_smem_bytes() {
+  return (size_t)kSumTile + (size_t)kK * kSumTile * sizeof(uint16_t);
 }
 
 // ================================================================= batches
@@ -1422,6 +1466,7 @@ struct BatchDecodeArgs {
 
 constexpr int kPrepThreads = 1024;
 constexpr uint32_t kSmemSearch = 2048;  // tensors whose first tiles fit in shared memory
+constexpr uint32_t kSmemSearchUnits = 1024;  // the same in the warp-unit kernel (less room)
 
 // One block: validate every tensor's stream once, and number the tiles that
 // actually exist (ceil(m / tile_bytes) per stream, none for a corrupt one)
@@ -1528,7 +1573,7 @@ __global__ void __launch_bounds__(kDThreads) k_decode_batch(const BatchDecodeArg
 // tensor by the prepare kernel; block b takes chunks b, b + grid, ...
 __global__ void __launch_bounds__(kDThreads, 4) k_index_count_batch(const BatchDecodeArgs a) {
   __shared__ uint32_t begin_s[kSmemSearch];
-  __shared__ uint32_t wtot_s[kDWarps];
+  __shared__ uint32_t wtot_s[2 * kDWarps];
   pdl_enter();
   const bool in_smem = a.count <= kSmemSearch;
   if (in_smem)
@@ -1539,8 +1584,8 @@ __global__ void __launch_bounds__(kDThreads, 4) k_index_count_batch(const BatchD
     const uint32_t id = find_tensor(begin_s, in_smem, a.prep, a.count, g, true);
     const BatchTensor &T = a.tensors[id];
     const BatchPrep &P = a.prep[id];
-    count_chunk(a.arena + T.arena_off + 4, P.m, g - P.cact_begin, a.loc + T.d_tile_begin,
-                a.cpre + T.d_chunk_begin + id, wtot_s);
+    count_chunk<false>(a.arena + T.arena_off + 4, P.m, g - P.cact_begin, a.loc + T.d_tile_begin,
+                       a.cpre + T.d_chunk_begin + id, nullptr, nullptr, wtot_s);
   }
 }
 
@@ -1556,7 +1601,7 @@ __global__ void __launch_bounds__(kDThreads) k_index_scan_batch(const BatchDecod
       if (threadIdx.x == 0) a.ok[id] = 0u;
       continue;
     }
-    const IndexOut io = {a.cpre + T.d_chunk_begin + id, nullptr, a.ok + id, T.groups};
+    const IndexOut io = {a.cpre + T.d_chunk_begin + id, a.ok + id, T.groups, nullptr};
     scan_chunks<kDThreads>(io, chunks_of(P.m), wsum, a.dev_status);
   }
 }
@@ -1567,12 +1612,12 @@ __global__ void __launch_bounds__(kDThreads) k_index_scan_batch(const BatchDecod
 template <int kMode>
 __global__ void __launch_bounds__(kDThreads, units_min_blocks<kMode>(true))
     k_decode_batch_units(const BatchDecodeArgs a) {
-  __shared__ UnitSmem sm;
-  __shared__ uint32_t begin_s[kSmemSearch];
+  __shared__ UnitSmem<kMode> sm;
+  __shared__ uint32_t begin_s[kSmemSearchUnits];
   __shared__ DecodeJob jobs[kDWarps];  // each warp's current tensor
-  fill_unit_tables(sm);
+  fill_lut(sm.d.lut);
   pdl_enter();
-  const bool in_smem = a.count <= kSmemSearch;
+  const bool in_smem = a.count <= kSmemSearchUnits;
   if (in_smem)
     for (uint32_t i = threadIdx.x; i < a.count; i += kDThreads) begin_s[i] = a.prep[i].act_begin;
   __syncthreads();
@@ -1603,9 +1648,10 @@ __global__ void __launch_bounds__(kDThreads, units_min_blocks<kMode>(true))
         j.cpre = a.cpre + T.d_chunk_begin + id;
       }
       __syncwarp();
+      fill_scaled_pairs(sm.sp[warp], j.scale, lane);
       cur = id;
     }
-    decode_unit<kMode>(j, gu - first, sm.d.lut, sm.pair, sm.wd[warp]);
+    decode_unit<kMode>(j, gu - first, sm.d.lut, sm.sp[warp], sm.wd[warp], unit_stage(sm, warp));
   }
 }
 
@@ -1640,7 +1686,6 @@ uint32_t decode_tile_payload_bytes(bool accumulate) {
   return accumulate ? DecodeShape<kAccumulate>::kTile : DecodeShape<kWrite>::kTile;
 }
 
-uint32_t decode_pages(uint64_t groups) { return (uint32_t)((groups + kPage - 1) / kPage); }
 
 static uint32_t persistent_grid(const DeviceInfo &dev, int occ, uint64_t work_blocks) {
   uint64_t grid = (uint64_t)dev.sm_count * (uint64_t)(occ > 0 ? occ : 1);
@@ -1687,9 +1732,10 @@ cudaError_t launch_decode(const DeviceInfo &dev, const uint8_t *in, const uint64
 
 // ---- indexed decode of up to kIndexPass streams --------------------------
 // Scratch: [ticket2, ok[kIndexPass]] (written by the scan), then each
-// stream's loc[] (one word per unit of its capacity), cpre[] (one per chunk,
-// plus the total) and, for two streams or more, page[] (one per 1024
-// groups).
+// stream's loc[] (one word per unit of its capacity) and cpre[] (one per
+// chunk, plus the total); for two streams or more also eloc[], ecpre[],
+// list[] (one word per possible entry: min(payload capacity, groups)) and
+// tfe[] (one per sum tile, plus the total).
 static size_t ix_head_bytes() { return align_up(4 + 4 * kIndexPass, 256); }
 
 IndexedLayout indexed_layout(const IndexedStream *s, int k, uint64_t n) {
@@ -1699,27 +1745,35 @@ IndexedLayout indexed_layout(const IndexedStream *s, int k, uint64_t n) {
   for (int i = 0; i < k; ++i) {
     const uint32_t units = decode_tiles_max(s[i].cap, groups);
     const uint32_t chunks = (units + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
-    L.loc_off[i] = at;
-    at = align_up(at + 4 * (size_t)units, 16);
-    L.cpre_off[i] = at;
-    at = align_up(at + 4 * ((size_t)chunks + 1), 16);
-    L.page_off[i] = at;
-    if (k > 1) at = align_up(at + 4 * (size_t)decode_pages(groups), 16);
+    auto take = [&at](size_t words) {
+      const size_t off = at;
+      at = align_up(at + 4 * words, 16);
+      return off;
+    };
+    L.loc_off[i] = take(units);
+    L.cpre_off[i] = take((size_t)chunks + 1);
+    if (k > 1) {
+      const uint64_t mcap = s[i].cap >= 4 ? s[i].cap - 4 : 0;
+      L.eloc_off[i] = take(units);
+      L.ecpre_off[i] = take((size_t)chunks + 1);
+      L.list_off[i] = take((size_t)(mcap < groups ? mcap : groups) + 1);
+      L.tfe_off[i] = take((size_t)sum_tiles(groups) + 1);
+    }
   }
   L.total_bytes = align_up(at, 256);
   return L;
 }
 
 // Blocks per SM: the warp-unit kernels (slots 0 dense output, 1
-// accumulate) and each k_decode_ix instantiation (slots 2, 3, 4: up to 2, 4
-// and 8 streams), with their shared memory.
-template <int kGt, int kK>
-static int ix_occupancy() {
-  constexpr size_t smem = ix_smem_bytes<kGt, kK>();
-  cudaFuncSetAttribute(k_decode_ix<kGt, kK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+// accumulate) and each k_apply_entries instantiation (slots 2, 3, 4: up to
+// 2, 4 and 8 streams), with their shared memory.
+template <int kK>
+static int apply_occupancy() {
+  constexpr size_t smem = apply_smem_bytes<kK>();
+  cudaFuncSetAttribute(k_apply_entries<kK>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)smem);
   int occ = 0;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_ix<kGt, kK>, kDThreads, smem);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_apply_entries<kK>, kDThreads, smem);
   return occ;
 }
 
@@ -1727,21 +1781,17 @@ void occupancy_decode_ix(int occ[5]) {
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ[0], k_decode_units<kWrite>, kDThreads, 0);
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ[1], k_decode_units<kAccumulate>, kDThreads,
                                                 0);
-  occ[2] = ix_occupancy<TLC_GT_ACC / 2, 2>();
-  occ[3] = ix_occupancy<TLC_GT_ACC / 4, 4>();
-  occ[4] = ix_occupancy<TLC_GT_ACC / 8, 8>();
+  occ[2] = apply_occupancy<2>();
+  occ[3] = apply_occupancy<4>();
+  occ[4] = apply_occupancy<8>();
 }
 
-template <int kGt, int kK>
-static cudaError_t launch_ix(const DeviceInfo &dev, const IxArgs &a, int occ_slot,
-                             cudaStream_t stream) {
-  constexpr size_t smem = ix_smem_bytes<kGt, kK>();
-  const uint32_t grid =
-      persistent_grid(dev, dev.occ_decode_ix[occ_slot], (a.groups + kGt - 1) / kGt);
-  timing_begin(kKindDecodeAccumulate, stream);
-  launch_k(k_decode_ix<kGt, kK>, grid, kDThreads, smem, stream, a);
-  timing_end(kKindDecodeAccumulate, stream);
-  return cudaGetLastError();
+template <int kK>
+static cudaError_t launch_apply(const DeviceInfo &dev, const IxArgs &a, int occ_slot,
+                               cudaStream_t stream) {
+  constexpr size_t smem = apply_smem_bytes<kK>();
+  const uint32_t grid = persistent_grid(dev, dev.occ_decode_ix[occ_slot], sum_tiles(a.groups));
+  return launch_k(k_apply_entries<kK>, grid, kDThreads, smem, stream, a);
 }
 
 cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s, int k, uint64_t n,
@@ -1760,25 +1810,33 @@ cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s,
   a.y = y;
   a.vec = (reinterpret_cast<uintptr_t>(y) & 15) == 0;
   a.dev_status = dev_status;
-  uint64_t chunks = 0, units_max = 0;
+  uint64_t chunks = 0, units_max = 0, units_all = 0;
   for (int i = 0; i < kIndexPass; ++i) {
     IxStream &S = a.s[i];
+    S = IxStream{};
     if (i < k) {
       S.in = s[i].in;
       S.len_dev = s[i].len_dev;
       S.cap = s[i].cap;
       S.loc = reinterpret_cast<uint32_t *>(base + L.loc_off[i]);
       S.cpre = reinterpret_cast<uint32_t *>(base + L.cpre_off[i]);
-      S.page = k > 1 ? reinterpret_cast<uint32_t *>(base + L.page_off[i]) : nullptr;
+      if (k > 1) {
+        S.eloc = reinterpret_cast<uint32_t *>(base + L.eloc_off[i]);
+        S.ecpre = reinterpret_cast<uint32_t *>(base + L.ecpre_off[i]);
+        S.list = reinterpret_cast<uint32_t *>(base + L.list_off[i]);
+        S.tfe = reinterpret_cast<uint32_t *>(base + L.tfe_off[i]);
+      }
       const uint32_t units = decode_tiles_max(s[i].cap, a.groups);
       chunks += (units + kDecodeChunkUnits - 1) / kDecodeChunkUnits;
+      units_all += units;
       if (units > units_max) units_max = units;
-    } else {
-      S = IxStream{};
     }
   }
   timing_begin(kKindDecodeCount, stream);
-  launch_k(k_index_count, persistent_grid(dev, 4, chunks), kDThreads, 0, stream, a);
+  if (k > 1)
+    launch_k(k_index_count<true>, persistent_grid(dev, 4, chunks), kDThreads, 0, stream, a);
+  else
+    launch_k(k_index_count<false>, persistent_grid(dev, 4, chunks), kDThreads, 0, stream, a);
   launch_k(k_index_scan, k, kScanThreads, 0, stream, a);
   timing_end(kKindDecodeCount, stream);
   cudaError_t e = cudaGetLastError();
@@ -1796,9 +1854,19 @@ cudaError_t launch_decode_indexed(const DeviceInfo &dev, const IndexedStream *s,
     timing_end(kind, stream);
     return cudaGetLastError();
   }
-  if (k == 2) return launch_ix<TLC_GT_ACC / 2, 2>(dev, a, 2, stream);
-  if (k <= 4) return launch_ix<TLC_GT_ACC / 4, 4>(dev, a, 3, stream);
-  return launch_ix<TLC_GT_ACC / 8, 8>(dev, a, 4, stream);
+  // several streams: every stream's entries (one warp per unit), then the
+  // sum tiles
+  timing_begin(kKindDecodeAccumulate, stream);
+  launch_k(k_index_entries, persistent_grid(dev, 8, (units_all + kDWarps - 1) / kDWarps),
+           kDThreads, 0, stream, a);
+  if (k == 2)
+    e = launch_apply<2>(dev, a, 2, stream);
+  else if (k <= 4)
+    e = launch_apply<4>(dev, a, 3, stream);
+  else
+    e = launch_apply<8>(dev, a, 4, stream);
+  timing_end(kKindDecodeAccumulate, stream);
+  return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // ---- plans ----------------------------------------------------------------

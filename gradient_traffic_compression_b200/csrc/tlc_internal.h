@@ -172,7 +172,6 @@ cudaError_t launch_decode_batch(const DeviceInfo &dev, const BatchPlanDev &p,
 int occupancy_quant_batch();
 int occupancy_decode_batch(bool accumulate, bool indexed);
 uint32_t decode_tile_payload_bytes(bool accumulate);
-uint32_t decode_pages(uint64_t groups);
 
 // Per-device facts for device d (initialised on first use); nullptr on error.
 const DeviceInfo *device_info(int d);
@@ -241,8 +240,9 @@ cudaError_t launch_decode(const DeviceInfo &dev, const uint8_t *in, const uint64
                           cudaStream_t stream);
 
 // Indexed decode of up to kIndexPass streams of n values each: the index
-// (a count and a scan launch) and one decode launch (dense output: exactly
-// one stream; accumulate: the streams added in order).  The scratch is
+// (a count and a scan launch), then one decode launch (dense output: exactly
+// one stream; accumulate of one stream) or, for a sum of several streams
+// (added in order), an entries launch and a sum-tile launch.  The scratch is
 // indexed_layout(..).total_bytes bytes; nothing in it needs clearing.
 constexpr int kIndexPass = 8;
 struct IndexedStream {
@@ -251,7 +251,8 @@ struct IndexedStream {
   uint64_t cap;
 };
 struct IndexedLayout {
-  size_t loc_off[kIndexPass], cpre_off[kIndexPass], page_off[kIndexPass];
+  size_t loc_off[kIndexPass], cpre_off[kIndexPass];
+  size_t eloc_off[kIndexPass], ecpre_off[kIndexPass], list_off[kIndexPass], tfe_off[kIndexPass];
   size_t total_bytes;
 };
 IndexedLayout indexed_layout(const IndexedStream *s, int k, uint64_t n);
