@@ -14,13 +14,13 @@
 //   k_absmax     x' = x + err and M = max|x'| (as a max over the uint32 bit
 //                patterns of |x'|; NaN/Inf sort above every finite value).
 //                It also clears the scan state that k_quant_zre uses.
-//   k_quant_zre  per tile of 4096 byte groups (20480 values): recompute x',
+//   k_quant_zre  per tile of 2048 byte groups (10240 values): recompute x',
 //                q = round(x'/(M s)), err' = x' - q M s (written back), pack
 //                the quartic bytes into shared memory, zero-run encode them,
 //                and place the tile's output with a decoupled look-back over
 //                earlier tiles.  Tiles are taken in order from a ticket
 //                counter, so every tile a tile waits on is already running.
-// Tensors of 384 tiles and more take a third launch instead of the
+// Tensors of 768 tiles and more take a third launch instead of the
 // per-tile look-back (the deferred-placement path): k_quant_zre tiles
 // write their summary and stage the bytes that follow their leading run,
 // and k_zre_place, one block per 32 tiles, scans the summaries (a
@@ -126,7 +126,7 @@ k_absmax(const float *__restrict__ x, const float *__restrict__ err, uint64_t n,
 // --------------------------------------------------------- k_quant_zre ----
 // Tile shape (compile-time knobs; defaults are the tuned values).
 #ifndef TLC_Q_ITERS
-#define TLC_Q_ITERS 4
+#define TLC_Q_ITERS 2
 #endif
 #ifndef TLC_Q_MINB
 #define TLC_Q_MINB 6
@@ -136,9 +136,9 @@ constexpr int kQWarps = kQThreads / kWarp;
 constexpr int kChunkElems = 640;   // one warp step: 32 lanes x 5 float4
 constexpr int kChunkGroups = 128;  // = kChunkElems / 5
 constexpr int kQIters = TLC_Q_ITERS;
-constexpr int kTileGroups = kQWarps * kQIters * kChunkGroups;  // 4096 by default
-constexpr uint64_t kTileElems = 5ull * kTileGroups;            // 20480 by default
-constexpr int kZBytes = kTileGroups / kQThreads;               // 16 per thread by default
+constexpr int kTileGroups = kQWarps * kQIters * kChunkGroups;  // 2048 by default
+constexpr uint64_t kTileElems = 5ull * kTileGroups;            // 10240 by default
+constexpr int kZBytes = kTileGroups / kQThreads;               // 8 per thread by default
 constexpr int kZWords = kZBytes / 4;                           // u32 words per thread
 static_assert((kZBytes == 8 || kZBytes % 16 == 0) && kTileGroups < 65536, "tile shape");
 #ifndef TLC_Q_LOOKV
@@ -147,7 +147,7 @@ static_assert((kZBytes == 8 || kZBytes % 16 == 0) && kTileGroups < 65536, "tile 
 constexpr int kLookV = TLC_Q_LOOKV;  // look-back words per lane per round trip
 // Tensors of at least this many tiles take the deferred-placement path.
 #ifndef TLC_DEFER_MIN_TILES
-#define TLC_DEFER_MIN_TILES 384
+#define TLC_DEFER_MIN_TILES 768
 #endif
 constexpr uint32_t kDeferMinTiles = TLC_DEFER_MIN_TILES;
 
@@ -700,7 +700,7 @@ __device__ __forceinline__ void zre_encode_tile(const TileJob &j, const DeferJob
   __syncthreads();
 }
 
-// One tile of 4096 byte groups (20480 values) of one tensor, fused: quantize
+// One tile of kTileGroups byte groups (5 kTileGroups values) of one tensor, fused: quantize
 // and update the error buffer, pack the quartic bytes into shared memory,
 // then zero-run encode them.  Whole block; ends synchronised.
 // kCount: the tile's non-zero values are added to the call's record.
@@ -867,8 +867,12 @@ __global__ void TLC_Q_BOUNDS k_quant_zre(const QuantArgs a) {
   for (;;) {
     if (threadIdx.x == 0) tile_id_s = atomicAdd(a.ticket, 1u);
     __syncthreads();
-    const uint32_t t = tile_id_s;
-    if (t >= a.n_tiles) break;
+    const uint32_t tk = tile_id_s;
+    if (tk >= a.n_tiles) break;
+    // Deferred tiles wait on no other tile, so they run last tile first:
+    // k_absmax swept x and err front to back, and the end of both is still
+    // in L2.  Look-back tiles keep ticket order (each waits on earlier ones).
+    const uint32_t t = kDeferred ? a.n_tiles - 1 - tk : tk;
     quant_tile<kDeferred, kRecord>(job, djob, t, scale, thr, sm, a.dev_status, a.max_polls);
   }
 }
@@ -1091,8 +1095,9 @@ __global__ void TLC_Q_BOUNDS k_quant_zre_batch(const BatchQuantArgs a) {
   for (;;) {
     if (threadIdx.x == 0) tile_id_s = atomicAdd(a.ticket, 1u);
     __syncthreads();
-    const uint32_t u = tile_id_s;
-    if (u >= a.n_tiles) break;
+    const uint32_t tk = tile_id_s;
+    if (tk >= a.n_tiles) break;
+    const uint32_t u = kDeferred ? a.n_tiles - 1 - tk : tk;  // as in k_quant_zre
     const uint32_t id = a.tile_tensor[u];
     const BatchTensor &T = a.tensors[id];
     const uint32_t t = u - T.q_tile_begin;

@@ -2,8 +2,8 @@
 // allocation, for callers that cannot allocate device memory (see tlc.h).
 //
 // The two compress kernels need a little scratch: one 64-bit status word per
-// tile of 4096 byte groups, a tile ticket, and one partial maximum per block
-// of the magnitude pass.  Here that scratch is a fixed array in the
+// compress tile (2048 byte groups), a tile ticket, and one partial maximum
+// per block of the magnitude pass.  Here that scratch is a fixed array in the
 // library's own device memory instead of a stream-ordered allocation.
 #include <atomic>
 #include <cstring>
@@ -15,9 +15,9 @@
 namespace {
 
 // The scratch, in every device that loads the library, for the life of the
-// process.  256 KiB holds the status words of n <= TLC_NOALLOC_MAX_N plus
-// the partial maxima of devices with up to 3000 SMs.
-constexpr size_t kScratchBytes = 256 * 1024;
+// process.  512 KiB holds the status words of n <= TLC_NOALLOC_MAX_N (52,429
+// tiles) plus the partial maxima of devices with up to 3000 SMs.
+constexpr size_t kScratchBytes = 512 * 1024;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;

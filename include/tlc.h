@@ -95,7 +95,7 @@ size_t tlc_compress_bound(size_t n);
  * unchanged and out holds no stream.
  * Host errors: TLC_ERR_INVALID_ARG if a pointer is NULL, n is out of range,
  * s is outside [1, 2) or NaN, out_cap is too small, or x/err/out overlap.
- * Scratch: about 8 bytes per 20480 values; from 384 * 20480 values on, also
+ * Scratch: about 8 bytes per 10240 values; from 768 * 10240 values on, also
  * a staging area of about n/5 bytes (the placement of the zero-run encoded
  * bytes then runs as a separate kernel). */
 tlc_status tlc_compress(const float *x, size_t n, float s, float *err,
@@ -143,8 +143,8 @@ tlc_status tlc_compress_recorded(const float *x, size_t n, float s, float *err,
  * does not expand to exactly ceil(n/5) groups.  Then y holds unspecified
  * values, but nothing outside y is written.
  * When min(in_cap - 4, ceil(n/5)) spans 16384 or more 512-byte units
- * (about 8 MiB; per stream in tlc_decompress_accumulate), a counting kernel
- * runs before the decode kernel; the result is the same. */
+ * (about 8 MiB), an index (a count kernel and a scan kernel) runs before the
+ * decode kernel; the result is the same. */
 tlc_status tlc_decompress(const uint8_t *in, const uint64_t *in_len,
                           size_t in_cap, size_t n, float *y,
                           int32_t *dev_status, tlc_stream_t stream);
@@ -253,7 +253,7 @@ tlc_status tlc_compress_noalloc(const float *x, size_t n, float s, float *err,
 
 /* Debug build.  libtlc_debug.so (the same sources compiled with
  * -DTLC_DEBUG) checks every index of its shared-memory staging, stream
- * placement and page tables before the access, and puts 256-byte canaries of
+ * placement and entry lists before the access, and puts 256-byte canaries of
  * 0xA5 on both sides of every scratch allocation, checked by a small kernel
  * when the scratch is freed.  A failing check never faults: it records its
  * location (source line | file id << 16; file ids 1 compress, 2 decode,

@@ -144,7 +144,8 @@ def mixed_case(seed, n, zero_frac=0.6):
 
 # ------------------------------------------------------------------ cases --
 
-TILE_VALUES = 20480          # compress tile: 4096 groups
+TILE_GROUPS = 2048           # compress tile
+TILE_VALUES = 5 * TILE_GROUPS
 RAGGED = sorted(set(
     list(range(1, 13)) + [19, 20, 21, 39, 40, 41, 639, 640, 641, 5119, 5120, 5121,
                           TILE_VALUES - 1, TILE_VALUES, TILE_VALUES + 1, TILE_VALUES + 5,
@@ -191,24 +192,24 @@ def _literal_groups_case(n, groups):
 
 RUN_CASES = {
     # runs that end exactly at, just past, or far past compress tile edges
-    # (4096 groups per tile), with lengths = 0, 1, 13 (mod 14) on each side
-    "edge_mod0": [4096 - 15, 4096 + 13],
-    "edge_mod1": [4096 - 16, 4096 + 14],
-    "edge_mod13": [4096 - 14, 4096 + 12],
-    "end_at_edge": [4096 - 1, 4096, 8191],
-    "start_at_edge": [4095, 4096 + 27],
-    "span_many_tiles": [100, 4096 * 5 + 57],
-    "span_exact_tiles": [4095, 4096 * 3 - 1],
+    # (TILE_GROUPS groups per tile), with lengths = 0, 1, 13 (mod 14) on each side
+    "edge_mod0": [TILE_GROUPS - 15, TILE_GROUPS + 13],
+    "edge_mod1": [TILE_GROUPS - 16, TILE_GROUPS + 14],
+    "edge_mod13": [TILE_GROUPS - 14, TILE_GROUPS + 12],
+    "end_at_edge": [TILE_GROUPS - 1, TILE_GROUPS, 2 * TILE_GROUPS - 1],
+    "start_at_edge": [TILE_GROUPS - 1, TILE_GROUPS + 27],
+    "span_many_tiles": [100, TILE_GROUPS * 5 + 57],
+    "span_exact_tiles": [TILE_GROUPS - 1, TILE_GROUPS * 3 - 1],
     "long_tail_run": [3],
-    "long_head_run": [4096 * 4 + 1],
-    "dense_then_empty": list(range(0, 300)) + [4096 * 2 + 7],
+    "long_head_run": [TILE_GROUPS * 4 + 1],
+    "dense_then_empty": list(range(0, 300)) + [TILE_GROUPS * 2 + 7],
 }
 
 
 @pytest.mark.parametrize("name", list(RUN_CASES))
 def test_runs_across_tiles(g, name):
     groups = RUN_CASES[name]
-    n = 5 * (4096 * 6 + 11) + 3
+    n = 5 * (TILE_GROUPS * 6 + 11) + 3
     x = _literal_groups_case(n, groups)
     st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
     assert_roundtrip_parity(g, st, n)
@@ -216,7 +217,7 @@ def test_runs_across_tiles(g, name):
 
 @pytest.mark.parametrize("tail", [0, 1, 13, 14, 15, 27, 28])
 def test_run_lengths_at_stream_end(g, tail):
-    gtot = 4096 * 2 + tail + 1
+    gtot = TILE_GROUPS * 2 + tail + 1
     n = 5 * gtot
     x = _literal_groups_case(n, [gtot - tail - 1])     # then `tail` zero groups
     st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
@@ -241,7 +242,7 @@ def test_dense_streams_at_decode_tile_edges(g, groups):
 
 
 def test_all_zero_and_single_values(g):
-    for n in (1, 5, 70, 71, 4096 * 5, 4096 * 5 * 3 + 1):
+    for n in (1, 5, 70, 71, TILE_GROUPS * 5, TILE_GROUPS * 5 * 3 + 1):
         st, _ = assert_compress_parity(g, np.zeros(n, np.float32), 1.0, np.zeros(n, np.float32))
         assert_roundtrip_parity(g, st, n)
     x = np.zeros(100003, np.float32)
@@ -499,11 +500,11 @@ def test_large_nonfinite_and_zero(g):
     assert_roundtrip_parity(g, st, n)
 
 
-# ---- the deferred-placement path (tensors of 384 tiles and more) ---------
-# Tiles there stage their bytes and a second kernel places them; below 384
+# ---- the deferred-placement path (tensors of 768 tiles and more) ---------
+# Tiles there stage their bytes and a second kernel places them; below 768
 # tiles the tiles place their own bytes.  Both must give the same streams.
 
-DEFER_TILES = 384
+DEFER_TILES = 768
 
 
 @pytest.mark.parametrize("n", [(DEFER_TILES - 1) * TILE_VALUES, (DEFER_TILES - 1) * TILE_VALUES + 1,
@@ -518,15 +519,15 @@ def test_deferred_threshold_sizes(g, n):
 @pytest.mark.parametrize("name", list(RUN_CASES))
 def test_deferred_runs_across_tiles(g, name):
     # the run cases of the look-back path, in a tensor that takes the deferred one
-    n = 5 * 4096 * (DEFER_TILES + 2) + 3
+    n = 5 * TILE_GROUPS * (DEFER_TILES + 2) + 3
     x = _literal_groups_case(n, RUN_CASES[name])
     st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
     assert_roundtrip_parity(g, st, n)
 
 
-@pytest.mark.parametrize("tail", [0, 1, 13, 14, 15, 27, 28, 4096 * 3 + 5])
+@pytest.mark.parametrize("tail", [0, 1, 13, 14, 15, 27, 28, TILE_GROUPS * 3 + 5])
 def test_deferred_run_lengths_at_stream_end(g, tail):
-    gtot = 4096 * DEFER_TILES + tail + 1
+    gtot = TILE_GROUPS * DEFER_TILES + tail + 1
     n = 5 * gtot
     x = _literal_groups_case(n, [gtot - tail - 1])
     st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
@@ -536,8 +537,8 @@ def test_deferred_run_lengths_at_stream_end(g, tail):
 def test_deferred_sparse_literals_every_tile(g):
     # one literal per tile at a drifting position: every tile has a leading
     # run whose remainder byte depends on the tiles before it
-    n = 5 * 4096 * (DEFER_TILES + 5)
-    groups = [t * 4096 + (t * 977) % 4096 for t in range(DEFER_TILES + 5)]
+    n = 5 * TILE_GROUPS * (DEFER_TILES + 5)
+    groups = [t * TILE_GROUPS + (t * 977) % TILE_GROUPS for t in range(DEFER_TILES + 5)]
     x = _literal_groups_case(n, groups)
     st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
     assert_roundtrip_parity(g, st, n)

@@ -4,7 +4,7 @@ framework's caching allocator, or a hot loop where allocation is forbidden).
 Its scratch is a fixed array inside the library, so the call itself never
 allocates.  It must produce exactly what tlc_compress produces.
 
-tlc_compress switches to a different placement of the encoded bytes from 384
+tlc_compress switches to a different placement of the encoded bytes from 768
 tiles (7,864,320 values) on, while the no-allocation call keeps the per-tile
 look-back at every size up to its limit of 2^29 values; the sizes below sit
 on both sides of that switch and at the limit, so the two paths are compared
@@ -25,8 +25,8 @@ import synth
 
 torch = pytest.importorskip("torch")
 
-TILE_VALUES = 5 * 4096          # values per compress tile
-DEFER_TILES = 384               # tlc_compress's placement switch, in tiles
+TILE_VALUES = 5 * 2048          # values per compress tile
+DEFER_TILES = 768               # tlc_compress's placement switch, in tiles
 
 
 @pytest.fixture(scope="module")
