@@ -34,7 +34,7 @@
 //   k_index_entries 2..8 streams: one warp per unit writes the unit's entries
 //                   (tile position and digit word) to the stream's list, in
 //                   group order, and the first entry of every sum tile.
-//   k_apply_entries 2..8 streams: tiles of 4096 groups; each stream's entries
+//   k_apply_entries 2..8 streams: tiles of 2048 groups; each stream's entries
 //                   of the tile go to shared memory with a per-group stream
 //                   mask, then each thread reads a marked group's acc values
 //                   once, adds the streams' values in stream order and
@@ -902,7 +902,7 @@ __device__ __forceinline__ uint32_t chunks_of(uint64_t m) {
 
 // Groups per tile of a sum of several streams.
 #ifndef TLC_SUM_TILE
-#define TLC_SUM_TILE 4096
+#define TLC_SUM_TILE 2048
 #endif
 constexpr uint32_t kSumTile = TLC_SUM_TILE;
 static_assert(kSumTile % 16 == 0 && kSumTile <= 65536, "a tile position fits 16 bits");
@@ -1308,8 +1308,16 @@ __global__ void __launch_bounds__(kDThreads) k_index_entries(const IxArgs a) {
 // group that some stream changes once, adds the marking streams' values in
 // stream order and writes them once.  No value is touched by two threads,
 // so the streams need no barrier between them.
+// Groups of a thread whose acc values are loaded together, and the blocks
+// per SM the kernel is compiled for.
+#ifndef TLC_SUM_AT
+#define TLC_SUM_AT 2
+#endif
+#ifndef TLC_SUM_MINB
+#define TLC_SUM_MINB 5
+#endif
 template <int kK>
-__global__ void __launch_bounds__(kDThreads, 3) k_apply_entries(const IxArgs a) {
+__global__ void __launch_bounds__(kDThreads, TLC_SUM_MINB) k_apply_entries(const IxArgs a) {
   extern __shared__ __align__(16) uint8_t dyn_s[];  // mask bytes, then digit words
   __shared__ float scale_s[kK];
   __shared__ const uint32_t *list_s[kK];  // per-lane stream choice: read from shared memory
@@ -1385,7 +1393,7 @@ __global__ void __launch_bounds__(kDThreads, 3) k_apply_entries(const IxArgs a) 
       if (i < gn && mb[i]) todo |= 1u << j;
     }
     while (todo) {
-      constexpr int kAt = 4;
+      constexpr int kAt = TLC_SUM_AT;
       uint32_t gi[kAt], tch[kAt];
 #pragma unroll
       for (int q = 0; q < kAt; ++q) {
