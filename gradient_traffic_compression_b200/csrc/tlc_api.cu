@@ -472,7 +472,7 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
 
   std::vector<tlc::BatchTensor> T(count);
   std::vector<tlc::BatchChunk> chunks;
-  std::vector<uint32_t> qtt, dtt;
+  std::vector<uint32_t> qtt, dtt, qct;
   std::vector<uint64_t> offsets(count + 1, 0);
   uint64_t n_dchunks = 0, n_qchunks = 0;
   for (int i = 0; i < count; ++i) {
@@ -490,6 +490,7 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
     for (uint32_t k = 0; k < t.q_tiles; ++k) qtt.push_back((uint32_t)i);
     t.q_chunk_begin = (uint32_t)n_qchunks;
     n_qchunks += tlc::compress_place_chunks(t.q_tiles);
+    for (uint32_t k = 0; k < tlc::compress_place_chunks(t.q_tiles); ++k) qct.push_back((uint32_t)i);
     t.d_tile_begin = (uint32_t)dtt.size();
     t.d_tiles = tlc::decode_tiles_max(t.cap, t.groups);  // 512-byte units
     for (uint32_t k = 0; k < t.d_tiles; ++k) dtt.push_back((uint32_t)i);
@@ -525,8 +526,9 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   const bool q_def = xs && tlc::compress_deferred_tiles(qtt.size());
   const size_t sz_QC = q_def ? tlc::align_up(8 * n_qchunks, 256) : 0;
   const size_t sz_QT = q_def ? (size_t)tlc::compress_stage_bytes_per_tile() * qtt.size() : 0;
+  const size_t sz_QCT = q_def ? tlc::align_up(4 * n_qchunks, 256) : 0;  // each chunk's tensor
   const size_t total = sz_T + sz_C + sz_Q + sz_D + sz_M + sz_QS + sz_DS + sz_P + 256 + sz_E +
-                       sz_S + sz_QC + sz_QT;
+                       sz_S + sz_QC + sz_QT + sz_QCT;
   tlc_plan_s *P = new tlc_plan_s();
   P->device = dev->device;
   P->count = count;
@@ -570,6 +572,8 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
   D.q_stage = q_def ? reinterpret_cast<uint8_t *>(zd + sz_DS + sz_P + 256 + sz_E + sz_S + sz_QC)
                     : nullptr;
   D.n_q_chunks = (uint32_t)n_qchunks;
+  uint32_t *qct_dev = q_def ? reinterpret_cast<uint32_t *>(b + total - sz_QCT) : nullptr;
+  D.q_chunk_tensor = qct_dev;
   ce = cudaMemcpy(b, T.data(), sizeof(tlc::BatchTensor) * count, cudaMemcpyHostToDevice);
   if (ce == cudaSuccess && !chunks.empty())
     ce = cudaMemcpy(b + sz_T, chunks.data(), sizeof(tlc::BatchChunk) * chunks.size(),
@@ -578,6 +582,8 @@ tlc_status tlc_plan_create(int count, const size_t *ns, const float *const *xs,
     ce = cudaMemcpy(b + sz_T + sz_C, qtt.data(), 4 * qtt.size(), cudaMemcpyHostToDevice);
   if (ce == cudaSuccess)
     ce = cudaMemcpy(b + sz_T + sz_C + sz_Q, dtt.data(), 4 * dtt.size(), cudaMemcpyHostToDevice);
+  if (ce == cudaSuccess && q_def)
+    ce = cudaMemcpy(qct_dev, qct.data(), 4 * qct.size(), cudaMemcpyHostToDevice);
   if (ce != cudaSuccess) {
     cudaFree(P->dmem);
     delete P;

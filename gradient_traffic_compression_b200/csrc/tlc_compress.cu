@@ -283,21 +283,24 @@ __device__ __forceinline__ ZScan zshfl_up(const ZScan &v, int d) {
   return r;
 }
 
-// The summary of a chunk of kPlaceTiles tiles in 64 bits (A, R < 2^20), as
-// the deferred path stores it per chunk.
+// The summary of a chunk of kPlaceTiles tiles, or of a span of kPlaceSpan
+// chunks, in 64 bits (A, R < 2^24: a segment emits at most one byte per
+// group), as the deferred path stores it.
 constexpr int kPlaceTiles = 32;
-static_assert((uint64_t)kPlaceTiles * kTileGroups < (1u << 20), "chunk A and R fit in 20 bits");
+constexpr int kPlaceSpan = 32;
+static_assert((uint64_t)kPlaceSpan * kPlaceTiles * kTileGroups < (1u << 24),
+              "span A and R fit in 24 bits");
 struct ChunkCodec {
   __device__ static uint64_t pack(const ZAgg &a) {
-    return (uint64_t)a.A | ((uint64_t)a.R << 20) | ((uint64_t)a.tc << 40) |
-           ((uint64_t)a.all << 44);
+    return (uint64_t)a.A | ((uint64_t)a.R << 24) | ((uint64_t)a.tc << 48) |
+           ((uint64_t)a.all << 52);
   }
   __device__ static ZAgg unpack(uint64_t w) {
     ZAgg a;
-    a.A = (uint32_t)(w & 0xfffffu);
-    a.R = (uint32_t)((w >> 20) & 0xfffffu);
-    a.tc = (uint32_t)((w >> 40) & 0xfu);
-    a.all = (uint32_t)((w >> 44) & 1u);
+    a.A = (uint32_t)(w & 0xffffffu);
+    a.R = (uint32_t)((w >> 24) & 0xffffffu);
+    a.tc = (uint32_t)((w >> 48) & 0xfu);
+    a.all = (uint32_t)((w >> 52) & 1u);
     return a;
   }
 };
@@ -322,7 +325,9 @@ struct DeferJob {
   uint32_t *aggs;     // each tile's summary (pack_agg32),
   uint8_t *stage;     // kTileGroups staged bytes per tile,
   uint32_t *ccount;   // finished tiles per 32-tile chunk (starts at 0),
-  uint64_t *cagg;     // and each chunk's summary (ChunkCodec)
+  uint64_t *cagg;     // each chunk's summary (ChunkCodec),
+  uint32_t *scount;   // or nullptr: finished chunks per 32-chunk span (starts at 0)
+  uint64_t *sagg;     // and each span's summary (ChunkCodec)
 };
 
 // Shared memory of one compress block.
@@ -779,7 +784,33 @@ __device__ __forceinline__ void quant_tile(const TileJob &j, const DeferJob &dj,
         const ZScan o = zshfl_up(v, d);
         if (lane >= d) v = zcombine(o, v);
       }
-      if (lane == 31) dj.cagg[c] = ChunkCodec::pack(v.a);
+      const uint64_t cw = ChunkCodec::pack(v.a);  // lane 31: the chunk's summary
+      if (lane == 31) dj.cagg[c] = cw;
+      if (dj.scount) {
+        // The same one level up: the last chunk of a 32-chunk span to be
+        // summed up sums up the span.
+        const uint32_t sp = c / kPlaceSpan;
+        const uint32_t n_chunks = (j.n_tiles + kPlaceTiles - 1) / kPlaceTiles;
+        uint32_t slast = 0;
+        if (lane == 31) {
+          const uint32_t size = (uint32_t)umin64(kPlaceSpan, n_chunks - sp * kPlaceSpan);
+          __threadfence();
+          slast = atomicAdd(dj.scount + sp, 1u) == size - 1 ? 1u : 0u;
+        }
+        if (__shfl_sync(0xffffffffu, slast, 31)) {
+          __threadfence();
+          const uint32_t cc = sp * kPlaceSpan + lane;
+          const uint64_t own = __shfl_sync(0xffffffffu, cw, 31);
+          ZScan w = {0u, {0u, 0u, 0u, 0u}};
+          if (cc < n_chunks) w = {1u, ChunkCodec::unpack(cc == c ? own : __ldcg(dj.cagg + cc))};
+#pragma unroll
+          for (int d = 1; d < 32; d <<= 1) {
+            const ZScan o = zshfl_up(w, d);
+            if (lane >= d) w = zcombine(o, w);
+          }
+          if (lane == 31) dj.sagg[sp] = ChunkCodec::pack(w.a);
+        }
+      }
     }
   }
 }
@@ -799,8 +830,10 @@ struct QuantArgs {
   uint32_t *aggs;    // deferred placement only: tile summaries,
   uint8_t *stage;    // staged bytes,
   uint32_t *ok;      // 1 if the step is finite (written by block 0),
-  uint32_t *ccount;  // chunk counters and
-  uint64_t *cagg;    // chunk summaries
+  uint32_t *ccount;  // chunk counters,
+  uint64_t *cagg;    // chunk summaries,
+  uint32_t *scount;  // span counters and
+  uint64_t *sagg;    // span summaries
   const float *x;
   float *err;
   uint64_t n;
@@ -863,7 +896,7 @@ __global__ void TLC_Q_BOUNDS k_quant_zre(const QuantArgs a) {
   const float scale = scale_s, thr = thr_s;
   const TileJob job = {a.x, a.err, a.n, a.groups, a.out, a.out_cap, a.out_len,
                        a.status, a.n_tiles, kVec, kRecord ? a.rec : nullptr};
-  const DeferJob djob = {a.aggs, a.stage, a.ccount, a.cagg};
+  const DeferJob djob = {a.aggs, a.stage, a.ccount, a.cagg, a.scount, a.sagg};
   for (;;) {
     if (threadIdx.x == 0) tile_id_s = atomicAdd(a.ticket, 1u);
     __syncthreads();
@@ -912,92 +945,55 @@ __device__ __forceinline__ void warp_copy(uint8_t *dst, const uint8_t *__restric
   if (ts + lane < len) dst[ts + lane] = src[ts + lane];
 }
 
-// Put the tiles' output in place, one block per kPlaceBlockTiles tiles of
-// one 32-tile chunk.  Warp 0 composes the summaries of all earlier chunks
-// (each lane a contiguous share, then a warp scan) into the chunk's incoming
-// prefix, scans the chunk's own tile summaries, and keeps the exclusive
-// prefixes of the block's tiles; then each warp writes one tile: the
-// leading run's bytes (full 14-chunks as 255, then, if the run ends in the
-// tile, its remainder byte) and the staged bytes.  The block of the last
-// tile writes the closing remainder and the length.  No block waits on
-// another.
-constexpr int kPlaceBlockTiles = 4;
-constexpr int kPlaceThreads = kPlaceBlockTiles * kWarp;
-static_assert(kPlaceTiles % kPlaceBlockTiles == 0, "blocks do not straddle chunks");
-__global__ void __launch_bounds__(kPlaceThreads)
-k_zre_place(const uint32_t *__restrict__ aggs, const uint64_t *__restrict__ cagg,
-            uint32_t n_tiles, const uint32_t *ok, const uint8_t *__restrict__ stage, uint8_t *out,
-            uint64_t out_cap, uint64_t *out_len, CompressRecord *rec) {
-  __shared__ uint32_t tC[kPlaceBlockTiles], tT[kPlaceBlockTiles], tA[kPlaceBlockTiles];
-  pdl_enter();
-  if (!*ok) return;  // non-finite step: nothing was encoded
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t b0 = blockIdx.x * kPlaceBlockTiles;  // the block's first tile
-  const uint32_t c = b0 / kPlaceTiles;
-  const uint32_t t0 = c * kPlaceTiles;
-  const uint32_t nv = (uint32_t)umin64(kPlaceTiles, n_tiles - t0);
-  if (warp == 0) {
-    // chunks [0, c): lane l folds [l * per, (l + 1) * per), loads first
-    const uint32_t per = (c + kWarp - 1) / kWarp;
-    ZScan p = {0u, {0u, 0u, 0u, 0u}};
-    const uint32_t pe = (uint32_t)umin64((uint64_t)(lane + 1) * per, c);
-    for (uint32_t i0 = lane * per; i0 < pe; i0 += 8) {
-      uint64_t w8[8];
+// The incoming prefix (emitted count C, run length mod 14) of chunk c:
+// warp 0 composes the summaries of all earlier spans (each lane a
+// contiguous share) and of the span's earlier chunks (one per lane), each by
+// a warp scan.  Every lane returns the same prefix.
+__device__ __forceinline__ void chunk_prefix(const uint64_t *__restrict__ cagg,
+                                             const uint64_t *__restrict__ sagg, uint32_t c,
+                                             int lane, uint32_t &C, uint32_t &tt) {
+  const uint32_t sp = c / kPlaceSpan;
+  const uint32_t per = (sp + kWarp - 1) / kWarp;
+  const uint32_t pe = (uint32_t)umin64((uint64_t)(lane + 1) * per, sp);
+  const uint32_t cc = sp * kPlaceSpan + lane;
+  const uint64_t cw = cc < c ? cagg[cc] : 0;
+  ZScan p = {0u, {0u, 0u, 0u, 0u}};
+  for (uint32_t i = lane * per; i < pe; ++i) p = zcombine(p, {1u, ChunkCodec::unpack(sagg[i])});
+  ZScan q = {0u, {0u, 0u, 0u, 0u}};
+  if (cc < c) q = {1u, ChunkCodec::unpack(cw)};
 #pragma unroll
-      for (int k = 0; k < 8; ++k) w8[k] = i0 + k < pe ? cagg[i0 + k] : 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k)
-        if (i0 + k < pe) p = zcombine(p, {1u, ChunkCodec::unpack(w8[k])});
-    }
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const ZScan o = zshfl_up(p, d);
-      if (lane >= d) p = zcombine(o, p);
-    }
-    uint32_t C = 0, tt = 0;
-    if (__shfl_sync(0xffffffffu, p.valid, 31)) {
-      ZAgg pa;
-      pa.all = __shfl_sync(0xffffffffu, p.a.all, 31);
-      pa.A = __shfl_sync(0xffffffffu, p.a.A, 31);
-      pa.R = __shfl_sync(0xffffffffu, p.a.R, 31);
-      pa.tc = __shfl_sync(0xffffffffu, p.a.tc, 31);
-      eval_agg(C, tt, pa);
-    }
-    // the chunk's own tiles, one per lane
-    uint32_t w = 0;
-    ZScan v = {0u, {0u, 0u, 0u, 0u}};
-    if ((uint32_t)lane < nv) {
-      w = aggs[t0 + lane];
-      v = {1u, unpack_agg32(w)};
-    }
-    ZScan inc = v;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const ZScan o = zshfl_up(inc, d);
-      if (lane >= d) inc = zcombine(o, inc);
-    }
-    ZScan exc = zshfl_up(inc, 1);
-    if (lane == 0) exc.valid = 0;
-    if (exc.valid) eval_agg(C, tt, exc.a);
-    const uint32_t k = t0 + lane - b0;  // this lane's tile within the block
-    if (k < kPlaceBlockTiles) {
-      tC[k] = C;
-      tT[k] = tt;
-      tA[k] = w;
-    }
-    if (t0 + nv == n_tiles && (uint32_t)lane == nv - 1 && k < kPlaceBlockTiles) {
-      // the stream's end: state after the last tile
-      eval_agg(C, tt, v.a);
-      if (tt && TLC_BOUND(4ull + C < out_cap)) out[4 + C] = remainder_byte(tt);
-      *out_len = 4ull + C + (tt ? 1u : 0u);
-      if (rec) rec->length = 4ull + C + (tt ? 1u : 0u);
-    }
+  for (int d = 1; d < 32; d <<= 1) {
+    const ZScan o = zshfl_up(p, d);
+    if (lane >= d) p = zcombine(o, p);
+    const ZScan oq = zshfl_up(q, d);
+    if (lane >= d) q = zcombine(oq, q);
   }
-  __syncthreads();
-  const uint32_t t = b0 + warp;
-  if (t >= n_tiles) return;
-  const ZAgg a = unpack_agg32(tA[warp]);
-  const uint32_t C = tC[warp], tin = tT[warp];
+  C = 0;
+  tt = 0;
+  if (__shfl_sync(0xffffffffu, p.valid, 31)) {
+    ZAgg pa;
+    pa.all = __shfl_sync(0xffffffffu, p.a.all, 31);
+    pa.A = __shfl_sync(0xffffffffu, p.a.A, 31);
+    pa.R = __shfl_sync(0xffffffffu, p.a.R, 31);
+    pa.tc = __shfl_sync(0xffffffffu, p.a.tc, 31);
+    eval_agg(C, tt, pa);
+  }
+  if (__shfl_sync(0xffffffffu, q.valid, 31)) {
+    ZAgg qa;
+    qa.all = __shfl_sync(0xffffffffu, q.a.all, 31);
+    qa.A = __shfl_sync(0xffffffffu, q.a.A, 31);
+    qa.R = __shfl_sync(0xffffffffu, q.a.R, 31);
+    qa.tc = __shfl_sync(0xffffffffu, q.a.tc, 31);
+    eval_agg(C, tt, qa);
+  }
+}
+
+// One tile's bytes in place, by one warp: the leading run's bytes (full
+// 14-chunks as 255, then, if the run ends in the tile, its remainder byte)
+// and the staged bytes, from the tile's incoming prefix (C, tin).
+__device__ __forceinline__ void place_tile(const ZAgg &a, uint32_t C, uint32_t tin,
+                                           const uint8_t *__restrict__ staged, uint8_t *out,
+                                           uint64_t out_cap, int lane) {
   const uint32_t lead = lead_count(a, tin);
   const uint32_t r = (tin + a.A) % 14u;
   const bool rem = !a.all && r;  // the run ends in the tile with a remainder
@@ -1006,9 +1002,70 @@ k_zre_place(const uint32_t *__restrict__ aggs, const uint64_t *__restrict__ cagg
   (void)TLC_CHECK((uint64_t)lead + a.R <= room);  // the tile's bytes fit the stream
   warp_fill_255(o, (uint32_t)umin64(lead - (rem ? 1u : 0u), room), lane);
   if (rem && lane == 0 && TLC_BOUND(lead - 1 < room)) o[lead - 1] = remainder_byte(r);
-  if (lead < room)
-    warp_copy(o + lead, stage + (uint64_t)t * kTileGroups, (uint32_t)umin64(a.R, room - lead),
-              lane);
+  if (lead < room) warp_copy(o + lead, staged, (uint32_t)umin64(a.R, room - lead), lane);
+}
+
+// Warp 0 of a placement block: from the chunk's incoming prefix (C, tt),
+// scan the chunk's nv tile summaries (w: lane l's tile l) and keep each
+// tile's exclusive prefix and summary in shared memory.  Lane nv - 1 gets
+// back in (C, tt) the state after the chunk's last tile.
+__device__ __forceinline__ void scan_chunk_tiles(uint32_t w, uint32_t nv, int lane, uint32_t &C,
+                                                 uint32_t &tt, uint32_t *tC, uint32_t *tT,
+                                                 uint32_t *tA) {
+  ZScan v = {0u, {0u, 0u, 0u, 0u}};
+  if ((uint32_t)lane < nv) v = {1u, unpack_agg32(w)};
+  ZScan inc = v;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const ZScan o = zshfl_up(inc, d);
+    if (lane >= d) inc = zcombine(o, inc);
+  }
+  ZScan exc = zshfl_up(inc, 1);
+  if (lane == 0) exc.valid = 0;
+  if (exc.valid) eval_agg(C, tt, exc.a);
+  tC[lane] = C;
+  tT[lane] = tt;
+  tA[lane] = w;
+  if ((uint32_t)lane < nv) eval_agg(C, tt, v.a);
+}
+
+// Put the tiles' output in place, one block per 32-tile chunk.  Warp 0
+// finds the chunk's incoming prefix (chunk_prefix), scans the chunk's own
+// tile summaries (one per lane) and keeps every tile's exclusive prefix in
+// shared memory; then each warp places every kPlaceWarps-th tile of the
+// chunk.  The block of the last tile writes the closing remainder and the
+// length.  No block waits on another, and one wave of blocks covers 2^28
+// values (820 chunks).
+constexpr int kPlaceWarps = 8;
+constexpr int kPlaceThreads = kPlaceWarps * kWarp;
+__global__ void __launch_bounds__(kPlaceThreads)
+k_zre_place(const uint32_t *__restrict__ aggs, const uint64_t *__restrict__ cagg,
+            const uint64_t *__restrict__ sagg, uint32_t n_tiles, const uint32_t *ok,
+            const uint8_t *__restrict__ stage, uint8_t *out, uint64_t out_cap, uint64_t *out_len,
+            CompressRecord *rec) {
+  __shared__ uint32_t tC[kPlaceTiles], tT[kPlaceTiles], tA[kPlaceTiles];
+  pdl_enter();
+  if (!*ok) return;  // non-finite step: nothing was encoded
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t c = blockIdx.x;
+  const uint32_t t0 = c * kPlaceTiles;
+  const uint32_t nv = (uint32_t)umin64(kPlaceTiles, n_tiles - t0);
+  if (warp == 0) {
+    const uint32_t w = (uint32_t)lane < nv ? aggs[t0 + lane] : 0u;
+    uint32_t C, tt;
+    chunk_prefix(cagg, sagg, c, lane, C, tt);
+    scan_chunk_tiles(w, nv, lane, C, tt, tC, tT, tA);
+    if (t0 + nv == n_tiles && (uint32_t)lane == nv - 1) {
+      // the stream's end: state after the last tile
+      if (tt && TLC_BOUND(4ull + C < out_cap)) out[4 + C] = remainder_byte(tt);
+      *out_len = 4ull + C + (tt ? 1u : 0u);
+      if (rec) rec->length = 4ull + C + (tt ? 1u : 0u);
+    }
+  }
+  __syncthreads();
+  for (uint32_t k = warp; k < nv; k += kPlaceWarps)
+    place_tile(unpack_agg32(tA[k]), tC[k], tT[k], stage + (uint64_t)(t0 + k) * kTileGroups, out,
+               out_cap, lane);
 }
 
 // ------------------------------------------------- batched (tensor lists) --
@@ -1081,6 +1138,8 @@ struct BatchQuantArgs {
   uint32_t *ccount;
   uint64_t *cagg;
   uint8_t *stage;
+  const uint32_t *chunk_tensor;  // tensor of each chunk (global numbering)
+  uint32_t n_chunks;
 };
 
 // Quantize + encode over a list of tensors: tiles of all tensors in one
@@ -1116,7 +1175,8 @@ __global__ void TLC_Q_BOUNDS k_quant_zre_batch(const BatchQuantArgs a) {
     if (kDeferred) {
       const DeferJob dj = {a.aggs + T.q_tile_begin,
                            a.stage + (uint64_t)T.q_tile_begin * kTileGroups,
-                           a.ccount + T.q_chunk_begin, a.cagg + T.q_chunk_begin};
+                           a.ccount + T.q_chunk_begin, a.cagg + T.q_chunk_begin, nullptr,
+                           nullptr};
       quant_tile<true>(job, dj, t, scale, thr, sm, a.dev_status, a.max_polls);
     } else {
       quant_tile<false>(job, DeferJob{}, t, scale, thr, sm, a.dev_status, a.max_polls);
@@ -1124,86 +1184,60 @@ __global__ void TLC_Q_BOUNDS k_quant_zre_batch(const BatchQuantArgs a) {
   }
 }
 
-// Deferred placement over a list of tensors, one warp per tile (global
-// numbering): the warp finds its tensor, composes the summaries of the
-// tensor's earlier 32-tile chunks, scans its own chunk, and writes its
-// tile's leading run and staged bytes; the warp of a tensor's last tile
-// writes the closing remainder byte and the length.  Tensors whose step is
-// non-finite are skipped (k_quant_zre_batch set their length to 0).
+// Deferred placement over a list of tensors, one block per 32-tile chunk
+// (all tensors' chunks in one numbering, chunk_tensor naming each one's
+// tensor): warp 0 composes the summaries of the tensor's earlier chunks
+// (each lane a contiguous share, then a warp scan) and scans the chunk's
+// tiles, then each warp places every kPlaceWarps-th tile of the chunk.  The
+// block of a tensor's last tile writes the closing remainder byte and the
+// length.  Tensors whose step is non-finite are skipped (k_quant_zre_batch
+// set their length to 0).
 __global__ void __launch_bounds__(kPlaceThreads) k_zre_place_batch(const BatchQuantArgs a) {
+  __shared__ uint32_t tC[kPlaceTiles], tT[kPlaceTiles], tA[kPlaceTiles];
   pdl_enter();
-  const int lane = threadIdx.x & 31;
-  const uint32_t u = blockIdx.x * (kPlaceThreads / kWarp) + (threadIdx.x >> 5);
-  if (u >= a.n_tiles) return;  // whole warp
-  const uint32_t id = a.tile_tensor[u];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t id = a.chunk_tensor[blockIdx.x];
   const BatchTensor &T = a.tensors[id];
   float scale = 0.0f, thr = 0.0f;
-  if (!scale_from_max(a.mbits[id], a.s, scale, thr)) return;
-  const uint32_t t = u - T.q_tile_begin;
-  const uint32_t c = t / kPlaceTiles;
+  if (!scale_from_max(a.mbits[id], a.s, scale, thr)) return;  // whole block
+  const uint32_t c = blockIdx.x - T.q_chunk_begin;
   const uint32_t t0 = c * kPlaceTiles;
   const uint32_t nv = (uint32_t)umin64(kPlaceTiles, T.q_tiles - t0);
-  const uint32_t *aggs = a.aggs + T.q_tile_begin;
-  const uint64_t *cagg = a.cagg + T.q_chunk_begin;
-  // chunks [0, c) of this tensor: lane l folds [l * per, (l + 1) * per)
-  const uint32_t per = (c + kWarp - 1) / kWarp;
-  ZScan p = {0u, {0u, 0u, 0u, 0u}};
-  const uint32_t pe = (uint32_t)umin64((uint64_t)(lane + 1) * per, c);
-  for (uint32_t i = lane * per; i < pe; ++i) p = zcombine(p, {1u, ChunkCodec::unpack(cagg[i])});
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const ZScan o = zshfl_up(p, d);
-    if (lane >= d) p = zcombine(o, p);
-  }
-  uint32_t C = 0, tt = 0;
-  if (__shfl_sync(0xffffffffu, p.valid, 31)) {
-    ZAgg pa;
-    pa.all = __shfl_sync(0xffffffffu, p.a.all, 31);
-    pa.A = __shfl_sync(0xffffffffu, p.a.A, 31);
-    pa.R = __shfl_sync(0xffffffffu, p.a.R, 31);
-    pa.tc = __shfl_sync(0xffffffffu, p.a.tc, 31);
-    eval_agg(C, tt, pa);
-  }
-  // the chunk's tiles, one per lane; this tile is lane t - t0
-  uint32_t w = 0;
-  ZScan v = {0u, {0u, 0u, 0u, 0u}};
-  if ((uint32_t)lane < nv) {
-    w = aggs[t0 + lane];
-    v = {1u, unpack_agg32(w)};
-  }
-  ZScan inc = v;
-#pragma unroll
-  for (int d = 1; d < 32; d <<= 1) {
-    const ZScan o = zshfl_up(inc, d);
-    if (lane >= d) inc = zcombine(o, inc);
-  }
-  ZScan exc = zshfl_up(inc, 1);
-  if (lane == 0) exc.valid = 0;
-  if (exc.valid) eval_agg(C, tt, exc.a);
-  const int me = (int)(t - t0);
-  C = __shfl_sync(0xffffffffu, C, me);
-  tt = __shfl_sync(0xffffffffu, tt, me);
-  w = __shfl_sync(0xffffffffu, w, me);
-  const ZAgg ag = unpack_agg32(w);
   uint8_t *out = a.arena + T.arena_off;
   const uint64_t out_cap = T.cap;
-  if (t == T.q_tiles - 1 && lane == 0) {
-    uint32_t Ce = C, te = tt;
-    eval_agg(Ce, te, ag);
-    if (te && TLC_BOUND(4ull + Ce < out_cap)) out[4 + Ce] = remainder_byte(te);
-    a.out_lens[id] = 4ull + Ce + (te ? 1u : 0u);
+  if (warp == 0) {
+    const uint32_t *aggs = a.aggs + T.q_tile_begin;
+    const uint64_t *cagg = a.cagg + T.q_chunk_begin;
+    const uint32_t w = (uint32_t)lane < nv ? aggs[t0 + lane] : 0u;
+    // chunks [0, c) of this tensor: lane l folds [l * per, (l + 1) * per)
+    const uint32_t per = (c + kWarp - 1) / kWarp;
+    ZScan p = {0u, {0u, 0u, 0u, 0u}};
+    const uint32_t pe = (uint32_t)umin64((uint64_t)(lane + 1) * per, c);
+    for (uint32_t i = lane * per; i < pe; ++i) p = zcombine(p, {1u, ChunkCodec::unpack(cagg[i])});
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const ZScan o = zshfl_up(p, d);
+      if (lane >= d) p = zcombine(o, p);
+    }
+    uint32_t C = 0, tt = 0;
+    if (__shfl_sync(0xffffffffu, p.valid, 31)) {
+      ZAgg pa;
+      pa.all = __shfl_sync(0xffffffffu, p.a.all, 31);
+      pa.A = __shfl_sync(0xffffffffu, p.a.A, 31);
+      pa.R = __shfl_sync(0xffffffffu, p.a.R, 31);
+      pa.tc = __shfl_sync(0xffffffffu, p.a.tc, 31);
+      eval_agg(C, tt, pa);
+    }
+    scan_chunk_tiles(w, nv, lane, C, tt, tC, tT, tA);
+    if (t0 + nv == T.q_tiles && (uint32_t)lane == nv - 1) {
+      if (tt && TLC_BOUND(4ull + C < out_cap)) out[4 + C] = remainder_byte(tt);
+      a.out_lens[id] = 4ull + C + (tt ? 1u : 0u);
+    }
   }
-  const uint32_t lead = lead_count(ag, tt);
-  const uint32_t r = (tt + ag.A) % 14u;
-  const bool rem = !ag.all && r;
-  uint8_t *o = out + 4ull + C;
-  const uint64_t room = out_cap > 4ull + C ? out_cap - 4ull - C : 0;
-  (void)TLC_CHECK((uint64_t)lead + ag.R <= room);  // the tile's bytes fit the stream
-  warp_fill_255(o, (uint32_t)umin64(lead - (rem ? 1u : 0u), room), lane);
-  if (rem && lane == 0 && TLC_BOUND(lead - 1 < room)) o[lead - 1] = remainder_byte(r);
-  if (lead < room)
-    warp_copy(o + lead, a.stage + (uint64_t)u * kTileGroups, (uint32_t)umin64(ag.R, room - lead),
-              lane);
+  __syncthreads();
+  for (uint32_t k = warp; k < nv; k += kPlaceWarps)
+    place_tile(unpack_agg32(tA[k]), tC[k], tT[k],
+               a.stage + (uint64_t)(T.q_tile_begin + t0 + k) * kTileGroups, out, out_cap, lane);
 }
 
 // Wait-limit check of the compress look-back: tile 1 looks back at a tile 0
@@ -1248,6 +1282,10 @@ bool compress_deferred_tiles(uint64_t n_tiles) { return n_tiles >= kDeferMinTile
 uint32_t compress_stage_bytes_per_tile() { return kTileGroups; }
 
 uint32_t compress_place_chunks(uint32_t n_tiles) { return (n_tiles + kPlaceTiles - 1) / kPlaceTiles; }
+
+uint32_t compress_place_spans(uint32_t n_tiles) {
+  return (compress_place_chunks(n_tiles) + kPlaceSpan - 1) / kPlaceSpan;
+}
 
 cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, float s,
                             float *err, uint8_t *out, uint64_t out_cap, uint64_t *out_len,
@@ -1297,14 +1335,19 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
   qa.ok = nullptr;
   qa.ccount = nullptr;
   qa.cagg = nullptr;
+  qa.scount = nullptr;
+  qa.sagg = nullptr;
   DeferredScratch ds = {};
   if (deferred) {
     ds = deferred_scratch_layout(scratch, n_part, n_tiles);
     qa.stage = ds.stage;
     qa.ok = ds.ok;
     qa.cagg = ds.cagg;
-    // the chunk counters follow the summaries in the (cleared) status area
+    qa.sagg = ds.sagg;
+    // the chunk counters, then the span counters, follow the summaries in
+    // the (cleared) status area: n_tiles + chunks + spans < 2 * n_tiles
     qa.ccount = qa.aggs + n_tiles;
+    qa.scount = qa.ccount + compress_place_chunks(n_tiles);
   }
 
   int occ = vec ? dev.occ_quant_vec : dev.occ_quant_scalar;
@@ -1321,9 +1364,8 @@ cudaError_t launch_compress(const DeviceInfo &dev, const float *x, uint64_t n, f
       launch_k(k_quant_zre<false, true>, grid, kQThreads, 0, stream, qa);
     timing_end(kKindQuantZre, stream);
     timing_begin(kKindZrePlace, stream);
-    const uint32_t n_blocks = (n_tiles + kPlaceBlockTiles - 1) / kPlaceBlockTiles;
-    launch_k(k_zre_place, n_blocks, kPlaceThreads, 0, stream, qa.aggs, ds.cagg, n_tiles, ds.ok,
-             ds.stage, out, out_cap, out_len, rec);
+    launch_k(k_zre_place, compress_place_chunks(n_tiles), kPlaceThreads, 0, stream, qa.aggs,
+             ds.cagg, ds.sagg, n_tiles, ds.ok, ds.stage, out, out_cap, out_len, rec);
     timing_end(kKindZrePlace, stream);
   } else {
     if (rec)
@@ -1365,6 +1407,8 @@ cudaError_t launch_compress_batch(const DeviceInfo &dev, const BatchPlanDev &p, 
   qa.ccount = qa.aggs + p.n_q_tiles;
   qa.cagg = p.q_cagg;
   qa.stage = p.q_stage;
+  qa.chunk_tensor = p.q_chunk_tensor;
+  qa.n_chunks = p.n_q_chunks;
   uint32_t grid = (uint32_t)dev.sm_count * (uint32_t)(dev.occ_quant_batch > 0 ? dev.occ_quant_batch : 1);
   if (grid > p.n_q_tiles) grid = p.n_q_tiles;
   timing_begin(kKindQuantZre, stream);
@@ -1374,10 +1418,8 @@ cudaError_t launch_compress_batch(const DeviceInfo &dev, const BatchPlanDev &p, 
     launch_k(k_quant_zre_batch<false>, grid, kQThreads, 0, stream, qa);
   timing_end(kKindQuantZre, stream);
   if (p.q_deferred) {
-    const uint32_t per_block = kPlaceThreads / kWarp;
     timing_begin(kKindZrePlace, stream);
-    launch_k(k_zre_place_batch, (p.n_q_tiles + per_block - 1) / per_block, kPlaceThreads, 0,
-             stream, qa);
+    launch_k(k_zre_place_batch, p.n_q_chunks, kPlaceThreads, 0, stream, qa);
     timing_end(kKindZrePlace, stream);
   }
   return cudaGetLastError();

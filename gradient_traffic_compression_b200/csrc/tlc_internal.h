@@ -61,22 +61,27 @@ inline CompressScratch compress_scratch_layout(void *base, uint32_t n_part, uint
 }
 
 // The deferred-placement path appends, after the look-back layout (whose
-// status words hold the tiles' summaries and the chunk counters there): the
-// placement chunks' summaries (compress_place_chunks u64), a finite-step
-// word, and a staging slot of compress_stage_bytes_per_tile() bytes per tile.
+// status words hold the tiles' summaries and the chunk and span counters
+// there): the placement chunks' summaries (compress_place_chunks u64), the
+// spans' summaries (compress_place_spans u64), a finite-step word, and a
+// staging slot of compress_stage_bytes_per_tile() bytes per tile.
 struct DeferredScratch {
   uint64_t *cagg;
+  uint64_t *sagg;
   uint32_t *ok;
   uint8_t *stage;
 };
 
 // Staging bytes per tile of the deferred-placement path (one tile's groups).
 uint32_t compress_stage_bytes_per_tile();
-// Placement chunks of the deferred path for n_tiles tiles.
+// Placement chunks (32 tiles) and spans (32 chunks) of the deferred path
+// for n_tiles tiles.
 uint32_t compress_place_chunks(uint32_t n_tiles);
+uint32_t compress_place_spans(uint32_t n_tiles);
 
 inline size_t deferred_head_bytes(uint32_t n_tiles) {
-  return align_up(8 * (size_t)compress_place_chunks(n_tiles) + 4, 256);
+  return align_up(8 * ((size_t)compress_place_chunks(n_tiles) + compress_place_spans(n_tiles)) + 4,
+                  256);
 }
 
 inline size_t deferred_scratch_bytes(uint32_t n_part, uint32_t n_tiles) {
@@ -88,7 +93,8 @@ inline DeferredScratch deferred_scratch_layout(void *base, uint32_t n_part, uint
   DeferredScratch d;
   char *p = static_cast<char *>(base) + compress_scratch_bytes(n_part, n_tiles);
   d.cagg = reinterpret_cast<uint64_t *>(p);
-  d.ok = reinterpret_cast<uint32_t *>(d.cagg + compress_place_chunks(n_tiles));
+  d.sagg = d.cagg + compress_place_chunks(n_tiles);
+  d.ok = reinterpret_cast<uint32_t *>(d.sagg + compress_place_spans(n_tiles));
   d.stage = reinterpret_cast<uint8_t *>(p + deferred_head_bytes(n_tiles));
   return d;
 }
@@ -156,6 +162,7 @@ struct BatchPlanDev {
   uint64_t *q_cagg;       // deferred placement: per 32-tile chunk summaries,
   uint8_t *q_stage;       // and the staged bytes, compress_stage_bytes_per_tile() per tile;
   uint32_t n_q_chunks;    // tile summaries and chunk counters sit in q_status
+  const uint32_t *q_chunk_tensor;  // deferred placement: the tensor of each chunk
   uint32_t *d_loc;        // indexed plans: units' first groups within their chunk (per
                           // tensor d_tiles words from d_tile_begin)
   uint32_t *d_cpre;       // and chunks' first groups (per tensor d_chunks + 1 words from

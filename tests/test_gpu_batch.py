@@ -227,11 +227,12 @@ def test_batch_counting_pass_large_plan(g):
 
 
 def test_batch_deferred_placement_many_tensors(g):
-    # 384 compress tiles or more in total: every tensor's tiles stage their
-    # bytes and a placement kernel writes the streams; small tensors of one
-    # tile sit beside a large one, one of them non-finite
+    # 768 compress tiles (of 10240 values) or more in total: every tensor's
+    # tiles stage their bytes and a placement kernel writes the streams;
+    # small tensors of a few tiles sit beside a large one of 35 placement
+    # chunks (32 tiles each) and a ragged end, one of them non-finite
     rng_sizes = (synth.uniforms(synth.key_for(140, 0), 150) * 60_000).astype(np.int64) + 1
-    sizes = [int(v) for v in rng_sizes] + [384 * 20480 + 12345]
+    sizes = [int(v) for v in rng_sizes] + [(32 * 34 + 5) * 10240 + 12345]
     xs, errs = [], []
     for i, n in enumerate(sizes):
         x, e = mixed(150 + i, n, zero_frac=(0.5 + 0.45 * (i % 3) / 2), sigma=1e-3)

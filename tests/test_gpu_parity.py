@@ -544,6 +544,29 @@ def test_deferred_sparse_literals_every_tile(g):
     assert_roundtrip_parity(g, st, n)
 
 
+# Placement composes 32-tile chunks, and spans of 32 chunks, of tile
+# summaries; these runs cross chunk and span edges, cover a whole empty span,
+# and give every chunk a leading run that depends on all before it.
+CHUNK_GROUPS = 32 * TILE_GROUPS
+SPAN_GROUPS = 32 * CHUNK_GROUPS
+SPAN_CASES = {
+    "span_edge_mod0": [SPAN_GROUPS - 15, SPAN_GROUPS + 13],
+    "span_edge_mod13": [2 * SPAN_GROUPS - 14, 2 * SPAN_GROUPS + 12],
+    "chunk_and_span_ends": [CHUNK_GROUPS - 1, SPAN_GROUPS - 1, SPAN_GROUPS,
+                            3 * SPAN_GROUPS - 1],
+    "empty_span": [5, 2 * SPAN_GROUPS + 40],
+    "one_per_chunk": [c * CHUNK_GROUPS + (c * 7919) % CHUNK_GROUPS for c in range(3 * 32 + 1)],
+}
+
+
+@pytest.mark.parametrize("name", list(SPAN_CASES))
+def test_deferred_runs_across_spans(g, name):
+    n = 5 * (3 * SPAN_GROUPS + 37 * TILE_GROUPS + 11) + 2
+    x = _literal_groups_case(n, SPAN_CASES[name])
+    st, _ = assert_compress_parity(g, x, 1.0, np.zeros(n, np.float32))
+    assert_roundtrip_parity(g, st, n)
+
+
 def test_deferred_dense_and_nonfinite(g):
     n = DEFER_TILES * TILE_VALUES + 77
     x = (synth.uniforms(synth.key_for(7, 5), n) * 2 - 1).astype(np.float32)
