@@ -1000,6 +1000,14 @@ __global__ void __launch_bounds__(kScanThreads) k_index_scan(const IxArgs a) {
 constexpr uint32_t kWarpGroups = TLC_WARP_GROUPS;
 static_assert(kWarpGroups % 16 == 0, "whole swizzle blocks of digit words");
 constexpr uint32_t kZeroDigits2 = 0x01550155u;  // two digit words of the zero group 121
+// A unit's literal-group list in the accumulate mode's sparse case (fewer
+// than one literal group per 16 groups, so at most 14 * 512 / 16 entries)
+// sits in the warp's window, one word per entry; an entry of a group past
+// the tensor is kNoListEntry.
+constexpr uint32_t kListCap = (kWarpGroups + 16) / 2;
+static_assert(kListCap >= 14 * kDecodeUnit / 16, "a sparse unit's literal list fits the window");
+static_assert(14 * kDecodeUnit <= (1u << 13), "a group offset within a unit fits 13 bits");
+constexpr uint32_t kNoListEntry = 0xffffffffu;
 
 __device__ __forceinline__ uint64_t unit_first_group(const uint32_t *cpre, const uint32_t *loc,
                                                      uint32_t u) {
@@ -1060,35 +1068,57 @@ __device__ __forceinline__ void decode_unit(const DecodeJob &j, uint32_t u, cons
     return;
   }
   if (kMode == kAccumulate && 16 * L < E) {
-    // long zero runs around a few literals: visit the literal groups only
-    // (each group's values loaded before any is added)
-    uint64_t g = O + excl;
+    // long zero runs around a few literals: the warp lists the unit's
+    // literal groups in its window (in group order: the group's offset from
+    // O in bits 0..12, its digit word in bits 13..22), then each lane takes
+    // list entries i and i + 32 of every 64 and loads both groups' values
+    // before adding to either, so no lane walks a run of literals alone
+    uint32_t lpre = lits;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const uint32_t t = __shfl_up_sync(0xffffffffu, lpre, d);
+      if (lane >= d) lpre += t;
+    }
+    uint32_t *list = reinterpret_cast<uint32_t *>(wd);
+    uint32_t at = lpre - lits, rel = excl;
 #pragma unroll
     for (int k = 0; k < 16; ++k) {
       if (k < nb) {
         const uint32_t b = (w[k >> 2] >> (8 * (k & 3))) & 0xffu;
         if (b >= 243u) {
-          g += b - 241u;
+          rel += b - 241u;
         } else {
-          if (b != 121u && g < j.groups) {
-            const uint32_t dg = lut[b];
-            float v[5];
-#pragma unroll
-            for (int d = 0; d < 5; ++d) {
-              const uint64_t ei = 5 * g + d;
-              v[d] = (((dg >> (2 * d)) & 3u) != 1u && ei < j.n) ? j.y[ei] : 0.0f;
-            }
-#pragma unroll
-            for (int d = 0; d < 5; ++d) {
-              const uint32_t dig = (dg >> (2 * d)) & 3u;
-              const uint64_t ei = 5 * g + d;
-              if (dig != 1u && ei < j.n) j.y[ei] = __fadd_rn(v[d], dequant(dig, j.scale));
-            }
-          }
-          ++g;
+          if (b != 121u && TLC_CHECK(at < kListCap))
+            list[at++] = O + rel < j.groups ? rel | ((uint32_t)lut[b] << 13) : kNoListEntry;
+          ++rel;
         }
       }
     }
+    __syncwarp();
+    for (uint32_t i = lane; i < L; i += 2 * kWarp) {
+      const uint32_t ea = list[i];
+      const uint32_t eb = i + kWarp < L ? list[i + kWarp] : kNoListEntry;
+      // each group's values in acc and how many of its five exist (n may
+      // end inside the last group)
+      const uint64_t ea5 = 5 * (O + (ea & 0x1fffu)), eb5 = 5 * (O + (eb & 0x1fffu));
+      float *ya = j.y + ea5, *yb = j.y + eb5;
+      const uint32_t na = ea == kNoListEntry ? 0u : (uint32_t)umin64(5, j.n - ea5);
+      const uint32_t nb2 = eb == kNoListEntry ? 0u : (uint32_t)umin64(5, j.n - eb5);
+      const uint32_t da = ea >> 13, db = eb >> 13;
+      float va[5], vb[5];
+#pragma unroll
+      for (int d = 0; d < 5; ++d) {
+        va[d] = (((da >> (2 * d)) & 3u) != 1u && (uint32_t)d < na) ? ya[d] : 0.0f;
+        vb[d] = (((db >> (2 * d)) & 3u) != 1u && (uint32_t)d < nb2) ? yb[d] : 0.0f;
+      }
+#pragma unroll
+      for (int d = 0; d < 5; ++d) {
+        const uint32_t qa = (da >> (2 * d)) & 3u, qb = (db >> (2 * d)) & 3u;
+        if (qa != 1u && (uint32_t)d < na) ya[d] = __fadd_rn(va[d], dequant(qa, j.scale));
+        if (qb != 1u && (uint32_t)d < nb2) yb[d] = __fadd_rn(vb[d], dequant(qb, j.scale));
+      }
+    }
+    __syncwarp();  // the window is free again for the warp's next unit
     return;
   }
   for (uint32_t w0 = 0; w0 < Ec; w0 += kWarpGroups) {
