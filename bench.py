@@ -620,9 +620,11 @@ def run_e2e(args, tlc, torch, dev, xs_h, n, cap, world):
 # ------------------------------------------- tensor sets and K streams ----
 
 def run_config_set(args, rank, world, local):
-    """Configs 2 and 4 (per-layer tensors, one call per tensor, error buffers
-    carried) and 5 (K = 8 workers' streams summed).  Same legs and timing as
-    the headline; extra lines, not the headline workload."""
+    """Configs 2 and 4 (per-layer tensors, one plan call per leg or one call
+    per tensor, error buffers carried) and 5 (K = 8 workers' streams summed),
+    with a fresh gradient set every step (--grads seeded steps of the
+    workload, taken in turn).  Same legs and timing as the headline; extra
+    lines, not the headline workload."""
     import torch
     import torch.distributed as dist
 
@@ -634,12 +636,21 @@ def run_config_set(args, rank, world, local):
     dev = torch.device("cuda", local)
     cfg = synth.CONFIGS[args.config]
     s = cfg["s"]
-    if args.config == 5:
-        xs_h = [synth.flat_tensor(5, worker=w) for w in range(cfg["k"])]
-    else:
-        xs_h = synth.tensor_set(args.config, rank)
-    xs = [torch.from_numpy(a).to(dev) for a in xs_h]
-    ns = [a.size for a in xs_h]
+    # A fresh gradient set every step: the workload's steps 0 .. P-1 (each
+    # rank its own), resident on the device and taken in turn, while the
+    # error buffers carry over from step to step.
+    P = max(1, args.grads)
+    sets = []
+    for k in range(P):
+        st_k = 1000 * rank + k
+        if args.config == 5:
+            xs_h = [synth.flat_tensor(5, step=st_k, worker=w) for w in range(cfg["k"])]
+        else:
+            xs_h = synth.tensor_set(args.config, st_k)
+        sets.append([torch.from_numpy(a).to(dev) for a in xs_h])
+        ns = [a.size for a in xs_h]
+        del xs_h
+    cur = [0]   # the gradient set of the current step
     total = sum(ns)
     errs = [torch.zeros(n, dtype=torch.float32, device=dev) for n in ns]
     caps = [tlc.tlc_compress_bound(n) for n in ns]
@@ -657,20 +668,24 @@ def run_config_set(args, rank, world, local):
 
     use_plan = args.config in (2, 4) and not args.per_tensor
     if use_plan:
-        plan = tlc.Plan(xs, errs, ys)
-        arena = torch.empty(plan.arena_bytes, dtype=torch.uint8, device=dev)
+        # a plan binds its tensors: one per gradient set, all sharing the
+        # error buffers, the outputs and the arena
+        plans = [tlc.Plan(xs, errs, ys) for xs in sets]
+        arena = torch.empty(plans[0].arena_bytes, dtype=torch.uint8, device=dev)
         acc_plan = tlc.Plan(ys=accs)
 
     def leg_compress():
         if use_plan:
-            plan.compress(s, arena, lens, status, strm[0])
+            plans[cur[0]].compress(s, arena, lens, status, strm[0])
             return
+        xs = sets[cur[0]]
         for i in range(len(ns)):
             tlc.tlc_compress(xs[i], s, errs[i], outs[i], lens[i:i + 1], status, strm[0])
 
     def leg_decompress():
         if use_plan:
-            plan.decompress(arena, lens, accumulate=False, dev_status=status, stream=strm[0])
+            plans[0].decompress(arena, lens, accumulate=False, dev_status=status,
+                                stream=strm[0])
         elif args.config != 5:
             for i in range(len(ns)):
                 tlc.tlc_decompress(outs[i], ns[i], ys[i], in_len=lens[i:i + 1], in_cap=caps[i],
@@ -694,6 +709,7 @@ def run_config_set(args, rank, world, local):
         for fn in leg_fns:
             fn()
             yield
+        cur[0] = (cur[0] + 1) % P
 
     for _ in range(max(3, args.warmup)):
         for _ in legs():
@@ -705,6 +721,8 @@ def run_config_set(args, rank, world, local):
     # small tensor set, so that the GPU, not the host's launch rate, sets the
     # time), replayed in the timed region; launches counted while captured
     reps = (16 if total < (1 << 24) else 1) if args.graph else 1
+    if args.graph:
+        reps = -(-reps // P) * P   # whole turns of the gradient sets per replay
     leg_graphs = []
     if args.graph:
         tlc.tlc_kernel_timing_kinds([])
@@ -723,9 +741,11 @@ def run_config_set(args, rank, world, local):
         for fn in leg_fns:
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=cs):
-                for _ in range(reps):
+                for r in range(reps):
+                    cur[0] = r % P
                     fn()
             leg_graphs.append(gr)
+        cur[0] = 0
         strm[0] = stream
         graph.replay()
         torch.cuda.synchronize()
@@ -782,6 +802,9 @@ def run_config_set(args, rank, world, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic",
         "config": {"workload": cfg["name"], "tensors": len(ns), "values": total, "s": s,
+                   "inputs": (f"a fresh gradient set each step: the workload's steps 0..{P - 1}, "
+                              "resident on the device and taken in turn, error buffers "
+                              "carried"),
                    "calls": ("one plan call per leg (tlc_compress_batch / "
                              "tlc_decompress_batch)" if use_plan else
                              "one C-ABI call per tensor and leg")
