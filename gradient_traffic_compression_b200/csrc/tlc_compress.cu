@@ -22,14 +22,16 @@
 //                counter, so every tile a tile waits on is already running.
 // Tensors of 768 tiles and more take a third launch instead of the
 // per-tile look-back (the deferred-placement path): k_quant_zre tiles
-// write their summary and stage the bytes that follow their leading run,
-// and k_zre_place, one block per 32 tiles, scans the summaries (a
-// look-back over 32-tile chunks) and writes every tile's bytes in place.
+// write their summary and stage the bytes that follow their leading run;
+// the last tile of every 32-tile chunk to finish sums up the chunk, and the
+// last chunk of every 32-chunk span the span; then k_zre_place, one block
+// per chunk, composes the summaries before its chunk (spans, then chunks),
+// scans its tiles' and writes every tile's bytes in place.  Nothing waits.
 // The look-back inside k_quant_zre holds each tile's memory stream for a
 // round trip to earlier tiles; moving it to a kernel with no other work
 // measured 10-18% less time for the two kernels together than for the
 // look-back k_quant_zre from 2^23 to 2^28 values (sparse and dense
-// streams), and more below 300 tiles.
+// streams).  Below 768 tiles the look-back is as fast or faster.
 //
 // Zero-run emission order.  A maximal run of L bytes equal to 121 emits
 // floor(L/14) bytes 255 (one at the end of each full chunk of 14), then, if

@@ -223,6 +223,68 @@ def test_indexed_decode_corrupt_streams(g):
         assert rc == 0 and np.array_equal(bits(y), bits(y_o))
 
 
+def sparse_units_stream(seed, n):
+    """A valid stream for n values made of 512-byte units of three kinds, in
+    turn: a run of 30 literal bytes and then full escapes (one lane's 16
+    bytes all literals), a literal every 5th byte (about 100 per unit, so a
+    warp goes round its list more than once), and escapes only.  Every unit
+    has fewer literal groups than 1 in 16 of its groups.  The stream ends
+    with a literal in the last group, whose values past n are set (242: all
+    digits 2), which the decoders must ignore."""
+    groups = (n + 4) // 5
+    lits = np.minimum((synth.uniforms(synth.key_for(seed, 0), groups // 10 + 64) * 243)
+                      .astype(np.int64), 242)
+    li = 0
+    out, total, u = [], 0, 0
+    while True:
+        unit = np.full(512, 255, np.int64)
+        kind = u % 3
+        if kind == 0:
+            unit[:30] = lits[li:li + 30]
+            li += 30
+        elif kind == 1:
+            k = len(unit[::5])
+            unit[::5] = lits[li:li + k]
+            li += k
+        e = int(np.where(unit >= 243, unit - 241, 1).sum())
+        if total + e + 64 > groups:
+            break
+        out.append(unit)
+        total += e
+        u += 1
+    rest = groups - total - 1          # zero groups before the last group
+    tail = [255] * (rest // 14)
+    r = rest % 14
+    if r == 1:
+        tail.append(121)
+    elif r:
+        tail.append(241 + r)
+    tail.append(242)
+    b = np.concatenate(out + [np.array(tail, np.int64)]).astype(np.uint8)
+    head = np.frombuffer(np.float32(0.0456).tobytes(), np.uint8)
+    return np.concatenate([head, b])
+
+
+@pytest.mark.parametrize("tail", [0, 1, 4])
+def test_indexed_accumulate_sparse_units_literal_lists(g, tail):
+    # one stream summed into acc: units with few literal groups are added
+    # from a per-warp list of those groups, two list entries per lane at a
+    # time; runs of literals, long lists and the last, partial group
+    n = LARGE_N - 1234 - tail
+    st = sparse_units_stream(990 + tail, n)
+    rc_o, y_o = oracle.decompress(st, n)
+    assert rc_o == 0
+    acc0 = synth.normal(synth.key_for(991, tail), n, 0.05)
+    acc0[::11] = -0.0
+    rc_o, a_o = oracle.decompress_accumulate([st], n, acc0)
+    cap = g.tlc_compress_bound(n)
+    for offset in (0, 1):
+        rc_g, a_g = accumulate(g, [st], n, acc0, caps=[cap], offset=offset)
+        assert rc_o == rc_g == 0 and np.array_equal(bits(a_g), bits(a_o))
+    rc_g, y_g = decompress(g, st, n, cap=cap)
+    assert rc_g == 0 and np.array_equal(bits(y_g), bits(y_o))
+
+
 # ---- several streams summed in one pass --------------------------------------
 
 @pytest.mark.parametrize("k", [2, 3, 5, 8, 9, 17])
